@@ -1,0 +1,9 @@
+"""CPU oracle for the multi-round dropless MoE layer forward.
+
+TEST INFRASTRUCTURE: imported only by tests/, the smoke check in
+__graft_entry__.py and the CPU-baseline leg of bench.py. The library never
+imports it and shares no code with it.
+"""
+from .moe_oracle import (bf16_to_f64, router_logits, select_topk, gates, plan,  # noqa: F401
+                         round_rows, silu, expert_hidden, expert_ffn, forward,
+                         forward_rounds, layer)
