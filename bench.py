@@ -1,0 +1,403 @@
+"""Benchmark: routed tokens/s of one multi-round dropless MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = moe_plan (router top-k + round planner) + moe_forward (all rounds of dispatch ->
+gate/up GEMM -> down GEMM -> combine) on one batch, inputs resident in HBM. L2 is flushed
+(a 256 MiB write) between timed steps, outside the timed events. Per-step device time comes
+from CUDA events on the launching stream; the job time is the max over ranks.
+
+Multi-GPU: the layer's experts all live on one GPU, so N GPUs run N independent replicas
+(weak scaling, no collective on the data path); torch.distributed is used only for the
+barrier and the max-over-ranks of the timing.
+
+--impl reference times the CPU oracle (float64 numpy) on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from dropless_moe_layer_b200 import workloads as wl  # noqa: E402
+
+DEFAULT_WORKLOAD = "4k-zipf1"
+METRIC = "routed tokens/s per MoE layer fwd (bf16, 1 B200); % of tensor/HBM roofline"
+UNIT = "tokens/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def workload_config(w):
+    desc = {"tiny-zipf1": "Zipf(1.0) expert popularity", "4k-zipf1": "Zipf(1.0) expert popularity",
+            "16k-uniform": "near-uniform routing", "16k-hot-expert": "one expert picked by ~50% of tokens",
+            "32k-zipf1.2-router-gemm": "Zipf(1.2) popularity, logits from the router GEMM"}.get(w.name, "")
+    return {"workload": f"{w.name}: T={w.T} d={w.d} E={w.E} top-{w.k} SwiGLU d_ff={w.F} C={w.C}; {desc}",
+            "T": w.T, "d": w.d, "E": w.E, "k": w.k, "d_ff": w.F, "C": w.C,
+            "router": "fp32 logits given" if w.router == "logits" else "bf16 router GEMM x W_r^T + b",
+            "l2": "flushed between timed steps (256 MiB write, outside the timed events)"}
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_step(w, host, tokens=None):
+    import oracle
+    out = oracle.layer(host["x"], host["w_gate_up"], host["w_down"], k=w.k, C=w.C,
+                       logits=host["logits"], w_router_bits=host["w_router"], bias=host["bias"],
+                       tokens=tokens)
+    return out
+
+
+def host_inputs(w):
+    inp = wl.generate(w, "cpu")
+    return {"x": wl.bf16_bits(inp["x"]), "w_gate_up": wl.bf16_bits(inp["w_gate_up"]),
+            "w_down": wl.bf16_bits(inp["w_down"]), "logits": wl.f32_host(inp["logits"]),
+            "w_router": wl.bf16_bits(inp["w_router"]), "bias": wl.f32_host(inp["bias"])}
+
+
+def oracle_sample_plan(w, host, budget_s):
+    """Pick a token sample so one oracle step takes about `budget_s` seconds: time a probe
+    on 64 tokens (plus the full-T router and plan) and scale."""
+    import numpy as np
+    probe = np.arange(min(64, w.T))
+    t0 = time.perf_counter()
+    oracle_step(w, host, tokens=probe)
+    dt = time.perf_counter() - t0
+    per_token = dt / len(probe)
+    n = w.T if per_token * w.T <= budget_s else max(64, int(budget_s / per_token))
+    if n >= w.T:
+        return None, f"full workload ({w.T} tokens), router + plan + forward"
+    rng = np.random.default_rng(12345)
+    tok = np.sort(rng.choice(w.T, size=n, replace=False))
+    return tok, (f"seeded sample of {n} of {w.T} tokens (all their top-{w.k} pairs) + the full "
+                 f"router/top-k/plan; throughput counts the sampled tokens")
+
+
+def cpu_baseline(w, steps=1, budget_s=15.0):
+    host = host_inputs(w)
+    tok, sample = oracle_sample_plan(w, host, budget_s)
+    n_tok = w.T if tok is None else len(tok)
+    times = []
+    for _ in range(max(1, steps)):
+        t0 = time.perf_counter()
+        oracle_step(w, host, tokens=tok)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    return {"value": n_tok * len(times) / total, "unit": UNIT, "cores": blas_threads(),
+            "kind": "oracle", "sample": sample, "seconds_per_step": total / len(times)}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    host = host_inputs(w)
+    budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    tok, sample = oracle_sample_plan(w, host, budget)
+    n_tok = w.T if tok is None else len(tok)
+    for _ in range(args.warmup):
+        oracle_step(w, host, tokens=tok)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(w, host, tokens=tok)
+    dt = time.perf_counter() - t0
+    value = n_tok * args.steps / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"moe_bench_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- algorithmic work
+
+def algorithmic_work(w, info):
+    """Per kernel kind, the algorithmic units of one step (flops for the GEMMs, bytes for the
+    rest), from the plan alone. Padding rows (C - n) are never counted."""
+    import numpy as np
+    load = np.array(info.load[:w.E], dtype=np.int64)
+    R = info.R
+    n = np.clip(load[None, :] - w.C * np.arange(R)[:, None], 0, w.C)
+    rows = int(n.sum())                       # = T * k
+    work = {
+        "router_gemm": ("hbm", (w.T * w.d * 2 + w.E * w.d * 2 + w.T * w.E * 4) if w.router == "gemm" else 0),
+        "topk": ("hbm", w.T * w.E * 4 + w.T * w.k * 8),
+        "plan": ("hbm", w.T * w.k * 4 * 6),
+        "dispatch": ("hbm", 2 * rows * w.d * 2),
+        "gate_up": ("tensor", 4 * rows * w.d * w.F),
+        "down": ("tensor", 2 * rows * w.F * w.d),
+    }
+    return work, rows
+
+
+def combine_bytes(w, round_np):
+    """combine reads every pair's expert row once (d bf16), writes each token's y row on every
+    round it has a pair in, and reads it back on every such round but the first."""
+    import numpy as np
+    T, d = w.T, w.d
+    rows = T * w.k * d * 2
+    spans = np.array([len(set(r)) for r in round_np.tolist()], dtype=np.int64)
+    writes = int(spans.sum()) * d * 4
+    reads = int((spans - 1).sum()) * d * 4
+    return rows + writes + reads
+
+
+# ----------------------------------------------------------------------------- GPU benchmark
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=[x.name for x in wl.WORKLOADS])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = wl.BY_NAME[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    import numpy as np
+    import torch
+
+    from dropless_moe_layer_b200 import moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    moe.load_library()
+    inp = wl.generate(w, dev)
+    layer = moe.DroplessMoE(w.T, w.d, w.E, w.k, w.F, w.C, device=dev)
+    y = torch.empty(w.T, w.d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        layer.plan(logits=inp["logits"], x=inp["x"] if w.router == "gemm" else None,
+                   w_router=inp["w_router"], bias=inp["bias"])
+        layer.forward(inp["x"], inp["w_gate_up"], inp["w_down"], y=y)
+
+    def timed(K, profile=False):
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        if profile:
+            moe.profile_enable(True)
+        launches0 = moe.launch_count()
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+        launches = moe.launch_count() - launches0
+        prof = moe.profile_read() if profile else None
+        if profile:
+            moe.profile_enable(False)
+        if dist is not None:
+            dist.barrier()
+        ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+        return ms, launches, prof
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if layer.device_status() != 0:
+        raise SystemExit("kernel wait timed out during warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    total_ms, launches, _ = timed(args.steps)
+    clk = clocks.stop()
+    if dist is not None:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = w.T * world * args.steps / (total_ms / 1e3)
+
+    # second timed pass with per-kernel events (for the roofline of the dominant kernel)
+    _, _, prof = timed(args.steps, profile=True)
+    info = layer.info
+    work, rows = algorithmic_work(w, info)
+    rnd = layer.plan_tensors()["round"].cpu().numpy()
+    work["combine"] = ("hbm", combine_bytes(w, rnd))
+    peaks, peak_src = load_peaks()
+    kinds = {k: v for k, v in prof.items() if v[0] > 0}
+    dom = max(kinds, key=lambda k: kinds[k][1])
+    bound, units_per_step = work[dom]
+    cnt, ms = kinds[dom]
+    per_launch_units = units_per_step * args.steps / cnt
+    avg_launch_s = ms / cnt / 1e3
+    if bound == "tensor":
+        achieved, peak, unit = per_launch_units / avg_launch_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    else:
+        achieved, peak, unit = per_launch_units / avg_launch_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    per_kernel = {}
+    for k, (c, t) in kinds.items():
+        b, u = work[k]
+        rate = u * args.steps / (t / 1e3)
+        per_kernel[k] = {"launches": c, "ms_total": round(t, 4), "share": round(t / sum(v[1] for v in kinds.values()), 4),
+                         "bound": b, ("TFLOP/s" if b == "tensor" else "GB/s"): round(rate / (1e12 if b == "tensor" else 1e9), 2)}
+
+    # end to end through the public API from pinned host buffers
+    host_x = inp["x"].cpu().pin_memory()
+    host_z = inp["logits"].cpu().pin_memory() if inp["logits"] is not None else None
+    host_y = torch.empty(w.T, w.d, dtype=torch.float32).pin_memory()
+    dx = torch.empty_like(inp["x"])
+    dz = torch.empty_like(inp["logits"]) if host_z is not None else None
+    h2d = host_x.numel() * 2 + (host_z.numel() * 4 if host_z is not None else 0)
+    d2h = host_y.numel() * 4
+
+    def e2e_step():
+        dx.copy_(host_x, non_blocking=True)
+        if dz is not None:
+            dz.copy_(host_z, non_blocking=True)
+        layer.plan(logits=dz, x=dx if w.router == "gemm" else None, w_router=inp["w_router"], bias=inp["bias"])
+        layer.forward(dx, inp["w_gate_up"], inp["w_down"], y=y)
+        host_y.copy_(y, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = 0.0
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev0.record(stream)
+        e2e_step()
+        ev1.record(stream)
+        ev1.synchronize()
+        e2e_ms += ev0.elapsed_time(ev1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = w.T * world * args.steps / (e2e_ms / 1e3)
+    status = layer.device_status()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(w),
+            "rounds": info.R, "routed_pairs_per_s": value * w.k,
+            "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                         "frac": achieved / peak, "peak_source": f"{peak_src} ({'bf16_tflops burst' if bound == 'tensor' else 'hbm_gbs copy'})",
+                         "traffic": None},
+            "kernels": per_kernel,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clk,
+            "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

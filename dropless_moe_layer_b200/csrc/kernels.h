@@ -1,0 +1,91 @@
+// kernels.h - internal launchers shared by the library's translation units.
+// Not part of the public C ABI (that is include/moe.h).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+// Workspace status word bits (header[kHdrStatus]).
+enum : int {
+  kStatusTimeoutProducer = 1,
+  kStatusTimeoutMma = 2,
+  kStatusTimeoutEpilogue = 4,
+};
+
+// Header words inside the workspace.
+enum : int {
+  kHdrR = 0,
+  kHdrMaxLoad = 1,
+  kHdrStatus = 2,
+  kHdrLoad = 64,      // copy of load[0..E-1], so one small copy brings the plan summary home
+  kHdrWords = 64 + 256,
+};
+
+constexpr int kPlanTokensPerBlock = 256;
+#define MOE_MAX_E_PLAN 256
+
+// Kernel kinds for profiling (same numbering as the public header).
+enum KernelKind : int {
+  kKindRouterGemm = 0,
+  kKindTopk = 1,
+  kKindPlan = 2,
+  kKindDispatch = 3,
+  kKindGateUp = 4,
+  kKindDown = 5,
+  kKindCombine = 6,
+};
+
+// Called around every launch (profiling and launch accounting).
+void launch_begin(int kind, cudaStream_t stream);
+void launch_end(int kind, cudaStream_t stream, int kernels = 1);
+
+int num_sms();
+
+// ---- router / top-k (router.cu)
+cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int renorm, int32_t* idx,
+                               float* gate, cudaStream_t stream);
+
+// ---- planner (plan.cu)
+struct PlanBuffers {
+  const int32_t* idx;     // [T, k]
+  int32_t* header;        // [kHdrWords]
+  int32_t* load;          // [E]
+  int32_t* offsets;       // [E + 1]
+  int32_t* block_base;    // [blocks, E]
+  int32_t* n;             // [max_rounds, E]
+  int32_t* row_off;       // [max_rounds, E]
+  int32_t* row_start;     // [max_rounds + 1]
+  int32_t* round;         // [T, k]
+  int32_t* slot;          // [T, k]
+  int32_t* row_token;     // [T * k]
+  int32_t* row_dst;       // [T * k]
+};
+cudaError_t launch_plan(const PlanBuffers& b, int T, int k, int E, int C, int max_rounds,
+                        cudaStream_t stream);
+
+// ---- dispatch / combine (dispatch_combine.cu)
+cudaError_t launch_dispatch(const uint16_t* x, uint16_t* buf, const int32_t* row_start,
+                            const int32_t* row_token, const int32_t* row_dst, int r, int rows,
+                            int d, cudaStream_t stream);
+cudaError_t launch_combine(const uint16_t* buf, float* y, const int32_t* idx, const float* gate,
+                           const int32_t* round, const int32_t* slot, int T, int k, int C, int d,
+                           int r, cudaStream_t stream);
+
+// ---- grouped GEMMs (grouped_gemm.cu)
+// gate_up: h[e][s] = bf16(silu(buf[e][s] W1_e^T) * (buf[e][s] W3_e^T)), s < n_dev[e]
+cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint16_t* h,
+                           const int32_t* n_dev, const int32_t* n_host, int E, int C, int d, int F,
+                           int32_t* status, cudaStream_t stream);
+// down: out[e][s] = bf16(h[e][s] W2_e^T), s < n_dev[e]
+cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out,
+                        const int32_t* n_dev, const int32_t* n_host, int E, int C, int d, int F,
+                        int32_t* status, cudaStream_t stream);
+// router GEMM: logits[t][e] = x[t] . w_router[e] + bias[e] (fp32 out)
+cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                               float* logits, int T, int d, int E, int32_t* status,
+                               cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,418 @@
+// moe_api.cu - the C ABI (include/moe.h): argument checks, the fixed workspace layout,
+// the router -> planner sequence and the round loop.
+//
+// The memory of the layer is fixed by the shape alone ("Frontier Pre-training at
+// Microsoft AI (MAI-Base-2)", Key claims, multi-round dropless MoE item: memory usage
+// is static whatever the token imbalance). moe_workspace_bytes() depends on
+// (T, d, E, k, d_ff, C) only; the routing decides how many rounds run, never how much
+// memory they use.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.h"
+#include "moe.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- accounting / profiling
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+constexpr int kProfMax = 4096;
+struct Profiler {
+  bool on = false;
+  bool created = false;
+  int n = 0;
+  int kind[kProfMax];
+  cudaEvent_t ev[2 * kProfMax];
+};
+Profiler g_prof;
+
+std::mutex g_sm_mutex;
+int g_sm_count[64] = {0};
+
+}  // namespace
+
+void launch_begin(int kind, cudaStream_t stream) {
+  (void)kind;
+  if (g_prof.on && g_prof.n < kProfMax) cudaEventRecord(g_prof.ev[2 * g_prof.n], stream);
+}
+
+void launch_end(int kind, cudaStream_t stream, int kernels) {
+  g_launches.fetch_add(static_cast<uint64_t>(kernels));
+  if (g_prof.on && g_prof.n < kProfMax) {
+    cudaEventRecord(g_prof.ev[2 * g_prof.n + 1], stream);
+    g_prof.kind[g_prof.n] = kind;
+    ++g_prof.n;
+  }
+}
+
+int num_sms() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  dev &= 63;
+  std::lock_guard<std::mutex> lock(g_sm_mutex);
+  if (g_sm_count[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    g_sm_count[dev] = n > 0 ? n : 1;
+  }
+  return g_sm_count[dev];
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+int check_shape(const moe_shape_t* s) {
+  if (s == nullptr) return MOE_ERR_INVALID_ARG;
+  if (s->flags & ~static_cast<uint32_t>(MOE_FLAG_RENORM_TOPK)) return MOE_ERR_INVALID_ARG;
+  if (s->T < 0 || s->E < 1 || s->E > MOE_MAX_EXPERTS || s->k < 1 || s->k > MOE_MAX_TOPK ||
+      s->k > s->E || s->C < 1)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s->d < 64 || s->d > 16384 || s->d % 64 != 0 || s->d_ff < 64 || s->d_ff > 16384 ||
+      s->d_ff % 64 != 0)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<long long>(s->T) * s->k >= (1ll << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<long long>(s->E) * s->C >= (1ll << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  const long long wide = s->d > s->d_ff ? s->d : s->d_ff;
+  if (static_cast<long long>(s->C) * wide * 2 >= (1ll << 40)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+int max_rounds_of(const moe_shape_t* s) { return s->T == 0 ? 0 : (s->T + s->C - 1) / s->C; }
+
+void make_layout(const moe_shape_t* s, moe_workspace_layout_t* L) {
+  std::memset(L, 0, sizeof(*L));
+  size_t off = 0;
+  auto take = [&](long long bytes) {
+    const size_t o = off;
+    off += (static_cast<size_t>(bytes) + 255) & ~static_cast<size_t>(255);
+    return o;
+  };
+  const long long T = s->T, E = s->E, k = s->k, C = s->C;
+  const int mr = max_rounds_of(s);
+  const int blocks = static_cast<int>((T + kPlanTokensPerBlock - 1) / kPlanTokensPerBlock);
+  L->header = take(kHdrWords * 4ll);
+  L->logits = take(T * E * 4);
+  L->topk_idx = take(T * k * 4);
+  L->gate = take(T * k * 4);
+  L->round = take(T * k * 4);
+  L->slot = take(T * k * 4);
+  L->load = take(E * 4);
+  L->offsets = take((E + 1) * 4);
+  L->block_base = take(static_cast<long long>(blocks) * E * 4);
+  L->n = take(static_cast<long long>(mr) * E * 4);
+  L->row_off = take(static_cast<long long>(mr) * E * 4);
+  L->row_start = take((mr + 1ll) * 4);
+  L->row_token = take(T * k * 4);
+  L->row_dst = take(T * k * 4);
+  L->buf = take(E * C * s->d * 2);
+  L->h = take(E * C * s->d_ff * 2);
+  L->total_bytes = off;
+  L->max_rounds = mr;
+  L->plan_blocks = blocks;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+int check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  static std::atomic<uint64_t> ok_mask{0}, bad_mask{0};
+  const uint64_t bit = 1ull << (dev & 63);
+  if (ok_mask.load() & bit) return MOE_OK;
+  if (bad_mask.load() & bit) return MOE_ERR_NO_DEVICE;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (major != 10) {
+    bad_mask.fetch_or(bit);
+    return MOE_ERR_NO_DEVICE;
+  }
+  ok_mask.fetch_or(bit);
+  return MOE_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Common checks of the calls that run a plan.
+int check_run(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
+              moe_workspace_layout_t* L) {
+  int st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (info == nullptr || ws == nullptr) return MOE_ERR_INVALID_ARG;
+  make_layout(shape, L);
+  if (ws_bytes < L->total_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned(ws, 256)) return MOE_ERR_MISALIGNED;
+  if (info->R < 0 || info->R > L->max_rounds) return MOE_ERR_INVALID_ARG;
+  return check_device();
+}
+
+void round_rows(const moe_shape_t* s, const moe_plan_info_t* info, int r, int32_t* n_host, int* rows) {
+  long long total = 0;
+  const long long base = static_cast<long long>(r) * s->C;
+  for (int e = 0; e < s->E; ++e) {
+    const long long rem = info->load[e] - base;
+    n_host[e] = rem <= 0 ? 0 : rem >= s->C ? s->C : static_cast<int32_t>(rem);
+    total += n_host[e];
+  }
+  *rows = static_cast<int>(total);
+}
+
+int do_dispatch(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
+                const moe_workspace_layout_t& L, int r, const uint16_t* x, cudaStream_t stream) {
+  int32_t n_host[MOE_MAX_EXPERTS];
+  int rows = 0;
+  round_rows(s, info, r, n_host, &rows);
+  return cuda_status(launch_dispatch(x, at<uint16_t>(ws, L.buf), at<int32_t>(ws, L.row_start),
+                                     at<int32_t>(ws, L.row_token), at<int32_t>(ws, L.row_dst), r, rows,
+                                     s->d, stream));
+}
+
+int do_gate_up(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
+               const moe_workspace_layout_t& L, int r, const uint16_t* w13, cudaStream_t stream) {
+  int32_t n_host[MOE_MAX_EXPERTS];
+  int rows = 0;
+  round_rows(s, info, r, n_host, &rows);
+  return cuda_status(launch_gate_up(at<uint16_t>(ws, L.buf), w13, at<uint16_t>(ws, L.h),
+                                    at<int32_t>(ws, L.n) + static_cast<size_t>(r) * s->E, n_host,
+                                    s->E, s->C, s->d, s->d_ff,
+                                    at<int32_t>(ws, L.header) + kHdrStatus, stream));
+}
+
+int do_down(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
+            const moe_workspace_layout_t& L, int r, const uint16_t* w2, cudaStream_t stream) {
+  int32_t n_host[MOE_MAX_EXPERTS];
+  int rows = 0;
+  round_rows(s, info, r, n_host, &rows);
+  return cuda_status(launch_down(at<uint16_t>(ws, L.h), w2, at<uint16_t>(ws, L.buf),
+                                 at<int32_t>(ws, L.n) + static_cast<size_t>(r) * s->E, n_host, s->E,
+                                 s->C, s->d, s->d_ff, at<int32_t>(ws, L.header) + kHdrStatus,
+                                 stream));
+}
+
+int do_combine(const moe_shape_t* s, void* ws, const moe_workspace_layout_t& L, int r, float* y,
+               cudaStream_t stream) {
+  return cuda_status(launch_combine(at<uint16_t>(ws, L.buf), y, at<int32_t>(ws, L.topk_idx),
+                                    at<float>(ws, L.gate), at<int32_t>(ws, L.round),
+                                    at<int32_t>(ws, L.slot), s->T, s->k, s->C, s->d, r, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_bytes(const moe_shape_t* shape) {
+  if (check_shape(shape) != MOE_OK) return 0;
+  moe_workspace_layout_t L;
+  make_layout(shape, &L);
+  return L.total_bytes;
+}
+
+int moe_workspace_layout(const moe_shape_t* shape, moe_workspace_layout_t* layout) {
+  const int st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (layout == nullptr) return MOE_ERR_INVALID_ARG;
+  make_layout(shape, layout);
+  return MOE_OK;
+}
+
+int moe_plan(const moe_shape_t* shape, const float* logits, const uint16_t* x,
+             const uint16_t* w_router, const float* bias, void* ws, size_t ws_bytes,
+             moe_plan_info_t* info, moe_stream_t stream_) {
+  int st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (ws == nullptr || info == nullptr) return MOE_ERR_INVALID_ARG;
+  if (logits == nullptr && shape->T > 0 && (x == nullptr || w_router == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  moe_workspace_layout_t L;
+  make_layout(shape, &L);
+  if (ws_bytes < L.total_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned(ws, 256) || !aligned(logits, 16) || !aligned(x, 16) || !aligned(w_router, 16) ||
+      !aligned(bias, 4))
+    return MOE_ERR_MISALIGNED;
+  if ((st = check_device()) != MOE_OK) return st;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const moe_shape_t& s = *shape;
+  int32_t* header = at<int32_t>(ws, L.header);
+  if (cudaMemsetAsync(header, 0, kHdrWords * 4, stream) != cudaSuccess) return MOE_ERR_CUDA;
+
+  const float* z = logits;
+  if (z == nullptr && s.T > 0) {
+    if ((st = cuda_status(launch_router_gemm(x, w_router, bias, at<float>(ws, L.logits), s.T, s.d,
+                                             s.E, header + kHdrStatus, stream))) != MOE_OK)
+      return st;
+    z = at<float>(ws, L.logits);
+  }
+  if ((st = cuda_status(launch_router_topk(z, s.T, s.E, s.k, (s.flags & MOE_FLAG_RENORM_TOPK) ? 1 : 0,
+                                           at<int32_t>(ws, L.topk_idx), at<float>(ws, L.gate),
+                                           stream))) != MOE_OK)
+    return st;
+  PlanBuffers pb;
+  pb.idx = at<int32_t>(ws, L.topk_idx);
+  pb.header = header;
+  pb.load = at<int32_t>(ws, L.load);
+  pb.offsets = at<int32_t>(ws, L.offsets);
+  pb.block_base = at<int32_t>(ws, L.block_base);
+  pb.n = at<int32_t>(ws, L.n);
+  pb.row_off = at<int32_t>(ws, L.row_off);
+  pb.row_start = at<int32_t>(ws, L.row_start);
+  pb.round = at<int32_t>(ws, L.round);
+  pb.slot = at<int32_t>(ws, L.slot);
+  pb.row_token = at<int32_t>(ws, L.row_token);
+  pb.row_dst = at<int32_t>(ws, L.row_dst);
+  if ((st = cuda_status(launch_plan(pb, s.T, s.k, s.E, s.C, L.max_rounds, stream))) != MOE_OK) return st;
+
+  int32_t host[kHdrWords];
+  if (cudaMemcpyAsync(host, header, sizeof(host), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (host[kHdrStatus] != 0) return MOE_ERR_TIMEOUT;
+
+  info->R = host[kHdrR];
+  info->max_load = host[kHdrMaxLoad];
+  for (int e = 0; e < MOE_MAX_EXPERTS; ++e) info->load[e] = e < s.E ? host[kHdrLoad + e] : 0;
+  info->logits = z;
+  info->topk_idx = pb.idx;
+  info->gate = at<float>(ws, L.gate);
+  info->round = pb.round;
+  info->slot = pb.slot;
+  info->offsets = pb.offsets;
+  info->n = pb.n;
+  return MOE_OK;
+}
+
+int moe_round_dispatch(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
+                       int32_t r, const uint16_t* x, moe_stream_t stream) {
+  moe_workspace_layout_t L;
+  int st = check_run(shape, info, ws, ws_bytes, &L);
+  if (st != MOE_OK) return st;
+  if (r < 0 || r >= info->R || x == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16)) return MOE_ERR_MISALIGNED;
+  return do_dispatch(shape, info, ws, L, r, x, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_round_gate_up(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
+                      int32_t r, const uint16_t* w_gate_up, moe_stream_t stream) {
+  moe_workspace_layout_t L;
+  int st = check_run(shape, info, ws, ws_bytes, &L);
+  if (st != MOE_OK) return st;
+  if (r < 0 || r >= info->R || w_gate_up == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(w_gate_up, 16)) return MOE_ERR_MISALIGNED;
+  return do_gate_up(shape, info, ws, L, r, w_gate_up, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_round_down(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
+                   int32_t r, const uint16_t* w_down, moe_stream_t stream) {
+  moe_workspace_layout_t L;
+  int st = check_run(shape, info, ws, ws_bytes, &L);
+  if (st != MOE_OK) return st;
+  if (r < 0 || r >= info->R || w_down == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(w_down, 16)) return MOE_ERR_MISALIGNED;
+  return do_down(shape, info, ws, L, r, w_down, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_round_combine(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
+                      int32_t r, float* y, moe_stream_t stream) {
+  moe_workspace_layout_t L;
+  int st = check_run(shape, info, ws, ws_bytes, &L);
+  if (st != MOE_OK) return st;
+  if (r < 0 || r >= info->R || y == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(y, 16)) return MOE_ERR_MISALIGNED;
+  return do_combine(shape, ws, L, r, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
+                const uint16_t* x, const uint16_t* w_gate_up, const uint16_t* w_down, float* y,
+                moe_stream_t stream_) {
+  moe_workspace_layout_t L;
+  int st = check_run(shape, info, ws, ws_bytes, &L);
+  if (st != MOE_OK) return st;
+  if (shape->T > 0 && (x == nullptr || w_gate_up == nullptr || w_down == nullptr || y == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(w_gate_up, 16) || !aligned(w_down, 16) || !aligned(y, 16))
+    return MOE_ERR_MISALIGNED;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  for (int r = 0; r < info->R; ++r) {
+    if ((st = do_dispatch(shape, info, ws, L, r, x, stream)) != MOE_OK) return st;
+    if ((st = do_gate_up(shape, info, ws, L, r, w_gate_up, stream)) != MOE_OK) return st;
+    if ((st = do_down(shape, info, ws, L, r, w_down, stream)) != MOE_OK) return st;
+    if ((st = do_combine(shape, ws, L, r, y, stream)) != MOE_OK) return st;
+  }
+  return MOE_OK;
+}
+
+int moe_device_status(const moe_shape_t* shape, void* ws, moe_stream_t stream_) {
+  const int st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (ws == nullptr) return MOE_ERR_INVALID_ARG;
+  moe_workspace_layout_t L;
+  make_layout(shape, &L);
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int32_t word = 0;
+  if (cudaMemcpyAsync(&word, at<int32_t>(ws, L.header) + kHdrStatus, 4, cudaMemcpyDeviceToHost, stream) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  return word != 0 ? MOE_ERR_TIMEOUT : MOE_OK;
+}
+
+const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MOE_ERR_MISALIGNED: return "misaligned pointer";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "a kernel wait timed out";
+    case MOE_ERR_NO_DEVICE: return "current device is not sm_100";
+    default: return "unknown status";
+  }
+}
+
+uint64_t moe_launch_count(void) { return g_launches.load(); }
+
+int moe_profile_enable(int on) {
+  if (on && !g_prof.created) {
+    for (int i = 0; i < 2 * kProfMax; ++i)
+      if (cudaEventCreate(&g_prof.ev[i]) != cudaSuccess) return MOE_ERR_CUDA;
+    g_prof.created = true;
+  }
+  g_prof.on = on != 0;
+  g_prof.n = 0;
+  return MOE_OK;
+}
+
+int moe_profile_read(int32_t counts[MOE_PROFILE_KINDS], double ms[MOE_PROFILE_KINDS]) {
+  if (counts == nullptr || ms == nullptr) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < MOE_PROFILE_KINDS; ++i) {
+    counts[i] = 0;
+    ms[i] = 0.0;
+  }
+  for (int i = 0; i < g_prof.n; ++i) {
+    if (cudaEventSynchronize(g_prof.ev[2 * i + 1]) != cudaSuccess) return MOE_ERR_CUDA;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]) != cudaSuccess) return MOE_ERR_CUDA;
+    counts[g_prof.kind[i]] += 1;
+    ms[g_prof.kind[i]] += t;
+  }
+  g_prof.n = 0;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,192 @@
+/*
+ * moe.h - C ABI of the multi-round dropless MoE layer forward for NVIDIA B200 (sm_100a).
+ *
+ * The method (sources, by page and section):
+ *   - "Frontier Pre-training at Microsoft AI (MAI-Base-2)", Key claims, the multi-round
+ *     dropless MoE item [section "Scaling MoE", Fig. 6]: each expert group runs one or
+ *     more dispatch -> compute -> collect rounds with a fixed per-expert token capacity;
+ *     overflow waits for another round; memory stays static whatever the imbalance;
+ *     capacity is tunable.
+ *   - "Microsoft AI's MAI-Base-2 trained on 16K GPUs with Muon", section "Expert groups
+ *     keep memory fixed when tokens pile up": a router sends each token to a few experts;
+ *     larger capacity costs memory, smaller capacity costs rounds.
+ *   - "MAI-Base-2: Microsoft's 2.8T Model is a BREAKTHROUGH" (transcript, 03:11): no token
+ *     is dropped.
+ *
+ * What this library computes (all experts on one GPU):
+ *   z = logits [T,E] fp32 (given, or x @ w_router^T + bias)
+ *   idx[t,0..k-1] = top-k experts of z[t] (logit descending, ties -> lower expert index)
+ *   gate[t,j]     = softmax(z[t])[idx[t,j]] (fp32; divided by the k gates' sum with
+ *                   MOE_FLAG_RENORM_TOPK)
+ *   rank(t,j)     = number of tokens t' < t that selected the same expert
+ *   round = rank / C, slot = rank % C, R = ceil(max_e load_e / C)
+ *   for r in 0..R-1:
+ *     dispatch: buf[e][slot] = x[t] for every pair in round r       (buf: [E, C, d] bf16)
+ *     experts:  h = bf16(silu(buf W1^T) * (buf W3^T)); out = bf16(h W2^T)   (grouped GEMMs)
+ *     combine:  y[t] += gate[t,j] * out[e][slot] for the round's pairs, j ascending
+ *   y [T, d] fp32 equals the capacity-free dropless MoE output up to bf16 rounding of the
+ *   expert intermediates.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, row-major, contiguous,
+ *     16-byte aligned. bf16 is passed as its uint16_t bit pattern. The workspace must be
+ *     256-byte aligned. The library allocates no device memory.
+ *   - Entry points return MOE_OK (0) or a negative moe_status; invalid arguments are found
+ *     on the host before any kernel is launched, and no entry point aborts the process.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *     Only moe_plan() synchronizes the stream (once, to learn the round count R).
+ *   - Faults of earlier asynchronous work surface as MOE_ERR_CUDA from a later call.
+ *   - Results are deterministic: the same inputs, C and GPU give the same bits.
+ *   - Shape limits: T >= 0, 1 <= E <= 256, 1 <= k <= min(E, 16), d and d_ff multiples of
+ *     64 in [64, 16384], C >= 1, T*k < 2^31, E*C < 2^31.
+ */
+#ifndef DROPLESS_MOE_H_
+#define DROPLESS_MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,         /* null pointer, bad round index, inconsistent plan info */
+  MOE_ERR_UNSUPPORTED_SHAPE = -2,   /* a shape limit above is violated */
+  MOE_ERR_WORKSPACE_TOO_SMALL = -3, /* ws_bytes < moe_workspace_bytes(shape) */
+  MOE_ERR_MISALIGNED = -4,          /* a pointer breaks the alignment rules */
+  MOE_ERR_CUDA = -5,                /* a CUDA runtime call failed (includes earlier faults) */
+  MOE_ERR_TIMEOUT = -6,             /* a kernel's bounded wait gave up; see moe_device_status */
+  MOE_ERR_NO_DEVICE = -7            /* current device is not an sm_100 GPU */
+} moe_status;
+
+/* moe_shape_t.flags */
+#define MOE_FLAG_RENORM_TOPK 1u     /* divide the k selected gates of a token by their sum */
+
+#define MOE_MAX_EXPERTS 256
+#define MOE_MAX_TOPK 16
+
+/* Layer shape. T tokens, hidden size d, E experts, top-k, SwiGLU inner size d_ff,
+ * per-expert capacity C of one round (the pages' tunable capacity). */
+typedef struct moe_shape {
+  int32_t T, d, E, k, d_ff, C;
+  uint32_t flags;
+} moe_shape_t;
+
+/* Host-side result of moe_plan(). Caller-owned; pass it unchanged to the calls that
+ * execute that plan on the same workspace. The device pointers point into the workspace. */
+typedef struct moe_plan_info {
+  int32_t R;                        /* number of rounds = ceil(max_load / C); 0 if T == 0 */
+  int32_t max_load;                 /* largest number of tokens routed to one expert */
+  int32_t load[MOE_MAX_EXPERTS];    /* tokens routed to each expert (first E entries) */
+  const float* logits;              /* [T, E] fp32 logits the plan used (caller's or computed) */
+  const int32_t* topk_idx;          /* [T, k] selected experts, best first */
+  const float* gate;                /* [T, k] gates */
+  const int32_t* round;             /* [T, k] round of each (token, expert) pair */
+  const int32_t* slot;              /* [T, k] row of the pair inside its expert's C rows */
+  const int32_t* offsets;           /* [E + 1] exclusive prefix sum of load */
+  const int32_t* n;                 /* [max_rounds, E] rows of expert e in round r */
+} moe_plan_info_t;
+
+/* Byte offsets of the sub-buffers inside the workspace (all 256-byte aligned). */
+typedef struct moe_workspace_layout {
+  size_t total_bytes;
+  size_t header;      /* int32[64]: R, max_load, status word, ... */
+  size_t logits;      /* f32 [T, E]   logits from the router GEMM */
+  size_t topk_idx;    /* i32 [T, k] */
+  size_t gate;        /* f32 [T, k] */
+  size_t round;       /* i32 [T, k] */
+  size_t slot;        /* i32 [T, k] */
+  size_t load;        /* i32 [E] */
+  size_t offsets;     /* i32 [E + 1] */
+  size_t block_base;  /* i32 [plan_blocks, E] planner scratch: per-block per-expert counts */
+  size_t n;           /* i32 [max_rounds, E] rows of expert e in round r */
+  size_t row_off;     /* i32 [max_rounds, E] first row of (round r, expert e) in the row list */
+  size_t row_start;   /* i32 [max_rounds + 1]: first row of round r in the round-major row list */
+  size_t row_token;   /* i32 [T * k] round-major row list: source token */
+  size_t row_dst;     /* i32 [T * k] round-major row list: destination e * C + slot */
+  size_t buf;         /* bf16 [E, C, d]: dispatch buffer; also the expert output of the round */
+  size_t h;           /* bf16 [E, C, d_ff]: SwiGLU activations of the round */
+  int32_t max_rounds; /* ceil(T / C): no expert can receive more than T tokens */
+  int32_t plan_blocks;
+} moe_workspace_layout_t;
+
+/* Bytes of device workspace for `shape`. Depends on the shape only, never on the
+ * routing: this is the layer's fixed memory. Returns 0 for an invalid shape. */
+MOE_API size_t moe_workspace_bytes(const moe_shape_t* shape);
+
+/* Fills *layout for `shape`. Returns MOE_OK or MOE_ERR_UNSUPPORTED_SHAPE / INVALID_ARG. */
+MOE_API int moe_workspace_layout(const moe_shape_t* shape, moe_workspace_layout_t* layout);
+
+/* Router + round planner.
+ *   logits   [T, E] fp32, or NULL to compute logits = x @ w_router^T + bias on tensor cores;
+ *   x        [T, d] bf16 (needed only when logits == NULL);
+ *   w_router [E, d] bf16 (nn.Linear layout; needed only when logits == NULL);
+ *   bias     [E] fp32 or NULL (used only when logits == NULL).
+ * Writes topk/gate/round/slot/load/offsets/n and the round-major row list into `ws`,
+ * then synchronizes `stream` once and fills *info (R, max_load, load[], device pointers).
+ * Non-finite logits give undefined routing. */
+MOE_API int moe_plan(const moe_shape_t* shape, const float* logits, const uint16_t* x,
+             const uint16_t* w_router, const float* bias, void* ws, size_t ws_bytes,
+             moe_plan_info_t* info, moe_stream_t stream);
+
+/* Executes all R rounds of the plan in `info` (from moe_plan on this `ws`):
+ *   x         [T, d] bf16
+ *   w_gate_up [E, 2*d_ff, d] bf16: rows 0..d_ff-1 = W1 (gate), rows d_ff..2*d_ff-1 = W3 (up)
+ *   w_down    [E, d, d_ff] bf16 (W2)
+ *   y         [T, d] fp32 output; every row is written (rows of tokens with pairs are
+ *             overwritten on their first round; T*k >= T pairs means every token has one).
+ * Asynchronous: no synchronization. */
+MOE_API int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
+                const uint16_t* x, const uint16_t* w_gate_up, const uint16_t* w_down, float* y,
+                moe_stream_t stream);
+
+/* The four steps of round r (0 <= r < info->R), as moe_forward runs them. Exposed so that
+ * each kernel can be checked and timed on its own; call them in this order per round.
+ *   dispatch: buf[e][s] = x[token] for the round's rows (bf16 copy)
+ *   gate_up:  h[e][s] = bf16(silu(buf[e][s] W1_e^T) * (buf[e][s] W3_e^T)) for s < n[r][e]
+ *   down:     buf[e][s] = bf16(h[e][s] W2_e^T) for s < n[r][e] (overwrites the dispatch rows)
+ *   combine:  y[t] = (t's first round ? 0 : y[t]) + sum_{j ascending, round(t,j)=r} gate*buf */
+MOE_API int moe_round_dispatch(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
+                       size_t ws_bytes, int32_t r, const uint16_t* x, moe_stream_t stream);
+MOE_API int moe_round_gate_up(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
+                      size_t ws_bytes, int32_t r, const uint16_t* w_gate_up, moe_stream_t stream);
+MOE_API int moe_round_down(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
+                   size_t ws_bytes, int32_t r, const uint16_t* w_down, moe_stream_t stream);
+MOE_API int moe_round_combine(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
+                      size_t ws_bytes, int32_t r, float* y, moe_stream_t stream);
+
+/* Synchronizes `stream` and reads the workspace status word that kernels set when a
+ * bounded wait gives up. Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_CUDA. */
+MOE_API int moe_device_status(const moe_shape_t* shape, void* ws, moe_stream_t stream);
+
+/* Human-readable text for a moe_status value (static storage). */
+MOE_API const char* moe_status_string(int status);
+
+/* Number of kernels this library has launched in this process (for accounting). */
+MOE_API uint64_t moe_launch_count(void);
+
+/* Per-kernel timing with CUDA events. While enabled, every launch made by the calls above
+ * is bracketed by two events on its stream; moe_profile_read() synchronizes on them and
+ * reports, per kernel kind, the launch count and the summed milliseconds. Kinds:
+ * 0 router GEMM, 1 top-k, 2 plan, 3 dispatch, 4 gate_up GEMM, 5 down GEMM, 6 combine.
+ * Up to 4096 launches are recorded between enable and read. Not thread-safe. */
+#define MOE_PROFILE_KINDS 7
+MOE_API int moe_profile_enable(int on);
+MOE_API int moe_profile_read(int32_t counts[MOE_PROFILE_KINDS], double ms[MOE_PROFILE_KINDS]);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DROPLESS_MOE_H_ */

@@ -1,0 +1,112 @@
+"""Host-side checks of the C ABI: the library builds, loads and exports every entry
+point that include/moe.h declares, and argument errors are reported as status codes
+without touching the GPU (these calls return before any CUDA call)."""
+import ctypes
+
+import pytest
+
+from dropless_moe_layer_b200 import build, moe
+from dropless_moe_layer_b200 import workloads as wl
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return moe.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = moe.header_symbols()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(lib, n), n
+    for n in ["moe_workspace_bytes", "moe_plan", "moe_forward"]:
+        assert n in names
+
+
+def test_status_strings(lib):
+    for code in moe.STATUS:
+        assert lib.moe_status_string(code)
+    assert lib.moe_status_string(12345) == b"unknown status"
+
+
+def _bytes_model(w):
+    """Workspace size from the layout rules: 256-byte aligned regions."""
+    def a(n):
+        return (n + 255) // 256 * 256
+    T, E, k, C, d, F = w.T, w.E, w.k, w.C, w.d, w.F
+    mr = (T + C - 1) // C
+    blocks = (T + 255) // 256
+    return (a(320 * 4) + a(T * E * 4) + 4 * a(T * k * 4) + a(E * 4) + a((E + 1) * 4)
+            + a(blocks * E * 4) + 2 * a(mr * E * 4) + a((mr + 1) * 4) + 2 * a(T * k * 4)
+            + a(E * C * d * 2) + a(E * C * F * 2))
+
+
+@pytest.mark.parametrize("w", wl.WORKLOADS, ids=lambda w: w.name)
+def test_workspace_is_fixed_by_shape(lib, w):
+    s = moe.make_shape(w.T, w.d, w.E, w.k, w.F, w.C)
+    n = moe.workspace_bytes(s)
+    assert n == _bytes_model(w)
+    # the round buffers dominate: E*C*(d + d_ff) bf16
+    assert n >= w.E * w.C * (w.d + w.F) * 2
+    lay = moe.workspace_layout(s)
+    assert lay.total_bytes == n
+    offs = [lay.header, lay.logits, lay.topk_idx, lay.gate, lay.round, lay.slot, lay.load,
+            lay.offsets, lay.block_base, lay.n, lay.row_off, lay.row_start, lay.row_token,
+            lay.row_dst, lay.buf, lay.h]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert lay.max_rounds == (w.T + w.C - 1) // w.C
+
+
+@pytest.mark.parametrize("kw", [
+    dict(E=0), dict(E=257), dict(k=0), dict(k=17, E=32), dict(k=5, E=4), dict(C=0),
+    dict(d=96), dict(d=32), dict(d_ff=100), dict(T=-1), dict(d=16448),
+])
+def test_bad_shapes_are_rejected(lib, kw):
+    base = dict(T=64, d=128, E=8, k=2, d_ff=128, C=16)
+    base.update(kw)
+    s = moe.make_shape(**base)
+    assert moe.workspace_bytes(s) == 0
+    lay = moe.WorkspaceLayout()
+    assert lib.moe_workspace_layout(ctypes.byref(s), ctypes.byref(lay)) == -2
+
+
+def test_bad_flags_rejected(lib):
+    s = moe.make_shape(64, 128, 8, 2, 128, 16)
+    s.flags = 4
+    assert moe.workspace_bytes(s) == 0
+
+
+def test_plan_argument_errors_without_gpu(lib):
+    s = moe.make_shape(64, 128, 8, 2, 128, 16)
+    need = moe.workspace_bytes(s)
+    info = moe.PlanInfo()
+    P = ctypes.byref
+    # null workspace / null info
+    assert lib.moe_plan(P(s), 4096, None, None, None, None, need, P(info), None) == -1
+    assert lib.moe_plan(P(s), 4096, None, None, None, 1 << 20, need, None, None) == -1
+    # neither logits nor (x, w_router)
+    assert lib.moe_plan(P(s), None, None, None, None, 1 << 20, need, P(info), None) == -1
+    # workspace too small
+    assert lib.moe_plan(P(s), 4096, None, None, None, 1 << 20, need - 1, P(info), None) == -3
+    # misaligned workspace / logits
+    assert lib.moe_plan(P(s), 4096, None, None, None, (1 << 20) + 16, need, P(info), None) == -4
+    assert lib.moe_plan(P(s), 4100, None, None, None, 1 << 20, need, P(info), None) == -4
+
+
+def test_forward_argument_errors_without_gpu(lib):
+    s = moe.make_shape(64, 128, 8, 2, 128, 16)
+    need = moe.workspace_bytes(s)
+    info = moe.PlanInfo()
+    info.R = 5                                   # more rounds than ceil(T / C) = 4
+    P = ctypes.byref
+    ws = 1 << 20
+    assert lib.moe_forward(P(s), P(info), ws, need, 4096, 4096, 4096, 4096, None) == -1
+    info.R = 1
+    assert lib.moe_forward(P(s), None, ws, need, 4096, 4096, 4096, 4096, None) == -1
+    assert lib.moe_forward(P(s), P(info), ws, need - 256, 4096, 4096, 4096, 4096, None) == -3
+    assert lib.moe_forward(P(s), P(info), ws + 8, need, 4096, 4096, 4096, 4096, None) == -4
+    for fn in ("moe_round_dispatch", "moe_round_gate_up", "moe_round_down", "moe_round_combine"):
+        f = getattr(lib, fn)
+        assert f(P(s), P(info), ws, need - 256, 0, 4096, None) == -3
+        assert f(P(s), P(info), ws + 64, need, 0, 4096, None) == -4
