@@ -100,18 +100,22 @@ def oracle_sample_plan(w, host, budget_s):
                  f"router/top-k/plan; throughput counts the sampled tokens")
 
 
-def cpu_baseline(w, steps=1, budget_s=15.0):
+def cpu_baseline(w, min_seconds=10.0, budget_s=15.0, max_steps=50):
+    """The oracle as it stands on the host cores: repeated steps (each the full workload, or
+    a seeded token sample when the full workload would exceed `budget_s`) until at least
+    `min_seconds` of CPU work has been timed."""
     host = host_inputs(w)
     tok, sample = oracle_sample_plan(w, host, budget_s)
     n_tok = w.T if tok is None else len(tok)
     times = []
-    for _ in range(max(1, steps)):
+    while sum(times) < min_seconds and len(times) < max_steps:
         t0 = time.perf_counter()
         oracle_step(w, host, tokens=tok)
         times.append(time.perf_counter() - t0)
     total = sum(times)
     return {"value": n_tok * len(times) / total, "unit": UNIT, "cores": blas_threads(),
-            "kind": "oracle", "sample": sample, "seconds_per_step": total / len(times)}
+            "kind": "oracle", "sample": f"{sample}; {len(times)} steps, {total:.1f} s",
+            "seconds_per_step": total / len(times)}
 
 
 def run_reference(args, w):
@@ -302,9 +306,23 @@ def main():
     if layer.device_status() != 0:
         raise SystemExit("kernel wait timed out during warm-up")
 
-    clocks = ClockSampler(local)
+    # nvidia-smi samples every 100 ms, longer than a short timed region: keep the GPU under
+    # the same load (untimed steps) for ~0.5 s on each side so the clock record covers it.
+    def load_for(seconds):
+        t_end = time.perf_counter() + seconds
+        while time.perf_counter() < t_end:
+            step()
+        torch.cuda.synchronize(dev)
+
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = str(local)
+    clocks = ClockSampler(gpu_id)
     clocks.start()
+    load_for(0.6)
     total_ms, launches, _ = timed(args.steps)
+    load_for(0.4)
     clk = clocks.stop()
     if dist is not None:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
