@@ -20,7 +20,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB_PATH = os.path.join(LIB_DIR, "libmoe.so")
 
-SOURCES = ["moe_api.cu", "router.cu", "plan.cu", "dispatch_combine.cu", "grouped_gemm.cu"]
+SOURCES = ["moe_api.cu", "router.cu", "plan.cu", "dispatch_combine.cu", "grouped_gemm.cu",
+           "noalloc.cu"]
 HEADERS = ["kernels.h", "sm100.cuh"]
 
 NVCC_FLAGS = [

@@ -381,6 +381,7 @@ const char* moe_status_string(int status) {
     case MOE_ERR_CUDA: return "CUDA error";
     case MOE_ERR_TIMEOUT: return "a kernel wait timed out";
     case MOE_ERR_NO_DEVICE: return "current device is not sm_100";
+    case MOE_ERR_NOALLOC_LIMIT: return "shape needs more scratch than moe_plan_noalloc's static array";
     default: return "unknown status";
   }
 }

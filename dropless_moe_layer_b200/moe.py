@@ -22,7 +22,7 @@ FLAG_RENORM_TOPK = 1
 
 STATUS = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED_SHAPE",
           -3: "MOE_ERR_WORKSPACE_TOO_SMALL", -4: "MOE_ERR_MISALIGNED", -5: "MOE_ERR_CUDA",
-          -6: "MOE_ERR_TIMEOUT", -7: "MOE_ERR_NO_DEVICE"}
+          -6: "MOE_ERR_TIMEOUT", -7: "MOE_ERR_NO_DEVICE", -8: "MOE_ERR_NOALLOC_LIMIT"}
 
 
 class Shape(ctypes.Structure):
@@ -83,6 +83,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_launch_count": (ctypes.c_uint64, []),
         "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
         "moe_profile_read": (ctypes.c_int, [P(c_i32), P(ctypes.c_double)]),
+        "moe_plan_noalloc": (ctypes.c_int, [P(Shape), c_vp, c_vp, c_vp, c_vp, c_vp, P(c_i32), P(c_i32), c_vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

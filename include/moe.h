@@ -67,7 +67,8 @@ typedef enum moe_status {
   MOE_ERR_MISALIGNED = -4,          /* a pointer breaks the alignment rules */
   MOE_ERR_CUDA = -5,                /* a CUDA runtime call failed (includes earlier faults) */
   MOE_ERR_TIMEOUT = -6,             /* a kernel's bounded wait gave up; see moe_device_status */
-  MOE_ERR_NO_DEVICE = -7            /* current device is not an sm_100 GPU */
+  MOE_ERR_NO_DEVICE = -7,           /* current device is not an sm_100 GPU */
+  MOE_ERR_NOALLOC_LIMIT = -8        /* moe_plan_noalloc: shape needs more than its static scratch */
 } moe_status;
 
 /* moe_shape_t.flags */
@@ -184,6 +185,33 @@ MOE_API uint64_t moe_launch_count(void);
 #define MOE_PROFILE_KINDS 7
 MOE_API int moe_profile_enable(int on);
 MOE_API int moe_profile_read(int32_t counts[MOE_PROFILE_KINDS], double ms[MOE_PROFILE_KINDS]);
+
+/* Routing and round plan with no device allocation at all.
+ *
+ * The pages have no counterpart to this call; it exists for callers that cannot
+ * allocate device memory when they route a batch: code running under a memory pool
+ * that already owns the device, plugins that a host framework hands only their input
+ * and output buffers, or services that forbid cudaMalloc after start-up. moe_plan()
+ * needs a caller-allocated workspace; this call keeps the planner's scratch in one
+ * static device array of MOE_NOALLOC_SCRATCH_BYTES inside the library instead. Every
+ * GPU that loads the library holds that array until the process exits.
+ *
+ *   logits   [T, E] fp32 device input (the router-GEMM form is not offered here);
+ *   topk_idx [T, k] int32, gate [T, k] fp32, round [T, k] int32, slot [T, k] int32:
+ *            device outputs, identical to what moe_plan() writes into its workspace;
+ *   R        host out: the number of rounds; load: host out [E] (may be NULL).
+ * Returns MOE_ERR_NOALLOC_LIMIT, launching nothing, when the shape's scratch
+ * (about 8*T*k + 8*ceil(T/C)*E + 4*ceil(T/256)*E bytes) exceeds the array. Calls no
+ * cudaMalloc, cudaFree or other allocating routine. The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress) with that device
+ * current; make that first call before any stream capture. All calls share the array
+ * and each one clears what must start at zero, but calls whose GPU work overlaps
+ * (other streams, other threads) race on it. Synchronizes `stream` once, like
+ * moe_plan(). */
+#define MOE_NOALLOC_SCRATCH_BYTES (16u << 20)
+MOE_API int moe_plan_noalloc(const moe_shape_t* shape, const float* logits, int32_t* topk_idx,
+                             float* gate, int32_t* round, int32_t* slot, int32_t* R,
+                             int32_t* load, moe_stream_t stream);
 
 #ifdef __cplusplus
 }
