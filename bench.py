@@ -228,6 +228,23 @@ def combine_bytes(w, round_np):
     return rows + writes + reads
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def max_over_ranks(value, dist=None, device="cpu"):
+    """The job's time: the maximum of `value` over all ranks (identity on one rank)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank, steps, world, job_ms):
+    """Whole-job tokens/s: the tokens all ranks processed divided by the job time."""
+    return tokens_per_rank * world * steps / (job_ms / 1e3)
+
+
 # ----------------------------------------------------------------------------- GPU benchmark
 
 def main():
@@ -324,11 +341,8 @@ def main():
     total_ms, launches, _ = timed(args.steps)
     load_for(0.4)
     clk = clocks.stop()
-    if dist is not None:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = w.T * world * args.steps / (total_ms / 1e3)
+    total_ms = max_over_ranks(total_ms, dist, dev)
+    value = job_throughput(w.T, args.steps, world, total_ms)
 
     # second timed pass with per-kernel events (for the roofline of the dominant kernel)
     _, _, prof = timed(args.steps, profile=True)
@@ -383,11 +397,8 @@ def main():
         ev1.record(stream)
         ev1.synchronize()
         e2e_ms += ev0.elapsed_time(ev1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = w.T * world * args.steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+    e2e_value = job_throughput(w.T, args.steps, world, e2e_ms)
     status = layer.device_status()
 
     cpu = None
