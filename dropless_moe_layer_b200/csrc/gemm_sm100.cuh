@@ -1,0 +1,420 @@
+// gemm_sm100.cuh - device side of the grouped expert GEMM on the 5th-generation tensor
+// cores (launched by grouped_gemm.cu).
+//
+// "Frontier Pre-training at Microsoft AI (MAI-Base-2)", Key claims, item on reducing
+// per-expert overhead [section "Reducing per-expert overhead"]: the experts of a group run
+// as one grouped GEMM. One GEMM phase covers every expert with rows in the round; expert e
+// multiplies its n[r][e] rows of the fixed [E, C, K] round buffer by its own weights.
+//
+// CTA layout (192 threads, one CTA per SM, persistent over tiles):
+//   warp 0      TMA producer: 3-D tiled loads (128-byte swizzle, no multicast) of the
+//               A tile (128 rows x 64 K) and the B tile into a 192 KB shared-memory ring of
+//               4 to 8 stages (more stages when the tile is narrower).
+//   warp 1      MMA issuer: one thread issues tcgen05.mma.cta_group::1.kind::f16 (bf16 x
+//               bf16 -> fp32, M = 128, N = bn <= 256, K = 16) into a TMEM accumulator;
+//               tcgen05.commit frees each stage and, after the last K block, hands the
+//               accumulator to the epilogue.
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
+//               32*(w%4)..+31, one output row per thread), the phase's math, 16-byte stores.
+// Two accumulators of 256 TMEM columns alternate, so tile i's epilogue overlaps tile i+1's
+// main loop. The pipeline counters live in the role threads (struct Pipe).
+//
+// Tiles are (group, 128-row block, N block). The N width is chosen per launch: the widest
+// candidate that still gives every SM a tile, else the narrowest, so thin rounds (few active
+// experts) spread over more SMs. Rows of a tile past the group's row count read
+// stale rows or TMA zero fill; they reach only accumulator rows that are never stored (an
+// MMA output row depends on its own A row only).
+//
+// Modes: SwiGLU (B = `width` rows of W1 (gate) stacked on the same rows of W3 (up), one MMA
+// of N = 2 * width; out = bf16(silu(gate) * up)), Bf16Out (out = bf16(A B^T)) and F32Bias
+// (out = fp32 A B^T + bias, for the router logits).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace gemm {
+
+using namespace sm100;
+
+constexpr int BM = 128;
+constexpr int BK = 64;            // bf16 elements in one 128-byte swizzle row
+constexpr int UMMA_K = 16;
+constexpr int kStages = 4;
+constexpr int kABytes = BM * BK * 2;
+constexpr int kBMaxRows = 256;
+constexpr int kStageBytes = kABytes + kBMaxRows * BK * 2;   // 48 KB
+constexpr int kAccCols = 256;
+constexpr int kTmemCols = 512;
+constexpr int kMaxGroups = MOE_MAX_E_PLAN;
+constexpr int kThreads = 192;
+constexpr int kMaxStages = 8;
+constexpr int kRingBytes = kStages * kStageBytes;           // 192 KB, re-cut per phase width
+constexpr int kBarBytes = (2 * kMaxStages + 5) * 8;
+constexpr int kMiscWords = 8;
+constexpr int kSmemBytes = 1024 + kRingBytes + kBarBytes + kMiscWords * 4 + 2 * (kMaxGroups + 1) * 4;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+
+enum Mode : int { kSwiGLU = 0, kBf16Out = 1, kF32Bias = 2 };
+
+struct Smem {
+  uint8_t* stage;
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* tfull;
+  uint64_t* tempty;
+  uint64_t* drain;
+  uint32_t* tmem_holder;
+  volatile int* abort;      // raised by any role of this CTA that gives up
+  int* width_idx;           // [2] chosen width of the two planned phases
+  int* tile_start[2];       // [groups + 1] tile prefix of the two planned phases
+};
+
+__device__ __forceinline__ Smem carve(uint8_t* raw) {
+  Smem s;
+  uint8_t* base = raw + ((1024u - (smem_addr(raw) & 1023u)) & 1023u);
+  s.stage = base;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kRingBytes);
+  s.full = bars;
+  s.empty = bars + kMaxStages;
+  s.tfull = bars + 2 * kMaxStages;
+  s.tempty = s.tfull + 2;
+  s.drain = s.tempty + 2;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(s.drain + 1);
+  s.tmem_holder = misc;
+  s.abort = reinterpret_cast<volatile int*>(misc + 1);
+  s.width_idx = reinterpret_cast<int*>(misc + 2);
+  s.tile_start[0] = reinterpret_cast<int*>(misc + kMiscWords);
+  s.tile_start[1] = s.tile_start[0] + kMaxGroups + 1;
+  return s;
+}
+
+// CTA set-up: barriers (thread 0) and the TMEM accumulators (warp 1). Ends synchronised.
+__device__ __forceinline__ uint32_t setup(const Smem& s) {
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kMaxStages; ++i) {
+      mbar_init(smem_addr(&s.full[i]), 1);
+      mbar_init(smem_addr(&s.empty[i]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_addr(&s.tfull[a]), 1);
+      mbar_init(smem_addr(&s.tempty[a]), 128);
+    }
+    mbar_init(smem_addr(s.drain), 1);
+    *s.abort = 0;
+    mbar_fence_init();
+  }
+  __syncwarp();   // every warp reconverges before the (aligned) CTA barrier
+  if ((threadIdx.x >> 5) == 1) {
+    tmem_alloc(smem_addr(s.tmem_holder), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  return *s.tmem_holder;
+}
+
+// CTA tear-down after every role is done: frees the TMEM accumulators.
+__device__ __forceinline__ void release_tmem(uint32_t tmem_base) {
+  if ((threadIdx.x >> 5) == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// One grouped GEMM.
+struct Phase {
+  int mode;
+  const CUtensorMap* a;
+  const CUtensorMap* b[3];     // B maps, one per candidate width
+  int widths[3];               // candidate N widths (SwiGLU: gate columns), widest first; 0 = none
+  int width_idx;               // >= 0: use widths[width_idx]; < 0: pick on the device
+  const int32_t* rows;         // rows of each group (device), or nullptr: rows_const for all
+  int rows_const;
+  int groups;
+  int num_k_blocks;            // K / 64
+  int n_total;                 // output columns (SwiGLU: d_ff)
+  int b_second_row;            // SwiGLU: first row of W3 inside B (= d_ff)
+  void* out;
+  long long out_group_stride;  // elements
+  int out_ld;                  // elements
+  const float* bias;           // F32Bias
+  int n_valid;                 // F32Bias: stored columns
+};
+
+// Pipeline counters; each role thread uses its own fields, and they persist across phases.
+struct Pipe {
+  int stage = 0;
+  uint32_t phase = 0;
+  int acc = 0;
+  uint32_t acc_phase = 0;
+  uint32_t issued = 0, issued_parity = 0;   // producer: stages with loads in flight
+};
+
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+// Warp 0 picks the phase's N width and writes its tile prefix into slot `which`.
+// The caller synchronises the CTA before run_phase.
+__device__ __forceinline__ void plan_phase(const Smem& s, const Phase& p, int which) {
+  if ((threadIdx.x >> 5) != 0) return;
+  const int lane = threadIdx.x & 31;
+  int mt = 0;
+  for (int g = lane; g < p.groups; g += 32) {
+    const int rows = p.rows ? p.rows[g] : p.rows_const;
+    mt += (rows + BM - 1) / BM;
+  }
+  mt = warp_sum(mt);
+  int wi = p.width_idx;          // chosen by the host when it knows the row counts
+  if (wi < 0) {
+    int last = -1;
+    for (int i = 0; i < 3; ++i) {
+      const int w = p.widths[i];
+      if (w <= 0 || p.n_total % w != 0) continue;
+      last = i;
+      if (static_cast<long long>(mt) * (p.n_total / w) >= gridDim.x) {
+        wi = i;
+        break;
+      }
+    }
+    if (wi < 0) wi = last;
+  }
+  const int n_tiles = p.n_total / p.widths[wi];
+  int* ts = s.tile_start[which];
+  int running = 0;
+  for (int g0 = 0; g0 < p.groups; g0 += 32) {
+    const int g = g0 + lane;
+    int cnt = 0;
+    if (g < p.groups) {
+      const int rows = p.rows ? p.rows[g] : p.rows_const;
+      cnt = ((rows + BM - 1) / BM) * n_tiles;
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (g < p.groups) ts[g] = running + incl - cnt;
+    running += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) {
+    ts[p.groups] = running;
+    s.width_idx[which] = wi;
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + __expf(-a)); }
+
+// Runs the CTA's share of the tiles of the phase planned in slot `which`. Returns when this
+// warp's role work is issued/done (the epilogue warps return after their last store). Every warp
+// leaves converged: a CTA barrier (which requires whole warps) may follow directly.
+__device__ __forceinline__ void run_phase(const Smem& s, uint32_t tmem_base, const Phase& p, int which,
+                                          Pipe& pipe, int32_t* status) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int* ts = s.tile_start[which];
+  const int wi = s.width_idx[which];
+  const int width = p.widths[wi];
+  const int bn = p.mode == kSwiGLU ? 2 * width : width;
+  const int n_tiles = p.n_total / width;
+  const int total = ts[p.groups];
+  // the 192 KB ring is cut into as many stages as this width allows (4 at N = 256, 8 at N <= 64)
+  const int stage_bytes = kABytes + bn * BK * 2;
+  const int nstages = min(kMaxStages, kRingBytes / stage_bytes);
+  auto decode = [&](int tile, int& g, int& mt, int& nt) {
+    int lo = 0, hi = p.groups - 1;   // largest g with ts[g] <= tile
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (ts[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    g = lo;
+    const int local = tile - ts[g];
+    mt = local / n_tiles;
+    nt = local - mt * n_tiles;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    const CUtensorMap* mb = p.b[wi];
+    const uint32_t tx = static_cast<uint32_t>(kABytes + bn * BK * 2);
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      int g, mt, nt;
+      decode(tile, g, mt, nt);
+      for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+        if (!mbar_wait(smem_addr(&s.empty[pipe.stage]), pipe.phase ^ 1u, s.abort)) {
+          ok = false;
+          break;
+        }
+        const uint32_t sA = smem_addr(s.stage + pipe.stage * stage_bytes);
+        const uint32_t sB = sA + kABytes;
+        const uint32_t fb = smem_addr(&s.full[pipe.stage]);
+        mbar_arrive_expect_tx(fb, tx);
+        tma_load_3d(sA, p.a, fb, kb * BK, mt * BM, g);
+        if (p.mode == kSwiGLU) {
+          tma_load_3d(sB, mb, fb, kb * BK, nt * width, g);
+          tma_load_3d(sB + width * BK * 2, mb, fb, kb * BK, p.b_second_row + nt * width, g);
+        } else {
+          tma_load_3d(sB, mb, fb, kb * BK, nt * width, g);
+        }
+        pipe.issued |= 1u << pipe.stage;
+        pipe.issued_parity = (pipe.issued_parity & ~(1u << pipe.stage)) | (pipe.phase << pipe.stage);
+        if (++pipe.stage == nstages) {
+          pipe.stage = 0;
+          pipe.phase ^= 1u;
+        }
+      }
+    }
+    if (!ok) {
+      atomicOr(status, kStatusTimeoutProducer);
+      *s.abort = 1;
+      for (int i = 0; i < nstages; ++i)   // let issued loads land before shared memory is reused
+        if ((pipe.issued >> i) & 1u) mbar_wait(smem_addr(&s.full[i]), (pipe.issued_parity >> i) & 1u, nullptr);
+    }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+    // ---------------------------------------------------------------- MMA issuer
+    const uint32_t idesc = idesc_bf16_f32(BM, bn);
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      if (!mbar_wait(smem_addr(&s.tempty[pipe.acc]), pipe.acc_phase ^ 1u, s.abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(pipe.acc * kAccCols);
+      for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+        if (!mbar_wait(smem_addr(&s.full[pipe.stage]), pipe.phase, s.abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sA = smem_addr(s.stage + pipe.stage * stage_bytes);
+        const uint64_t adesc = smem_desc_sw128(sA);
+        const uint64_t bdesc = smem_desc_sw128(sA + kABytes);
+#pragma unroll
+        for (int kk = 0; kk < BK / UMMA_K; ++kk)   // +32 bytes along K per step
+          mma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+        mma_commit(smem_addr(&s.empty[pipe.stage]));
+        if (++pipe.stage == nstages) {
+          pipe.stage = 0;
+          pipe.phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      mma_commit(smem_addr(&s.tfull[pipe.acc]));
+      pipe.acc ^= 1;
+      if (pipe.acc == 0) pipe.acc_phase ^= 1u;
+    }
+    if (!ok) {
+      atomicOr(status, kStatusTimeoutMma);
+      *s.abort = 1;
+      mma_commit(smem_addr(s.drain));   // wait for every MMA already issued
+      mbar_wait(smem_addr(s.drain), 0, nullptr);
+    }
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int g, mt, nt;
+      decode(tile, g, mt, nt);
+      // every lane waits; the outcome is made warp-uniform before the warp-wide TMEM loads
+      const bool ready = __all_sync(0xffffffffu, mbar_wait(smem_addr(&s.tfull[pipe.acc]), pipe.acc_phase, s.abort));
+      if (!ready) {
+        if (lane == 0) atomicOr(status, kStatusTimeoutEpilogue);
+        *s.abort = 1;
+        break;
+      }
+      tc_fence_after();
+      const int row = mt * BM + q * 32 + lane;
+      const int rows_g = p.rows ? p.rows[g] : p.rows_const;
+      const bool valid = row < rows_g;
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                          static_cast<uint32_t>(pipe.acc * kAccCols);
+      if (p.mode == kSwiGLU) {
+        uint16_t* orow = static_cast<uint16_t*>(p.out) + g * p.out_group_stride +
+                         static_cast<long long>(row) * p.out_ld + nt * width;
+        for (int c = 0; c < width; c += 32) {
+          uint32_t gv[32], uv[32];
+          tmem_ld32(tb + c, gv);
+          tmem_ld32(tb + width + c, uv);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float h0 = silu_f(__uint_as_float(gv[2 * i])) * __uint_as_float(uv[2 * i]);
+            const float h1 = silu_f(__uint_as_float(gv[2 * i + 1])) * __uint_as_float(uv[2 * i + 1]);
+            pk[i] = pack_bf16x2(h0, h1);
+          }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+      } else if (p.mode == kBf16Out) {
+        uint16_t* orow = static_cast<uint16_t*>(p.out) + g * p.out_group_stride +
+                         static_cast<long long>(row) * p.out_ld + nt * width;
+        for (int c = 0; c < bn; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tb + c, v);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+      } else {
+        float* orow = static_cast<float*>(p.out) + static_cast<long long>(row) * p.out_ld;
+        for (int c = 0; c < bn; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tb + c, v);
+          tmem_wait_ld();
+          if (valid) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int col = nt * width + c + i;
+              if (col < p.n_valid) orow[col] = __uint_as_float(v[i]) + (p.bias ? p.bias[col] : 0.f);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_addr(&s.tempty[pipe.acc]));
+      pipe.acc ^= 1;
+      if (pipe.acc == 0) pipe.acc_phase ^= 1u;
+    }
+    __syncwarp();
+  }
+}
+
+// Host side: tensor maps (cached) for a 3-D bf16 tensor [groups][rows][inner], box = 64 x
+// box_rows x 1, 128-byte swizzle, zero fill out of bounds.
+cudaError_t make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                     uint64_t groups, uint32_t box_rows);
+
+}  // namespace gemm
+}  // namespace moe

@@ -6,7 +6,31 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#ifndef MOE_PDL
+#define MOE_PDL 1   // 0: plain stream-ordered launches (the kernels' dependency waits are no-ops)
+#endif
+
 namespace moe {
+
+// Launch `kernel` with programmatic stream serialization: it may begin (and run its
+// prologue) while the previous kernel in the stream drains. Every kernel of this library
+// calls grid_dependency_wait() before it touches memory that an earlier kernel writes or
+// reads, so stream order is preserved for data; only launch latency is hidden.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = MOE_PDL;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
 
 // Workspace status word bits (header[kHdrStatus]).
 enum : int {
@@ -76,13 +100,16 @@ cudaError_t launch_combine(const uint16_t* buf, float* y, const int32_t* idx, co
 
 // ---- grouped GEMMs (grouped_gemm.cu)
 // gate_up: h[e][s] = bf16(silu(buf[e][s] W1_e^T) * (buf[e][s] W3_e^T)), s < n_dev[e]
+// n_dev: rows per expert this round on the device (read by the kernel); n_host: the same on
+// the host (picks the tile width and the grid).
 cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint16_t* h,
                            const int32_t* n_dev, const int32_t* n_host, int E, int C, int d, int F,
                            int32_t* status, cudaStream_t stream);
 // down: out[e][s] = bf16(h[e][s] W2_e^T), s < n_dev[e]
-cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out,
-                        const int32_t* n_dev, const int32_t* n_host, int E, int C, int d, int F,
-                        int32_t* status, cudaStream_t stream);
+cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out, const int32_t* n_dev,
+                        const int32_t* n_host, int E, int C, int d, int F, int32_t* status,
+                        cudaStream_t stream);
+
 // router GEMM: logits[t][e] = x[t] . w_router[e] + bias[e] (fp32 out)
 cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* w_router, const float* bias,
                                float* logits, int T, int d, int E, int32_t* status,

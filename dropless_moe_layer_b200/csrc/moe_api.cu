@@ -189,9 +189,8 @@ int do_gate_up(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
   int rows = 0;
   round_rows(s, info, r, n_host, &rows);
   return cuda_status(launch_gate_up(at<uint16_t>(ws, L.buf), w13, at<uint16_t>(ws, L.h),
-                                    at<int32_t>(ws, L.n) + static_cast<size_t>(r) * s->E, n_host,
-                                    s->E, s->C, s->d, s->d_ff,
-                                    at<int32_t>(ws, L.header) + kHdrStatus, stream));
+                                    at<int32_t>(ws, L.n) + static_cast<size_t>(r) * s->E, n_host, s->E,
+                                    s->C, s->d, s->d_ff, at<int32_t>(ws, L.header) + kHdrStatus, stream));
 }
 
 int do_down(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
@@ -201,8 +200,7 @@ int do_down(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
   round_rows(s, info, r, n_host, &rows);
   return cuda_status(launch_down(at<uint16_t>(ws, L.h), w2, at<uint16_t>(ws, L.buf),
                                  at<int32_t>(ws, L.n) + static_cast<size_t>(r) * s->E, n_host, s->E,
-                                 s->C, s->d, s->d_ff, at<int32_t>(ws, L.header) + kHdrStatus,
-                                 stream));
+                                 s->C, s->d, s->d_ff, at<int32_t>(ws, L.header) + kHdrStatus, stream));
 }
 
 int do_combine(const moe_shape_t* s, void* ws, const moe_workspace_layout_t& L, int r, float* y,

@@ -22,6 +22,7 @@
 //                     pair's row in the round-major list (source token, destination
 //                     e * C + slot) that dispatch copies from.
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace moe {
 
@@ -35,6 +36,8 @@ __global__ void __launch_bounds__(kTPB) plan_count_kernel(const int32_t* __restr
                                                           int32_t* __restrict__ block_base) {
   __shared__ int cnt[MOE_MAX_E_PLAN];
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  sm100::grid_dependency_wait();
+  sm100::grid_launch_dependents();
   __syncthreads();
   const int t = blockIdx.x * kTPB + threadIdx.x;
   if (t < T) {
@@ -78,6 +81,8 @@ __global__ void __launch_bounds__(kTPB) plan_scan_kernel(int32_t* __restrict__ b
   __shared__ int chunk_total;
   const int e = blockIdx.x;
   int carry = 0;
+  sm100::grid_dependency_wait();
+  sm100::grid_launch_dependents();
   for (int b0 = 0; b0 < blocks; b0 += kTPB) {
     const int b = b0 + threadIdx.x;
     const int c = b < blocks ? block_base[static_cast<size_t>(b) * E + e] : 0;
@@ -103,6 +108,8 @@ __global__ void __launch_bounds__(kTPB) plan_finalize_kernel(const int32_t* __re
   __shared__ int s_load[MOE_MAX_E_PLAN];
   __shared__ int s_max;
   const int e = threadIdx.x;
+  sm100::grid_dependency_wait();
+  sm100::grid_launch_dependents();
   const int le = e < E ? load[e] : 0;
   if (e < MOE_MAX_E_PLAN) s_load[e] = le;
   if (threadIdx.x == 0) s_max = 0;
@@ -166,6 +173,8 @@ __global__ void __launch_bounds__(kTPB) plan_rank_kernel(const int32_t* __restri
   __shared__ uint32_t mask[kWarps][MOE_MAX_E_PLAN];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) mask[i / E][i % E] = 0u;
+  sm100::grid_dependency_wait();
+  sm100::grid_launch_dependents();
   __syncthreads();
   const int t = blockIdx.x * kTPB + threadIdx.x;
   const bool valid = t < T;
@@ -195,15 +204,19 @@ cudaError_t launch_plan(const PlanBuffers& b, int T, int k, int E, int C, int ma
                         cudaStream_t stream) {
   const int blocks = (T + kTPB - 1) / kTPB;
   launch_begin(kKindPlan, stream);
-  if (blocks > 0) plan_count_kernel<<<blocks, kTPB, 0, stream>>>(b.idx, T, k, E, b.block_base);
-  plan_scan_kernel<<<E, kTPB, 0, stream>>>(b.block_base, blocks, E, b.load);
-  plan_finalize_kernel<<<1, kTPB, 0, stream>>>(b.load, E, C, max_rounds, b.offsets, b.header, b.n,
-                                               b.row_off, b.row_start);
-  if (blocks > 0)
-    plan_rank_kernel<<<blocks, kTPB, 0, stream>>>(b.idx, T, k, E, C, b.block_base, b.row_off,
-                                                  b.round, b.slot, b.row_token, b.row_dst);
+  cudaError_t err = cudaSuccess;
+  if (blocks > 0 && err == cudaSuccess)
+    err = launch_pdl(plan_count_kernel, dim3(blocks), dim3(kTPB), 0, stream, b.idx, T, k, E, b.block_base);
+  if (err == cudaSuccess)
+    err = launch_pdl(plan_scan_kernel, dim3(E), dim3(kTPB), 0, stream, b.block_base, blocks, E, b.load);
+  if (err == cudaSuccess)
+    err = launch_pdl(plan_finalize_kernel, dim3(1), dim3(kTPB), 0, stream, b.load, E, C, max_rounds,
+                     b.offsets, b.header, b.n, b.row_off, b.row_start);
+  if (blocks > 0 && err == cudaSuccess)
+    err = launch_pdl(plan_rank_kernel, dim3(blocks), dim3(kTPB), 0, stream, b.idx, T, k, E, C,
+                     b.block_base, b.row_off, b.round, b.slot, b.row_token, b.row_dst);
   launch_end(kKindPlan, stream, blocks > 0 ? 4 : 2);
-  return cudaGetLastError();
+  return err;
 }
 
 }  // namespace moe

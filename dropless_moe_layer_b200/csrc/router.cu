@@ -15,6 +15,7 @@
 #include <climits>
 
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace moe {
 
@@ -25,6 +26,8 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
                                                           float* __restrict__ gate_out) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  sm100::grid_dependency_wait();
+  sm100::grid_launch_dependents();
   if (t >= T) return;
   const float* row = logits + static_cast<size_t>(t) * E;
 
@@ -94,16 +97,11 @@ cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int ren
   const dim3 grid((T + warps_per_block - 1) / warps_per_block), block(32 * warps_per_block);
   launch_begin(kKindTopk, stream);
   const int vpl = (E + 31) / 32;
-  if (vpl <= 1)
-    router_topk_kernel<1><<<grid, block, 0, stream>>>(logits, T, E, k, renorm, idx, gate);
-  else if (vpl <= 2)
-    router_topk_kernel<2><<<grid, block, 0, stream>>>(logits, T, E, k, renorm, idx, gate);
-  else if (vpl <= 4)
-    router_topk_kernel<4><<<grid, block, 0, stream>>>(logits, T, E, k, renorm, idx, gate);
-  else
-    router_topk_kernel<8><<<grid, block, 0, stream>>>(logits, T, E, k, renorm, idx, gate);
+  auto kern = vpl <= 1 ? router_topk_kernel<1> : vpl <= 2 ? router_topk_kernel<2>
+            : vpl <= 4 ? router_topk_kernel<4> : router_topk_kernel<8>;
+  const cudaError_t err = launch_pdl(kern, grid, block, 0, stream, logits, T, E, k, renorm, idx, gate);
   launch_end(kKindTopk, stream);
-  return cudaGetLastError();
+  return err;
 }
 
 }  // namespace moe

@@ -197,5 +197,40 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+
+// Where a kernel lets its successor launch: 1 = after the kernel's own work (the successor
+// then only hides its launch latency and prologue behind this kernel's tail), 0 = right
+// after this kernel's own dependency wait (the successor's blocks may sit resident, waiting,
+// for the whole of this kernel).
+#ifndef MOE_PDL_LATE_TRIGGER
+#define MOE_PDL_LATE_TRIGGER 1
+#endif
+
+// Block until every grid this one depends on (the previous kernel in the stream when
+// launched with programmatic stream serialization) has completed and its memory is
+// visible. A no-op for a normal launch. Waiting is done by the hardware, not by a spin.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allow the next kernel in the stream to begin launching (its blocks still wait for this
+// grid to complete in grid_dependency_wait before touching its results).
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Trigger points for the two placements above; call both, in this order, in every kernel.
+__device__ __forceinline__ void pdl_trigger_early() {
+#if !MOE_PDL_LATE_TRIGGER
+  grid_launch_dependents();
+#endif
+}
+__device__ __forceinline__ void pdl_trigger_late() {
+#if MOE_PDL_LATE_TRIGGER
+  grid_launch_dependents();
+#endif
+}
+
 }  // namespace sm100
 }  // namespace moe

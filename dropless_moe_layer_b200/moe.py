@@ -59,11 +59,13 @@ def header_symbols() -> list[str]:
     return re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)
 
 
-def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Load libmoe.so (built in-tree by dropless_moe_layer_b200.build). Raises if missing."""
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load libmoe.so (built in-tree by dropless_moe_layer_b200.build, or the file named by
+    the MOE_LIBRARY_PATH environment variable). Raises if it is missing."""
     global _lib
     if _lib is not None:
         return _lib
+    path = path or os.environ.get("MOE_LIBRARY_PATH") or LIB_PATH
     if not os.path.exists(path):
         raise RuntimeError(f"libmoe.so not found at {path}; build it with "
                            "`python -m dropless_moe_layer_b200.build`")

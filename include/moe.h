@@ -141,7 +141,8 @@ MOE_API int moe_plan(const moe_shape_t* shape, const float* logits, const uint16
              const uint16_t* w_router, const float* bias, void* ws, size_t ws_bytes,
              moe_plan_info_t* info, moe_stream_t stream);
 
-/* Executes all R rounds of the plan in `info` (from moe_plan on this `ws`):
+/* Executes all R rounds of the plan in `info` (from moe_plan on this `ws`), four kernels per
+ * round launched with programmatic dependent launch:
  *   x         [T, d] bf16
  *   w_gate_up [E, 2*d_ff, d] bf16: rows 0..d_ff-1 = W1 (gate), rows d_ff..2*d_ff-1 = W3 (up)
  *   w_down    [E, d, d_ff] bf16 (W2)
