@@ -72,7 +72,10 @@ struct CombineArgs {
 };
 
 // The whole warp combines token t for round r (no-op if t has no pair in round r).
-__device__ __forceinline__ void combine_token(const CombineArgs& a, int t, int r) {
+// With `only_expert` >= 0 the warp stands for one row of the round (token t's pair with that
+// expert) and does the work only if that pair is t's first pair in the round, so that every
+// active token is combined exactly once when the round is walked row by row.
+__device__ __forceinline__ void combine_token(const CombineArgs& a, int t, int r, int only_expert = -1) {
   const int lane = threadIdx.x & 31;
   const size_t pbase = static_cast<size_t>(t) * a.k;
   // lane j < k holds pair j's round, expert, slot and gate (four independent loads)
@@ -86,6 +89,7 @@ __device__ __forceinline__ void combine_token(const CombineArgs& a, int t, int r
   }
   const uint32_t here = __ballot_sync(0xffffffffu, my_round == r);
   if (here == 0u) return;
+  if (only_expert >= 0 && __shfl_sync(0xffffffffu, my_idx, __ffs(here) - 1) != only_expert) return;
   const int first_round = __reduce_min_sync(0xffffffffu, my_round);
   const bool fresh = first_round == r;
   const int npairs = __popc(here);

@@ -9,11 +9,12 @@
 // dispatch: one warp per row of the round-major row list (built by the planner, so
 //   the round's rows are one contiguous range with no empty experts to skip); 16-byte
 //   vector loads and stores, eight in flight per lane.
-// combine:  one warp per token. It finds the token's pairs that fall in this round
-//   (ballot over the k round numbers), starts from zero on the token's first round
-//   and from the running y otherwise, and adds gate * out[e][slot] in ascending j.
-//   The order of additions is fixed by (round, j), so y is bitwise reproducible; no
-//   atomics are used.
+// combine:  one warp per token, or, when the round holds fewer rows than there are tokens,
+//   one warp per row of the round (the row of a token's first pair in the round does the
+//   token's work). It finds the token's pairs that fall in this round (ballot over the k
+//   round numbers), starts from zero on the token's first round and from the running y
+//   otherwise, and adds gate * out[e][slot] in ascending j. The order of additions is
+//   fixed by (round, j), so y is bitwise reproducible; no atomics are used.
 #include "copy_phases.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -37,11 +38,21 @@ __global__ void __launch_bounds__(32 * kDispatchWarps)
   sm100::pdl_trigger_late();
 }
 
-__global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const copy::CombineArgs a, int r) {
-  const int t = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+// by_rows == 0: warp w combines token w. by_rows == 1: warp w stands for row w of the round's
+// contiguous row range (fewer warps when the round holds fewer rows than there are tokens).
+__global__ void __launch_bounds__(32 * kCombineWarps)
+    combine_kernel(const copy::CombineArgs a, int r, int by_rows, const int32_t* __restrict__ row_start,
+                   const int32_t* __restrict__ row_token, const int32_t* __restrict__ row_dst) {
+  const int w = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+  int t = w, expert = -1;
+  if (by_rows) {                       // plan data: written before this forward
+    const int row = row_start[r] + w;
+    t = row < row_start[r + 1] ? row_token[row] : a.T;
+    if (t < a.T) expert = row_dst[row] / a.C;
+  }
   sm100::grid_dependency_wait();      // buf comes from the round's down GEMM, y from earlier rounds
   sm100::pdl_trigger_early();
-  if (t < a.T) copy::combine_token(a, t, r);
+  if (t < a.T) copy::combine_token(a, t, r, expert);
   sm100::pdl_trigger_late();
 }
 
@@ -64,13 +75,18 @@ cudaError_t launch_dispatch(const uint16_t* x, uint16_t* buf, const int32_t* row
 }
 
 cudaError_t launch_combine(const uint16_t* buf, float* y, const int32_t* idx, const float* gate,
-                           const int32_t* round, const int32_t* slot, int T, int k, int C, int d,
-                           int r, cudaStream_t stream) {
+                           const int32_t* round, const int32_t* slot, const int32_t* row_start,
+                           const int32_t* row_token, const int32_t* row_dst, int T, int k, int C, int d,
+                           int r, int rows, cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
-  const int blocks = (T + kCombineWarps - 1) / kCombineWarps;
+  const int by_rows = rows < T ? 1 : 0;
+  const int warps = by_rows ? rows : T;
+  if (warps <= 0) return cudaSuccess;
+  const int blocks = (warps + kCombineWarps - 1) / kCombineWarps;
   launch_begin(kKindCombine, stream);
   const copy::CombineArgs a{buf, y, idx, gate, round, slot, T, k, C, d};
-  const cudaError_t err = launch_pdl(combine_kernel, dim3(blocks), dim3(32 * kCombineWarps), 0, stream, a, r);
+  const cudaError_t err = launch_pdl(combine_kernel, dim3(blocks), dim3(32 * kCombineWarps), 0, stream, a, r,
+                                     by_rows, row_start, row_token, row_dst);
   launch_end(kKindCombine, stream);
   return err;
 }

@@ -94,9 +94,12 @@ cudaError_t launch_plan(const PlanBuffers& b, int T, int k, int E, int C, int ma
 cudaError_t launch_dispatch(const uint16_t* x, uint16_t* buf, const int32_t* row_start,
                             const int32_t* row_token, const int32_t* row_dst, int r, int rows,
                             int d, cudaStream_t stream);
+// rows: rows of round r (host copy); the kernel walks the round's rows instead of all T
+// tokens when there are fewer of them.
 cudaError_t launch_combine(const uint16_t* buf, float* y, const int32_t* idx, const float* gate,
-                           const int32_t* round, const int32_t* slot, int T, int k, int C, int d,
-                           int r, cudaStream_t stream);
+                           const int32_t* round, const int32_t* slot, const int32_t* row_start,
+                           const int32_t* row_token, const int32_t* row_dst, int T, int k, int C, int d,
+                           int r, int rows, cudaStream_t stream);
 
 // ---- grouped GEMMs (grouped_gemm.cu)
 // gate_up: h[e][s] = bf16(silu(buf[e][s] W1_e^T) * (buf[e][s] W3_e^T)), s < n_dev[e]

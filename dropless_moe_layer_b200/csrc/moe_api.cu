@@ -203,11 +203,16 @@ int do_down(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
                                  s->C, s->d, s->d_ff, at<int32_t>(ws, L.header) + kHdrStatus, stream));
 }
 
-int do_combine(const moe_shape_t* s, void* ws, const moe_workspace_layout_t& L, int r, float* y,
-               cudaStream_t stream) {
+int do_combine(const moe_shape_t* s, const moe_plan_info_t* info, void* ws, const moe_workspace_layout_t& L,
+               int r, float* y, cudaStream_t stream) {
+  int32_t n_host[MOE_MAX_EXPERTS];
+  int rows = 0;
+  round_rows(s, info, r, n_host, &rows);
   return cuda_status(launch_combine(at<uint16_t>(ws, L.buf), y, at<int32_t>(ws, L.topk_idx),
                                     at<float>(ws, L.gate), at<int32_t>(ws, L.round),
-                                    at<int32_t>(ws, L.slot), s->T, s->k, s->C, s->d, r, stream));
+                                    at<int32_t>(ws, L.slot), at<int32_t>(ws, L.row_start),
+                                    at<int32_t>(ws, L.row_token), at<int32_t>(ws, L.row_dst), s->T, s->k,
+                                    s->C, s->d, r, rows, stream));
 }
 
 }  // namespace
@@ -331,7 +336,7 @@ int moe_round_combine(const moe_shape_t* shape, const moe_plan_info_t* info, voi
   if (st != MOE_OK) return st;
   if (r < 0 || r >= info->R || y == nullptr) return MOE_ERR_INVALID_ARG;
   if (!aligned(y, 16)) return MOE_ERR_MISALIGNED;
-  return do_combine(shape, ws, L, r, y, reinterpret_cast<cudaStream_t>(stream));
+  return do_combine(shape, info, ws, L, r, y, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
@@ -349,7 +354,7 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
     if ((st = do_dispatch(shape, info, ws, L, r, x, stream)) != MOE_OK) return st;
     if ((st = do_gate_up(shape, info, ws, L, r, w_gate_up, stream)) != MOE_OK) return st;
     if ((st = do_down(shape, info, ws, L, r, w_down, stream)) != MOE_OK) return st;
-    if ((st = do_combine(shape, ws, L, r, y, stream)) != MOE_OK) return st;
+    if ((st = do_combine(shape, info, ws, L, r, y, stream)) != MOE_OK) return st;
   }
   return MOE_OK;
 }
