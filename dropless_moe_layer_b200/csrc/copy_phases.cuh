@@ -101,9 +101,13 @@ __device__ __forceinline__ void combine_token(const CombineArgs& a, int t, int r
   const unsigned long long prow = lane < npairs ? static_cast<unsigned long long>(e_p) * a.C + s_p : 0ull;
   const float pgate = lane < npairs ? g_p : 0.f;
   float* yrow = a.y + static_cast<size_t>(t) * a.d;
-  for (int c = lane * 8; c < a.d; c += 32 * 8) {
+  // Every lane runs the same iterations (the shuffles below need the whole warp); lanes past
+  // the end of the row (d < 256) only skip the loads and stores.
+  for (int c0 = 0; c0 < a.d; c0 += 32 * 8) {
+    const int c = c0 + lane * 8;
+    const bool col = c < a.d;
     float acc[8];
-    if (fresh) {
+    if (fresh || !col) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
     } else {
@@ -120,7 +124,7 @@ __device__ __forceinline__ void combine_token(const CombineArgs& a, int t, int r
         const int p = p0 + u;
         const unsigned long long row = __shfl_sync(0xffffffffu, prow, p & 31);
         g[u] = __shfl_sync(0xffffffffu, pgate, p & 31);
-        q[u] = p < npairs ? *reinterpret_cast<const uint4*>(a.buf + row * a.d + c) : make_uint4(0, 0, 0, 0);
+        q[u] = (p < npairs && col) ? *reinterpret_cast<const uint4*>(a.buf + row * a.d + c) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -132,8 +136,10 @@ __device__ __forceinline__ void combine_token(const CombineArgs& a, int t, int r
         }
       }
     }
-    *reinterpret_cast<float4*>(yrow + c) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    *reinterpret_cast<float4*>(yrow + c + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    if (col) {
+      *reinterpret_cast<float4*>(yrow + c) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      *reinterpret_cast<float4*>(yrow + c + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
   }
 }
 

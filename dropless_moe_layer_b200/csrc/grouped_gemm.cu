@@ -1,17 +1,56 @@
-// grouped_gemm.cu - stand-alone launches of the grouped expert GEMM (one round's gate/up or
-// down GEMM, or the router logits GEMM) and the host-side tensor-map cache. The device code
-// is in gemm_sm100.cuh.
+// grouped_gemm.cu - launches of the grouped expert GEMM (one round's gate/up or down GEMM, or
+// the router logits GEMM), optionally carrying the neighbouring round's copy step on extra
+// warps, and the host-side tensor-map cache. The GEMM device code is in gemm_sm100.cuh.
 #include <cuda.h>
 
 #include <atomic>
 #include <mutex>
 
+#include "copy_phases.cuh"
 #include "gemm_sm100.cuh"
 #include "kernels.h"
 
 namespace moe {
 
 namespace gemm {
+
+// Copy work that rides along with a GEMM launch on warps 6..9 ("copy warps"), overlapping
+// the tensor-core work: the previous round's combine next to a gate/up GEMM, the next round's
+// dispatch next to a down GEMM. It shares no data with the GEMM it rides with.
+constexpr int kCopyWarps = 4;
+constexpr int kLaunchThreads = kThreads + 32 * kCopyWarps;
+
+enum SideKind : int { kSideNone = 0, kSideDispatch = 1, kSideCombine = 2 };
+
+struct SideArgs {
+  int kind;
+  int r;                       // round the side work belongs to
+  const int32_t* row_start;
+  const int32_t* row_token;
+  const int32_t* row_dst;
+  const uint4* x;              // dispatch
+  uint4* buf;
+  int vecs;
+  copy::CombineArgs comb;      // combine
+  int by_rows;
+};
+
+__device__ __forceinline__ void side_work(const SideArgs& sa) {
+  const int cw = blockIdx.x * kCopyWarps + ((threadIdx.x >> 5) - kThreads / 32);
+  const int warps = gridDim.x * kCopyWarps;
+  if (sa.kind == kSideDispatch) {
+    copy::dispatch_rows(sa.x, sa.buf, sa.row_token, sa.row_dst, sa.row_start[sa.r], sa.row_start[sa.r + 1],
+                        sa.vecs, cw, warps);
+  } else if (sa.kind == kSideCombine) {
+    if (sa.by_rows) {
+      const int begin = sa.row_start[sa.r], end = sa.row_start[sa.r + 1];
+      for (int row = begin + cw; row < end; row += warps)
+        copy::combine_token(sa.comb, sa.row_token[row], sa.r, sa.row_dst[row] / sa.comb.C);
+    } else {
+      for (int t = cw; t < sa.comb.T; t += warps) copy::combine_token(sa.comb, t, sa.r);
+    }
+  }
+}
 
 struct KernelArgs {
   int mode;
@@ -31,10 +70,10 @@ struct KernelArgs {
   int32_t* status;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kLaunchThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb0,
                         const __grid_constant__ CUtensorMap tb1, const __grid_constant__ CUtensorMap tb2,
-                        const KernelArgs args) {
+                        const KernelArgs args, const SideArgs side) {
   extern __shared__ uint8_t smem_raw[];
   const Smem s = carve(smem_raw);
   if (threadIdx.x == 0) {
@@ -68,7 +107,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   grid_dependency_wait();
   pdl_trigger_early();
   Pipe pipe;
-  run_phase(s, tmem, p, 0, pipe, args.status);
+  if (threadIdx.x < kThreads)
+    run_phase(s, tmem, p, 0, pipe, args.status);
+  else
+    side_work(side);
   tc_fence_before();
   __syncthreads();
   pdl_trigger_late();               // after every role of this CTA is done
@@ -193,8 +235,8 @@ static long long choose_width(const int32_t* n_host, int groups, int rows_const,
 }
 
 static cudaError_t run(const CUtensorMap& a, const CUtensorMap* b, const KernelArgs& args, long long tiles,
-                       int kind, cudaStream_t stream) {
-  if (tiles <= 0) return cudaSuccess;
+                       const SideArgs& side, int kind, cudaStream_t stream) {
+  if (tiles <= 0 && side.kind == kSideNone) return cudaSuccess;
   static std::atomic<uint64_t> configured{0};   // one bit per device ordinal
   int dev = 0;
   cudaGetDevice(&dev);
@@ -206,9 +248,10 @@ static cudaError_t run(const CUtensorMap& a, const CUtensorMap* b, const KernelA
     configured.fetch_or(bit);
   }
   launch_begin(kind, stream);
-  const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
-  const cudaError_t err = launch_pdl(grouped_gemm_kernel, dim3(grid), dim3(kThreads), kSmemBytes, stream,
-                                     a, b[0], b[1], b[2], args);
+  // with side work every SM takes part in the copy; otherwise one CTA per tile, at most one per SM
+  const int grid = side.kind != kSideNone ? num_sms() : static_cast<int>(tiles < num_sms() ? tiles : num_sms());
+  const cudaError_t err = launch_pdl(grouped_gemm_kernel, dim3(grid), dim3(kLaunchThreads), kSmemBytes, stream,
+                                     a, b[0], b[1], b[2], args, side);
   launch_end(kind, stream);
   return err;
 }
@@ -232,9 +275,27 @@ cudaError_t make_down_maps(const uint16_t* h, const uint16_t* w_down, int E, int
   return gemm::make_b_maps(mb, w_down, F, d, E, kDownWidths, d);
 }
 
+static gemm::SideArgs make_side(const RoundCopy* copy) {
+  gemm::SideArgs sd{};
+  sd.kind = gemm::kSideNone;
+  if (copy == nullptr) return sd;
+  sd.kind = copy->combine ? gemm::kSideCombine : gemm::kSideDispatch;
+  sd.r = copy->r;
+  sd.row_start = copy->row_start;
+  sd.row_token = copy->row_token;
+  sd.row_dst = copy->row_dst;
+  sd.x = reinterpret_cast<const uint4*>(copy->x);
+  sd.buf = reinterpret_cast<uint4*>(copy->buf);
+  sd.vecs = copy->d / 8;
+  sd.comb = copy::CombineArgs{copy->out, copy->y, copy->idx, copy->gate, copy->round, copy->slot,
+                              copy->T, copy->k, copy->C, copy->d};
+  sd.by_rows = copy->rows < copy->T ? 1 : 0;
+  return sd;
+}
+
 cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint16_t* h,
                            const int32_t* n_dev, const int32_t* n_host, int E, int C, int d, int F,
-                           int32_t* status, cudaStream_t stream) {
+                           int32_t* status, const RoundCopy* copy, cudaStream_t stream) {
   CUtensorMap ma, mb[3];
   cudaError_t e = make_gate_up_maps(buf, w_gate_up, E, C, d, F, &ma, mb);
   if (e != cudaSuccess) return e;
@@ -251,12 +312,12 @@ cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint1
   a.out_ld = F;
   a.status = status;
   const long long tiles = gemm::choose_width(n_host, E, 0, F, a);
-  return gemm::run(ma, mb, a, tiles, kKindGateUp, stream);
+  return gemm::run(ma, mb, a, tiles, make_side(copy), kKindGateUp, stream);
 }
 
 cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out, const int32_t* n_dev,
                         const int32_t* n_host, int E, int C, int d, int F, int32_t* status,
-                        cudaStream_t stream) {
+                        const RoundCopy* copy, cudaStream_t stream) {
   CUtensorMap ma, mb[3];
   cudaError_t e = make_down_maps(h, w_down, E, C, d, F, &ma, mb);
   if (e != cudaSuccess) return e;
@@ -272,7 +333,7 @@ cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out
   a.out_ld = d;
   a.status = status;
   const long long tiles = gemm::choose_width(n_host, E, 0, d, a);
-  return gemm::run(ma, mb, a, tiles, kKindDown, stream);
+  return gemm::run(ma, mb, a, tiles, make_side(copy), kKindDown, stream);
 }
 
 cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* w_router, const float* bias,
@@ -299,7 +360,7 @@ cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* w_router, cons
   a.bias = bias;
   a.status = status;
   const long long tiles = gemm::choose_width(nullptr, 1, T, bn, a);
-  return gemm::run(ma, mb, a, tiles, kKindRouterGemm, stream);
+  return gemm::run(ma, mb, a, tiles, make_side(nullptr), kKindRouterGemm, stream);
 }
 
 }  // namespace moe

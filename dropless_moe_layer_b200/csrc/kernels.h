@@ -103,15 +103,35 @@ cudaError_t launch_combine(const uint16_t* buf, float* y, const int32_t* idx, co
 
 // ---- grouped GEMMs (grouped_gemm.cu)
 // gate_up: h[e][s] = bf16(silu(buf[e][s] W1_e^T) * (buf[e][s] W3_e^T)), s < n_dev[e]
+// A copy step of a neighbouring round carried by a GEMM launch on extra warps: a dispatch
+// (x -> buf rows of round r) or a combine (gate * out -> y for round r).
+struct RoundCopy {
+  bool combine;
+  int r;
+  int rows;                  // rows of round r (host copy)
+  const int32_t* row_start;
+  const int32_t* row_token;
+  const int32_t* row_dst;
+  const uint16_t* x;         // dispatch
+  uint16_t* buf;
+  const uint16_t* out;       // combine
+  float* y;
+  const int32_t* idx;
+  const float* gate;
+  const int32_t* round;
+  const int32_t* slot;
+  int T, k, C, d;
+};
+
 // n_dev: rows per expert this round on the device (read by the kernel); n_host: the same on
-// the host (picks the tile width and the grid).
+// the host (picks the tile width and the grid). copy: optional side copy step, or null.
 cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint16_t* h,
                            const int32_t* n_dev, const int32_t* n_host, int E, int C, int d, int F,
-                           int32_t* status, cudaStream_t stream);
+                           int32_t* status, const RoundCopy* copy, cudaStream_t stream);
 // down: out[e][s] = bf16(h[e][s] W2_e^T), s < n_dev[e]
 cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out, const int32_t* n_dev,
                         const int32_t* n_host, int E, int C, int d, int F, int32_t* status,
-                        cudaStream_t stream);
+                        const RoundCopy* copy, cudaStream_t stream);
 
 // router GEMM: logits[t][e] = x[t] . w_router[e] + bias[e] (fp32 out)
 cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* w_router, const float* bias,

@@ -117,6 +117,7 @@ void make_layout(const moe_shape_t* s, moe_workspace_layout_t* L) {
   L->row_dst = take(T * k * 4);
   L->buf = take(E * C * s->d * 2);
   L->h = take(E * C * s->d_ff * 2);
+  L->out = take(E * C * s->d * 2);
   L->total_bytes = off;
   L->max_rounds = mr;
   L->plan_blocks = blocks;
@@ -183,24 +184,57 @@ int do_dispatch(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
                                      s->d, stream));
 }
 
+// Copy steps up to this many bytes of rows ride on a GEMM launch (its 4 copy warps per SM);
+// larger ones get their own kernel, which reaches full HBM bandwidth.
+constexpr size_t kFuseCopyBytes = 32ull << 20;
+
+// The copy step of round `cr` carried by a GEMM launch (a combine, or a dispatch of x).
+RoundCopy make_copy(const moe_shape_t* s, const moe_plan_info_t* info, void* ws, const moe_workspace_layout_t& L,
+                    bool combine, int cr, const uint16_t* x, float* y) {
+  int32_t n_host[MOE_MAX_EXPERTS];
+  RoundCopy c{};
+  c.combine = combine;
+  c.r = cr;
+  round_rows(s, info, cr, n_host, &c.rows);
+  c.row_start = at<int32_t>(ws, L.row_start);
+  c.row_token = at<int32_t>(ws, L.row_token);
+  c.row_dst = at<int32_t>(ws, L.row_dst);
+  c.x = x;
+  c.buf = at<uint16_t>(ws, L.buf);
+  c.out = at<uint16_t>(ws, L.out);
+  c.y = y;
+  c.idx = at<int32_t>(ws, L.topk_idx);
+  c.gate = at<float>(ws, L.gate);
+  c.round = at<int32_t>(ws, L.round);
+  c.slot = at<int32_t>(ws, L.slot);
+  c.T = s->T;
+  c.k = s->k;
+  c.C = s->C;
+  c.d = s->d;
+  return c;
+}
+
 int do_gate_up(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
-               const moe_workspace_layout_t& L, int r, const uint16_t* w13, cudaStream_t stream) {
+               const moe_workspace_layout_t& L, int r, const uint16_t* w13, const RoundCopy* copy,
+               cudaStream_t stream) {
   int32_t n_host[MOE_MAX_EXPERTS];
   int rows = 0;
   round_rows(s, info, r, n_host, &rows);
   return cuda_status(launch_gate_up(at<uint16_t>(ws, L.buf), w13, at<uint16_t>(ws, L.h),
                                     at<int32_t>(ws, L.n) + static_cast<size_t>(r) * s->E, n_host, s->E,
-                                    s->C, s->d, s->d_ff, at<int32_t>(ws, L.header) + kHdrStatus, stream));
+                                    s->C, s->d, s->d_ff, at<int32_t>(ws, L.header) + kHdrStatus, copy,
+                                    stream));
 }
 
 int do_down(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
-            const moe_workspace_layout_t& L, int r, const uint16_t* w2, cudaStream_t stream) {
+            const moe_workspace_layout_t& L, int r, const uint16_t* w2, const RoundCopy* copy,
+            cudaStream_t stream) {
   int32_t n_host[MOE_MAX_EXPERTS];
   int rows = 0;
   round_rows(s, info, r, n_host, &rows);
-  return cuda_status(launch_down(at<uint16_t>(ws, L.h), w2, at<uint16_t>(ws, L.buf),
+  return cuda_status(launch_down(at<uint16_t>(ws, L.h), w2, at<uint16_t>(ws, L.out),
                                  at<int32_t>(ws, L.n) + static_cast<size_t>(r) * s->E, n_host, s->E,
-                                 s->C, s->d, s->d_ff, at<int32_t>(ws, L.header) + kHdrStatus, stream));
+                                 s->C, s->d, s->d_ff, at<int32_t>(ws, L.header) + kHdrStatus, copy, stream));
 }
 
 int do_combine(const moe_shape_t* s, const moe_plan_info_t* info, void* ws, const moe_workspace_layout_t& L,
@@ -208,7 +242,7 @@ int do_combine(const moe_shape_t* s, const moe_plan_info_t* info, void* ws, cons
   int32_t n_host[MOE_MAX_EXPERTS];
   int rows = 0;
   round_rows(s, info, r, n_host, &rows);
-  return cuda_status(launch_combine(at<uint16_t>(ws, L.buf), y, at<int32_t>(ws, L.topk_idx),
+  return cuda_status(launch_combine(at<uint16_t>(ws, L.out), y, at<int32_t>(ws, L.topk_idx),
                                     at<float>(ws, L.gate), at<int32_t>(ws, L.round),
                                     at<int32_t>(ws, L.slot), at<int32_t>(ws, L.row_start),
                                     at<int32_t>(ws, L.row_token), at<int32_t>(ws, L.row_dst), s->T, s->k,
@@ -316,7 +350,7 @@ int moe_round_gate_up(const moe_shape_t* shape, const moe_plan_info_t* info, voi
   if (st != MOE_OK) return st;
   if (r < 0 || r >= info->R || w_gate_up == nullptr) return MOE_ERR_INVALID_ARG;
   if (!aligned(w_gate_up, 16)) return MOE_ERR_MISALIGNED;
-  return do_gate_up(shape, info, ws, L, r, w_gate_up, reinterpret_cast<cudaStream_t>(stream));
+  return do_gate_up(shape, info, ws, L, r, w_gate_up, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int moe_round_down(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
@@ -326,7 +360,7 @@ int moe_round_down(const moe_shape_t* shape, const moe_plan_info_t* info, void* 
   if (st != MOE_OK) return st;
   if (r < 0 || r >= info->R || w_down == nullptr) return MOE_ERR_INVALID_ARG;
   if (!aligned(w_down, 16)) return MOE_ERR_MISALIGNED;
-  return do_down(shape, info, ws, L, r, w_down, reinterpret_cast<cudaStream_t>(stream));
+  return do_down(shape, info, ws, L, r, w_down, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int moe_round_combine(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
@@ -350,11 +384,32 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
   if (!aligned(x, 16) || !aligned(w_gate_up, 16) || !aligned(w_down, 16) || !aligned(y, 16))
     return MOE_ERR_MISALIGNED;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  for (int r = 0; r < info->R; ++r) {
-    if ((st = do_dispatch(shape, info, ws, L, r, x, stream)) != MOE_OK) return st;
-    if ((st = do_gate_up(shape, info, ws, L, r, w_gate_up, stream)) != MOE_OK) return st;
-    if ((st = do_down(shape, info, ws, L, r, w_down, stream)) != MOE_OK) return st;
-    if ((st = do_combine(shape, info, ws, L, r, y, stream)) != MOE_OK) return st;
+  // Launch order. A small copy step (a thin round: at most kFuseCopyBytes of rows) rides on
+  // the neighbouring GEMM launch: combine(r-1) on gate/up(r), dispatch(r+1) on down(r). A large
+  // one runs as its own full-bandwidth kernel right after down(r). Each launch depends only on
+  // the one before it (PDL wait), and no two steps of one launch touch the same buffer:
+  // dispatch writes buf, gate/up reads buf and writes h, down reads h and writes out, combine
+  // reads out and updates y. A run of thin rounds thus costs two launches per round.
+  const int R = info->R;
+  if (R == 0) return MOE_OK;
+  auto small = [&](int rr) {
+    int32_t n_host[MOE_MAX_EXPERTS];
+    int rows = 0;
+    round_rows(shape, info, rr, n_host, &rows);
+    return static_cast<size_t>(rows) * shape->d * 2 <= kFuseCopyBytes;
+  };
+  if ((st = do_dispatch(shape, info, ws, L, 0, x, stream)) != MOE_OK) return st;
+  for (int r = 0; r < R; ++r) {
+    const bool fuse_combine = r > 0 && small(r - 1);
+    const RoundCopy comb = make_copy(shape, info, ws, L, true, r > 0 ? r - 1 : 0, x, y);
+    if ((st = do_gate_up(shape, info, ws, L, r, w_gate_up, fuse_combine ? &comb : nullptr, stream)) != MOE_OK)
+      return st;
+    const bool next = r + 1 < R;
+    const bool fuse_dispatch = next && small(r + 1);
+    const RoundCopy disp = make_copy(shape, info, ws, L, false, next ? r + 1 : r, x, y);
+    if ((st = do_down(shape, info, ws, L, r, w_down, fuse_dispatch ? &disp : nullptr, stream)) != MOE_OK) return st;
+    if (next && !fuse_dispatch && (st = do_dispatch(shape, info, ws, L, r + 1, x, stream)) != MOE_OK) return st;
+    if (!(next && small(r)) && (st = do_combine(shape, info, ws, L, r, y, stream)) != MOE_OK) return st;
   }
   return MOE_OK;
 }

@@ -39,7 +39,7 @@ class PlanInfo(ctypes.Structure):
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [(name, c_sz) for name in (
         "total_bytes", "header", "logits", "topk_idx", "gate", "round", "slot", "load",
-        "offsets", "block_base", "n", "row_off", "row_start", "row_token", "row_dst", "buf", "h")
+        "offsets", "block_base", "n", "row_off", "row_start", "row_token", "row_dst", "buf", "h", "out")
     ] + [("max_rounds", c_i32), ("plan_blocks", c_i32)]
 
 
@@ -279,6 +279,11 @@ class DroplessMoE:
         import torch
         s, L = self.shape, self.layout
         return self._view(L.buf, s.E * s.C * s.d, torch.bfloat16).view(s.E, s.C, s.d)
+
+    def output_buffer(self):
+        import torch
+        s, L = self.shape, self.layout
+        return self._view(L.out, s.E * s.C * s.d, torch.bfloat16).view(s.E, s.C, s.d)
 
     def hidden_buffer(self):
         import torch

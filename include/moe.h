@@ -22,7 +22,8 @@
  *   round = rank / C, slot = rank % C, R = ceil(max_e load_e / C)
  *   for r in 0..R-1:
  *     dispatch: buf[e][slot] = x[t] for every pair in round r       (buf: [E, C, d] bf16)
- *     experts:  h = bf16(silu(buf W1^T) * (buf W3^T)); out = bf16(h W2^T)   (grouped GEMMs)
+ *     experts:  h = bf16(silu(buf W1^T) * (buf W3^T)); out = bf16(h W2^T)   (grouped GEMMs,
+ *               out: [E, C, d] bf16)
  *     combine:  y[t] += gate[t,j] * out[e][slot] for the round's pairs, j ascending
  *   y [T, d] fp32 equals the capacity-free dropless MoE output up to bf16 rounding of the
  *   expert intermediates.
@@ -116,8 +117,9 @@ typedef struct moe_workspace_layout {
   size_t row_start;   /* i32 [max_rounds + 1]: first row of round r in the round-major row list */
   size_t row_token;   /* i32 [T * k] round-major row list: source token */
   size_t row_dst;     /* i32 [T * k] round-major row list: destination e * C + slot */
-  size_t buf;         /* bf16 [E, C, d]: dispatch buffer; also the expert output of the round */
+  size_t buf;         /* bf16 [E, C, d]: dispatch buffer of the round */
   size_t h;           /* bf16 [E, C, d_ff]: SwiGLU activations of the round */
+  size_t out;         /* bf16 [E, C, d]: expert outputs of the round */
   int32_t max_rounds; /* ceil(T / C): no expert can receive more than T tokens */
   int32_t plan_blocks;
 } moe_workspace_layout_t;
@@ -141,8 +143,10 @@ MOE_API int moe_plan(const moe_shape_t* shape, const float* logits, const uint16
              const uint16_t* w_router, const float* bias, void* ws, size_t ws_bytes,
              moe_plan_info_t* info, moe_stream_t stream);
 
-/* Executes all R rounds of the plan in `info` (from moe_plan on this `ws`), four kernels per
- * round launched with programmatic dependent launch:
+/* Executes all R rounds of the plan in `info` (from moe_plan on this `ws`), kernels launched
+ * with programmatic dependent launch: per round the gate/up and the down GEMM; a thin round's
+ * dispatch and combine ride on the neighbouring GEMM launches (extra warps), a large round's get
+ * their own kernels. Arguments:
  *   x         [T, d] bf16
  *   w_gate_up [E, 2*d_ff, d] bf16: rows 0..d_ff-1 = W1 (gate), rows d_ff..2*d_ff-1 = W3 (up)
  *   w_down    [E, d, d_ff] bf16 (W2)
@@ -157,8 +161,8 @@ MOE_API int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, v
  * each kernel can be checked and timed on its own; call them in this order per round.
  *   dispatch: buf[e][s] = x[token] for the round's rows (bf16 copy)
  *   gate_up:  h[e][s] = bf16(silu(buf[e][s] W1_e^T) * (buf[e][s] W3_e^T)) for s < n[r][e]
- *   down:     buf[e][s] = bf16(h[e][s] W2_e^T) for s < n[r][e] (overwrites the dispatch rows)
- *   combine:  y[t] = (t's first round ? 0 : y[t]) + sum_{j ascending, round(t,j)=r} gate*buf */
+ *   down:     out[e][s] = bf16(h[e][s] W2_e^T) for s < n[r][e]
+ *   combine:  y[t] = (t's first round ? 0 : y[t]) + sum_{j ascending, round(t,j)=r} gate*out */
 MOE_API int moe_round_dispatch(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
                        size_t ws_bytes, int32_t r, const uint16_t* x, moe_stream_t stream);
 MOE_API int moe_round_gate_up(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,

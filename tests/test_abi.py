@@ -39,7 +39,7 @@ def _bytes_model(w):
     blocks = (T + 255) // 256
     return (a(320 * 4) + a(T * E * 4) + 4 * a(T * k * 4) + a(E * 4) + a((E + 1) * 4)
             + a(blocks * E * 4) + 2 * a(mr * E * 4) + a((mr + 1) * 4) + 2 * a(T * k * 4)
-            + a(E * C * d * 2) + a(E * C * F * 2))
+            + a(E * C * d * 2) + a(E * C * F * 2) + a(E * C * d * 2))
 
 
 @pytest.mark.parametrize("w", wl.WORKLOADS, ids=lambda w: w.name)
@@ -47,13 +47,13 @@ def test_workspace_is_fixed_by_shape(lib, w):
     s = moe.make_shape(w.T, w.d, w.E, w.k, w.F, w.C)
     n = moe.workspace_bytes(s)
     assert n == _bytes_model(w)
-    # the round buffers dominate: E*C*(d + d_ff) bf16
-    assert n >= w.E * w.C * (w.d + w.F) * 2
+    # the round buffers dominate: E*C*(2d + d_ff) bf16 (dispatch rows, activations, outputs)
+    assert n >= w.E * w.C * (2 * w.d + w.F) * 2
     lay = moe.workspace_layout(s)
     assert lay.total_bytes == n
     offs = [lay.header, lay.logits, lay.topk_idx, lay.gate, lay.round, lay.slot, lay.load,
             lay.offsets, lay.block_base, lay.n, lay.row_off, lay.row_start, lay.row_token,
-            lay.row_dst, lay.buf, lay.h]
+            lay.row_dst, lay.buf, lay.h, lay.out]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     assert lay.max_rounds == (w.T + w.C - 1) // w.C
 

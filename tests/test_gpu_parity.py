@@ -161,7 +161,7 @@ def test_round_steps_against_oracle(name):
         layer.round_step("gate_up", r, inp["w_gate_up"])
         h = bits(layer.hidden_buffer())
         layer.round_step("down", r, inp["w_down"])
-        out = bits(layer.round_buffer())
+        out = bits(layer.output_buffer())
         for e in range(w.E):
             n = int(p["n"][r, e])
             if n == 0:
