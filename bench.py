@@ -36,6 +36,34 @@ UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM traffic per launch of a kernel, from an ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum, averaged over the launches of one layer step; summaries in profiles/),
+# valid only while the kernel's sources hash to the recorded value.
+TRAFFIC_SOURCES = ["sm100.cuh", "gemm_sm100.cuh", "copy_phases.cuh", "grouped_gemm.cu"]
+TRAFFIC = {
+    ("4k-zipf1", "gate_up"): {"bytes_per_launch": 20.22e6 + 0.50e6,
+                              "sources_sha1": "5a7f8bf5a51e3abde51578fcb03dedff101be348"},
+    ("4k-zipf1", "down"): {"bytes_per_launch": 9.12e6 + 0.02e6,
+                           "sources_sha1": "5a7f8bf5a51e3abde51578fcb03dedff101be348"},
+}
+
+
+def sources_sha1():
+    import hashlib
+    h = hashlib.sha1()
+    for f in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, "dropless_moe_layer_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload, kernel):
+    rec = TRAFFIC.get((workload, kernel))
+    if rec is None or rec["sources_sha1"] != sources_sha1():
+        return None
+    return rec["bytes_per_launch"]
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -414,7 +442,7 @@ def main():
             "rounds": info.R, "routed_pairs_per_s": value * w.k,
             "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                          "frac": achieved / peak, "peak_source": f"{peak_src} ({'bf16_tflops burst' if bound == 'tensor' else 'hbm_gbs copy'})",
-                         "traffic": None},
+                         "traffic": measured_traffic(w.name, dom)},
             "kernels": per_kernel,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
