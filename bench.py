@@ -225,35 +225,59 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- algorithmic work
 
-def algorithmic_work(w, info):
-    """Per kernel kind, the algorithmic units of one step (flops for the GEMMs, bytes for the
-    rest), from the plan alone. Padding rows (C - n) are never counted."""
+def round_rows(w, info):
+    """n[r][e]: rows of expert e in round r, from the plan's loads."""
     import numpy as np
     load = np.array(info.load[:w.E], dtype=np.int64)
-    R = info.R
-    n = np.clip(load[None, :] - w.C * np.arange(R)[:, None], 0, w.C)
-    rows = int(n.sum())                       # = T * k
+    return np.clip(load[None, :] - w.C * np.arange(info.R)[:, None], 0, w.C)
+
+
+def combine_bytes(w, round_np, rounds=None):
+    """combine reads every pair's expert row once (d bf16), writes each token's y row on every
+    round it has a pair in, and reads it back on every such round but the first. `rounds`
+    restricts the count to a set of rounds."""
+    import numpy as np
+    T, d = w.T, w.d
+    total = 0
+    for t_rounds in round_np.tolist():
+        seen = sorted(set(t_rounds))
+        for i, r in enumerate(seen):
+            if rounds is not None and r not in rounds:
+                continue
+            total += t_rounds.count(r) * d * 2 + d * 4 + (d * 4 if i > 0 else 0)
+    return total
+
+
+def algorithmic_work(w, info, r0, round_np):
+    """Per kernel kind, the algorithmic units of one step, from the plan alone (padding rows
+    C - n never count). Per-round kernels cover rounds [0, r0), the pipelined launch [r0, R).
+    GEMMs: flops (tensor-bound). Copies: bytes (HBM-bound). The pipelined launch runs all four
+    steps of its rounds; its bound is the larger of its tensor time (6 n d F flops per
+    (round, expert)) and its HBM time (the weights, 6 d F bytes per active (round, expert),
+    plus its copies' and its GEMM operands' bytes), each at the measured peak."""
+    n = round_rows(w, info)
+    per = n[:r0].sum()
+    pipe = n[r0:]
+    prow = int(pipe.sum())
+    d, F = w.d, w.F
     work = {
         "router_gemm": ("hbm", (w.T * w.d * 2 + w.E * w.d * 2 + w.T * w.E * 4) if w.router == "gemm" else 0),
         "topk": ("hbm", w.T * w.E * 4 + w.T * w.k * 8),
         "plan": ("hbm", w.T * w.k * 4 * 6),
-        "dispatch": ("hbm", 2 * rows * w.d * 2),
-        "gate_up": ("tensor", 4 * rows * w.d * w.F),
-        "down": ("tensor", 2 * rows * w.F * w.d),
+        "dispatch": ("hbm", 2 * int(per) * d * 2),
+        "gate_up": ("tensor", 4 * int(per) * d * F),
+        "down": ("tensor", 2 * int(per) * F * d),
+        "combine": ("hbm", combine_bytes(w, round_np, set(range(r0))) if r0 > 0 else 0),
     }
-    return work, rows
-
-
-def combine_bytes(w, round_np):
-    """combine reads every pair's expert row once (d bf16), writes each token's y row on every
-    round it has a pair in, and reads it back on every such round but the first."""
-    import numpy as np
-    T, d = w.T, w.d
-    rows = T * w.k * d * 2
-    spans = np.array([len(set(r)) for r in round_np.tolist()], dtype=np.int64)
-    writes = int(spans.sum()) * d * 4
-    reads = int((spans - 1).sum()) * d * 4
-    return rows + writes + reads
+    if prow:
+        flops = 6 * prow * d * F
+        active = int((pipe > 0).sum())
+        bytes_ = (active * 6 * d * F                  # weights of each active (round, expert)
+                  + 2 * prow * d * 2                  # dispatch: x rows in, buf rows out
+                  + prow * (d + F) * 2 * 2            # GEMM operands: buf, h (twice), out
+                  + combine_bytes(w, round_np, set(range(r0, info.R))))
+        work["pipeline"] = ("mixed", (flops, bytes_))
+    return work
 
 
 # ----------------------------------------------------------------------------- ranks
@@ -375,13 +399,27 @@ def main():
     # second timed pass with per-kernel events (for the roofline of the dominant kernel)
     _, _, prof = timed(args.steps, profile=True)
     info = layer.info
-    work, rows = algorithmic_work(w, info)
     rnd = layer.plan_tensors()["round"].cpu().numpy()
-    work["combine"] = ("hbm", combine_bytes(w, rnd))
     peaks, peak_src = load_peaks()
     kinds = {k: v for k, v in prof.items() if v[0] > 0}
+    # per-round launches cover rounds [0, r0): one gate/up launch per round and step
+    r0 = kinds["gate_up"][0] // args.steps if "gate_up" in kinds else 0
+    if "pipeline" not in kinds:
+        r0 = info.R
+    work = algorithmic_work(w, info, r0, rnd)
+
+    def resolve(kind):
+        """(bound, units per step) of a kind; a mixed launch takes its slower roofline."""
+        b, u = work[kind]
+        if b != "mixed":
+            return b, u
+        flops, bytes_ = u
+        t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+        t_hbm = bytes_ / (peaks["hbm_gbs"] * 1e9)
+        return ("tensor", flops) if t_tensor >= t_hbm else ("hbm", bytes_)
+
     dom = max(kinds, key=lambda k: kinds[k][1])
-    bound, units_per_step = work[dom]
+    bound, units_per_step = resolve(dom)
     cnt, ms = kinds[dom]
     per_launch_units = units_per_step * args.steps / cnt
     avg_launch_s = ms / cnt / 1e3
@@ -391,10 +429,14 @@ def main():
         achieved, peak, unit = per_launch_units / avg_launch_s / 1e9, peaks["hbm_gbs"], "GB/s"
     per_kernel = {}
     for k, (c, t) in kinds.items():
-        b, u = work[k]
+        b, u = resolve(k)
         rate = u * args.steps / (t / 1e3)
         per_kernel[k] = {"launches": c, "ms_total": round(t, 4), "share": round(t / sum(v[1] for v in kinds.values()), 4),
                          "bound": b, ("TFLOP/s" if b == "tensor" else "GB/s"): round(rate / (1e12 if b == "tensor" else 1e9), 2)}
+    if "pipeline" in work:
+        flops, bytes_ = work["pipeline"][1]
+        per_kernel.setdefault("pipeline", {}).update(
+            {"rounds": [r0, info.R], "flops_per_step": flops, "bytes_per_step": bytes_})
 
     # end to end through the public API from pinned host buffers
     host_x = inp["x"].cpu().pin_memory()
@@ -439,7 +481,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(w),
-            "rounds": info.R, "routed_pairs_per_s": value * w.k,
+            "rounds": info.R, "pipelined_rounds": [r0, info.R], "routed_pairs_per_s": value * w.k,
             "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                          "frac": achieved / peak, "peak_source": f"{peak_src} ({'bf16_tflops burst' if bound == 'tensor' else 'hbm_gbs copy'})",
                          "traffic": measured_traffic(w.name, dom)},

@@ -220,6 +220,48 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ float silu_f(float a) { return a / (1.0f + __expf(-a)); }
 
+// Epilogue of one accumulator row (this thread's TMEM lane; tb = lane base + accumulator
+// column): SwiGLU of `width` gate columns (TMEM columns [0, width)) with the matching up
+// columns ([width, 2 width)), bf16, 16-byte stores to orow[0, width). The TMEM loads are
+// warp-wide, so every lane runs them; only rows with `valid` store.
+__device__ __forceinline__ void store_swiglu(uint32_t tb, int width, uint16_t* orow, bool valid) {
+  for (int c = 0; c < width; c += 32) {
+    uint32_t gv[32], uv[32];
+    tmem_ld32(tb + c, gv);
+    tmem_ld32(tb + width + c, uv);
+    tmem_wait_ld();
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float h0 = silu_f(__uint_as_float(gv[2 * i])) * __uint_as_float(uv[2 * i]);
+      const float h1 = silu_f(__uint_as_float(gv[2 * i + 1])) * __uint_as_float(uv[2 * i + 1]);
+      pk[i] = pack_bf16x2(h0, h1);
+    }
+    if (valid) {
+      uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    }
+  }
+}
+
+// Same for a plain bf16 result of `cols` columns.
+__device__ __forceinline__ void store_bf16(uint32_t tb, int cols, uint16_t* orow, bool valid) {
+  for (int c = 0; c < cols; c += 32) {
+    uint32_t v[32];
+    tmem_ld32(tb + c, v);
+    tmem_wait_ld();
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+    if (valid) {
+      uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    }
+  }
+}
+
 // Runs the CTA's share of the tiles of the phase planned in slot `which`. Returns when this
 // warp's role work is issued/done (the epilogue warps return after their last store). Every warp
 // leaves converged: a CTA barrier (which requires whole warps) may follow directly.
@@ -353,40 +395,11 @@ __device__ __forceinline__ void run_phase(const Smem& s, uint32_t tmem_base, con
       if (p.mode == kSwiGLU) {
         uint16_t* orow = static_cast<uint16_t*>(p.out) + g * p.out_group_stride +
                          static_cast<long long>(row) * p.out_ld + nt * width;
-        for (int c = 0; c < width; c += 32) {
-          uint32_t gv[32], uv[32];
-          tmem_ld32(tb + c, gv);
-          tmem_ld32(tb + width + c, uv);
-          tmem_wait_ld();
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float h0 = silu_f(__uint_as_float(gv[2 * i])) * __uint_as_float(uv[2 * i]);
-            const float h1 = silu_f(__uint_as_float(gv[2 * i + 1])) * __uint_as_float(uv[2 * i + 1]);
-            pk[i] = pack_bf16x2(h0, h1);
-          }
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-          }
-        }
+        store_swiglu(tb, width, orow, valid);
       } else if (p.mode == kBf16Out) {
         uint16_t* orow = static_cast<uint16_t*>(p.out) + g * p.out_group_stride +
                          static_cast<long long>(row) * p.out_ld + nt * width;
-        for (int c = 0; c < bn; c += 32) {
-          uint32_t v[32];
-          tmem_ld32(tb + c, v);
-          tmem_wait_ld();
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-          }
-        }
+        store_bf16(tb, bn, orow, valid);
       } else {
         float* orow = static_cast<float*>(p.out) + static_cast<long long>(row) * p.out_ld;
         for (int c = 0; c < bn; c += 32) {

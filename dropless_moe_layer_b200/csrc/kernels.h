@@ -37,6 +37,7 @@ enum : int {
   kStatusTimeoutProducer = 1,
   kStatusTimeoutMma = 2,
   kStatusTimeoutEpilogue = 4,
+  kStatusTimeoutPipeline = 8,   // a dependency wait of the pipelined-rounds kernel gave up
 };
 
 // Header words inside the workspace.
@@ -51,6 +52,22 @@ enum : int {
 constexpr int kPlanTokensPerBlock = 256;
 #define MOE_MAX_E_PLAN 256
 
+// Pipelined-rounds kernel (round_pipeline.cu): fixed tile widths and the layout of its
+// dependency counters inside the workspace ("sync" region, int32, all zero between launches).
+constexpr int kPipeRowBlock = 128;   // rows of a tile (one 128-row block of an expert's C rows)
+constexpr int kPipeGuWidth = 32;     // gate columns per gate/up tile (MMA N = 64)
+constexpr int kPipeDnWidth = 64;     // output columns per down tile (MMA N = 64)
+enum : int {
+  kSyncGuTotal = 0,    // gate/up tile quarters finished (all blocks, all rounds of the launch)
+  kSyncDnTotal = 1,    // down tile quarters finished
+  kSyncCombTotal = 2,  // combine items finished
+  kSyncAbort = 3,      // raised by any CTA that gave up a wait
+  kSyncExit = 4,       // CTAs that finished (the last one zeroes the region)
+  kSyncBlocks = 32,    // then disp[E * MB], gu[E * MB], dn[E * MB], MB = ceil(C / 128)
+};
+__host__ __device__ inline long long pipe_row_blocks(int C) { return (C + kPipeRowBlock - 1) / kPipeRowBlock; }
+__host__ __device__ inline long long pipe_sync_words(int E, int C) { return kSyncBlocks + 3ll * E * pipe_row_blocks(C); }
+
 // Kernel kinds for profiling (same numbering as the public header).
 enum KernelKind : int {
   kKindRouterGemm = 0,
@@ -60,6 +77,7 @@ enum KernelKind : int {
   kKindGateUp = 4,
   kKindDown = 5,
   kKindCombine = 6,
+  kKindPipeline = 7,
 };
 
 // Called around every launch (profiling and launch accounting).
@@ -86,6 +104,9 @@ struct PlanBuffers {
   int32_t* slot;          // [T, k]
   int32_t* row_token;     // [T * k]
   int32_t* row_dst;       // [T * k]
+  int32_t* mb_prefix;     // [max_rounds, E + 1] 128-row blocks of experts < e in round r, or null
+  int32_t* sync;          // pipelined-rounds counters to zero ([sync_words]), or null
+  long long sync_words;
 };
 cudaError_t launch_plan(const PlanBuffers& b, int T, int k, int E, int C, int max_rounds,
                         cudaStream_t stream);
@@ -132,6 +153,33 @@ cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint1
 cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out, const int32_t* n_dev,
                         const int32_t* n_host, int E, int C, int d, int F, int32_t* status,
                         const RoundCopy* copy, cudaStream_t stream);
+
+// ---- pipelined rounds (round_pipeline.cu)
+// Rounds [r0, R) of the layer in one persistent launch (one CTA per SM): dispatch, gate/up
+// GEMM, down GEMM and combine of consecutive rounds overlap, ordered by dependency counters
+// instead of kernel boundaries. Expects rounds < r0 fully done (y holds their sums).
+struct PipelineArgs {
+  const uint16_t* x;
+  const uint16_t* w_gate_up;
+  const uint16_t* w_down;
+  uint16_t* buf;
+  uint16_t* h;
+  uint16_t* out;
+  float* y;
+  const int32_t* idx;
+  const float* gate;
+  const int32_t* round;
+  const int32_t* slot;
+  const int32_t* n;          // [max_rounds, E]
+  const int32_t* row_start;  // [max_rounds + 1]
+  const int32_t* row_token;
+  const int32_t* row_dst;
+  const int32_t* mb_prefix;  // [max_rounds, E + 1]
+  int32_t* sync;
+  int32_t* status;
+  int T, k, E, C, d, F, r0, R;
+};
+cudaError_t launch_round_pipeline(const PipelineArgs& a, cudaStream_t stream);
 
 // router GEMM: logits[t][e] = x[t] . w_router[e] + bias[e] (fp32 out)
 cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* w_router, const float* bias,

@@ -74,7 +74,9 @@ namespace {
 
 int check_shape(const moe_shape_t* s) {
   if (s == nullptr) return MOE_ERR_INVALID_ARG;
-  if (s->flags & ~static_cast<uint32_t>(MOE_FLAG_RENORM_TOPK)) return MOE_ERR_INVALID_ARG;
+  if (s->flags & ~static_cast<uint32_t>(MOE_FLAG_RENORM_TOPK | MOE_FLAG_PER_ROUND | MOE_FLAG_PIPELINE_ALL))
+    return MOE_ERR_INVALID_ARG;
+  if ((s->flags & MOE_FLAG_PER_ROUND) && (s->flags & MOE_FLAG_PIPELINE_ALL)) return MOE_ERR_INVALID_ARG;
   if (s->T < 0 || s->E < 1 || s->E > MOE_MAX_EXPERTS || s->k < 1 || s->k > MOE_MAX_TOPK ||
       s->k > s->E || s->C < 1)
     return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -118,6 +120,8 @@ void make_layout(const moe_shape_t* s, moe_workspace_layout_t* L) {
   L->buf = take(E * C * s->d * 2);
   L->h = take(E * C * s->d_ff * 2);
   L->out = take(E * C * s->d * 2);
+  L->mb_prefix = take(static_cast<long long>(mr) * (E + 1) * 4);
+  L->sync = take(pipe_sync_words(s->E, s->C) * 4);
   L->total_bytes = off;
   L->max_rounds = mr;
   L->plan_blocks = blocks;
@@ -312,6 +316,9 @@ int moe_plan(const moe_shape_t* shape, const float* logits, const uint16_t* x,
   pb.slot = at<int32_t>(ws, L.slot);
   pb.row_token = at<int32_t>(ws, L.row_token);
   pb.row_dst = at<int32_t>(ws, L.row_dst);
+  pb.mb_prefix = at<int32_t>(ws, L.mb_prefix);
+  pb.sync = at<int32_t>(ws, L.sync);
+  pb.sync_words = pipe_sync_words(s.E, s.C);
   if ((st = cuda_status(launch_plan(pb, s.T, s.k, s.E, s.C, L.max_rounds, stream))) != MOE_OK) return st;
 
   int32_t host[kHdrWords];
@@ -384,12 +391,6 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
   if (!aligned(x, 16) || !aligned(w_gate_up, 16) || !aligned(w_down, 16) || !aligned(y, 16))
     return MOE_ERR_MISALIGNED;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  // Launch order. A small copy step (a thin round: at most kFuseCopyBytes of rows) rides on
-  // the neighbouring GEMM launch: combine(r-1) on gate/up(r), dispatch(r+1) on down(r). A large
-  // one runs as its own full-bandwidth kernel right after down(r). Each launch depends only on
-  // the one before it (PDL wait), and no two steps of one launch touch the same buffer:
-  // dispatch writes buf, gate/up reads buf and writes h, down reads h and writes out, combine
-  // reads out and updates y. A run of thin rounds thus costs two launches per round.
   const int R = info->R;
   if (R == 0) return MOE_OK;
   auto small = [&](int rr) {
@@ -398,18 +399,57 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
     round_rows(shape, info, rr, n_host, &rows);
     return static_cast<size_t>(rows) * shape->d * 2 <= kFuseCopyBytes;
   };
-  if ((st = do_dispatch(shape, info, ws, L, 0, x, stream)) != MOE_OK) return st;
-  for (int r = 0; r < R; ++r) {
+  // Rounds [0, r0) run as per-round launches, [r0, R) in one pipelined launch.
+  int r0 = R;
+  if (shape->flags & MOE_FLAG_PIPELINE_ALL) r0 = 0;
+  // Per-round launch order. A small copy step (a thin round: at most kFuseCopyBytes of rows)
+  // rides on the neighbouring GEMM launch: combine(r-1) on gate/up(r), dispatch(r+1) on
+  // down(r). A large one runs as its own full-bandwidth kernel right after down(r). Each launch
+  // depends only on the one before it (PDL wait), and no two steps of one launch touch the same
+  // buffer: dispatch writes buf, gate/up reads buf and writes h, down reads h and writes out,
+  // combine reads out and updates y. A run of thin rounds thus costs two launches per round.
+  if (r0 > 0 && (st = do_dispatch(shape, info, ws, L, 0, x, stream)) != MOE_OK) return st;
+  for (int r = 0; r < r0; ++r) {
     const bool fuse_combine = r > 0 && small(r - 1);
     const RoundCopy comb = make_copy(shape, info, ws, L, true, r > 0 ? r - 1 : 0, x, y);
     if ((st = do_gate_up(shape, info, ws, L, r, w_gate_up, fuse_combine ? &comb : nullptr, stream)) != MOE_OK)
       return st;
-    const bool next = r + 1 < R;
+    const bool next = r + 1 < r0;
     const bool fuse_dispatch = next && small(r + 1);
     const RoundCopy disp = make_copy(shape, info, ws, L, false, next ? r + 1 : r, x, y);
     if ((st = do_down(shape, info, ws, L, r, w_down, fuse_dispatch ? &disp : nullptr, stream)) != MOE_OK) return st;
     if (next && !fuse_dispatch && (st = do_dispatch(shape, info, ws, L, r + 1, x, stream)) != MOE_OK) return st;
     if (!(next && small(r)) && (st = do_combine(shape, info, ws, L, r, y, stream)) != MOE_OK) return st;
+  }
+  if (r0 < R) {
+    PipelineArgs p{};
+    p.x = x;
+    p.w_gate_up = w_gate_up;
+    p.w_down = w_down;
+    p.buf = at<uint16_t>(ws, L.buf);
+    p.h = at<uint16_t>(ws, L.h);
+    p.out = at<uint16_t>(ws, L.out);
+    p.y = y;
+    p.idx = at<int32_t>(ws, L.topk_idx);
+    p.gate = at<float>(ws, L.gate);
+    p.round = at<int32_t>(ws, L.round);
+    p.slot = at<int32_t>(ws, L.slot);
+    p.n = at<int32_t>(ws, L.n);
+    p.row_start = at<int32_t>(ws, L.row_start);
+    p.row_token = at<int32_t>(ws, L.row_token);
+    p.row_dst = at<int32_t>(ws, L.row_dst);
+    p.mb_prefix = at<int32_t>(ws, L.mb_prefix);
+    p.sync = at<int32_t>(ws, L.sync);
+    p.status = at<int32_t>(ws, L.header) + kHdrStatus;
+    p.T = shape->T;
+    p.k = shape->k;
+    p.E = shape->E;
+    p.C = shape->C;
+    p.d = shape->d;
+    p.F = shape->d_ff;
+    p.r0 = r0;
+    p.R = R;
+    if ((st = cuda_status(launch_round_pipeline(p, stream))) != MOE_OK) return st;
   }
   return MOE_OK;
 }

@@ -103,7 +103,10 @@ __global__ void __launch_bounds__(kTPB) plan_finalize_kernel(const int32_t* __re
                                                              int32_t* __restrict__ header,
                                                              int32_t* __restrict__ n,
                                                              int32_t* __restrict__ row_off,
-                                                             int32_t* __restrict__ row_start) {
+                                                             int32_t* __restrict__ row_start,
+                                                             int32_t* __restrict__ mb_prefix,
+                                                             int32_t* __restrict__ sync,
+                                                             long long sync_words) {
   __shared__ int warp_sums[kWarps];
   __shared__ int s_load[MOE_MAX_E_PLAN];
   __shared__ int s_max;
@@ -135,11 +138,13 @@ __global__ void __launch_bounds__(kTPB) plan_finalize_kernel(const int32_t* __re
     row_start[r] = static_cast<int>(s);
   }
   __syncthreads();
-  // n[r][e] and row_off[r][e] = row_start[r] + sum_{e' < e} n[r][e'], one warp per round.
+  // n[r][e] and row_off[r][e] = row_start[r] + sum_{e' < e} n[r][e'], one warp per round;
+  // with mb_prefix, also the prefix over experts of their 128-row blocks in the round.
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int r = warp; r < R; r += kWarps) {
     const long long base_r = static_cast<long long>(r) * C;
     int running = row_start[r];
+    int running_mb = 0;
     for (int e0 = 0; e0 < E; e0 += 32) {
       const int x = e0 + lane;
       int nv = 0;
@@ -147,19 +152,30 @@ __global__ void __launch_bounds__(kTPB) plan_finalize_kernel(const int32_t* __re
         const long long rem = s_load[x] - base_r;
         nv = rem <= 0 ? 0 : (rem >= C ? C : static_cast<int>(rem));
       }
-      int incl = nv;
+      const int mb = (nv + kPipeRowBlock - 1) / kPipeRowBlock;
+      int incl = nv, incl_mb = mb;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const int o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
+        const int om = __shfl_up_sync(0xffffffffu, incl_mb, off);
+        if (lane >= off) {
+          incl += o;
+          incl_mb += om;
+        }
       }
       if (x < E) {
         n[static_cast<size_t>(r) * E + x] = nv;
         row_off[static_cast<size_t>(r) * E + x] = running + incl - nv;
+        if (mb_prefix) mb_prefix[static_cast<size_t>(r) * (E + 1) + x] = running_mb + incl_mb - mb;
       }
       running += __shfl_sync(0xffffffffu, incl, 31);
+      running_mb += __shfl_sync(0xffffffffu, incl_mb, 31);
     }
+    if (mb_prefix && lane == 0) mb_prefix[static_cast<size_t>(r) * (E + 1) + E] = running_mb;
   }
+  // the pipelined-rounds kernel expects its counters at zero
+  if (sync)
+    for (long long i = threadIdx.x; i < sync_words; i += blockDim.x) sync[i] = 0;
 }
 
 __global__ void __launch_bounds__(kTPB) plan_rank_kernel(const int32_t* __restrict__ idx, int T, int k,
@@ -211,7 +227,8 @@ cudaError_t launch_plan(const PlanBuffers& b, int T, int k, int E, int C, int ma
     err = launch_pdl(plan_scan_kernel, dim3(E), dim3(kTPB), 0, stream, b.block_base, blocks, E, b.load);
   if (err == cudaSuccess)
     err = launch_pdl(plan_finalize_kernel, dim3(1), dim3(kTPB), 0, stream, b.load, E, C, max_rounds,
-                     b.offsets, b.header, b.n, b.row_off, b.row_start);
+                     b.offsets, b.header, b.n, b.row_off, b.row_start, b.mb_prefix, b.sync,
+                     b.sync_words);
   if (blocks > 0 && err == cudaSuccess)
     err = launch_pdl(plan_rank_kernel, dim3(blocks), dim3(kTPB), 0, stream, b.idx, T, k, E, C,
                      b.block_base, b.row_off, b.round, b.slot, b.row_token, b.row_dst);

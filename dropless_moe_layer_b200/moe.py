@@ -16,9 +16,12 @@ from .build import LIB_PATH, ROOT
 c_i32, c_u32, c_sz, c_vp = ctypes.c_int32, ctypes.c_uint32, ctypes.c_size_t, ctypes.c_void_p
 
 MAX_EXPERTS = 256
-PROFILE_KINDS = 7
-PROFILE_NAMES = ["router_gemm", "topk", "plan", "dispatch", "gate_up", "down", "combine"]
+PROFILE_KINDS = 8
+PROFILE_NAMES = ["router_gemm", "topk", "plan", "dispatch", "gate_up", "down", "combine", "pipeline"]
 FLAG_RENORM_TOPK = 1
+FLAG_PER_ROUND = 2
+FLAG_PIPELINE_ALL = 4
+SCHEDULES = {"auto": 0, "per_round": FLAG_PER_ROUND, "pipeline": FLAG_PIPELINE_ALL}
 
 STATUS = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED_SHAPE",
           -3: "MOE_ERR_WORKSPACE_TOO_SMALL", -4: "MOE_ERR_MISALIGNED", -5: "MOE_ERR_CUDA",
@@ -39,7 +42,8 @@ class PlanInfo(ctypes.Structure):
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [(name, c_sz) for name in (
         "total_bytes", "header", "logits", "topk_idx", "gate", "round", "slot", "load",
-        "offsets", "block_base", "n", "row_off", "row_start", "row_token", "row_dst", "buf", "h", "out")
+        "offsets", "block_base", "n", "row_off", "row_start", "row_token", "row_dst", "buf", "h", "out",
+        "mb_prefix", "sync")
     ] + [("max_rounds", c_i32), ("plan_blocks", c_i32)]
 
 
@@ -107,8 +111,10 @@ def _check(call: str, status: int) -> None:
         raise MoeError(call, status)
 
 
-def make_shape(T: int, d: int, E: int, k: int, d_ff: int, C: int, renorm: bool = False) -> Shape:
-    return Shape(T, d, E, k, d_ff, C, FLAG_RENORM_TOPK if renorm else 0)
+def make_shape(T: int, d: int, E: int, k: int, d_ff: int, C: int, renorm: bool = False,
+               schedule: str = "auto") -> Shape:
+    """schedule: "auto" (trailing small rounds pipelined), "per_round" or "pipeline"."""
+    return Shape(T, d, E, k, d_ff, C, (FLAG_RENORM_TOPK if renorm else 0) | SCHEDULES[schedule])
 
 
 # ------------------------------------------------------------------------- raw-pointer calls
@@ -202,9 +208,9 @@ class DroplessMoE:
     """
 
     def __init__(self, T: int, d: int, E: int, k: int, d_ff: int, C: int, renorm: bool = False,
-                 device=None):
+                 device=None, schedule: str = "auto"):
         import torch
-        self.shape = make_shape(T, d, E, k, d_ff, C, renorm)
+        self.shape = make_shape(T, d, E, k, d_ff, C, renorm, schedule)
         self.ws_bytes = workspace_bytes(self.shape)
         if self.ws_bytes == 0:
             raise ValueError(f"unsupported shape T={T} d={d} E={E} k={k} d_ff={d_ff} C={C}")
@@ -289,6 +295,13 @@ class DroplessMoE:
         import torch
         s, L = self.shape, self.layout
         return self._view(L.h, s.E * s.C * s.d_ff, torch.bfloat16).view(s.E, s.C, s.d_ff)
+
+    def sync_counters(self):
+        """The pipelined launch's dependency counters (all zero between calls)."""
+        import torch
+        s, L = self.shape, self.layout
+        words = 32 + 3 * s.E * ((s.C + 127) // 128)
+        return self._view(L.sync, words, torch.int32)
 
     def round_step(self, step: str, r: int, ptr_tensor, stream=None) -> None:
         fn = dict(dispatch=round_dispatch, gate_up=round_gate_up, down=round_down,

@@ -74,6 +74,10 @@ typedef enum moe_status {
 
 /* moe_shape_t.flags */
 #define MOE_FLAG_RENORM_TOPK 1u     /* divide the k selected gates of a token by their sum */
+/* Launch schedule of moe_forward (results are identical; only the overlap of rounds differs).
+ * Default: per-round launches. */
+#define MOE_FLAG_PER_ROUND 2u       /* every round as per-round launches */
+#define MOE_FLAG_PIPELINE_ALL 4u    /* every round in the pipelined launch */
 
 #define MOE_MAX_EXPERTS 256
 #define MOE_MAX_TOPK 16
@@ -120,6 +124,9 @@ typedef struct moe_workspace_layout {
   size_t buf;         /* bf16 [E, C, d]: dispatch buffer of the round */
   size_t h;           /* bf16 [E, C, d_ff]: SwiGLU activations of the round */
   size_t out;         /* bf16 [E, C, d]: expert outputs of the round */
+  size_t mb_prefix;   /* i32 [max_rounds, E + 1]: 128-row blocks of experts < e in round r */
+  size_t sync;        /* i32 [32 + 3 * E * ceil(C / 128)]: pipelined launch's dependency
+                         counters (zero between calls) */
   int32_t max_rounds; /* ceil(T / C): no expert can receive more than T tokens */
   int32_t plan_blocks;
 } moe_workspace_layout_t;
@@ -143,10 +150,13 @@ MOE_API int moe_plan(const moe_shape_t* shape, const float* logits, const uint16
              const uint16_t* w_router, const float* bias, void* ws, size_t ws_bytes,
              moe_plan_info_t* info, moe_stream_t stream);
 
-/* Executes all R rounds of the plan in `info` (from moe_plan on this `ws`), kernels launched
- * with programmatic dependent launch: per round the gate/up and the down GEMM; a thin round's
- * dispatch and combine ride on the neighbouring GEMM launches (extra warps), a large round's get
- * their own kernels. Arguments:
+/* Executes all R rounds of the plan in `info` (from moe_plan on this `ws`).
+ * Per-round launches (programmatic dependent launch): per round the gate/up and the down GEMM;
+ * a thin round's dispatch and combine ride on the neighbouring GEMM launches (extra warps), a
+ * large round's get their own kernels. Pipelined launch: one persistent cooperative kernel (one
+ * CTA per SM) runs a run of rounds, their dispatch, GEMM tiles and combine overlapping under
+ * dependency counters kept in the workspace; a wait that exceeds 2 s sets the status word
+ * (moe_device_status) and the launch unwinds. shape->flags choose the schedule. Arguments:
  *   x         [T, d] bf16
  *   w_gate_up [E, 2*d_ff, d] bf16: rows 0..d_ff-1 = W1 (gate), rows d_ff..2*d_ff-1 = W3 (up)
  *   w_down    [E, d, d_ff] bf16 (W2)
@@ -185,9 +195,10 @@ MOE_API uint64_t moe_launch_count(void);
 /* Per-kernel timing with CUDA events. While enabled, every launch made by the calls above
  * is bracketed by two events on its stream; moe_profile_read() synchronizes on them and
  * reports, per kernel kind, the launch count and the summed milliseconds. Kinds:
- * 0 router GEMM, 1 top-k, 2 plan, 3 dispatch, 4 gate_up GEMM, 5 down GEMM, 6 combine.
+ * 0 router GEMM, 1 top-k, 2 plan, 3 dispatch, 4 gate_up GEMM, 5 down GEMM, 6 combine,
+ * 7 pipelined rounds (all four steps of its rounds in one launch).
  * Up to 4096 launches are recorded between enable and read. Not thread-safe. */
-#define MOE_PROFILE_KINDS 7
+#define MOE_PROFILE_KINDS 8
 MOE_API int moe_profile_enable(int on);
 MOE_API int moe_profile_read(int32_t counts[MOE_PROFILE_KINDS], double ms[MOE_PROFILE_KINDS]);
 

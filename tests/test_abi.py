@@ -39,7 +39,8 @@ def _bytes_model(w):
     blocks = (T + 255) // 256
     return (a(320 * 4) + a(T * E * 4) + 4 * a(T * k * 4) + a(E * 4) + a((E + 1) * 4)
             + a(blocks * E * 4) + 2 * a(mr * E * 4) + a((mr + 1) * 4) + 2 * a(T * k * 4)
-            + a(E * C * d * 2) + a(E * C * F * 2) + a(E * C * d * 2))
+            + a(E * C * d * 2) + a(E * C * F * 2) + a(E * C * d * 2)
+            + a(mr * (E + 1) * 4) + a((32 + 3 * E * ((C + 127) // 128)) * 4))
 
 
 @pytest.mark.parametrize("w", wl.WORKLOADS, ids=lambda w: w.name)
@@ -53,7 +54,7 @@ def test_workspace_is_fixed_by_shape(lib, w):
     assert lay.total_bytes == n
     offs = [lay.header, lay.logits, lay.topk_idx, lay.gate, lay.round, lay.slot, lay.load,
             lay.offsets, lay.block_base, lay.n, lay.row_off, lay.row_start, lay.row_token,
-            lay.row_dst, lay.buf, lay.h, lay.out]
+            lay.row_dst, lay.buf, lay.h, lay.out, lay.mb_prefix, lay.sync]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     assert lay.max_rounds == (w.T + w.C - 1) // w.C
 
@@ -73,8 +74,12 @@ def test_bad_shapes_are_rejected(lib, kw):
 
 def test_bad_flags_rejected(lib):
     s = moe.make_shape(64, 128, 8, 2, 128, 16)
-    s.flags = 4
-    assert moe.workspace_bytes(s) == 0
+    for flags in (8, 1 << 31, moe.FLAG_PER_ROUND | moe.FLAG_PIPELINE_ALL):
+        s.flags = flags
+        assert moe.workspace_bytes(s) == 0
+    for schedule in moe.SCHEDULES:   # the schedule flags do not change the fixed memory
+        assert moe.workspace_bytes(moe.make_shape(64, 128, 8, 2, 128, 16, schedule=schedule)) == \
+            moe.workspace_bytes(moe.make_shape(64, 128, 8, 2, 128, 16))
 
 
 def test_plan_argument_errors_without_gpu(lib):

@@ -60,9 +60,12 @@ def rel_err(got, ref):
     return float(np.max(np.abs(got - ref)) / max(np.max(np.abs(ref)), 1e-30))
 
 
-def run_gpu(w, inp, C=None, renorm=False):
+SCHEDULES = ["auto", "per_round", "pipeline"]
+
+
+def run_gpu(w, inp, C=None, renorm=False, schedule="auto"):
     C = C or w.C
-    layer = moe.DroplessMoE(w.T, w.d, w.E, w.k, w.F, C, renorm=renorm)
+    layer = moe.DroplessMoE(w.T, w.d, w.E, w.k, w.F, C, renorm=renorm, schedule=schedule)
     y = layer(inp["x"], inp["w_gate_up"], inp["w_down"], logits=inp["logits"],
               w_router=inp["w_router"], bias=inp["bias"])
     torch.cuda.synchronize()
@@ -101,11 +104,12 @@ def sample_tokens(T, p, count, seed):
 
 # ----------------------------------------------------------------------------- workloads
 
+@pytest.mark.parametrize("schedule", SCHEDULES)
 @pytest.mark.parametrize("name", ["tiny-zipf1", "4k-zipf1"])
-def test_workload_full_parity(name):
+def test_workload_full_parity(name, schedule):
     w = wl.BY_NAME[name]
     inp = wl.generate(w, "cuda")
-    layer, y = run_gpu(w, inp)
+    layer, y = run_gpu(w, inp, schedule=schedule)
     z = inp["logits"].cpu().numpy()
     idx, g, p = check_plan(layer, w, w.C, z)
     assert p["R"] >= 2
@@ -191,12 +195,13 @@ EDGE = [
 ]
 
 
+@pytest.mark.parametrize("schedule", ["per_round", "pipeline"])
 @pytest.mark.parametrize("cfg", EDGE, ids=lambda c: "T{T}-d{d}-E{E}-k{k}-F{F}-C{C}".format(**c))
-def test_edge_shapes(cfg):
+def test_edge_shapes(cfg, schedule):
     w = wl.custom(name="edge", T=cfg["T"], d=cfg["d"], E=cfg["E"], k=cfg["k"], F=cfg["F"], C=cfg["C"],
                   bias="zipf", zipf_s=1.0, seed=cfg["T"])
     inp = wl.generate(w, "cuda")
-    layer, y = run_gpu(w, inp)
+    layer, y = run_gpu(w, inp, schedule=schedule)
     idx, g, p = check_plan(layer, w, w.C, inp["logits"].cpu().numpy())
     ref = oracle.forward(bits(inp["x"]), LazyExperts(inp["w_gate_up"]), LazyExperts(inp["w_down"]), idx, g)
     assert rel_err(y.cpu().numpy().astype(np.float64), ref) <= Y_TOL
@@ -275,3 +280,32 @@ def test_capacity_changes_rounds_not_result():
     for C, y in ys.items():
         assert rel_err(y, base) <= 1e-5, C
     assert layer.info.R == 1
+
+
+def test_schedules_give_identical_bits():
+    """The launch schedule changes which rounds overlap, never the arithmetic: every output
+    element is the same K-ordered fp32 sum and every token's pairs are combined in the same
+    (round, j) order, whatever the tile widths and the launch boundaries."""
+    w = wl.BY_NAME["4k-zipf1"]
+    inp = wl.generate(w, "cuda")
+    ys = {sch: run_gpu(w, inp, schedule=sch)[1] for sch in SCHEDULES}
+    assert torch.equal(ys["per_round"], ys["pipeline"])
+    assert torch.equal(ys["auto"], ys["pipeline"])
+
+
+def test_pipeline_counters_return_to_zero_and_repeat():
+    """One plan, two pipelined forwards: the dependency counters are zero after each launch
+    (the last CTA clears them), so the second call starts clean and gives the same bits."""
+    w = wl.BY_NAME["tiny-zipf1"]
+    inp = wl.generate(w, "cuda")
+    layer = moe.DroplessMoE(w.T, w.d, w.E, w.k, w.F, w.C, schedule="pipeline")
+    layer.plan(logits=inp["logits"])
+    assert int(layer.sync_counters().abs().sum()) == 0
+    y1 = layer.forward(inp["x"], inp["w_gate_up"], inp["w_down"])
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    assert int(layer.sync_counters().abs().sum()) == 0
+    y2 = layer.forward(inp["x"], inp["w_gate_up"], inp["w_down"])
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    assert torch.equal(y1, y2)
