@@ -307,6 +307,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=[x.name for x in wl.WORKLOADS])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--schedule", default="auto", choices=["auto", "per_round", "pipeline"],
+                    help="moe_forward launch schedule (the layer's results are identical)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = wl.BY_NAME[args.workload]
@@ -335,7 +337,7 @@ def main():
 
     moe.load_library()
     inp = wl.generate(w, dev)
-    layer = moe.DroplessMoE(w.T, w.d, w.E, w.k, w.F, w.C, device=dev)
+    layer = moe.DroplessMoE(w.T, w.d, w.E, w.k, w.F, w.C, device=dev, schedule=args.schedule)
     y = torch.empty(w.T, w.d, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -480,7 +482,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(w),
+            "config": dict(workload_config(w), schedule=args.schedule),
             "rounds": info.R, "pipelined_rounds": [r0, info.R], "routed_pairs_per_s": value * w.k,
             "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                          "frac": achieved / peak, "peak_source": f"{peak_src} ({'bf16_tflops burst' if bound == 'tensor' else 'hbm_gbs copy'})",

@@ -71,74 +71,156 @@ struct CombineArgs {
   int T, k, C, d;
 };
 
-// The whole warp combines token t for round r (no-op if t has no pair in round r).
-// With `only_expert` >= 0 the warp stands for one row of the round (token t's pair with that
-// expert) and does the work only if that pair is t's first pair in the round, so that every
-// active token is combined exactly once when the round is walked row by row.
-__device__ __forceinline__ void combine_token(const CombineArgs& a, int t, int r, int only_expert = -1) {
+// One token's pairs in one round, spread over the warp (every lane holds the same scalars;
+// lane p < npairs holds pair p's source row and gate, pairs in ascending j).
+struct TokenPairs {
+  int npairs;               // pairs of the token in round r (0: nothing to do)
+  bool fresh;               // r is the token's first round: y starts from zero
+  int prev_round;           // the token's latest round before r, or -1
+  int first_expert;         // expert of the token's first pair in round r
+  int e, s;                 // this lane's pair (expert, slot), lane < npairs
+  unsigned long long prow;  // e * C + s
+  float pgate;
+};
+
+// A token's plan entries as loaded: lane j < k holds pair j's round, expert, slot and gate.
+struct PairLoads {
+  int round, idx, slot;
+  float gate;
+};
+
+// Issues the four independent loads; nothing waits for them until token_pairs() uses them, so
+// a warp can fetch the next token's entries while it combines the current one.
+__device__ __forceinline__ PairLoads load_pairs(const CombineArgs& a, int t) {
   const int lane = threadIdx.x & 31;
-  const size_t pbase = static_cast<size_t>(t) * a.k;
-  // lane j < k holds pair j's round, expert, slot and gate (four independent loads)
-  int my_round = INT_MAX, my_idx = 0, my_slot = 0;
-  float my_gate = 0.f;
+  PairLoads l{INT_MAX, 0, 0, 0.f};
   if (lane < a.k) {
-    my_round = a.round[pbase + lane];
-    my_idx = a.idx[pbase + lane];
-    my_slot = a.slot[pbase + lane];
-    my_gate = a.gate[pbase + lane];
+    const size_t i = static_cast<size_t>(t) * a.k + lane;
+    l.round = a.round[i];
+    l.idx = a.idx[i];
+    l.slot = a.slot[i];
+    l.gate = a.gate[i];
   }
+  return l;
+}
+
+__device__ __forceinline__ TokenPairs token_pairs(const CombineArgs& a, const PairLoads& l, int r) {
+  const int lane = threadIdx.x & 31;
+  const int my_round = l.round, my_idx = l.idx, my_slot = l.slot;
+  const float my_gate = l.gate;
+  TokenPairs tp;
   const uint32_t here = __ballot_sync(0xffffffffu, my_round == r);
-  if (here == 0u) return;
-  if (only_expert >= 0 && __shfl_sync(0xffffffffu, my_idx, __ffs(here) - 1) != only_expert) return;
-  const int first_round = __reduce_min_sync(0xffffffffu, my_round);
-  const bool fresh = first_round == r;
-  const int npairs = __popc(here);
-  // Lane p holds the source row and gate of the p-th pair of this round (ascending j).
-  const int jp = lane < npairs ? static_cast<int>(__fns(here, 0, lane + 1)) : 0;
-  const int e_p = __shfl_sync(0xffffffffu, my_idx, jp);
-  const int s_p = __shfl_sync(0xffffffffu, my_slot, jp);
-  const float g_p = __shfl_sync(0xffffffffu, my_gate, jp);
-  const unsigned long long prow = lane < npairs ? static_cast<unsigned long long>(e_p) * a.C + s_p : 0ull;
-  const float pgate = lane < npairs ? g_p : 0.f;
+  tp.npairs = __popc(here);
+  tp.first_expert = __shfl_sync(0xffffffffu, my_idx, here ? __ffs(here) - 1 : 0);
+  tp.fresh = __reduce_min_sync(0xffffffffu, my_round) == r;
+  tp.prev_round = __reduce_max_sync(0xffffffffu, my_round < r ? my_round : -1);
+  const int jp = lane < tp.npairs ? static_cast<int>(__fns(here, 0, lane + 1)) : 0;
+  tp.e = __shfl_sync(0xffffffffu, my_idx, jp);
+  tp.s = __shfl_sync(0xffffffffu, my_slot, jp);
+  const float g = __shfl_sync(0xffffffffu, my_gate, jp);
+  tp.prow = lane < tp.npairs ? static_cast<unsigned long long>(tp.e) * a.C + tp.s : 0ull;
+  tp.pgate = lane < tp.npairs ? g : 0.f;
+  return tp;
+}
+
+// y[t] = (fresh ? 0 : y[t]) + sum over the round's pairs (ascending j) of gate * out row, fp32
+// FMAs. kLaneCols columns per lane per pass (8 or 16): 16 halves the passes over a row, so
+// more loads are in flight when few warps do the work. The whole warp runs it.
+template <int kLaneCols = 8>
+__device__ __forceinline__ void accumulate_token(const CombineArgs& a, int t, const TokenPairs& tp) {
+  static_assert(kLaneCols == 8 || kLaneCols == 16, "lane width");
+  constexpr int kVecs = kLaneCols / 8;   // bf16 x 8 per 16-byte load
+  const int lane = threadIdx.x & 31;
+  const int npairs = tp.npairs;
   float* yrow = a.y + static_cast<size_t>(t) * a.d;
   // Every lane runs the same iterations (the shuffles below need the whole warp); lanes past
-  // the end of the row (d < 256) only skip the loads and stores.
-  for (int c0 = 0; c0 < a.d; c0 += 32 * 8) {
-    const int c = c0 + lane * 8;
+  // the end of the row only skip the loads and stores.
+  for (int c0 = 0; c0 < a.d; c0 += 32 * kLaneCols) {
+    const int c = c0 + lane * kLaneCols;
     const bool col = c < a.d;
-    float acc[8];
-    if (fresh || !col) {
+    float acc[kLaneCols];
+    if (tp.fresh || !col) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      for (int i = 0; i < kLaneCols; ++i) acc[i] = 0.f;
     } else {
-      const float4 u = *reinterpret_cast<const float4*>(yrow + c);
-      const float4 v = *reinterpret_cast<const float4*>(yrow + c + 4);
-      acc[0] = u.x; acc[1] = u.y; acc[2] = u.z; acc[3] = u.w;
-      acc[4] = v.x; acc[5] = v.y; acc[6] = v.z; acc[7] = v.w;
+#pragma unroll
+      for (int i = 0; i < kLaneCols; i += 4) {
+        const float4 u = *reinterpret_cast<const float4*>(yrow + c + i);
+        acc[i] = u.x; acc[i + 1] = u.y; acc[i + 2] = u.z; acc[i + 3] = u.w;
+      }
     }
     for (int p0 = 0; p0 < npairs; p0 += 4) {
-      uint4 q[4];
+      uint4 q[4][kVecs];
       float g[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {               // up to four rows in flight per lane
         const int p = p0 + u;
-        const unsigned long long row = __shfl_sync(0xffffffffu, prow, p & 31);
-        g[u] = __shfl_sync(0xffffffffu, pgate, p & 31);
-        q[u] = (p < npairs && col) ? *reinterpret_cast<const uint4*>(a.buf + row * a.d + c) : make_uint4(0, 0, 0, 0);
+        const unsigned long long row = __shfl_sync(0xffffffffu, tp.prow, p & 31);
+        g[u] = __shfl_sync(0xffffffffu, tp.pgate, p & 31);
+#pragma unroll
+        for (int v = 0; v < kVecs; ++v)
+          q[u][v] = (p < npairs && col) ? *reinterpret_cast<const uint4*>(a.buf + row * a.d + c + 8 * v)
+                                        : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         if (p0 + u < npairs) {
-          float f[8];
-          bf16x8_to_f32(q[u], f);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] = __fmaf_rn(g[u], f[i], acc[i]);
+          for (int v = 0; v < kVecs; ++v) {
+            float f[8];
+            bf16x8_to_f32(q[u][v], f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[8 * v + i] = __fmaf_rn(g[u], f[i], acc[8 * v + i]);
+          }
         }
       }
     }
     if (col) {
-      *reinterpret_cast<float4*>(yrow + c) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      *reinterpret_cast<float4*>(yrow + c + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+#pragma unroll
+      for (int i = 0; i < kLaneCols; i += 4)
+        *reinterpret_cast<float4*>(yrow + c + i) = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
+    }
+  }
+}
+
+// The whole warp combines token t for round r (no-op if t has no pair in round r).
+// With `only_expert` >= 0 the warp stands for one row of the round (token t's pair with that
+// expert) and does the work only if that pair is t's first pair in the round, so that every
+// active token is combined exactly once when the round is walked row by row.
+template <int kLaneCols = 8>
+__device__ __forceinline__ void combine_token(const CombineArgs& a, int t, int r, int only_expert = -1) {
+  const TokenPairs tp = token_pairs(a, load_pairs(a, t), r);
+  if (tp.npairs == 0) return;
+  if (only_expert >= 0 && tp.first_expert != only_expert) return;
+  accumulate_token<kLaneCols>(a, t, tp);
+}
+
+// One warp copies rows [0, nr) (nr <= 32) of a slice of the round-major row list: row i goes
+// from x[tok[i]] to buf[dst[i]]. The row list entries are read once (lane i holds row i) and the
+// copy is flattened over (row, 16-byte vector) so that 16 loads per lane are in flight, whatever
+// the row length. Every shuffle runs on all 32 lanes.
+__device__ __forceinline__ void copy_rows_flat(const uint4* __restrict__ x, uint4* __restrict__ buf,
+                                               int tok_lane, int dst_lane, int nr, int vecs) {
+  const int lane = threadIdx.x & 31;
+  const int units = nr * vecs;
+  constexpr int kInFlight = 16;
+  for (int u0 = 0; u0 < units; u0 += 32 * kInFlight) {
+    uint4 v[kInFlight];
+#pragma unroll
+    for (int i = 0; i < kInFlight; ++i) {
+      const int u = u0 + i * 32 + lane;
+      const int uc = u < units ? u : units - 1;
+      const int row = uc / vecs;
+      const int t = __shfl_sync(0xffffffffu, tok_lane, row);
+      if (u < units) v[i] = __ldg(x + static_cast<size_t>(t) * vecs + (uc - row * vecs));
+    }
+#pragma unroll
+    for (int i = 0; i < kInFlight; ++i) {
+      const int u = u0 + i * 32 + lane;
+      const int uc = u < units ? u : units - 1;
+      const int row = uc / vecs;
+      const int dst = __shfl_sync(0xffffffffu, dst_lane, row);
+      if (u < units) buf[static_cast<size_t>(dst) * vecs + (uc - row * vecs)] = v[i];
     }
   }
 }

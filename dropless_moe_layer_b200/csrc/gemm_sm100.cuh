@@ -218,7 +218,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + __expf(-a)); }
+// silu(a) = a * sigmoid(a) = a / (1 + e^-a), with the fast division (at most 2 ulp; it returns 0
+// once 1 + e^-a exceeds 2^126, where silu(a) is below 1e-36 in magnitude anyway).
+__device__ __forceinline__ float silu_f(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 
 // Epilogue of one accumulator row (this thread's TMEM lane; tb = lane base + accumulator
 // column): SwiGLU of `width` gate columns (TMEM columns [0, width)) with the matching up

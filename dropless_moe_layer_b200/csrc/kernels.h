@@ -54,19 +54,26 @@ constexpr int kPlanTokensPerBlock = 256;
 
 // Pipelined-rounds kernel (round_pipeline.cu): fixed tile widths and the layout of its
 // dependency counters inside the workspace ("sync" region, int32, all zero between launches).
+// Round r of a launch starting at round r0 uses buffer set p = (r - r0) & 1.
 constexpr int kPipeRowBlock = 128;   // rows of a tile (one 128-row block of an expert's C rows)
 constexpr int kPipeGuWidth = 32;     // gate columns per gate/up tile (MMA N = 64)
 constexpr int kPipeDnWidth = 64;     // output columns per down tile (MMA N = 64)
+// Every counter has its own 32-byte sector (a stride of 8 words) and the round-level counters
+// their own 256-byte slots, so that polls and atomic adds on different counters do not queue
+// behind each other in one L2 line.
+constexpr int kSyncStride = 8;       // words between per-block counters
 enum : int {
-  kSyncGuTotal = 0,    // gate/up tile quarters finished (all blocks, all rounds of the launch)
-  kSyncDnTotal = 1,    // down tile quarters finished
-  kSyncCombTotal = 2,  // combine items finished
-  kSyncAbort = 3,      // raised by any CTA that gave up a wait
-  kSyncExit = 4,       // CTAs that finished (the last one zeroes the region)
-  kSyncBlocks = 32,    // then disp[E * MB], gu[E * MB], dn[E * MB], MB = ceil(C / 128)
+  kSyncAbort = 128,        // raised by any CTA that gave up a wait
+  kSyncExit = 160,         // CTAs that finished (the last one zeroes the region)
+  kSyncDnTotal = 192,      // [2] (stride 64) down tile quarters finished, per buffer set
+  kSyncNextTask = 384,     // next GEMM tile of the list to claim
+  kSyncBlocks = 448,       // then disp, gu, dn, rd: [2][E * MB] each, MB = ceil(C / 128)
 };
+constexpr int kSyncSetStride = 64;
 __host__ __device__ inline long long pipe_row_blocks(int C) { return (C + kPipeRowBlock - 1) / kPipeRowBlock; }
-__host__ __device__ inline long long pipe_sync_words(int E, int C) { return kSyncBlocks + 3ll * E * pipe_row_blocks(C); }
+__host__ __device__ inline long long pipe_sync_words(int E, int C) {
+  return kSyncBlocks + 8ll * E * pipe_row_blocks(C) * kSyncStride;
+}
 
 // Kernel kinds for profiling (same numbering as the public header).
 enum KernelKind : int {
@@ -107,6 +114,7 @@ struct PlanBuffers {
   int32_t* mb_prefix;     // [max_rounds, E + 1] 128-row blocks of experts < e in round r, or null
   int32_t* sync;          // pipelined-rounds counters to zero ([sync_words]), or null
   long long sync_words;
+  unsigned long long* tok_flag;   // [T] per-token combine progress to zero, or null
 };
 cudaError_t launch_plan(const PlanBuffers& b, int T, int k, int E, int C, int max_rounds,
                         cudaStream_t stream);
@@ -162,9 +170,9 @@ struct PipelineArgs {
   const uint16_t* x;
   const uint16_t* w_gate_up;
   const uint16_t* w_down;
-  uint16_t* buf;
-  uint16_t* h;
-  uint16_t* out;
+  uint16_t* buf[2];          // two buffer sets: round r uses set (r - r0) & 1
+  uint16_t* h[2];
+  uint16_t* out[2];
   float* y;
   const int32_t* idx;
   const float* gate;
@@ -176,6 +184,8 @@ struct PipelineArgs {
   const int32_t* row_dst;
   const int32_t* mb_prefix;  // [max_rounds, E + 1]
   int32_t* sync;
+  unsigned long long* tok_flag;  // [T] (gen << 32) | (last round combined in this launch + 1)
+  unsigned long long gen;        // launch generation (increases from launch to launch)
   int32_t* status;
   int T, k, E, C, d, F, r0, R;
 };

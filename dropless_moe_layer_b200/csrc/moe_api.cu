@@ -122,6 +122,12 @@ void make_layout(const moe_shape_t* s, moe_workspace_layout_t* L) {
   L->out = take(E * C * s->d * 2);
   L->mb_prefix = take(static_cast<long long>(mr) * (E + 1) * 4);
   L->sync = take(pipe_sync_words(s->E, s->C) * 4);
+  L->tok_flag = take(T * 8);
+  if (!(s->flags & MOE_FLAG_PER_ROUND)) {   // second buffer set of the pipelined launch
+    L->buf2 = take(E * C * s->d * 2);
+    L->h2 = take(E * C * s->d_ff * 2);
+    L->out2 = take(E * C * s->d * 2);
+  }
   L->total_bytes = off;
   L->max_rounds = mr;
   L->plan_blocks = blocks;
@@ -319,6 +325,7 @@ int moe_plan(const moe_shape_t* shape, const float* logits, const uint16_t* x,
   pb.mb_prefix = at<int32_t>(ws, L.mb_prefix);
   pb.sync = at<int32_t>(ws, L.sync);
   pb.sync_words = pipe_sync_words(s.E, s.C);
+  pb.tok_flag = at<unsigned long long>(ws, L.tok_flag);
   if ((st = cuda_status(launch_plan(pb, s.T, s.k, s.E, s.C, L.max_rounds, stream))) != MOE_OK) return st;
 
   int32_t host[kHdrWords];
@@ -400,8 +407,25 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
     return static_cast<size_t>(rows) * shape->d * 2 <= kFuseCopyBytes;
   };
   // Rounds [0, r0) run as per-round launches, [r0, R) in one pipelined launch.
+  // A round is thin when even 128-column tiles of its gate/up GEMM would leave SMs idle: its
+  // steps are latency-bound and gain from overlapping their neighbours. The pipelined launch
+  // takes the trailing run of thin rounds (its 32-column tiles suit thin rounds only).
+  auto thin = [&](int rr) {
+    long long blocks = 0;
+    const long long base = static_cast<long long>(rr) * shape->C;
+    for (int e = 0; e < shape->E; ++e) {
+      const long long rem = info->load[e] - base;
+      const long long n = rem <= 0 ? 0 : (rem >= shape->C ? shape->C : rem);
+      blocks += (n + kPipeRowBlock - 1) / kPipeRowBlock;
+    }
+    return blocks * (shape->d_ff / 128 > 0 ? shape->d_ff / 128 : 1) < num_sms();
+  };
   int r0 = R;
-  if (shape->flags & MOE_FLAG_PIPELINE_ALL) r0 = 0;
+  if (shape->flags & MOE_FLAG_PIPELINE_ALL) {
+    r0 = 0;
+  } else if (!(shape->flags & MOE_FLAG_PER_ROUND)) {
+    while (r0 > 0 && thin(r0 - 1)) --r0;
+  }
   // Per-round launch order. A small copy step (a thin round: at most kFuseCopyBytes of rows)
   // rides on the neighbouring GEMM launch: combine(r-1) on gate/up(r), dispatch(r+1) on
   // down(r). A large one runs as its own full-bandwidth kernel right after down(r). Each launch
@@ -426,9 +450,12 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
     p.x = x;
     p.w_gate_up = w_gate_up;
     p.w_down = w_down;
-    p.buf = at<uint16_t>(ws, L.buf);
-    p.h = at<uint16_t>(ws, L.h);
-    p.out = at<uint16_t>(ws, L.out);
+    p.buf[0] = at<uint16_t>(ws, L.buf);
+    p.h[0] = at<uint16_t>(ws, L.h);
+    p.out[0] = at<uint16_t>(ws, L.out);
+    p.buf[1] = at<uint16_t>(ws, L.buf2);
+    p.h[1] = at<uint16_t>(ws, L.h2);
+    p.out[1] = at<uint16_t>(ws, L.out2);
     p.y = y;
     p.idx = at<int32_t>(ws, L.topk_idx);
     p.gate = at<float>(ws, L.gate);
@@ -440,6 +467,7 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
     p.row_dst = at<int32_t>(ws, L.row_dst);
     p.mb_prefix = at<int32_t>(ws, L.mb_prefix);
     p.sync = at<int32_t>(ws, L.sync);
+    p.tok_flag = at<unsigned long long>(ws, L.tok_flag);
     p.status = at<int32_t>(ws, L.header) + kHdrStatus;
     p.T = shape->T;
     p.k = shape->k;

@@ -104,9 +104,7 @@ __global__ void __launch_bounds__(kTPB) plan_finalize_kernel(const int32_t* __re
                                                              int32_t* __restrict__ n,
                                                              int32_t* __restrict__ row_off,
                                                              int32_t* __restrict__ row_start,
-                                                             int32_t* __restrict__ mb_prefix,
-                                                             int32_t* __restrict__ sync,
-                                                             long long sync_words) {
+                                                             int32_t* __restrict__ mb_prefix) {
   __shared__ int warp_sums[kWarps];
   __shared__ int s_load[MOE_MAX_E_PLAN];
   __shared__ int s_max;
@@ -173,9 +171,6 @@ __global__ void __launch_bounds__(kTPB) plan_finalize_kernel(const int32_t* __re
     }
     if (mb_prefix && lane == 0) mb_prefix[static_cast<size_t>(r) * (E + 1) + E] = running_mb;
   }
-  // the pipelined-rounds kernel expects its counters at zero
-  if (sync)
-    for (long long i = threadIdx.x; i < sync_words; i += blockDim.x) sync[i] = 0;
 }
 
 __global__ void __launch_bounds__(kTPB) plan_rank_kernel(const int32_t* __restrict__ idx, int T, int k,
@@ -185,7 +180,9 @@ __global__ void __launch_bounds__(kTPB) plan_rank_kernel(const int32_t* __restri
                                                          int32_t* __restrict__ round_out,
                                                          int32_t* __restrict__ slot_out,
                                                          int32_t* __restrict__ row_token,
-                                                         int32_t* __restrict__ row_dst) {
+                                                         int32_t* __restrict__ row_dst,
+                                                         unsigned long long* __restrict__ tok_flag,
+                                                         int32_t* __restrict__ sync, long long sync_words) {
   __shared__ uint32_t mask[kWarps][MOE_MAX_E_PLAN];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) mask[i / E][i % E] = 0u;
@@ -194,6 +191,10 @@ __global__ void __launch_bounds__(kTPB) plan_rank_kernel(const int32_t* __restri
   __syncthreads();
   const int t = blockIdx.x * kTPB + threadIdx.x;
   const bool valid = t < T;
+  // the pipelined-rounds kernel expects its counters and token flags at zero
+  if (valid && tok_flag) tok_flag[t] = 0ull;
+  if (sync)
+    for (long long i = t; i < sync_words; i += static_cast<long long>(gridDim.x) * kTPB) sync[i] = 0;
   if (valid)
     for (int j = 0; j < k; ++j) atomicOr(&mask[warp][idx[static_cast<size_t>(t) * k + j]], 1u << lane);
   __syncthreads();
@@ -227,11 +228,11 @@ cudaError_t launch_plan(const PlanBuffers& b, int T, int k, int E, int C, int ma
     err = launch_pdl(plan_scan_kernel, dim3(E), dim3(kTPB), 0, stream, b.block_base, blocks, E, b.load);
   if (err == cudaSuccess)
     err = launch_pdl(plan_finalize_kernel, dim3(1), dim3(kTPB), 0, stream, b.load, E, C, max_rounds,
-                     b.offsets, b.header, b.n, b.row_off, b.row_start, b.mb_prefix, b.sync,
-                     b.sync_words);
+                     b.offsets, b.header, b.n, b.row_off, b.row_start, b.mb_prefix);
   if (blocks > 0 && err == cudaSuccess)
     err = launch_pdl(plan_rank_kernel, dim3(blocks), dim3(kTPB), 0, stream, b.idx, T, k, E, C,
-                     b.block_base, b.row_off, b.round, b.slot, b.row_token, b.row_dst);
+                     b.block_base, b.row_off, b.round, b.slot, b.row_token, b.row_dst, b.tok_flag,
+                     b.sync, b.sync_words);
   launch_end(kKindPlan, stream, blocks > 0 ? 4 : 2);
   return err;
 }

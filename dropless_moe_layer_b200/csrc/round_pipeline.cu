@@ -9,34 +9,43 @@
 // launches each step pays a launch, a prologue and a pipeline fill. Here one CTA per SM runs
 // rounds [r0, R) and consecutive rounds overlap wherever the data allows.
 //
-// Roles of a CTA (320 threads):
-//   warps 0..5  the tcgen05 GEMM pipeline of gemm_sm100.cuh (TMA producer, MMA issuer, four
-//               epilogue warps) over the GEMM tile list below, tiles dealt round-robin to CTAs;
-//   warps 6..9  copy warps: the dispatch rows and combine items of every round, dealt
-//               round-robin over all copy warps of the grid.
+// Roles of a CTA (512 threads):
+//   warps 0..5    the tcgen05 GEMM pipeline of gemm_sm100.cuh (TMA producer, MMA issuer, four
+//                 epilogue warps) over the GEMM tile list below: the producer claims the next
+//                 tile of the list (a global counter) when it is ready for one, and passes its
+//                 index to the MMA and epilogue warps through a small shared-memory ring;
+//   warps 6..9    dispatch warps: each round's rows, in contiguous slices per warp of the grid;
+//   warps 10..15  combine warps: each round's combine items, round-robin over the grid's warps.
 // GEMM tile list, for r = r0..R-1: the gate/up tiles of round r (128 rows x 32 gate columns,
 // MMA N = 64, every column slice of a 128-row block before the next block), then its down
-// tiles (128 rows x 64 output columns). Copy steps: dispatch(r0), then for each r:
-// dispatch(r + 1), combine(r).
+// tiles (128 rows x 64 output columns).
 //
-// Dependencies, tracked by cumulative int32 counters in the workspace (zero before a launch;
-// the last CTA to finish zeroes them again). Every wait is bounded in time.
-//   gate/up(r, e, m)  after dispatch(r) rows of block (e, m)     buf is its A operand
-//                     after down(r-1) of block (e, m)           it overwrites h
-//   down(r, e, m)     after gate/up(r) of block (e, m)          h is its A operand
-//                     after combine(r-1)                        it overwrites out
-//   dispatch(r)       after every gate/up tile of round r-1     it overwrites buf
-//   combine(r)        after every down tile of round r          it reads out
-//                     after combine(r-1)                        y accumulates in round order
-// Each dependency points to a step earlier in the order
-//   D(r0) G(r0) N(r0) D(r0+1) C(r0) G(r0+1) N(r0+1) D(r0+2) C(r0+1) ...
-// and every role takes its own steps in that order. With every CTA resident (a cooperative
+// Round r uses buffer set p = (r - r0) & 1 (buf, h and out exist twice), so a round's buffers
+// are reused two rounds later and consecutive rounds do not wait on each other's reads.
+// Dependencies, tracked by int32 counters per buffer set in the workspace (zero before a
+// launch; the last CTA to finish zeroes them again). Every wait is bounded in time.
+//   dispatch(r, e, m) after gate/up(r-2) of block (e, m)        it overwrites buf[p]
+//   gate/up(r, e, m)  after dispatch(r) rows of block (e, m)     buf[p] is its A operand
+//                     after down(r-2) of block (e, m)           it overwrites h[p]
+//   down(r, e, m)     after gate/up(r) of block (e, m)          h[p] is its A operand
+//                     after combine(r-2) read block (e, m)      it overwrites out[p]
+//   combine(r, t)     after down(r) of the blocks holding t's    it reads out[p]
+//                     round-r rows
+//                     after combine(r', t), r' = t's previous   y[t] accumulates in round order
+//                     round (a per-token flag)
+// A counter of set p only ever receives the contributions of rounds of set p in round order
+// (round r+2 of a set cannot start its step before round r's is complete), so "count >=
+// target" means exactly "the earlier rounds of the set are done". Each dependency points to a
+// step earlier in the order
+//   D(r0) G(r0) N(r0)  D(r0+1) G(r0+1) N(r0+1) C(r0)  D(r0+2) G(r0+2) N(r0+2) C(r0+1) ...
+// and every role takes its own steps in that order (a combine warp its items round by round). With every CTA resident (a cooperative
 // launch of one CTA per SM) the earliest unfinished step always has its inputs and a role that
 // is working on it, so the launch cannot deadlock.
 //
-// Memory ordering: a producer of data issues its stores, a generic-to-async proxy fence and a
-// gpu-scope fence, then a release add on the counter; a consumer acquires the counter and, before
-// a TMA load, issues the proxy fence as well.
+// Memory ordering: the threads that wrote a step's data issue a generic-to-async proxy fence
+// (the data may next be read by TMA) and meet at __syncwarp; one lane then adds to the counter
+// with release semantics (cumulative over the warp's writes). A consumer acquires the counter
+// and, before a TMA load, issues the proxy fence as well.
 #include <cuda.h>
 
 #include <atomic>
@@ -58,9 +67,13 @@ constexpr int kPStages = kRingBytes / kPStageBytes;        // 8
 static_assert(kPStages <= kMaxStages, "ring stages");
 static_assert(kPipeDnWidth == kBN, "both GEMMs use one stage geometry");
 static_assert(kPipeRowBlock == BM, "row blocks are GEMM tiles");
-constexpr int kPipeCopyWarps = 4;
-constexpr int kPipeThreads = kThreads + 32 * kPipeCopyWarps;
+constexpr int kDispWarps = 4;
+constexpr int kCombWarps = 6;
+constexpr int kFirstDispWarp = kThreads / 32;
+constexpr int kFirstCombWarp = kFirstDispWarp + kDispWarps;
+constexpr int kPipeThreads = kThreads + 32 * (kDispWarps + kCombWarps);
 constexpr int kEpiWarps = 4;
+constexpr int kRing = 4;   // claimed tiles in flight between the producer and the consumers
 
 #ifdef MOE_TRACE
 // Diagnostic build only (-DMOE_TRACE): %globaltimer stamps of the launch, written to a buffer
@@ -109,16 +122,6 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-__device__ __forceinline__ int ld_acquire_cta_shared(const int* p) {
-  int v;
-  asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void st_release_cta_shared(int* p, int v) {
-  asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(p)), "r"(v) : "memory");
-}
-
 // Marks the launch as failed: status bit plus the abort word every wait watches.
 __device__ __forceinline__ void give_up(const PipelineArgs& a) {
   atomicOr(a.status, kStatusTimeoutPipeline);
@@ -131,26 +134,11 @@ __device__ bool wait_counter(const PipelineArgs& a, const int32_t* p, int target
   if (ld_acquire(p) >= target) return true;
   const uint64_t t0 = global_timer_ns();
   unsigned ns = 32;
-  while (true) {
+  for (uint32_t i = 1;; ++i) {
     __nanosleep(ns);
     if (ld_acquire(p) >= target) return true;
     if (ns < 256) ns <<= 1;
-    if (ld_relaxed(a.sync + kSyncAbort) != 0) return false;
-    if (global_timer_ns() - t0 > MOE_WAIT_LIMIT_NS) {
-      give_up(a);
-      return false;
-    }
-  }
-}
-
-// Same on a value that another warp of this CTA publishes in shared memory.
-__device__ bool wait_shared(const PipelineArgs& a, const int* p, int target) {
-  if (ld_acquire_cta_shared(p) >= target) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-    __nanosleep(64);
-    if (ld_acquire_cta_shared(p) >= target) return true;
-    if (ld_relaxed(a.sync + kSyncAbort) != 0) return false;
+    if ((i & 7) == 0 && ld_relaxed(a.sync + kSyncAbort) != 0) return false;
     if (global_timer_ns() - t0 > MOE_WAIT_LIMIT_NS) {
       give_up(a);
       return false;
@@ -160,11 +148,10 @@ __device__ bool wait_shared(const PipelineArgs& a, const int* p, int target) {
 
 // Walks the GEMM tile list forward, one round at a time.
 struct Cursor {
-  int r = 0;            // round of the tiles in [base, end)
+  int r = 0;             // round of the tiles in [base, end)
   int base = 0;
   int end = 0;
-  int gu_tiles = 0;     // gate/up tiles of round r (the first ones of the round)
-  int comb_before = 0;  // combine items of rounds r0..r-1
+  int gu_tiles = 0;      // gate/up tiles of round r (the first ones of the round)
 };
 
 __device__ __forceinline__ void cursor_load(Cursor& c, const PipelineArgs& a) {
@@ -176,7 +163,6 @@ __device__ __forceinline__ void cursor_load(Cursor& c, const PipelineArgs& a) {
 __device__ __forceinline__ void cursor_init(Cursor& c, const PipelineArgs& a) {
   c.r = a.r0;
   c.base = 0;
-  c.comb_before = 0;
   cursor_load(c, a);
 }
 
@@ -190,8 +176,6 @@ __device__ __forceinline__ int combine_items(const PipelineArgs& a, int r, bool*
 // Moves the cursor to the round holding `task`; false past the last round.
 __device__ __forceinline__ bool cursor_seek(Cursor& c, const PipelineArgs& a, int task) {
   while (task >= c.end) {
-    bool by_rows;
-    c.comb_before += combine_items(a, c.r, &by_rows);
     c.base = c.end;
     if (++c.r >= a.R) return false;
     cursor_load(c, a);
@@ -230,132 +214,204 @@ __device__ __forceinline__ void decode(const Cursor& c, const PipelineArgs& a, i
 }
 
 struct Counters {
-  int32_t* disp;   // [E * MB] dispatch rows written into block (e, m), all rounds
-  int32_t* gu;     // [E * MB] gate/up tile quarters finished on block (e, m)
-  int32_t* dn;     // [E * MB] down tile quarters finished on block (e, m)
-  int mb;          // 128-row blocks per expert = ceil(C / 128)
+  int32_t* disp[2];   // [E * MB] per set: dispatch rows written into block (e, m)
+  int32_t* gu[2];     // [E * MB] per set: gate/up tile quarters finished on block (e, m)
+  int32_t* dn[2];     // [E * MB] per set: down tile quarters finished on block (e, m)
+  int32_t* rd[2];     // [E * MB] per set: rows of block (e, m) of out read by the combine
+  int mb;             // 128-row blocks per expert = ceil(C / 128)
 };
 
 __device__ __forceinline__ Counters counters(const PipelineArgs& a) {
   Counters k;
   k.mb = static_cast<int>(pipe_row_blocks(a.C));
-  k.disp = a.sync + kSyncBlocks;
-  k.gu = k.disp + static_cast<size_t>(a.E) * k.mb;
-  k.dn = k.gu + static_cast<size_t>(a.E) * k.mb;
+  const size_t n = static_cast<size_t>(a.E) * k.mb * kSyncStride;
+  int32_t* base = a.sync + kSyncBlocks;
+  for (int p = 0; p < 2; ++p) {
+    k.disp[p] = base + p * n;
+    k.gu[p] = base + (2 + p) * n;
+    k.dn[p] = base + (4 + p) * n;
+    k.rd[p] = base + (6 + p) * n;
+  }
   return k;
 }
 
-// Producer: every input of tile t is in memory.
+// Producer: every input of tile t is in memory and its output buffer is free.
 __device__ bool wait_inputs(const PipelineArgs& a, const Counters& cn, const Cursor& c, const Tile& t) {
-  const int blk = t.e * cn.mb + t.m;
-  const int rr = t.r - a.r0;   // rounds of this launch before t.r
+  const int blk = (t.e * cn.mb + t.m) * kSyncStride;
+  const int p = (t.r - a.r0) & 1;
+  const int q = (t.r - a.r0) >> 1;   // earlier rounds of this launch on the same buffer set
   if (t.gu) {
     const int full = min(BM, a.C - t.m * BM);
     const int nv = a.n[static_cast<size_t>(t.r) * a.E + t.e] - t.m * BM;
     const int rows = nv < 0 ? 0 : (nv > BM ? BM : nv);
-    if (!wait_counter(a, cn.disp + blk, rr * full + rows)) return false;
-    if (rr > 0 && !wait_counter(a, cn.dn + blk, rr * kEpiWarps * (a.d / kPipeDnWidth))) return false;
+    if (!wait_counter(a, cn.disp[p] + blk, q * full + rows)) return false;
+    if (q > 0 && !wait_counter(a, cn.dn[p] + blk, q * kEpiWarps * (a.d / kPipeDnWidth))) return false;
   } else {
-    if (!wait_counter(a, cn.gu + blk, (rr + 1) * kEpiWarps * (a.F / kPipeGuWidth))) return false;
-    if (rr > 0 && !wait_counter(a, a.sync + kSyncCombTotal, c.comb_before)) return false;
+    if (!wait_counter(a, cn.gu[p] + blk, (q + 1) * kEpiWarps * (a.F / kPipeGuWidth))) return false;
+    if (q > 0 && !wait_counter(a, cn.rd[p] + blk, q * min(BM, a.C - t.m * BM))) return false;
   }
   return true;
 }
 
-// Copy warps: a round-level wait. Copy warp 0 of the CTA polls the global counter and publishes
-// what it saw in shared memory; the other copy warps wait on that word.
-__device__ bool round_wait(const PipelineArgs& a, int* seen, const int32_t* counter, int target, int cwarp) {
+// Dispatch warps: round r's rows x[token] -> buf[p][e][slot], each warp a contiguous slice.
+__device__ void dispatch_role(const PipelineArgs& a, const Counters& cn) {
   const int lane = threadIdx.x & 31;
-  int ok = 1;
-  if (lane == 0) {
-    if (cwarp == 0) {
-      ok = wait_counter(a, counter, target);
-      if (ok) st_release_cta_shared(seen, target);
-    } else {
-      ok = wait_shared(a, seen, target);
+  const int dw = (threadIdx.x >> 5) - kFirstDispWarp;
+  const int gw = blockIdx.x * kDispWarps + dw;
+  const int W = gridDim.x * kDispWarps;
+  const int vecs = a.d / 8;
+  for (int r = a.r0; r < a.R; ++r) {
+    const int p = (r - a.r0) & 1;
+    const int q = (r - a.r0) >> 1;
+    // block (e, m) of buf[p] is free once every gate/up tile of it in round r-2 has read it
+    const int war_target = q * kEpiWarps * (a.F / kPipeGuWidth);
+    const int begin = a.row_start[r], rows = a.row_start[r + 1] - begin;
+    const int chunk = (rows + W - 1) / W;
+    const int lo = gw * chunk, hi = min(rows, lo + chunk);
+    MOE_TRACE_DO(if (lane == 0 && lo < hi) trace_min(trace_round(r, 0), global_timer_ns()));
+    for (int b = lo; b < hi; b += 32) {
+      const int nr = min(32, hi - b);
+      int tok = 0, dst = 0, blk = -1;
+      if (lane < nr) {
+        tok = a.row_token[begin + b + lane];
+        dst = a.row_dst[begin + b + lane];
+        const int e = dst / a.C;
+        blk = (e * cn.mb + (dst - e * a.C) / BM) * kSyncStride;
+      }
+      // rows are in (expert, slot) order: runs of rows of the same block
+      const int prev = __shfl_up_sync(0xffffffffu, blk, 1);
+      const bool head = lane < nr && (lane == 0 || prev != blk);
+      const uint32_t heads = __ballot_sync(0xffffffffu, head);
+      const uint32_t later = lane == 31 ? 0u : (heads & ~((2u << lane) - 1u));
+      const int run_end = later ? __ffs(later) - 1 : nr;
+      if (q > 0) {
+        int ok = 1;
+        if (head) ok = wait_counter(a, cn.gu[p] + blk, war_target);
+        if (!__all_sync(0xffffffffu, ok)) return;
+        fence_proxy_async();
+      }
+      copy::copy_rows_flat(reinterpret_cast<const uint4*>(a.x), reinterpret_cast<uint4*>(a.buf[p]), tok, dst,
+                           nr, vecs);
+      fence_proxy_async();   // the rows are read next by TMA (the async proxy)
+      __syncwarp();
+      if (head) red_release(cn.disp[p] + blk, run_end - lane);
     }
+    MOE_TRACE_DO(if (lane == 0 && lo < hi) trace_max(trace_round(r, 1), global_timer_ns()));
   }
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
-  return ok != 0;
 }
 
-// The four copy warps of this CTA: dispatch rows and combine items of rounds r0..R-1.
-__device__ void copy_role(const PipelineArgs& a, const Counters& cn, int* seen) {
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Bounded wait (one thread) until the token flag reaches `target`.
+__device__ bool wait_flag(const PipelineArgs& a, const unsigned long long* p, unsigned long long target) {
+  if (ld_acquire_u64(p) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    __nanosleep(32);
+    if (ld_acquire_u64(p) >= target) return true;
+    if ((i & 7) == 0 && ld_relaxed(a.sync + kSyncAbort) != 0) return false;
+    if (global_timer_ns() - t0 > MOE_WAIT_LIMIT_NS) {
+      give_up(a);
+      return false;
+    }
+  }
+}
+
+// Combine warps: y[t] (+)= gate * out[p][e][slot] for round r. A token waits only for the down
+// tiles of the blocks its own round-r rows live in, and for its own previous round's combine;
+// once its rows are read it counts them on their blocks, which the down GEMM two rounds later
+// waits for before it overwrites them.
+__device__ void combine_role(const PipelineArgs& a, const Counters& cn) {
   const int lane = threadIdx.x & 31;
-  const int cwarp = (threadIdx.x >> 5) - kThreads / 32;
-  const int gw = blockIdx.x * kPipeCopyWarps + cwarp;
-  const int W = gridDim.x * kPipeCopyWarps;
-  const int vecs = a.d / 8;
-  const copy::CombineArgs comb{a.out, a.y, a.idx, a.gate, a.round, a.slot, a.T, a.k, a.C, a.d};
-
-  auto dispatch_round = [&](int r) {
-    const int begin = a.row_start[r], rows = a.row_start[r + 1] - begin;
-    MOE_TRACE_DO(if (lane == 0 && gw < rows) trace_min(trace_round(r, 0), global_timer_ns()));
-    for (int i = gw; i < rows; i += W) {
-      const int row = begin + i;
-      const int t = a.row_token[row], dst = a.row_dst[row];
-      const int e = dst / a.C, m = (dst - e * a.C) / BM;
-      copy::dispatch_row(reinterpret_cast<const uint4*>(a.x), reinterpret_cast<uint4*>(a.buf), t, dst, vecs, lane);
-      fence_proxy_async();   // the row is read next by TMA (the async proxy)
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) red_release(cn.disp + e * cn.mb + m, 1);
-    }
-    MOE_TRACE_DO(if (lane == 0 && gw < rows) trace_max(trace_round(r, 1), global_timer_ns()));
-  };
-
-  dispatch_round(a.r0);
-  int gu_through = 0, dn_through = 0, comb_before = 0;
+  const int cw = (threadIdx.x >> 5) - kFirstCombWarp;
+  const int gw = blockIdx.x * kCombWarps + cw;
+  const int W = gridDim.x * kCombWarps;
+  int dn_cum[2] = {0, 0};
   for (int r = a.r0; r < a.R; ++r) {
+    const int p = (r - a.r0) & 1;
+    const int q = (r - a.r0) >> 1;
     const int mblocks = a.mb_prefix[static_cast<size_t>(r) * (a.E + 1) + a.E];
-    gu_through += mblocks * kEpiWarps * (a.F / kPipeGuWidth);
-    dn_through += mblocks * kEpiWarps * (a.d / kPipeDnWidth);
-    if (r + 1 < a.R) {
-      // buf is free once every gate/up tile of round r has read it
-      if (!round_wait(a, &seen[0], a.sync + kSyncGuTotal, gu_through, cwarp)) return;
-      fence_proxy_async();
-      dispatch_round(r + 1);
-    }
-    if (!round_wait(a, &seen[1], a.sync + kSyncDnTotal, dn_through, cwarp)) return;
-    if (!round_wait(a, &seen[2], a.sync + kSyncCombTotal, comb_before, cwarp)) return;
+    dn_cum[p] += mblocks * kEpiWarps * (a.d / kPipeDnWidth);
+    const int blk_target = (q + 1) * kEpiWarps * (a.d / kPipeDnWidth);
+    const copy::CombineArgs comb{a.out[p], a.y, a.idx, a.gate, a.round, a.slot, a.T, a.k, a.C, a.d};
     bool by_rows;
     const int items = combine_items(a, r, &by_rows);
     MOE_TRACE_DO(if (lane == 0 && gw < items) trace_min(trace_round(r, 2), global_timer_ns()));
-    int done = 0;
-    for (int u = gw; u < items; u += W, ++done) {
-      if (by_rows) {
-        const int row = a.row_start[r] + u;
-        copy::combine_token(comb, a.row_token[row], r, a.row_dst[row] / a.C);
-      } else {
-        copy::combine_token(comb, u, r);
+    bool round_done = false;   // every down tile of round r seen finished
+    // this warp's items u = gw + i * W, 32 at a time: lane i fetches item i's token first
+    for (int base = gw; base < items; base += 32 * W) {
+      const int u_l = base + lane * W;
+      int t_l = u_l, only_l = -1;
+      if (by_rows && u_l < items) {
+        const int row = a.row_start[r] + u_l;
+        t_l = a.row_token[row];
+        only_l = a.row_dst[row] / a.C;
+      }
+      const int n_here = min(32, (items - base + W - 1) / W);
+      copy::PairLoads next = copy::load_pairs(comb, __shfl_sync(0xffffffffu, t_l, 0));
+      for (int i = 0; i < n_here; ++i) {
+        const int t = __shfl_sync(0xffffffffu, t_l, i);
+        const int only = __shfl_sync(0xffffffffu, only_l, i);
+        const copy::PairLoads cur = next;
+        if (i + 1 < n_here) next = copy::load_pairs(comb, __shfl_sync(0xffffffffu, t_l, i + 1));
+        const copy::TokenPairs tp = copy::token_pairs(comb, cur, r);
+        if (tp.npairs == 0 || (only >= 0 && tp.first_expert != only)) continue;
+        const int blk = (tp.e * cn.mb + tp.s / BM) * kSyncStride;   // this lane's pair's block
+        if (!round_done) {
+          int ok = 1;
+          if (lane == 0) round_done = ld_acquire(a.sync + kSyncDnTotal + p * kSyncSetStride) >= dn_cum[p];
+          round_done = __shfl_sync(0xffffffffu, round_done ? 1 : 0, 0) != 0;
+          if (!round_done && lane < tp.npairs) ok = wait_counter(a, cn.dn[p] + blk, blk_target);
+          if (!__all_sync(0xffffffffu, ok)) return;
+        }
+        if (tp.prev_round >= a.r0) {   // y[t] holds the previous round's sum once its flag is set
+          int ok = 1;
+          if (lane == 0) ok = wait_flag(a, a.tok_flag + t, (a.gen << 32) | static_cast<unsigned>(tp.prev_round + 1));
+          if (!__shfl_sync(0xffffffffu, ok, 0)) return;
+        }
+        __syncwarp();
+        copy::accumulate_token<16>(comb, t, tp);
+        __syncwarp();
+        if (lane == 0) st_release_u64(a.tok_flag + t, (a.gen << 32) | static_cast<unsigned>(r + 1));
+        if (lane < tp.npairs) red_release(cn.rd[p] + blk, 1);   // this pair's out row is read
       }
     }
-    if (done > 0) {
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) red_release(a.sync + kSyncCombTotal, done);
-      MOE_TRACE_DO(if (lane == 0) trace_max(trace_round(r, 3), global_timer_ns()));
-    }
-    comb_before += items;
+    MOE_TRACE_DO(if (lane == 0 && gw < items) trace_max(trace_round(r, 3), global_timer_ns()));
   }
 }
 
 __global__ void __launch_bounds__(kPipeThreads, 1)
-    round_pipeline_kernel(const __grid_constant__ CUtensorMap a_gu, const __grid_constant__ CUtensorMap b_gu,
-                          const __grid_constant__ CUtensorMap a_dn, const __grid_constant__ CUtensorMap b_dn,
+    round_pipeline_kernel(const __grid_constant__ CUtensorMap a_gu0, const __grid_constant__ CUtensorMap a_gu1,
+                          const __grid_constant__ CUtensorMap b_gu, const __grid_constant__ CUtensorMap a_dn0,
+                          const __grid_constant__ CUtensorMap a_dn1, const __grid_constant__ CUtensorMap b_dn,
                           const PipelineArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ int seen[3];
   __shared__ int last_cta;
+  // tile ring: the producer publishes each claimed tile (-1: no more) to the MMA issuer and the
+  // four epilogue warps
+  __shared__ uint64_t ring_full[kRing], ring_empty[kRing];
+  __shared__ int ring_task[kRing];
   const Smem s = carve(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    tma_prefetch_desc(&a_gu);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(smem_addr(&ring_full[i]), 1);
+      mbar_init(smem_addr(&ring_empty[i]), 1 + kEpiWarps);
+    }
+    tma_prefetch_desc(&a_gu0);
+    tma_prefetch_desc(&a_gu1);
     tma_prefetch_desc(&b_gu);
-    tma_prefetch_desc(&a_dn);
+    tma_prefetch_desc(&a_dn0);
+    tma_prefetch_desc(&a_dn1);
     tma_prefetch_desc(&b_dn);
-    seen[0] = seen[1] = seen[2] = 0;
   }
   const uint32_t tmem = setup(s);
   grid_dependency_wait();
@@ -378,11 +434,26 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
           tma_load_3d(sB, &b_dn, fb, kb * BK, t.nt * kPipeDnWidth, t.e);
         }
       };
-      for (int task = blockIdx.x; ok; task += gridDim.x) {
-        if (!cursor_seek(c, a, task)) break;
+      int slot = 0;
+      uint32_t rphase = 0;
+      while (ok) {
+        const int task = atomicAdd(a.sync + kSyncNextTask, 1);
+        const bool have = cursor_seek(c, a, task);
+        if (!mbar_wait(smem_addr(&ring_empty[slot]), rphase ^ 1u, s.abort)) {
+          ok = false;
+          break;
+        }
+        ring_task[slot] = have ? task : -1;
+        mbar_arrive(smem_addr(&ring_full[slot]));
+        if (++slot == kRing) {
+          slot = 0;
+          rphase ^= 1u;
+        }
+        if (!have) break;
         Tile t;
         decode(c, a, task, t);
-        const CUtensorMap* ma = t.gu ? &a_gu : &a_dn;
+        const bool set1 = ((t.r - a.r0) & 1) != 0;
+        const CUtensorMap* ma = t.gu ? (set1 ? &a_gu1 : &a_gu0) : (set1 ? &a_dn1 : &a_dn0);
         // Weights do not depend on earlier steps: the B tiles of the first stages are requested
         // before the wait for this tile's A rows, so they arrive while it waits.
         const int pre = t.kb < kPStages ? t.kb : kPStages;
@@ -454,8 +525,20 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int task = blockIdx.x; ok; task += gridDim.x) {
-        if (!cursor_seek(c, a, task)) break;
+      int slot = 0;
+      uint32_t rphase = 0;
+      while (ok) {
+        if (!mbar_wait(smem_addr(&ring_full[slot]), rphase, s.abort)) {
+          ok = false;
+          break;
+        }
+        const int task = ring_task[slot];
+        mbar_arrive(smem_addr(&ring_empty[slot]));
+        if (++slot == kRing) {
+          slot = 0;
+          rphase ^= 1u;
+        }
+        if (task < 0 || !cursor_seek(c, a, task)) break;
         Tile t;
         decode(c, a, task, t);
         if (!mbar_wait(smem_addr(&s.tempty[acc]), acc_phase ^ 1u, s.abort)) {
@@ -505,8 +588,25 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     cursor_init(c, a);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int task = blockIdx.x;; task += gridDim.x) {
-      if (!cursor_seek(c, a, task)) break;
+    int slot = 0;
+    uint32_t rphase = 0;
+    while (true) {
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&ring_full[slot]), rphase, s.abort))) {
+        if (lane == 0) {
+          atomicOr(a.status, kStatusTimeoutEpilogue);
+          atomicExch(a.sync + kSyncAbort, 1);
+        }
+        *s.abort = 1;
+        break;
+      }
+      const int task = ring_task[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&ring_empty[slot]));
+      if (++slot == kRing) {
+        slot = 0;
+        rphase ^= 1u;
+      }
+      if (task < 0 || !cursor_seek(c, a, task)) break;
       Tile t;
       decode(c, a, task, t);
       const bool ready = __all_sync(0xffffffffu, mbar_wait(smem_addr(&s.tfull[acc]), acc_phase, s.abort));
@@ -523,11 +623,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       const int row = t.m * BM + q * 32 + lane;
       const bool valid = row < a.n[static_cast<size_t>(t.r) * a.E + t.e];
       const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kAccCols);
+      const int p = (t.r - a.r0) & 1;
       if (t.gu) {
-        uint16_t* orow = a.h + (static_cast<size_t>(t.e) * a.C + row) * a.F + t.nt * kPipeGuWidth;
+        uint16_t* orow = a.h[p] + (static_cast<size_t>(t.e) * a.C + row) * a.F + t.nt * kPipeGuWidth;
         store_swiglu(tb, kPipeGuWidth, orow, valid);
       } else {
-        uint16_t* orow = a.out + (static_cast<size_t>(t.e) * a.C + row) * a.d + t.nt * kPipeDnWidth;
+        uint16_t* orow = a.out[p] + (static_cast<size_t>(t.e) * a.C + row) * a.d + t.nt * kPipeDnWidth;
         store_bf16(tb, kPipeDnWidth, orow, valid);
       }
       tc_fence_before();
@@ -536,18 +637,20 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       if (acc == 0) acc_phase ^= 1u;
       // this warp's quarter of the tile is in memory
       fence_proxy_async();
-      __threadfence();
       __syncwarp();
       if (lane == 0) {
-        const int blk = t.e * cn.mb + t.m;
-        red_release((t.gu ? cn.gu : cn.dn) + blk, 1);
-        red_release(a.sync + (t.gu ? kSyncGuTotal : kSyncDnTotal), 1);
+        const int blk = (t.e * cn.mb + t.m) * kSyncStride;
+        red_release((t.gu ? cn.gu[p] : cn.dn[p]) + blk, 1);
+        if (!t.gu) red_release(a.sync + kSyncDnTotal + p * kSyncSetStride, 1);
         MOE_TRACE_DO(if (warp == 2) trace_task(task, 2, global_timer_ns()));
       }
     }
     __syncwarp();
+  } else if (warp < kFirstCombWarp) {
+    dispatch_role(a, cn);
+    __syncwarp();
   } else {
-    copy_role(a, cn, seen);
+    combine_role(a, cn);
     __syncwarp();
   }
 
@@ -579,10 +682,16 @@ extern "C" MOE_API int moe_trace_set(void* buffer) {
 
 cudaError_t launch_round_pipeline(const PipelineArgs& a, cudaStream_t stream) {
   if (a.r0 >= a.R) return cudaSuccess;
-  CUtensorMap m_agu, m_bgu, m_adn, m_bdn;
-  cudaError_t e = gemm::make_map(&m_agu, a.buf, a.d, a.C, a.E, BM);
+  if (a.tok_flag == nullptr) return cudaErrorInvalidValue;
+  for (int p = 0; p < 2; ++p)
+    if (a.buf[p] == nullptr || a.h[p] == nullptr || a.out[p] == nullptr) return cudaErrorInvalidValue;
+  CUtensorMap m_agu[2], m_bgu, m_adn[2], m_bdn;
+  cudaError_t e = cudaSuccess;
+  for (int p = 0; p < 2 && e == cudaSuccess; ++p) {
+    e = gemm::make_map(&m_agu[p], a.buf[p], a.d, a.C, a.E, BM);
+    if (e == cudaSuccess) e = gemm::make_map(&m_adn[p], a.h[p], a.F, a.C, a.E, BM);
+  }
   if (e == cudaSuccess) e = gemm::make_map(&m_bgu, a.w_gate_up, a.d, 2ull * a.F, a.E, kPipeGuWidth);
-  if (e == cudaSuccess) e = gemm::make_map(&m_adn, a.h, a.F, a.C, a.E, BM);
   if (e == cudaSuccess) e = gemm::make_map(&m_bdn, a.w_down, a.F, a.d, a.E, kPipeDnWidth);
   if (e != cudaSuccess) return e;
   static std::atomic<uint64_t> configured{0};   // one bit per device ordinal
@@ -607,7 +716,13 @@ cudaError_t launch_round_pipeline(const PipelineArgs& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   launch_begin(kKindPipeline, stream);
-  e = cudaLaunchKernelEx(&cfg, round_pipeline_kernel, m_agu, m_bgu, m_adn, m_bdn, a);
+  // token flags hold (generation << 32) | (round + 1): a flag left by an earlier launch on the
+  // same workspace is below every target of this one, so the flags are never cleared between
+  // launches (the planner zeroes them once per plan)
+  static std::atomic<unsigned long long> generation{0};
+  PipelineArgs args = a;
+  args.gen = generation.fetch_add(1) + 1;
+  e = cudaLaunchKernelEx(&cfg, round_pipeline_kernel, m_agu[0], m_agu[1], m_bgu, m_adn[0], m_adn[1], m_bdn, args);
   launch_end(kKindPipeline, stream);
   return e;
 }

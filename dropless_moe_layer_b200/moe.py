@@ -43,7 +43,7 @@ class WorkspaceLayout(ctypes.Structure):
     _fields_ = [(name, c_sz) for name in (
         "total_bytes", "header", "logits", "topk_idx", "gate", "round", "slot", "load",
         "offsets", "block_base", "n", "row_off", "row_start", "row_token", "row_dst", "buf", "h", "out",
-        "mb_prefix", "sync")
+        "mb_prefix", "sync", "tok_flag", "buf2", "h2", "out2")
     ] + [("max_rounds", c_i32), ("plan_blocks", c_i32)]
 
 
@@ -300,7 +300,7 @@ class DroplessMoE:
         """The pipelined launch's dependency counters (all zero between calls)."""
         import torch
         s, L = self.shape, self.layout
-        words = 32 + 3 * s.E * ((s.C + 127) // 128)
+        words = 448 + 8 * s.E * ((s.C + 127) // 128) * 8
         return self._view(L.sync, words, torch.int32)
 
     def round_step(self, step: str, r: int, ptr_tensor, stream=None) -> None:

@@ -75,7 +75,11 @@ typedef enum moe_status {
 /* moe_shape_t.flags */
 #define MOE_FLAG_RENORM_TOPK 1u     /* divide the k selected gates of a token by their sum */
 /* Launch schedule of moe_forward (results are identical; only the overlap of rounds differs).
- * Default: per-round launches. */
+ * Default: the trailing run of thin rounds (whose gate/up GEMM has fewer 128-row x 128-column
+ * tiles than the GPU has SMs) runs in one pipelined launch, the rounds before it as per-round
+ * launches. The pipelined launch
+ * alternates two sets of round buffers, so the workspace holds a second set unless
+ * MOE_FLAG_PER_ROUND is given. */
 #define MOE_FLAG_PER_ROUND 2u       /* every round as per-round launches */
 #define MOE_FLAG_PIPELINE_ALL 4u    /* every round in the pipelined launch */
 
@@ -125,8 +129,12 @@ typedef struct moe_workspace_layout {
   size_t h;           /* bf16 [E, C, d_ff]: SwiGLU activations of the round */
   size_t out;         /* bf16 [E, C, d]: expert outputs of the round */
   size_t mb_prefix;   /* i32 [max_rounds, E + 1]: 128-row blocks of experts < e in round r */
-  size_t sync;        /* i32 [32 + 3 * E * ceil(C / 128)]: pipelined launch's dependency
+  size_t sync;        /* i32 [448 + 64 * E * ceil(C / 128)]: pipelined launch's dependency
                          counters (zero between calls) */
+  size_t tok_flag;    /* u64 [T]: pipelined launch's per-token combine progress */
+  size_t buf2;        /* second buffer set of the pipelined launch (rounds alternate sets); */
+  size_t h2;          /* absent (0) with MOE_FLAG_PER_ROUND, which never uses it */
+  size_t out2;
   int32_t max_rounds; /* ceil(T / C): no expert can receive more than T tokens */
   int32_t plan_blocks;
 } moe_workspace_layout_t;

@@ -30,8 +30,9 @@ def test_status_strings(lib):
     assert lib.moe_status_string(12345) == b"unknown status"
 
 
-def _bytes_model(w):
-    """Workspace size from the layout rules: 256-byte aligned regions."""
+def _bytes_model(w, per_round=False):
+    """Workspace size from the layout rules: 256-byte aligned regions; a second set of round
+    buffers unless the schedule is per-round only."""
     def a(n):
         return (n + 255) // 256 * 256
     T, E, k, C, d, F = w.T, w.E, w.k, w.C, w.d, w.F
@@ -40,7 +41,8 @@ def _bytes_model(w):
     return (a(320 * 4) + a(T * E * 4) + 4 * a(T * k * 4) + a(E * 4) + a((E + 1) * 4)
             + a(blocks * E * 4) + 2 * a(mr * E * 4) + a((mr + 1) * 4) + 2 * a(T * k * 4)
             + a(E * C * d * 2) + a(E * C * F * 2) + a(E * C * d * 2)
-            + a(mr * (E + 1) * 4) + a((32 + 3 * E * ((C + 127) // 128)) * 4))
+            + a(mr * (E + 1) * 4) + a((448 + 8 * E * ((C + 127) // 128) * 8) * 4) + a(T * 8)
+            + (0 if per_round else a(E * C * d * 2) + a(E * C * F * 2) + a(E * C * d * 2)))
 
 
 @pytest.mark.parametrize("w", wl.WORKLOADS, ids=lambda w: w.name)
@@ -54,9 +56,14 @@ def test_workspace_is_fixed_by_shape(lib, w):
     assert lay.total_bytes == n
     offs = [lay.header, lay.logits, lay.topk_idx, lay.gate, lay.round, lay.slot, lay.load,
             lay.offsets, lay.block_base, lay.n, lay.row_off, lay.row_start, lay.row_token,
-            lay.row_dst, lay.buf, lay.h, lay.out, lay.mb_prefix, lay.sync]
+            lay.row_dst, lay.buf, lay.h, lay.out]
+    offs += [lay.mb_prefix, lay.sync, lay.tok_flag, lay.buf2, lay.h2, lay.out2]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     assert lay.max_rounds == (w.T + w.C - 1) // w.C
+    s1 = moe.make_shape(w.T, w.d, w.E, w.k, w.F, w.C, schedule="per_round")
+    assert moe.workspace_bytes(s1) == _bytes_model(w, per_round=True)
+    lay1 = moe.workspace_layout(s1)
+    assert lay1.buf2 == lay1.h2 == lay1.out2 == 0
 
 
 @pytest.mark.parametrize("kw", [
@@ -77,9 +84,11 @@ def test_bad_flags_rejected(lib):
     for flags in (8, 1 << 31, moe.FLAG_PER_ROUND | moe.FLAG_PIPELINE_ALL):
         s.flags = flags
         assert moe.workspace_bytes(s) == 0
-    for schedule in moe.SCHEDULES:   # the schedule flags do not change the fixed memory
-        assert moe.workspace_bytes(moe.make_shape(64, 128, 8, 2, 128, 16, schedule=schedule)) == \
-            moe.workspace_bytes(moe.make_shape(64, 128, 8, 2, 128, 16))
+    # the pipelined schedules share one layout; per-round only drops the second buffer set
+    assert moe.workspace_bytes(moe.make_shape(64, 128, 8, 2, 128, 16, schedule="pipeline")) == \
+        moe.workspace_bytes(moe.make_shape(64, 128, 8, 2, 128, 16))
+    assert moe.workspace_bytes(moe.make_shape(64, 128, 8, 2, 128, 16, schedule="per_round")) < \
+        moe.workspace_bytes(moe.make_shape(64, 128, 8, 2, 128, 16))
 
 
 def test_plan_argument_errors_without_gpu(lib):
