@@ -114,7 +114,6 @@ struct PlanBuffers {
   int32_t* mb_prefix;     // [max_rounds, E + 1] 128-row blocks of experts < e in round r, or null
   int32_t* sync;          // pipelined-rounds counters to zero ([sync_words]), or null
   long long sync_words;
-  unsigned long long* tok_flag;   // [T] per-token combine progress to zero, or null
 };
 cudaError_t launch_plan(const PlanBuffers& b, int T, int k, int E, int C, int max_rounds,
                         cudaStream_t stream);
@@ -184,8 +183,6 @@ struct PipelineArgs {
   const int32_t* row_dst;
   const int32_t* mb_prefix;  // [max_rounds, E + 1]
   int32_t* sync;
-  unsigned long long* tok_flag;  // [T] (gen << 32) | (last round combined in this launch + 1)
-  unsigned long long gen;        // launch generation (increases from launch to launch)
   int32_t* status;
   int T, k, E, C, d, F, r0, R;
 };

@@ -122,7 +122,6 @@ void make_layout(const moe_shape_t* s, moe_workspace_layout_t* L) {
   L->out = take(E * C * s->d * 2);
   L->mb_prefix = take(static_cast<long long>(mr) * (E + 1) * 4);
   L->sync = take(pipe_sync_words(s->E, s->C) * 4);
-  L->tok_flag = take(T * 8);
   if (!(s->flags & MOE_FLAG_PER_ROUND)) {   // second buffer set of the pipelined launch
     L->buf2 = take(E * C * s->d * 2);
     L->h2 = take(E * C * s->d_ff * 2);
@@ -325,7 +324,6 @@ int moe_plan(const moe_shape_t* shape, const float* logits, const uint16_t* x,
   pb.mb_prefix = at<int32_t>(ws, L.mb_prefix);
   pb.sync = at<int32_t>(ws, L.sync);
   pb.sync_words = pipe_sync_words(s.E, s.C);
-  pb.tok_flag = at<unsigned long long>(ws, L.tok_flag);
   if ((st = cuda_status(launch_plan(pb, s.T, s.k, s.E, s.C, L.max_rounds, stream))) != MOE_OK) return st;
 
   int32_t host[kHdrWords];
@@ -467,7 +465,6 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
     p.row_dst = at<int32_t>(ws, L.row_dst);
     p.mb_prefix = at<int32_t>(ws, L.mb_prefix);
     p.sync = at<int32_t>(ws, L.sync);
-    p.tok_flag = at<unsigned long long>(ws, L.tok_flag);
     p.status = at<int32_t>(ws, L.header) + kHdrStatus;
     p.T = shape->T;
     p.k = shape->k;

@@ -181,7 +181,6 @@ __global__ void __launch_bounds__(kTPB) plan_rank_kernel(const int32_t* __restri
                                                          int32_t* __restrict__ slot_out,
                                                          int32_t* __restrict__ row_token,
                                                          int32_t* __restrict__ row_dst,
-                                                         unsigned long long* __restrict__ tok_flag,
                                                          int32_t* __restrict__ sync, long long sync_words) {
   __shared__ uint32_t mask[kWarps][MOE_MAX_E_PLAN];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -191,8 +190,7 @@ __global__ void __launch_bounds__(kTPB) plan_rank_kernel(const int32_t* __restri
   __syncthreads();
   const int t = blockIdx.x * kTPB + threadIdx.x;
   const bool valid = t < T;
-  // the pipelined-rounds kernel expects its counters and token flags at zero
-  if (valid && tok_flag) tok_flag[t] = 0ull;
+  // the pipelined-rounds kernel expects its counters at zero
   if (sync)
     for (long long i = t; i < sync_words; i += static_cast<long long>(gridDim.x) * kTPB) sync[i] = 0;
   if (valid)
@@ -231,8 +229,8 @@ cudaError_t launch_plan(const PlanBuffers& b, int T, int k, int E, int C, int ma
                      b.offsets, b.header, b.n, b.row_off, b.row_start, b.mb_prefix);
   if (blocks > 0 && err == cudaSuccess)
     err = launch_pdl(plan_rank_kernel, dim3(blocks), dim3(kTPB), 0, stream, b.idx, T, k, E, C,
-                     b.block_base, b.row_off, b.round, b.slot, b.row_token, b.row_dst, b.tok_flag,
-                     b.sync, b.sync_words);
+                     b.block_base, b.row_off, b.round, b.slot, b.row_token, b.row_dst, b.sync,
+                     b.sync_words);
   launch_end(kKindPlan, stream, blocks > 0 ? 4 : 2);
   return err;
 }

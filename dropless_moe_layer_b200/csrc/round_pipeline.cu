@@ -15,10 +15,10 @@
 //                 tile of the list (a global counter) when it is ready for one, and passes its
 //                 index to the MMA and epilogue warps through a small shared-memory ring;
 //   warps 6..9    dispatch warps: each round's rows, in contiguous slices per warp of the grid;
-//   warps 10..15  combine warps: each round's combine items, round-robin over the grid's warps.
-// GEMM tile list, for r = r0..R-1: the gate/up tiles of round r (128 rows x 32 gate columns,
-// MMA N = 64, every column slice of a 128-row block before the next block), then its down
-// tiles (128 rows x 64 output columns).
+//   warps 10..15  combine warps: each owns a fixed set of tokens and combines them round by round.
+// GEMM tile list: gate/up tiles (128 rows x 32 gate columns, MMA N = 64, every column slice of
+// a 128-row block before the next block) and down tiles (128 rows x 64 output columns), phase
+// by phase in the order G(r0) G(r0+1) N(r0) G(r0+2) N(r0+1) ... N(R-1).
 //
 // Round r uses buffer set p = (r - r0) & 1 (buf, h and out exist twice), so a round's buffers
 // are reused two rounds later and consecutive rounds do not wait on each other's reads.
@@ -30,14 +30,14 @@
 //   down(r, e, m)     after gate/up(r) of block (e, m)          h[p] is its A operand
 //                     after combine(r-2) read block (e, m)      it overwrites out[p]
 //   combine(r, t)     after down(r) of the blocks holding t's    it reads out[p]
-//                     round-r rows
-//                     after combine(r', t), r' = t's previous   y[t] accumulates in round order
-//                     round (a per-token flag)
+//                     round-r rows (y[t] accumulates in round order by construction: one
+//                     warp owns token t for all rounds)
 // A counter of set p only ever receives the contributions of rounds of set p in round order
 // (round r+2 of a set cannot start its step before round r's is complete), so "count >=
 // target" means exactly "the earlier rounds of the set are done". Each dependency points to a
 // step earlier in the order
-//   D(r0) G(r0) N(r0)  D(r0+1) G(r0+1) N(r0+1) C(r0)  D(r0+2) G(r0+2) N(r0+2) C(r0+1) ...
+//   D(r0) G(r0)  D(r0+1) G(r0+1) N(r0)  D(r0+2) G(r0+2) N(r0+1) C(r0)  D(r0+3) G(r0+3) N(r0+2)
+//   C(r0+1) ...
 // and every role takes its own steps in that order (a combine warp its items round by round). With every CTA resident (a cooperative
 // launch of one CTA per SM) the earliest unfinished step always has its inputs and a role that
 // is working on it, so the launch cannot deadlock.
@@ -146,40 +146,53 @@ __device__ bool wait_counter(const PipelineArgs& a, const int32_t* p, int target
   }
 }
 
-// Walks the GEMM tile list forward, one round at a time.
+// Walks the GEMM tile list forward, one phase (the gate/up or the down tiles of one round) at a
+// time. Phase order: G(r0), then for each r: G(r + 1), N(r) -- the gate/up tiles run one round
+// ahead, so that CTAs waiting for a round's gate/up results are not the ones that could start
+// the next round's gate/up.
 struct Cursor {
-  int r = 0;             // round of the tiles in [base, end)
-  int base = 0;
-  int end = 0;
-  int gu_tiles = 0;      // gate/up tiles of round r (the first ones of the round)
+  bool gu = true;        // phase kind: gate/up (else down)
+  int r = 0;             // round of the phase
+  int base = 0;          // first task of the phase
+  int end = 0;           // one past its last task
 };
 
 __device__ __forceinline__ void cursor_load(Cursor& c, const PipelineArgs& a) {
   const int mblocks = a.mb_prefix[static_cast<size_t>(c.r) * (a.E + 1) + a.E];
-  c.gu_tiles = mblocks * (a.F / kPipeGuWidth);
-  c.end = c.base + c.gu_tiles + mblocks * (a.d / kPipeDnWidth);
+  c.end = c.base + mblocks * (c.gu ? a.F / kPipeGuWidth : a.d / kPipeDnWidth);
 }
 
 __device__ __forceinline__ void cursor_init(Cursor& c, const PipelineArgs& a) {
+  c.gu = true;
   c.r = a.r0;
   c.base = 0;
   cursor_load(c, a);
 }
 
-// Combine items of round r: its rows when there are fewer rows than tokens, else its tokens.
-__device__ __forceinline__ int combine_items(const PipelineArgs& a, int r, bool* by_rows) {
-  const int rows = a.row_start[r + 1] - a.row_start[r];
-  *by_rows = rows < a.T;
-  return rows < a.T ? rows : a.T;
+// The phase after the cursor's; false at the end of the list.
+__device__ __forceinline__ bool cursor_next(Cursor& c, const PipelineArgs& a) {
+  if (c.gu && c.r == a.r0) {          // G(r0) -> G(r0 + 1), or N(r0) with one round
+    if (c.r + 1 < a.R) ++c.r; else c.gu = false;
+  } else if (c.gu) {                  // G(r) -> N(r - 1)
+    c.gu = false;
+    --c.r;
+  } else if (c.r + 2 < a.R) {         // N(r) -> G(r + 2)
+    c.gu = true;
+    c.r += 2;
+  } else if (c.r + 1 < a.R) {         // N(r) -> N(r + 1) at the end of the list
+    ++c.r;
+  } else {
+    return false;
+  }
+  c.base = c.end;
+  cursor_load(c, a);
+  return true;
 }
 
-// Moves the cursor to the round holding `task`; false past the last round.
+// Moves the cursor to the phase holding `task`; false past the end of the list.
 __device__ __forceinline__ bool cursor_seek(Cursor& c, const PipelineArgs& a, int task) {
-  while (task >= c.end) {
-    c.base = c.end;
-    if (++c.r >= a.R) return false;
-    cursor_load(c, a);
-  }
+  while (task >= c.end)
+    if (!cursor_next(c, a)) return false;
   return true;
 }
 
@@ -189,18 +202,11 @@ struct Tile {
 };
 
 __device__ __forceinline__ void decode(const Cursor& c, const PipelineArgs& a, int task, Tile& t) {
-  int local = task - c.base;
+  const int local = task - c.base;
   t.r = c.r;
-  t.gu = local < c.gu_tiles;
-  int per;
-  if (t.gu) {
-    per = a.F / kPipeGuWidth;
-    t.kb = a.d / BK;
-  } else {
-    local -= c.gu_tiles;
-    per = a.d / kPipeDnWidth;
-    t.kb = a.F / BK;
-  }
+  t.gu = c.gu;
+  const int per = c.gu ? a.F / kPipeGuWidth : a.d / kPipeDnWidth;
+  t.kb = c.gu ? a.d / BK : a.F / BK;
   const int blk = local / per;
   t.nt = local - blk * per;
   const int32_t* pre = a.mb_prefix + static_cast<size_t>(c.r) * (a.E + 1);
@@ -300,33 +306,10 @@ __device__ void dispatch_role(const PipelineArgs& a, const Counters& cn) {
   }
 }
 
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
-  asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-// Bounded wait (one thread) until the token flag reaches `target`.
-__device__ bool wait_flag(const PipelineArgs& a, const unsigned long long* p, unsigned long long target) {
-  if (ld_acquire_u64(p) >= target) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t i = 1;; ++i) {
-    __nanosleep(32);
-    if (ld_acquire_u64(p) >= target) return true;
-    if ((i & 7) == 0 && ld_relaxed(a.sync + kSyncAbort) != 0) return false;
-    if (global_timer_ns() - t0 > MOE_WAIT_LIMIT_NS) {
-      give_up(a);
-      return false;
-    }
-  }
-}
-
-// Combine warps: y[t] (+)= gate * out[p][e][slot] for round r. A token waits only for the down
-// tiles of the blocks its own round-r rows live in, and for its own previous round's combine;
+// Combine warps: y[t] (+)= gate * out[p][e][slot] for round r. Each warp owns the tokens
+// t = gw + i * W and combines them round by round, so a token's y row is only ever touched by
+// one warp, each lane always on the same columns: the rounds are added in order by program
+// order alone. A token waits only for the down tiles of the blocks its round-r rows live in;
 // once its rows are read it counts them on their blocks, which the down GEMM two rounds later
 // waits for before it overwrites them.
 __device__ void combine_role(const PipelineArgs& a, const Counters& cn) {
@@ -334,6 +317,7 @@ __device__ void combine_role(const PipelineArgs& a, const Counters& cn) {
   const int cw = (threadIdx.x >> 5) - kFirstCombWarp;
   const int gw = blockIdx.x * kCombWarps + cw;
   const int W = gridDim.x * kCombWarps;
+  const long long span = 32ll * W;   // tokens per chunk (lane i holds the chunk's i-th token)
   int dn_cum[2] = {0, 0};
   for (int r = a.r0; r < a.R; ++r) {
     const int p = (r - a.r0) & 1;
@@ -342,28 +326,23 @@ __device__ void combine_role(const PipelineArgs& a, const Counters& cn) {
     dn_cum[p] += mblocks * kEpiWarps * (a.d / kPipeDnWidth);
     const int blk_target = (q + 1) * kEpiWarps * (a.d / kPipeDnWidth);
     const copy::CombineArgs comb{a.out[p], a.y, a.idx, a.gate, a.round, a.slot, a.T, a.k, a.C, a.d};
-    bool by_rows;
-    const int items = combine_items(a, r, &by_rows);
-    MOE_TRACE_DO(if (lane == 0 && gw < items) trace_min(trace_round(r, 2), global_timer_ns()));
     bool round_done = false;   // every down tile of round r seen finished
-    // this warp's items u = gw + i * W, 32 at a time: lane i fetches item i's token first
-    for (int base = gw; base < items; base += 32 * W) {
-      const int u_l = base + lane * W;
-      int t_l = u_l, only_l = -1;
-      if (by_rows && u_l < items) {
-        const int row = a.row_start[r] + u_l;
-        t_l = a.row_token[row];
-        only_l = a.row_dst[row] / a.C;
-      }
-      const int n_here = min(32, (items - base + W - 1) / W);
-      copy::PairLoads next = copy::load_pairs(comb, __shfl_sync(0xffffffffu, t_l, 0));
-      for (int i = 0; i < n_here; ++i) {
-        const int t = __shfl_sync(0xffffffffu, t_l, i);
-        const int only = __shfl_sync(0xffffffffu, only_l, i);
+    MOE_TRACE_DO(if (lane == 0) trace_min(trace_round(r, 2), global_timer_ns()));
+    for (long long c0 = gw; c0 < a.T; c0 += span) {
+      const long long tl = c0 + static_cast<long long>(lane) * W;
+      bool has = false;
+      if (tl < a.T)
+        for (int j = 0; j < a.k; ++j) has |= a.round[tl * a.k + j] == r;
+      uint32_t todo = __ballot_sync(0xffffffffu, has);
+      if (todo == 0u) continue;
+      copy::PairLoads next = copy::load_pairs(comb, static_cast<int>(c0 + static_cast<long long>(__ffs(todo) - 1) * W));
+      while (todo) {
+        const int i = __ffs(todo) - 1;
+        todo &= todo - 1;
+        const int t = static_cast<int>(c0 + static_cast<long long>(i) * W);
         const copy::PairLoads cur = next;
-        if (i + 1 < n_here) next = copy::load_pairs(comb, __shfl_sync(0xffffffffu, t_l, i + 1));
+        if (todo) next = copy::load_pairs(comb, static_cast<int>(c0 + static_cast<long long>(__ffs(todo) - 1) * W));
         const copy::TokenPairs tp = copy::token_pairs(comb, cur, r);
-        if (tp.npairs == 0 || (only >= 0 && tp.first_expert != only)) continue;
         const int blk = (tp.e * cn.mb + tp.s / BM) * kSyncStride;   // this lane's pair's block
         if (!round_done) {
           int ok = 1;
@@ -372,19 +351,12 @@ __device__ void combine_role(const PipelineArgs& a, const Counters& cn) {
           if (!round_done && lane < tp.npairs) ok = wait_counter(a, cn.dn[p] + blk, blk_target);
           if (!__all_sync(0xffffffffu, ok)) return;
         }
-        if (tp.prev_round >= a.r0) {   // y[t] holds the previous round's sum once its flag is set
-          int ok = 1;
-          if (lane == 0) ok = wait_flag(a, a.tok_flag + t, (a.gen << 32) | static_cast<unsigned>(tp.prev_round + 1));
-          if (!__shfl_sync(0xffffffffu, ok, 0)) return;
-        }
-        __syncwarp();
         copy::accumulate_token<16>(comb, t, tp);
         __syncwarp();
-        if (lane == 0) st_release_u64(a.tok_flag + t, (a.gen << 32) | static_cast<unsigned>(r + 1));
         if (lane < tp.npairs) red_release(cn.rd[p] + blk, 1);   // this pair's out row is read
       }
     }
-    MOE_TRACE_DO(if (lane == 0 && gw < items) trace_max(trace_round(r, 3), global_timer_ns()));
+    MOE_TRACE_DO(if (lane == 0) trace_max(trace_round(r, 3), global_timer_ns()));
   }
 }
 
@@ -682,7 +654,6 @@ extern "C" MOE_API int moe_trace_set(void* buffer) {
 
 cudaError_t launch_round_pipeline(const PipelineArgs& a, cudaStream_t stream) {
   if (a.r0 >= a.R) return cudaSuccess;
-  if (a.tok_flag == nullptr) return cudaErrorInvalidValue;
   for (int p = 0; p < 2; ++p)
     if (a.buf[p] == nullptr || a.h[p] == nullptr || a.out[p] == nullptr) return cudaErrorInvalidValue;
   CUtensorMap m_agu[2], m_bgu, m_adn[2], m_bdn;
@@ -716,13 +687,7 @@ cudaError_t launch_round_pipeline(const PipelineArgs& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   launch_begin(kKindPipeline, stream);
-  // token flags hold (generation << 32) | (round + 1): a flag left by an earlier launch on the
-  // same workspace is below every target of this one, so the flags are never cleared between
-  // launches (the planner zeroes them once per plan)
-  static std::atomic<unsigned long long> generation{0};
-  PipelineArgs args = a;
-  args.gen = generation.fetch_add(1) + 1;
-  e = cudaLaunchKernelEx(&cfg, round_pipeline_kernel, m_agu[0], m_agu[1], m_bgu, m_adn[0], m_adn[1], m_bdn, args);
+  e = cudaLaunchKernelEx(&cfg, round_pipeline_kernel, m_agu[0], m_agu[1], m_bgu, m_adn[0], m_adn[1], m_bdn, a);
   launch_end(kKindPipeline, stream);
   return e;
 }

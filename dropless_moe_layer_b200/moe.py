@@ -43,7 +43,7 @@ class WorkspaceLayout(ctypes.Structure):
     _fields_ = [(name, c_sz) for name in (
         "total_bytes", "header", "logits", "topk_idx", "gate", "round", "slot", "load",
         "offsets", "block_base", "n", "row_off", "row_start", "row_token", "row_dst", "buf", "h", "out",
-        "mb_prefix", "sync", "tok_flag", "buf2", "h2", "out2")
+        "mb_prefix", "sync", "buf2", "h2", "out2")
     ] + [("max_rounds", c_i32), ("plan_blocks", c_i32)]
 
 

@@ -131,7 +131,6 @@ typedef struct moe_workspace_layout {
   size_t mb_prefix;   /* i32 [max_rounds, E + 1]: 128-row blocks of experts < e in round r */
   size_t sync;        /* i32 [448 + 64 * E * ceil(C / 128)]: pipelined launch's dependency
                          counters (zero between calls) */
-  size_t tok_flag;    /* u64 [T]: pipelined launch's per-token combine progress */
   size_t buf2;        /* second buffer set of the pipelined launch (rounds alternate sets); */
   size_t h2;          /* absent (0) with MOE_FLAG_PER_ROUND, which never uses it */
   size_t out2;

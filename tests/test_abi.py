@@ -41,7 +41,7 @@ def _bytes_model(w, per_round=False):
     return (a(320 * 4) + a(T * E * 4) + 4 * a(T * k * 4) + a(E * 4) + a((E + 1) * 4)
             + a(blocks * E * 4) + 2 * a(mr * E * 4) + a((mr + 1) * 4) + 2 * a(T * k * 4)
             + a(E * C * d * 2) + a(E * C * F * 2) + a(E * C * d * 2)
-            + a(mr * (E + 1) * 4) + a((448 + 8 * E * ((C + 127) // 128) * 8) * 4) + a(T * 8)
+            + a(mr * (E + 1) * 4) + a((448 + 8 * E * ((C + 127) // 128) * 8) * 4)
             + (0 if per_round else a(E * C * d * 2) + a(E * C * F * 2) + a(E * C * d * 2)))
 
 
@@ -57,7 +57,7 @@ def test_workspace_is_fixed_by_shape(lib, w):
     offs = [lay.header, lay.logits, lay.topk_idx, lay.gate, lay.round, lay.slot, lay.load,
             lay.offsets, lay.block_base, lay.n, lay.row_off, lay.row_start, lay.row_token,
             lay.row_dst, lay.buf, lay.h, lay.out]
-    offs += [lay.mb_prefix, lay.sync, lay.tok_flag, lay.buf2, lay.h2, lay.out2]
+    offs += [lay.mb_prefix, lay.sync, lay.buf2, lay.h2, lay.out2]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     assert lay.max_rounds == (w.T + w.C - 1) // w.C
     s1 = moe.make_shape(w.T, w.d, w.E, w.k, w.F, w.C, schedule="per_round")
