@@ -185,6 +185,7 @@ struct PipelineArgs {
   int32_t* sync;
   int32_t* status;
   int T, k, E, C, d, F, r0, R;
+  int r0_dispatched;         // 1: round r0's rows are already in buf (set 0) when the launch starts
 };
 cudaError_t launch_round_pipeline(const PipelineArgs& a, cudaStream_t stream);
 

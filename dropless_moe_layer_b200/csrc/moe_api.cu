@@ -407,7 +407,8 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
   // Rounds [0, r0) run as per-round launches, [r0, R) in one pipelined launch.
   // A round is thin when even 128-column tiles of its gate/up GEMM would leave SMs idle: its
   // steps are latency-bound and gain from overlapping their neighbours. The pipelined launch
-  // takes the trailing run of thin rounds (its 32-column tiles suit thin rounds only).
+  // takes the trailing run of thin rounds (its 32-column tiles and its copy warps suit thin
+  // rounds only; a large round's copies get full-bandwidth kernels of their own).
   auto thin = [&](int rr) {
     long long blocks = 0;
     const long long base = static_cast<long long>(rr) * shape->C;
@@ -430,18 +431,20 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
   // depends only on the one before it (PDL wait), and no two steps of one launch touch the same
   // buffer: dispatch writes buf, gate/up reads buf and writes h, down reads h and writes out,
   // combine reads out and updates y. A run of thin rounds thus costs two launches per round.
-  if (r0 > 0 && (st = do_dispatch(shape, info, ws, L, 0, x, stream)) != MOE_OK) return st;
+  // The first pipelined round is dispatched here too (by the dispatch kernel, or on the last
+  // per-round down GEMM), so the pipelined launch starts with its rows in place.
+  if ((st = do_dispatch(shape, info, ws, L, 0, x, stream)) != MOE_OK) return st;
   for (int r = 0; r < r0; ++r) {
     const bool fuse_combine = r > 0 && small(r - 1);
     const RoundCopy comb = make_copy(shape, info, ws, L, true, r > 0 ? r - 1 : 0, x, y);
     if ((st = do_gate_up(shape, info, ws, L, r, w_gate_up, fuse_combine ? &comb : nullptr, stream)) != MOE_OK)
       return st;
-    const bool next = r + 1 < r0;
+    const bool next = r + 1 < R;
     const bool fuse_dispatch = next && small(r + 1);
     const RoundCopy disp = make_copy(shape, info, ws, L, false, next ? r + 1 : r, x, y);
     if ((st = do_down(shape, info, ws, L, r, w_down, fuse_dispatch ? &disp : nullptr, stream)) != MOE_OK) return st;
     if (next && !fuse_dispatch && (st = do_dispatch(shape, info, ws, L, r + 1, x, stream)) != MOE_OK) return st;
-    if (!(next && small(r)) && (st = do_combine(shape, info, ws, L, r, y, stream)) != MOE_OK) return st;
+    if (!(r + 1 < r0 && small(r)) && (st = do_combine(shape, info, ws, L, r, y, stream)) != MOE_OK) return st;
   }
   if (r0 < R) {
     PipelineArgs p{};
@@ -474,6 +477,7 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
     p.F = shape->d_ff;
     p.r0 = r0;
     p.R = R;
+    p.r0_dispatched = 1;
     if ((st = cuda_status(launch_round_pipeline(p, stream))) != MOE_OK) return st;
   }
   return MOE_OK;

@@ -250,7 +250,9 @@ __device__ bool wait_inputs(const PipelineArgs& a, const Counters& cn, const Cur
     const int full = min(BM, a.C - t.m * BM);
     const int nv = a.n[static_cast<size_t>(t.r) * a.E + t.e] - t.m * BM;
     const int rows = nv < 0 ? 0 : (nv > BM ? BM : nv);
-    if (!wait_counter(a, cn.disp[p] + blk, q * full + rows)) return false;
+    // round r0's rows were dispatched by an earlier kernel: set 0 counts them as present
+    const int pre = a.r0_dispatched && p == 0 ? full : 0;
+    if (!wait_counter(a, cn.disp[p] + blk, q * full + rows - pre)) return false;
     if (q > 0 && !wait_counter(a, cn.dn[p] + blk, q * kEpiWarps * (a.d / kPipeDnWidth))) return false;
   } else {
     if (!wait_counter(a, cn.gu[p] + blk, (q + 1) * kEpiWarps * (a.F / kPipeGuWidth))) return false;
@@ -266,7 +268,7 @@ __device__ void dispatch_role(const PipelineArgs& a, const Counters& cn) {
   const int gw = blockIdx.x * kDispWarps + dw;
   const int W = gridDim.x * kDispWarps;
   const int vecs = a.d / 8;
-  for (int r = a.r0; r < a.R; ++r) {
+  for (int r = a.r0 + (a.r0_dispatched ? 1 : 0); r < a.R; ++r) {
     const int p = (r - a.r0) & 1;
     const int q = (r - a.r0) >> 1;
     // block (e, m) of buf[p] is free once every gate/up tile of it in round r-2 has read it
