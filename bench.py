@@ -37,21 +37,20 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # DRAM traffic per launch of a kernel, from an ncu capture (dram__bytes_read.sum +
-# dram__bytes_write.sum, averaged over the launches of one layer step; summaries in profiles/),
-# valid only while the kernel's sources hash to the recorded value.
-TRAFFIC_SOURCES = ["sm100.cuh", "gemm_sm100.cuh", "copy_phases.cuh", "grouped_gemm.cu"]
+# dram__bytes_write.sum per launch; summaries in profiles/), valid only while the kernel's
+# sources hash to the recorded value.
 TRAFFIC = {
-    ("4k-zipf1", "gate_up"): {"bytes_per_launch": 20.22e6 + 0.50e6,
-                              "sources_sha1": "5a7f8bf5a51e3abde51578fcb03dedff101be348"},
-    ("4k-zipf1", "down"): {"bytes_per_launch": 9.12e6 + 0.02e6,
-                           "sources_sha1": "5a7f8bf5a51e3abde51578fcb03dedff101be348"},
+    ("4k-zipf1", "pipeline"): {
+        "bytes_per_launch": 67.483904e6 + 14.387712e6,
+        "sources": ["sm100.cuh", "gemm_sm100.cuh", "copy_phases.cuh", "kernels.h", "round_pipeline.cu"],
+        "sources_sha1": "7c1fb8cf357e09fc1cb1cfa0024d51a76baadd45"},
 }
 
 
-def sources_sha1():
+def sources_sha1(files):
     import hashlib
     h = hashlib.sha1()
-    for f in TRAFFIC_SOURCES:
+    for f in files:
         with open(os.path.join(ROOT, "dropless_moe_layer_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
@@ -59,7 +58,7 @@ def sources_sha1():
 
 def measured_traffic(workload, kernel):
     rec = TRAFFIC.get((workload, kernel))
-    if rec is None or rec["sources_sha1"] != sources_sha1():
+    if rec is None or rec["sources_sha1"] != sources_sha1(rec["sources"]):
         return None
     return rec["bytes_per_launch"]
 
