@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(32 * kCombineWarps)
   }
   sm100::grid_dependency_wait();      // buf comes from the round's down GEMM, y from earlier rounds
   sm100::pdl_trigger_early();
-  if (t < a.T) copy::combine_token(a, t, r, expert);
+  if (t < a.T) copy::combine_token<16>(a, t, r, expert);   // 16 columns per lane: more loads in flight
   sm100::pdl_trigger_late();
 }
 

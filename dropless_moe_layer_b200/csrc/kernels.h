@@ -45,6 +45,7 @@ enum : int {
   kHdrR = 0,
   kHdrMaxLoad = 1,
   kHdrStatus = 2,
+  kHdrScanDone = 3,   // planner: expert scans finished (the last one finalizes the plan)
   kHdrLoad = 64,      // copy of load[0..E-1], so one small copy brings the plan summary home
   kHdrWords = 64 + 256,
 };
@@ -94,8 +95,10 @@ void launch_end(int kind, cudaStream_t stream, int kernels = 1);
 int num_sms();
 
 // ---- router / top-k (router.cu)
+// block_counts: [ceil(T / 256), E] pair counts per block of 256 tokens and expert, added with
+// atomics (the caller zeroes it first); the planner's first input.
 cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int renorm, int32_t* idx,
-                               float* gate, cudaStream_t stream);
+                               float* gate, int32_t* block_counts, cudaStream_t stream);
 
 // ---- planner (plan.cu)
 struct PlanBuffers {
@@ -103,7 +106,7 @@ struct PlanBuffers {
   int32_t* header;        // [kHdrWords]
   int32_t* load;          // [E]
   int32_t* offsets;       // [E + 1]
-  int32_t* block_base;    // [blocks, E]
+  int32_t* block_base;    // [blocks, E]: per-block pair counts from the top-k kernel
   int32_t* n;             // [max_rounds, E]
   int32_t* row_off;       // [max_rounds, E]
   int32_t* row_start;     // [max_rounds + 1]

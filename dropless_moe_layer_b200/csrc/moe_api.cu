@@ -104,6 +104,7 @@ void make_layout(const moe_shape_t* s, moe_workspace_layout_t* L) {
   const int mr = max_rounds_of(s);
   const int blocks = static_cast<int>((T + kPlanTokensPerBlock - 1) / kPlanTokensPerBlock);
   L->header = take(kHdrWords * 4ll);
+  L->block_base = take(static_cast<long long>(blocks) * E * 4);   // right after the header: one memset
   L->logits = take(T * E * 4);
   L->topk_idx = take(T * k * 4);
   L->gate = take(T * k * 4);
@@ -111,7 +112,6 @@ void make_layout(const moe_shape_t* s, moe_workspace_layout_t* L) {
   L->slot = take(T * k * 4);
   L->load = take(E * 4);
   L->offsets = take((E + 1) * 4);
-  L->block_base = take(static_cast<long long>(blocks) * E * 4);
   L->n = take(static_cast<long long>(mr) * E * 4);
   L->row_off = take(static_cast<long long>(mr) * E * 4);
   L->row_start = take((mr + 1ll) * 4);
@@ -295,7 +295,10 @@ int moe_plan(const moe_shape_t* shape, const float* logits, const uint16_t* x,
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   const moe_shape_t& s = *shape;
   int32_t* header = at<int32_t>(ws, L.header);
-  if (cudaMemsetAsync(header, 0, kHdrWords * 4, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  // the header and the per-block pair counts start at zero (one memset: they are adjacent)
+  if (cudaMemsetAsync(header, 0, L.block_base - L.header + static_cast<size_t>(L.plan_blocks) * s.E * 4, stream) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
 
   const float* z = logits;
   if (z == nullptr && s.T > 0) {
@@ -306,7 +309,7 @@ int moe_plan(const moe_shape_t* shape, const float* logits, const uint16_t* x,
   }
   if ((st = cuda_status(launch_router_topk(z, s.T, s.E, s.k, (s.flags & MOE_FLAG_RENORM_TOPK) ? 1 : 0,
                                            at<int32_t>(ws, L.topk_idx), at<float>(ws, L.gate),
-                                           stream))) != MOE_OK)
+                                           at<int32_t>(ws, L.block_base), stream))) != MOE_OK)
     return st;
   PlanBuffers pb;
   pb.idx = at<int32_t>(ws, L.topk_idx);

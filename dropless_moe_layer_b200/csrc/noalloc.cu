@@ -74,9 +74,9 @@ extern "C" MOE_API int moe_plan_noalloc(const moe_shape_t* shape, const float* l
     return o;
   };
   const size_t o_header = take(moe::kHdrWords * 4ll);
+  const size_t o_block = take(static_cast<long long>(blocks) * E * 4);   // adjacent: one memset
   const size_t o_load = take(E * 4);
   const size_t o_offsets = take((E + 1) * 4);
-  const size_t o_block = take(static_cast<long long>(blocks) * E * 4);
   const size_t o_n = take(static_cast<long long>(max_rounds) * E * 4);
   const size_t o_row_off = take(static_cast<long long>(max_rounds) * E * 4);
   const size_t o_row_start = take((max_rounds + 1ll) * 4);
@@ -96,9 +96,10 @@ extern "C" MOE_API int moe_plan_noalloc(const moe_shape_t* shape, const float* l
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
 
   int32_t* header = reinterpret_cast<int32_t*>(scratch + o_header);
-  if (cudaMemsetAsync(header, 0, moe::kHdrWords * 4, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(header, 0, o_block - o_header + static_cast<size_t>(blocks) * E * 4, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
   if (moe::launch_router_topk(logits, s.T, s.E, s.k, (s.flags & MOE_FLAG_RENORM_TOPK) ? 1 : 0, topk_idx,
-                              gate, stream) != cudaSuccess)
+                              gate, reinterpret_cast<int32_t*>(scratch + o_block), stream) != cudaSuccess)
     return MOE_ERR_CUDA;
   moe::PlanBuffers pb;
   pb.idx = topk_idx;

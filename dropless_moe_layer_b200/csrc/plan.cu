@@ -10,13 +10,13 @@
 //   rank(t, j) = #{t' < t : expert idx[t, j] is among t's choices}
 //   round = rank / C, slot = rank % C, R = ceil(max_e load_e / C)
 //
-// Four small kernels, all integer (bit-exact, deterministic):
-//   1. plan_count:    per block of 256 tokens, per-expert pair counts.
-//   2. plan_scan:     one CTA per expert: exclusive scan of the block counts over
-//                     blocks (the block's base rank) and the expert's load.
-//   3. plan_finalize: one CTA: expert offsets, max load, R, n[r][e], the round-major
-//                     row positions row_off[r][e] and row_start[r].
-//   4. plan_rank:     per block of 256 tokens: the stable rank of each pair inside its
+// Integer work only (bit-exact, deterministic), after the top-k kernel has counted the pairs
+// of every block of 256 tokens per expert (router.cu):
+//   1. plan_scan:     one CTA per expert: exclusive scan of the block counts over
+//                     blocks (the block's base rank) and the expert's load; the last CTA
+//                     to finish then computes the expert offsets, max load, R, n[r][e],
+//                     the round-major row positions row_off[r][e] and row_start[r].
+//   2. plan_rank:     per block of 256 tokens: the stable rank of each pair inside its
 //                     block from per-warp lane bitmasks (popcount of lower lanes and
 //                     lower warps), plus the block base; writes round, slot and the
 //                     pair's row in the round-major list (source token, destination
@@ -30,23 +30,6 @@ namespace {
 
 constexpr int kTPB = kPlanTokensPerBlock;   // tokens per block = threads per block
 constexpr int kWarps = kTPB / 32;
-
-__global__ void __launch_bounds__(kTPB) plan_count_kernel(const int32_t* __restrict__ idx, int T,
-                                                          int k, int E,
-                                                          int32_t* __restrict__ block_base) {
-  __shared__ int cnt[MOE_MAX_E_PLAN];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
-  sm100::grid_dependency_wait();
-  sm100::grid_launch_dependents();
-  __syncthreads();
-  const int t = blockIdx.x * kTPB + threadIdx.x;
-  if (t < T) {
-    for (int j = 0; j < k; ++j) atomicAdd(&cnt[idx[static_cast<size_t>(t) * k + j]], 1);
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x)
-    block_base[static_cast<size_t>(blockIdx.x) * E + e] = cnt[e];
-}
 
 // Block-wide inclusive scan of one int per thread (blockDim.x == 256).
 __device__ int block_inclusive_scan(int v, int* warp_sums) {
@@ -73,12 +56,26 @@ __device__ int block_inclusive_scan(int v, int* warp_sums) {
   return v;
 }
 
-// One CTA per expert e: block_base[b][e] <- sum_{b' < b} count[b'][e]; load[e] <- total.
+__device__ void finalize_plan(const int32_t* __restrict__ load, int E, int C, int max_rounds,
+                              int32_t* __restrict__ offsets, int32_t* __restrict__ header,
+                              int32_t* __restrict__ n, int32_t* __restrict__ row_off,
+                              int32_t* __restrict__ row_start, int32_t* __restrict__ mb_prefix,
+                              int* warp_sums);
+
+// One CTA per expert e: block_base[b][e] <- sum_{b' < b} count[b'][e]; load[e] <- total. The
+// last CTA to finish (a counter in the header) then finalizes the plan.
 __global__ void __launch_bounds__(kTPB) plan_scan_kernel(int32_t* __restrict__ block_base,
-                                                         int blocks, int E,
-                                                         int32_t* __restrict__ load) {
+                                                         int blocks, int E, int C, int max_rounds,
+                                                         int32_t* __restrict__ load,
+                                                         int32_t* __restrict__ offsets,
+                                                         int32_t* __restrict__ header,
+                                                         int32_t* __restrict__ n,
+                                                         int32_t* __restrict__ row_off,
+                                                         int32_t* __restrict__ row_start,
+                                                         int32_t* __restrict__ mb_prefix) {
   __shared__ int warp_sums[kWarps];
   __shared__ int chunk_total;
+  __shared__ int is_last;
   const int e = blockIdx.x;
   int carry = 0;
   sm100::grid_dependency_wait();
@@ -93,25 +90,28 @@ __global__ void __launch_bounds__(kTPB) plan_scan_kernel(int32_t* __restrict__ b
     carry += chunk_total;
     __syncthreads();
   }
-  if (threadIdx.x == 0) load[e] = carry;
+  if (threadIdx.x == 0) {
+    load[e] = carry;
+    __threadfence();   // load[e] is visible before this CTA counts itself done
+    is_last = atomicAdd(header + kHdrScanDone, 1) == E - 1;
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  finalize_plan(load, E, C, max_rounds, offsets, header, n, row_off, row_start, mb_prefix, warp_sums);
 }
 
-// One CTA: offsets, max load, R, n[r][e], row_off[r][e], row_start[r].
-__global__ void __launch_bounds__(kTPB) plan_finalize_kernel(const int32_t* __restrict__ load, int E,
-                                                             int C, int max_rounds,
-                                                             int32_t* __restrict__ offsets,
-                                                             int32_t* __restrict__ header,
-                                                             int32_t* __restrict__ n,
-                                                             int32_t* __restrict__ row_off,
-                                                             int32_t* __restrict__ row_start,
-                                                             int32_t* __restrict__ mb_prefix) {
-  __shared__ int warp_sums[kWarps];
+// One CTA (the last expert scan to finish): offsets, max load, R, n[r][e], row_off[r][e],
+// row_start[r], and the per-round 128-row block prefix.
+__device__ void finalize_plan(const int32_t* __restrict__ load, int E, int C, int max_rounds,
+                              int32_t* __restrict__ offsets, int32_t* __restrict__ header,
+                              int32_t* __restrict__ n, int32_t* __restrict__ row_off,
+                              int32_t* __restrict__ row_start, int32_t* __restrict__ mb_prefix,
+                              int* warp_sums) {
   __shared__ int s_load[MOE_MAX_E_PLAN];
   __shared__ int s_max;
   const int e = threadIdx.x;
-  sm100::grid_dependency_wait();
-  sm100::grid_launch_dependents();
-  const int le = e < E ? load[e] : 0;
+  const int le = e < E ? __ldcg(load + e) : 0;   // written by the other CTAs of this grid
   if (e < MOE_MAX_E_PLAN) s_load[e] = le;
   if (threadIdx.x == 0) s_max = 0;
   const int inc = block_inclusive_scan(le, warp_sums);
@@ -219,19 +219,14 @@ cudaError_t launch_plan(const PlanBuffers& b, int T, int k, int E, int C, int ma
                         cudaStream_t stream) {
   const int blocks = (T + kTPB - 1) / kTPB;
   launch_begin(kKindPlan, stream);
-  cudaError_t err = cudaSuccess;
-  if (blocks > 0 && err == cudaSuccess)
-    err = launch_pdl(plan_count_kernel, dim3(blocks), dim3(kTPB), 0, stream, b.idx, T, k, E, b.block_base);
-  if (err == cudaSuccess)
-    err = launch_pdl(plan_scan_kernel, dim3(E), dim3(kTPB), 0, stream, b.block_base, blocks, E, b.load);
-  if (err == cudaSuccess)
-    err = launch_pdl(plan_finalize_kernel, dim3(1), dim3(kTPB), 0, stream, b.load, E, C, max_rounds,
-                     b.offsets, b.header, b.n, b.row_off, b.row_start, b.mb_prefix);
+  cudaError_t err = launch_pdl(plan_scan_kernel, dim3(E), dim3(kTPB), 0, stream, b.block_base, blocks, E, C,
+                               max_rounds, b.load, b.offsets, b.header, b.n, b.row_off, b.row_start,
+                               b.mb_prefix);
   if (blocks > 0 && err == cudaSuccess)
     err = launch_pdl(plan_rank_kernel, dim3(blocks), dim3(kTPB), 0, stream, b.idx, T, k, E, C,
                      b.block_base, b.row_off, b.round, b.slot, b.row_token, b.row_dst, b.sync,
                      b.sync_words);
-  launch_end(kKindPlan, stream, blocks > 0 ? 4 : 2);
+  launch_end(kKindPlan, stream, blocks > 0 ? 2 : 1);
   return err;
 }
 

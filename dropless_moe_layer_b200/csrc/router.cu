@@ -10,7 +10,8 @@
 // Each lane holds up to 8 logits (E <= 256) in registers. The softmax max and sum are
 // warp butterfly reductions (fixed order, so deterministic). Top-k is k rounds of a
 // warp arg-max under the total order (logit desc, index asc); the winner is marked
-// taken in its owner lane.
+// taken in its owner lane. The kernel also counts, for the planner, the pairs of every block
+// of 256 tokens per expert.
 #include <cfloat>
 #include <climits>
 
@@ -23,7 +24,8 @@ template <int VPL>
 __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits, int T,
                                                           int E, int k, int renorm,
                                                           int32_t* __restrict__ idx_out,
-                                                          float* __restrict__ gate_out) {
+                                                          float* __restrict__ gate_out,
+                                                          int32_t* __restrict__ block_counts) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   sm100::grid_dependency_wait();
@@ -87,11 +89,13 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     if (renorm) my_gate = my_gate / gsum;
     idx_out[static_cast<size_t>(t) * k + lane] = my_idx;
     gate_out[static_cast<size_t>(t) * k + lane] = my_gate;
+    // the planner's per-block counts (integer adds: the order does not matter)
+    atomicAdd(block_counts + static_cast<size_t>(t / kPlanTokensPerBlock) * E + my_idx, 1);
   }
 }
 
 cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int renorm, int32_t* idx,
-                               float* gate, cudaStream_t stream) {
+                               float* gate, int32_t* block_counts, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   const int warps_per_block = 8;
   const dim3 grid((T + warps_per_block - 1) / warps_per_block), block(32 * warps_per_block);
@@ -99,7 +103,8 @@ cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int ren
   const int vpl = (E + 31) / 32;
   auto kern = vpl <= 1 ? router_topk_kernel<1> : vpl <= 2 ? router_topk_kernel<2>
             : vpl <= 4 ? router_topk_kernel<4> : router_topk_kernel<8>;
-  const cudaError_t err = launch_pdl(kern, grid, block, 0, stream, logits, T, E, k, renorm, idx, gate);
+  const cudaError_t err = launch_pdl(kern, grid, block, 0, stream, logits, T, E, k, renorm, idx, gate,
+                                     block_counts);
   launch_end(kKindTopk, stream);
   return err;
 }

@@ -54,8 +54,8 @@ def test_workspace_is_fixed_by_shape(lib, w):
     assert n >= w.E * w.C * (2 * w.d + w.F) * 2
     lay = moe.workspace_layout(s)
     assert lay.total_bytes == n
-    offs = [lay.header, lay.logits, lay.topk_idx, lay.gate, lay.round, lay.slot, lay.load,
-            lay.offsets, lay.block_base, lay.n, lay.row_off, lay.row_start, lay.row_token,
+    offs = [lay.header, lay.block_base, lay.logits, lay.topk_idx, lay.gate, lay.round, lay.slot, lay.load,
+            lay.offsets, lay.n, lay.row_off, lay.row_start, lay.row_token,
             lay.row_dst, lay.buf, lay.h, lay.out]
     offs += [lay.mb_prefix, lay.sync, lay.buf2, lay.h2, lay.out2]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
