@@ -35,8 +35,11 @@ Readings where the pages are silent (each listed in the design notes):
   * selection order and ties: by logit descending, equal logits (+0 == -0) broken
     by the lower expert index.
   * which pairs go first: in ascending token order within each expert.
-  * no capacity borrowing between experts: each expert owns C rows per round, so
-    the round count is R = ceil(max_e load_e / C).
+  * by default no capacity borrowing between experts: each expert owns C rows per
+    round, so the round count is R = ceil(max_e load_e / C). `plan_borrow` states the
+    pages' fuller rule (an overloaded expert takes capacity other experts leave unused,
+    else an extra round); the order in which spare rows are handed out is not given,
+    and the reading taken is "ascending expert index".
   * expert FFN: SwiGLU without biases, f(x) = W2 (silu(W1 x) * (W3 x)).
 """
 from __future__ import annotations
@@ -143,6 +146,68 @@ def plan(idx, E: int, C: int) -> dict:
                 max_load=max_load, n=n, offsets=offsets, C=C)
 
 
+def plan_borrow(idx, E: int, C: int) -> dict:
+    """Round plan with capacity borrowing.
+
+    "Frontier Pre-training at Microsoft AI (MAI-Base-2)", Key claims, multi-round dropless
+    MoE item: overflow tokens use unused capacity of other experts of the same group, and
+    only otherwise go to an extra round; "MAI-Base-2: Microsoft details its new training
+    infrastructure", section "Optimizations to prevent memory loss": the system can reuse
+    capacity other experts leave unallocated. A round holds at most E*C rows (the fixed
+    buffer). Reading where the pages are silent: in each round every expert first takes up
+    to C of its pending pairs; the rows left unused by that are handed to experts that still
+    have pending pairs, in ascending expert index, each taking what it has pending or what is
+    left. An expert's pairs still go in ascending token order: its pairs with ranks
+    [start[r, e], start[r, e] + n[r, e]) form its rows of round r, at slots 0 .. n[r, e]-1.
+    Written as the plain loop over rounds.
+    """
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    if C < 1:
+        raise ValueError("capacity C must be >= 1")
+    count = [0] * E
+    rank = np.empty((T, k), dtype=np.int64)
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            rank[t, j] = count[e]
+            count[e] += 1
+    load = np.array(count, dtype=np.int64)
+    pending = load.copy()
+    rounds = []
+    while pending.sum() > 0:
+        own = np.minimum(pending, C)                 # each expert's own C rows first
+        spare = E * C - int(own.sum())               # rows nobody took that way
+        extra = np.zeros(E, dtype=np.int64)
+        for e in range(E):                           # lent in ascending expert order
+            want = int(pending[e] - own[e])
+            take = min(want, spare)
+            extra[e] = take
+            spare -= take
+        n_r = own + extra
+        rounds.append(n_r)
+        pending = pending - n_r
+    R = len(rounds)
+    n = np.array(rounds, dtype=np.int64).reshape(R, E)
+    start = np.zeros((R + 1, E), dtype=np.int64)     # start[r, e]: pairs of e in rounds < r
+    for r in range(R):
+        start[r + 1] = start[r] + n[r]
+    rnd = np.empty((T, k), dtype=np.int64)
+    slot = np.empty((T, k), dtype=np.int64)
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            r = 0
+            while rank[t, j] >= start[r + 1, e]:
+                r += 1
+            rnd[t, j] = r
+            slot[t, j] = rank[t, j] - start[r, e]
+    max_load = int(load.max()) if E > 0 else 0
+    offsets = np.concatenate([[0], np.cumsum(load)]).astype(np.int64)
+    return dict(rank=rank, round=rnd, slot=slot, load=load, R=R, max_load=max_load, n=n,
+                offsets=offsets, C=C)
+
+
 def round_rows(p: dict, idx, r: int) -> list:
     """The rows of round r as (expert, slot, token, j) tuples, ordered by expert then
     slot: the contents of the round's fixed [E, C, d] dispatch buffer."""
@@ -208,33 +273,39 @@ def forward(x_bits, w_gate_up_bits, w_down_bits, idx, gate, tokens=None) -> np.n
     return y
 
 
-def forward_rounds(x_bits, w_gate_up_bits, w_down_bits, idx, gate, C: int) -> tuple:
+def forward_rounds(x_bits, w_gate_up_bits, w_down_bits, idx, gate, C: int,
+                   borrow: bool = False) -> tuple:
     """Literal multi-round executor (tiny inputs only).
 
-    For r = 0 .. R-1: dispatch copies the round's pairs into a fixed [E, C, d] buffer
-    at (expert, slot); compute runs each expert's FFN on its first n[r, e] rows;
-    collect writes gate * output back to the pair. The buffer never grows with the
-    routing. Returns (y, plan, max rows any round held for one expert)."""
+    For r = 0 .. R-1: dispatch copies the round's pairs into a fixed buffer of E*C rows;
+    compute runs each expert's FFN on its n[r, e] rows; collect writes gate * output back
+    to the pair. Without borrowing the buffer is [E, C, d] (expert e's rows at e*C + slot);
+    with borrowing (`plan_borrow`) an expert may hold more than C rows of a round, so the
+    round's rows are packed expert after expert (expert e's rows at
+    sum_{e' < e} n[r, e'] + slot). Either way the buffer never grows with the routing.
+    Returns (y, plan, max rows any round held for one expert)."""
     idx = np.asarray(idx)
     gate = np.asarray(gate, dtype=np.float64)
     T, k = idx.shape
     E = w_gate_up_bits.shape[0]
     d = w_down_bits.shape[1]
-    p = plan(idx, E, C)
+    p = plan_borrow(idx, E, C) if borrow else plan(idx, E, C)
     x = bf16_to_f64(x_bits)
-    buf = np.zeros((E, C, d), dtype=np.float64)
+    buf = np.zeros((E * C, d), dtype=np.float64)
     terms = np.zeros((T, k, d), dtype=np.float64)
     peak = 0
     for r in range(p["R"]):
+        n_r = [int(v) for v in p["n"][r]]
+        base = [e * C for e in range(E)] if not borrow else [sum(n_r[:e]) for e in range(E)]
         rows = round_rows(p, idx, r)
         for (e, s, t, j) in rows:                      # dispatch
-            buf[e, s, :] = x[t]
+            buf[base[e] + s, :] = x[t]
         outs = {}
         for e in range(E):                             # compute
-            n = int(p["n"][r, e])
+            n = n_r[e]
             peak = max(peak, n)
             if n:
-                outs[e] = expert_ffn(buf[e, :n], bf16_to_f64(w_gate_up_bits[e]),
+                outs[e] = expert_ffn(buf[base[e]:base[e] + n], bf16_to_f64(w_gate_up_bits[e]),
                                      bf16_to_f64(w_down_bits[e]))
         for (e, s, t, j) in rows:                      # collect
             terms[t, j, :] = gate[t, j] * outs[e][s]

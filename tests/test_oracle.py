@@ -195,6 +195,117 @@ def test_plan_special_cases():
     assert empty["R"] == 0 and empty["load"].sum() == 0
 
 
+# ----------------------------------------------------------------------------- capacity borrowing
+
+def test_plan_borrow_worked_example():
+    g = _read_golden("plan_borrow_worked_example.txt")
+    T, E, k, C = (int(g[key][0]) for key in ("T", "E", "k", "C"))
+    z = np.array([float(v) for v in g["logits"]], dtype=np.float32).reshape(T, E)
+    idx = oracle.select_topk(z, k)
+    np.testing.assert_array_equal(idx, np.array(g["idx"], int).reshape(T, k))
+    p = oracle.plan_borrow(idx, E, C)
+    np.testing.assert_array_equal(p["round"], np.array(g["round"], int).reshape(T, k))
+    np.testing.assert_array_equal(p["slot"], np.array(g["slot"], int).reshape(T, k))
+    np.testing.assert_array_equal(p["load"], np.array(g["load"], int))
+    assert p["R"] == int(g["R"][0])
+    np.testing.assert_array_equal(p["n"], np.array(g["n"], int).reshape(p["R"], E))
+    for r in range(p["R"]):
+        want = []
+        for item in g[f"round{r}"]:
+            es, t = item.split("=")
+            e, s = es.split(":")
+            want.append((int(e), int(s), int(t)))
+        got = [(e, s, t) for (e, s, t, j) in oracle.round_rows(p, idx, r)]
+        assert got == sorted(want)
+
+
+def _check_borrow_invariants(idx, p, E, C):
+    """What the borrowing rule fixes, whatever order spare rows are lent in."""
+    T, k = idx.shape
+    load = p["load"]
+    assert load.sum() == T * k
+    np.testing.assert_array_equal(p["n"].sum(0), load)                  # every pair once
+    assert np.all(p["n"].sum(1) <= E * C)                                # fixed round buffer
+    pending = load.copy()
+    for r in range(p["R"]):
+        n_r = p["n"][r]
+        assert np.all(n_r >= np.minimum(pending, C))                      # own capacity first
+        if n_r.sum() < E * C:                                            # spare left over:
+            assert np.array_equal(n_r, pending)                           # nothing was waiting
+        pending = pending - n_r
+    assert not pending.any()
+    total = T * k
+    assert p["R"] >= math.ceil(total / (E * C))                           # pool bound
+    assert p["R"] <= math.ceil(load.max() / C) if total else p["R"] == 0  # never worse
+    for e in range(E):                                                    # stable token order
+        ts, js = np.nonzero(idx == e)
+        start = np.concatenate([[0], np.cumsum(p["n"][:, e])])
+        rk = start[p["round"][ts, js]] + p["slot"][ts, js]
+        np.testing.assert_array_equal(rk, np.arange(ts.size))
+
+
+@pytest.mark.parametrize("name", ["tiny-zipf1", "4k-zipf1"])
+def test_plan_borrow_invariants_on_workloads(name):
+    w = wl.BY_NAME[name]
+    z = wl.generate(w, "cpu", routing_only=True)["logits"].numpy()
+    idx = oracle.select_topk(z, w.k)
+    p = oracle.plan_borrow(idx, w.E, w.C)
+    _check_borrow_invariants(idx, p, w.E, w.C)
+    assert p["R"] < oracle.plan(idx, w.E, w.C)["R"]                      # skewed: fewer rounds
+
+
+def test_plan_borrow_special_cases():
+    rng = np.random.default_rng(5)
+    z = rng.standard_normal((300, 7)).astype(np.float32)
+    idx = oracle.select_topk(z, 3)
+    # one round exactly when all pairs fit the pool: R = 1 iff T*k <= E*C
+    for C in (128, 129, 130, 200):
+        p = oracle.plan_borrow(idx, 7, C)
+        _check_borrow_invariants(idx, p, 7, C)
+        assert (p["R"] == 1) == (900 <= 7 * C)
+    # nobody over capacity: borrowing changes nothing
+    base = oracle.plan(idx, 7, C=10_000)
+    bor = oracle.plan_borrow(idx, 7, C=10_000)
+    for key in ("round", "slot", "n"):
+        np.testing.assert_array_equal(base[key], bor[key])
+    # a single expert has nobody to borrow from
+    one = np.zeros((50, 1), np.int64)
+    for key in ("round", "slot", "n"):
+        np.testing.assert_array_equal(oracle.plan(one, 1, 7)[key], oracle.plan_borrow(one, 1, 7)[key])
+    # every pair on one expert of eight: the whole pool each round
+    hot = np.zeros((100, 1), np.int64)
+    p = oracle.plan_borrow(hot, 8, 4)
+    assert p["R"] == math.ceil(100 / 32) and list(p["n"][:, 0]) == [32, 32, 32, 4]
+    empty = oracle.plan_borrow(np.zeros((0, 2), np.int64), 5, 3)
+    assert empty["R"] == 0
+    # two overloaded experts, two spare rows: the lower expert index takes them (the reading)
+    two = np.array([[0]] * 4 + [[1]] * 4, np.int64)
+    p = oracle.plan_borrow(two, 3, 2)
+    np.testing.assert_array_equal(p["n"], [[4, 2, 0], [0, 2, 0]])
+    np.testing.assert_array_equal(p["round"][:, 0], [0, 0, 0, 0, 0, 0, 1, 1])
+    np.testing.assert_array_equal(p["slot"][:, 0], [0, 1, 2, 3, 0, 1, 0, 1])
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_borrowing_rounds_do_not_change_the_output(seed):
+    """The pooled round executor with borrowing gives the capacity-free output."""
+    rng = np.random.default_rng(40 + seed)
+    T, E, k, d, F = 24, 5, 2, 8, 16
+    z = rng.standard_normal((T, E)).astype(np.float32)
+    z[:, 0] += 3.0                                                        # one hot expert
+    x = _rand_bf16_bits(rng, (T, d))
+    w13 = _rand_bf16_bits(rng, (E, 2 * F, d), 0.3)
+    w2 = _rand_bf16_bits(rng, (E, d, F), 0.3)
+    idx = oracle.select_topk(z, k)
+    g = oracle.gates(z, idx)
+    y_free = oracle.forward(x, w13, w2, idx, g)
+    for C in (1, 2, 3, 5, 24):
+        y, p, peak = oracle.forward_rounds(x, w13, w2, idx, g, C, borrow=True)
+        assert p["R"] <= oracle.plan(idx, E, C)["R"]
+        assert peak <= E * C
+        np.testing.assert_allclose(y, y_free, rtol=1e-12, atol=1e-14)
+
+
 # ----------------------------------------------------------------------------- expert math
 
 def _torch_swiglu(x, w1, w3, w2):
