@@ -224,9 +224,12 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- algorithmic work
 
-def round_rows(w, info):
-    """n[r][e]: rows of expert e in round r, from the plan's loads."""
+def round_rows(w, info, n_plan=None):
+    """n[r][e]: rows of expert e in round r (the device plan's when given, else from the loads
+    by the no-borrowing rule)."""
     import numpy as np
+    if n_plan is not None:
+        return np.asarray(n_plan, dtype=np.int64)
     load = np.array(info.load[:w.E], dtype=np.int64)
     return np.clip(load[None, :] - w.C * np.arange(info.R)[:, None], 0, w.C)
 
@@ -247,14 +250,14 @@ def combine_bytes(w, round_np, rounds=None):
     return total
 
 
-def algorithmic_work(w, info, r0, round_np):
+def algorithmic_work(w, info, r0, round_np, n_plan=None):
     """Per kernel kind, the algorithmic units of one step, from the plan alone (padding rows
     C - n never count). Per-round kernels cover rounds [0, r0), the pipelined launch [r0, R).
     GEMMs: flops (tensor-bound). Copies: bytes (HBM-bound). The pipelined launch runs all four
     steps of its rounds; its bound is the larger of its tensor time (6 n d F flops per
     (round, expert)) and its HBM time (the weights, 6 d F bytes per active (round, expert),
     plus its copies' and its GEMM operands' bytes), each at the measured peak."""
-    n = round_rows(w, info)
+    n = round_rows(w, info, n_plan)
     per = n[:r0].sum()
     pipe = n[r0:]
     prow = int(pipe.sum())
@@ -308,6 +311,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--schedule", default="auto", choices=["auto", "per_round", "pipeline"],
                     help="moe_forward launch schedule (the layer's results are identical)")
+    ap.add_argument("--borrow", action="store_true",
+                    help="capacity borrowing between experts (fewer rounds; not the default plan)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = wl.BY_NAME[args.workload]
@@ -336,7 +341,8 @@ def main():
 
     moe.load_library()
     inp = wl.generate(w, dev)
-    layer = moe.DroplessMoE(w.T, w.d, w.E, w.k, w.F, w.C, device=dev, schedule=args.schedule)
+    layer = moe.DroplessMoE(w.T, w.d, w.E, w.k, w.F, w.C, device=dev, schedule=args.schedule,
+                            borrow=args.borrow)
     y = torch.empty(w.T, w.d, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -407,7 +413,7 @@ def main():
     r0 = kinds["gate_up"][0] // args.steps if "gate_up" in kinds else 0
     if "pipeline" not in kinds:
         r0 = info.R
-    work = algorithmic_work(w, info, r0, rnd)
+    work = algorithmic_work(w, info, r0, rnd, layer.plan_tensors()["n"].cpu().numpy())
 
     def resolve(kind):
         """(bound, units per step) of a kind; a mixed launch takes its slower roofline."""
@@ -481,7 +487,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": dict(workload_config(w), schedule=args.schedule),
+            "config": dict(workload_config(w), schedule=args.schedule, capacity_borrowing=args.borrow),
             "rounds": info.R, "pipelined_rounds": [r0, info.R], "routed_pairs_per_s": value * w.k,
             "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                          "frac": achieved / peak, "peak_source": f"{peak_src} ({'bf16_tflops burst' if bound == 'tensor' else 'hbm_gbs copy'})",

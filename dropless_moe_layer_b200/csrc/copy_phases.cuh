@@ -69,6 +69,11 @@ struct CombineArgs {
   const int32_t* round;
   const int32_t* slot;
   int T, k, C, d;
+  // Pooled round rows (capacity borrowing): the pair (e, slot) of round r is row
+  // row_off[r][e] - row_start[r] + slot of buf. Null: row e * C + slot.
+  const int32_t* row_off;
+  const int32_t* row_start;
+  int E;
 };
 
 // One token's pairs in one round, spread over the warp (every lane holds the same scalars;
@@ -77,7 +82,7 @@ struct TokenPairs {
   int npairs;               // pairs of the token in round r (0: nothing to do)
   bool fresh;               // r is the token's first round: y starts from zero
   int prev_round;           // the token's latest round before r, or -1
-  int first_expert;         // expert of the token's first pair in round r
+  unsigned long long first_row;   // buffer row of the token's first pair in round r
   int e, s;                 // this lane's pair (expert, slot), lane < npairs
   unsigned long long prow;  // e * C + s
   float pgate;
@@ -111,14 +116,18 @@ __device__ __forceinline__ TokenPairs token_pairs(const CombineArgs& a, const Pa
   TokenPairs tp;
   const uint32_t here = __ballot_sync(0xffffffffu, my_round == r);
   tp.npairs = __popc(here);
-  tp.first_expert = __shfl_sync(0xffffffffu, my_idx, here ? __ffs(here) - 1 : 0);
   tp.fresh = __reduce_min_sync(0xffffffffu, my_round) == r;
   tp.prev_round = __reduce_max_sync(0xffffffffu, my_round < r ? my_round : -1);
   const int jp = lane < tp.npairs ? static_cast<int>(__fns(here, 0, lane + 1)) : 0;
   tp.e = __shfl_sync(0xffffffffu, my_idx, jp);
   tp.s = __shfl_sync(0xffffffffu, my_slot, jp);
   const float g = __shfl_sync(0xffffffffu, my_gate, jp);
-  tp.prow = lane < tp.npairs ? static_cast<unsigned long long>(tp.e) * a.C + tp.s : 0ull;
+  unsigned long long row = 0ull;
+  if (lane < tp.npairs)
+    row = a.row_off ? static_cast<unsigned long long>(a.row_off[static_cast<size_t>(r) * a.E + tp.e] - a.row_start[r] + tp.s)
+                    : static_cast<unsigned long long>(tp.e) * a.C + tp.s;
+  tp.prow = row;
+  tp.first_row = __shfl_sync(0xffffffffu, row, 0);
   tp.pgate = lane < tp.npairs ? g : 0.f;
   return tp;
 }
@@ -184,14 +193,14 @@ __device__ __forceinline__ void accumulate_token(const CombineArgs& a, int t, co
 }
 
 // The whole warp combines token t for round r (no-op if t has no pair in round r).
-// With `only_expert` >= 0 the warp stands for one row of the round (token t's pair with that
-// expert) and does the work only if that pair is t's first pair in the round, so that every
-// active token is combined exactly once when the round is walked row by row.
+// With `only_row` >= 0 the warp stands for one buffer row of the round (one of token t's pairs)
+// and does the work only if that row is t's first pair in the round, so that every active
+// token is combined exactly once when the round is walked row by row.
 template <int kLaneCols = 8>
-__device__ __forceinline__ void combine_token(const CombineArgs& a, int t, int r, int only_expert = -1) {
+__device__ __forceinline__ void combine_token(const CombineArgs& a, int t, int r, long long only_row = -1) {
   const TokenPairs tp = token_pairs(a, load_pairs(a, t), r);
   if (tp.npairs == 0) return;
-  if (only_expert >= 0 && tp.first_expert != only_expert) return;
+  if (only_row >= 0 && tp.first_row != static_cast<unsigned long long>(only_row)) return;
   accumulate_token<kLaneCols>(a, t, tp);
 }
 

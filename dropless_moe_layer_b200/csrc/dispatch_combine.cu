@@ -44,15 +44,16 @@ __global__ void __launch_bounds__(32 * kCombineWarps)
     combine_kernel(const copy::CombineArgs a, int r, int by_rows, const int32_t* __restrict__ row_start,
                    const int32_t* __restrict__ row_token, const int32_t* __restrict__ row_dst) {
   const int w = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
-  int t = w, expert = -1;
+  int t = w;
+  long long buf_row = -1;
   if (by_rows) {                       // plan data: written before this forward
     const int row = row_start[r] + w;
     t = row < row_start[r + 1] ? row_token[row] : a.T;
-    if (t < a.T) expert = row_dst[row] / a.C;
+    if (t < a.T) buf_row = row_dst[row];
   }
   sm100::grid_dependency_wait();      // buf comes from the round's down GEMM, y from earlier rounds
   sm100::pdl_trigger_early();
-  if (t < a.T) copy::combine_token<16>(a, t, r, expert);   // 16 columns per lane: more loads in flight
+  if (t < a.T) copy::combine_token<16>(a, t, r, buf_row);   // 16 columns per lane: more loads in flight
   sm100::pdl_trigger_late();
 }
 
@@ -77,14 +78,14 @@ cudaError_t launch_dispatch(const uint16_t* x, uint16_t* buf, const int32_t* row
 cudaError_t launch_combine(const uint16_t* buf, float* y, const int32_t* idx, const float* gate,
                            const int32_t* round, const int32_t* slot, const int32_t* row_start,
                            const int32_t* row_token, const int32_t* row_dst, int T, int k, int C, int d,
-                           int r, int rows, cudaStream_t stream) {
+                           int r, int rows, const int32_t* row_off, int E, cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
   const int by_rows = rows < T ? 1 : 0;
   const int warps = by_rows ? rows : T;
   if (warps <= 0) return cudaSuccess;
   const int blocks = (warps + kCombineWarps - 1) / kCombineWarps;
   launch_begin(kKindCombine, stream);
-  const copy::CombineArgs a{buf, y, idx, gate, round, slot, T, k, C, d};
+  const copy::CombineArgs a{buf, y, idx, gate, round, slot, T, k, C, d, row_off, row_off ? row_start : nullptr, E};
   const cudaError_t err = launch_pdl(combine_kernel, dim3(blocks), dim3(32 * kCombineWarps), 0, stream, a, r,
                                      by_rows, row_start, row_token, row_dst);
   launch_end(kKindCombine, stream);

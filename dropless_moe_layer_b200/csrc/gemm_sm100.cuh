@@ -145,6 +145,10 @@ struct Phase {
   int out_ld;                  // elements
   const float* bias;           // F32Bias
   int n_valid;                 // F32Bias: stored columns
+  // Pooled rows (capacity borrowing): group g's rows start at row group_row[g] - *group_row_base
+  // of a single [rows, K] operand and output, instead of at row 0 of group g. Null: per group.
+  const int32_t* group_row;
+  const int32_t* group_row_base;
 };
 
 // Pipeline counters; each role thread uses its own fields, and they persist across phases.
@@ -300,6 +304,11 @@ __device__ __forceinline__ void run_phase(const Smem& s, uint32_t tmem_base, con
     for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
       int g, mt, nt;
       decode(tile, g, mt, nt);
+      int a_row = mt * BM, a_grp = g;
+      if (p.group_row) {
+        a_row += p.group_row[g] - *p.group_row_base;
+        a_grp = 0;
+      }
       for (int kb = 0; kb < p.num_k_blocks; ++kb) {
         if (!mbar_wait(smem_addr(&s.empty[pipe.stage]), pipe.phase ^ 1u, s.abort)) {
           ok = false;
@@ -309,7 +318,7 @@ __device__ __forceinline__ void run_phase(const Smem& s, uint32_t tmem_base, con
         const uint32_t sB = sA + kABytes;
         const uint32_t fb = smem_addr(&s.full[pipe.stage]);
         mbar_arrive_expect_tx(fb, tx);
-        tma_load_3d(sA, p.a, fb, kb * BK, mt * BM, g);
+        tma_load_3d(sA, p.a, fb, kb * BK, a_row, a_grp);
         if (p.mode == kSwiGLU) {
           tma_load_3d(sB, mb, fb, kb * BK, nt * width, g);
           tma_load_3d(sB + width * BK * 2, mb, fb, kb * BK, p.b_second_row + nt * width, g);
@@ -394,13 +403,14 @@ __device__ __forceinline__ void run_phase(const Smem& s, uint32_t tmem_base, con
       const bool valid = row < rows_g;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(pipe.acc * kAccCols);
+      const long long orow_off = p.group_row
+                                     ? static_cast<long long>(p.group_row[g] - *p.group_row_base + row) * p.out_ld
+                                     : g * p.out_group_stride + static_cast<long long>(row) * p.out_ld;
       if (p.mode == kSwiGLU) {
-        uint16_t* orow = static_cast<uint16_t*>(p.out) + g * p.out_group_stride +
-                         static_cast<long long>(row) * p.out_ld + nt * width;
+        uint16_t* orow = static_cast<uint16_t*>(p.out) + orow_off + nt * width;
         store_swiglu(tb, width, orow, valid);
       } else if (p.mode == kBf16Out) {
-        uint16_t* orow = static_cast<uint16_t*>(p.out) + g * p.out_group_stride +
-                         static_cast<long long>(row) * p.out_ld + nt * width;
+        uint16_t* orow = static_cast<uint16_t*>(p.out) + orow_off + nt * width;
         store_bf16(tb, bn, orow, valid);
       } else {
         float* orow = static_cast<float*>(p.out) + static_cast<long long>(row) * p.out_ld;

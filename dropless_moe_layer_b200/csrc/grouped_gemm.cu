@@ -45,7 +45,7 @@ __device__ __forceinline__ void side_work(const SideArgs& sa) {
     if (sa.by_rows) {
       const int begin = sa.row_start[sa.r], end = sa.row_start[sa.r + 1];
       for (int row = begin + cw; row < end; row += warps)
-        copy::combine_token(sa.comb, sa.row_token[row], sa.r, sa.row_dst[row] / sa.comb.C);
+        copy::combine_token(sa.comb, sa.row_token[row], sa.r, sa.row_dst[row]);
     } else {
       for (int t = cw; t < sa.comb.T; t += warps) copy::combine_token(sa.comb, t, sa.r);
     }
@@ -68,6 +68,8 @@ struct KernelArgs {
   const float* bias;
   int n_valid;
   int32_t* status;
+  const int32_t* group_row;        // pooled rows (see Phase), or null
+  const int32_t* group_row_base;
 };
 
 __global__ void __launch_bounds__(kLaunchThreads, 1)
@@ -100,6 +102,8 @@ __global__ void __launch_bounds__(kLaunchThreads, 1)
   p.out_ld = args.out_ld;
   p.bias = args.bias;
   p.n_valid = args.n_valid;
+  p.group_row = args.group_row;
+  p.group_row_base = args.group_row_base;
   plan_phase(s, p, 0);              // reads only the row counts (plan data)
   __syncthreads();
   // Everything above overlaps the previous kernel; the operands, and the output buffer that
@@ -262,15 +266,18 @@ extern const int kGateUpWidths[3] = {128, 64, 32};   // gate columns per tile (M
 extern const int kDownWidths[3] = {256, 128, 64};
 
 cudaError_t make_gate_up_maps(const uint16_t* buf, const uint16_t* w_gate_up, int E, int C, int d, int F,
-                              CUtensorMap* ma, CUtensorMap* mb) {
-  cudaError_t e = gemm::make_map(ma, buf, d, C, E, gemm::BM);
+                              CUtensorMap* ma, CUtensorMap* mb, bool pooled) {
+  // A: [E][C][d] per expert, or pooled [1][E*C][d] (rows located by the group offsets)
+  cudaError_t e = pooled ? gemm::make_map(ma, buf, d, static_cast<uint64_t>(E) * C, 1, gemm::BM)
+                         : gemm::make_map(ma, buf, d, C, E, gemm::BM);
   if (e != cudaSuccess) return e;
   return gemm::make_b_maps(mb, w_gate_up, d, 2ull * F, E, kGateUpWidths, F);
 }
 
 cudaError_t make_down_maps(const uint16_t* h, const uint16_t* w_down, int E, int C, int d, int F,
-                           CUtensorMap* ma, CUtensorMap* mb) {
-  cudaError_t e = gemm::make_map(ma, h, F, C, E, gemm::BM);
+                           CUtensorMap* ma, CUtensorMap* mb, bool pooled) {
+  cudaError_t e = pooled ? gemm::make_map(ma, h, F, static_cast<uint64_t>(E) * C, 1, gemm::BM)
+                         : gemm::make_map(ma, h, F, C, E, gemm::BM);
   if (e != cudaSuccess) return e;
   return gemm::make_b_maps(mb, w_down, F, d, E, kDownWidths, d);
 }
@@ -288,16 +295,18 @@ static gemm::SideArgs make_side(const RoundCopy* copy) {
   sd.buf = reinterpret_cast<uint4*>(copy->buf);
   sd.vecs = copy->d / 8;
   sd.comb = copy::CombineArgs{copy->out, copy->y, copy->idx, copy->gate, copy->round, copy->slot,
-                              copy->T, copy->k, copy->C, copy->d};
+                              copy->T, copy->k, copy->C, copy->d, copy->row_off,
+                              copy->row_off ? copy->row_start : nullptr, copy->E};
   sd.by_rows = copy->rows < copy->T ? 1 : 0;
   return sd;
 }
 
 cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint16_t* h,
                            const int32_t* n_dev, const int32_t* n_host, int E, int C, int d, int F,
-                           int32_t* status, const RoundCopy* copy, cudaStream_t stream) {
+                           int32_t* status, const RoundCopy* copy, const int32_t* group_row,
+                           const int32_t* group_row_base, cudaStream_t stream) {
   CUtensorMap ma, mb[3];
-  cudaError_t e = make_gate_up_maps(buf, w_gate_up, E, C, d, F, &ma, mb);
+  cudaError_t e = make_gate_up_maps(buf, w_gate_up, E, C, d, F, &ma, mb, group_row != nullptr);
   if (e != cudaSuccess) return e;
   gemm::KernelArgs a{};
   a.mode = gemm::kSwiGLU;
@@ -311,15 +320,18 @@ cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint1
   a.out_group_stride = static_cast<long long>(C) * F;
   a.out_ld = F;
   a.status = status;
+  a.group_row = group_row;
+  a.group_row_base = group_row_base;
   const long long tiles = gemm::choose_width(n_host, E, 0, F, a);
   return gemm::run(ma, mb, a, tiles, make_side(copy), kKindGateUp, stream);
 }
 
 cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out, const int32_t* n_dev,
                         const int32_t* n_host, int E, int C, int d, int F, int32_t* status,
-                        const RoundCopy* copy, cudaStream_t stream) {
+                        const RoundCopy* copy, const int32_t* group_row, const int32_t* group_row_base,
+                        cudaStream_t stream) {
   CUtensorMap ma, mb[3];
-  cudaError_t e = make_down_maps(h, w_down, E, C, d, F, &ma, mb);
+  cudaError_t e = make_down_maps(h, w_down, E, C, d, F, &ma, mb, group_row != nullptr);
   if (e != cudaSuccess) return e;
   gemm::KernelArgs a{};
   a.mode = gemm::kBf16Out;
@@ -332,6 +344,8 @@ cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out
   a.out_group_stride = static_cast<long long>(C) * d;
   a.out_ld = d;
   a.status = status;
+  a.group_row = group_row;
+  a.group_row_base = group_row_base;
   const long long tiles = gemm::choose_width(n_host, E, 0, d, a);
   return gemm::run(ma, mb, a, tiles, make_side(copy), kKindDown, stream);
 }

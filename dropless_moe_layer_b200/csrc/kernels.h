@@ -117,6 +117,7 @@ struct PlanBuffers {
   int32_t* mb_prefix;     // [max_rounds, E + 1] 128-row blocks of experts < e in round r, or null
   int32_t* sync;          // pipelined-rounds counters to zero ([sync_words]), or null
   long long sync_words;
+  int borrow;             // 1: capacity borrowing (rows packed per round, n[r][e] may exceed C)
 };
 cudaError_t launch_plan(const PlanBuffers& b, int T, int k, int E, int C, int max_rounds,
                         cudaStream_t stream);
@@ -127,10 +128,12 @@ cudaError_t launch_dispatch(const uint16_t* x, uint16_t* buf, const int32_t* row
                             int d, cudaStream_t stream);
 // rows: rows of round r (host copy); the kernel walks the round's rows instead of all T
 // tokens when there are fewer of them.
+// row_off: pooled round rows (capacity borrowing: pair (e, slot) of round r at buffer row
+// row_off[r][e] - row_start[r] + slot), or null for the per-expert [E, C, d] buffer.
 cudaError_t launch_combine(const uint16_t* buf, float* y, const int32_t* idx, const float* gate,
                            const int32_t* round, const int32_t* slot, const int32_t* row_start,
                            const int32_t* row_token, const int32_t* row_dst, int T, int k, int C, int d,
-                           int r, int rows, cudaStream_t stream);
+                           int r, int rows, const int32_t* row_off, int E, cudaStream_t stream);
 
 // ---- grouped GEMMs (grouped_gemm.cu)
 // gate_up: h[e][s] = bf16(silu(buf[e][s] W1_e^T) * (buf[e][s] W3_e^T)), s < n_dev[e]
@@ -152,17 +155,23 @@ struct RoundCopy {
   const int32_t* round;
   const int32_t* slot;
   int T, k, C, d;
+  const int32_t* row_off;    // pooled round rows (capacity borrowing), or null
+  int E;
 };
 
 // n_dev: rows per expert this round on the device (read by the kernel); n_host: the same on
 // the host (picks the tile width and the grid). copy: optional side copy step, or null.
+// group_row / group_row_base: pooled round rows (capacity borrowing: expert e's rows start at
+// buffer row group_row[e] - *group_row_base), or null for the per-expert [E, C, .] buffers.
 cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint16_t* h,
                            const int32_t* n_dev, const int32_t* n_host, int E, int C, int d, int F,
-                           int32_t* status, const RoundCopy* copy, cudaStream_t stream);
+                           int32_t* status, const RoundCopy* copy, const int32_t* group_row,
+                           const int32_t* group_row_base, cudaStream_t stream);
 // down: out[e][s] = bf16(h[e][s] W2_e^T), s < n_dev[e]
 cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out, const int32_t* n_dev,
                         const int32_t* n_host, int E, int C, int d, int F, int32_t* status,
-                        const RoundCopy* copy, cudaStream_t stream);
+                        const RoundCopy* copy, const int32_t* group_row, const int32_t* group_row_base,
+                        cudaStream_t stream);
 
 // ---- pipelined rounds (round_pipeline.cu)
 // Rounds [r0, R) of the layer in one persistent launch (one CTA per SM): dispatch, gate/up

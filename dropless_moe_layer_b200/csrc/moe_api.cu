@@ -74,9 +74,11 @@ namespace {
 
 int check_shape(const moe_shape_t* s) {
   if (s == nullptr) return MOE_ERR_INVALID_ARG;
-  if (s->flags & ~static_cast<uint32_t>(MOE_FLAG_RENORM_TOPK | MOE_FLAG_PER_ROUND | MOE_FLAG_PIPELINE_ALL))
+  if (s->flags & ~static_cast<uint32_t>(MOE_FLAG_RENORM_TOPK | MOE_FLAG_PER_ROUND | MOE_FLAG_PIPELINE_ALL |
+                                        MOE_FLAG_BORROW))
     return MOE_ERR_INVALID_ARG;
   if ((s->flags & MOE_FLAG_PER_ROUND) && (s->flags & MOE_FLAG_PIPELINE_ALL)) return MOE_ERR_INVALID_ARG;
+  if ((s->flags & MOE_FLAG_BORROW) && (s->flags & MOE_FLAG_PIPELINE_ALL)) return MOE_ERR_INVALID_ARG;
   if (s->T < 0 || s->E < 1 || s->E > MOE_MAX_EXPERTS || s->k < 1 || s->k > MOE_MAX_TOPK ||
       s->k > s->E || s->C < 1)
     return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -122,7 +124,7 @@ void make_layout(const moe_shape_t* s, moe_workspace_layout_t* L) {
   L->out = take(E * C * s->d * 2);
   L->mb_prefix = take(static_cast<long long>(mr) * (E + 1) * 4);
   L->sync = take(pipe_sync_words(s->E, s->C) * 4);
-  if (!(s->flags & MOE_FLAG_PER_ROUND)) {   // second buffer set of the pipelined launch
+  if (!(s->flags & (MOE_FLAG_PER_ROUND | MOE_FLAG_BORROW))) {   // second buffer set of the pipelined launch
     L->buf2 = take(E * C * s->d * 2);
     L->h2 = take(E * C * s->d_ff * 2);
     L->out2 = take(E * C * s->d * 2);
@@ -172,13 +174,40 @@ int check_run(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, s
   return check_device();
 }
 
+bool borrowing(const moe_shape_t* s) { return (s->flags & MOE_FLAG_BORROW) != 0; }
+
+// Rows of each expert in round r, on the host, from the loads: the same integer rule as the
+// planner's (min(C, what is left) without borrowing; with borrowing, the planner's
+// round-by-round lending of the E*C pool, replayed up to round r).
 void round_rows(const moe_shape_t* s, const moe_plan_info_t* info, int r, int32_t* n_host, int* rows) {
   long long total = 0;
-  const long long base = static_cast<long long>(r) * s->C;
-  for (int e = 0; e < s->E; ++e) {
-    const long long rem = info->load[e] - base;
-    n_host[e] = rem <= 0 ? 0 : rem >= s->C ? s->C : static_cast<int32_t>(rem);
-    total += n_host[e];
+  if (!borrowing(s)) {
+    const long long base = static_cast<long long>(r) * s->C;
+    for (int e = 0; e < s->E; ++e) {
+      const long long rem = info->load[e] - base;
+      n_host[e] = rem <= 0 ? 0 : rem >= s->C ? s->C : static_cast<int32_t>(rem);
+      total += n_host[e];
+    }
+    *rows = static_cast<int>(total);
+    return;
+  }
+  long long pending[MOE_MAX_EXPERTS];
+  for (int e = 0; e < s->E; ++e) pending[e] = info->load[e];
+  const long long pool = static_cast<long long>(s->E) * s->C;
+  for (int rr = 0; rr <= r; ++rr) {
+    long long own_sum = 0;
+    for (int e = 0; e < s->E; ++e) own_sum += pending[e] < s->C ? pending[e] : s->C;
+    long long spare = pool - own_sum;
+    total = 0;
+    for (int e = 0; e < s->E; ++e) {
+      const long long own = pending[e] < s->C ? pending[e] : s->C;
+      const long long want = pending[e] - own;
+      const long long extra = want < spare ? want : spare;
+      spare -= extra;
+      n_host[e] = static_cast<int32_t>(own + extra);
+      pending[e] -= own + extra;
+      total += n_host[e];
+    }
   }
   *rows = static_cast<int>(total);
 }
@@ -220,6 +249,8 @@ RoundCopy make_copy(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
   c.k = s->k;
   c.C = s->C;
   c.d = s->d;
+  c.row_off = borrowing(s) ? at<int32_t>(ws, L.row_off) : nullptr;
+  c.E = s->E;
   return c;
 }
 
@@ -229,10 +260,12 @@ int do_gate_up(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
   int32_t n_host[MOE_MAX_EXPERTS];
   int rows = 0;
   round_rows(s, info, r, n_host, &rows);
+  const bool pooled = borrowing(s);
   return cuda_status(launch_gate_up(at<uint16_t>(ws, L.buf), w13, at<uint16_t>(ws, L.h),
                                     at<int32_t>(ws, L.n) + static_cast<size_t>(r) * s->E, n_host, s->E,
                                     s->C, s->d, s->d_ff, at<int32_t>(ws, L.header) + kHdrStatus, copy,
-                                    stream));
+                                    pooled ? at<int32_t>(ws, L.row_off) + static_cast<size_t>(r) * s->E : nullptr,
+                                    pooled ? at<int32_t>(ws, L.row_start) + r : nullptr, stream));
 }
 
 int do_down(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
@@ -241,9 +274,12 @@ int do_down(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
   int32_t n_host[MOE_MAX_EXPERTS];
   int rows = 0;
   round_rows(s, info, r, n_host, &rows);
+  const bool pooled = borrowing(s);
   return cuda_status(launch_down(at<uint16_t>(ws, L.h), w2, at<uint16_t>(ws, L.out),
                                  at<int32_t>(ws, L.n) + static_cast<size_t>(r) * s->E, n_host, s->E,
-                                 s->C, s->d, s->d_ff, at<int32_t>(ws, L.header) + kHdrStatus, copy, stream));
+                                 s->C, s->d, s->d_ff, at<int32_t>(ws, L.header) + kHdrStatus, copy,
+                                 pooled ? at<int32_t>(ws, L.row_off) + static_cast<size_t>(r) * s->E : nullptr,
+                                 pooled ? at<int32_t>(ws, L.row_start) + r : nullptr, stream));
 }
 
 int do_combine(const moe_shape_t* s, const moe_plan_info_t* info, void* ws, const moe_workspace_layout_t& L,
@@ -255,7 +291,8 @@ int do_combine(const moe_shape_t* s, const moe_plan_info_t* info, void* ws, cons
                                     at<float>(ws, L.gate), at<int32_t>(ws, L.round),
                                     at<int32_t>(ws, L.slot), at<int32_t>(ws, L.row_start),
                                     at<int32_t>(ws, L.row_token), at<int32_t>(ws, L.row_dst), s->T, s->k,
-                                    s->C, s->d, r, rows, stream));
+                                    s->C, s->d, r, rows, borrowing(s) ? at<int32_t>(ws, L.row_off) : nullptr,
+                                    s->E, stream));
 }
 
 }  // namespace
@@ -327,6 +364,7 @@ int moe_plan(const moe_shape_t* shape, const float* logits, const uint16_t* x,
   pb.mb_prefix = at<int32_t>(ws, L.mb_prefix);
   pb.sync = at<int32_t>(ws, L.sync);
   pb.sync_words = pipe_sync_words(s.E, s.C);
+  pb.borrow = (s.flags & MOE_FLAG_BORROW) ? 1 : 0;
   if ((st = cuda_status(launch_plan(pb, s.T, s.k, s.E, s.C, L.max_rounds, stream))) != MOE_OK) return st;
 
   int32_t host[kHdrWords];
@@ -425,7 +463,7 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
   int r0 = R;
   if (shape->flags & MOE_FLAG_PIPELINE_ALL) {
     r0 = 0;
-  } else if (!(shape->flags & MOE_FLAG_PER_ROUND)) {
+  } else if (!(shape->flags & (MOE_FLAG_PER_ROUND | MOE_FLAG_BORROW))) {   // borrowing: per-round only
     while (r0 > 0 && thin(r0 - 1)) --r0;
   }
   // Per-round launch order. A small copy step (a thin round: at most kFuseCopyBytes of rows)

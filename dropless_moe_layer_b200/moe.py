@@ -21,6 +21,7 @@ PROFILE_NAMES = ["router_gemm", "topk", "plan", "dispatch", "gate_up", "down", "
 FLAG_RENORM_TOPK = 1
 FLAG_PER_ROUND = 2
 FLAG_PIPELINE_ALL = 4
+FLAG_BORROW = 8
 SCHEDULES = {"auto": 0, "per_round": FLAG_PER_ROUND, "pipeline": FLAG_PIPELINE_ALL}
 
 STATUS = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED_SHAPE",
@@ -112,9 +113,11 @@ def _check(call: str, status: int) -> None:
 
 
 def make_shape(T: int, d: int, E: int, k: int, d_ff: int, C: int, renorm: bool = False,
-               schedule: str = "auto") -> Shape:
-    """schedule: "auto" (trailing small rounds pipelined), "per_round" or "pipeline"."""
-    return Shape(T, d, E, k, d_ff, C, (FLAG_RENORM_TOPK if renorm else 0) | SCHEDULES[schedule])
+               schedule: str = "auto", borrow: bool = False) -> Shape:
+    """schedule: "auto" (trailing thin rounds pipelined), "per_round" or "pipeline";
+    borrow: capacity borrowing between experts (MOE_FLAG_BORROW)."""
+    return Shape(T, d, E, k, d_ff, C, (FLAG_RENORM_TOPK if renorm else 0) | SCHEDULES[schedule] |
+                 (FLAG_BORROW if borrow else 0))
 
 
 # ------------------------------------------------------------------------- raw-pointer calls
@@ -208,9 +211,9 @@ class DroplessMoE:
     """
 
     def __init__(self, T: int, d: int, E: int, k: int, d_ff: int, C: int, renorm: bool = False,
-                 device=None, schedule: str = "auto"):
+                 device=None, schedule: str = "auto", borrow: bool = False):
         import torch
-        self.shape = make_shape(T, d, E, k, d_ff, C, renorm, schedule)
+        self.shape = make_shape(T, d, E, k, d_ff, C, renorm, schedule, borrow)
         self.ws_bytes = workspace_bytes(self.shape)
         if self.ws_bytes == 0:
             raise ValueError(f"unsupported shape T={T} d={d} E={E} k={k} d_ff={d_ff} C={C}")

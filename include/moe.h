@@ -82,6 +82,18 @@ typedef enum moe_status {
  * MOE_FLAG_PER_ROUND is given. */
 #define MOE_FLAG_PER_ROUND 2u       /* every round as per-round launches */
 #define MOE_FLAG_PIPELINE_ALL 4u    /* every round in the pipelined launch */
+/* Capacity borrowing ("Frontier Pre-training at Microsoft AI (MAI-Base-2)", Key claims,
+ * multi-round dropless MoE item: overflow tokens use unused capacity of other experts of the
+ * group, otherwise an extra round). Each round still holds at most E*C rows (the same fixed
+ * buffers), but an overloaded expert takes the rows other experts leave unused: every expert
+ * first takes up to C of its pending pairs, then the unused rows go to experts with pairs
+ * pending, in ascending expert index. An expert may then hold more than C rows of a round, so
+ * the round's rows are packed expert after expert (pair (e, slot) of round r at buffer row
+ * row_off[r][e] - row_start[r] + slot, the layout's row lists) and `slot` counts from 0 within
+ * the expert's rows of the round, up to n[r][e]-1. R never exceeds ceil(max_load / C) and is
+ * 1 whenever T*k <= E*C. Runs as per-round launches (not with MOE_FLAG_PIPELINE_ALL); y is the
+ * same layer output. Off by default: the default plan is R = ceil(max_load / C). */
+#define MOE_FLAG_BORROW 8u
 
 #define MOE_MAX_EXPERTS 256
 #define MOE_MAX_TOPK 16

@@ -81,9 +81,13 @@ def test_bad_shapes_are_rejected(lib, kw):
 
 def test_bad_flags_rejected(lib):
     s = moe.make_shape(64, 128, 8, 2, 128, 16)
-    for flags in (8, 1 << 31, moe.FLAG_PER_ROUND | moe.FLAG_PIPELINE_ALL):
+    for flags in (16, 1 << 31, moe.FLAG_PER_ROUND | moe.FLAG_PIPELINE_ALL,
+                  moe.FLAG_BORROW | moe.FLAG_PIPELINE_ALL):
         s.flags = flags
         assert moe.workspace_bytes(s) == 0
+    # borrowing runs per round: no second buffer set, like the per-round schedule
+    assert moe.workspace_bytes(moe.make_shape(64, 128, 8, 2, 128, 16, borrow=True)) == \
+        moe.workspace_bytes(moe.make_shape(64, 128, 8, 2, 128, 16, schedule="per_round"))
     # the pipelined schedules share one layout; per-round only drops the second buffer set
     assert moe.workspace_bytes(moe.make_shape(64, 128, 8, 2, 128, 16, schedule="pipeline")) == \
         moe.workspace_bytes(moe.make_shape(64, 128, 8, 2, 128, 16))

@@ -63,9 +63,9 @@ def rel_err(got, ref):
 SCHEDULES = ["auto", "per_round", "pipeline"]
 
 
-def run_gpu(w, inp, C=None, renorm=False, schedule="auto"):
+def run_gpu(w, inp, C=None, renorm=False, schedule="auto", borrow=False):
     C = C or w.C
-    layer = moe.DroplessMoE(w.T, w.d, w.E, w.k, w.F, C, renorm=renorm, schedule=schedule)
+    layer = moe.DroplessMoE(w.T, w.d, w.E, w.k, w.F, C, renorm=renorm, schedule=schedule, borrow=borrow)
     y = layer(inp["x"], inp["w_gate_up"], inp["w_down"], logits=inp["logits"],
               w_router=inp["w_router"], bias=inp["bias"])
     torch.cuda.synchronize()
@@ -73,14 +73,14 @@ def run_gpu(w, inp, C=None, renorm=False, schedule="auto"):
     return layer, y
 
 
-def check_plan(layer, w, C, z, renorm=False):
+def check_plan(layer, w, C, z, renorm=False, borrow=False):
     """Routing and plan bit-exact against the oracle on the logits the GPU used."""
     pt = layer.plan_tensors()
     idx_ref = oracle.select_topk(z, w.k)
     np.testing.assert_array_equal(pt["topk_idx"].cpu().numpy(), idx_ref)
     g_ref = oracle.gates(z, idx_ref, renorm)
     np.testing.assert_allclose(pt["gate"].cpu().numpy(), g_ref, rtol=GATE_RTOL, atol=1e-12)
-    p = oracle.plan(idx_ref, w.E, C)
+    p = oracle.plan_borrow(idx_ref, w.E, C) if borrow else oracle.plan(idx_ref, w.E, C)
     info = layer.info
     assert info.R == p["R"] and info.max_load == p["max_load"]
     assert list(info.load)[:w.E] == list(p["load"])
@@ -309,3 +309,46 @@ def test_pipeline_counters_return_to_zero_and_repeat():
     torch.cuda.synchronize()
     assert layer.device_status() == 0
     assert torch.equal(y1, y2)
+
+
+# ----------------------------------------------------------------------------- capacity borrowing
+
+@pytest.mark.parametrize("name", ["tiny-zipf1", "4k-zipf1"])
+def test_borrow_full_parity(name):
+    """Capacity borrowing: the plan bit-exact against the oracle's borrowing plan (fewer
+    rounds on skewed routing), y the same layer output."""
+    w = wl.BY_NAME[name]
+    inp = wl.generate(w, "cuda")
+    layer, y = run_gpu(w, inp, borrow=True)
+    z = inp["logits"].cpu().numpy()
+    idx, g, p = check_plan(layer, w, w.C, z, borrow=True)
+    assert p["R"] < oracle.plan(idx, w.E, w.C)["R"]
+    ref = oracle.forward(bits(inp["x"]), LazyExperts(inp["w_gate_up"]), LazyExperts(inp["w_down"]), idx, g)
+    assert rel_err(y.cpu().numpy().astype(np.float64), ref) <= Y_TOL
+
+
+@pytest.mark.parametrize("cfg", EDGE, ids=lambda c: "T{T}-d{d}-E{E}-k{k}-F{F}-C{C}".format(**c))
+def test_borrow_edge_shapes(cfg):
+    w = wl.custom(name="edge", T=cfg["T"], d=cfg["d"], E=cfg["E"], k=cfg["k"], F=cfg["F"], C=cfg["C"],
+                  bias="zipf", zipf_s=1.0, seed=cfg["T"])
+    inp = wl.generate(w, "cuda")
+    layer, y = run_gpu(w, inp, borrow=True)
+    idx, g, p = check_plan(layer, w, w.C, inp["logits"].cpu().numpy(), borrow=True)
+    ref = oracle.forward(bits(inp["x"]), LazyExperts(inp["w_gate_up"]), LazyExperts(inp["w_down"]), idx, g)
+    assert rel_err(y.cpu().numpy().astype(np.float64), ref) <= Y_TOL
+
+
+def test_borrow_sampled_parity_hot_expert():
+    """16k-hot-expert with borrowing: the hot expert's overflow fills the other experts'
+    unused rows; plan on every token, y on a token sample."""
+    w = wl.BY_NAME["16k-hot-expert"]
+    inp = wl.generate(w, "cuda")
+    layer, y = run_gpu(w, inp, borrow=True)
+    z = inp["logits"].cpu().numpy()
+    idx, g, p = check_plan(layer, w, w.C, z, borrow=True)
+    assert p["R"] < oracle.plan(idx, w.E, w.C)["R"]
+    tok = sample_tokens(w.T, p, 64, seed=w.seed)
+    ref = oracle.forward(LazyRows(inp["x"]), LazyExperts(inp["w_gate_up"]), LazyExperts(inp["w_down"]), idx, g,
+                         tokens=tok)
+    got = y[torch.as_tensor(tok, device="cuda")].cpu().numpy().astype(np.float64)
+    assert rel_err(got, ref) <= Y_TOL
