@@ -171,6 +171,8 @@ int check_run(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, s
   if (ws_bytes < L->total_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
   if (!aligned(ws, 256)) return MOE_ERR_MISALIGNED;
   if (info->R < 0 || info->R > L->max_rounds) return MOE_ERR_INVALID_ARG;
+  // the plan was made for this kind of plan (with or without borrowing)
+  if ((info->plan_flags ^ shape->flags) & MOE_FLAG_BORROW) return MOE_ERR_INVALID_ARG;
   return check_device();
 }
 
@@ -383,6 +385,7 @@ int moe_plan(const moe_shape_t* shape, const float* logits, const uint16_t* x,
   info->slot = pb.slot;
   info->offsets = pb.offsets;
   info->n = pb.n;
+  info->plan_flags = s.flags & MOE_FLAG_BORROW;
   return MOE_OK;
 }
 
@@ -474,19 +477,26 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
   // combine reads out and updates y. A run of thin rounds thus costs two launches per round.
   // The first pipelined round is dispatched here too (by the dispatch kernel, or on the last
   // per-round down GEMM), so the pipelined launch starts with its rows in place.
+  // Rounds [rb, re) as per-round launches, round rb's rows already dispatched and the combine
+  // of round rb-1 already issued.
+  auto per_round = [&](int rb, int re) -> int {
+    int rc = MOE_OK;
+    for (int r = rb; r < re; ++r) {
+      const bool fuse_combine = r > rb && small(r - 1);
+      const RoundCopy comb = make_copy(shape, info, ws, L, true, r > 0 ? r - 1 : 0, x, y);
+      if ((rc = do_gate_up(shape, info, ws, L, r, w_gate_up, fuse_combine ? &comb : nullptr, stream)) != MOE_OK)
+        return rc;
+      const bool next = r + 1 < R;
+      const bool fuse_dispatch = next && small(r + 1);
+      const RoundCopy disp = make_copy(shape, info, ws, L, false, next ? r + 1 : r, x, y);
+      if ((rc = do_down(shape, info, ws, L, r, w_down, fuse_dispatch ? &disp : nullptr, stream)) != MOE_OK) return rc;
+      if (next && !fuse_dispatch && (rc = do_dispatch(shape, info, ws, L, r + 1, x, stream)) != MOE_OK) return rc;
+      if (!(r + 1 < re && small(r)) && (rc = do_combine(shape, info, ws, L, r, y, stream)) != MOE_OK) return rc;
+    }
+    return rc;
+  };
   if ((st = do_dispatch(shape, info, ws, L, 0, x, stream)) != MOE_OK) return st;
-  for (int r = 0; r < r0; ++r) {
-    const bool fuse_combine = r > 0 && small(r - 1);
-    const RoundCopy comb = make_copy(shape, info, ws, L, true, r > 0 ? r - 1 : 0, x, y);
-    if ((st = do_gate_up(shape, info, ws, L, r, w_gate_up, fuse_combine ? &comb : nullptr, stream)) != MOE_OK)
-      return st;
-    const bool next = r + 1 < R;
-    const bool fuse_dispatch = next && small(r + 1);
-    const RoundCopy disp = make_copy(shape, info, ws, L, false, next ? r + 1 : r, x, y);
-    if ((st = do_down(shape, info, ws, L, r, w_down, fuse_dispatch ? &disp : nullptr, stream)) != MOE_OK) return st;
-    if (next && !fuse_dispatch && (st = do_dispatch(shape, info, ws, L, r + 1, x, stream)) != MOE_OK) return st;
-    if (!(r + 1 < r0 && small(r)) && (st = do_combine(shape, info, ws, L, r, y, stream)) != MOE_OK) return st;
-  }
+  if ((st = per_round(0, r0)) != MOE_OK) return st;
   if (r0 < R) {
     PipelineArgs p{};
     p.x = x;
@@ -519,7 +529,13 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
     p.r0 = r0;
     p.R = R;
     p.r0_dispatched = 1;
-    if ((st = cuda_status(launch_round_pipeline(p, stream))) != MOE_OK) return st;
+    const cudaError_t e = launch_round_pipeline(p, stream);
+    if (e == cudaErrorCooperativeLaunchTooLarge) {
+      // not every SM is available to this context (a partitioned GPU): run those rounds per round
+      cudaGetLastError();
+      return per_round(r0, R);
+    }
+    if ((st = cuda_status(e)) != MOE_OK) return st;
   }
   return MOE_OK;
 }

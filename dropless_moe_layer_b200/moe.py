@@ -37,7 +37,7 @@ class Shape(ctypes.Structure):
 class PlanInfo(ctypes.Structure):
     _fields_ = [("R", c_i32), ("max_load", c_i32), ("load", c_i32 * MAX_EXPERTS),
                 ("logits", c_vp), ("topk_idx", c_vp), ("gate", c_vp), ("round", c_vp),
-                ("slot", c_vp), ("offsets", c_vp), ("n", c_vp)]
+                ("slot", c_vp), ("offsets", c_vp), ("n", c_vp), ("plan_flags", c_u32)]
 
 
 class WorkspaceLayout(ctypes.Structure):

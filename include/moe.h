@@ -118,6 +118,8 @@ typedef struct moe_plan_info {
   const int32_t* slot;              /* [T, k] row of the pair inside its expert's C rows */
   const int32_t* offsets;           /* [E + 1] exclusive prefix sum of load */
   const int32_t* n;                 /* [max_rounds, E] rows of expert e in round r */
+  uint32_t plan_flags;              /* the shape flags that decide the plan (MOE_FLAG_BORROW);
+                                       calls that run the plan reject a shape whose flags differ */
 } moe_plan_info_t;
 
 /* Byte offsets of the sub-buffers inside the workspace (all 256-byte aligned). */

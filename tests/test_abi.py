@@ -128,3 +128,11 @@ def test_forward_argument_errors_without_gpu(lib):
         f = getattr(lib, fn)
         assert f(P(s), P(info), ws, need - 256, 0, 4096, None) == -3
         assert f(P(s), P(info), ws + 64, need, 0, 4096, None) == -4
+    # a plan made with capacity borrowing cannot be run as a plan without it, nor the reverse
+    sb = moe.make_shape(64, 128, 8, 2, 128, 16, borrow=True)
+    need_b = moe.workspace_bytes(sb)
+    info.plan_flags = moe.FLAG_BORROW
+    assert lib.moe_forward(P(s), P(info), ws, need, 4096, 4096, 4096, 4096, None) == -1
+    assert lib.moe_round_combine(P(s), P(info), ws, need, 0, 4096, None) == -1
+    info.plan_flags = 0
+    assert lib.moe_forward(P(sb), P(info), ws, need_b, 4096, 4096, 4096, 4096, None) == -1
