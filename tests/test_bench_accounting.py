@@ -1,0 +1,54 @@
+"""The benchmark's algorithmic-work accounting (pure host logic): the per-kernel units of one
+step add up to the layer's totals however the rounds are split between per-round launches and
+the pipelined launch, and nothing counts padding rows."""
+import types
+
+import numpy as np
+import pytest
+
+import bench
+import oracle
+from dropless_moe_layer_b200 import workloads as wl
+
+
+def _plan(name, borrow=False):
+    w = wl.BY_NAME[name]
+    z = wl.generate(w, "cpu", routing_only=True)["logits"].numpy()
+    idx = oracle.select_topk(z, w.k)
+    p = (oracle.plan_borrow if borrow else oracle.plan)(idx, w.E, w.C)
+    info = types.SimpleNamespace(load=list(p["load"]) + [0] * (256 - w.E), R=p["R"])
+    return w, p, info
+
+
+@pytest.mark.parametrize("name", ["tiny-zipf1", "4k-zipf1"])
+def test_work_totals_do_not_depend_on_the_split(name):
+    w, p, info = _plan(name)
+    pairs = w.T * w.k
+    for r0 in range(0, p["R"] + 1):
+        work = bench.algorithmic_work(w, info, r0, p["round"], p["n"])
+        flops = work["gate_up"][1] + work["down"][1]
+        if "pipeline" in work:
+            flops += work["pipeline"][1][0]
+        assert flops == 6 * pairs * w.d * w.F                      # every pair's GEMM work once
+        comb = work["combine"][1] + (bench.combine_bytes(w, p["round"], set(range(r0, p["R"])))
+                                     if r0 < p["R"] else 0)
+        assert comb == bench.combine_bytes(w, p["round"])          # combine bytes split exactly
+        assert ("pipeline" in work) == (r0 < p["R"])
+
+
+def test_combine_bytes_closed_form():
+    """Each pair's row is read once; each token writes y once per round it has pairs in and
+    reads it back on every such round but its first."""
+    w, p, info = _plan("tiny-zipf1")
+    spans = np.array([len(set(r)) for r in p["round"].tolist()])
+    want = w.T * w.k * w.d * 2 + spans.sum() * w.d * 4 + (spans - 1).sum() * w.d * 4
+    assert bench.combine_bytes(w, p["round"]) == want
+
+
+def test_borrowing_plan_rows_feed_the_accounting():
+    """With borrowing an expert may hold more than C rows of a round: the accounting takes the
+    plan's own n, so the GEMM work still counts every pair once."""
+    w, p, info = _plan("4k-zipf1", borrow=True)
+    assert p["n"].max() > w.C
+    work = bench.algorithmic_work(w, info, p["R"], p["round"], p["n"])
+    assert work["gate_up"][1] + work["down"][1] == 6 * w.T * w.k * w.d * w.F
