@@ -1,11 +1,16 @@
 """Benchmark: routed tokens/s of one multi-round dropless MoE layer forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+                    [--schedule auto|per_round|pipeline] [--borrow]
 
 One step = moe_plan (router top-k + round planner) + moe_forward (all rounds of dispatch ->
 gate/up GEMM -> down GEMM -> combine) on one batch, inputs resident in HBM. L2 is flushed
 (a 256 MiB write) between timed steps, outside the timed events. Per-step device time comes
-from CUDA events on the launching stream; the job time is the max over ranks.
+from CUDA events on the launching stream; the job time is the max over ranks. The `e2e` key
+times the same calls with each step's inputs copied in from pinned host memory and its result
+copied out, the copies of neighbouring steps overlapping the compute (the sequential form is
+reported beside it). --borrow turns on capacity borrowing (not the plan the metric is defined
+on; reported as such in `config`).
 
 Multi-GPU: the layer's experts all live on one GPU, so N GPUs run N independent replicas
 (weak scaling, no collective on the data path); torch.distributed is used only for the

@@ -285,6 +285,9 @@ class DroplessMoE:
         )
 
     def round_buffer(self):
+        """The dispatch buffer as [E, C, d] (expert e's rows at e, 0..). With capacity borrowing
+        the round's rows are packed instead: row row_off[r][e] - row_start[r] + slot of the
+        flattened [E * C, d] view."""
         import torch
         s, L = self.shape, self.layout
         return self._view(L.buf, s.E * s.C * s.d, torch.bfloat16).view(s.E, s.C, s.d)
