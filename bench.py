@@ -43,21 +43,45 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic per launch of a kernel, from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum per launch; summaries in profiles/), valid only while the kernel's
-# sources hash to the recorded value.
+# sources, with comments and blank space taken out, hash to the recorded value.
 TRAFFIC = {
     ("4k-zipf1", "pipeline"): {
         "bytes_per_launch": 67.653888e6 + 13.169408e6,
         "sources": ["sm100.cuh", "gemm_sm100.cuh", "copy_phases.cuh", "kernels.h", "round_pipeline.cu"],
-        "sources_sha1": "301617e10d4489f33286ca315f162b3e7a966e5b"},
+        "sources_sha1": "5eedc768a5e12125b43c8dc1e1ed41004ae8d580"},
 }
+
+
+def code_tokens(src):
+    """C++ source without its comments, each line's blank space collapsed, blank lines dropped:
+    an edit to comments or layout leaves it unchanged, an edit to code does not."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        if src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif src[i] in "\"'":
+            q, j = src[i], i + 1
+            while j < n and src[j] != q:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(src[i])
+            i += 1
+    return "\n".join(" ".join(l.split()) for l in "".join(out).splitlines() if l.strip())
 
 
 def sources_sha1(files):
     import hashlib
     h = hashlib.sha1()
     for f in files:
-        with open(os.path.join(ROOT, "dropless_moe_layer_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "dropless_moe_layer_b200", "csrc", f)) as fh:
+            h.update(code_tokens(fh.read()).encode())
     return h.hexdigest()
 
 

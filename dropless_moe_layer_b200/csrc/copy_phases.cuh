@@ -79,13 +79,13 @@ struct CombineArgs {
 // One token's pairs in one round, spread over the warp (every lane holds the same scalars;
 // lane p < npairs holds pair p's source row and gate, pairs in ascending j).
 struct TokenPairs {
-  int npairs;               // pairs of the token in round r (0: nothing to do)
-  bool fresh;               // r is the token's first round: y starts from zero
-  int prev_round;           // the token's latest round before r, or -1
+  int npairs;                     // pairs of the token in round r (0: nothing to do)
+  bool fresh;                     // r is the token's first round: y starts from zero
+  int prev_round;                 // the token's latest round before r, or -1
   unsigned long long first_row;   // buffer row of the token's first pair in round r
-  int e, s;                 // this lane's pair (expert, slot), lane < npairs
-  unsigned long long prow;  // e * C + s
-  float pgate;
+  int e, s;                       // this lane's pair (expert, slot), lane < npairs
+  unsigned long long prow;        // its buffer row: e * C + s, or the pooled row
+  float pgate;                    // its gate (0 for lanes >= npairs)
 };
 
 // A token's plan entries as loaded: lane j < k holds pair j's round, expert, slot and gate.

@@ -38,9 +38,9 @@
 // step earlier in the order
 //   D(r0) G(r0)  D(r0+1) G(r0+1) N(r0)  D(r0+2) G(r0+2) N(r0+1) C(r0)  D(r0+3) G(r0+3) N(r0+2)
 //   C(r0+1) ...
-// and every role takes its own steps in that order (a combine warp its items round by round). With every CTA resident (a cooperative
-// launch of one CTA per SM) the earliest unfinished step always has its inputs and a role that
-// is working on it, so the launch cannot deadlock.
+// and every role takes its own steps in that order (a combine warp its tokens round by round).
+// With every CTA resident (a cooperative launch of one CTA per SM) the earliest unfinished step
+// always has its inputs and a role that is working on it, so the launch cannot deadlock.
 //
 // Memory ordering: the threads that wrote a step's data issue a generic-to-async proxy fence
 // (the data may next be read by TMA) and meet at __syncwarp; one lane then adds to the counter

@@ -52,3 +52,13 @@ def test_borrowing_plan_rows_feed_the_accounting():
     assert p["n"].max() > w.C
     work = bench.algorithmic_work(w, info, p["R"], p["round"], p["n"])
     assert work["gate_up"][1] + work["down"][1] == 6 * w.T * w.k * w.d * w.F
+
+
+def test_traffic_record_ignores_comments_not_code():
+    """The recorded DRAM traffic stays attached to a kernel across edits of its comments and
+    layout, and is dropped by an edit of its code."""
+    src = 'int a = 1; // note\n/* block\n comment */ const char* s = "//kept";\n\n  char c = \'/\';\n'
+    assert bench.code_tokens(src) == 'int a = 1;\nconst char* s = "//kept";\nchar c = \'/\';'
+    reflowed = 'int   a = 1;   // another note\n  const char* s = "//kept"; // x\nchar c = \'/\';'
+    assert bench.code_tokens(reflowed) == bench.code_tokens(src)
+    assert bench.code_tokens(src.replace("a = 1", "a = 2")) != bench.code_tokens(src)
