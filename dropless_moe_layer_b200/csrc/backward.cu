@@ -1,0 +1,799 @@
+// backward.cu - backward pass of the multi-round dropless MoE layer, with per-round recompute.
+//
+// "Microsoft AI's MAI-Base-2 trained on 16K GPUs with Muon", section "Expert groups keep memory
+// fixed when tokens pile up": the backward pass recomputes each expert group on the same round
+// schedule as the forward, so its memory stays as static as the forward's. "Frontier
+// Pre-training at Microsoft AI (MAI-Base-2)", Key claims, multi-round dropless MoE item
+// [section "Scaling MoE", Fig. 6]: the backward uses fine-grained per-expert-group recompute.
+//
+// Per expert e and row x (a pair (t, j) of the round): a = W1 x, b = W3 x, s = silu(a),
+// h = s * b, out = W2 h, y[t] += gate * out. Given dy (fp32):
+//   dgate = <dy, out> = <W2^T dy, h>        dh = gate * W2^T dy
+//   db = dh * s, da = dh * b * silu'(a)     dx[t] += W1^T da + W3^T db
+//   dW2_e += (gate dy) h^T = dy (gate h)^T  dW1_e += da x^T, dW3_e += db x^T
+//   dz = softmax Jacobian applied to dgate (renormalised gates: the quotient rule first).
+//
+// Per round r, with the forward's plan (rows of expert e in round r at e * C + slot):
+//   dispatch   x rows -> xbuf, bf16(dy) rows -> dybuf, the pair's gate -> row_gate
+//   transpose  xbuf -> xT, dybuf -> dyT ([E][d][Cp], Cp = C rounded up to 128: K-major over the
+//              round's rows for the weight-gradient GEMMs;
+//              zeros past the expert's rows up to the next multiple of 64)
+//   recompute  [a | b] = xbuf W13^T (tensor cores); epilogue keeps a, b (bf16, row-major) and
+//              writes bf16(gate * h) transposed (hgT [E][F][Cp])
+//   dh         W2^T dy as dybuf (W2^T)^T (tensor cores, B = W2 transposed once per call);
+//              epilogue: the SwiGLU backward (da, db from a, b and the gate), dgate partial sums
+//              <W2^T dy, h> per 64..256-column tile, dab = [da | db] row-major and transposed
+//   dx         dab W13 (tensor cores, B = W13 transposed once per call) -> dxbuf (bf16)
+//   combine    dx[t] = (first round of t ? 0 : dx[t]) + sum of the token's dxbuf rows, ascending
+//              j; dgate[t, j] = sum of its row's partials in tile order (no atomics anywhere)
+//   wgrad      dW2 += dyT hgT^T and dW13 += dabT xT^T over K = the round's rows of each expert
+//              (tensor cores; fp32 read-add-write of the caller's gradient, one CTA per tile)
+// After the last round: dz from dgate and the logits (one warp per token).
+//
+// Every operand of a tensor-core step is bf16 (fp32 accumulate); a and b are kept as bf16 between
+// the recompute and the dh epilogue. Rows of a tile past the expert's row count never reach a
+// row-major store; in the transposed buffers they are written as zeros, so the weight-gradient
+// GEMMs may read K up to the next multiple of 64 without a mask.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <atomic>
+
+#include "copy_phases.cuh"
+#include "gemm_sm100.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace bwd {
+
+using namespace sm100;
+using gemm::BK;
+using gemm::BM;
+using gemm::Pipe;
+using gemm::Smem;
+
+enum Mode : int { kRecompute = 0, kDh = 1, kDx = 2, kWgrad = 3 };
+
+struct GemmArgs {
+  int mode;
+  int width;                  // output columns per tile (kRecompute: gate columns, MMA N = 2x)
+  const int32_t* rows;        // [E] rows of each expert in this round (the round's n)
+  int groups;                 // E
+  int m_total;                // kWgrad: output rows per expert (the M extent)
+  int n_total;                // output columns per expert
+  int num_k_blocks;           // K / 64 (all but kWgrad, whose K is the expert's rows)
+  int C, F;
+  int cpad;                   // row stride of the transposed buffers (multiple of 128, >= C)
+  void* out;                  // kRecompute: ab; kDh: dab; kDx: dxbuf; kWgrad: the fp32 gradient
+  long long out_group_stride; // elements (kWgrad)
+  int out_ld;                 // elements (kWgrad, kDx)
+  uint16_t* out_t;            // kRecompute: hgT [E][F][cpad]; kDh: dabT [E][2F][cpad]
+  const uint16_t* ab;         // kDh: [E * C][2F] a | b
+  const float* row_gate;      // kRecompute, kDh: [E * C] gate of the pair in each row
+  float* dgate_part;          // kDh: [E * C][dgate_ld] partial sums of <W2^T dy, h>
+  int dgate_ld;
+  int32_t* status;
+};
+
+__device__ __forceinline__ uint16_t bf16_bits(float v) {
+  const __nv_bfloat16 b = __float2bfloat16_rn(v);
+  return *reinterpret_cast<const uint16_t*>(&b);
+}
+
+__device__ __forceinline__ int tiles_of(const GemmArgs& p, int g, int n_tiles) {
+  const int rows = p.rows[g];
+  if (p.mode == kWgrad) return rows > 0 ? ((p.m_total + BM - 1) / BM) * n_tiles : 0;
+  return ((rows + BM - 1) / BM) * n_tiles;
+}
+
+__device__ __forceinline__ int k_blocks_of(const GemmArgs& p, int g) {
+  return p.mode == kWgrad ? (p.rows[g] + BK - 1) / BK : p.num_k_blocks;
+}
+
+// Warp 0 writes the tile prefix over the experts into s.tile_start[0].
+__device__ __forceinline__ void plan_tiles(const Smem& s, const GemmArgs& p, int n_tiles) {
+  if ((threadIdx.x >> 5) != 0) return;
+  const int lane = threadIdx.x & 31;
+  int* ts = s.tile_start[0];
+  int running = 0;
+  for (int g0 = 0; g0 < p.groups; g0 += 32) {
+    const int g = g0 + lane;
+    const int cnt = g < p.groups ? tiles_of(p, g, n_tiles) : 0;
+    int incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (g < p.groups) ts[g] = running + incl - cnt;
+    running += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) ts[p.groups] = running;
+  __syncwarp();
+}
+
+// ---------------------------------------------------------------- epilogues (one row per thread)
+
+// a, b of 32 columns: row-major bf16 into ab, and bf16(gate * silu(a) * b) transposed into hgT.
+__device__ __forceinline__ void epi_recompute(const GemmArgs& p, uint32_t tb, int g, int row, bool valid,
+                                              int nt) {
+  const long long rrow = static_cast<long long>(g) * p.C + row;
+  const float gv = valid ? p.row_gate[rrow] : 0.f;
+  uint16_t* ab = static_cast<uint16_t*>(p.out);
+  for (int c = 0; c < p.width; c += 32) {
+    uint32_t av[32], bv[32];
+    tmem_ld32(tb + c, av);
+    tmem_ld32(tb + p.width + c, bv);
+    tmem_wait_ld();
+    const int col0 = nt * p.width + c;
+    if (valid) {
+      uint32_t pa[16], pb[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        pa[i] = gemm::pack_bf16x2(__uint_as_float(av[2 * i]), __uint_as_float(av[2 * i + 1]));
+        pb[i] = gemm::pack_bf16x2(__uint_as_float(bv[2 * i]), __uint_as_float(bv[2 * i + 1]));
+      }
+      uint4* da = reinterpret_cast<uint4*>(ab + rrow * 2 * p.F + col0);
+      uint4* db = reinterpret_cast<uint4*>(ab + rrow * 2 * p.F + p.F + col0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        da[i] = make_uint4(pa[4 * i], pa[4 * i + 1], pa[4 * i + 2], pa[4 * i + 3]);
+        db[i] = make_uint4(pb[4 * i], pb[4 * i + 1], pb[4 * i + 2], pb[4 * i + 3]);
+      }
+    }
+    uint16_t* tcol = p.out_t + (static_cast<long long>(g) * p.F + col0) * p.cpad + row;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float a = __uint_as_float(av[i]), b = __uint_as_float(bv[i]);
+      tcol[static_cast<long long>(i) * p.cpad] = valid ? bf16_bits(gv * gemm::silu_f(a) * b) : uint16_t(0);
+    }
+  }
+}
+
+// The accumulator holds W2^T dy for 32-column chunks of the tile; a, b come from the recompute.
+__device__ __forceinline__ void epi_dh(const GemmArgs& p, uint32_t tb, int g, int row, bool valid, int nt) {
+  const long long rrow = static_cast<long long>(g) * p.C + row;
+  const float gv = valid ? p.row_gate[rrow] : 0.f;
+  uint16_t* dab = static_cast<uint16_t*>(p.out);
+  float part = 0.f;
+  for (int c = 0; c < p.width; c += 32) {
+    uint32_t v[32];
+    tmem_ld32(tb + c, v);
+    tmem_wait_ld();
+    const int col0 = nt * p.width + c;
+    uint16_t* tda = p.out_t + (static_cast<long long>(g) * 2 * p.F + col0) * p.cpad + row;
+    uint16_t* tdb = tda + static_cast<long long>(p.F) * p.cpad;
+    if (valid) {
+      const uint4* aq = reinterpret_cast<const uint4*>(p.ab + rrow * 2 * p.F + col0);
+      const uint4* bq = reinterpret_cast<const uint4*>(p.ab + rrow * 2 * p.F + p.F + col0);
+      uint32_t pda[16], pdb[16];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float af[8], bf[8];
+        copy::bf16x8_to_f32(aq[u], af);
+        copy::bf16x8_to_f32(bq[u], bf);
+        float dav[8], dbv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float a = af[i], b = bf[i];
+          const float dhu = __uint_as_float(v[8 * u + i]);
+          const float sig = __fdividef(1.0f, 1.0f + __expf(-a));
+          const float s = a * sig;
+          part = __fmaf_rn(dhu, s * b, part);
+          const float dh = gv * dhu;
+          dbv[i] = dh * s;
+          dav[i] = dh * b * (sig * (1.0f + a * (1.0f - sig)));
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          pda[4 * u + i] = gemm::pack_bf16x2(dav[2 * i], dav[2 * i + 1]);
+          pdb[4 * u + i] = gemm::pack_bf16x2(dbv[2 * i], dbv[2 * i + 1]);
+        }
+      }
+      uint4* oda = reinterpret_cast<uint4*>(dab + rrow * 2 * p.F + col0);
+      uint4* odb = reinterpret_cast<uint4*>(dab + rrow * 2 * p.F + p.F + col0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        oda[i] = make_uint4(pda[4 * i], pda[4 * i + 1], pda[4 * i + 2], pda[4 * i + 3]);
+        odb[i] = make_uint4(pdb[4 * i], pdb[4 * i + 1], pdb[4 * i + 2], pdb[4 * i + 3]);
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        tda[static_cast<long long>(2 * i) * p.cpad] = static_cast<uint16_t>(pda[i] & 0xFFFFu);
+        tda[static_cast<long long>(2 * i + 1) * p.cpad] = static_cast<uint16_t>(pda[i] >> 16);
+        tdb[static_cast<long long>(2 * i) * p.cpad] = static_cast<uint16_t>(pdb[i] & 0xFFFFu);
+        tdb[static_cast<long long>(2 * i + 1) * p.cpad] = static_cast<uint16_t>(pdb[i] >> 16);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        tda[static_cast<long long>(i) * p.cpad] = 0;
+        tdb[static_cast<long long>(i) * p.cpad] = 0;
+      }
+    }
+  }
+  if (valid) p.dgate_part[rrow * p.dgate_ld + nt] = part;
+}
+
+// fp32 gradient tile row: out[g][row][nt * width + c] += accumulator.
+__device__ __forceinline__ void epi_wgrad(const GemmArgs& p, uint32_t tb, int g, int row, bool valid, int nt) {
+  float* o = static_cast<float*>(p.out) + g * p.out_group_stride + static_cast<long long>(row) * p.out_ld +
+             nt * p.width;
+  for (int c = 0; c < p.width; c += 32) {
+    uint32_t v[32];
+    tmem_ld32(tb + c, v);
+    tmem_wait_ld();
+    if (valid) {
+      float4* q = reinterpret_cast<float4*>(o + c);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float4 u = q[i];
+        u.x += __uint_as_float(v[4 * i]);
+        u.y += __uint_as_float(v[4 * i + 1]);
+        u.z += __uint_as_float(v[4 * i + 2]);
+        u.w += __uint_as_float(v[4 * i + 3]);
+        q[i] = u;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- the GEMM kernel
+
+__global__ void __launch_bounds__(gemm::kThreads, 1)
+    bwd_gemm_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
+                    const GemmArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  const Smem s = gemm::carve(smem_raw);
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&ta);
+    tma_prefetch_desc(&tb);
+  }
+  const uint32_t tmem_base = gemm::setup(s);
+  const int n_tiles = p.n_total / p.width;
+  plan_tiles(s, p, n_tiles);        // reads only the round's row counts (plan data)
+  __syncthreads();
+  grid_dependency_wait();
+  pdl_trigger_early();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int* ts = s.tile_start[0];
+  const int total = ts[p.groups];
+  const int bn = p.mode == kRecompute ? 2 * p.width : p.width;
+  const int stage_bytes = gemm::kABytes + bn * BK * 2;
+  const int nstages = min(gemm::kMaxStages, gemm::kRingBytes / stage_bytes);
+  auto decode = [&](int tile, int& g, int& mt, int& nt) {
+    int lo = 0, hi = p.groups - 1;   // largest g with ts[g] <= tile
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (ts[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    g = lo;
+    const int local = tile - ts[g];
+    mt = local / n_tiles;
+    nt = local - mt * n_tiles;
+  };
+  Pipe pipe;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      const uint32_t tx = static_cast<uint32_t>(stage_bytes);
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        int g, mt, nt;
+        decode(tile, g, mt, nt);
+        const int kbs = k_blocks_of(p, g);
+        for (int kb = 0; kb < kbs; ++kb) {
+          if (!mbar_wait(smem_addr(&s.empty[pipe.stage]), pipe.phase ^ 1u, s.abort)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sA = smem_addr(s.stage + pipe.stage * stage_bytes);
+          const uint32_t sB = sA + gemm::kABytes;
+          const uint32_t fb = smem_addr(&s.full[pipe.stage]);
+          mbar_arrive_expect_tx(fb, tx);
+          tma_load_3d(sA, &ta, fb, kb * BK, mt * BM, g);
+          if (p.mode == kRecompute) {
+            tma_load_3d(sB, &tb, fb, kb * BK, nt * p.width, g);
+            tma_load_3d(sB + p.width * BK * 2, &tb, fb, kb * BK, p.F + nt * p.width, g);
+          } else {
+            tma_load_3d(sB, &tb, fb, kb * BK, nt * p.width, g);
+          }
+          pipe.issued |= 1u << pipe.stage;
+          pipe.issued_parity = (pipe.issued_parity & ~(1u << pipe.stage)) | (pipe.phase << pipe.stage);
+          if (++pipe.stage == nstages) {
+            pipe.stage = 0;
+            pipe.phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        atomicOr(p.status, kStatusTimeoutProducer);
+        *s.abort = 1;
+        for (int i = 0; i < nstages; ++i)   // let issued loads land before the CTA exits
+          if ((pipe.issued >> i) & 1u) mbar_wait(smem_addr(&s.full[i]), (pipe.issued_parity >> i) & 1u, nullptr);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      const uint32_t idesc = idesc_bf16_f32(BM, bn);
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        int g, mt, nt;
+        decode(tile, g, mt, nt);
+        const int kbs = k_blocks_of(p, g);
+        if (!mbar_wait(smem_addr(&s.tempty[pipe.acc]), pipe.acc_phase ^ 1u, s.abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(pipe.acc * gemm::kAccCols);
+        for (int kb = 0; kb < kbs; ++kb) {
+          if (!mbar_wait(smem_addr(&s.full[pipe.stage]), pipe.phase, s.abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sA = smem_addr(s.stage + pipe.stage * stage_bytes);
+          const uint64_t adesc = smem_desc_sw128(sA);
+          const uint64_t bdesc = smem_desc_sw128(sA + gemm::kABytes);
+#pragma unroll
+          for (int kk = 0; kk < BK / gemm::UMMA_K; ++kk)
+            mma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+          mma_commit(smem_addr(&s.empty[pipe.stage]));
+          if (++pipe.stage == nstages) {
+            pipe.stage = 0;
+            pipe.phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(smem_addr(&s.tfull[pipe.acc]));
+        pipe.acc ^= 1;
+        if (pipe.acc == 0) pipe.acc_phase ^= 1u;
+      }
+      if (!ok) {
+        atomicOr(p.status, kStatusTimeoutMma);
+        *s.abort = 1;
+        mma_commit(smem_addr(s.drain));   // wait for every MMA already issued
+        mbar_wait(smem_addr(s.drain), 0, nullptr);
+      }
+    }
+    __syncwarp();
+  } else {
+    // -------------------------------------------------------------- epilogue (warps 2..5)
+    const int q = warp & 3;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int g, mt, nt;
+      decode(tile, g, mt, nt);
+      const bool ready =
+          __all_sync(0xffffffffu, mbar_wait(smem_addr(&s.tfull[pipe.acc]), pipe.acc_phase, s.abort));
+      if (!ready) {
+        if (lane == 0) atomicOr(p.status, kStatusTimeoutEpilogue);
+        *s.abort = 1;
+        break;
+      }
+      tc_fence_after();
+      const int row = mt * BM + q * 32 + lane;
+      const bool valid = row < (p.mode == kWgrad ? p.m_total : p.rows[g]);
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(pipe.acc * gemm::kAccCols);
+      if (p.mode == kRecompute) {
+        epi_recompute(p, tbase, g, row, valid, nt);
+      } else if (p.mode == kDh) {
+        epi_dh(p, tbase, g, row, valid, nt);
+      } else if (p.mode == kDx) {
+        uint16_t* orow = static_cast<uint16_t*>(p.out) +
+                         (static_cast<long long>(g) * p.C + row) * p.out_ld + nt * p.width;
+        gemm::store_bf16(tbase, p.width, orow, valid);
+      } else {
+        epi_wgrad(p, tbase, g, row, valid, nt);
+      }
+      tc_fence_before();
+      mbar_arrive(smem_addr(&s.tempty[pipe.acc]));
+      pipe.acc ^= 1;
+      if (pipe.acc == 0) pipe.acc_phase ^= 1u;
+    }
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  pdl_trigger_late();
+  gemm::release_tmem(tmem_base);
+}
+
+// ---------------------------------------------------------------- copy and small kernels
+
+constexpr int kWarps = 8;
+
+// One warp per row of round r: x row -> xbuf, bf16(dy row) -> dybuf, the pair's gate -> row_gate.
+__global__ void __launch_bounds__(32 * kWarps)
+    bwd_dispatch_kernel(const uint16_t* __restrict__ x, const float* __restrict__ dy,
+                        const int32_t* __restrict__ idx, const float* __restrict__ gate,
+                        const int32_t* __restrict__ row_start, const int32_t* __restrict__ row_token,
+                        const int32_t* __restrict__ row_dst, uint16_t* __restrict__ xbuf,
+                        uint16_t* __restrict__ dybuf, float* __restrict__ row_gate, int r, int k, int C, int d) {
+  grid_dependency_wait();
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * kWarps;
+  const int begin = row_start[r], end = row_start[r + 1];
+  const int vecs = d / 8;
+  for (int row = begin + blockIdx.x * kWarps + (threadIdx.x >> 5); row < end; row += warps) {
+    const int t = row_token[row];
+    const int dst = row_dst[row];
+    const int e = dst / C;
+    const bool mine = lane < k && idx[static_cast<size_t>(t) * k + lane] == e;
+    const uint32_t hit = __ballot_sync(0xffffffffu, mine);
+    if (lane == 0 && hit) row_gate[dst] = gate[static_cast<size_t>(t) * k + (__ffs(hit) - 1)];
+    const uint4* xs = reinterpret_cast<const uint4*>(x) + static_cast<size_t>(t) * vecs;
+    uint4* xd = reinterpret_cast<uint4*>(xbuf) + static_cast<size_t>(dst) * vecs;
+    const float4* ys = reinterpret_cast<const float4*>(dy) + static_cast<size_t>(t) * (d / 4);
+    uint4* yd = reinterpret_cast<uint4*>(dybuf) + static_cast<size_t>(dst) * vecs;
+    for (int v = lane; v < vecs; v += 32) {
+      xd[v] = __ldg(xs + v);
+      const float4 lo = __ldg(ys + 2 * v), hi = __ldg(ys + 2 * v + 1);
+      yd[v] = make_uint4(gemm::pack_bf16x2(lo.x, lo.y), gemm::pack_bf16x2(lo.z, lo.w),
+                         gemm::pack_bf16x2(hi.x, hi.y), gemm::pack_bf16x2(hi.z, hi.w));
+    }
+  }
+  pdl_trigger_early();
+  pdl_trigger_late();
+}
+
+// Batched transpose of bf16 [G][R][Ccols] into [G][Ccols][Rp]: dst[g][c][r] = src[g][r][c] for
+// r < valid(g), 0 for valid(g) <= r < fill(g), nothing written past fill(g). valid(g) = R and
+// fill(g) = R without `valid_rows`; with it valid(g) = valid_rows[g] and fill(g) = valid(g)
+// rounded up to 64. A block moves one 64 x 64 tile through shared memory; Ccols, R (without
+// valid_rows) and Rp are multiples of 64. Two tensors can share the launch (blockIdx.z >= G
+// picks the second pair).
+struct TransposeArgs {
+  const uint16_t* src[2];
+  uint16_t* dst[2];
+  int G, R, Ccols, Rp;
+  const int32_t* valid_rows;   // [G] or null
+};
+
+__global__ void __launch_bounds__(256) transpose_kernel(const TransposeArgs a) {
+  __shared__ uint16_t tile[64][66];
+  grid_dependency_wait();
+  const int which = blockIdx.z >= a.G ? 1 : 0;
+  const int g = blockIdx.z - which * a.G;
+  const int c0 = blockIdx.x * 64, r0 = blockIdx.y * 64;
+  const int valid = a.valid_rows ? a.valid_rows[g] : a.R;
+  const int fill = a.valid_rows ? (valid + 63) / 64 * 64 : a.R;
+  if (r0 < fill) {
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
+    const uint16_t* src = (which ? a.src[1] : a.src[0]) + static_cast<size_t>(g) * a.R * a.Ccols;
+    uint16_t* dst = (which ? a.dst[1] : a.dst[0]) + static_cast<size_t>(g) * a.Ccols * a.Rp;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int rr = ty + 8 * i;
+      const int r = r0 + rr;
+      uint32_t v = 0;
+      if (r < valid) v = *reinterpret_cast<const uint32_t*>(src + static_cast<size_t>(r) * a.Ccols + c0 + 2 * tx);
+      tile[rr][2 * tx] = static_cast<uint16_t>(v & 0xFFFFu);
+      tile[rr][2 * tx + 1] = static_cast<uint16_t>(v >> 16);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int cc = ty + 8 * i;
+      const uint32_t v = static_cast<uint32_t>(tile[2 * tx][cc]) | (static_cast<uint32_t>(tile[2 * tx + 1][cc]) << 16);
+      *reinterpret_cast<uint32_t*>(dst + static_cast<size_t>(c0 + cc) * a.Rp + r0 + 2 * tx) = v;
+    }
+  }
+  pdl_trigger_early();
+  pdl_trigger_late();
+}
+
+// One warp per token with pairs in round r: dx[t] (+)= its pairs' dxbuf rows (gate 1, ascending j),
+// dgate[t, j] = sum over the row's `parts` partials, in order.
+__global__ void __launch_bounds__(32 * kWarps)
+    bwd_combine_kernel(const copy::CombineArgs a, int r, const float* __restrict__ dgate_part, int dgate_ld,
+                       int parts, float* __restrict__ dgate) {
+  grid_dependency_wait();
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * kWarps;
+  for (int t = blockIdx.x * kWarps + (threadIdx.x >> 5); t < a.T; t += warps) {
+    const copy::PairLoads l = copy::load_pairs(a, t);
+    const copy::TokenPairs tp = copy::token_pairs(a, l, r);
+    if (tp.npairs == 0) continue;
+    copy::accumulate_token<8>(a, t, tp);
+    const uint32_t here = __ballot_sync(0xffffffffu, l.round == r);
+    if (lane < tp.npairs) {
+      const int j = static_cast<int>(__fns(here, 0, lane + 1));
+      const float* pr = dgate_part + tp.prow * dgate_ld;
+      float sum = 0.f;
+      for (int i = 0; i < parts; ++i) sum += pr[i];
+      dgate[static_cast<size_t>(t) * a.k + j] = sum;
+    }
+  }
+  pdl_trigger_early();
+  pdl_trigger_late();
+}
+
+// One warp per token: dz[t, e] = p_e (dp_e - sum_e' p_e' dp_e'), p = softmax(z[t]) in fp32,
+// dp_e = the token's dgate of expert e (0 if not selected); with renormalised gates
+// dp_{e_j} = (dgate_j - sum_i g_i dgate_i) / sum_i p_{e_i}.
+__global__ void __launch_bounds__(32 * kWarps)
+    gate_grad_kernel(const float* __restrict__ z, const int32_t* __restrict__ idx,
+                     const float* __restrict__ dgate, int T, int E, int k, int renorm, float* __restrict__ dz) {
+  grid_dependency_wait();
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * kWarps;
+  for (int t = blockIdx.x * kWarps + (threadIdx.x >> 5); t < T; t += warps) {
+    const float* zt = z + static_cast<size_t>(t) * E;
+    float m = __int_as_float(0xff800000);   // -inf
+    for (int e = lane; e < E; e += 32) m = fmaxf(m, zt[e]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    float S = 0.f;
+    for (int e = lane; e < E; e += 32) S += __expf(zt[e] - m);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) S += __shfl_xor_sync(0xffffffffu, S, off);
+    const float invS = 1.0f / S;
+    int ej = -1;
+    float psel = 0.f, dg = 0.f;
+    if (lane < k) {
+      ej = idx[static_cast<size_t>(t) * k + lane];
+      psel = __expf(zt[ej] - m) * invS;
+      dg = dgate[static_cast<size_t>(t) * k + lane];
+    }
+    float dps = dg;
+    if (renorm) {
+      float ssel = psel;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ssel += __shfl_xor_sync(0xffffffffu, ssel, off);
+      float gd = psel * dg;           // sum_i g_i dgate_i = (sum_i p_i dgate_i) / ssel
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) gd += __shfl_xor_sync(0xffffffffu, gd, off);
+      dps = lane < k ? (dg - gd / ssel) / ssel : 0.f;
+    }
+    float c = psel * dps;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      float dpe = 0.f;
+      for (int j = 0; j < k; ++j) {
+        const int ejj = __shfl_sync(0xffffffffu, ej, j);
+        const float dpj = __shfl_sync(0xffffffffu, dps, j);
+        if (ejj == e) dpe = dpj;
+      }
+      if (e < E) dz[static_cast<size_t>(t) * E + e] = __expf(zt[e] - m) * invS * (dpe - c);
+    }
+  }
+  pdl_trigger_early();
+  pdl_trigger_late();
+}
+
+__global__ void __launch_bounds__(256) fill_kernel(float* __restrict__ p, long long n, float v) {
+  grid_dependency_wait();
+  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n; i += static_cast<long long>(gridDim.x) * 256)
+    p[i] = v;
+  pdl_trigger_early();
+  pdl_trigger_late();
+}
+
+}  // namespace bwd
+
+// ---------------------------------------------------------------- host side
+
+namespace {
+
+int grid_for(long long warps_needed) {
+  const long long blocks = (warps_needed + bwd::kWarps - 1) / bwd::kWarps;
+  const long long cap = 8ll * num_sms();
+  return static_cast<int>(blocks < 1 ? 1 : blocks < cap ? blocks : cap);
+}
+
+// Widest candidate whose tile count reaches the SM count, else the narrowest that divides n_total.
+int pick_width(const int* widths, int n_widths, long long mtiles, int n_total) {
+  int last = -1;
+  for (int i = 0; i < n_widths; ++i) {
+    if (n_total % widths[i] != 0) continue;
+    last = widths[i];
+    if (mtiles * (n_total / widths[i]) >= num_sms()) return widths[i];
+  }
+  return last;
+}
+
+cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b, const bwd::GemmArgs& args, long long tiles,
+                     cudaStream_t stream) {
+  if (tiles <= 0) return cudaSuccess;
+  static std::atomic<uint64_t> configured{0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(bwd::bwd_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
+  launch_begin(kKindBackward, stream);
+  const cudaError_t err = launch_pdl(bwd::bwd_gemm_kernel, dim3(grid), dim3(gemm::kThreads), gemm::kSmemBytes,
+                                     stream, a, b, args);
+  launch_end(kKindBackward, stream);
+  return err;
+}
+
+}  // namespace
+
+long long backward_cpad(int C) { return (C + 127) / 128 * 128ll; }
+
+cudaError_t launch_backward_prepare(const BackwardArgs& a, cudaStream_t stream) {
+  const int E = a.E, d = a.d, F = a.F;
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(a.dw_gate_up, 0, static_cast<size_t>(E) * 2 * F * d * 4, stream)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(a.dw_down, 0, static_cast<size_t>(E) * d * F * 4, stream)) != cudaSuccess) return e;
+  // W2 [E][d][F] -> W2^T [E][F][d]; W13 [E][2F][d] -> W13^T [E][d][2F]
+  bwd::TransposeArgs t1{{a.w_down, nullptr}, {a.w2t, nullptr}, E, d, F, d, nullptr};
+  launch_begin(kKindBackward, stream);
+  e = launch_pdl(bwd::transpose_kernel, dim3(F / 64, d / 64, E), dim3(256), 0, stream, t1);
+  launch_end(kKindBackward, stream);
+  if (e != cudaSuccess) return e;
+  bwd::TransposeArgs t2{{a.w_gate_up, nullptr}, {a.w13t, nullptr}, E, 2 * F, d, 2 * F, nullptr};
+  launch_begin(kKindBackward, stream);
+  e = launch_pdl(bwd::transpose_kernel, dim3(d / 64, 2 * F / 64, E), dim3(256), 0, stream, t2);
+  launch_end(kKindBackward, stream);
+  if (e != cudaSuccess) return e;
+  const long long pairs = static_cast<long long>(a.T) * a.k;
+  if (pairs > 0) {
+    launch_begin(kKindBackward, stream);
+    e = launch_pdl(bwd::fill_kernel, dim3(static_cast<unsigned>((pairs + 255) / 256 < 4096 ? (pairs + 255) / 256 : 4096)),
+                   dim3(256), 0, stream, a.ones, pairs, 1.0f);
+    launch_end(kKindBackward, stream);
+  }
+  return e;
+}
+
+cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n_host, int rows,
+                                  cudaStream_t stream) {
+  const int E = a.E, C = a.C, d = a.d, F = a.F;
+  const long long cpad = backward_cpad(C);
+  const int32_t* n_dev = a.n + static_cast<size_t>(r) * E;
+  cudaError_t e;
+  // dispatch x, dy and the gates of the round's rows
+  launch_begin(kKindBackward, stream);
+  e = launch_pdl(bwd::bwd_dispatch_kernel, dim3(grid_for(rows)), dim3(32 * bwd::kWarps), 0, stream, a.x, a.dy,
+                 a.idx, a.gate, a.row_start, a.row_token, a.row_dst, a.xbuf, a.dybuf, a.row_gate, r, a.k, C, d);
+  launch_end(kKindBackward, stream);
+  if (e != cudaSuccess) return e;
+  // xbuf, dybuf -> xT, dyT (K-major over the round's rows)
+  bwd::TransposeArgs tr{{a.xbuf, a.dybuf}, {a.xt, a.dyt}, E, C, d, static_cast<int>(cpad), n_dev};
+  launch_begin(kKindBackward, stream);
+  e = launch_pdl(bwd::transpose_kernel, dim3(d / 64, static_cast<unsigned>(cpad / 64), 2 * E), dim3(256), 0, stream,
+                 tr);
+  launch_end(kKindBackward, stream);
+  if (e != cudaSuccess) return e;
+
+  long long mt = 0;
+  int active = 0;
+  for (int g = 0; g < E; ++g) {
+    mt += (n_host[g] + gemm::BM - 1) / gemm::BM;
+    active += n_host[g] > 0 ? 1 : 0;
+  }
+  bwd::GemmArgs base{};
+  base.rows = n_dev;
+  base.groups = E;
+  base.C = C;
+  base.F = F;
+  base.cpad = static_cast<int>(cpad);
+  base.status = a.status;
+
+  // recompute: [a | b] = xbuf W13^T
+  {
+    static const int kW[3] = {128, 64, 32};
+    bwd::GemmArgs g = base;
+    g.mode = bwd::kRecompute;
+    g.width = pick_width(kW, 3, mt, F);
+    g.n_total = F;
+    g.num_k_blocks = d / gemm::BK;
+    g.out = a.ab;
+    g.out_t = a.hgt;
+    g.row_gate = a.row_gate;
+    CUtensorMap ma, mb;
+    if ((e = gemm::make_map(&ma, a.xbuf, d, C, E, gemm::BM)) != cudaSuccess) return e;
+    if ((e = gemm::make_map(&mb, a.w_gate_up, d, 2ull * F, E, static_cast<uint32_t>(g.width))) != cudaSuccess) return e;
+    if ((e = run_gemm(ma, mb, g, mt * (F / g.width), stream)) != cudaSuccess) return e;
+  }
+  // dh = W2^T dy with the SwiGLU backward in its epilogue
+  int parts = 0;
+  {
+    static const int kW[3] = {256, 128, 64};
+    bwd::GemmArgs g = base;
+    g.mode = bwd::kDh;
+    g.width = pick_width(kW, 3, mt, F);
+    parts = F / g.width;
+    g.n_total = F;
+    g.num_k_blocks = d / gemm::BK;
+    g.out = a.dab;
+    g.out_t = a.dabt;
+    g.ab = a.ab;
+    g.row_gate = a.row_gate;
+    g.dgate_part = a.dgate_part;
+    g.dgate_ld = F / 64;
+    CUtensorMap ma, mb;
+    if ((e = gemm::make_map(&ma, a.dybuf, d, C, E, gemm::BM)) != cudaSuccess) return e;
+    if ((e = gemm::make_map(&mb, a.w2t, d, F, E, static_cast<uint32_t>(g.width))) != cudaSuccess) return e;
+    if ((e = run_gemm(ma, mb, g, mt * parts, stream)) != cudaSuccess) return e;
+  }
+  // dx rows = dab W13
+  {
+    static const int kW[3] = {256, 128, 64};
+    bwd::GemmArgs g = base;
+    g.mode = bwd::kDx;
+    g.width = pick_width(kW, 3, mt, d);
+    g.n_total = d;
+    g.num_k_blocks = 2 * F / gemm::BK;
+    g.out = a.dxbuf;
+    g.out_ld = d;
+    CUtensorMap ma, mb;
+    if ((e = gemm::make_map(&ma, a.dab, 2ull * F, C, E, gemm::BM)) != cudaSuccess) return e;
+    if ((e = gemm::make_map(&mb, a.w13t, 2ull * F, d, E, static_cast<uint32_t>(g.width))) != cudaSuccess) return e;
+    if ((e = run_gemm(ma, mb, g, mt * (d / g.width), stream)) != cudaSuccess) return e;
+  }
+  // combine dx and gather dgate
+  {
+    const copy::CombineArgs ca{a.dxbuf, a.dx, a.idx, a.ones, a.round, a.slot, a.T, a.k, C, d,
+                               nullptr, nullptr, E};
+    launch_begin(kKindBackward, stream);
+    e = launch_pdl(bwd::bwd_combine_kernel, dim3(grid_for(a.T)), dim3(32 * bwd::kWarps), 0, stream, ca, r,
+                   static_cast<const float*>(a.dgate_part), F / 64, parts, a.dgate);
+    launch_end(kKindBackward, stream);
+    if (e != cudaSuccess) return e;
+  }
+  // weight gradients over K = the round's rows of each expert
+  {
+    static const int kW[3] = {256, 128, 64};
+    bwd::GemmArgs g = base;
+    g.mode = bwd::kWgrad;
+    g.m_total = d;
+    g.n_total = F;
+    g.width = pick_width(kW, 3, static_cast<long long>(active) * ((d + gemm::BM - 1) / gemm::BM), F);
+    g.out = a.dw_down;
+    g.out_group_stride = static_cast<long long>(d) * F;
+    g.out_ld = F;
+    CUtensorMap ma, mb;
+    if ((e = gemm::make_map(&ma, a.dyt, static_cast<uint64_t>(cpad), d, E, gemm::BM)) != cudaSuccess) return e;
+    if ((e = gemm::make_map(&mb, a.hgt, static_cast<uint64_t>(cpad), F, E, static_cast<uint32_t>(g.width))) !=
+        cudaSuccess)
+      return e;
+    const long long tiles = static_cast<long long>(active) * ((d + gemm::BM - 1) / gemm::BM) * (F / g.width);
+    if ((e = run_gemm(ma, mb, g, tiles, stream)) != cudaSuccess) return e;
+  }
+  {
+    static const int kW[3] = {256, 128, 64};
+    bwd::GemmArgs g = base;
+    g.mode = bwd::kWgrad;
+    g.m_total = 2 * F;
+    g.n_total = d;
+    g.width = pick_width(kW, 3, static_cast<long long>(active) * ((2 * F + gemm::BM - 1) / gemm::BM), d);
+    g.out = a.dw_gate_up;
+    g.out_group_stride = 2ll * F * d;
+    g.out_ld = d;
+    CUtensorMap ma, mb;
+    if ((e = gemm::make_map(&ma, a.dabt, static_cast<uint64_t>(cpad), 2ull * F, E, gemm::BM)) != cudaSuccess) return e;
+    if ((e = gemm::make_map(&mb, a.xt, static_cast<uint64_t>(cpad), d, E, static_cast<uint32_t>(g.width))) !=
+        cudaSuccess)
+      return e;
+    const long long tiles = static_cast<long long>(active) * ((2 * F + gemm::BM - 1) / gemm::BM) * (d / g.width);
+    if ((e = run_gemm(ma, mb, g, tiles, stream)) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_backward_gates(const BackwardArgs& a, cudaStream_t stream) {
+  if (a.T <= 0) return cudaSuccess;
+  launch_begin(kKindBackward, stream);
+  const cudaError_t e = launch_pdl(bwd::gate_grad_kernel, dim3(grid_for(a.T)), dim3(32 * bwd::kWarps), 0, stream,
+                                   a.logits, a.idx, static_cast<const float*>(a.dgate), a.T, a.E, a.k, a.renorm, a.dz);
+  launch_end(kKindBackward, stream);
+  return e;
+}
+
+}  // namespace moe

@@ -161,9 +161,9 @@ int check_device() {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-// Common checks of the calls that run a plan.
-int check_run(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
-              moe_workspace_layout_t* L) {
+// Common argument checks of the calls that run a plan (no CUDA call).
+int check_plan_args(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
+                    moe_workspace_layout_t* L) {
   int st = check_shape(shape);
   if (st != MOE_OK) return st;
   if (info == nullptr || ws == nullptr) return MOE_ERR_INVALID_ARG;
@@ -173,7 +173,14 @@ int check_run(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, s
   if (info->R < 0 || info->R > L->max_rounds) return MOE_ERR_INVALID_ARG;
   // the plan was made for this kind of plan (with or without borrowing)
   if ((info->plan_flags ^ shape->flags) & MOE_FLAG_BORROW) return MOE_ERR_INVALID_ARG;
-  return check_device();
+  return MOE_OK;
+}
+
+// The same, then the device check.
+int check_run(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
+              moe_workspace_layout_t* L) {
+  const int st = check_plan_args(shape, info, ws, ws_bytes, L);
+  return st != MOE_OK ? st : check_device();
 }
 
 bool borrowing(const moe_shape_t* s) { return (s->flags & MOE_FLAG_BORROW) != 0; }
@@ -297,9 +304,126 @@ int do_combine(const moe_shape_t* s, const moe_plan_info_t* info, void* ws, cons
                                     s->E, stream));
 }
 
+void make_backward_layout(const moe_shape_t* s, moe_backward_layout_t* L) {
+  std::memset(L, 0, sizeof(*L));
+  size_t off = 0;
+  auto take = [&](long long bytes) {
+    const size_t o = off;
+    off += (static_cast<size_t>(bytes) + 255) & ~static_cast<size_t>(255);
+    return o;
+  };
+  const long long T = s->T, E = s->E, k = s->k, C = s->C, d = s->d, F = s->d_ff;
+  const long long cpad = backward_cpad(s->C);
+  L->xbuf = take(E * C * d * 2);
+  L->dybuf = take(E * C * d * 2);
+  L->row_gate = take(E * C * 4);
+  L->xt = take(E * d * cpad * 2);
+  L->dyt = take(E * d * cpad * 2);
+  L->ab = take(E * C * 2 * F * 2);
+  L->hgt = take(E * F * cpad * 2);
+  L->dab = take(E * C * 2 * F * 2);
+  L->dabt = take(E * 2 * F * cpad * 2);
+  L->dgate_part = take(E * C * (F / 64) * 4);
+  L->dxbuf = take(E * C * d * 2);
+  L->dgate = take(T * k * 4);
+  L->ones = take(T * k * 4);
+  L->w2t = take(E * F * d * 2);
+  L->w13t = take(E * d * 2 * F * 2);
+  L->total_bytes = off;
+  L->cpad = static_cast<int32_t>(cpad);
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t moe_backward_workspace_bytes(const moe_shape_t* shape) {
+  if (check_shape(shape) != MOE_OK) return 0;
+  moe_backward_layout_t L;
+  make_backward_layout(shape, &L);
+  return L.total_bytes;
+}
+
+int moe_backward_workspace_layout(const moe_shape_t* shape, moe_backward_layout_t* layout) {
+  const int st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (layout == nullptr) return MOE_ERR_INVALID_ARG;
+  make_backward_layout(shape, layout);
+  return MOE_OK;
+}
+
+int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
+                 void* bws, size_t bws_bytes, const uint16_t* x, const uint16_t* w_gate_up,
+                 const uint16_t* w_down, const float* dy, float* dx, float* dw_gate_up, float* dw_down,
+                 float* dz, moe_stream_t stream_) {
+  moe_workspace_layout_t L;
+  int st = check_plan_args(shape, info, ws, ws_bytes, &L);
+  if (st != MOE_OK) return st;
+  if (borrowing(shape)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (bws == nullptr || w_gate_up == nullptr || w_down == nullptr || dw_gate_up == nullptr ||
+      dw_down == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (shape->T > 0 && (x == nullptr || dy == nullptr || dx == nullptr || dz == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  moe_backward_layout_t B;
+  make_backward_layout(shape, &B);
+  if (bws_bytes < B.total_bytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned(bws, 256) || !aligned(x, 16) || !aligned(w_gate_up, 16) || !aligned(w_down, 16) ||
+      !aligned(dy, 16) || !aligned(dx, 16) || !aligned(dw_gate_up, 16) || !aligned(dw_down, 16) ||
+      !aligned(dz, 16))
+    return MOE_ERR_MISALIGNED;
+  if ((st = check_device()) != MOE_OK) return st;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  BackwardArgs a{};
+  a.x = x;
+  a.w_gate_up = w_gate_up;
+  a.w_down = w_down;
+  a.dy = dy;
+  a.logits = info->logits;
+  a.idx = at<int32_t>(ws, L.topk_idx);
+  a.gate = at<float>(ws, L.gate);
+  a.round = at<int32_t>(ws, L.round);
+  a.slot = at<int32_t>(ws, L.slot);
+  a.n = at<int32_t>(ws, L.n);
+  a.row_start = at<int32_t>(ws, L.row_start);
+  a.row_token = at<int32_t>(ws, L.row_token);
+  a.row_dst = at<int32_t>(ws, L.row_dst);
+  a.dx = dx;
+  a.dw_gate_up = dw_gate_up;
+  a.dw_down = dw_down;
+  a.dz = dz;
+  a.xbuf = at<uint16_t>(bws, B.xbuf);
+  a.dybuf = at<uint16_t>(bws, B.dybuf);
+  a.row_gate = at<float>(bws, B.row_gate);
+  a.xt = at<uint16_t>(bws, B.xt);
+  a.dyt = at<uint16_t>(bws, B.dyt);
+  a.ab = at<uint16_t>(bws, B.ab);
+  a.hgt = at<uint16_t>(bws, B.hgt);
+  a.dab = at<uint16_t>(bws, B.dab);
+  a.dabt = at<uint16_t>(bws, B.dabt);
+  a.dgate_part = at<float>(bws, B.dgate_part);
+  a.dxbuf = at<uint16_t>(bws, B.dxbuf);
+  a.dgate = at<float>(bws, B.dgate);
+  a.ones = at<float>(bws, B.ones);
+  a.w2t = at<uint16_t>(bws, B.w2t);
+  a.w13t = at<uint16_t>(bws, B.w13t);
+  a.status = at<int32_t>(ws, L.header) + kHdrStatus;
+  a.T = shape->T;
+  a.k = shape->k;
+  a.E = shape->E;
+  a.C = shape->C;
+  a.d = shape->d;
+  a.F = shape->d_ff;
+  a.renorm = (shape->flags & MOE_FLAG_RENORM_TOPK) ? 1 : 0;
+  if ((st = cuda_status(launch_backward_prepare(a, stream))) != MOE_OK) return st;
+  for (int r = 0; r < info->R; ++r) {
+    int32_t n_host[MOE_MAX_EXPERTS];
+    int rows = 0;
+    round_rows(shape, info, r, n_host, &rows);
+    if ((st = cuda_status(launch_backward_round(a, r, n_host, rows, stream))) != MOE_OK) return st;
+  }
+  return cuda_status(launch_backward_gates(a, stream));
+}
 
 size_t moe_workspace_bytes(const moe_shape_t* shape) {
   if (check_shape(shape) != MOE_OK) return 0;

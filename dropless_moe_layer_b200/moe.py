@@ -16,8 +16,9 @@ from .build import LIB_PATH, ROOT
 c_i32, c_u32, c_sz, c_vp = ctypes.c_int32, ctypes.c_uint32, ctypes.c_size_t, ctypes.c_void_p
 
 MAX_EXPERTS = 256
-PROFILE_KINDS = 8
-PROFILE_NAMES = ["router_gemm", "topk", "plan", "dispatch", "gate_up", "down", "combine", "pipeline"]
+PROFILE_KINDS = 9
+PROFILE_NAMES = ["router_gemm", "topk", "plan", "dispatch", "gate_up", "down", "combine", "pipeline",
+                 "backward"]
 FLAG_RENORM_TOPK = 1
 FLAG_PER_ROUND = 2
 FLAG_PIPELINE_ALL = 4
@@ -46,6 +47,13 @@ class WorkspaceLayout(ctypes.Structure):
         "offsets", "block_base", "n", "row_off", "row_start", "row_token", "row_dst", "buf", "h", "out",
         "mb_prefix", "sync", "buf2", "h2", "out2")
     ] + [("max_rounds", c_i32), ("plan_blocks", c_i32)]
+
+
+class BackwardLayout(ctypes.Structure):
+    _fields_ = [(name, c_sz) for name in (
+        "total_bytes", "xbuf", "dybuf", "row_gate", "xt", "dyt", "ab", "hgt", "dab", "dabt",
+        "dgate_part", "dxbuf", "dgate", "ones", "w2t", "w13t")
+    ] + [("cpad", c_i32)]
 
 
 class MoeError(RuntimeError):
@@ -91,6 +99,10 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
         "moe_profile_read": (ctypes.c_int, [P(c_i32), P(ctypes.c_double)]),
         "moe_plan_noalloc": (ctypes.c_int, [P(Shape), c_vp, c_vp, c_vp, c_vp, c_vp, P(c_i32), P(c_i32), c_vp]),
+        "moe_backward_workspace_bytes": (c_sz, [P(Shape)]),
+        "moe_backward_workspace_layout": (ctypes.c_int, [P(Shape), P(BackwardLayout)]),
+        "moe_backward": (ctypes.c_int, [P(Shape), P(PlanInfo), c_vp, c_sz, c_vp, c_sz, c_vp, c_vp, c_vp,
+                                        c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -145,6 +157,25 @@ def forward(shape: Shape, info: PlanInfo, ws: int, ws_bytes: int, x: int, w_gate
             w_down: int, y: int, stream: int) -> None:
     _check("moe_forward", load_library().moe_forward(ctypes.byref(shape), ctypes.byref(info), ws, ws_bytes,
                                                      x, w_gate_up, w_down, y, stream or None))
+
+
+def backward_workspace_bytes(shape: Shape) -> int:
+    return int(load_library().moe_backward_workspace_bytes(ctypes.byref(shape)))
+
+
+def backward_layout(shape: Shape) -> BackwardLayout:
+    lay = BackwardLayout()
+    _check("moe_backward_workspace_layout",
+           load_library().moe_backward_workspace_layout(ctypes.byref(shape), ctypes.byref(lay)))
+    return lay
+
+
+def backward(shape: Shape, info: PlanInfo, ws: int, ws_bytes: int, bws: int, bws_bytes: int, x: int,
+             w_gate_up: int, w_down: int, dy: int, dx: int, dw_gate_up: int, dw_down: int, dz: int,
+             stream: int) -> None:
+    _check("moe_backward", load_library().moe_backward(ctypes.byref(shape), ctypes.byref(info), ws, ws_bytes,
+                                                       bws, bws_bytes, x, w_gate_up, w_down, dy, dx,
+                                                       dw_gate_up, dw_down, dz, stream or None))
 
 
 def _round_call(name: str, shape: Shape, info: PlanInfo, ws: int, ws_bytes: int, r: int, ptr: int,
@@ -204,7 +235,7 @@ def _need(t, dtype, shape, name):
 
 
 class DroplessMoE:
-    """A fixed-memory dropless MoE layer forward on one B200.
+    """A fixed-memory dropless MoE layer (forward, and backward with recompute) on one B200.
 
     The workspace (the layer's fixed memory) is allocated once, from the shape alone.
     `plan()` routes one batch; `forward()` runs its rounds; `__call__` does both.
@@ -262,6 +293,30 @@ class DroplessMoE:
         self.plan(logits=logits, x=x if logits is None else None, w_router=w_router, bias=bias,
                   stream=stream)
         return self.forward(x, w_gate_up, w_down, y=y, stream=stream)
+
+    def backward(self, x, w_gate_up, w_down, dy, stream=None) -> dict:
+        """Gradients of the last planned forward given dy [T, d] fp32: dx [T, d], dw_gate_up
+        [E, 2 d_ff, d], dw_down [E, d, d_ff], dz [T, E] (all fp32), recomputing each round's
+        expert activations on the forward's round schedule. The backward workspace is
+        allocated on first use (its size depends on the shape only)."""
+        import torch
+        s = self.shape
+        if self.info is None:
+            raise RuntimeError("plan() first")
+        _need(x, torch.bfloat16, (s.T, s.d), "x")
+        _need(w_gate_up, torch.bfloat16, (s.E, 2 * s.d_ff, s.d), "w_gate_up")
+        _need(w_down, torch.bfloat16, (s.E, s.d, s.d_ff), "w_down")
+        _need(dy, torch.float32, (s.T, s.d), "dy")
+        if getattr(self, "bworkspace", None) is None:
+            self.bws_bytes = backward_workspace_bytes(s)
+            self.bworkspace = torch.empty(self.bws_bytes, dtype=torch.uint8, device=self.device)
+        f32 = dict(dtype=torch.float32, device=self.device)
+        g = dict(dx=torch.empty(s.T, s.d, **f32), dw_gate_up=torch.empty(s.E, 2 * s.d_ff, s.d, **f32),
+                 dw_down=torch.empty(s.E, s.d, s.d_ff, **f32), dz=torch.empty(s.T, s.E, **f32))
+        backward(s, self.info, self.ws, self.ws_bytes, int(self.bworkspace.data_ptr()), self.bws_bytes,
+                 _ptr(x), _ptr(w_gate_up), _ptr(w_down), _ptr(dy), _ptr(g["dx"]), _ptr(g["dw_gate_up"]),
+                 _ptr(g["dw_down"]), _ptr(g["dz"]), self._stream(stream))
+        return g
 
     # -- views of the plan and of the round buffers (for checking and inspection)
     def _view(self, off: int, count: int, dtype):

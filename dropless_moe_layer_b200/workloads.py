@@ -1,4 +1,4 @@
-"""Seeded synthetic workloads for the multi-round dropless MoE layer forward.
+"""Seeded synthetic workloads for the multi-round dropless MoE layer (forward and backward).
 
 This module only draws random inputs. It holds none of the layer's arithmetic:
 no routing, no planning, no expert math. Both the CUDA path and the CPU oracle
@@ -143,6 +143,16 @@ def generate(w: Workload, device: str | torch.device = "cpu",
     out["w_gate_up"] = (_randn(gen, (w.E, 2 * w.F, w.d), device) * 0.02).to(torch.bfloat16)
     out["w_down"] = (_randn(gen, (w.E, w.d, w.F), device) * 0.02).to(torch.bfloat16)
     return out
+
+
+def generate_dy(w: Workload, device: str | torch.device = "cpu") -> torch.Tensor:
+    """The output gradient dy [T, d] fp32 of a backward pass over workload `w`: N(0, 1) drawn
+    from its own generator, seeded with the workload's seed + 1000, so that the forward inputs
+    above are the same with or without it."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed + 1000)
+    return _randn(gen, (w.T, w.d), device).contiguous()
 
 
 def bf16_bits(t: Optional[torch.Tensor]):

@@ -203,6 +203,59 @@ MOE_API int moe_round_down(const moe_shape_t* shape, const moe_plan_info_t* info
 MOE_API int moe_round_combine(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
                       size_t ws_bytes, int32_t r, float* y, moe_stream_t stream);
 
+/* ---------------------------------------------------------------- backward pass
+ *
+ * "Microsoft AI's MAI-Base-2 trained on 16K GPUs with Muon", section "Expert groups keep
+ * memory fixed when tokens pile up": the backward pass recomputes each expert group on the
+ * forward's round schedule, so its memory is as static as the forward's. moe_backward runs
+ * the R rounds of the plan in `info` again: per round it re-dispatches the round's x rows and
+ * dy rows, recomputes the SwiGLU pre-activations on the tensor cores, and adds the round's
+ * weight gradients into the caller's fp32 gradients; nothing it holds grows with the routing.
+ *
+ * Its own workspace `bws` (device, caller-owned, 256-byte aligned) holds the per-round buffers
+ * and transposed copies of the weights; its size depends on the shape only. */
+typedef struct moe_backward_layout {
+  size_t total_bytes;
+  size_t xbuf;        /* bf16 [E * C, d]     the round's x rows */
+  size_t dybuf;       /* bf16 [E * C, d]     the round's dy rows */
+  size_t row_gate;    /* f32  [E * C]        the gate of the pair in each row */
+  size_t xt;          /* bf16 [E, d, cpad]   xbuf transposed per expert (K-major over rows) */
+  size_t dyt;         /* bf16 [E, d, cpad]   dybuf transposed per expert */
+  size_t ab;          /* bf16 [E * C, 2 d_ff] recomputed a = W1 x, b = W3 x */
+  size_t hgt;         /* bf16 [E, d_ff, cpad] gate * silu(a) * b, transposed per expert */
+  size_t dab;         /* bf16 [E * C, 2 d_ff] [da | db] */
+  size_t dabt;        /* bf16 [E, 2 d_ff, cpad] [da | db] transposed per expert */
+  size_t dgate_part;  /* f32  [E * C, d_ff / 64] per-tile partial sums of dgate */
+  size_t dxbuf;       /* bf16 [E * C, d]     per-pair dx rows of the round */
+  size_t dgate;       /* f32  [T, k]         dL/dgate */
+  size_t ones;        /* f32  [T, k]         unit gates of the dx combine */
+  size_t w2t;         /* bf16 [E, d_ff, d]   W2 transposed */
+  size_t w13t;        /* bf16 [E, d, 2 d_ff] W13 transposed */
+  int32_t cpad;       /* C rounded up to a multiple of 128 */
+} moe_backward_layout_t;
+
+/* Bytes of the backward workspace for `shape` (0 for an invalid shape). */
+MOE_API size_t moe_backward_workspace_bytes(const moe_shape_t* shape);
+MOE_API int moe_backward_workspace_layout(const moe_shape_t* shape, moe_backward_layout_t* layout);
+
+/* Gradients of the layer output y (moe_forward with the same plan, inputs and weights) given
+ * dy = dL/dy:
+ *   dx         [T, d] fp32 out: through the experts (the router's share, dz W_r, is the
+ *              caller's: dz is returned for it)
+ *   dw_gate_up [E, 2*d_ff, d] fp32 out (overwritten), same row order as w_gate_up
+ *   dw_down    [E, d, d_ff] fp32 out (overwritten)
+ *   dz         [T, E] fp32 out: dL/dlogits through the softmax gates of info->logits (the
+ *              top-k selection passes no gradient)
+ * ws holds the plan (moe_plan) and is only read, except for its status word; x, w_gate_up,
+ * w_down as in moe_forward; dy [T, d] fp32. Operands of the tensor-core steps are bf16 (dy, a,
+ * b, gate * h, da, db rounded to bf16) with fp32 accumulation. Plans made with MOE_FLAG_BORROW
+ * are rejected (MOE_ERR_UNSUPPORTED_SHAPE). A bounded wait that gives up sets the status word
+ * (moe_device_status). Asynchronous: no synchronization. */
+MOE_API int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
+                         void* bws, size_t bws_bytes, const uint16_t* x, const uint16_t* w_gate_up,
+                         const uint16_t* w_down, const float* dy, float* dx, float* dw_gate_up,
+                         float* dw_down, float* dz, moe_stream_t stream);
+
 /* Synchronizes `stream` and reads the workspace status word that kernels set when a
  * bounded wait gives up. Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_CUDA. */
 MOE_API int moe_device_status(const moe_shape_t* shape, void* ws, moe_stream_t stream);
@@ -217,9 +270,10 @@ MOE_API uint64_t moe_launch_count(void);
  * is bracketed by two events on its stream; moe_profile_read() synchronizes on them and
  * reports, per kernel kind, the launch count and the summed milliseconds. Kinds:
  * 0 router GEMM, 1 top-k, 2 plan, 3 dispatch, 4 gate_up GEMM, 5 down GEMM, 6 combine,
- * 7 pipelined rounds (all four steps of its rounds in one launch).
+ * 7 pipelined rounds (all four steps of its rounds in one launch), 8 backward (every launch
+ * of moe_backward).
  * Up to 4096 launches are recorded between enable and read. Not thread-safe. */
-#define MOE_PROFILE_KINDS 8
+#define MOE_PROFILE_KINDS 9
 MOE_API int moe_profile_enable(int on);
 MOE_API int moe_profile_read(int32_t counts[MOE_PROFILE_KINDS], double ms[MOE_PROFILE_KINDS]);
 

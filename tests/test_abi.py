@@ -136,3 +136,50 @@ def test_forward_argument_errors_without_gpu(lib):
     assert lib.moe_round_combine(P(s), P(info), ws, need, 0, 4096, None) == -1
     info.plan_flags = 0
     assert lib.moe_forward(P(sb), P(info), ws, need_b, 4096, 4096, 4096, 4096, None) == -1
+
+
+def _backward_bytes_model(w):
+    """Backward workspace from its layout rules: per-round buffers of E*C rows, the transposed
+    copies with C rounded up to 128, the weights transposed once, [T, k] dgate and unit gates."""
+    def a(n):
+        return (n + 255) // 256 * 256
+    T, E, k, C, d, F = w.T, w.E, w.k, w.C, w.d, w.F
+    cp = (C + 127) // 128 * 128
+    return (3 * a(E * C * d * 2) + a(E * C * 4) + 2 * a(E * d * cp * 2) + 2 * a(E * C * 2 * F * 2)
+            + a(E * F * cp * 2) + a(E * 2 * F * cp * 2) + a(E * C * (F // 64) * 4) + 2 * a(T * k * 4)
+            + a(E * F * d * 2) + a(E * d * 2 * F * 2))
+
+
+@pytest.mark.parametrize("w", wl.WORKLOADS, ids=lambda w: w.name)
+def test_backward_workspace_is_fixed_by_shape(lib, w):
+    s = moe.make_shape(w.T, w.d, w.E, w.k, w.F, w.C)
+    n = moe.backward_workspace_bytes(s)
+    assert n == _backward_bytes_model(w)
+    lay = moe.backward_layout(s)
+    assert lay.total_bytes == n and lay.cpad % 128 == 0 and w.C <= lay.cpad < w.C + 128
+    offs = [lay.xbuf, lay.dybuf, lay.row_gate, lay.xt, lay.dyt, lay.ab, lay.hgt, lay.dab, lay.dabt,
+            lay.dgate_part, lay.dxbuf, lay.dgate, lay.ones, lay.w2t, lay.w13t]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    s.flags = 16
+    assert moe.backward_workspace_bytes(s) == 0
+
+
+def test_backward_argument_errors_without_gpu(lib):
+    s = moe.make_shape(64, 128, 8, 2, 128, 16)
+    need, bneed = moe.workspace_bytes(s), moe.backward_workspace_bytes(s)
+    info = moe.PlanInfo()
+    info.R = 1
+    P = ctypes.byref
+    ws, bws, p = 1 << 20, 1 << 24, 4096
+    f = lib.moe_backward
+    assert f(P(s), None, ws, need, bws, bneed, p, p, p, p, p, p, p, p, None) == -1
+    assert f(P(s), P(info), ws, need, None, bneed, p, p, p, p, p, p, p, p, None) == -1
+    assert f(P(s), P(info), ws, need, bws, bneed - 256, p, p, p, p, p, p, p, p, None) == -3
+    assert f(P(s), P(info), ws, need, bws + 64, bneed, p, p, p, p, p, p, p, p, None) == -4
+    assert f(P(s), P(info), ws, need, bws, bneed, p, p, p, p + 4, p, p, p, p, None) == -4
+    assert f(P(s), P(info), ws, need, bws, bneed, p, p, p, None, p, p, p, p, None) == -1
+    # plans with capacity borrowing are not supported by the backward
+    sb = moe.make_shape(64, 128, 8, 2, 128, 16, borrow=True)
+    info.plan_flags = moe.FLAG_BORROW
+    assert f(P(sb), P(info), ws, moe.workspace_bytes(sb), bws, moe.backward_workspace_bytes(sb),
+             p, p, p, p, p, p, p, p, None) == -2
