@@ -328,6 +328,120 @@ def job_throughput(tokens_per_rank, steps, world, job_ms):
     return tokens_per_rank * world * steps / (job_ms / 1e3)
 
 
+# ----------------------------------------------------------------------------- backward pass
+
+BWD_METRIC = ("routed tokens/s per MoE layer backward with per-round recompute (bf16, 1 B200); "
+              "% of tensor roofline")
+
+
+def backward_flops(w):
+    """Tensor-core work of one backward pass: per routed pair the recompute of a and b (4 d d_ff),
+    W2^T dy (2 d d_ff), dx = [da | db] W13 (4 d d_ff), dW2 (2 d d_ff) and dW1, dW3 (4 d d_ff)."""
+    return 16 * w.T * w.k * w.d * w.F
+
+
+def backward_cpu_baseline(w, budget_s=12.0):
+    """The oracle's backward on the host cores, on a seeded token sample (all the sampled tokens'
+    pairs), scaled to tokens/s."""
+    import numpy as np
+
+    import oracle
+    host = host_inputs(w)
+    z = host["logits"] if host["logits"] is not None else oracle.router_logits(host["x"], host["w_router"],
+                                                                              host["bias"])
+    dy = wl.generate_dy(w, "cpu").numpy().astype(np.float64)
+    rng = np.random.default_rng(12345)
+
+    def run(n):
+        tok = np.sort(rng.choice(w.T, size=min(n, w.T), replace=False))
+        zs = z[tok]
+        t0 = time.perf_counter()
+        oracle.backward(host["x"][tok], host["w_gate_up"], host["w_down"], zs, oracle.select_topk(zs, w.k),
+                        dy[tok])
+        return len(tok), time.perf_counter() - t0
+
+    n, dt = run(64)
+    n_tok = w.T if dt / n * w.T <= budget_s else max(64, int(budget_s / (dt / n)))
+    n, dt = run(n_tok)
+    return {"value": n / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"seeded sample of {n} of {w.T} tokens (all their top-{w.k} pairs), oracle.backward, "
+                      f"{dt:.1f} s"}
+
+
+def bench_backward(args, w):
+    import torch
+
+    from dropless_moe_layer_b200 import moe
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    moe.load_library()
+    inp = wl.generate(w, dev)
+    dy = wl.generate_dy(w, dev)
+    layer = moe.DroplessMoE(w.T, w.d, w.E, w.k, w.F, w.C, device=dev)
+    layer.plan(logits=inp["logits"], x=inp["x"] if w.router == "gemm" else None,
+               w_router=inp["w_router"], bias=inp["bias"])
+    layer.forward(inp["x"], inp["w_gate_up"], inp["w_down"])
+    info = layer.info
+    bws_bytes = moe.backward_workspace_bytes(layer.shape)
+    bws = torch.empty(bws_bytes, dtype=torch.uint8, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = dict(dx=torch.empty(w.T, w.d, **f32), dw_gate_up=torch.empty(w.E, 2 * w.F, w.d, **f32),
+             dw_down=torch.empty(w.E, w.d, w.F, **f32), dz=torch.empty(w.T, w.E, **f32))
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        moe.backward(layer.shape, info, layer.ws, layer.ws_bytes, int(bws.data_ptr()), bws_bytes,
+                     int(inp["x"].data_ptr()), int(inp["w_gate_up"].data_ptr()), int(inp["w_down"].data_ptr()),
+                     int(dy.data_ptr()), int(g["dx"].data_ptr()), int(g["dw_gate_up"].data_ptr()),
+                     int(g["dw_down"].data_ptr()), int(g["dz"].data_ptr()), int(stream.cuda_stream))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    launches0 = moe.launch_count()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    launches = moe.launch_count() - launches0
+    total_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends))
+    # one more pass with per-launch events, for the per-kernel split
+    moe.profile_enable(True)
+    flush.fill_(1)
+    step()
+    torch.cuda.synchronize(dev)
+    prof = {k: v for k, v in moe.profile_read().items() if v[0] > 0}
+    moe.profile_enable(False)
+    status = layer.device_status()
+    peaks, peak_src = load_peaks()
+    flops = backward_flops(w)
+    gemm_ms = prof["backward_gemm"][1]
+    achieved = flops / (gemm_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops"]
+    ms = total_ms / args.steps
+    line = {
+        "metric": BWD_METRIC, "pass": "backward", "value": w.T / (ms / 1e3), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w), "rounds": info.R,
+        "roofline": {"kernel": "backward_gemm", "bound": "tensor", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_src} (bf16_tflops burst)", "traffic": None,
+                     "flops_per_step": flops},
+        "whole_pass_tflops": flops / (ms / 1e3) / 1e12,
+        "kernels": {k: {"launches": c, "ms": round(t, 4)} for k, (c, t) in prof.items()},
+        "cpu_baseline": None if args.no_cpu_baseline else backward_cpu_baseline(w),
+        "gpu_launches": launches,
+        "device_status": status,
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- GPU benchmark
 
 def main():
@@ -342,9 +456,15 @@ def main():
                     help="moe_forward launch schedule (the layer's results are identical)")
     ap.add_argument("--borrow", action="store_true",
                     help="capacity borrowing between experts (fewer rounds; not the default plan)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (moe_backward) instead of the forward step; prints "
+                         "its own line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = wl.BY_NAME[args.workload]
+    if args.backward:
+        bench_backward(args, w)
+        return
     if args.impl == "reference":
         run_reference(args, w)
         return

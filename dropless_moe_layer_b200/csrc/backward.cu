@@ -614,10 +614,10 @@ cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b, const bwd::Gemm
     configured.fetch_or(bit);
   }
   const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
-  launch_begin(kKindBackward, stream);
+  launch_begin(kKindBackwardGemm, stream);
   const cudaError_t err = launch_pdl(bwd::bwd_gemm_kernel, dim3(grid), dim3(gemm::kThreads), gemm::kSmemBytes,
                                      stream, a, b, args);
-  launch_end(kKindBackward, stream);
+  launch_end(kKindBackwardGemm, stream);
   return err;
 }
 
@@ -632,21 +632,21 @@ cudaError_t launch_backward_prepare(const BackwardArgs& a, cudaStream_t stream) 
   if ((e = cudaMemsetAsync(a.dw_down, 0, static_cast<size_t>(E) * d * F * 4, stream)) != cudaSuccess) return e;
   // W2 [E][d][F] -> W2^T [E][F][d]; W13 [E][2F][d] -> W13^T [E][d][2F]
   bwd::TransposeArgs t1{{a.w_down, nullptr}, {a.w2t, nullptr}, E, d, F, d, nullptr};
-  launch_begin(kKindBackward, stream);
+  launch_begin(kKindBackwardCopy, stream);
   e = launch_pdl(bwd::transpose_kernel, dim3(F / 64, d / 64, E), dim3(256), 0, stream, t1);
-  launch_end(kKindBackward, stream);
+  launch_end(kKindBackwardCopy, stream);
   if (e != cudaSuccess) return e;
   bwd::TransposeArgs t2{{a.w_gate_up, nullptr}, {a.w13t, nullptr}, E, 2 * F, d, 2 * F, nullptr};
-  launch_begin(kKindBackward, stream);
+  launch_begin(kKindBackwardCopy, stream);
   e = launch_pdl(bwd::transpose_kernel, dim3(d / 64, 2 * F / 64, E), dim3(256), 0, stream, t2);
-  launch_end(kKindBackward, stream);
+  launch_end(kKindBackwardCopy, stream);
   if (e != cudaSuccess) return e;
   const long long pairs = static_cast<long long>(a.T) * a.k;
   if (pairs > 0) {
-    launch_begin(kKindBackward, stream);
+    launch_begin(kKindBackwardCopy, stream);
     e = launch_pdl(bwd::fill_kernel, dim3(static_cast<unsigned>((pairs + 255) / 256 < 4096 ? (pairs + 255) / 256 : 4096)),
                    dim3(256), 0, stream, a.ones, pairs, 1.0f);
-    launch_end(kKindBackward, stream);
+    launch_end(kKindBackwardCopy, stream);
   }
   return e;
 }
@@ -658,17 +658,17 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
   const int32_t* n_dev = a.n + static_cast<size_t>(r) * E;
   cudaError_t e;
   // dispatch x, dy and the gates of the round's rows
-  launch_begin(kKindBackward, stream);
+  launch_begin(kKindBackwardCopy, stream);
   e = launch_pdl(bwd::bwd_dispatch_kernel, dim3(grid_for(rows)), dim3(32 * bwd::kWarps), 0, stream, a.x, a.dy,
                  a.idx, a.gate, a.row_start, a.row_token, a.row_dst, a.xbuf, a.dybuf, a.row_gate, r, a.k, C, d);
-  launch_end(kKindBackward, stream);
+  launch_end(kKindBackwardCopy, stream);
   if (e != cudaSuccess) return e;
   // xbuf, dybuf -> xT, dyT (K-major over the round's rows)
   bwd::TransposeArgs tr{{a.xbuf, a.dybuf}, {a.xt, a.dyt}, E, C, d, static_cast<int>(cpad), n_dev};
-  launch_begin(kKindBackward, stream);
+  launch_begin(kKindBackwardCopy, stream);
   e = launch_pdl(bwd::transpose_kernel, dim3(d / 64, static_cast<unsigned>(cpad / 64), 2 * E), dim3(256), 0, stream,
                  tr);
-  launch_end(kKindBackward, stream);
+  launch_end(kKindBackwardCopy, stream);
   if (e != cudaSuccess) return e;
 
   long long mt = 0;
@@ -741,10 +741,10 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
   {
     const copy::CombineArgs ca{a.dxbuf, a.dx, a.idx, a.ones, a.round, a.slot, a.T, a.k, C, d,
                                nullptr, nullptr, E};
-    launch_begin(kKindBackward, stream);
+    launch_begin(kKindBackwardCopy, stream);
     e = launch_pdl(bwd::bwd_combine_kernel, dim3(grid_for(a.T)), dim3(32 * bwd::kWarps), 0, stream, ca, r,
                    static_cast<const float*>(a.dgate_part), F / 64, parts, a.dgate);
-    launch_end(kKindBackward, stream);
+    launch_end(kKindBackwardCopy, stream);
     if (e != cudaSuccess) return e;
   }
   // weight gradients over K = the round's rows of each expert
@@ -789,10 +789,10 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
 
 cudaError_t launch_backward_gates(const BackwardArgs& a, cudaStream_t stream) {
   if (a.T <= 0) return cudaSuccess;
-  launch_begin(kKindBackward, stream);
+  launch_begin(kKindBackwardCopy, stream);
   const cudaError_t e = launch_pdl(bwd::gate_grad_kernel, dim3(grid_for(a.T)), dim3(32 * bwd::kWarps), 0, stream,
                                    a.logits, a.idx, static_cast<const float*>(a.dgate), a.T, a.E, a.k, a.renorm, a.dz);
-  launch_end(kKindBackward, stream);
+  launch_end(kKindBackwardCopy, stream);
   return e;
 }
 

@@ -86,7 +86,8 @@ enum KernelKind : int {
   kKindDown = 5,
   kKindCombine = 6,
   kKindPipeline = 7,
-  kKindBackward = 8,
+  kKindBackwardGemm = 8,
+  kKindBackwardCopy = 9,
 };
 
 // Called around every launch (profiling and launch accounting).
