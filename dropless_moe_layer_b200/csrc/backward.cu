@@ -27,7 +27,8 @@
 //   combine    dx[t] = (first round of t ? 0 : dx[t]) + sum of the token's dxbuf rows, ascending
 //              j; dgate[t, j] = sum of its row's partials in tile order (no atomics anywhere)
 //   wgrad      dW2 += dyT hgT^T and dW13 += dabT xT^T over K = the round's rows of each expert
-//              (tensor cores; fp32 read-add-write of the caller's gradient, one CTA per tile)
+//              (tensor cores; fp32 read-add-write of the caller's gradient, one CTA per tile;
+//              round 0 stores instead: it holds every expert that has rows)
 // After the last round: dz from dgate and the logits (one warp per token).
 //
 // Every operand of a tensor-core step is bf16 (fp32 accumulate); a and b are kept as bf16 between
@@ -72,6 +73,7 @@ struct GemmArgs {
   const float* row_gate;      // kRecompute, kDh: [E * C] gate of the pair in each row
   float* dgate_part;          // kDh: [E * C][dgate_ld] partial sums of <W2^T dy, h>
   int dgate_ld;
+  int overwrite;              // kWgrad: store the tile instead of adding it (round 0)
   int32_t* status;
 };
 
@@ -215,7 +217,8 @@ __device__ __forceinline__ void epi_dh(const GemmArgs& p, uint32_t tb, int g, in
   if (valid) p.dgate_part[rrow * p.dgate_ld + nt] = part;
 }
 
-// fp32 gradient tile row: out[g][row][nt * width + c] += accumulator.
+// fp32 gradient tile row: out[g][row][nt * width + c] += accumulator (= accumulator when
+// `overwrite`: round 0, the first round of every expert that has rows at all).
 __device__ __forceinline__ void epi_wgrad(const GemmArgs& p, uint32_t tb, int g, int row, bool valid, int nt) {
   float* o = static_cast<float*>(p.out) + g * p.out_group_stride + static_cast<long long>(row) * p.out_ld +
              nt * p.width;
@@ -227,7 +230,7 @@ __device__ __forceinline__ void epi_wgrad(const GemmArgs& p, uint32_t tb, int g,
       float4* q = reinterpret_cast<float4*>(o + c);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        float4 u = q[i];
+        float4 u = p.overwrite ? make_float4(0.f, 0.f, 0.f, 0.f) : q[i];
         u.x += __uint_as_float(v[4 * i]);
         u.y += __uint_as_float(v[4 * i + 1]);
         u.z += __uint_as_float(v[4 * i + 2]);
@@ -625,11 +628,18 @@ cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b, const bwd::Gemm
 
 long long backward_cpad(int C) { return (C + 127) / 128 * 128ll; }
 
-cudaError_t launch_backward_prepare(const BackwardArgs& a, cudaStream_t stream) {
+cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_host, cudaStream_t stream) {
   const int E = a.E, d = a.d, F = a.F;
   cudaError_t e;
-  if ((e = cudaMemsetAsync(a.dw_gate_up, 0, static_cast<size_t>(E) * 2 * F * d * 4, stream)) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(a.dw_down, 0, static_cast<size_t>(E) * d * F * 4, stream)) != cudaSuccess) return e;
+  // Round 0 holds every expert that has rows at all (an expert with rows in round r > 0 has C
+  // in round 0), and its weight-gradient tiles are stored, not added: only experts without
+  // rows need zeroing.
+  const size_t per13 = static_cast<size_t>(2) * F * d, per2 = static_cast<size_t>(d) * F;
+  for (int x = 0; x < E; ++x) {
+    if (load_host[x] > 0) continue;
+    if ((e = cudaMemsetAsync(a.dw_gate_up + x * per13, 0, per13 * 4, stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(a.dw_down + x * per2, 0, per2 * 4, stream)) != cudaSuccess) return e;
+  }
   // W2 [E][d][F] -> W2^T [E][F][d]; W13 [E][2F][d] -> W13^T [E][d][2F]
   bwd::TransposeArgs t1{{a.w_down, nullptr}, {a.w2t, nullptr}, E, d, F, d, nullptr};
   launch_begin(kKindBackwardCopy, stream);
@@ -756,6 +766,7 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g.n_total = F;
     g.width = pick_width(kW, 3, static_cast<long long>(active) * ((d + gemm::BM - 1) / gemm::BM), F);
     g.out = a.dw_down;
+    g.overwrite = r == 0;
     g.out_group_stride = static_cast<long long>(d) * F;
     g.out_ld = F;
     CUtensorMap ma, mb;
@@ -774,6 +785,7 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g.n_total = d;
     g.width = pick_width(kW, 3, static_cast<long long>(active) * ((2 * F + gemm::BM - 1) / gemm::BM), d);
     g.out = a.dw_gate_up;
+    g.overwrite = r == 0;
     g.out_group_stride = 2ll * F * d;
     g.out_ld = d;
     CUtensorMap ma, mb;

@@ -245,8 +245,9 @@ struct BackwardArgs {
 };
 // Row stride of the transposed per-round buffers: C rounded up to 128 (a whole GEMM row tile).
 long long backward_cpad(int C);
-// Zeroes the weight gradients, transposes the weights, fills the unit gates.
-cudaError_t launch_backward_prepare(const BackwardArgs& a, cudaStream_t stream);
+// Zeroes the weight gradients of experts without rows (load_host: host copy of the loads),
+// transposes the weights, fills the unit gates.
+cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_host, cudaStream_t stream);
 // One round: dispatch, transposes, recompute, dh (+ SwiGLU backward), dx GEMM, dx combine and
 // dgate, weight gradients. n_host / rows: the round's rows per expert and in total.
 cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n_host, int rows,

@@ -415,7 +415,7 @@ int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws
   a.d = shape->d;
   a.F = shape->d_ff;
   a.renorm = (shape->flags & MOE_FLAG_RENORM_TOPK) ? 1 : 0;
-  if ((st = cuda_status(launch_backward_prepare(a, stream))) != MOE_OK) return st;
+  if ((st = cuda_status(launch_backward_prepare(a, info->load, stream))) != MOE_OK) return st;
   for (int r = 0; r < info->R; ++r) {
     int32_t n_host[MOE_MAX_EXPERTS];
     int rows = 0;

@@ -100,3 +100,18 @@ def test_backward_is_deterministic():
     torch.cuda.synchronize()
     for n in NAMES:
         assert torch.equal(g1[n], g2[n]), n
+
+
+def test_backward_empty_batch():
+    """No tokens: no rounds; the weight gradients are all zero."""
+    layer = moe.DroplessMoE(0, 128, 8, 2, 128, 16)
+    layer.plan(logits=torch.empty(0, 8, dtype=torch.float32, device="cuda"))
+    x = torch.empty(0, 128, dtype=torch.bfloat16, device="cuda")
+    w13 = torch.randn(8, 256, 128, device="cuda").to(torch.bfloat16)
+    w2 = torch.randn(8, 128, 128, device="cuda").to(torch.bfloat16)
+    layer.forward(x, w13, w2)
+    g = layer.backward(x, w13, w2, torch.empty(0, 128, dtype=torch.float32, device="cuda"))
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    assert g["dx"].shape == (0, 128) and g["dz"].shape == (0, 8)
+    assert torch.count_nonzero(g["dw_gate_up"]) == 0 and torch.count_nonzero(g["dw_down"]) == 0
