@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(LIB_DIR, "libmoe.so")
 
 SOURCES = ["moe_api.cu", "router.cu", "plan.cu", "dispatch_combine.cu", "grouped_gemm.cu",
            "round_pipeline.cu", "noalloc.cu", "backward.cu"]
-HEADERS = ["kernels.h", "sm100.cuh", "gemm_sm100.cuh", "copy_phases.cuh"]
+HEADERS = ["kernels.h", "backward.h", "sm100.cuh", "gemm_sm100.cuh", "copy_phases.cuh"]
 
 NVCC_FLAGS = [
     "-std=c++17", "-O3", "-lineinfo",

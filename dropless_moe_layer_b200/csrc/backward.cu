@@ -42,6 +42,7 @@
 
 #include "copy_phases.cuh"
 #include "gemm_sm100.cuh"
+#include "backward.h"
 #include "kernels.h"
 
 namespace moe {

@@ -86,8 +86,6 @@ enum KernelKind : int {
   kKindDown = 5,
   kKindCombine = 6,
   kKindPipeline = 7,
-  kKindBackwardGemm = 8,
-  kKindBackwardCopy = 9,
 };
 
 // Called around every launch (profiling and launch accounting).
@@ -202,58 +200,6 @@ struct PipelineArgs {
   int r0_dispatched;         // 1: round r0's rows are already in buf (set 0) when the launch starts
 };
 cudaError_t launch_round_pipeline(const PipelineArgs& a, cudaStream_t stream);
-
-// ---- backward with per-round recompute (backward.cu)
-// Device pointers of one backward call: the forward's plan (read only), the caller's tensors and
-// gradients, and the backward workspace's buffers (moe_backward_layout_t).
-struct BackwardArgs {
-  const uint16_t* x;          // [T, d]
-  const uint16_t* w_gate_up;  // [E, 2F, d]
-  const uint16_t* w_down;     // [E, d, F]
-  const float* dy;            // [T, d]
-  const float* logits;        // [T, E] the logits the plan used
-  const int32_t* idx;         // plan: [T, k]
-  const float* gate;          // plan: [T, k]
-  const int32_t* round;       // plan: [T, k]
-  const int32_t* slot;        // plan: [T, k]
-  const int32_t* n;           // plan: [max_rounds, E]
-  const int32_t* row_start;   // plan: [max_rounds + 1]
-  const int32_t* row_token;   // plan: round-major row list
-  const int32_t* row_dst;
-  float* dx;                  // [T, d]
-  float* dw_gate_up;          // [E, 2F, d]
-  float* dw_down;             // [E, d, F]
-  float* dz;                  // [T, E]
-  // backward workspace
-  uint16_t* xbuf;             // [E * C, d]
-  uint16_t* dybuf;            // [E * C, d]
-  float* row_gate;            // [E * C]
-  uint16_t* xt;               // [E, d, cpad]
-  uint16_t* dyt;              // [E, d, cpad]
-  uint16_t* ab;               // [E * C, 2F]
-  uint16_t* hgt;              // [E, F, cpad]
-  uint16_t* dab;              // [E * C, 2F]
-  uint16_t* dabt;             // [E, 2F, cpad]
-  float* dgate_part;          // [E * C, F / 64]
-  uint16_t* dxbuf;            // [E * C, d]
-  float* dgate;               // [T, k]
-  float* ones;                // [T, k]
-  uint16_t* w2t;              // [E, F, d]
-  uint16_t* w13t;             // [E, d, 2F]
-  int32_t* status;
-  int T, k, E, C, d, F, renorm;
-};
-// Row stride of the transposed per-round buffers: C rounded up to 128 (a whole GEMM row tile).
-long long backward_cpad(int C);
-// Zeroes the weight gradients of experts without rows (load_host: host copy of the loads),
-// transposes the weights, fills the unit gates.
-cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_host, cudaStream_t stream);
-// One round: dispatch, transposes, recompute, dh (+ SwiGLU backward), dx GEMM, dx combine and
-// dgate, weight gradients. n_host / rows: the round's rows per expert and in total.
-cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n_host, int rows,
-                                  cudaStream_t stream);
-// dz from dgate and the logits, after the last round.
-cudaError_t launch_backward_gates(const BackwardArgs& a, cudaStream_t stream);
 
 // router GEMM: logits[t][e] = x[t] . w_router[e] + bias[e] (fp32 out)
 cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* w_router, const float* bias,

@@ -13,6 +13,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "backward.h"
 #include "kernels.h"
 #include "moe.h"
 
