@@ -183,3 +183,18 @@ def test_backward_argument_errors_without_gpu(lib):
     info.plan_flags = moe.FLAG_BORROW
     assert f(P(sb), P(info), ws, moe.workspace_bytes(sb), bws, moe.backward_workspace_bytes(sb),
              p, p, p, p, p, p, p, p, None) == -2
+
+
+@pytest.mark.parametrize("cmd", [["gcc", "-std=c99", "-x", "c"], ["g++", "-std=c++11", "-x", "c++"]],
+                         ids=["c99", "c++11"])
+def test_public_header_is_plain_c(cmd):
+    """include/moe.h is a C ABI: it compiles on its own, warning-free, as C99 and as C++11."""
+    import os
+    import shutil
+    import subprocess
+    if shutil.which(cmd[0]) is None:
+        pytest.skip(f"{cmd[0]} not installed")
+    header = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe.h")
+    out = subprocess.run(cmd + ["-fsyntax-only", "-Wall", "-Wextra", "-Werror", header],
+                         capture_output=True, text=True)
+    assert out.returncode == 0, out.stderr
