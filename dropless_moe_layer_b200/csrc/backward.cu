@@ -14,10 +14,10 @@
 //   dz = softmax Jacobian applied to dgate (renormalised gates: the quotient rule first).
 //
 // Per round r, with the forward's plan (rows of expert e in round r at e * C + slot):
-//   dispatch   x rows -> xbuf, bf16(dy) rows -> dybuf, the pair's gate -> row_gate
-//   transpose  xbuf -> xT, dybuf -> dyT ([E][d][Cp], Cp = C rounded up to 128: K-major over the
-//              round's rows for the weight-gradient GEMMs;
-//              zeros past the expert's rows up to the next multiple of 64)
+//   gather     x rows -> xbuf, bf16(dy) rows -> dybuf (row-major) and, in the same pass, xT, dyT
+//              ([E][d][Cp], Cp = C rounded up to 128: K-major over the round's rows for the
+//              weight-gradient GEMMs; zeros past the expert's rows up to the next multiple of 64);
+//              the pair's gate -> row_gate
 //   recompute  [a | b] = xbuf W13^T (tensor cores); epilogue keeps a, b (bf16, row-major) and
 //              writes bf16(gate * h) transposed (hgT [E][F][Cp])
 //   dh         W2^T dy as dybuf (W2^T)^T (tensor cores, B = W2 transposed once per call);
@@ -27,6 +27,7 @@
 //   combine    dx[t] = (first round of t ? 0 : dx[t]) + sum of the token's dxbuf rows, ascending
 //              j; dgate[t, j] = sum of its row's partials in tile order (no atomics anywhere)
 //   wgrad      dW2 += dyT hgT^T and dW13 += dabT xT^T over K = the round's rows of each expert
+//              (one launch together with the dx GEMM: the three are independent)
 //              (tensor cores; fp32 read-add-write of the caller's gradient, one CTA per tile;
 //              round 0 stores instead: it holds every expert that has rows)
 // After the last round: dz from dgate and the logits (one warp per token).
@@ -93,11 +94,10 @@ __device__ __forceinline__ int k_blocks_of(const GemmArgs& p, int g) {
   return p.mode == kWgrad ? (p.rows[g] + BK - 1) / BK : p.num_k_blocks;
 }
 
-// Warp 0 writes the tile prefix over the experts into s.tile_start[0].
-__device__ __forceinline__ void plan_tiles(const Smem& s, const GemmArgs& p, int n_tiles) {
+// Warp 0 writes the tile prefix over the experts into ts[0 .. groups].
+__device__ __forceinline__ void plan_tiles(int* ts, const GemmArgs& p, int n_tiles) {
   if ((threadIdx.x >> 5) != 0) return;
   const int lane = threadIdx.x & 31;
-  int* ts = s.tile_start[0];
   int running = 0;
   for (int g0 = 0; g0 < p.groups; g0 += 32) {
     const int g = g0 + lane;
@@ -244,78 +244,113 @@ __device__ __forceinline__ void epi_wgrad(const GemmArgs& p, uint32_t tb, int g,
 
 // ---------------------------------------------------------------- the GEMM kernel
 
+// One launch runs up to three independent GEMMs ("phases") back to back over one tile list:
+// phase 0's tiles, then phase 1's, then phase 2's. All phases share one stage geometry (the
+// widest: a 128-row A tile and a 256-row B tile, 48 KB, 4 stages), because the ring's slot
+// barriers assume that a slot always covers the same bytes.
+constexpr int kMaxPhases = 3;
+constexpr int kStageBytes = gemm::kABytes + 256 * BK * 2;
+constexpr int kStages = gemm::kRingBytes / kStageBytes;
+static_assert(kStages >= 2 && kStages <= gemm::kMaxStages, "ring stages");
+constexpr int kTileStride = gemm::kMaxGroups + 1;
+// gemm::carve's layout, with room for one tile prefix per phase after the misc words.
+constexpr int kSmemBytes = 1024 + gemm::kRingBytes + gemm::kBarBytes + gemm::kMiscWords * 4 +
+                           kMaxPhases * kTileStride * 4;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+
+struct Launch {
+  GemmArgs ph[kMaxPhases];
+  int phases;
+};
+
 __global__ void __launch_bounds__(gemm::kThreads, 1)
-    bwd_gemm_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
-                    const GemmArgs p) {
+    bwd_gemm_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap tb0,
+                    const __grid_constant__ CUtensorMap ta1, const __grid_constant__ CUtensorMap tb1,
+                    const __grid_constant__ CUtensorMap ta2, const __grid_constant__ CUtensorMap tb2,
+                    const __grid_constant__ Launch L) {
   extern __shared__ uint8_t smem_raw[];
   const Smem s = gemm::carve(smem_raw);
   if (threadIdx.x == 0) {
-    tma_prefetch_desc(&ta);
-    tma_prefetch_desc(&tb);
+    tma_prefetch_desc(&ta0);
+    tma_prefetch_desc(&tb0);
   }
   const uint32_t tmem_base = gemm::setup(s);
-  const int n_tiles = p.n_total / p.width;
-  plan_tiles(s, p, n_tiles);        // reads only the round's row counts (plan data)
+  int* ts[kMaxPhases];
+  for (int q = 0; q < kMaxPhases; ++q) ts[q] = s.tile_start[0] + q * kTileStride;
+  for (int q = 0; q < L.phases; ++q)     // reads only the round's row counts (plan data)
+    plan_tiles(ts[q], L.ph[q], L.ph[q].n_total / L.ph[q].width);
   __syncthreads();
   grid_dependency_wait();
   pdl_trigger_early();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int* ts = s.tile_start[0];
-  const int total = ts[p.groups];
-  const int bn = p.mode == kRecompute ? 2 * p.width : p.width;
-  const int stage_bytes = gemm::kABytes + bn * BK * 2;
-  const int nstages = min(gemm::kMaxStages, gemm::kRingBytes / stage_bytes);
-  auto decode = [&](int tile, int& g, int& mt, int& nt) {
-    int lo = 0, hi = p.groups - 1;   // largest g with ts[g] <= tile
+  int first[kMaxPhases + 1];             // first tile of each phase in the launch's list
+  first[0] = 0;
+  for (int q = 0; q < kMaxPhases; ++q) first[q + 1] = first[q] + (q < L.phases ? ts[q][L.ph[q].groups] : 0);
+  const int total = first[L.phases];
+  auto decode = [&](int tile, int& q, int& g, int& mt, int& nt) {
+    q = 0;
+    while (q + 1 < L.phases && tile >= first[q + 1]) ++q;
+    const GemmArgs& p = L.ph[q];
+    const int* t = ts[q];
+    const int local0 = tile - first[q];
+    int lo = 0, hi = p.groups - 1;       // largest g with t[g] <= local0
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (ts[mid] <= tile) lo = mid; else hi = mid - 1;
+      if (t[mid] <= local0) lo = mid; else hi = mid - 1;
     }
     g = lo;
-    const int local = tile - ts[g];
+    const int n_tiles = p.n_total / p.width;
+    const int local = local0 - t[g];
     mt = local / n_tiles;
     nt = local - mt * n_tiles;
   };
+  auto map_a = [&](int q) { return q == 0 ? &ta0 : q == 1 ? &ta1 : &ta2; };
+  auto map_b = [&](int q) { return q == 0 ? &tb0 : q == 1 ? &tb1 : &tb2; };
+  auto bn_of = [&](const GemmArgs& p) { return p.mode == kRecompute ? 2 * p.width : p.width; };
   Pipe pipe;
+  int32_t* status = L.ph[0].status;
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA producer
-      const uint32_t tx = static_cast<uint32_t>(stage_bytes);
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-        int g, mt, nt;
-        decode(tile, g, mt, nt);
+        int q, g, mt, nt;
+        decode(tile, q, g, mt, nt);
+        const GemmArgs& p = L.ph[q];
+        const CUtensorMap* ma = map_a(q);
+        const CUtensorMap* mb = map_b(q);
+        const uint32_t tx = static_cast<uint32_t>(gemm::kABytes + bn_of(p) * BK * 2);
         const int kbs = k_blocks_of(p, g);
         for (int kb = 0; kb < kbs; ++kb) {
           if (!mbar_wait(smem_addr(&s.empty[pipe.stage]), pipe.phase ^ 1u, s.abort)) {
             ok = false;
             break;
           }
-          const uint32_t sA = smem_addr(s.stage + pipe.stage * stage_bytes);
+          const uint32_t sA = smem_addr(s.stage + pipe.stage * kStageBytes);
           const uint32_t sB = sA + gemm::kABytes;
           const uint32_t fb = smem_addr(&s.full[pipe.stage]);
           mbar_arrive_expect_tx(fb, tx);
-          tma_load_3d(sA, &ta, fb, kb * BK, mt * BM, g);
+          tma_load_3d(sA, ma, fb, kb * BK, mt * BM, g);
           if (p.mode == kRecompute) {
-            tma_load_3d(sB, &tb, fb, kb * BK, nt * p.width, g);
-            tma_load_3d(sB + p.width * BK * 2, &tb, fb, kb * BK, p.F + nt * p.width, g);
+            tma_load_3d(sB, mb, fb, kb * BK, nt * p.width, g);
+            tma_load_3d(sB + p.width * BK * 2, mb, fb, kb * BK, p.F + nt * p.width, g);
           } else {
-            tma_load_3d(sB, &tb, fb, kb * BK, nt * p.width, g);
+            tma_load_3d(sB, mb, fb, kb * BK, nt * p.width, g);
           }
           pipe.issued |= 1u << pipe.stage;
           pipe.issued_parity = (pipe.issued_parity & ~(1u << pipe.stage)) | (pipe.phase << pipe.stage);
-          if (++pipe.stage == nstages) {
+          if (++pipe.stage == kStages) {
             pipe.stage = 0;
             pipe.phase ^= 1u;
           }
         }
       }
       if (!ok) {
-        atomicOr(p.status, kStatusTimeoutProducer);
+        atomicOr(status, kStatusTimeoutProducer);
         *s.abort = 1;
-        for (int i = 0; i < nstages; ++i)   // let issued loads land before the CTA exits
+        for (int i = 0; i < kStages; ++i)   // let issued loads land before the CTA exits
           if ((pipe.issued >> i) & 1u) mbar_wait(smem_addr(&s.full[i]), (pipe.issued_parity >> i) & 1u, nullptr);
       }
     }
@@ -323,11 +358,12 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
-      const uint32_t idesc = idesc_bf16_f32(BM, bn);
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-        int g, mt, nt;
-        decode(tile, g, mt, nt);
+        int q, g, mt, nt;
+        decode(tile, q, g, mt, nt);
+        const GemmArgs& p = L.ph[q];
+        const uint32_t idesc = idesc_bf16_f32(BM, bn_of(p));
         const int kbs = k_blocks_of(p, g);
         if (!mbar_wait(smem_addr(&s.tempty[pipe.acc]), pipe.acc_phase ^ 1u, s.abort)) {
           ok = false;
@@ -341,14 +377,14 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sA = smem_addr(s.stage + pipe.stage * stage_bytes);
+          const uint32_t sA = smem_addr(s.stage + pipe.stage * kStageBytes);
           const uint64_t adesc = smem_desc_sw128(sA);
           const uint64_t bdesc = smem_desc_sw128(sA + gemm::kABytes);
 #pragma unroll
           for (int kk = 0; kk < BK / gemm::UMMA_K; ++kk)
             mma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
           mma_commit(smem_addr(&s.empty[pipe.stage]));
-          if (++pipe.stage == nstages) {
+          if (++pipe.stage == kStages) {
             pipe.stage = 0;
             pipe.phase ^= 1u;
           }
@@ -359,7 +395,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         if (pipe.acc == 0) pipe.acc_phase ^= 1u;
       }
       if (!ok) {
-        atomicOr(p.status, kStatusTimeoutMma);
+        atomicOr(status, kStatusTimeoutMma);
         *s.abort = 1;
         mma_commit(smem_addr(s.drain));   // wait for every MMA already issued
         mbar_wait(smem_addr(s.drain), 0, nullptr);
@@ -368,21 +404,22 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     __syncwarp();
   } else {
     // -------------------------------------------------------------- epilogue (warps 2..5)
-    const int q = warp & 3;
+    const int qw = warp & 3;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      int g, mt, nt;
-      decode(tile, g, mt, nt);
+      int q, g, mt, nt;
+      decode(tile, q, g, mt, nt);
+      const GemmArgs& p = L.ph[q];
       const bool ready =
           __all_sync(0xffffffffu, mbar_wait(smem_addr(&s.tfull[pipe.acc]), pipe.acc_phase, s.abort));
       if (!ready) {
-        if (lane == 0) atomicOr(p.status, kStatusTimeoutEpilogue);
+        if (lane == 0) atomicOr(status, kStatusTimeoutEpilogue);
         *s.abort = 1;
         break;
       }
       tc_fence_after();
-      const int row = mt * BM + q * 32 + lane;
+      const int row = mt * BM + qw * 32 + lane;
       const bool valid = row < (p.mode == kWgrad ? p.m_total : p.rows[g]);
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) +
                              static_cast<uint32_t>(pipe.acc * gemm::kAccCols);
       if (p.mode == kRecompute) {
         epi_recompute(p, tbase, g, row, valid, nt);
@@ -411,40 +448,6 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
 // ---------------------------------------------------------------- copy and small kernels
 
 constexpr int kWarps = 8;
-
-// One warp per row of round r: x row -> xbuf, bf16(dy row) -> dybuf, the pair's gate -> row_gate.
-__global__ void __launch_bounds__(32 * kWarps)
-    bwd_dispatch_kernel(const uint16_t* __restrict__ x, const float* __restrict__ dy,
-                        const int32_t* __restrict__ idx, const float* __restrict__ gate,
-                        const int32_t* __restrict__ row_start, const int32_t* __restrict__ row_token,
-                        const int32_t* __restrict__ row_dst, uint16_t* __restrict__ xbuf,
-                        uint16_t* __restrict__ dybuf, float* __restrict__ row_gate, int r, int k, int C, int d) {
-  grid_dependency_wait();
-  const int lane = threadIdx.x & 31;
-  const int warps = gridDim.x * kWarps;
-  const int begin = row_start[r], end = row_start[r + 1];
-  const int vecs = d / 8;
-  for (int row = begin + blockIdx.x * kWarps + (threadIdx.x >> 5); row < end; row += warps) {
-    const int t = row_token[row];
-    const int dst = row_dst[row];
-    const int e = dst / C;
-    const bool mine = lane < k && idx[static_cast<size_t>(t) * k + lane] == e;
-    const uint32_t hit = __ballot_sync(0xffffffffu, mine);
-    if (lane == 0 && hit) row_gate[dst] = gate[static_cast<size_t>(t) * k + (__ffs(hit) - 1)];
-    const uint4* xs = reinterpret_cast<const uint4*>(x) + static_cast<size_t>(t) * vecs;
-    uint4* xd = reinterpret_cast<uint4*>(xbuf) + static_cast<size_t>(dst) * vecs;
-    const float4* ys = reinterpret_cast<const float4*>(dy) + static_cast<size_t>(t) * (d / 4);
-    uint4* yd = reinterpret_cast<uint4*>(dybuf) + static_cast<size_t>(dst) * vecs;
-    for (int v = lane; v < vecs; v += 32) {
-      xd[v] = __ldg(xs + v);
-      const float4 lo = __ldg(ys + 2 * v), hi = __ldg(ys + 2 * v + 1);
-      yd[v] = make_uint4(gemm::pack_bf16x2(lo.x, lo.y), gemm::pack_bf16x2(lo.z, lo.w),
-                         gemm::pack_bf16x2(hi.x, hi.y), gemm::pack_bf16x2(hi.z, hi.w));
-    }
-  }
-  pdl_trigger_early();
-  pdl_trigger_late();
-}
 
 // Batched transpose of bf16 [G][R][Ccols] into [G][Ccols][Rp]: dst[g][c][r] = src[g][r][c] for
 // r < valid(g), 0 for valid(g) <= r < fill(g), nothing written past fill(g). valid(g) = R and
@@ -486,6 +489,85 @@ __global__ void __launch_bounds__(256) transpose_kernel(const TransposeArgs a) {
       const int cc = ty + 8 * i;
       const uint32_t v = static_cast<uint32_t>(tile[2 * tx][cc]) | (static_cast<uint32_t>(tile[2 * tx + 1][cc]) << 16);
       *reinterpret_cast<uint32_t*>(dst + static_cast<size_t>(c0 + cc) * a.Rp + r0 + 2 * tx) = v;
+    }
+  }
+  pdl_trigger_early();
+  pdl_trigger_late();
+}
+
+// Dispatch and transpose of round r in one pass. A block takes 64 rows (s0 ..) of expert e's
+// rows in the round and 64 columns (c0 ..): the rows' tokens come from the round-major row list
+// (row_off[r][e] + s), their x and dy slices are copied row-major into xbuf and dybuf (dy as
+// bf16) and, through a shared-memory tile, transposed into xT and dyT ([E][d][cpad]); rows from
+// n[r][e] up to the next multiple of 64 are zeros in the transposed copies only. The blocks of
+// the first column slice also write each row's gate.
+struct GatherArgs {
+  const uint16_t* x;
+  const float* dy;
+  const int32_t* idx;
+  const float* gate;
+  const int32_t* n;           // [max_rounds, E]
+  const int32_t* row_off;     // [max_rounds, E] first row of (round, expert) in the row list
+  const int32_t* row_token;
+  uint16_t* xbuf;
+  uint16_t* dybuf;
+  float* row_gate;
+  uint16_t* xt;
+  uint16_t* dyt;
+  int r, E, C, d, k, cpad;
+};
+
+__global__ void __launch_bounds__(256) bwd_gather_kernel(const __grid_constant__ GatherArgs a) {
+  __shared__ uint16_t tx_tile[64][66];
+  __shared__ uint16_t ty_tile[64][66];
+  __shared__ int tok[64];
+  grid_dependency_wait();
+  const int e = blockIdx.z, c0 = blockIdx.x * 64, s0 = blockIdx.y * 64;
+  const int ne = a.n[static_cast<size_t>(a.r) * a.E + e];
+  const int fill = (ne + 63) / 64 * 64;
+  if (s0 < fill) {
+    const int base = a.row_off[static_cast<size_t>(a.r) * a.E + e];
+    if (threadIdx.x < 64) {
+      const int sr = s0 + threadIdx.x;
+      tok[threadIdx.x] = sr < ne ? a.row_token[base + sr] : -1;
+    }
+    __syncthreads();
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int rr = ty + 8 * i;
+      const int t = tok[rr];
+      uint32_t xv = 0, yv = 0;
+      if (t >= 0) {
+        xv = *reinterpret_cast<const uint32_t*>(a.x + static_cast<size_t>(t) * a.d + c0 + 2 * tx);
+        const float2 dv = *reinterpret_cast<const float2*>(a.dy + static_cast<size_t>(t) * a.d + c0 + 2 * tx);
+        yv = gemm::pack_bf16x2(dv.x, dv.y);
+        const size_t orow = (static_cast<size_t>(e) * a.C + s0 + rr) * a.d + c0 + 2 * tx;
+        *reinterpret_cast<uint32_t*>(a.xbuf + orow) = xv;
+        *reinterpret_cast<uint32_t*>(a.dybuf + orow) = yv;
+      }
+      tx_tile[rr][2 * tx] = static_cast<uint16_t>(xv & 0xFFFFu);
+      tx_tile[rr][2 * tx + 1] = static_cast<uint16_t>(xv >> 16);
+      ty_tile[rr][2 * tx] = static_cast<uint16_t>(yv & 0xFFFFu);
+      ty_tile[rr][2 * tx + 1] = static_cast<uint16_t>(yv >> 16);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int cc = ty + 8 * i;
+      const size_t o = (static_cast<size_t>(e) * a.d + c0 + cc) * a.cpad + s0 + 2 * tx;
+      *reinterpret_cast<uint32_t*>(a.xt + o) =
+          static_cast<uint32_t>(tx_tile[2 * tx][cc]) | (static_cast<uint32_t>(tx_tile[2 * tx + 1][cc]) << 16);
+      *reinterpret_cast<uint32_t*>(a.dyt + o) =
+          static_cast<uint32_t>(ty_tile[2 * tx][cc]) | (static_cast<uint32_t>(ty_tile[2 * tx + 1][cc]) << 16);
+    }
+    if (c0 == 0 && threadIdx.x < 64) {
+      const int t = tok[threadIdx.x];
+      if (t >= 0) {
+        int j = 0;
+        while (j + 1 < a.k && a.idx[static_cast<size_t>(t) * a.k + j] != e) ++j;
+        a.row_gate[static_cast<size_t>(e) * a.C + s0 + threadIdx.x] = a.gate[static_cast<size_t>(t) * a.k + j];
+      }
     }
   }
   pdl_trigger_early();
@@ -604,8 +686,9 @@ int pick_width(const int* widths, int n_widths, long long mtiles, int n_total) {
   return last;
 }
 
-cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b, const bwd::GemmArgs& args, long long tiles,
-                     cudaStream_t stream) {
+// One launch of up to three GEMM phases (maps a[q], b[q], args[q]); tiles = the sum of their tiles.
+cudaError_t run_gemm(const CUtensorMap* a, const CUtensorMap* b, const bwd::GemmArgs* args, int phases,
+                     long long tiles, cudaStream_t stream) {
   if (tiles <= 0) return cudaSuccess;
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
@@ -613,14 +696,21 @@ cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b, const bwd::Gemm
   const uint64_t bit = 1ull << (dev & 63);
   if (!(configured.load() & bit)) {
     const cudaError_t e =
-        cudaFuncSetAttribute(bwd::bwd_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::kSmemBytes);
+        cudaFuncSetAttribute(bwd::bwd_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::kSmemBytes);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
+  bwd::Launch L{};
+  L.phases = phases;
+  for (int q = 0; q < phases; ++q) L.ph[q] = args[q];
+  const CUtensorMap& a1 = a[phases > 1 ? 1 : 0];
+  const CUtensorMap& b1 = b[phases > 1 ? 1 : 0];
+  const CUtensorMap& a2 = a[phases > 2 ? 2 : 0];
+  const CUtensorMap& b2 = b[phases > 2 ? 2 : 0];
   const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
   launch_begin(kKindBackwardGemm, stream);
-  const cudaError_t err = launch_pdl(bwd::bwd_gemm_kernel, dim3(grid), dim3(gemm::kThreads), gemm::kSmemBytes,
-                                     stream, a, b, args);
+  const cudaError_t err = launch_pdl(bwd::bwd_gemm_kernel, dim3(grid), dim3(gemm::kThreads), bwd::kSmemBytes,
+                                     stream, a[0], b[0], a1, b1, a2, b2, L);
   launch_end(kKindBackwardGemm, stream);
   return err;
 }
@@ -664,23 +754,21 @@ cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_h
 
 cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n_host, int rows,
                                   cudaStream_t stream) {
+  (void)rows;
   const int E = a.E, C = a.C, d = a.d, F = a.F;
   const long long cpad = backward_cpad(C);
   const int32_t* n_dev = a.n + static_cast<size_t>(r) * E;
   cudaError_t e;
-  // dispatch x, dy and the gates of the round's rows
-  launch_begin(kKindBackwardCopy, stream);
-  e = launch_pdl(bwd::bwd_dispatch_kernel, dim3(grid_for(rows)), dim3(32 * bwd::kWarps), 0, stream, a.x, a.dy,
-                 a.idx, a.gate, a.row_start, a.row_token, a.row_dst, a.xbuf, a.dybuf, a.row_gate, r, a.k, C, d);
-  launch_end(kKindBackwardCopy, stream);
-  if (e != cudaSuccess) return e;
-  // xbuf, dybuf -> xT, dyT (K-major over the round's rows)
-  bwd::TransposeArgs tr{{a.xbuf, a.dybuf}, {a.xt, a.dyt}, E, C, d, static_cast<int>(cpad), n_dev};
-  launch_begin(kKindBackwardCopy, stream);
-  e = launch_pdl(bwd::transpose_kernel, dim3(d / 64, static_cast<unsigned>(cpad / 64), 2 * E), dim3(256), 0, stream,
-                 tr);
-  launch_end(kKindBackwardCopy, stream);
-  if (e != cudaSuccess) return e;
+  // dispatch and transpose x, dy; the rows' gates
+  {
+    const bwd::GatherArgs ga{a.x, a.dy, a.idx, a.gate, a.n, a.row_off, a.row_token, a.xbuf, a.dybuf,
+                             a.row_gate, a.xt, a.dyt, r, E, C, d, a.k, static_cast<int>(cpad)};
+    launch_begin(kKindBackwardCopy, stream);
+    e = launch_pdl(bwd::bwd_gather_kernel, dim3(d / 64, static_cast<unsigned>(cpad / 64), E), dim3(256), 0, stream,
+                   ga);
+    launch_end(kKindBackwardCopy, stream);
+    if (e != cudaSuccess) return e;
+  }
 
   long long mt = 0;
   int active = 0;
@@ -695,6 +783,7 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
   base.F = F;
   base.cpad = static_cast<int>(cpad);
   base.status = a.status;
+  static const int kWide[3] = {256, 128, 64};
 
   // recompute: [a | b] = xbuf W13^T
   {
@@ -710,15 +799,14 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     CUtensorMap ma, mb;
     if ((e = gemm::make_map(&ma, a.xbuf, d, C, E, gemm::BM)) != cudaSuccess) return e;
     if ((e = gemm::make_map(&mb, a.w_gate_up, d, 2ull * F, E, static_cast<uint32_t>(g.width))) != cudaSuccess) return e;
-    if ((e = run_gemm(ma, mb, g, mt * (F / g.width), stream)) != cudaSuccess) return e;
+    if ((e = run_gemm(&ma, &mb, &g, 1, mt * (F / g.width), stream)) != cudaSuccess) return e;
   }
   // dh = W2^T dy with the SwiGLU backward in its epilogue
   int parts = 0;
   {
-    static const int kW[3] = {256, 128, 64};
     bwd::GemmArgs g = base;
     g.mode = bwd::kDh;
-    g.width = pick_width(kW, 3, mt, F);
+    g.width = pick_width(kWide, 3, mt, F);
     parts = F / g.width;
     g.n_total = F;
     g.num_k_blocks = d / gemm::BK;
@@ -731,22 +819,53 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     CUtensorMap ma, mb;
     if ((e = gemm::make_map(&ma, a.dybuf, d, C, E, gemm::BM)) != cudaSuccess) return e;
     if ((e = gemm::make_map(&mb, a.w2t, d, F, E, static_cast<uint32_t>(g.width))) != cudaSuccess) return e;
-    if ((e = run_gemm(ma, mb, g, mt * parts, stream)) != cudaSuccess) return e;
+    if ((e = run_gemm(&ma, &mb, &g, 1, mt * parts, stream)) != cudaSuccess) return e;
   }
-  // dx rows = dab W13
+  // one launch: dx rows = dab W13, dW2 (+)= dyT hgT^T, dW13 (+)= dabT xT^T (K = the round's rows)
   {
-    static const int kW[3] = {256, 128, 64};
-    bwd::GemmArgs g = base;
-    g.mode = bwd::kDx;
-    g.width = pick_width(kW, 3, mt, d);
-    g.n_total = d;
-    g.num_k_blocks = 2 * F / gemm::BK;
-    g.out = a.dxbuf;
-    g.out_ld = d;
-    CUtensorMap ma, mb;
-    if ((e = gemm::make_map(&ma, a.dab, 2ull * F, C, E, gemm::BM)) != cudaSuccess) return e;
-    if ((e = gemm::make_map(&mb, a.w13t, 2ull * F, d, E, static_cast<uint32_t>(g.width))) != cudaSuccess) return e;
-    if ((e = run_gemm(ma, mb, g, mt * (d / g.width), stream)) != cudaSuccess) return e;
+    bwd::GemmArgs g[3] = {base, base, base};
+    CUtensorMap ma[3], mb[3];
+    long long tiles = 0;
+    g[0].mode = bwd::kDx;
+    g[0].width = pick_width(kWide, 3, mt, d);
+    g[0].n_total = d;
+    g[0].num_k_blocks = 2 * F / gemm::BK;
+    g[0].out = a.dxbuf;
+    g[0].out_ld = d;
+    if ((e = gemm::make_map(&ma[0], a.dab, 2ull * F, C, E, gemm::BM)) != cudaSuccess) return e;
+    if ((e = gemm::make_map(&mb[0], a.w13t, 2ull * F, d, E, static_cast<uint32_t>(g[0].width))) != cudaSuccess)
+      return e;
+    tiles += mt * (d / g[0].width);
+    const long long mt_w2 = static_cast<long long>(active) * ((d + gemm::BM - 1) / gemm::BM);
+    const long long mt_w13 = static_cast<long long>(active) * ((2 * F + gemm::BM - 1) / gemm::BM);
+    g[1].mode = bwd::kWgrad;
+    g[1].m_total = d;
+    g[1].n_total = F;
+    g[1].width = pick_width(kWide, 3, mt_w2, F);
+    g[1].out = a.dw_down;
+    g[1].overwrite = r == 0;
+    g[1].out_group_stride = static_cast<long long>(d) * F;
+    g[1].out_ld = F;
+    if ((e = gemm::make_map(&ma[1], a.dyt, static_cast<uint64_t>(cpad), d, E, gemm::BM)) != cudaSuccess) return e;
+    if ((e = gemm::make_map(&mb[1], a.hgt, static_cast<uint64_t>(cpad), F, E, static_cast<uint32_t>(g[1].width))) !=
+        cudaSuccess)
+      return e;
+    tiles += mt_w2 * (F / g[1].width);
+    g[2].mode = bwd::kWgrad;
+    g[2].m_total = 2 * F;
+    g[2].n_total = d;
+    g[2].width = pick_width(kWide, 3, mt_w13, d);
+    g[2].out = a.dw_gate_up;
+    g[2].overwrite = r == 0;
+    g[2].out_group_stride = 2ll * F * d;
+    g[2].out_ld = d;
+    if ((e = gemm::make_map(&ma[2], a.dabt, static_cast<uint64_t>(cpad), 2ull * F, E, gemm::BM)) != cudaSuccess)
+      return e;
+    if ((e = gemm::make_map(&mb[2], a.xt, static_cast<uint64_t>(cpad), d, E, static_cast<uint32_t>(g[2].width))) !=
+        cudaSuccess)
+      return e;
+    tiles += mt_w13 * (d / g[2].width);
+    if ((e = run_gemm(ma, mb, g, 3, tiles, stream)) != cudaSuccess) return e;
   }
   // combine dx and gather dgate
   {
@@ -756,48 +875,8 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     e = launch_pdl(bwd::bwd_combine_kernel, dim3(grid_for(a.T)), dim3(32 * bwd::kWarps), 0, stream, ca, r,
                    static_cast<const float*>(a.dgate_part), F / 64, parts, a.dgate);
     launch_end(kKindBackwardCopy, stream);
-    if (e != cudaSuccess) return e;
   }
-  // weight gradients over K = the round's rows of each expert
-  {
-    static const int kW[3] = {256, 128, 64};
-    bwd::GemmArgs g = base;
-    g.mode = bwd::kWgrad;
-    g.m_total = d;
-    g.n_total = F;
-    g.width = pick_width(kW, 3, static_cast<long long>(active) * ((d + gemm::BM - 1) / gemm::BM), F);
-    g.out = a.dw_down;
-    g.overwrite = r == 0;
-    g.out_group_stride = static_cast<long long>(d) * F;
-    g.out_ld = F;
-    CUtensorMap ma, mb;
-    if ((e = gemm::make_map(&ma, a.dyt, static_cast<uint64_t>(cpad), d, E, gemm::BM)) != cudaSuccess) return e;
-    if ((e = gemm::make_map(&mb, a.hgt, static_cast<uint64_t>(cpad), F, E, static_cast<uint32_t>(g.width))) !=
-        cudaSuccess)
-      return e;
-    const long long tiles = static_cast<long long>(active) * ((d + gemm::BM - 1) / gemm::BM) * (F / g.width);
-    if ((e = run_gemm(ma, mb, g, tiles, stream)) != cudaSuccess) return e;
-  }
-  {
-    static const int kW[3] = {256, 128, 64};
-    bwd::GemmArgs g = base;
-    g.mode = bwd::kWgrad;
-    g.m_total = 2 * F;
-    g.n_total = d;
-    g.width = pick_width(kW, 3, static_cast<long long>(active) * ((2 * F + gemm::BM - 1) / gemm::BM), d);
-    g.out = a.dw_gate_up;
-    g.overwrite = r == 0;
-    g.out_group_stride = 2ll * F * d;
-    g.out_ld = d;
-    CUtensorMap ma, mb;
-    if ((e = gemm::make_map(&ma, a.dabt, static_cast<uint64_t>(cpad), 2ull * F, E, gemm::BM)) != cudaSuccess) return e;
-    if ((e = gemm::make_map(&mb, a.xt, static_cast<uint64_t>(cpad), d, E, static_cast<uint32_t>(g.width))) !=
-        cudaSuccess)
-      return e;
-    const long long tiles = static_cast<long long>(active) * ((2 * F + gemm::BM - 1) / gemm::BM) * (d / g.width);
-    if ((e = run_gemm(ma, mb, g, tiles, stream)) != cudaSuccess) return e;
-  }
-  return cudaSuccess;
+  return e;
 }
 
 cudaError_t launch_backward_gates(const BackwardArgs& a, cudaStream_t stream) {

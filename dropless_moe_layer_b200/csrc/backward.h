@@ -29,6 +29,7 @@ struct BackwardArgs {
   const int32_t* slot;        // plan: [T, k]
   const int32_t* n;           // plan: [max_rounds, E]
   const int32_t* row_start;   // plan: [max_rounds + 1]
+  const int32_t* row_off;     // plan: [max_rounds, E] first row of (round, expert) in the row list
   const int32_t* row_token;   // plan: round-major row list
   const int32_t* row_dst;
   float* dx;                  // [T, d]

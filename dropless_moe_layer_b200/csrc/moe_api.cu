@@ -387,6 +387,7 @@ int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws
   a.slot = at<int32_t>(ws, L.slot);
   a.n = at<int32_t>(ws, L.n);
   a.row_start = at<int32_t>(ws, L.row_start);
+  a.row_off = at<int32_t>(ws, L.row_off);
   a.row_token = at<int32_t>(ws, L.row_token);
   a.row_dst = at<int32_t>(ws, L.row_dst);
   a.dx = dx;
