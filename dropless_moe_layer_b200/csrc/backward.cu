@@ -66,11 +66,18 @@ struct GemmArgs {
   int n_total;                // output columns per expert
   int num_k_blocks;           // K / 64 (all but kWgrad, whose K is the expert's rows)
   int C, F;
-  int cpad;                   // row stride of the transposed buffers (multiple of 128, >= C)
+  int t_ld;                   // elements per row of the transposed buffers: C rounded up to 128
+                              // per expert, or the pooled width with capacity borrowing
+  // Pooled round rows (capacity borrowing): expert g's rows of the round start at row
+  // group_row[g] - *group_row_base of the E*C-row buffers, and at column seg(g) = sum over
+  // g' < g of rows(g') rounded up to 64 of the single [rows_t][t_ld] transposed buffers. Null:
+  // rows at g * C, transposed buffers per expert ([E][rows_t][t_ld]).
+  const int32_t* group_row;
+  const int32_t* group_row_base;
   void* out;                  // kRecompute: ab; kDh: dab; kDx: dxbuf; kWgrad: the fp32 gradient
   long long out_group_stride; // elements (kWgrad)
   int out_ld;                 // elements (kWgrad, kDx)
-  uint16_t* out_t;            // kRecompute: hgT [E][F][cpad]; kDh: dabT [E][2F][cpad]
+  uint16_t* out_t;            // kRecompute: hgT (F rows); kDh: dabT (2F rows)
   const uint16_t* ab;         // kDh: [E * C][2F] a | b
   const float* row_gate;      // kRecompute, kDh: [E * C] gate of the pair in each row
   float* dgate_part;          // kDh: [E * C][dgate_ld] partial sums of <W2^T dy, h>
@@ -94,33 +101,57 @@ __device__ __forceinline__ int k_blocks_of(const GemmArgs& p, int g) {
   return p.mode == kWgrad ? (p.rows[g] + BK - 1) / BK : p.num_k_blocks;
 }
 
-// Warp 0 writes the tile prefix over the experts into ts[0 .. groups].
-__device__ __forceinline__ void plan_tiles(int* ts, const GemmArgs& p, int n_tiles) {
-  if ((threadIdx.x >> 5) != 0) return;
+// Exclusive prefix over the experts of cnt(g), written to out[0 .. groups] by warp 0.
+template <typename Count>
+__device__ __forceinline__ void warp_prefix(int* out, int groups, Count cnt_of) {
   const int lane = threadIdx.x & 31;
   int running = 0;
-  for (int g0 = 0; g0 < p.groups; g0 += 32) {
+  for (int g0 = 0; g0 < groups; g0 += 32) {
     const int g = g0 + lane;
-    const int cnt = g < p.groups ? tiles_of(p, g, n_tiles) : 0;
+    const int cnt = g < groups ? cnt_of(g) : 0;
     int incl = cnt;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int o = __shfl_up_sync(0xffffffffu, incl, off);
       if (lane >= off) incl += o;
     }
-    if (g < p.groups) ts[g] = running + incl - cnt;
+    if (g < groups) out[g] = running + incl - cnt;
     running += __shfl_sync(0xffffffffu, incl, 31);
   }
-  if (lane == 0) ts[p.groups] = running;
+  if (lane == 0) out[groups] = running;
   __syncwarp();
+}
+
+// Warp 0 writes the tile prefix over the experts into ts[0 .. groups] and, for pooled rows, the
+// experts' first columns in the transposed buffers into seg[0 .. groups].
+__device__ __forceinline__ void plan_tiles(int* ts, int* seg, const GemmArgs& p, int n_tiles) {
+  if ((threadIdx.x >> 5) != 0) return;
+  warp_prefix(ts, p.groups, [&](int g) { return tiles_of(p, g, n_tiles); });
+  if (p.group_row) warp_prefix(seg, p.groups, [&](int g) { return (p.rows[g] + BK - 1) / BK * BK; });
+}
+
+// Row of expert g's row `row` in the E*C-row buffers.
+__device__ __forceinline__ long long row_of(const GemmArgs& p, int g, int row) {
+  return p.group_row ? static_cast<long long>(p.group_row[g] - *p.group_row_base) + row
+                     : static_cast<long long>(g) * p.C + row;
+}
+
+// Element (r, c) of expert g's part of a transposed buffer with rows_t rows: c is the expert's row.
+__device__ __forceinline__ long long t_index(const GemmArgs& p, const int* seg, int g, int rows_t, int r,
+                                             int c) {
+  return p.group_row ? static_cast<long long>(r) * p.t_ld + seg[g] + c
+                     : (static_cast<long long>(g) * rows_t + r) * p.t_ld + c;
 }
 
 // ---------------------------------------------------------------- epilogues (one row per thread)
 
 // a, b of 32 columns: row-major bf16 into ab, and bf16(gate * silu(a) * b) transposed into hgT.
-__device__ __forceinline__ void epi_recompute(const GemmArgs& p, uint32_t tb, int g, int row, bool valid,
-                                              int nt) {
-  const long long rrow = static_cast<long long>(g) * p.C + row;
+__device__ __forceinline__ void epi_recompute(const GemmArgs& p, const int* seg, uint32_t tb, int g, int row,
+                                              bool valid, int nt) {
+  const long long rrow = row_of(p, g, row);
+  // transposed rows are written up to the expert's rows rounded up to 64 (zeros past them): the
+  // weight-gradient GEMMs read K in blocks of 64, and with pooled rows the next expert follows
+  const bool in_t = row < (p.rows[g] + BK - 1) / BK * BK;
   const float gv = valid ? p.row_gate[rrow] : 0.f;
   uint16_t* ab = static_cast<uint16_t*>(p.out);
   for (int c = 0; c < p.width; c += 32) {
@@ -144,18 +175,22 @@ __device__ __forceinline__ void epi_recompute(const GemmArgs& p, uint32_t tb, in
         db[i] = make_uint4(pb[4 * i], pb[4 * i + 1], pb[4 * i + 2], pb[4 * i + 3]);
       }
     }
-    uint16_t* tcol = p.out_t + (static_cast<long long>(g) * p.F + col0) * p.cpad + row;
+    if (in_t) {
+      uint16_t* tcol = p.out_t + t_index(p, seg, g, p.F, col0, row);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float a = __uint_as_float(av[i]), b = __uint_as_float(bv[i]);
-      tcol[static_cast<long long>(i) * p.cpad] = valid ? bf16_bits(gv * gemm::silu_f(a) * b) : uint16_t(0);
+      for (int i = 0; i < 32; ++i) {
+        const float a = __uint_as_float(av[i]), b = __uint_as_float(bv[i]);
+        tcol[static_cast<long long>(i) * p.t_ld] = valid ? bf16_bits(gv * gemm::silu_f(a) * b) : uint16_t(0);
+      }
     }
   }
 }
 
 // The accumulator holds W2^T dy for 32-column chunks of the tile; a, b come from the recompute.
-__device__ __forceinline__ void epi_dh(const GemmArgs& p, uint32_t tb, int g, int row, bool valid, int nt) {
-  const long long rrow = static_cast<long long>(g) * p.C + row;
+__device__ __forceinline__ void epi_dh(const GemmArgs& p, const int* seg, uint32_t tb, int g, int row, bool valid,
+                                       int nt) {
+  const long long rrow = row_of(p, g, row);
+  const bool in_t = row < (p.rows[g] + BK - 1) / BK * BK;
   const float gv = valid ? p.row_gate[rrow] : 0.f;
   uint16_t* dab = static_cast<uint16_t*>(p.out);
   float part = 0.f;
@@ -164,8 +199,8 @@ __device__ __forceinline__ void epi_dh(const GemmArgs& p, uint32_t tb, int g, in
     tmem_ld32(tb + c, v);
     tmem_wait_ld();
     const int col0 = nt * p.width + c;
-    uint16_t* tda = p.out_t + (static_cast<long long>(g) * 2 * p.F + col0) * p.cpad + row;
-    uint16_t* tdb = tda + static_cast<long long>(p.F) * p.cpad;
+    uint16_t* tda = p.out_t + t_index(p, seg, g, 2 * p.F, col0, row);
+    uint16_t* tdb = tda + static_cast<long long>(p.F) * p.t_ld;
     if (valid) {
       const uint4* aq = reinterpret_cast<const uint4*>(p.ab + rrow * 2 * p.F + col0);
       const uint4* bq = reinterpret_cast<const uint4*>(p.ab + rrow * 2 * p.F + p.F + col0);
@@ -202,16 +237,16 @@ __device__ __forceinline__ void epi_dh(const GemmArgs& p, uint32_t tb, int g, in
       }
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        tda[static_cast<long long>(2 * i) * p.cpad] = static_cast<uint16_t>(pda[i] & 0xFFFFu);
-        tda[static_cast<long long>(2 * i + 1) * p.cpad] = static_cast<uint16_t>(pda[i] >> 16);
-        tdb[static_cast<long long>(2 * i) * p.cpad] = static_cast<uint16_t>(pdb[i] & 0xFFFFu);
-        tdb[static_cast<long long>(2 * i + 1) * p.cpad] = static_cast<uint16_t>(pdb[i] >> 16);
+        tda[static_cast<long long>(2 * i) * p.t_ld] = static_cast<uint16_t>(pda[i] & 0xFFFFu);
+        tda[static_cast<long long>(2 * i + 1) * p.t_ld] = static_cast<uint16_t>(pda[i] >> 16);
+        tdb[static_cast<long long>(2 * i) * p.t_ld] = static_cast<uint16_t>(pdb[i] & 0xFFFFu);
+        tdb[static_cast<long long>(2 * i + 1) * p.t_ld] = static_cast<uint16_t>(pdb[i] >> 16);
       }
-    } else {
+    } else if (in_t) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        tda[static_cast<long long>(i) * p.cpad] = 0;
-        tdb[static_cast<long long>(i) * p.cpad] = 0;
+        tda[static_cast<long long>(i) * p.t_ld] = 0;
+        tdb[static_cast<long long>(i) * p.t_ld] = 0;
       }
     }
   }
@@ -253,9 +288,10 @@ constexpr int kStageBytes = gemm::kABytes + 256 * BK * 2;
 constexpr int kStages = gemm::kRingBytes / kStageBytes;
 static_assert(kStages >= 2 && kStages <= gemm::kMaxStages, "ring stages");
 constexpr int kTileStride = gemm::kMaxGroups + 1;
-// gemm::carve's layout, with room for one tile prefix per phase after the misc words.
+// gemm::carve's layout, with room for a tile prefix and a pooled-column prefix per phase after
+// the misc words.
 constexpr int kSmemBytes = 1024 + gemm::kRingBytes + gemm::kBarBytes + gemm::kMiscWords * 4 +
-                           kMaxPhases * kTileStride * 4;
+                           2 * kMaxPhases * kTileStride * 4;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 struct Launch {
@@ -276,9 +312,13 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   }
   const uint32_t tmem_base = gemm::setup(s);
   int* ts[kMaxPhases];
-  for (int q = 0; q < kMaxPhases; ++q) ts[q] = s.tile_start[0] + q * kTileStride;
+  int* seg[kMaxPhases];
+  for (int q = 0; q < kMaxPhases; ++q) {
+    ts[q] = s.tile_start[0] + q * kTileStride;
+    seg[q] = s.tile_start[0] + (kMaxPhases + q) * kTileStride;
+  }
   for (int q = 0; q < L.phases; ++q)     // reads only the round's row counts (plan data)
-    plan_tiles(ts[q], L.ph[q], L.ph[q].n_total / L.ph[q].width);
+    plan_tiles(ts[q], seg[q], L.ph[q], L.ph[q].n_total / L.ph[q].width);
   __syncthreads();
   grid_dependency_wait();
   pdl_trigger_early();
@@ -332,12 +372,22 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           const uint32_t sB = sA + gemm::kABytes;
           const uint32_t fb = smem_addr(&s.full[pipe.stage]);
           mbar_arrive_expect_tx(fb, tx);
-          tma_load_3d(sA, ma, fb, kb * BK, mt * BM, g);
-          if (p.mode == kRecompute) {
-            tma_load_3d(sB, mb, fb, kb * BK, nt * p.width, g);
-            tma_load_3d(sB + p.width * BK * 2, mb, fb, kb * BK, p.F + nt * p.width, g);
+          if (p.mode == kWgrad) {
+            // both operands are transposed buffers, K = the expert's rows: per expert, or from
+            // its pooled first column (a multiple of 64, so the coordinate stays 16-byte aligned)
+            const int k0 = p.group_row ? seg[q][g] + kb * BK : kb * BK;
+            const int grp = p.group_row ? 0 : g;
+            tma_load_3d(sA, ma, fb, k0, mt * BM, grp);
+            tma_load_3d(sB, mb, fb, k0, nt * p.width, grp);
           } else {
-            tma_load_3d(sB, mb, fb, kb * BK, nt * p.width, g);
+            const int a_row = p.group_row ? static_cast<int>(row_of(p, g, mt * BM)) : mt * BM;
+            tma_load_3d(sA, ma, fb, kb * BK, a_row, p.group_row ? 0 : g);
+            if (p.mode == kRecompute) {
+              tma_load_3d(sB, mb, fb, kb * BK, nt * p.width, g);
+              tma_load_3d(sB + p.width * BK * 2, mb, fb, kb * BK, p.F + nt * p.width, g);
+            } else {
+              tma_load_3d(sB, mb, fb, kb * BK, nt * p.width, g);
+            }
           }
           pipe.issued |= 1u << pipe.stage;
           pipe.issued_parity = (pipe.issued_parity & ~(1u << pipe.stage)) | (pipe.phase << pipe.stage);
@@ -422,12 +472,11 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) +
                              static_cast<uint32_t>(pipe.acc * gemm::kAccCols);
       if (p.mode == kRecompute) {
-        epi_recompute(p, tbase, g, row, valid, nt);
+        epi_recompute(p, seg[q], tbase, g, row, valid, nt);
       } else if (p.mode == kDh) {
-        epi_dh(p, tbase, g, row, valid, nt);
+        epi_dh(p, seg[q], tbase, g, row, valid, nt);
       } else if (p.mode == kDx) {
-        uint16_t* orow = static_cast<uint16_t*>(p.out) +
-                         (static_cast<long long>(g) * p.C + row) * p.out_ld + nt * p.width;
+        uint16_t* orow = static_cast<uint16_t*>(p.out) + row_of(p, g, row) * p.out_ld + nt * p.width;
         gemm::store_bf16(tbase, p.width, orow, valid);
       } else {
         epi_wgrad(p, tbase, g, row, valid, nt);
@@ -495,12 +544,16 @@ __global__ void __launch_bounds__(256) transpose_kernel(const TransposeArgs a) {
   pdl_trigger_late();
 }
 
-// Dispatch and transpose of round r in one pass. A block takes 64 rows (s0 ..) of expert e's
-// rows in the round and 64 columns (c0 ..): the rows' tokens come from the round-major row list
+// Dispatch and transpose of round r in one pass. A block takes 64 rows of one expert's rows in
+// the round and 64 columns (c0 ..): the rows' tokens come from the round-major row list
 // (row_off[r][e] + s), their x and dy slices are copied row-major into xbuf and dybuf (dy as
-// bf16) and, through a shared-memory tile, transposed into xT and dyT ([E][d][cpad]); rows from
-// n[r][e] up to the next multiple of 64 are zeros in the transposed copies only. The blocks of
-// the first column slice also write each row's gate.
+// bf16) and, through a shared-memory tile, transposed into xT and dyT; rows from n[r][e] up to
+// the next multiple of 64 are zeros in the transposed copies only. The blocks of the first
+// column slice also write each row's gate.
+// Per-expert rows (no borrowing): block (x, y, e) takes expert e's rows 64y.., at e * C + s in the
+// row-major buffers and at [e][c][s] (t_ld per row) in the transposed ones. Pooled rows
+// (borrowing): block (x, y) takes pooled transposed columns 64y.., which lie in the segment of
+// one expert (segments are the experts' rows rounded up to 64, in expert order) or past the last.
 struct GatherArgs {
   const uint16_t* x;
   const float* dy;
@@ -508,25 +561,59 @@ struct GatherArgs {
   const float* gate;
   const int32_t* n;           // [max_rounds, E]
   const int32_t* row_off;     // [max_rounds, E] first row of (round, expert) in the row list
+  const int32_t* row_start;   // [max_rounds + 1]
   const int32_t* row_token;
   uint16_t* xbuf;
   uint16_t* dybuf;
   float* row_gate;
   uint16_t* xt;
   uint16_t* dyt;
-  int r, E, C, d, k, cpad;
+  int r, E, C, d, k, t_ld, pooled;
 };
 
 __global__ void __launch_bounds__(256) bwd_gather_kernel(const __grid_constant__ GatherArgs a) {
   __shared__ uint16_t tx_tile[64][66];
   __shared__ uint16_t ty_tile[64][66];
   __shared__ int tok[64];
+  __shared__ int blk[3];      // expert, its first row of this block, its rows (pooled mode)
   grid_dependency_wait();
-  const int e = blockIdx.z, c0 = blockIdx.x * 64, s0 = blockIdx.y * 64;
-  const int ne = a.n[static_cast<size_t>(a.r) * a.E + e];
+  const int c0 = blockIdx.x * 64;
+  const int32_t* nr = a.n + static_cast<size_t>(a.r) * a.E;
+  int e, s0, ne;
+  if (!a.pooled) {
+    e = blockIdx.z;
+    s0 = blockIdx.y * 64;
+    ne = nr[e];
+  } else {
+    if (threadIdx.x == 0) {
+      const int col = blockIdx.y * 64;
+      int acc = 0, found = -1, first = 0, rows = 0;
+      for (int x = 0; x < a.E; ++x) {
+        const int len = (nr[x] + 63) / 64 * 64;
+        if (col < acc + len) {
+          found = x;
+          first = col - acc;
+          rows = nr[x];
+          break;
+        }
+        acc += len;
+      }
+      blk[0] = found;
+      blk[1] = first;
+      blk[2] = rows;
+    }
+    __syncthreads();
+    e = blk[0];
+    s0 = blk[1];
+    ne = blk[2];
+  }
   const int fill = (ne + 63) / 64 * 64;
-  if (s0 < fill) {
+  if (e >= 0 && s0 < fill) {
     const int base = a.row_off[static_cast<size_t>(a.r) * a.E + e];
+    const long long dst0 = a.pooled ? static_cast<long long>(base - a.row_start[a.r])
+                                    : static_cast<long long>(e) * a.C;   // row-major row of s = 0
+    const long long tcol0 = a.pooled ? static_cast<long long>(blockIdx.y) * 64
+                                     : static_cast<long long>(e) * a.d * a.t_ld + s0;   // + c * t_ld
     if (threadIdx.x < 64) {
       const int sr = s0 + threadIdx.x;
       tok[threadIdx.x] = sr < ne ? a.row_token[base + sr] : -1;
@@ -542,7 +629,7 @@ __global__ void __launch_bounds__(256) bwd_gather_kernel(const __grid_constant__
         xv = *reinterpret_cast<const uint32_t*>(a.x + static_cast<size_t>(t) * a.d + c0 + 2 * tx);
         const float2 dv = *reinterpret_cast<const float2*>(a.dy + static_cast<size_t>(t) * a.d + c0 + 2 * tx);
         yv = gemm::pack_bf16x2(dv.x, dv.y);
-        const size_t orow = (static_cast<size_t>(e) * a.C + s0 + rr) * a.d + c0 + 2 * tx;
+        const size_t orow = static_cast<size_t>(dst0 + s0 + rr) * a.d + c0 + 2 * tx;
         *reinterpret_cast<uint32_t*>(a.xbuf + orow) = xv;
         *reinterpret_cast<uint32_t*>(a.dybuf + orow) = yv;
       }
@@ -555,7 +642,7 @@ __global__ void __launch_bounds__(256) bwd_gather_kernel(const __grid_constant__
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int cc = ty + 8 * i;
-      const size_t o = (static_cast<size_t>(e) * a.d + c0 + cc) * a.cpad + s0 + 2 * tx;
+      const size_t o = static_cast<size_t>(tcol0 + static_cast<long long>(c0 + cc) * a.t_ld) + 2 * tx;
       *reinterpret_cast<uint32_t*>(a.xt + o) =
           static_cast<uint32_t>(tx_tile[2 * tx][cc]) | (static_cast<uint32_t>(tx_tile[2 * tx + 1][cc]) << 16);
       *reinterpret_cast<uint32_t*>(a.dyt + o) =
@@ -566,7 +653,7 @@ __global__ void __launch_bounds__(256) bwd_gather_kernel(const __grid_constant__
       if (t >= 0) {
         int j = 0;
         while (j + 1 < a.k && a.idx[static_cast<size_t>(t) * a.k + j] != e) ++j;
-        a.row_gate[static_cast<size_t>(e) * a.C + s0 + threadIdx.x] = a.gate[static_cast<size_t>(t) * a.k + j];
+        a.row_gate[dst0 + s0 + threadIdx.x] = a.gate[static_cast<size_t>(t) * a.k + j];
       }
     }
   }
@@ -717,7 +804,10 @@ cudaError_t run_gemm(const CUtensorMap* a, const CUtensorMap* b, const bwd::Gemm
 
 }  // namespace
 
-long long backward_cpad(int C) { return (C + 127) / 128 * 128ll; }
+long long backward_t_ld(int E, int C, bool pooled) {
+  const long long w = pooled ? static_cast<long long>(E) * C + 64ll * E : static_cast<long long>(C);
+  return (w + 127) / 128 * 128;
+}
 
 cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_host, cudaStream_t stream) {
   const int E = a.E, d = a.d, F = a.F;
@@ -756,16 +846,20 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
                                   cudaStream_t stream) {
   (void)rows;
   const int E = a.E, C = a.C, d = a.d, F = a.F;
-  const long long cpad = backward_cpad(C);
+  const long long t_ld = a.t_ld;
+  const bool pooled = a.pooled != 0;
   const int32_t* n_dev = a.n + static_cast<size_t>(r) * E;
+  // A operands [E][C][K] per expert, or pooled [1][E * C][K]; transposed [E][rows][t_ld] or [1][rows][t_ld]
+  const uint64_t a_rows = pooled ? static_cast<uint64_t>(E) * C : static_cast<uint64_t>(C);
+  const uint64_t groups = pooled ? 1 : static_cast<uint64_t>(E);
   cudaError_t e;
   // dispatch and transpose x, dy; the rows' gates
   {
-    const bwd::GatherArgs ga{a.x, a.dy, a.idx, a.gate, a.n, a.row_off, a.row_token, a.xbuf, a.dybuf,
-                             a.row_gate, a.xt, a.dyt, r, E, C, d, a.k, static_cast<int>(cpad)};
+    const bwd::GatherArgs ga{a.x, a.dy, a.idx, a.gate, a.n, a.row_off, a.row_start, a.row_token, a.xbuf, a.dybuf,
+                             a.row_gate, a.xt, a.dyt, r, E, C, d, a.k, static_cast<int>(t_ld), pooled ? 1 : 0};
     launch_begin(kKindBackwardCopy, stream);
-    e = launch_pdl(bwd::bwd_gather_kernel, dim3(d / 64, static_cast<unsigned>(cpad / 64), E), dim3(256), 0, stream,
-                   ga);
+    e = launch_pdl(bwd::bwd_gather_kernel, dim3(d / 64, static_cast<unsigned>(t_ld / 64), pooled ? 1 : E), dim3(256),
+                   0, stream, ga);
     launch_end(kKindBackwardCopy, stream);
     if (e != cudaSuccess) return e;
   }
@@ -781,7 +875,9 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
   base.groups = E;
   base.C = C;
   base.F = F;
-  base.cpad = static_cast<int>(cpad);
+  base.t_ld = static_cast<int>(t_ld);
+  base.group_row = pooled ? a.row_off + static_cast<size_t>(r) * E : nullptr;
+  base.group_row_base = pooled ? a.row_start + r : nullptr;
   base.status = a.status;
   static const int kWide[3] = {256, 128, 64};
 
@@ -797,7 +893,7 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g.out_t = a.hgt;
     g.row_gate = a.row_gate;
     CUtensorMap ma, mb;
-    if ((e = gemm::make_map(&ma, a.xbuf, d, C, E, gemm::BM)) != cudaSuccess) return e;
+    if ((e = gemm::make_map(&ma, a.xbuf, d, a_rows, groups, gemm::BM)) != cudaSuccess) return e;
     if ((e = gemm::make_map(&mb, a.w_gate_up, d, 2ull * F, E, static_cast<uint32_t>(g.width))) != cudaSuccess) return e;
     if ((e = run_gemm(&ma, &mb, &g, 1, mt * (F / g.width), stream)) != cudaSuccess) return e;
   }
@@ -817,7 +913,7 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g.dgate_part = a.dgate_part;
     g.dgate_ld = F / 64;
     CUtensorMap ma, mb;
-    if ((e = gemm::make_map(&ma, a.dybuf, d, C, E, gemm::BM)) != cudaSuccess) return e;
+    if ((e = gemm::make_map(&ma, a.dybuf, d, a_rows, groups, gemm::BM)) != cudaSuccess) return e;
     if ((e = gemm::make_map(&mb, a.w2t, d, F, E, static_cast<uint32_t>(g.width))) != cudaSuccess) return e;
     if ((e = run_gemm(&ma, &mb, &g, 1, mt * parts, stream)) != cudaSuccess) return e;
   }
@@ -832,7 +928,7 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g[0].num_k_blocks = 2 * F / gemm::BK;
     g[0].out = a.dxbuf;
     g[0].out_ld = d;
-    if ((e = gemm::make_map(&ma[0], a.dab, 2ull * F, C, E, gemm::BM)) != cudaSuccess) return e;
+    if ((e = gemm::make_map(&ma[0], a.dab, 2ull * F, a_rows, groups, gemm::BM)) != cudaSuccess) return e;
     if ((e = gemm::make_map(&mb[0], a.w13t, 2ull * F, d, E, static_cast<uint32_t>(g[0].width))) != cudaSuccess)
       return e;
     tiles += mt * (d / g[0].width);
@@ -846,8 +942,8 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g[1].overwrite = r == 0;
     g[1].out_group_stride = static_cast<long long>(d) * F;
     g[1].out_ld = F;
-    if ((e = gemm::make_map(&ma[1], a.dyt, static_cast<uint64_t>(cpad), d, E, gemm::BM)) != cudaSuccess) return e;
-    if ((e = gemm::make_map(&mb[1], a.hgt, static_cast<uint64_t>(cpad), F, E, static_cast<uint32_t>(g[1].width))) !=
+    if ((e = gemm::make_map(&ma[1], a.dyt, static_cast<uint64_t>(t_ld), d, groups, gemm::BM)) != cudaSuccess) return e;
+    if ((e = gemm::make_map(&mb[1], a.hgt, static_cast<uint64_t>(t_ld), F, groups, static_cast<uint32_t>(g[1].width))) !=
         cudaSuccess)
       return e;
     tiles += mt_w2 * (F / g[1].width);
@@ -859,9 +955,9 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g[2].overwrite = r == 0;
     g[2].out_group_stride = 2ll * F * d;
     g[2].out_ld = d;
-    if ((e = gemm::make_map(&ma[2], a.dabt, static_cast<uint64_t>(cpad), 2ull * F, E, gemm::BM)) != cudaSuccess)
+    if ((e = gemm::make_map(&ma[2], a.dabt, static_cast<uint64_t>(t_ld), 2ull * F, groups, gemm::BM)) != cudaSuccess)
       return e;
-    if ((e = gemm::make_map(&mb[2], a.xt, static_cast<uint64_t>(cpad), d, E, static_cast<uint32_t>(g[2].width))) !=
+    if ((e = gemm::make_map(&mb[2], a.xt, static_cast<uint64_t>(t_ld), d, groups, static_cast<uint32_t>(g[2].width))) !=
         cudaSuccess)
       return e;
     tiles += mt_w13 * (d / g[2].width);
@@ -870,7 +966,7 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
   // combine dx and gather dgate
   {
     const copy::CombineArgs ca{a.dxbuf, a.dx, a.idx, a.ones, a.round, a.slot, a.T, a.k, C, d,
-                               nullptr, nullptr, E};
+                               pooled ? a.row_off : nullptr, pooled ? a.row_start : nullptr, E};
     launch_begin(kKindBackwardCopy, stream);
     e = launch_pdl(bwd::bwd_combine_kernel, dim3(grid_for(a.T)), dim3(32 * bwd::kWarps), 0, stream, ca, r,
                    static_cast<const float*>(a.dgate_part), F / 64, parts, a.dgate);

@@ -40,12 +40,12 @@ struct BackwardArgs {
   uint16_t* xbuf;             // [E * C, d]
   uint16_t* dybuf;            // [E * C, d]
   float* row_gate;            // [E * C]
-  uint16_t* xt;               // [E, d, cpad]
-  uint16_t* dyt;              // [E, d, cpad]
+  uint16_t* xt;               // [E, d, t_ld], or [d, t_ld] pooled
+  uint16_t* dyt;              // the same
   uint16_t* ab;               // [E * C, 2F]
-  uint16_t* hgt;              // [E, F, cpad]
+  uint16_t* hgt;              // [E, F, t_ld], or [F, t_ld] pooled
   uint16_t* dab;              // [E * C, 2F]
-  uint16_t* dabt;             // [E, 2F, cpad]
+  uint16_t* dabt;             // [E, 2F, t_ld], or [2F, t_ld] pooled
   float* dgate_part;          // [E * C, F / 64]
   uint16_t* dxbuf;            // [E * C, d]
   float* dgate;               // [T, k]
@@ -54,9 +54,13 @@ struct BackwardArgs {
   uint16_t* w13t;             // [E, d, 2F]
   int32_t* status;
   int T, k, E, C, d, F, renorm;
+  int pooled;                 // capacity borrowing: pooled round rows (see the plan's row_off)
+  long long t_ld;             // elements per row of the transposed buffers
 };
-// Row stride of the transposed per-round buffers: C rounded up to 128 (a whole GEMM row tile).
-long long backward_cpad(int C);
+// Elements per row of the transposed per-round buffers: C rounded up to 128 (a whole GEMM row
+// tile) per expert; with pooled rows E * C + 64 * E (every expert's segment rounded up to 64)
+// rounded up to 128, one row for all experts.
+long long backward_t_ld(int E, int C, bool pooled);
 // Zeroes the weight gradients of experts without rows (load_host: host copy of the loads),
 // transposes the weights, fills the unit gates.
 cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_host, cudaStream_t stream);

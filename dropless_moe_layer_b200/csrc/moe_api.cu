@@ -314,16 +314,18 @@ void make_backward_layout(const moe_shape_t* s, moe_backward_layout_t* L) {
     return o;
   };
   const long long T = s->T, E = s->E, k = s->k, C = s->C, d = s->d, F = s->d_ff;
-  const long long cpad = backward_cpad(s->C);
+  const bool pooled = (s->flags & MOE_FLAG_BORROW) != 0;
+  const long long t_ld = backward_t_ld(s->E, s->C, pooled);
+  const long long tg = pooled ? 1 : E;   // transposed buffers: one per expert, or one pooled
   L->xbuf = take(E * C * d * 2);
   L->dybuf = take(E * C * d * 2);
   L->row_gate = take(E * C * 4);
-  L->xt = take(E * d * cpad * 2);
-  L->dyt = take(E * d * cpad * 2);
+  L->xt = take(tg * d * t_ld * 2);
+  L->dyt = take(tg * d * t_ld * 2);
   L->ab = take(E * C * 2 * F * 2);
-  L->hgt = take(E * F * cpad * 2);
+  L->hgt = take(tg * F * t_ld * 2);
   L->dab = take(E * C * 2 * F * 2);
-  L->dabt = take(E * 2 * F * cpad * 2);
+  L->dabt = take(tg * 2 * F * t_ld * 2);
   L->dgate_part = take(E * C * (F / 64) * 4);
   L->dxbuf = take(E * C * d * 2);
   L->dgate = take(T * k * 4);
@@ -331,7 +333,12 @@ void make_backward_layout(const moe_shape_t* s, moe_backward_layout_t* L) {
   L->w2t = take(E * F * d * 2);
   L->w13t = take(E * d * 2 * F * 2);
   L->total_bytes = off;
-  L->cpad = static_cast<int32_t>(cpad);
+  L->cpad = static_cast<int32_t>(t_ld);
+}
+
+// The pooled transposed row (borrowing) must stay within int32 element offsets.
+bool backward_shape_ok(const moe_shape_t* s) {
+  return backward_t_ld(s->E, s->C, (s->flags & MOE_FLAG_BORROW) != 0) < (1ll << 31);
 }
 
 }  // namespace
@@ -339,7 +346,7 @@ void make_backward_layout(const moe_shape_t* s, moe_backward_layout_t* L) {
 extern "C" {
 
 size_t moe_backward_workspace_bytes(const moe_shape_t* shape) {
-  if (check_shape(shape) != MOE_OK) return 0;
+  if (check_shape(shape) != MOE_OK || !backward_shape_ok(shape)) return 0;
   moe_backward_layout_t L;
   make_backward_layout(shape, &L);
   return L.total_bytes;
@@ -348,6 +355,7 @@ size_t moe_backward_workspace_bytes(const moe_shape_t* shape) {
 int moe_backward_workspace_layout(const moe_shape_t* shape, moe_backward_layout_t* layout) {
   const int st = check_shape(shape);
   if (st != MOE_OK) return st;
+  if (!backward_shape_ok(shape)) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (layout == nullptr) return MOE_ERR_INVALID_ARG;
   make_backward_layout(shape, layout);
   return MOE_OK;
@@ -360,7 +368,7 @@ int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws
   moe_workspace_layout_t L;
   int st = check_plan_args(shape, info, ws, ws_bytes, &L);
   if (st != MOE_OK) return st;
-  if (borrowing(shape)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!backward_shape_ok(shape)) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (bws == nullptr || w_gate_up == nullptr || w_down == nullptr || dw_gate_up == nullptr ||
       dw_down == nullptr)
     return MOE_ERR_INVALID_ARG;
@@ -417,6 +425,8 @@ int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws
   a.d = shape->d;
   a.F = shape->d_ff;
   a.renorm = (shape->flags & MOE_FLAG_RENORM_TOPK) ? 1 : 0;
+  a.pooled = borrowing(shape) ? 1 : 0;
+  a.t_ld = B.cpad;
   if ((st = cuda_status(launch_backward_prepare(a, info->load, stream))) != MOE_OK) return st;
   for (int r = 0; r < info->R; ++r) {
     int32_t n_host[MOE_MAX_EXPERTS];

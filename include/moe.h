@@ -219,19 +219,22 @@ typedef struct moe_backward_layout {
   size_t xbuf;        /* bf16 [E * C, d]     the round's x rows */
   size_t dybuf;       /* bf16 [E * C, d]     the round's dy rows */
   size_t row_gate;    /* f32  [E * C]        the gate of the pair in each row */
-  size_t xt;          /* bf16 [E, d, cpad]   xbuf transposed per expert (K-major over rows) */
-  size_t dyt;         /* bf16 [E, d, cpad]   dybuf transposed per expert */
+  size_t xt;          /* bf16 [E, d, cpad]   xbuf transposed per expert (K-major over rows);
+                         with MOE_FLAG_BORROW [d, cpad], pooled */
+  size_t dyt;         /* bf16, dybuf transposed, the same shape */
   size_t ab;          /* bf16 [E * C, 2 d_ff] recomputed a = W1 x, b = W3 x */
-  size_t hgt;         /* bf16 [E, d_ff, cpad] gate * silu(a) * b, transposed per expert */
+  size_t hgt;         /* bf16 [E, d_ff, cpad] gate * silu(a) * b, transposed ([d_ff, cpad] pooled) */
   size_t dab;         /* bf16 [E * C, 2 d_ff] [da | db] */
-  size_t dabt;        /* bf16 [E, 2 d_ff, cpad] [da | db] transposed per expert */
+  size_t dabt;        /* bf16 [E, 2 d_ff, cpad] [da | db] transposed ([2 d_ff, cpad] pooled) */
   size_t dgate_part;  /* f32  [E * C, d_ff / 64] per-tile partial sums of dgate */
   size_t dxbuf;       /* bf16 [E * C, d]     per-pair dx rows of the round */
   size_t dgate;       /* f32  [T, k]         dL/dgate */
   size_t ones;        /* f32  [T, k]         unit gates of the dx combine */
   size_t w2t;         /* bf16 [E, d_ff, d]   W2 transposed */
   size_t w13t;        /* bf16 [E, d, 2 d_ff] W13 transposed */
-  int32_t cpad;       /* C rounded up to a multiple of 128 */
+  int32_t cpad;       /* elements per row of the transposed buffers: C rounded up to 128 (one
+                         buffer per expert); with MOE_FLAG_BORROW, E * C + 64 * E rounded up to
+                         128 (one pooled buffer, every expert's rows rounded up to 64) */
 } moe_backward_layout_t;
 
 /* Bytes of the backward workspace for `shape` (0 for an invalid shape). */
@@ -249,7 +252,7 @@ MOE_API int moe_backward_workspace_layout(const moe_shape_t* shape, moe_backward
  * ws holds the plan (moe_plan) and is only read, except for its status word; x, w_gate_up,
  * w_down as in moe_forward; dy [T, d] fp32. Operands of the tensor-core steps are bf16 (dy, a,
  * b, gate * h, da, db rounded to bf16) with fp32 accumulation. Plans made with MOE_FLAG_BORROW
- * are rejected (MOE_ERR_UNSUPPORTED_SHAPE). A bounded wait that gives up sets the status word
+ * run on their pooled round rows. A bounded wait that gives up sets the status word
  * (moe_device_status). Asynchronous: no synchronization. */
 MOE_API int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
                          void* bws, size_t bws_bytes, const uint16_t* x, const uint16_t* w_gate_up,

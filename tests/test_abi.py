@@ -138,15 +138,18 @@ def test_forward_argument_errors_without_gpu(lib):
     assert lib.moe_forward(P(sb), P(info), ws, need_b, 4096, 4096, 4096, 4096, None) == -1
 
 
-def _backward_bytes_model(w):
+def _backward_bytes_model(w, borrow=False):
     """Backward workspace from its layout rules: per-round buffers of E*C rows, the transposed
-    copies with C rounded up to 128, the weights transposed once, [T, k] dgate and unit gates."""
+    copies with C rounded up to 128 per expert (with borrowing one pooled copy whose rows hold
+    E*C + 64*E columns rounded up to 128), the weights transposed once, [T, k] dgate and unit
+    gates."""
     def a(n):
         return (n + 255) // 256 * 256
     T, E, k, C, d, F = w.T, w.E, w.k, w.C, w.d, w.F
-    cp = (C + 127) // 128 * 128
-    return (3 * a(E * C * d * 2) + a(E * C * 4) + 2 * a(E * d * cp * 2) + 2 * a(E * C * 2 * F * 2)
-            + a(E * F * cp * 2) + a(E * 2 * F * cp * 2) + a(E * C * (F // 64) * 4) + 2 * a(T * k * 4)
+    cp = (E * C + 64 * E + 127) // 128 * 128 if borrow else (C + 127) // 128 * 128
+    tg = 1 if borrow else E
+    return (3 * a(E * C * d * 2) + a(E * C * 4) + 2 * a(tg * d * cp * 2) + 2 * a(E * C * 2 * F * 2)
+            + a(tg * F * cp * 2) + a(tg * 2 * F * cp * 2) + a(E * C * (F // 64) * 4) + 2 * a(T * k * 4)
             + a(E * F * d * 2) + a(E * d * 2 * F * 2))
 
 
@@ -160,6 +163,9 @@ def test_backward_workspace_is_fixed_by_shape(lib, w):
     offs = [lay.xbuf, lay.dybuf, lay.row_gate, lay.xt, lay.dyt, lay.ab, lay.hgt, lay.dab, lay.dabt,
             lay.dgate_part, lay.dxbuf, lay.dgate, lay.ones, lay.w2t, lay.w13t]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    sb = moe.make_shape(w.T, w.d, w.E, w.k, w.F, w.C, borrow=True)
+    assert moe.backward_workspace_bytes(sb) == _backward_bytes_model(w, borrow=True)
+    assert moe.backward_layout(sb).cpad == (w.E * w.C + 64 * w.E + 127) // 128 * 128
     s.flags = 16
     assert moe.backward_workspace_bytes(s) == 0
 
@@ -178,11 +184,13 @@ def test_backward_argument_errors_without_gpu(lib):
     assert f(P(s), P(info), ws, need, bws + 64, bneed, p, p, p, p, p, p, p, p, None) == -4
     assert f(P(s), P(info), ws, need, bws, bneed, p, p, p, p + 4, p, p, p, p, None) == -4
     assert f(P(s), P(info), ws, need, bws, bneed, p, p, p, None, p, p, p, p, None) == -1
-    # plans with capacity borrowing are not supported by the backward
+    # a plan with capacity borrowing runs on a borrowing shape (its argument checks pass and
+    # the call reaches the device check), and only on one
     sb = moe.make_shape(64, 128, 8, 2, 128, 16, borrow=True)
     info.plan_flags = moe.FLAG_BORROW
     assert f(P(sb), P(info), ws, moe.workspace_bytes(sb), bws, moe.backward_workspace_bytes(sb),
-             p, p, p, p, p, p, p, p, None) == -2
+             p, p, p, p, p, p, p, p, None) not in (-1, -2, -3, -4)
+    assert f(P(s), P(info), ws, need, bws, bneed, p, p, p, p, p, p, p, p, None) == -1
 
 
 @pytest.mark.parametrize("cmd", [["gcc", "-std=c99", "-x", "c"], ["g++", "-std=c++11", "-x", "c++"]],

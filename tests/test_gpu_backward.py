@@ -30,8 +30,8 @@ def rel_err(got, ref):
     return float(np.max(np.abs(got - ref)) / max(np.max(np.abs(ref)), 1e-30))
 
 
-def run_backward(w, inp, dy, renorm=False):
-    layer = moe.DroplessMoE(w.T, w.d, w.E, w.k, w.F, w.C, renorm=renorm)
+def run_backward(w, inp, dy, renorm=False, borrow=False):
+    layer = moe.DroplessMoE(w.T, w.d, w.E, w.k, w.F, w.C, renorm=renorm, borrow=borrow)
     layer(inp["x"], inp["w_gate_up"], inp["w_down"], logits=inp["logits"])
     g = layer.backward(inp["x"], inp["w_gate_up"], inp["w_down"], dy)
     torch.cuda.synchronize()
@@ -115,3 +115,25 @@ def test_backward_empty_batch():
     assert layer.device_status() == 0
     assert g["dx"].shape == (0, 128) and g["dz"].shape == (0, 8)
     assert torch.count_nonzero(g["dw_gate_up"]) == 0 and torch.count_nonzero(g["dw_down"]) == 0
+
+
+@pytest.mark.parametrize("name", ["tiny-zipf1", "4k-zipf1"])
+def test_backward_borrow_full_parity(name):
+    """With capacity borrowing the rounds hold pooled rows; the gradients do not depend on the
+    plan."""
+    w = wl.BY_NAME[name]
+    inp = wl.generate(w, "cuda")
+    dy = wl.generate_dy(w, "cuda")
+    layer, g = run_backward(w, inp, dy, borrow=True)
+    assert layer.info.R < (max(layer.info.load[:w.E]) + w.C - 1) // w.C    # borrowing saved rounds
+    check(w, inp, dy, g)
+
+
+@pytest.mark.parametrize("cfg", EDGE, ids=lambda c: "T{T}-d{d}-E{E}-k{k}-F{F}-C{C}".format(**c))
+def test_backward_borrow_edge_shapes(cfg):
+    w = wl.custom(name="edge", T=cfg["T"], d=cfg["d"], E=cfg["E"], k=cfg["k"], F=cfg["F"], C=cfg["C"],
+                  bias="zipf", zipf_s=1.0, seed=cfg["T"])
+    inp = wl.generate(w, "cuda")
+    dy = wl.generate_dy(w, "cuda")
+    layer, g = run_backward(w, inp, dy, borrow=True)
+    check(w, inp, dy, g)
