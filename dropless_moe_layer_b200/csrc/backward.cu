@@ -13,13 +13,15 @@
 //   dW2_e += (gate dy) h^T = dy (gate h)^T  dW1_e += da x^T, dW3_e += db x^T
 //   dz = softmax Jacobian applied to dgate (renormalised gates: the quotient rule first).
 //
-// Per round r, with the forward's plan (rows of expert e in round r at e * C + slot):
+// Per round r, with the forward's plan (rows of expert e in round r at e * C + slot; with
+// capacity borrowing pooled, at row_off[r][e] - row_start[r] + slot):
 //   gather     x rows -> xbuf, bf16(dy) rows -> dybuf (row-major) and, in the same pass, xT, dyT
-//              ([E][d][Cp], Cp = C rounded up to 128: K-major over the round's rows for the
-//              weight-gradient GEMMs; zeros past the expert's rows up to the next multiple of 64);
-//              the pair's gate -> row_gate
+//              (K-major over the round's rows for the weight-gradient GEMMs: [E][d][Cp] with
+//              Cp = C rounded up to 128, or pooled [d][E * C + 64 E rounded up to 128] with each
+//              expert's rows rounded up to 64; zeros past the expert's rows up to the next
+//              multiple of 64); the pair's gate -> row_gate
 //   recompute  [a | b] = xbuf W13^T (tensor cores); epilogue keeps a, b (bf16, row-major) and
-//              writes bf16(gate * h) transposed (hgT [E][F][Cp])
+//              writes bf16(gate * h) transposed (hgT, F rows)
 //   dh         W2^T dy as dybuf (W2^T)^T (tensor cores, B = W2 transposed once per call);
 //              epilogue: the SwiGLU backward (da, db from a, b and the gate), dgate partial sums
 //              <W2^T dy, h> per 64..256-column tile, dab = [da | db] row-major and transposed
@@ -27,15 +29,16 @@
 //   combine    dx[t] = (first round of t ? 0 : dx[t]) + sum of the token's dxbuf rows, ascending
 //              j; dgate[t, j] = sum of its row's partials in tile order (no atomics anywhere)
 //   wgrad      dW2 += dyT hgT^T and dW13 += dabT xT^T over K = the round's rows of each expert
-//              (one launch together with the dx GEMM: the three are independent)
 //              (tensor cores; fp32 read-add-write of the caller's gradient, one CTA per tile;
-//              round 0 stores instead: it holds every expert that has rows)
+//              round 0 stores instead: it holds every expert that has rows); one launch with
+//              the dx GEMM, as the three are independent
 // After the last round: dz from dgate and the logits (one warp per token).
 //
 // Every operand of a tensor-core step is bf16 (fp32 accumulate); a and b are kept as bf16 between
 // the recompute and the dh epilogue. Rows of a tile past the expert's row count never reach a
-// row-major store; in the transposed buffers they are written as zeros, so the weight-gradient
-// GEMMs may read K up to the next multiple of 64 without a mask.
+// row-major store; in the transposed buffers they are written as zeros up to the next multiple of
+// 64 (and no further: with pooled rows the next expert's rows follow), so the weight-gradient
+// GEMMs may read K in blocks of 64 without a mask.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
