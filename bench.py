@@ -334,6 +334,10 @@ BWD_METRIC = ("routed tokens/s per MoE layer backward with per-round recompute (
               "% of tensor roofline")
 
 
+# Tensor-core flops per routed pair, in units of d * d_ff, of each backward GEMM launch kind.
+BWD_KIND_FLOPS = {"backward_recompute": 4, "backward_dh": 2, "backward_dx_wgrad": 10}
+
+
 def backward_flops(w):
     """Tensor-core work of one backward pass: per routed pair the recompute of a and b (4 d d_ff),
     W2^T dy (2 d d_ff), dx = [da | db] W13 (4 d d_ff), dW2 (2 d d_ff) and dW1, dW3 (4 d d_ff)."""
@@ -421,7 +425,7 @@ def bench_backward(args, w):
     status = layer.device_status()
     peaks, peak_src = load_peaks()
     flops = backward_flops(w)
-    gemm_ms = prof["backward_gemm"][1]
+    gemm_ms = sum(prof[k][1] for k in moe.BACKWARD_GEMM_KINDS if k in prof)
     achieved = flops / (gemm_ms / 1e3) / 1e12
     peak = peaks["bf16_tflops"]
     ms = total_ms / args.steps
@@ -429,12 +433,16 @@ def bench_backward(args, w):
         "metric": BWD_METRIC, "pass": "backward", "value": w.T / (ms / 1e3), "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w), "rounds": info.R,
-        "roofline": {"kernel": "backward_gemm", "bound": "tensor", "achieved": achieved, "peak": peak,
+        "roofline": {"kernel": "backward GEMMs (" + ", ".join(moe.BACKWARD_GEMM_KINDS) + ")", "bound": "tensor",
+                     "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{peak_src} (bf16_tflops burst)", "traffic": None,
                      "flops_per_step": flops},
         "whole_pass_tflops": flops / (ms / 1e3) / 1e12,
-        "kernels": {k: {"launches": c, "ms": round(t, 4)} for k, (c, t) in prof.items()},
+        "kernels": {k: dict({"launches": c, "ms": round(t, 4)},
+                            **({"TFLOP/s": round(BWD_KIND_FLOPS[k] * w.T * w.k * w.d * w.F / (t / 1e3) / 1e12, 1)}
+                               if k in BWD_KIND_FLOPS else {}))
+                    for k, (c, t) in prof.items()},
         "cpu_baseline": None if args.no_cpu_baseline else backward_cpu_baseline(w),
         "gpu_launches": launches,
         "device_status": status,

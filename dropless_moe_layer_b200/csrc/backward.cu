@@ -778,7 +778,7 @@ int pick_width(const int* widths, int n_widths, long long mtiles, int n_total) {
 
 // One launch of up to three GEMM phases (maps a[q], b[q], args[q]); tiles = the sum of their tiles.
 cudaError_t run_gemm(const CUtensorMap* a, const CUtensorMap* b, const bwd::GemmArgs* args, int phases,
-                     long long tiles, cudaStream_t stream) {
+                     long long tiles, int kind, cudaStream_t stream) {
   if (tiles <= 0) return cudaSuccess;
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
@@ -798,10 +798,10 @@ cudaError_t run_gemm(const CUtensorMap* a, const CUtensorMap* b, const bwd::Gemm
   const CUtensorMap& a2 = a[phases > 2 ? 2 : 0];
   const CUtensorMap& b2 = b[phases > 2 ? 2 : 0];
   const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
-  launch_begin(kKindBackwardGemm, stream);
+  launch_begin(kind, stream);
   const cudaError_t err = launch_pdl(bwd::bwd_gemm_kernel, dim3(grid), dim3(gemm::kThreads), bwd::kSmemBytes,
                                      stream, a[0], b[0], a1, b1, a2, b2, L);
-  launch_end(kKindBackwardGemm, stream);
+  launch_end(kind, stream);
   return err;
 }
 
@@ -898,7 +898,8 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     CUtensorMap ma, mb;
     if ((e = gemm::make_map(&ma, a.xbuf, d, a_rows, groups, gemm::BM)) != cudaSuccess) return e;
     if ((e = gemm::make_map(&mb, a.w_gate_up, d, 2ull * F, E, static_cast<uint32_t>(g.width))) != cudaSuccess) return e;
-    if ((e = run_gemm(&ma, &mb, &g, 1, mt * (F / g.width), stream)) != cudaSuccess) return e;
+    if ((e = run_gemm(&ma, &mb, &g, 1, mt * (F / g.width), kKindBackwardRecompute, stream)) != cudaSuccess)
+      return e;
   }
   // dh = W2^T dy with the SwiGLU backward in its epilogue
   int parts = 0;
@@ -918,7 +919,7 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     CUtensorMap ma, mb;
     if ((e = gemm::make_map(&ma, a.dybuf, d, a_rows, groups, gemm::BM)) != cudaSuccess) return e;
     if ((e = gemm::make_map(&mb, a.w2t, d, F, E, static_cast<uint32_t>(g.width))) != cudaSuccess) return e;
-    if ((e = run_gemm(&ma, &mb, &g, 1, mt * parts, stream)) != cudaSuccess) return e;
+    if ((e = run_gemm(&ma, &mb, &g, 1, mt * parts, kKindBackwardDh, stream)) != cudaSuccess) return e;
   }
   // one launch: dx rows = dab W13, dW2 (+)= dyT hgT^T, dW13 (+)= dabT xT^T (K = the round's rows)
   {
@@ -964,7 +965,7 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
         cudaSuccess)
       return e;
     tiles += mt_w13 * (d / g[2].width);
-    if ((e = run_gemm(ma, mb, g, 3, tiles, stream)) != cudaSuccess) return e;
+    if ((e = run_gemm(ma, mb, g, 3, tiles, kKindBackwardDxWgrad, stream)) != cudaSuccess) return e;
   }
   // combine dx and gather dgate
   {

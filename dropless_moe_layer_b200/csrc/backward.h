@@ -11,8 +11,10 @@ namespace moe {
 
 // Kernel kinds of the backward's launches for profiling (after the forward's KernelKind values;
 // same numbering as the public header).
-constexpr int kKindBackwardGemm = 8;
-constexpr int kKindBackwardCopy = 9;
+constexpr int kKindBackwardRecompute = 8;
+constexpr int kKindBackwardDh = 9;
+constexpr int kKindBackwardDxWgrad = 10;
+constexpr int kKindBackwardCopy = 11;
 
 // ---- backward with per-round recompute (backward.cu)
 // Device pointers of one backward call: the forward's plan (read only), the caller's tensors and

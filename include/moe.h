@@ -273,11 +273,11 @@ MOE_API uint64_t moe_launch_count(void);
  * is bracketed by two events on its stream; moe_profile_read() synchronizes on them and
  * reports, per kernel kind, the launch count and the summed milliseconds. Kinds:
  * 0 router GEMM, 1 top-k, 2 plan, 3 dispatch, 4 gate_up GEMM, 5 down GEMM, 6 combine,
- * 7 pipelined rounds (all four steps of its rounds in one launch), 8 backward GEMMs (recompute,
- * dh, dx and weight gradients), 9 the backward's other launches (dispatch, transposes, dx
- * combine, gate gradient, fills).
+ * 7 pipelined rounds (all four steps of its rounds in one launch); backward: 8 recompute GEMM,
+ * 9 dh GEMM (with the SwiGLU backward), 10 dx and weight-gradient GEMMs (one launch a round),
+ * 11 its other launches (gather, weight transposes, dx combine, gate gradient, fills).
  * Up to 4096 launches are recorded between enable and read. Not thread-safe. */
-#define MOE_PROFILE_KINDS 10
+#define MOE_PROFILE_KINDS 12
 MOE_API int moe_profile_enable(int on);
 MOE_API int moe_profile_read(int32_t counts[MOE_PROFILE_KINDS], double ms[MOE_PROFILE_KINDS]);
 

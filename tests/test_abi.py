@@ -206,3 +206,13 @@ def test_public_header_is_plain_c(cmd):
     out = subprocess.run(cmd + ["-fsyntax-only", "-Wall", "-Wextra", "-Werror", header],
                          capture_output=True, text=True)
     assert out.returncode == 0, out.stderr
+
+
+def test_profile_kinds_agree_with_the_header():
+    import os
+    import re
+    header = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe.h")
+    with open(header) as f:
+        n = int(re.search(r"#define MOE_PROFILE_KINDS (\d+)", f.read()).group(1))
+    assert moe.PROFILE_KINDS == n == len(moe.PROFILE_NAMES)
+    assert set(moe.BACKWARD_GEMM_KINDS) <= set(moe.PROFILE_NAMES)

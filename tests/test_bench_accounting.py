@@ -62,3 +62,12 @@ def test_traffic_record_ignores_comments_not_code():
     reflowed = 'int   a = 1;   // another note\n  const char* s = "//kept"; // x\nchar c = \'/\';'
     assert bench.code_tokens(reflowed) == bench.code_tokens(src)
     assert bench.code_tokens(src.replace("a = 1", "a = 2")) != bench.code_tokens(src)
+
+
+def test_backward_flops_split_by_launch_kind():
+    """The backward's GEMM launch kinds account for all of its tensor-core work: 16 d d_ff flops
+    per routed pair (recompute 4, dh 2, dx 4, dW2 2, dW1 and dW3 4)."""
+    from dropless_moe_layer_b200 import moe
+    w = wl.BY_NAME["4k-zipf1"]
+    assert set(bench.BWD_KIND_FLOPS) == set(moe.BACKWARD_GEMM_KINDS)
+    assert sum(bench.BWD_KIND_FLOPS.values()) * w.T * w.k * w.d * w.F == bench.backward_flops(w)
