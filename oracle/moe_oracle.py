@@ -44,8 +44,6 @@ Readings where the pages are silent (each listed in the design notes):
 """
 from __future__ import annotations
 
-import math
-
 import numpy as np
 
 
