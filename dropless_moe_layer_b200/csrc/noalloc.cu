@@ -9,15 +9,19 @@
 // file-scope device array of fixed size. The caller passes only the logits and the
 // four [T, k] output arrays.
 //
-// The array is MOE_NOALLOC_SCRATCH_BYTES large and every GPU that loads this library
-// holds it until the process exits. All calls share it: two calls whose work overlaps
-// on the GPU (different streams, or different host threads) race on it. The contents
-// left by the previous call are never trusted: the header (status word included) is
-// cleared by every call and every other region is fully rewritten before it is read.
+// The array is MOE_NOALLOC_SCRATCH_BYTES large. CUDA reserves it on a device when it loads
+// this file's code there: at context creation under eager module loading, and under lazy
+// loading (the CUDA 12 default) at the first moe_plan_noalloc() on that device, whose address
+// lookup loads it. From then on the device holds it until the process exits. So a caller that
+// must not allocate later makes one call per device at start-up (a batch of T = 0 will do),
+// before its memory pool takes the device and before any stream capture. All calls share the
+// array: two calls whose work overlaps on the GPU (different streams, or different host
+// threads) race on it. The contents left by the previous call are never trusted: the header
+// (status word included) is cleared by every call and every other region is fully rewritten
+// before it is read.
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <mutex>
 
 #include "kernels.h"
 #include "moe.h"
@@ -26,21 +30,13 @@ namespace {
 
 static __device__ __align__(256) uint8_t g_plan_scratch[MOE_NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_plan_scratch, resolved once per device ordinal with that device
-// current (host code must not use the symbol itself as a device pointer).
-std::mutex g_scratch_mutex;
-void* g_scratch_ptr[64] = {nullptr};
-
+// Device address of g_plan_scratch on the current device. Host code must not use the symbol
+// itself as a device pointer. The address is looked up on every call, not cached: a cached
+// address would outlive the context it belongs to (cudaDeviceReset tears the module down).
 int scratch_for_current_device(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_plan_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_plan_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+  *out = p;
   return MOE_OK;
 }
 

@@ -75,33 +75,6 @@ constexpr int kPipeThreads = kThreads + 32 * (kDispWarps + kCombWarps);
 constexpr int kEpiWarps = 4;
 constexpr int kRing = 4;   // claimed tiles in flight between the producer and the consumers
 
-#ifdef MOE_TRACE
-// Diagnostic build only (-DMOE_TRACE): %globaltimer stamps of the launch, written to a buffer
-// that moe_trace_set() installs. Layout (u64): [0] first CTA start (min), [1] last CTA end
-// (max); from 16, eight words per GEMM tile: inputs ready, first load issued, epilogue done,
-// CTA, first stage consumed by the MMA, last MMA committed, accumulator seen by the epilogue,
-// last load issued; from 16 + 8 * kTraceTasks, eight words per round: dispatch start (min),
-// dispatch end (max), combine start (min), combine end (max).
-constexpr int kTraceTasks = 1 << 16;
-constexpr int kTraceRounds = 4096;
-__device__ unsigned long long* g_trace = nullptr;
-__device__ __forceinline__ void trace_min(long long i, unsigned long long v) {
-  if (g_trace) atomicMin(g_trace + i, v);
-}
-__device__ __forceinline__ void trace_max(long long i, unsigned long long v) {
-  if (g_trace) atomicMax(g_trace + i, v);
-}
-__device__ __forceinline__ void trace_task(int task, int word, unsigned long long v) {
-  if (g_trace && task < kTraceTasks) g_trace[16 + 8ll * task + word] = v;
-}
-__device__ __forceinline__ long long trace_round(int r, int word) {
-  return 16 + 8ll * kTraceTasks + 8ll * (r < kTraceRounds ? r : kTraceRounds - 1) + word;
-}
-#define MOE_TRACE_DO(x) x
-#else
-#define MOE_TRACE_DO(x)
-#endif
-
 __device__ __forceinline__ int ld_acquire(const int32_t* p) {
   int v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -276,7 +249,6 @@ __device__ void dispatch_role(const PipelineArgs& a, const Counters& cn) {
     const int begin = a.row_start[r], rows = a.row_start[r + 1] - begin;
     const int chunk = (rows + W - 1) / W;
     const int lo = gw * chunk, hi = min(rows, lo + chunk);
-    MOE_TRACE_DO(if (lane == 0 && lo < hi) trace_min(trace_round(r, 0), global_timer_ns()));
     for (int b = lo; b < hi; b += 32) {
       const int nr = min(32, hi - b);
       int tok = 0, dst = 0, blk = -1;
@@ -304,7 +276,6 @@ __device__ void dispatch_role(const PipelineArgs& a, const Counters& cn) {
       __syncwarp();
       if (head) red_release(cn.disp[p] + blk, run_end - lane);
     }
-    MOE_TRACE_DO(if (lane == 0 && lo < hi) trace_max(trace_round(r, 1), global_timer_ns()));
   }
 }
 
@@ -329,7 +300,6 @@ __device__ void combine_role(const PipelineArgs& a, const Counters& cn) {
     const int blk_target = (q + 1) * kEpiWarps * (a.d / kPipeDnWidth);
     const copy::CombineArgs comb{a.out[p], a.y, a.idx, a.gate, a.round, a.slot, a.T, a.k, a.C, a.d};
     bool round_done = false;   // every down tile of round r seen finished
-    MOE_TRACE_DO(if (lane == 0) trace_min(trace_round(r, 2), global_timer_ns()));
     for (long long c0 = gw; c0 < a.T; c0 += span) {
       const long long tl = c0 + static_cast<long long>(lane) * W;
       bool has = false;
@@ -358,7 +328,6 @@ __device__ void combine_role(const PipelineArgs& a, const Counters& cn) {
         if (lane < tp.npairs) red_release(cn.rd[p] + blk, 1);   // this pair's out row is read
       }
     }
-    MOE_TRACE_DO(if (lane == 0) trace_max(trace_round(r, 3), global_timer_ns()));
   }
 }
 
@@ -390,7 +359,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
   const uint32_t tmem = setup(s);
   grid_dependency_wait();
   const Counters cn = counters(a);
-  MOE_TRACE_DO(if (threadIdx.x == 0) trace_min(0, global_timer_ns()));
 
   if (warp == 0) {
     if (lane == 0) {
@@ -432,7 +400,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         // before the wait for this tile's A rows, so they arrive while it waits.
         const int pre = t.kb < kPStages ? t.kb : kPStages;
         const int first = stage;
-        MOE_TRACE_DO(trace_task(task, 1, global_timer_ns()); trace_task(task, 3, blockIdx.x));
         int armed = 0;
         for (; armed < pre; ++armed) {
           if (!mbar_wait(smem_addr(&s.empty[stage]), phase ^ 1u, s.abort)) {
@@ -451,7 +418,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
           }
         }
         const bool inputs = ok && wait_inputs(a, cn, c, t);
-        MOE_TRACE_DO(trace_task(task, 0, global_timer_ns()));
         fence_proxy_async();
         // A loads of the armed stages (issued even when giving up, so every armed stage completes)
         for (int i = 0; i < armed; ++i) {
@@ -479,7 +445,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             phase ^= 1u;
           }
         }
-        MOE_TRACE_DO(trace_task(task, 7, global_timer_ns()));
       }
       if (!ok) {
         atomicOr(a.status, kStatusTimeoutProducer);
@@ -527,7 +492,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             break;
           }
           tc_fence_after();
-          MOE_TRACE_DO(if (kb == 0) trace_task(task, 4, global_timer_ns()));
           const uint32_t sA = smem_addr(s.stage + stage * kPStageBytes);
           const uint64_t adesc = smem_desc_sw128(sA);
           const uint64_t bdesc = smem_desc_sw128(sA + kABytes);
@@ -542,7 +506,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         }
         if (!ok) break;
         mma_commit(smem_addr(&s.tfull[acc]));
-        MOE_TRACE_DO(trace_task(task, 5, global_timer_ns()));
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
@@ -593,7 +556,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         break;
       }
       tc_fence_after();
-      MOE_TRACE_DO(if (warp == 2 && lane == 0) trace_task(task, 6, global_timer_ns()));
       const int row = t.m * BM + q * 32 + lane;
       const bool valid = row < a.n[static_cast<size_t>(t.r) * a.E + t.e];
       const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kAccCols);
@@ -616,7 +578,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         const int blk = (t.e * cn.mb + t.m) * kSyncStride;
         red_release((t.gu ? cn.gu[p] : cn.dn[p]) + blk, 1);
         if (!t.gu) red_release(a.sync + kSyncDnTotal + p * kSyncSetStride, 1);
-        MOE_TRACE_DO(if (warp == 2) trace_task(task, 2, global_timer_ns()));
       }
     }
     __syncwarp();
@@ -630,7 +591,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  MOE_TRACE_DO(if (threadIdx.x == 0) trace_max(1, global_timer_ns()));
   if (threadIdx.x == 0) {
     __threadfence();
     last_cta = atomicAdd(a.sync + kSyncExit, 1) == static_cast<int>(gridDim.x) - 1;
@@ -646,13 +606,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
 }
 
 }  // namespace
-
-#ifdef MOE_TRACE
-extern "C" MOE_API int moe_trace_set(void* buffer) {
-  unsigned long long* p = static_cast<unsigned long long*>(buffer);
-  return cudaMemcpyToSymbol(g_trace, &p, sizeof(p)) == cudaSuccess ? 0 : -5;
-}
-#endif
 
 cudaError_t launch_round_pipeline(const PipelineArgs& a, cudaStream_t stream) {
   if (a.r0 >= a.R) return cudaSuccess;

@@ -288,8 +288,9 @@ MOE_API int moe_profile_read(int32_t counts[MOE_PROFILE_KINDS], double ms[MOE_PR
  * that already owns the device, plugins that a host framework hands only their input
  * and output buffers, or services that forbid cudaMalloc after start-up. moe_plan()
  * needs a caller-allocated workspace; this call keeps the planner's scratch in one
- * static device array of MOE_NOALLOC_SCRATCH_BYTES inside the library instead. Every
- * GPU that loads the library holds that array until the process exits.
+ * static device array of MOE_NOALLOC_SCRATCH_BYTES inside the library instead. A GPU
+ * holds that array from the moment it loads the library's code (its first
+ * moe_plan_noalloc() call under lazy module loading) until the process exits.
  *
  *   logits   [T, E] fp32 device input (the router-GEMM form is not offered here);
  *   topk_idx [T, k] int32, gate [T, k] fp32, round [T, k] int32, slot [T, k] int32:
@@ -297,12 +298,14 @@ MOE_API int moe_profile_read(int32_t counts[MOE_PROFILE_KINDS], double ms[MOE_PR
  *   R        host out: the number of rounds; load: host out [E] (may be NULL).
  * Returns MOE_ERR_NOALLOC_LIMIT, launching nothing, when the shape's scratch
  * (about 8*T*k + 8*ceil(T/C)*E + 4*ceil(T/256)*E bytes) exceeds the array. Calls no
- * cudaMalloc, cudaFree or other allocating routine. The first call on each device
- * looks up the array's device address (cudaGetSymbolAddress) with that device
- * current; make that first call before any stream capture. All calls share the array
- * and each one clears what must start at zero, but calls whose GPU work overlaps
- * (other streams, other threads) race on it. Synchronizes `stream` once, like
- * moe_plan(). */
+ * cudaMalloc, cudaFree or other allocating routine. Every call looks up the array's
+ * device address (cudaGetSymbolAddress) on the current device. Under CUDA's lazy module
+ * loading (the default) that lookup is also what makes the device reserve the array, so
+ * the FIRST call on each device may need 16 MiB of free device memory: make one call per
+ * device at start-up (T = 0 will do), before a memory pool takes the device and before
+ * any stream capture. All calls share the array and each one clears what must start at
+ * zero, but calls whose GPU work overlaps (other streams, other threads) race on it.
+ * Synchronizes `stream` once, like moe_plan(). */
 #define MOE_NOALLOC_SCRATCH_BYTES (16u << 20)
 MOE_API int moe_plan_noalloc(const moe_shape_t* shape, const float* logits, int32_t* topk_idx,
                              float* gate, int32_t* round, int32_t* slot, int32_t* R,
