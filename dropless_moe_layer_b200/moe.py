@@ -100,6 +100,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
         "moe_profile_read": (ctypes.c_int, [P(c_i32), P(ctypes.c_double)]),
         "moe_plan_noalloc": (ctypes.c_int, [P(Shape), c_vp, c_vp, c_vp, c_vp, c_vp, P(c_i32), P(c_i32), c_vp]),
+        "moe_ep_exchange_plan": (ctypes.c_int, [P(Shape), c_i32, c_i32, P(c_i32), c_i32, P(c_i32), P(c_i32),
+                                                P(c_i32), P(c_i32), P(c_i32), P(c_i32), P(c_i32)]),
         "moe_backward_workspace_bytes": (c_sz, [P(Shape)]),
         "moe_backward_workspace_layout": (ctypes.c_int, [P(Shape), P(BackwardLayout)]),
         "moe_backward": (ctypes.c_int, [P(Shape), P(PlanInfo), c_vp, c_sz, c_vp, c_sz, c_vp, c_vp, c_vp,
@@ -218,6 +220,29 @@ def profile_read() -> dict:
     ms = (ctypes.c_double * PROFILE_KINDS)()
     _check("moe_profile_read", load_library().moe_profile_read(counts, ms))
     return {PROFILE_NAMES[i]: (int(counts[i]), float(ms[i])) for i in range(PROFILE_KINDS)}
+
+
+def ep_exchange_plan(shape: Shape, G: int, rank: int, loads) -> dict:
+    """Exchange tables of an expert-parallel rank (moe_ep_exchange_plan; host code, no GPU).
+    loads: [G, E] integer array of every rank's pair counts per expert. Returns numpy arrays:
+    R, base [E], send_counts / send_offsets / recv_counts / recv_offsets [R, G], n_owned [R, E/G]."""
+    import numpy as np
+    E = shape.E
+    lo = np.ascontiguousarray(np.asarray(loads, dtype=np.int32).reshape(G, E))
+    P = ctypes.POINTER(c_i32)
+    R = c_i32(0)
+    base = np.zeros(E, dtype=np.int32)
+    lib = load_library()
+    _check("moe_ep_exchange_plan", lib.moe_ep_exchange_plan(ctypes.byref(shape), G, rank, lo.ctypes.data_as(P), 0,
+                                                            ctypes.byref(R), base.ctypes.data_as(P), None, None,
+                                                            None, None, None))
+    nr = R.value
+    out = {k: np.zeros((nr, G), dtype=np.int32) for k in ("send_counts", "send_offsets", "recv_counts", "recv_offsets")}
+    out["n_owned"] = np.zeros((nr, E // G if G > 0 else 0), dtype=np.int32)
+    _check("moe_ep_exchange_plan", lib.moe_ep_exchange_plan(
+        ctypes.byref(shape), G, rank, lo.ctypes.data_as(P), nr, ctypes.byref(R), base.ctypes.data_as(P),
+        *[out[k].ctypes.data_as(P) for k in ("send_counts", "send_offsets", "recv_counts", "recv_offsets", "n_owned")]))
+    return dict(out, R=nr, base=base)
 
 
 # ------------------------------------------------------------------------- torch marshalling

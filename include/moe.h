@@ -281,6 +281,41 @@ MOE_API uint64_t moe_launch_count(void);
 MOE_API int moe_profile_enable(int on);
 MOE_API int moe_profile_read(int32_t counts[MOE_PROFILE_KINDS], double ms[MOE_PROFILE_KINDS]);
 
+/* ---------------------------------------------------------------- expert parallelism
+ *
+ * "Frontier Pre-training at Microsoft AI (MAI-Base-2)", Key claims, the multi-round dropless
+ * MoE item [section "Scaling MoE", Fig. 6]: the experts are split into groups, one group per
+ * expert-parallel rank, and every group runs dispatch -> compute -> collect rounds with a fixed
+ * per-expert capacity; the token metadata stays on the device. Over G ranks, rank g owns the
+ * E/G contiguous experts [g E/G, (g+1) E/G). An expert's capacity C per round is shared by all
+ * source ranks, which fill it in (source rank, token) order: the job's plan is the single-GPU
+ * plan of the ranks' batches concatenated in rank order, and every rank runs the same
+ * R = ceil(max_e total_e / C) rounds. In round r, rank s sends rank g its pairs of round r
+ * whose expert g owns, in (expert, slot) order; rank g receives the chunks in source order.
+ *
+ * Exchange tables of rank `rank` from the pair counts of every rank. Host code only: no CUDA
+ * call, no device memory; every rank computes its own tables from the same all-gathered counts.
+ *   shape      this rank's layer shape (T = this rank's tokens; E, k, C as on every rank)
+ *   loads      host in [G, E]: loads[s][e] = pairs of rank s routed to expert e (this rank's
+ *              row must add up to T * k)
+ *   max_rounds rows of the per-round arrays below
+ *   R          host out: rounds of the job (filled even when it exceeds max_rounds)
+ *   base       host out [E] or NULL: pairs of expert e on the ranks before this one (this rank's
+ *              pairs of e hold the global ranks base[e] .. base[e] + loads[rank][e] - 1)
+ *   send_counts, send_offsets  host out [max_rounds, G] or NULL: rows this rank sends rank g
+ *              in round r, and their position in its packed round-r rows (exclusive prefix)
+ *   recv_counts, recv_offsets  host out [max_rounds, G] or NULL: rows this rank receives from
+ *              rank s in round r, and their position in its received rows (exclusive prefix)
+ *   n_owned    host out [max_rounds, E / G] or NULL: rows of each expert this rank owns in
+ *              round r, from all ranks (at most C)
+ * Returns MOE_ERR_INVALID_ARG for G < 1, E not a multiple of G, a rank out of range, a
+ * negative count, this rank's counts not adding up to T * k, or R > max_rounds with an
+ * array to fill. */
+MOE_API int moe_ep_exchange_plan(const moe_shape_t* shape, int32_t G, int32_t rank, const int32_t* loads,
+                                 int32_t max_rounds, int32_t* R, int32_t* base, int32_t* send_counts,
+                                 int32_t* send_offsets, int32_t* recv_counts, int32_t* recv_offsets,
+                                 int32_t* n_owned);
+
 /* Routing and round plan with no device allocation at all.
  *
  * The pages have no counterpart to this call; it exists for callers that cannot

@@ -9,3 +9,4 @@ from .moe_oracle import (bf16_to_f64, router_logits, select_topk, gates, plan, p
                          forward_rounds, layer)
 from .moe_backward import (silu_grad, expert_backward, gates_backward, router_backward,  # noqa: F401
                            backward, backward_rounds)
+from .moe_ep import owner, ep_plan, ep_forward  # noqa: F401
