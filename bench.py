@@ -300,7 +300,9 @@ def algorithmic_work(w, info, r0, round_np, n_plan=None):
         "router_gemm": ("hbm", (w.T * w.d * 2 + w.E * w.d * 2 + w.T * w.E * 4) if w.router == "gemm" else 0),
         "topk": ("hbm", w.T * w.E * 4 + w.T * w.k * 8),
         "plan": ("hbm", w.T * w.k * 4 * 6),
-        "dispatch": ("hbm", 2 * int(per) * d * 2),
+        # the per-round gate/up GEMMs gather their rows from x; only the pipelined launch's first
+        # round is dispatched into a buffer (x rows in, buffer rows out) before that launch
+        "dispatch": ("hbm", 2 * int(pipe[0].sum()) * d * 2 if len(pipe) else 0),
         "gate_up": ("tensor", 4 * int(per) * d * F),
         "down": ("tensor", 2 * int(per) * F * d),
         "combine": ("hbm", combine_bytes(w, round_np, set(range(r0))) if r0 > 0 else 0),
@@ -318,7 +320,8 @@ def algorithmic_work(w, info, r0, round_np, n_plan=None):
 
 def layer_roofline_s(w, info, round_np, peaks, tensor_tflops, n_plan=None):
     """Lower bound on one step's time from the layer's algorithmic work alone:
-    the bytes of the router GEMM, top-k, plan, dispatch and combine at the HBM peak, plus,
+    the bytes of the router GEMM, top-k, plan, the reads of the pairs' x rows and the combine at
+    the HBM peak, plus,
     for every expert that has rows in a round, the larger of its GEMM time (6 n d d_ff flops
     at the tensor peak) and the time to stream its weights once (6 d d_ff bytes at the HBM
     peak). Returns (seconds, parts)."""
@@ -328,7 +331,8 @@ def layer_roofline_s(w, info, round_np, peaks, tensor_tflops, n_plan=None):
     pt = tensor_tflops * 1e12
     copy_bytes = ((w.T * w.d * 2 + w.E * w.d * 2 + w.T * w.E * 4) if w.router == "gemm" else 0)
     copy_bytes += w.T * w.E * 4 + w.T * w.k * 8 + w.T * w.k * 4 * 6
-    copy_bytes += 2 * int(n.sum()) * d * 2 + combine_bytes(w, round_np)
+    # every pair's x row is read once (the gate/up GEMM gathers it; no dispatch buffer is needed)
+    copy_bytes += int(n.sum()) * d * 2 + combine_bytes(w, round_np)
     t_copy = copy_bytes / bw
     n = np.asarray(n)
     active = n[n > 0].astype(np.float64)

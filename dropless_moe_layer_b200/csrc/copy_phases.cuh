@@ -43,13 +43,22 @@ __device__ __forceinline__ void dispatch_row(const uint4* __restrict__ x, uint4*
 }
 
 // Rows [begin, end) of the round-major row list, spread over `warps` warps (this one is `w`).
+// With dbg (debug bounds checks) a row whose token is not below T or whose destination is not
+// below buf_rows is recorded and skipped.
 __device__ __forceinline__ void dispatch_rows(const uint4* __restrict__ x, uint4* __restrict__ buf,
                                               const int32_t* __restrict__ row_token,
                                               const int32_t* __restrict__ row_dst, int begin, int end,
-                                              int vecs, int w, int warps) {
+                                              int vecs, int w, int warps, int32_t* dbg = nullptr, int T = 0,
+                                              long long buf_rows = 0) {
   const int lane = threadIdx.x & 31;
-  for (int row = begin + w; row < end; row += warps)
-    dispatch_row(x, buf, row_token[row], row_dst[row], vecs, lane);
+  for (int row = begin + w; row < end; row += warps) {
+    const int t = row_token[row], dst = row_dst[row];
+    if (dbg != nullptr && (t < 0 || t >= T || dst < 0 || dst >= buf_rows)) {
+      if (lane == 0) record_bad(dbg, kBadDispatchRow, row);
+      continue;
+    }
+    dispatch_row(x, buf, t, dst, vecs, lane);
+  }
 }
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& q, float (&f)[8]) {
@@ -74,6 +83,10 @@ struct CombineArgs {
   const int32_t* row_off;
   const int32_t* row_start;
   int E;
+  // Debug bounds checks (MOE_FLAG_DEBUG_BOUNDS): the workspace header, else null; a pair whose
+  // expert is not below E or whose buffer row is not below rows_cap makes the token skipped.
+  int32_t* dbg;
+  long long rows_cap;
 };
 
 // One token's pairs in one round, spread over the warp (every lane holds the same scalars;
@@ -123,12 +136,21 @@ __device__ __forceinline__ TokenPairs token_pairs(const CombineArgs& a, const Pa
   tp.s = __shfl_sync(0xffffffffu, my_slot, jp);
   const float g = __shfl_sync(0xffffffffu, my_gate, jp);
   unsigned long long row = 0ull;
-  if (lane < tp.npairs)
+  const bool e_ok = a.dbg == nullptr || (tp.e >= 0 && tp.e < a.E);   // checked before it indexes row_off
+  if (lane < tp.npairs && e_ok)
     row = a.row_off ? static_cast<unsigned long long>(a.row_off[static_cast<size_t>(r) * a.E + tp.e] - a.row_start[r] + tp.s)
                     : static_cast<unsigned long long>(tp.e) * a.C + tp.s;
   tp.prow = row;
   tp.first_row = __shfl_sync(0xffffffffu, row, 0);
   tp.pgate = lane < tp.npairs ? g : 0.f;
+  if (a.dbg != nullptr) {
+    const bool bad = lane < tp.npairs && (!e_ok || tp.s < 0 || row >= static_cast<unsigned long long>(a.rows_cap));
+    const uint32_t any = __ballot_sync(0xffffffffu, bad);
+    if (any) {
+      if (lane == __ffs(any) - 1) record_bad(a.dbg, kBadCombinePair, static_cast<int>(row));
+      tp.npairs = 0;
+    }
+  }
   return tp;
 }
 

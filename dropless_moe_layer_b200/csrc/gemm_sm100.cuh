@@ -149,7 +149,22 @@ struct Phase {
   // of a single [rows, K] operand and output, instead of at row 0 of group g. Null: per group.
   const int32_t* group_row;
   const int32_t* group_row_base;
+  // Fused gather (gate/up of a round): the A rows are not read from a dispatch buffer but
+  // gathered straight from x through the 2-D map `a` (box: 64 columns x 1 row); row i of group
+  // g is x[gather_rows[gather_off[g] + i]] (the round-major row list). Null: tiled A loads.
+  const int32_t* gather_rows;
+  const int32_t* gather_off;
+  // Debug bounds checks (MOE_FLAG_DEBUG_BOUNDS): a group's row count above rows_cap (the buffer
+  // rows a group may hold) is recorded in the header dbg and clamped. rows_cap 0: unchecked.
+  int rows_cap;
+  int32_t* dbg;
 };
+
+// Rows of group g (clamped to rows_cap under the debug bounds checks).
+__device__ __forceinline__ int group_rows(const Phase& p, int g) {
+  const int r = p.rows ? p.rows[g] : p.rows_const;
+  return (p.rows_cap > 0 && r > p.rows_cap) ? p.rows_cap : r;
+}
 
 // Pipeline counters; each role thread uses its own fields, and they persist across phases.
 struct Pipe {
@@ -168,18 +183,27 @@ __device__ __forceinline__ int warp_sum(int v) {
 
 // Warp 0 picks the phase's N width and writes its tile prefix into slot `which`.
 // The caller synchronises the CTA before run_phase.
+// Warp 0 of CTA 0 records groups whose row count is above rows_cap (debug bounds checks).
+__device__ __forceinline__ void check_group_rows(const Phase& p) {
+  if (p.rows_cap <= 0 || p.dbg == nullptr || p.rows == nullptr || blockIdx.x != 0) return;
+  for (int g = threadIdx.x & 31; g < p.groups; g += 32)
+    if (p.rows[g] < 0 || p.rows[g] > p.rows_cap) record_bad(p.dbg, kBadGemmRows, g);
+}
+
 __device__ __forceinline__ void plan_phase(const Smem& s, const Phase& p, int which) {
   if ((threadIdx.x >> 5) != 0) return;
   const int lane = threadIdx.x & 31;
+  check_group_rows(p);
   int mt = 0;
   for (int g = lane; g < p.groups; g += 32) {
-    const int rows = p.rows ? p.rows[g] : p.rows_const;
+    const int rows = group_rows(p, g);
     mt += (rows + BM - 1) / BM;
   }
   mt = warp_sum(mt);
   int wi = p.width_idx;          // chosen by the host when it knows the row counts
   if (wi < 0) {
     int last = -1;
+#pragma unroll
     for (int i = 0; i < 3; ++i) {
       const int w = p.widths[i];
       if (w <= 0 || p.n_total % w != 0) continue;
@@ -191,14 +215,14 @@ __device__ __forceinline__ void plan_phase(const Smem& s, const Phase& p, int wh
     }
     if (wi < 0) wi = last;
   }
-  const int n_tiles = p.n_total / p.widths[wi];
+  const int n_tiles = p.n_total / (wi == 0 ? p.widths[0] : wi == 1 ? p.widths[1] : p.widths[2]);
   int* ts = s.tile_start[which];
   int running = 0;
   for (int g0 = 0; g0 < p.groups; g0 += 32) {
     const int g = g0 + lane;
     int cnt = 0;
     if (g < p.groups) {
-      const int rows = p.rows ? p.rows[g] : p.rows_const;
+      const int rows = group_rows(p, g);
       cnt = ((rows + BM - 1) / BM) * n_tiles;
     }
     int incl = cnt;
@@ -271,12 +295,17 @@ __device__ __forceinline__ void store_bf16(uint32_t tb, int cols, uint16_t* orow
 // Runs the CTA's share of the tiles of the phase planned in slot `which`. Returns when this
 // warp's role work is issued/done (the epilogue warps return after their last store). Every warp
 // leaves converged: a CTA barrier (which requires whole warps) may follow directly.
+// kGather: the phase gathers its A rows (Phase::gather_rows); a separate instantiation, so that the
+// tiled form keeps its register budget.
+template <bool kGather>
 __device__ __forceinline__ void run_phase(const Smem& s, uint32_t tmem_base, const Phase& p, int which,
                                           Pipe& pipe, int32_t* status) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int* ts = s.tile_start[which];
   const int wi = s.width_idx[which];
-  const int width = p.widths[wi];
+  // explicit selects instead of indexing p.widths / p.b with wi: the Phase then stays in registers
+  const int width = wi == 0 ? p.widths[0] : wi == 1 ? p.widths[1] : p.widths[2];
+  const CUtensorMap* const b_map = wi == 0 ? p.b[0] : wi == 1 ? p.b[1] : p.b[2];
   const int bn = p.mode == kSwiGLU ? 2 * width : width;
   const int n_tiles = p.n_total / width;
   const int total = ts[p.groups];
@@ -295,10 +324,63 @@ __device__ __forceinline__ void run_phase(const Smem& s, uint32_t tmem_base, con
     nt = local - mt * n_tiles;
   };
 
-  if (warp == 0) {
+  if (kGather && warp == 0) {
+    // ---------------------------------------------------------------- TMA producer, fused gather
+    // The whole warp produces: lane l gathers rows 4l .. 4l+3 of the A tile (one 4-row TMA
+    // gather per k block, 512 bytes of the tile each), lane 0 also loads the B tile. Every lane
+    // keeps the same pipeline counters.
+    const CUtensorMap* mb = b_map;
+    const uint32_t tx = static_cast<uint32_t>(kABytes + bn * BK * 2);
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      int g, mt, nt;
+      decode(tile, g, mt, nt);
+      const int rows_g = group_rows(p, g);
+      const int first = p.gather_off[g];
+      int tok[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {   // rows past the group's end repeat its first row (never stored)
+        const int i = mt * BM + 4 * lane + q;
+        tok[q] = p.gather_rows[first + (i < rows_g ? i : 0)];
+      }
+      for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&s.empty[pipe.stage]), pipe.phase ^ 1u, s.abort))) {
+          ok = false;
+          break;
+        }
+        const uint32_t sA = smem_addr(s.stage + pipe.stage * stage_bytes);
+        const uint32_t sB = sA + kABytes;
+        const uint32_t fb = smem_addr(&s.full[pipe.stage]);
+        if (lane == 0) mbar_arrive_expect_tx(fb, tx);
+        __syncwarp();
+        tma_gather4_2d(sA + lane * 4 * BK * 2, p.a, fb, kb * BK, tok[0], tok[1], tok[2], tok[3]);
+        if (lane == 0) {
+          if (p.mode == kSwiGLU) {
+            tma_load_3d(sB, mb, fb, kb * BK, nt * width, g);
+            tma_load_3d(sB + width * BK * 2, mb, fb, kb * BK, p.b_second_row + nt * width, g);
+          } else {
+            tma_load_3d(sB, mb, fb, kb * BK, nt * width, g);
+          }
+        }
+        pipe.issued |= 1u << pipe.stage;
+        pipe.issued_parity = (pipe.issued_parity & ~(1u << pipe.stage)) | (pipe.phase << pipe.stage);
+        if (++pipe.stage == nstages) {
+          pipe.stage = 0;
+          pipe.phase ^= 1u;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      atomicOr(status, kStatusTimeoutProducer);
+      *s.abort = 1;
+      for (int i = 0; i < nstages; ++i)   // let issued loads land before shared memory is reused
+        if ((pipe.issued >> i) & 1u) mbar_wait(smem_addr(&s.full[i]), (pipe.issued_parity >> i) & 1u, nullptr);
+    }
+    __syncwarp();
+  } else if (warp == 0) {
     if (lane == 0) {
     // ---------------------------------------------------------------- TMA producer
-    const CUtensorMap* mb = p.b[wi];
+    const CUtensorMap* mb = b_map;
     const uint32_t tx = static_cast<uint32_t>(kABytes + bn * BK * 2);
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
@@ -399,7 +481,7 @@ __device__ __forceinline__ void run_phase(const Smem& s, uint32_t tmem_base, con
       }
       tc_fence_after();
       const int row = mt * BM + q * 32 + lane;
-      const int rows_g = p.rows ? p.rows[g] : p.rows_const;
+      const int rows_g = group_rows(p, g);
       const bool valid = row < rows_g;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(pipe.acc * kAccCols);
@@ -429,6 +511,260 @@ __device__ __forceinline__ void run_phase(const Smem& s, uint32_t tmem_base, con
       }
       tc_fence_before();
       mbar_arrive(smem_addr(&s.tempty[pipe.acc]));
+      pipe.acc ^= 1;
+      if (pipe.acc == 0) pipe.acc_phase ^= 1u;
+    }
+    __syncwarp();
+  }
+}
+
+// ================================================================ CTA-pair form (cta_group::2)
+//
+// The same grouped GEMM on tiles of 256 rows x 256 columns shared by the two CTAs of a cluster
+// of two. CTA c of the pair loads A rows [128 c, 128 c + 128) of the tile and B rows
+// [128 c, 128 c + 128) of its 256 (SwiGLU: c = 0 the tile's 128 gate rows, c = 1 the same 128
+// up rows; Bf16Out: the two halves of the 256 output columns) into its own shared memory; the
+// leader's one thread issues the M = 256, N = 256 MMA for both, which reads the peer's halves
+// at the same offsets and leaves accumulator rows [128 c, 128 c + 128) in CTA c's TMEM. Per
+// k block a CTA's shared memory then holds 32 KB for 2 x 128 x 256 x 64 flops, half the bytes
+// per flop of the single-CTA tile, which is what lets the tensor pipe run near its peak: the
+// single-CTA 128 x 256 tile needs more shared-memory bandwidth (TMA writes plus MMA reads)
+// than an SM has. No load is multicast.
+//
+// Barriers: full[s] lives in the leader (one arrive with the pair's bytes, both CTAs' TMA
+// loads complete on it); empty[s] and tfull[a] in both CTAs (the leader's commit arrives on
+// both); tempty[a] in the leader (one arrive per epilogue warp of either CTA: 8).
+constexpr int kPairRows = 2 * BM;        // rows of a pair tile
+constexpr int kPairBn = 256;             // MMA N of a pair tile
+constexpr int kPairBHalf = kPairBn / 2;  // B rows per CTA
+constexpr int kPairStageBytes = kABytes + kPairBHalf * BK * 2;   // 32 KB
+constexpr int kPairStages = kRingBytes / kPairStageBytes;        // 6
+static_assert(kPairStages <= kMaxStages, "pair ring stages");
+constexpr int kEpiWarpsPair = 8;         // arrivals on the leader's tempty per tile
+
+// Set-up of both CTAs of a pair: barriers (thread 0 of each), the pair's TMEM (warp 1 of each),
+// then a cluster barrier, so that no CTA signals its peer before the peer's barriers exist.
+__device__ __forceinline__ uint32_t setup_pair(const Smem& s) {
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kMaxStages; ++i) {
+      mbar_init(smem_addr(&s.full[i]), 1);
+      mbar_init(smem_addr(&s.empty[i]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_addr(&s.tfull[a]), 1);
+      mbar_init(smem_addr(&s.tempty[a]), kEpiWarpsPair);
+    }
+    mbar_init(smem_addr(s.drain), 1);
+    *s.abort = 0;
+    mbar_fence_init();
+  }
+  __syncwarp();
+  if ((threadIdx.x >> 5) == 1) {
+    tmem_alloc_pair(smem_addr(s.tmem_holder), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  return *s.tmem_holder;
+}
+
+// Tear-down of both CTAs once every role of this CTA is done: a cluster barrier (no peer still
+// reads this CTA's shared memory or signals its barriers), then the pair's TMEM is freed.
+__device__ __forceinline__ void release_tmem_pair(uint32_t tmem_base) {
+  tc_fence_before();
+  cluster_sync();
+  if ((threadIdx.x >> 5) == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
+// Warp 0 writes the phase's tile prefix over 256-row blocks into slot `which` (fixed width).
+__device__ __forceinline__ void plan_phase_pair(const Smem& s, const Phase& p, int which, int width) {
+  if ((threadIdx.x >> 5) != 0) return;
+  const int lane = threadIdx.x & 31;
+  check_group_rows(p);
+  const int n_tiles = p.n_total / width;
+  int* ts = s.tile_start[which];
+  int running = 0;
+  for (int g0 = 0; g0 < p.groups; g0 += 32) {
+    const int g = g0 + lane;
+    int cnt = 0;
+    if (g < p.groups) {
+      const int rows = group_rows(p, g);
+      cnt = ((rows + kPairRows - 1) / kPairRows) * n_tiles;
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (g < p.groups) ts[g] = running + incl - cnt;
+    running += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) ts[p.groups] = running;
+  __syncwarp();
+}
+
+// The pair's share of the tiles: pair `pair` of `pairs` takes tiles pair, pair + pairs, ...
+// `width`: SwiGLU gate columns per tile (128; the B tile is those gate rows and the same up
+// rows), Bf16Out output columns (256). Modes SwiGLU and Bf16Out only.
+__device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base, const Phase& p, int which,
+                                               int width, int pair, int pairs, Pipe& pipe, int32_t* status) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t cta = cluster_rank();
+  const int* ts = s.tile_start[which];
+  const int n_tiles = p.n_total / width;
+  const int total = ts[p.groups];
+  auto decode = [&](int tile, int& g, int& mp, int& nt) {
+    int lo = 0, hi = p.groups - 1;   // largest g with ts[g] <= tile
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (ts[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    g = lo;
+    const int local = tile - ts[g];
+    mp = local / n_tiles;
+    nt = local - mp * n_tiles;
+  };
+  // B rows of this CTA's half of a tile
+  auto b_row = [&](int nt) {
+    return p.mode == kSwiGLU ? static_cast<int>(cta) * p.b_second_row + nt * width
+                             : nt * width + static_cast<int>(cta) * kPairBHalf;
+  };
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer (both CTAs)
+    const uint32_t tx = 2u * kPairStageBytes;   // the pair's bytes per stage, counted by the leader
+    bool ok = true;
+    const bool gather = p.gather_rows != nullptr;
+    for (int tile = pair; ok && tile < total; tile += pairs) {
+      int g, mp, nt;
+      decode(tile, g, mp, nt);
+      const int row0 = mp * kPairRows + static_cast<int>(cta) * BM;   // this CTA's first A row
+      int tok[4] = {0, 0, 0, 0};
+      if (gather) {
+        const int rows_g = group_rows(p, g);
+        const int first = p.gather_off[g];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {   // rows past the group's end repeat its first row (never stored)
+          const int i = row0 + 4 * lane + q;
+          tok[q] = p.gather_rows[first + (i < rows_g ? i : 0)];
+        }
+      }
+      int a_row = row0, a_grp = g;
+      if (p.group_row) {
+        a_row += p.group_row[g] - *p.group_row_base;
+        a_grp = 0;
+      }
+      for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&s.empty[pipe.stage]), pipe.phase ^ 1u, s.abort))) {
+          ok = false;
+          break;
+        }
+        const uint32_t sA = smem_addr(s.stage + pipe.stage * kPairStageBytes);
+        const uint32_t sB = sA + kABytes;
+        const uint32_t fb_local = smem_addr(&s.full[pipe.stage]);
+        const uint32_t fb = peer_addr(fb_local, 0);   // the leader's full barrier
+        if (cta == 0 && lane == 0) mbar_arrive_expect_tx(fb_local, tx);
+        __syncwarp();
+        if (gather) {
+          tma_gather4_2d_pair(sA + lane * 4 * BK * 2, p.a, fb, kb * BK, tok[0], tok[1], tok[2], tok[3]);
+        } else if (lane == 0) {
+          tma_load_3d_pair(sA, p.a, fb, kb * BK, a_row, a_grp);
+        }
+        if (lane == 0) tma_load_3d_pair(sB, p.b[0], fb, kb * BK, b_row(nt), g);
+        pipe.issued |= 1u << pipe.stage;
+        if (++pipe.stage == kPairStages) {
+          pipe.stage = 0;
+          pipe.phase ^= 1u;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      atomicOr(status, kStatusTimeoutProducer);
+      *s.abort = 1;
+      // loads already issued complete on the leader's barriers, which this CTA cannot wait on:
+      // give them time to land before the pair's shared memory is released
+      const uint64_t t0 = global_timer_ns();
+      while (global_timer_ns() - t0 < 200000ull) {
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && cta == 0) {
+    // ---------------------------------------------------------------- MMA issuer (leader only)
+    const uint32_t idesc = idesc_bf16_f32(kPairRows, kPairBn);
+    bool ok = true;
+    for (int tile = pair; ok && tile < total; tile += pairs) {
+      if (!mbar_wait(smem_addr(&s.tempty[pipe.acc]), pipe.acc_phase ^ 1u, s.abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(pipe.acc * kAccCols);
+      for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+        if (!mbar_wait(smem_addr(&s.full[pipe.stage]), pipe.phase, s.abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sA = smem_addr(s.stage + pipe.stage * kPairStageBytes);
+        const uint64_t adesc = smem_desc_sw128(sA);
+        const uint64_t bdesc = smem_desc_sw128(sA + kABytes);
+#pragma unroll
+        for (int kk = 0; kk < BK / UMMA_K; ++kk)
+          mma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+        mma_commit_pair(smem_addr(&s.empty[pipe.stage]), 3);
+        if (++pipe.stage == kPairStages) {
+          pipe.stage = 0;
+          pipe.phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      mma_commit_pair(smem_addr(&s.tfull[pipe.acc]), 3);
+      pipe.acc ^= 1;
+      if (pipe.acc == 0) pipe.acc_phase ^= 1u;
+    }
+    if (!ok) {
+      atomicOr(status, kStatusTimeoutMma);
+      *s.abort = 1;
+      mma_commit_pair(smem_addr(s.drain), 1);   // wait for every MMA already issued
+      mbar_wait(smem_addr(s.drain), 0, nullptr);
+    }
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    for (int tile = pair; tile < total; tile += pairs) {
+      int g, mp, nt;
+      decode(tile, g, mp, nt);
+      const bool ready = __all_sync(0xffffffffu, mbar_wait(smem_addr(&s.tfull[pipe.acc]), pipe.acc_phase, s.abort));
+      if (!ready) {
+        if (lane == 0) atomicOr(status, kStatusTimeoutEpilogue);
+        *s.abort = 1;
+        break;
+      }
+      tc_fence_after();
+      const int row = mp * kPairRows + static_cast<int>(cta) * BM + q * 32 + lane;
+      const int rows_g = group_rows(p, g);
+      const bool valid = row < rows_g;
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                          static_cast<uint32_t>(pipe.acc * kAccCols);
+      const long long orow_off = p.group_row
+                                     ? static_cast<long long>(p.group_row[g] - *p.group_row_base + row) * p.out_ld
+                                     : g * p.out_group_stride + static_cast<long long>(row) * p.out_ld;
+      uint16_t* orow = static_cast<uint16_t*>(p.out) + orow_off + nt * width;
+      if (p.mode == kSwiGLU)
+        store_swiglu(tb, width, orow, valid);
+      else
+        store_bf16(tb, kPairBn, orow, valid);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(peer_addr(smem_addr(&s.tempty[pipe.acc]), 0));
       pipe.acc ^= 1;
       if (pipe.acc == 0) pipe.acc_phase ^= 1u;
     }

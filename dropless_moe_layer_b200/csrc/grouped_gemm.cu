@@ -33,6 +33,9 @@ struct SideArgs {
   int vecs;
   copy::CombineArgs comb;      // combine
   int by_rows;
+  int32_t* dbg;                // debug bounds checks: the workspace header, else null
+  int T;
+  long long buf_rows;
 };
 
 __device__ __forceinline__ void side_work(const SideArgs& sa) {
@@ -40,12 +43,18 @@ __device__ __forceinline__ void side_work(const SideArgs& sa) {
   const int warps = gridDim.x * kCopyWarps;
   if (sa.kind == kSideDispatch) {
     copy::dispatch_rows(sa.x, sa.buf, sa.row_token, sa.row_dst, sa.row_start[sa.r], sa.row_start[sa.r + 1],
-                        sa.vecs, cw, warps);
+                        sa.vecs, cw, warps, sa.dbg, sa.T, sa.buf_rows);
   } else if (sa.kind == kSideCombine) {
     if (sa.by_rows) {
       const int begin = sa.row_start[sa.r], end = sa.row_start[sa.r + 1];
-      for (int row = begin + cw; row < end; row += warps)
-        copy::combine_token(sa.comb, sa.row_token[row], sa.r, sa.row_dst[row]);
+      for (int row = begin + cw; row < end; row += warps) {
+        const int t = sa.row_token[row];
+        if (sa.dbg != nullptr && (t < 0 || t >= sa.T)) {
+          if ((threadIdx.x & 31) == 0) record_bad(sa.dbg, kBadCombineToken, row);
+          continue;
+        }
+        copy::combine_token(sa.comb, t, sa.r, sa.row_dst[row]);
+      }
     } else {
       for (int t = cw; t < sa.comb.T; t += warps) copy::combine_token(sa.comb, t, sa.r);
     }
@@ -70,8 +79,12 @@ struct KernelArgs {
   int32_t* status;
   const int32_t* group_row;        // pooled rows (see Phase), or null
   const int32_t* group_row_base;
+  const int32_t* gather_rows;      // fused gather of the A rows (see Phase), or null
+  const int32_t* gather_off;
+  int rows_cap;                    // debug bounds checks (see Phase): 0 = unchecked
 };
 
+template <bool kGather>
 __global__ void __launch_bounds__(kLaunchThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb0,
                         const __grid_constant__ CUtensorMap tb1, const __grid_constant__ CUtensorMap tb2,
@@ -104,6 +117,10 @@ __global__ void __launch_bounds__(kLaunchThreads, 1)
   p.n_valid = args.n_valid;
   p.group_row = args.group_row;
   p.group_row_base = args.group_row_base;
+  p.gather_rows = args.gather_rows;
+  p.gather_off = args.gather_off;
+  p.rows_cap = args.rows_cap;
+  p.dbg = args.rows_cap > 0 ? args.status - kHdrStatus : nullptr;
   plan_phase(s, p, 0);              // reads only the row counts (plan data)
   __syncthreads();
   // Everything above overlaps the previous kernel; the operands, and the output buffer that
@@ -112,13 +129,65 @@ __global__ void __launch_bounds__(kLaunchThreads, 1)
   pdl_trigger_early();
   Pipe pipe;
   if (threadIdx.x < kThreads)
-    run_phase(s, tmem, p, 0, pipe, args.status);
+    run_phase<kGather>(s, tmem, p, 0, pipe, args.status);
   else
     side_work(side);
   tc_fence_before();
   __syncthreads();
   pdl_trigger_late();               // after every role of this CTA is done
   release_tmem(tmem);
+}
+
+// The CTA-pair form (gemm_sm100.cuh, run_phase_pair), launched as clusters of two CTAs: 256 x
+// 256 tiles, one B map with 128-row boxes, a fixed width (SwiGLU 128 gate columns, Bf16Out 256).
+__global__ void __launch_bounds__(kLaunchThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
+                             const KernelArgs args, const SideArgs side, int width) {
+  extern __shared__ uint8_t smem_raw[];
+  const Smem s = carve(smem_raw);
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&ta);
+    tma_prefetch_desc(&tb);
+  }
+  const uint32_t tmem = setup_pair(s);
+  Phase p;
+  p.mode = args.mode;
+  p.a = &ta;
+  p.b[0] = &tb;
+  p.b[1] = &tb;
+  p.b[2] = &tb;
+  for (int i = 0; i < 3; ++i) p.widths[i] = args.widths[i];
+  p.width_idx = 0;
+  p.rows = args.rows;
+  p.rows_const = args.rows_const;
+  p.groups = args.groups;
+  p.num_k_blocks = args.num_k_blocks;
+  p.n_total = args.n_total;
+  p.b_second_row = args.b_second_row;
+  p.out = args.out;
+  p.out_group_stride = args.out_group_stride;
+  p.out_ld = args.out_ld;
+  p.bias = args.bias;
+  p.n_valid = args.n_valid;
+  p.group_row = args.group_row;
+  p.group_row_base = args.group_row_base;
+  p.gather_rows = args.gather_rows;
+  p.gather_off = args.gather_off;
+  p.rows_cap = args.rows_cap;
+  p.dbg = args.rows_cap > 0 ? args.status - kHdrStatus : nullptr;
+  plan_phase_pair(s, p, 0, width);
+  __syncthreads();
+  grid_dependency_wait();
+  pdl_trigger_early();
+  Pipe pipe;
+  if (threadIdx.x < kThreads)
+    run_phase_pair(s, tmem, p, 0, width, blockIdx.x >> 1, gridDim.x >> 1, pipe, args.status);
+  else
+    side_work(side);
+  tc_fence_before();
+  __syncthreads();
+  pdl_trigger_late();
+  release_tmem_pair(tmem);
 }
 
 // ------------------------------------------------------------------ tensor maps
@@ -141,15 +210,17 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// groups == 0 encodes a 2-D map [rows][inner] (the row-gather form: box_rows must be 1).
 static cudaError_t encode_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
                               uint64_t groups, uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
+  const cuuint32_t rank = groups == 0 ? 2 : 3;
   const cuuint64_t dims[3] = {inner, rows, groups};
   const cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(BK), box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult res = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+  const CUresult res = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -246,16 +317,93 @@ static cudaError_t run(const CUtensorMap& a, const CUtensorMap* b, const KernelA
   cudaGetDevice(&dev);
   const uint64_t bit = 1ull << (dev & 63);
   if (!(configured.load() & bit)) {
-    const cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
   launch_begin(kind, stream);
   // with side work every SM takes part in the copy; otherwise one CTA per tile, at most one per SM
   const int grid = side.kind != kSideNone ? num_sms() : static_cast<int>(tiles < num_sms() ? tiles : num_sms());
-  const cudaError_t err = launch_pdl(grouped_gemm_kernel, dim3(grid), dim3(kLaunchThreads), kSmemBytes, stream,
-                                     a, b[0], b[1], b[2], args, side);
+  const cudaError_t err = args.gather_rows
+                              ? launch_pdl(grouped_gemm_kernel<true>, dim3(grid), dim3(kLaunchThreads), kSmemBytes,
+                                           stream, a, b[0], b[1], b[2], args, side)
+                              : launch_pdl(grouped_gemm_kernel<false>, dim3(grid), dim3(kLaunchThreads), kSmemBytes,
+                                           stream, a, b[0], b[1], b[2], args, side);
+  launch_end(kind, stream);
+  return err;
+}
+
+#ifndef MOE_GEMM_PAIR
+#define MOE_GEMM_PAIR 1   // 0: never use the CTA-pair form
+#endif
+
+// Clusters of two that fit on the device at once (one CTA per SM), per device ordinal.
+static int pair_clusters() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  dev &= 63;
+  int v = cached[dev].load();
+  if (v > 0) return v;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (num_sms() / 2));
+  cfg.blockDim = dim3(kLaunchThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaFuncSetAttribute(grouped_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+          cudaSuccess ||
+      cudaOccupancyMaxActiveClusters(&n, grouped_gemm_pair_kernel, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = -1;   // no pair form on this device
+  }
+  cached[dev].store(n);
+  return n;
+}
+
+// Whether a round's GEMM runs in the CTA-pair form: its 256-row tiles must keep every cluster
+// busy and pad at most kPairPadding more rows than the 128-row tiles of the single-CTA form.
+static bool use_pair(const int32_t* n_host, int groups, int n_total, int width) {
+  if (!MOE_GEMM_PAIR || n_host == nullptr || n_total % width != 0) return false;
+  long long pair_tiles = 0, rows_pair = 0, rows_single = 0;
+  for (int g = 0; g < groups; ++g) {
+    pair_tiles += (n_host[g] + kPairRows - 1) / kPairRows;
+    rows_pair += static_cast<long long>((n_host[g] + kPairRows - 1) / kPairRows) * kPairRows;
+    rows_single += static_cast<long long>((n_host[g] + BM - 1) / BM) * BM;
+  }
+  pair_tiles *= n_total / width;
+  const int clusters = pair_clusters();
+  return clusters > 0 && pair_tiles >= clusters && rows_pair * 100 <= rows_single * 115;
+}
+
+static cudaError_t run_pair(const CUtensorMap& a, const CUtensorMap& b, const KernelArgs& args, int width,
+                            const SideArgs& side, int kind, cudaStream_t stream) {
+  const int clusters = pair_clusters();   // every cluster takes part; the device counts the tiles
+  launch_begin(kind, stream);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(kLaunchThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = MOE_PDL;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel, a, b, args, side, width);
   launch_end(kind, stream);
   return err;
 }
@@ -296,7 +444,11 @@ static gemm::SideArgs make_side(const RoundCopy* copy) {
   sd.vecs = copy->d / 8;
   sd.comb = copy::CombineArgs{copy->out, copy->y, copy->idx, copy->gate, copy->round, copy->slot,
                               copy->T, copy->k, copy->C, copy->d, copy->row_off,
-                              copy->row_off ? copy->row_start : nullptr, copy->E};
+                              copy->row_off ? copy->row_start : nullptr, copy->E, copy->dbg,
+                              static_cast<long long>(copy->E) * copy->C};
+  sd.dbg = copy->dbg;
+  sd.T = copy->T;
+  sd.buf_rows = static_cast<long long>(copy->E) * copy->C;
   sd.by_rows = copy->rows < copy->T ? 1 : 0;
   return sd;
 }
@@ -304,10 +456,14 @@ static gemm::SideArgs make_side(const RoundCopy* copy) {
 cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint16_t* h,
                            const int32_t* n_dev, const int32_t* n_host, int E, int C, int d, int F,
                            int32_t* status, const RoundCopy* copy, const int32_t* group_row,
-                           const int32_t* group_row_base, cudaStream_t stream) {
+                           const int32_t* group_row_base, const GatherA* gather, cudaStream_t stream,
+                           int rows_cap) {
   CUtensorMap ma, mb[3];
   cudaError_t e = make_gate_up_maps(buf, w_gate_up, E, C, d, F, &ma, mb, group_row != nullptr);
   if (e != cudaSuccess) return e;
+  if (gather != nullptr) {   // A rows straight from x: a 2-D map whose box is one row high
+    if ((e = gemm::make_map(&ma, gather->x, d, gather->T, 0, 1)) != cudaSuccess) return e;
+  }
   gemm::KernelArgs a{};
   a.mode = gemm::kSwiGLU;
   for (int i = 0; i < 3; ++i) a.widths[i] = kGateUpWidths[i];
@@ -322,6 +478,11 @@ cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint1
   a.status = status;
   a.group_row = group_row;
   a.group_row_base = group_row_base;
+  a.gather_rows = gather ? gather->row_token : nullptr;
+  a.gather_off = gather ? gather->row_off : nullptr;
+  a.rows_cap = rows_cap;
+  if (gemm::use_pair(n_host, E, F, 128))   // mb[0]: 128-row boxes of W1 and of W3
+    return gemm::run_pair(ma, mb[0], a, 128, make_side(copy), kKindGateUp, stream);
   const long long tiles = gemm::choose_width(n_host, E, 0, F, a);
   return gemm::run(ma, mb, a, tiles, make_side(copy), kKindGateUp, stream);
 }
@@ -329,7 +490,7 @@ cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint1
 cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out, const int32_t* n_dev,
                         const int32_t* n_host, int E, int C, int d, int F, int32_t* status,
                         const RoundCopy* copy, const int32_t* group_row, const int32_t* group_row_base,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, int rows_cap) {
   CUtensorMap ma, mb[3];
   cudaError_t e = make_down_maps(h, w_down, E, C, d, F, &ma, mb, group_row != nullptr);
   if (e != cudaSuccess) return e;
@@ -346,6 +507,12 @@ cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out
   a.status = status;
   a.group_row = group_row;
   a.group_row_base = group_row_base;
+  a.rows_cap = rows_cap;
+  if (gemm::use_pair(n_host, E, d, gemm::kPairBn)) {   // each CTA loads 128 of the tile's 256 W2 rows
+    CUtensorMap mb_half;
+    if ((e = gemm::make_map(&mb_half, w_down, F, d, E, gemm::kPairBHalf)) != cudaSuccess) return e;
+    return gemm::run_pair(ma, mb_half, a, gemm::kPairBn, make_side(copy), kKindDown, stream);
+  }
   const long long tiles = gemm::choose_width(n_host, E, 0, d, a);
   return gemm::run(ma, mb, a, tiles, make_side(copy), kKindDown, stream);
 }

@@ -38,6 +38,8 @@ enum : int {
   kStatusTimeoutMma = 2,
   kStatusTimeoutEpilogue = 4,
   kStatusTimeoutPipeline = 8,   // a dependency wait of the pipelined-rounds kernel gave up
+  kStatusBounds = 16,           // a debug bounds check failed (MOE_FLAG_DEBUG_BOUNDS)
+  kStatusCanary = 32,           // a workspace guard word was overwritten (MOE_FLAG_DEBUG_BOUNDS)
 };
 
 // Header words inside the workspace.
@@ -46,9 +48,28 @@ enum : int {
   kHdrMaxLoad = 1,
   kHdrStatus = 2,
   kHdrScanDone = 3,   // planner: expert scans finished (the last one finalizes the plan)
+  kHdrBadKind = 4,    // first failed debug check: what failed (BadKind), 0 = none
+  kHdrBadValue = 5,   // ... and the offending index or guard number
   kHdrLoad = 64,      // copy of load[0..E-1], so one small copy brings the plan summary home
   kHdrWords = 64 + 256,
 };
+
+// What a failed debug check was checking (header word kHdrBadKind).
+enum BadKind : int {
+  kBadPlanPair = 1,      // planner: a pair's expert, round or row position out of range
+  kBadDispatchRow = 2,   // dispatch: a row's source token or destination row out of range
+  kBadCombinePair = 3,   // combine: a pair's expert or buffer row out of range
+  kBadCombineToken = 4,  // combine: a row's token out of range
+  kBadGemmRows = 5,      // GEMM: an expert's row count above the buffer's rows
+  kBadCanary = 6,        // a guard after a workspace region was overwritten (value: guard number)
+};
+
+// With MOE_FLAG_DEBUG_BOUNDS the kernels get the workspace header (else null) and check every
+// plan index before they use it; a failed check lands here and the access is skipped. Never traps.
+__device__ __forceinline__ void record_bad(int32_t* hdr, int kind, int value) {
+  atomicOr(hdr + kHdrStatus, kind == kBadCanary ? kStatusCanary : kStatusBounds);
+  if (atomicCAS(hdr + kHdrBadKind, 0, kind) == 0) atomicExch(hdr + kHdrBadValue, value);
+}
 
 constexpr int kPlanTokensPerBlock = 256;
 #define MOE_MAX_E_PLAN 256
@@ -118,14 +139,18 @@ struct PlanBuffers {
   int32_t* sync;          // pipelined-rounds counters to zero ([sync_words]), or null
   long long sync_words;
   int borrow;             // 1: capacity borrowing (rows packed per round, n[r][e] may exceed C)
+  int32_t* dbg;           // the header when MOE_FLAG_DEBUG_BOUNDS is set, else null
 };
 cudaError_t launch_plan(const PlanBuffers& b, int T, int k, int E, int C, int max_rounds,
                         cudaStream_t stream);
 
 // ---- dispatch / combine (dispatch_combine.cu)
+// dbg: the workspace header when MOE_FLAG_DEBUG_BOUNDS is set (row checks against T tokens and
+// buf_rows buffer rows), else null.
 cudaError_t launch_dispatch(const uint16_t* x, uint16_t* buf, const int32_t* row_start,
                             const int32_t* row_token, const int32_t* row_dst, int r, int rows,
-                            int d, cudaStream_t stream);
+                            int d, cudaStream_t stream, int32_t* dbg = nullptr, int T = 0,
+                            long long buf_rows = 0);
 // rows: rows of round r (host copy); the kernel walks the round's rows instead of all T
 // tokens when there are fewer of them.
 // row_off: pooled round rows (capacity borrowing: pair (e, slot) of round r at buffer row
@@ -133,7 +158,18 @@ cudaError_t launch_dispatch(const uint16_t* x, uint16_t* buf, const int32_t* row
 cudaError_t launch_combine(const uint16_t* buf, float* y, const int32_t* idx, const float* gate,
                            const int32_t* round, const int32_t* slot, const int32_t* row_start,
                            const int32_t* row_token, const int32_t* row_dst, int T, int k, int C, int d,
-                           int r, int rows, const int32_t* row_off, int E, cudaStream_t stream);
+                           int r, int rows, const int32_t* row_off, int E, cudaStream_t stream,
+                           int32_t* dbg = nullptr);
+
+// Guard words after the workspace regions (MOE_FLAG_DEBUG_BOUNDS): fill writes the pattern into
+// every guard; check compares it and records the first guard found changed.
+constexpr int kMaxGuards = 32;
+constexpr int kGuardBytes = 256;
+struct GuardList {
+  int n;
+  unsigned long long off[kMaxGuards];   // byte offsets of the guards inside the workspace
+};
+cudaError_t launch_guards(uint8_t* ws, const GuardList& g, int check, int32_t* hdr, cudaStream_t stream);
 
 // ---- grouped GEMMs (grouped_gemm.cu)
 // gate_up: h[e][s] = bf16(silu(buf[e][s] W1_e^T) * (buf[e][s] W3_e^T)), s < n_dev[e]
@@ -157,8 +193,21 @@ struct RoundCopy {
   int T, k, C, d;
   const int32_t* row_off;    // pooled round rows (capacity borrowing), or null
   int E;
+  int32_t* dbg;              // the header when MOE_FLAG_DEBUG_BOUNDS is set, else null
 };
 
+// Fused gather of a gate/up GEMM's A rows: row i of expert e's rows in the round is
+// x[row_token[row_off[e] + i]] (row_off: the round's row of the row_off table), read by TMA row
+// gathers instead of from the dispatch buffer, which the round then never needs.
+struct GatherA {
+  const uint16_t* x;         // [T, d] bf16
+  int T;
+  const int32_t* row_token;  // the round-major row list's source tokens
+  const int32_t* row_off;    // [E]: position of expert e's first row of the round in the list
+};
+
+// rows_cap > 0 (debug bounds checks): an expert's device row count above it is recorded in the
+// header and clamped.
 // n_dev: rows per expert this round on the device (read by the kernel); n_host: the same on
 // the host (picks the tile width and the grid). copy: optional side copy step, or null.
 // group_row / group_row_base: pooled round rows (capacity borrowing: expert e's rows start at
@@ -166,12 +215,13 @@ struct RoundCopy {
 cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint16_t* h,
                            const int32_t* n_dev, const int32_t* n_host, int E, int C, int d, int F,
                            int32_t* status, const RoundCopy* copy, const int32_t* group_row,
-                           const int32_t* group_row_base, cudaStream_t stream);
+                           const int32_t* group_row_base, const GatherA* gather, cudaStream_t stream,
+                           int rows_cap = 0);
 // down: out[e][s] = bf16(h[e][s] W2_e^T), s < n_dev[e]
 cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out, const int32_t* n_dev,
                         const int32_t* n_host, int E, int C, int d, int F, int32_t* status,
                         const RoundCopy* copy, const int32_t* group_row, const int32_t* group_row_base,
-                        cudaStream_t stream);
+                        cudaStream_t stream, int rows_cap = 0);
 
 // ---- pipelined rounds (round_pipeline.cu)
 // Rounds [r0, R) of the layer in one persistent launch (one CTA per SM): dispatch, gate/up

@@ -76,8 +76,9 @@ namespace {
 int check_shape(const moe_shape_t* s) {
   if (s == nullptr) return MOE_ERR_INVALID_ARG;
   if (s->flags & ~static_cast<uint32_t>(MOE_FLAG_RENORM_TOPK | MOE_FLAG_PER_ROUND | MOE_FLAG_PIPELINE_ALL |
-                                        MOE_FLAG_BORROW))
+                                        MOE_FLAG_BORROW | MOE_FLAG_DEBUG_BOUNDS))
     return MOE_ERR_INVALID_ARG;
+  if ((s->flags & MOE_FLAG_DEBUG_BOUNDS) && (s->flags & MOE_FLAG_PIPELINE_ALL)) return MOE_ERR_INVALID_ARG;
   if ((s->flags & MOE_FLAG_PER_ROUND) && (s->flags & MOE_FLAG_PIPELINE_ALL)) return MOE_ERR_INVALID_ARG;
   if ((s->flags & MOE_FLAG_BORROW) && (s->flags & MOE_FLAG_PIPELINE_ALL)) return MOE_ERR_INVALID_ARG;
   if (s->T < 0 || s->E < 1 || s->E > MOE_MAX_EXPERTS || s->k < 1 || s->k > MOE_MAX_TOPK ||
@@ -95,12 +96,22 @@ int check_shape(const moe_shape_t* s) {
 
 int max_rounds_of(const moe_shape_t* s) { return s->T == 0 ? 0 : (s->T + s->C - 1) / s->C; }
 
-void make_layout(const moe_shape_t* s, moe_workspace_layout_t* L) {
+bool debug_bounds(const moe_shape_t* s) { return (s->flags & MOE_FLAG_DEBUG_BOUNDS) != 0; }
+
+// With MOE_FLAG_DEBUG_BOUNDS every region is followed by a guard of kGuardBytes (listed in
+// *guards when given), which moe_plan fills and moe_device_status checks.
+void make_layout(const moe_shape_t* s, moe_workspace_layout_t* L, GuardList* guards = nullptr) {
   std::memset(L, 0, sizeof(*L));
   size_t off = 0;
+  const bool dbg = debug_bounds(s);
+  if (guards) guards->n = 0;
   auto take = [&](long long bytes) {
     const size_t o = off;
     off += (static_cast<size_t>(bytes) + 255) & ~static_cast<size_t>(255);
+    if (dbg) {
+      if (guards && guards->n < kMaxGuards) guards->off[guards->n++] = off;
+      off += kGuardBytes;
+    }
     return o;
   };
   const long long T = s->T, E = s->E, k = s->k, C = s->C;
@@ -125,7 +136,7 @@ void make_layout(const moe_shape_t* s, moe_workspace_layout_t* L) {
   L->out = take(E * C * s->d * 2);
   L->mb_prefix = take(static_cast<long long>(mr) * (E + 1) * 4);
   L->sync = take(pipe_sync_words(s->E, s->C) * 4);
-  if (!(s->flags & (MOE_FLAG_PER_ROUND | MOE_FLAG_BORROW))) {   // second buffer set of the pipelined launch
+  if (!(s->flags & (MOE_FLAG_PER_ROUND | MOE_FLAG_BORROW | MOE_FLAG_DEBUG_BOUNDS))) {   // pipelined launch's 2nd set
     L->buf2 = take(E * C * s->d * 2);
     L->h2 = take(E * C * s->d_ff * 2);
     L->out2 = take(E * C * s->d * 2);
@@ -162,6 +173,8 @@ int check_device() {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+bool borrowing(const moe_shape_t* s);
+
 // Common argument checks of the calls that run a plan (no CUDA call).
 int check_plan_args(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
                     moe_workspace_layout_t* L) {
@@ -174,6 +187,21 @@ int check_plan_args(const moe_shape_t* shape, const moe_plan_info_t* info, void*
   if (info->R < 0 || info->R > L->max_rounds) return MOE_ERR_INVALID_ARG;
   // the plan was made for this kind of plan (with or without borrowing)
   if ((info->plan_flags ^ shape->flags) & MOE_FLAG_BORROW) return MOE_ERR_INVALID_ARG;
+  if (debug_bounds(shape)) {
+    // debug bounds checks, on the host before any launch: the plan summary must be one that the
+    // planner can have produced for this shape
+    long long sum = 0;
+    int max_load = 0;
+    for (int e = 0; e < shape->E; ++e) {
+      if (info->load[e] < 0 || info->load[e] > shape->T) return MOE_ERR_INVALID_ARG;
+      sum += info->load[e];
+      max_load = info->load[e] > max_load ? info->load[e] : max_load;
+    }
+    if (sum != static_cast<long long>(shape->T) * shape->k || max_load != info->max_load) return MOE_ERR_INVALID_ARG;
+    const int r_own = (max_load + shape->C - 1) / shape->C;   // rounds without borrowing
+    if (!borrowing(shape) ? info->R != r_own : (info->R > r_own || (shape->T > 0 && info->R < 1)))
+      return MOE_ERR_INVALID_ARG;
+  }
   return MOE_OK;
 }
 
@@ -222,6 +250,18 @@ void round_rows(const moe_shape_t* s, const moe_plan_info_t* info, int r, int32_
   *rows = static_cast<int>(total);
 }
 
+// The workspace header for the kernels' debug bounds checks, or null when they are off.
+int32_t* debug_ptr(const moe_shape_t* s, void* ws, const moe_workspace_layout_t& L) {
+  return debug_bounds(s) ? at<int32_t>(ws, L.header) : nullptr;
+}
+
+// Most rows one expert may hold in a round (checked by the GEMMs under debug bounds checks).
+int rows_cap(const moe_shape_t* s) {
+  if (!debug_bounds(s)) return 0;
+  const long long cap = borrowing(s) ? static_cast<long long>(s->E) * s->C : s->C;
+  return static_cast<int>(cap);
+}
+
 int do_dispatch(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
                 const moe_workspace_layout_t& L, int r, const uint16_t* x, cudaStream_t stream) {
   int32_t n_host[MOE_MAX_EXPERTS];
@@ -229,12 +269,19 @@ int do_dispatch(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
   round_rows(s, info, r, n_host, &rows);
   return cuda_status(launch_dispatch(x, at<uint16_t>(ws, L.buf), at<int32_t>(ws, L.row_start),
                                      at<int32_t>(ws, L.row_token), at<int32_t>(ws, L.row_dst), r, rows,
-                                     s->d, stream));
+                                     s->d, stream, debug_ptr(s, ws, L), s->T,
+                                     static_cast<long long>(s->E) * s->C));
 }
 
 // Copy steps up to this many bytes of rows ride on a GEMM launch (its 4 copy warps per SM);
-// larger ones get their own kernel, which reaches full HBM bandwidth.
+// larger ones ride there only when the copy's estimated time, at about kSideCopyGBs, stays below
+// the GEMM's at about kGemmTflops; otherwise they get their own kernel at full HBM bandwidth.
 constexpr size_t kFuseCopyBytes = 32ull << 20;
+#ifndef MOE_SIDE_COPY_GBS
+#define MOE_SIDE_COPY_GBS 2000.0
+#endif
+constexpr double kSideCopyGBs = MOE_SIDE_COPY_GBS;
+constexpr double kGemmTflops = 1100.0;
 
 // The copy step of round `cr` carried by a GEMM launch (a combine, or a dispatch of x).
 RoundCopy make_copy(const moe_shape_t* s, const moe_plan_info_t* info, void* ws, const moe_workspace_layout_t& L,
@@ -261,21 +308,26 @@ RoundCopy make_copy(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
   c.d = s->d;
   c.row_off = borrowing(s) ? at<int32_t>(ws, L.row_off) : nullptr;
   c.E = s->E;
+  c.dbg = debug_ptr(s, ws, L);
   return c;
 }
 
+// x_gather: gather the round's A rows from x (the forward's own rounds), or null to read them
+// from the dispatch buffer that moe_round_dispatch filled.
 int do_gate_up(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
                const moe_workspace_layout_t& L, int r, const uint16_t* w13, const RoundCopy* copy,
-               cudaStream_t stream) {
+               const uint16_t* x_gather, cudaStream_t stream) {
   int32_t n_host[MOE_MAX_EXPERTS];
   int rows = 0;
   round_rows(s, info, r, n_host, &rows);
   const bool pooled = borrowing(s);
+  GatherA g{x_gather, s->T, at<int32_t>(ws, L.row_token), at<int32_t>(ws, L.row_off) + static_cast<size_t>(r) * s->E};
   return cuda_status(launch_gate_up(at<uint16_t>(ws, L.buf), w13, at<uint16_t>(ws, L.h),
                                     at<int32_t>(ws, L.n) + static_cast<size_t>(r) * s->E, n_host, s->E,
                                     s->C, s->d, s->d_ff, at<int32_t>(ws, L.header) + kHdrStatus, copy,
                                     pooled ? at<int32_t>(ws, L.row_off) + static_cast<size_t>(r) * s->E : nullptr,
-                                    pooled ? at<int32_t>(ws, L.row_start) + r : nullptr, stream));
+                                    pooled ? at<int32_t>(ws, L.row_start) + r : nullptr,
+                                    x_gather ? &g : nullptr, stream, rows_cap(s)));
 }
 
 int do_down(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
@@ -289,7 +341,7 @@ int do_down(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
                                  at<int32_t>(ws, L.n) + static_cast<size_t>(r) * s->E, n_host, s->E,
                                  s->C, s->d, s->d_ff, at<int32_t>(ws, L.header) + kHdrStatus, copy,
                                  pooled ? at<int32_t>(ws, L.row_off) + static_cast<size_t>(r) * s->E : nullptr,
-                                 pooled ? at<int32_t>(ws, L.row_start) + r : nullptr, stream));
+                                 pooled ? at<int32_t>(ws, L.row_start) + r : nullptr, stream, rows_cap(s)));
 }
 
 int do_combine(const moe_shape_t* s, const moe_plan_info_t* info, void* ws, const moe_workspace_layout_t& L,
@@ -302,7 +354,7 @@ int do_combine(const moe_shape_t* s, const moe_plan_info_t* info, void* ws, cons
                                     at<int32_t>(ws, L.slot), at<int32_t>(ws, L.row_start),
                                     at<int32_t>(ws, L.row_token), at<int32_t>(ws, L.row_dst), s->T, s->k,
                                     s->C, s->d, r, rows, borrowing(s) ? at<int32_t>(ws, L.row_off) : nullptr,
-                                    s->E, stream));
+                                    s->E, stream, debug_ptr(s, ws, L)));
 }
 
 void make_backward_layout(const moe_shape_t* s, moe_backward_layout_t* L) {
@@ -474,6 +526,12 @@ int moe_plan(const moe_shape_t* shape, const float* logits, const uint16_t* x,
   if (cudaMemsetAsync(header, 0, L.block_base - L.header + static_cast<size_t>(L.plan_blocks) * s.E * 4, stream) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
+  if (debug_bounds(&s)) {   // the guards after every region (the memset above covers the first)
+    GuardList guards;
+    moe_workspace_layout_t L2;
+    make_layout(&s, &L2, &guards);
+    if ((st = cuda_status(launch_guards(static_cast<uint8_t*>(ws), guards, 0, header, stream))) != MOE_OK) return st;
+  }
 
   const float* z = logits;
   if (z == nullptr && s.T > 0) {
@@ -503,6 +561,7 @@ int moe_plan(const moe_shape_t* shape, const float* logits, const uint16_t* x,
   pb.sync = at<int32_t>(ws, L.sync);
   pb.sync_words = pipe_sync_words(s.E, s.C);
   pb.borrow = (s.flags & MOE_FLAG_BORROW) ? 1 : 0;
+  pb.dbg = debug_bounds(&s) ? header : nullptr;
   if ((st = cuda_status(launch_plan(pb, s.T, s.k, s.E, s.C, L.max_rounds, stream))) != MOE_OK) return st;
 
   int32_t host[kHdrWords];
@@ -542,7 +601,7 @@ int moe_round_gate_up(const moe_shape_t* shape, const moe_plan_info_t* info, voi
   if (st != MOE_OK) return st;
   if (r < 0 || r >= info->R || w_gate_up == nullptr) return MOE_ERR_INVALID_ARG;
   if (!aligned(w_gate_up, 16)) return MOE_ERR_MISALIGNED;
-  return do_gate_up(shape, info, ws, L, r, w_gate_up, nullptr, reinterpret_cast<cudaStream_t>(stream));
+  return do_gate_up(shape, info, ws, L, r, w_gate_up, nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int moe_round_down(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
@@ -602,36 +661,51 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
   int r0 = R;
   if (shape->flags & MOE_FLAG_PIPELINE_ALL) {
     r0 = 0;
-  } else if (!(shape->flags & (MOE_FLAG_PER_ROUND | MOE_FLAG_BORROW))) {   // borrowing: per-round only
+  } else if (!(shape->flags & (MOE_FLAG_PER_ROUND | MOE_FLAG_BORROW | MOE_FLAG_DEBUG_BOUNDS))) {
+    // borrowing and the debug bounds checks run per round only
     while (r0 > 0 && thin(r0 - 1)) --r0;
   }
-  // Per-round launch order. A small copy step (a thin round: at most kFuseCopyBytes of rows)
-  // rides on the neighbouring GEMM launch: combine(r-1) on gate/up(r), dispatch(r+1) on
-  // down(r). A large one runs as its own full-bandwidth kernel right after down(r). Each launch
-  // depends only on the one before it (PDL wait), and no two steps of one launch touch the same
-  // buffer: dispatch writes buf, gate/up reads buf and writes h, down reads h and writes out,
-  // combine reads out and updates y. A run of thin rounds thus costs two launches per round.
-  // The first pipelined round is dispatched here too (by the dispatch kernel, or on the last
-  // per-round down GEMM), so the pipelined launch starts with its rows in place.
-  // Rounds [rb, re) as per-round launches, round rb's rows already dispatched and the combine
-  // of round rb-1 already issued.
+  // Per-round launch order. The gate/up GEMM of a round gathers its rows straight from x (TMA
+  // row gathers of the round-major row list), so these rounds need no dispatch step. A round's
+  // combine rides on the next round's gate/up launch as its copy warps when it is small (at most
+  // kFuseCopyBytes of rows) or when its estimated time there stays below that GEMM's; otherwise it
+  // runs as its own full-bandwidth kernel right after its down GEMM. Each launch depends only on
+  // the one before it (PDL wait), and no two steps of one launch touch the same buffer: gate/up
+  // reads x and writes h, down reads h and writes out, combine reads out and updates y. The first
+  // pipelined round is dispatched into buf here too (on the last per-round down GEMM's copy warps,
+  // or by the dispatch kernel), so the pipelined launch starts with its rows in place.
+  auto rows_of = [&](int rr) {
+    int32_t n_host[MOE_MAX_EXPERTS];
+    int rows = 0;
+    round_rows(shape, info, rr, n_host, &rows);
+    return rows;
+  };
+  auto combine_rides = [&](int rc, int rg) {
+    if (small(rc)) return true;
+    // copy warps move about kSideCopyGBs; the GEMM runs at about kGemmTflops
+    const double rows_c = rows_of(rc), tokens_c = rows_c < shape->T ? rows_c : shape->T;
+    const double t_copy = (2.0 * rows_c + 8.0 * tokens_c) * shape->d / (kSideCopyGBs * 1e9);
+    const double t_gemm = 4.0 * rows_of(rg) * shape->d * shape->d_ff / (kGemmTflops * 1e12);
+    return t_copy <= t_gemm;
+  };
   auto per_round = [&](int rb, int re) -> int {
     int rc = MOE_OK;
     for (int r = rb; r < re; ++r) {
-      const bool fuse_combine = r > rb && small(r - 1);
+      const bool fuse_combine = r > rb && combine_rides(r - 1, r);
       const RoundCopy comb = make_copy(shape, info, ws, L, true, r > 0 ? r - 1 : 0, x, y);
-      if ((rc = do_gate_up(shape, info, ws, L, r, w_gate_up, fuse_combine ? &comb : nullptr, stream)) != MOE_OK)
+      if ((rc = do_gate_up(shape, info, ws, L, r, w_gate_up, fuse_combine ? &comb : nullptr, x, stream)) != MOE_OK)
         return rc;
-      const bool next = r + 1 < R;
-      const bool fuse_dispatch = next && small(r + 1);
-      const RoundCopy disp = make_copy(shape, info, ws, L, false, next ? r + 1 : r, x, y);
+      const bool pipe_next = r + 1 == re && re < R;   // the pipelined launch takes round r + 1
+      const bool fuse_dispatch = pipe_next && small(r + 1);
+      const RoundCopy disp = make_copy(shape, info, ws, L, false, pipe_next ? r + 1 : r, x, y);
       if ((rc = do_down(shape, info, ws, L, r, w_down, fuse_dispatch ? &disp : nullptr, stream)) != MOE_OK) return rc;
-      if (next && !fuse_dispatch && (rc = do_dispatch(shape, info, ws, L, r + 1, x, stream)) != MOE_OK) return rc;
-      if (!(r + 1 < re && small(r)) && (rc = do_combine(shape, info, ws, L, r, y, stream)) != MOE_OK) return rc;
+      if (pipe_next && !fuse_dispatch && (rc = do_dispatch(shape, info, ws, L, r + 1, x, stream)) != MOE_OK) return rc;
+      if (!(r + 1 < re && combine_rides(r, r + 1)) && (rc = do_combine(shape, info, ws, L, r, y, stream)) != MOE_OK)
+        return rc;
     }
     return rc;
   };
-  if ((st = do_dispatch(shape, info, ws, L, 0, x, stream)) != MOE_OK) return st;
+  if (r0 == 0 && (st = do_dispatch(shape, info, ws, L, 0, x, stream)) != MOE_OK) return st;
   if ((st = per_round(0, r0)) != MOE_OK) return st;
   if (r0 < R) {
     PipelineArgs p{};
@@ -683,11 +757,19 @@ int moe_device_status(const moe_shape_t* shape, void* ws, moe_stream_t stream_) 
   moe_workspace_layout_t L;
   make_layout(shape, &L);
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (debug_bounds(shape)) {   // compare every guard word first
+    GuardList guards;
+    make_layout(shape, &L, &guards);
+    if (cuda_status(launch_guards(static_cast<uint8_t*>(ws), guards, 1, at<int32_t>(ws, L.header), stream)) !=
+        MOE_OK)
+      return MOE_ERR_CUDA;
+  }
   int32_t word = 0;
   if (cudaMemcpyAsync(&word, at<int32_t>(ws, L.header) + kHdrStatus, 4, cudaMemcpyDeviceToHost, stream) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word & (kStatusBounds | kStatusCanary)) return MOE_ERR_BOUNDS;
   return word != 0 ? MOE_ERR_TIMEOUT : MOE_OK;
 }
 
@@ -702,6 +784,7 @@ const char* moe_status_string(int status) {
     case MOE_ERR_TIMEOUT: return "a kernel wait timed out";
     case MOE_ERR_NO_DEVICE: return "current device is not sm_100";
     case MOE_ERR_NOALLOC_LIMIT: return "shape needs more scratch than moe_plan_noalloc's static array";
+    case MOE_ERR_BOUNDS: return "a debug bounds check failed or a workspace guard was overwritten";
     default: return "unknown status";
   }
 }

@@ -114,6 +114,7 @@ extern "C" MOE_API int moe_plan_noalloc(const moe_shape_t* shape, const float* l
   pb.sync = nullptr;
   pb.sync_words = 0;
   pb.borrow = (s.flags & MOE_FLAG_BORROW) ? 1 : 0;
+  pb.dbg = nullptr;
   if (moe::launch_plan(pb, s.T, s.k, s.E, s.C, max_rounds, stream) != cudaSuccess) return MOE_ERR_CUDA;
 
   int32_t host[moe::kHdrWords];

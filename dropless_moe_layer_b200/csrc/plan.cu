@@ -244,7 +244,8 @@ __global__ void __launch_bounds__(kTPB) plan_rank_kernel(const int32_t* __restri
                                                          const int32_t* __restrict__ n,
                                                          const int32_t* __restrict__ row_start,
                                                          int borrow, int max_rounds,
-                                                         int32_t* __restrict__ sync, long long sync_words) {
+                                                         int32_t* __restrict__ sync, long long sync_words,
+                                                         int32_t* dbg) {
   __shared__ uint32_t mask[kWarps][MOE_MAX_E_PLAN];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) mask[i / E][i % E] = 0u;
@@ -257,13 +258,21 @@ __global__ void __launch_bounds__(kTPB) plan_rank_kernel(const int32_t* __restri
   if (sync)
     for (long long i = t; i < sync_words; i += static_cast<long long>(gridDim.x) * kTPB) sync[i] = 0;
   if (valid)
-    for (int j = 0; j < k; ++j) atomicOr(&mask[warp][idx[static_cast<size_t>(t) * k + j]], 1u << lane);
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[static_cast<size_t>(t) * k + j];
+      if (dbg != nullptr && (e < 0 || e >= E)) {   // debug bounds checks: an expert out of range
+        record_bad(dbg, kBadPlanPair, t * k + j);
+        continue;
+      }
+      atomicOr(&mask[warp][e], 1u << lane);
+    }
   __syncthreads();
   if (!valid) return;
   const uint32_t lower = (1u << lane) - 1u;
   for (int j = 0; j < k; ++j) {
     const size_t p = static_cast<size_t>(t) * k + j;
     const int e = idx[p];
+    if (dbg != nullptr && (e < 0 || e >= E)) continue;   // recorded above
     int rank = block_base[static_cast<size_t>(blockIdx.x) * E + e];
     for (int w = 0; w < warp; ++w) rank += __popc(mask[w][e]);
     rank += __popc(mask[warp][e] & lower);
@@ -280,7 +289,15 @@ __global__ void __launch_bounds__(kTPB) plan_rank_kernel(const int32_t* __restri
     }
     round_out[p] = r;
     slot_out[p] = s;
+    if (dbg != nullptr && (r < 0 || r >= max_rounds)) {
+      record_bad(dbg, kBadPlanPair, static_cast<int>(p));
+      continue;
+    }
     const int pos = row_off[static_cast<size_t>(r) * E + e] + s;
+    if (dbg != nullptr && (pos < 0 || static_cast<long long>(pos) >= static_cast<long long>(T) * k)) {
+      record_bad(dbg, kBadPlanPair, static_cast<int>(p));
+      continue;
+    }
     row_token[pos] = t;
     // round buffer row: expert e's C rows, or with borrowing the round's rows packed in order
     row_dst[pos] = borrow ? pos - row_start[r] : e * C + s;
@@ -299,7 +316,7 @@ cudaError_t launch_plan(const PlanBuffers& b, int T, int k, int E, int C, int ma
   if (blocks > 0 && err == cudaSuccess)
     err = launch_pdl(plan_rank_kernel, dim3(blocks), dim3(kTPB), 0, stream, b.idx, T, k, E, C,
                      b.block_base, b.row_off, b.round, b.slot, b.row_token, b.row_dst, b.n, b.row_start,
-                     b.borrow, max_rounds, b.sync, b.sync_words);
+                     b.borrow, max_rounds, b.sync, b.sync_words, b.dbg);
   launch_end(kKindPlan, stream, blocks > 0 ? 2 : 1);
   return err;
 }

@@ -24,11 +24,12 @@ FLAG_RENORM_TOPK = 1
 FLAG_PER_ROUND = 2
 FLAG_PIPELINE_ALL = 4
 FLAG_BORROW = 8
+FLAG_DEBUG_BOUNDS = 16
 SCHEDULES = {"auto": 0, "per_round": FLAG_PER_ROUND, "pipeline": FLAG_PIPELINE_ALL}
 
 STATUS = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED_SHAPE",
           -3: "MOE_ERR_WORKSPACE_TOO_SMALL", -4: "MOE_ERR_MISALIGNED", -5: "MOE_ERR_CUDA",
-          -6: "MOE_ERR_TIMEOUT", -7: "MOE_ERR_NO_DEVICE", -8: "MOE_ERR_NOALLOC_LIMIT"}
+          -6: "MOE_ERR_TIMEOUT", -7: "MOE_ERR_NO_DEVICE", -8: "MOE_ERR_NOALLOC_LIMIT", -9: "MOE_ERR_BOUNDS"}
 
 
 class Shape(ctypes.Structure):
@@ -128,11 +129,12 @@ def _check(call: str, status: int) -> None:
 
 
 def make_shape(T: int, d: int, E: int, k: int, d_ff: int, C: int, renorm: bool = False,
-               schedule: str = "auto", borrow: bool = False) -> Shape:
+               schedule: str = "auto", borrow: bool = False, debug_bounds: bool = False) -> Shape:
     """schedule: "auto" (trailing thin rounds pipelined), "per_round" or "pipeline";
-    borrow: capacity borrowing between experts (MOE_FLAG_BORROW)."""
+    borrow: capacity borrowing between experts (MOE_FLAG_BORROW); debug_bounds: the library's
+    index checks and workspace guards (MOE_FLAG_DEBUG_BOUNDS)."""
     return Shape(T, d, E, k, d_ff, C, (FLAG_RENORM_TOPK if renorm else 0) | SCHEDULES[schedule] |
-                 (FLAG_BORROW if borrow else 0))
+                 (FLAG_BORROW if borrow else 0) | (FLAG_DEBUG_BOUNDS if debug_bounds else 0))
 
 
 # ------------------------------------------------------------------------- raw-pointer calls
@@ -268,9 +270,9 @@ class DroplessMoE:
     """
 
     def __init__(self, T: int, d: int, E: int, k: int, d_ff: int, C: int, renorm: bool = False,
-                 device=None, schedule: str = "auto", borrow: bool = False):
+                 device=None, schedule: str = "auto", borrow: bool = False, debug_bounds: bool = False):
         import torch
-        self.shape = make_shape(T, d, E, k, d_ff, C, renorm, schedule, borrow)
+        self.shape = make_shape(T, d, E, k, d_ff, C, renorm, schedule, borrow, debug_bounds)
         self.ws_bytes = workspace_bytes(self.shape)
         if self.ws_bytes == 0:
             raise ValueError(f"unsupported shape T={T} d={d} E={E} k={k} d_ff={d_ff} C={C}")

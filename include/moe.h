@@ -69,7 +69,9 @@ typedef enum moe_status {
   MOE_ERR_CUDA = -5,                /* a CUDA runtime call failed (includes earlier faults) */
   MOE_ERR_TIMEOUT = -6,             /* a kernel's bounded wait gave up; see moe_device_status */
   MOE_ERR_NO_DEVICE = -7,           /* current device is not an sm_100 GPU */
-  MOE_ERR_NOALLOC_LIMIT = -8        /* moe_plan_noalloc: shape needs more than its static scratch */
+  MOE_ERR_NOALLOC_LIMIT = -8,       /* moe_plan_noalloc: shape needs more than its static scratch */
+  MOE_ERR_BOUNDS = -9               /* MOE_FLAG_DEBUG_BOUNDS: a plan index was out of range, or a
+                                       workspace guard was overwritten; see moe_device_status */
 } moe_status;
 
 /* moe_shape_t.flags */
@@ -94,6 +96,21 @@ typedef enum moe_status {
  * 1 whenever T*k <= E*C. Runs as per-round launches (not with MOE_FLAG_PIPELINE_ALL); y is the
  * same layer output. Off by default: the default plan is R = ceil(max_load / C). */
 #define MOE_FLAG_BORROW 8u
+/* Debug bounds checks, a stand-in for a memory checker (off by default; slower). With this flag:
+ *   - the calls that run a plan first check its summary on the host (loads non-negative, at most
+ *     T and adding up to T*k, max_load their maximum, R the round count of those loads) and return
+ *     MOE_ERR_INVALID_ARG, launching nothing, when it cannot be the planner's;
+ *   - the planner, dispatch, combine and the GEMMs check every plan index before they use it
+ *     (expert < E, round < the workspace's rounds, row-list position < T*k, source token < T,
+ *     buffer row < E*C, rows of an expert in a round <= C, or <= E*C with MOE_FLAG_BORROW); a
+ *     failed check is recorded in the workspace header and the access is skipped, never trapped;
+ *   - the workspace holds a 256-byte guard after every region (moe_workspace_bytes grows by
+ *     256 bytes per region), which moe_plan fills and moe_device_status verifies;
+ *   - moe_forward runs every round as per-round launches (not with MOE_FLAG_PIPELINE_ALL);
+ *   - moe_device_status returns MOE_ERR_BOUNDS after a failed check or a changed guard.
+ * Results are bit-identical to the per-round schedule without the flag. The backward pass and
+ * moe_plan_noalloc do not check. */
+#define MOE_FLAG_DEBUG_BOUNDS 16u
 
 #define MOE_MAX_EXPERTS 256
 #define MOE_MAX_TOPK 16
@@ -260,7 +277,8 @@ MOE_API int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, 
                          float* dw_down, float* dz, moe_stream_t stream);
 
 /* Synchronizes `stream` and reads the workspace status word that kernels set when a
- * bounded wait gives up. Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_CUDA. */
+ * bounded wait gives up. With MOE_FLAG_DEBUG_BOUNDS it first verifies the workspace guards.
+ * Returns MOE_OK, MOE_ERR_TIMEOUT, MOE_ERR_BOUNDS or MOE_ERR_CUDA. */
 MOE_API int moe_device_status(const moe_shape_t* shape, void* ws, moe_stream_t stream);
 
 /* Human-readable text for a moe_status value (static storage). */

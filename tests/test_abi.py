@@ -81,8 +81,8 @@ def test_bad_shapes_are_rejected(lib, kw):
 
 def test_bad_flags_rejected(lib):
     s = moe.make_shape(64, 128, 8, 2, 128, 16)
-    for flags in (16, 1 << 31, moe.FLAG_PER_ROUND | moe.FLAG_PIPELINE_ALL,
-                  moe.FLAG_BORROW | moe.FLAG_PIPELINE_ALL):
+    for flags in (32, 1 << 31, moe.FLAG_PER_ROUND | moe.FLAG_PIPELINE_ALL,
+                  moe.FLAG_BORROW | moe.FLAG_PIPELINE_ALL, moe.FLAG_DEBUG_BOUNDS | moe.FLAG_PIPELINE_ALL):
         s.flags = flags
         assert moe.workspace_bytes(s) == 0
     # borrowing runs per round: no second buffer set, like the per-round schedule
@@ -166,7 +166,7 @@ def test_backward_workspace_is_fixed_by_shape(lib, w):
     sb = moe.make_shape(w.T, w.d, w.E, w.k, w.F, w.C, borrow=True)
     assert moe.backward_workspace_bytes(sb) == _backward_bytes_model(w, borrow=True)
     assert moe.backward_layout(sb).cpad == (w.E * w.C + 64 * w.E + 127) // 128 * 128
-    s.flags = 16
+    s.flags = 32          # not a flag
     assert moe.backward_workspace_bytes(s) == 0
 
 
