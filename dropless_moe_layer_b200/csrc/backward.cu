@@ -291,10 +291,11 @@ constexpr int kStageBytes = gemm::kABytes + 256 * BK * 2;
 constexpr int kStages = gemm::kRingBytes / kStageBytes;
 static_assert(kStages >= 2 && kStages <= gemm::kMaxStages, "ring stages");
 constexpr int kTileStride = gemm::kMaxGroups + 1;
-// gemm::carve's layout, with room for a tile prefix and a pooled-column prefix per phase after
+// gemm::carve's layout (ring, the forward's output staging, which this kernel leaves unused,
+// barriers, misc words), with room for a tile prefix and a pooled-column prefix per phase after
 // the misc words.
-constexpr int kSmemBytes = 1024 + gemm::kRingBytes + gemm::kBarBytes + gemm::kMiscWords * 4 +
-                           2 * kMaxPhases * kTileStride * 4;
+constexpr int kSmemBytes = 1024 + gemm::kRingBytes + gemm::kOutStagingBytes + gemm::kBarBytes +
+                           gemm::kMiscWords * 4 + 2 * kMaxPhases * kTileStride * 4;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 struct Launch {

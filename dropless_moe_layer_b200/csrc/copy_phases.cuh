@@ -23,21 +23,68 @@
 namespace moe {
 namespace copy {
 
+// Streaming accesses for copies that run beside a GEMM (the copy warps of a GEMM launch): an L2
+// evict-first policy, so that the copy's bytes, each touched once, do not push the GEMM's weight
+// and activation tiles out of the L2. kStream = false: plain accesses.
+__device__ __forceinline__ uint64_t stream_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+template <bool kStream>
+__device__ __forceinline__ uint4 ld_u4(const uint4* p, uint64_t pol) {
+  if constexpr (!kStream) return __ldg(p);
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p), "l"(pol));
+  return v;
+}
+template <bool kStream>
+__device__ __forceinline__ void st_u4(uint4* p, const uint4& v, uint64_t pol) {
+  if constexpr (!kStream) {
+    *p = v;
+  } else {
+    asm volatile("st.global.L1::no_allocate.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x),
+                 "r"(v.y), "r"(v.z), "r"(v.w), "l"(pol)
+                 : "memory");
+  }
+}
+template <bool kStream>
+__device__ __forceinline__ float4 ld_f4(const float* p, uint64_t pol) {
+  if constexpr (!kStream) return *reinterpret_cast<const float4*>(p);
+  float4 v;
+  asm volatile("ld.global.L1::no_allocate.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p), "l"(pol));
+  return v;
+}
+template <bool kStream>
+__device__ __forceinline__ void st_f4(float* p, const float4& v, uint64_t pol) {
+  if constexpr (!kStream) {
+    *reinterpret_cast<float4*>(p) = v;
+  } else {
+    asm volatile("st.global.L1::no_allocate.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v.x),
+                 "f"(v.y), "f"(v.z), "f"(v.w), "l"(pol)
+                 : "memory");
+  }
+}
+
+template <bool kStream = false>
 __device__ __forceinline__ void dispatch_row(const uint4* __restrict__ x, uint4* __restrict__ buf, int t,
                                              int dst, int vecs, int lane) {
   const uint4* src = x + static_cast<size_t>(t) * vecs;
   uint4* out = buf + static_cast<size_t>(dst) * vecs;
+  const uint64_t pol = kStream ? stream_policy() : 0;
   for (int v0 = 0; v0 < vecs; v0 += 8 * 32) {
     uint4 tmp[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int v = v0 + u * 32 + lane;
-      if (v < vecs) tmp[u] = __ldg(src + v);
+      if (v < vecs) tmp[u] = ld_u4<kStream>(src + v, pol);
     }
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int v = v0 + u * 32 + lane;
-      if (v < vecs) out[v] = tmp[u];
+      if (v < vecs) st_u4<kStream>(out + v, tmp[u], pol);
     }
   }
 }
@@ -45,6 +92,7 @@ __device__ __forceinline__ void dispatch_row(const uint4* __restrict__ x, uint4*
 // Rows [begin, end) of the round-major row list, spread over `warps` warps (this one is `w`).
 // With dbg (debug bounds checks) a row whose token is not below T or whose destination is not
 // below buf_rows is recorded and skipped.
+template <bool kStream = false>
 __device__ __forceinline__ void dispatch_rows(const uint4* __restrict__ x, uint4* __restrict__ buf,
                                               const int32_t* __restrict__ row_token,
                                               const int32_t* __restrict__ row_dst, int begin, int end,
@@ -57,7 +105,7 @@ __device__ __forceinline__ void dispatch_rows(const uint4* __restrict__ x, uint4
       if (lane == 0) record_bad(dbg, kBadDispatchRow, row);
       continue;
     }
-    dispatch_row(x, buf, t, dst, vecs, lane);
+    dispatch_row<kStream>(x, buf, t, dst, vecs, lane);
   }
 }
 
@@ -84,7 +132,8 @@ struct CombineArgs {
   const int32_t* row_start;
   int E;
   // Debug bounds checks (MOE_FLAG_DEBUG_BOUNDS): the workspace header, else null; a pair whose
-  // expert is not below E or whose buffer row is not below rows_cap makes the token skipped.
+  // expert is not below E, whose slot is not below C (per-expert rows) or whose buffer row is not
+  // below rows_cap makes the token skipped.
   int32_t* dbg;
   long long rows_cap;
 };
@@ -144,7 +193,9 @@ __device__ __forceinline__ TokenPairs token_pairs(const CombineArgs& a, const Pa
   tp.first_row = __shfl_sync(0xffffffffu, row, 0);
   tp.pgate = lane < tp.npairs ? g : 0.f;
   if (a.dbg != nullptr) {
-    const bool bad = lane < tp.npairs && (!e_ok || tp.s < 0 || row >= static_cast<unsigned long long>(a.rows_cap));
+    // a slot past C lands in the next expert's rows of the [E, C, d] buffer: checked on its own
+    const bool bad = lane < tp.npairs && (!e_ok || tp.s < 0 || (a.row_off == nullptr && tp.s >= a.C) ||
+                                          row >= static_cast<unsigned long long>(a.rows_cap));
     const uint32_t any = __ballot_sync(0xffffffffu, bad);
     if (any) {
       if (lane == __ffs(any) - 1) record_bad(a.dbg, kBadCombinePair, static_cast<int>(row));
@@ -155,13 +206,15 @@ __device__ __forceinline__ TokenPairs token_pairs(const CombineArgs& a, const Pa
 }
 
 // y[t] = (fresh ? 0 : y[t]) + sum over the round's pairs (ascending j) of gate * out row, fp32
-// FMAs. kLaneCols columns per lane per pass (8 or 16): 16 halves the passes over a row, so
-// more loads are in flight when few warps do the work. The whole warp runs it.
-template <int kLaneCols = 8>
+// FMAs. kLaneCols columns per lane per pass (8, 16 or 32): wider passes mean fewer dependent
+// passes over a row and more loads in flight, which matters when few warps do the work (the
+// copy warps of a GEMM launch). The whole warp runs it.
+template <int kLaneCols = 8, bool kStream = false>
 __device__ __forceinline__ void accumulate_token(const CombineArgs& a, int t, const TokenPairs& tp) {
-  static_assert(kLaneCols == 8 || kLaneCols == 16, "lane width");
+  static_assert(kLaneCols == 8 || kLaneCols == 16 || kLaneCols == 32, "lane width");
   constexpr int kVecs = kLaneCols / 8;   // bf16 x 8 per 16-byte load
   const int lane = threadIdx.x & 31;
+  const uint64_t pol = kStream ? stream_policy() : 0;
   const int npairs = tp.npairs;
   float* yrow = a.y + static_cast<size_t>(t) * a.d;
   // Every lane runs the same iterations (the shuffles below need the whole warp); lanes past
@@ -176,7 +229,7 @@ __device__ __forceinline__ void accumulate_token(const CombineArgs& a, int t, co
     } else {
 #pragma unroll
       for (int i = 0; i < kLaneCols; i += 4) {
-        const float4 u = *reinterpret_cast<const float4*>(yrow + c + i);
+        const float4 u = ld_f4<kStream>(yrow + c + i, pol);
         acc[i] = u.x; acc[i + 1] = u.y; acc[i + 2] = u.z; acc[i + 3] = u.w;
       }
     }
@@ -190,7 +243,7 @@ __device__ __forceinline__ void accumulate_token(const CombineArgs& a, int t, co
         g[u] = __shfl_sync(0xffffffffu, tp.pgate, p & 31);
 #pragma unroll
         for (int v = 0; v < kVecs; ++v)
-          q[u][v] = (p < npairs && col) ? *reinterpret_cast<const uint4*>(a.buf + row * a.d + c + 8 * v)
+          q[u][v] = (p < npairs && col) ? ld_u4<kStream>(reinterpret_cast<const uint4*>(a.buf + row * a.d + c + 8 * v), pol)
                                         : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
@@ -209,7 +262,7 @@ __device__ __forceinline__ void accumulate_token(const CombineArgs& a, int t, co
     if (col) {
 #pragma unroll
       for (int i = 0; i < kLaneCols; i += 4)
-        *reinterpret_cast<float4*>(yrow + c + i) = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
+        st_f4<kStream>(yrow + c + i, make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]), pol);
     }
   }
 }
@@ -218,12 +271,12 @@ __device__ __forceinline__ void accumulate_token(const CombineArgs& a, int t, co
 // With `only_row` >= 0 the warp stands for one buffer row of the round (one of token t's pairs)
 // and does the work only if that row is t's first pair in the round, so that every active
 // token is combined exactly once when the round is walked row by row.
-template <int kLaneCols = 8>
+template <int kLaneCols = 8, bool kStream = false>
 __device__ __forceinline__ void combine_token(const CombineArgs& a, int t, int r, long long only_row = -1) {
   const TokenPairs tp = token_pairs(a, load_pairs(a, t), r);
   if (tp.npairs == 0) return;
   if (only_row >= 0 && tp.first_row != static_cast<unsigned long long>(only_row)) return;
-  accumulate_token<kLaneCols>(a, t, tp);
+  accumulate_token<kLaneCols, kStream>(a, t, tp);
 }
 
 // One warp copies rows [0, nr) (nr <= 32) of a slice of the round-major row list: row i goes

@@ -54,15 +54,22 @@ constexpr int kMaxGroups = MOE_MAX_E_PLAN;
 constexpr int kThreads = 192;
 constexpr int kMaxStages = 8;
 constexpr int kRingBytes = kStages * kStageBytes;           // 192 KB, re-cut per phase width
+// TMA-store epilogue: each epilogue warp stages 32 rows x 32 columns of bf16 (2 KB, 64-byte
+// swizzle) in one of its two buffers, then stores them with one bulk tensor store.
+constexpr int kOutChunkCols = 32;
+constexpr int kOutChunkBytes = 32 * kOutChunkCols * 2;
+constexpr int kOutStagingBytes = 4 * 2 * kOutChunkBytes;    // 16 KB
 constexpr int kBarBytes = (2 * kMaxStages + 5) * 8;
 constexpr int kMiscWords = 8;
-constexpr int kSmemBytes = 1024 + kRingBytes + kBarBytes + kMiscWords * 4 + 2 * (kMaxGroups + 1) * 4;
+constexpr int kSmemBytes =
+    1024 + kRingBytes + kOutStagingBytes + kBarBytes + kMiscWords * 4 + 2 * (kMaxGroups + 1) * 4;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 enum Mode : int { kSwiGLU = 0, kBf16Out = 1, kF32Bias = 2 };
 
 struct Smem {
   uint8_t* stage;
+  uint8_t* out_stage;       // TMA-store staging of the epilogue warps (1024-byte aligned)
   uint64_t* full;
   uint64_t* empty;
   uint64_t* tfull;
@@ -78,7 +85,8 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   Smem s;
   uint8_t* base = raw + ((1024u - (smem_addr(raw) & 1023u)) & 1023u);
   s.stage = base;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kRingBytes);
+  s.out_stage = base + kRingBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kRingBytes + kOutStagingBytes);
   s.full = bars;
   s.empty = bars + kMaxStages;
   s.tfull = bars + 2 * kMaxStages;
@@ -149,15 +157,13 @@ struct Phase {
   // of a single [rows, K] operand and output, instead of at row 0 of group g. Null: per group.
   const int32_t* group_row;
   const int32_t* group_row_base;
-  // Fused gather (gate/up of a round): the A rows are not read from a dispatch buffer but
-  // gathered straight from x through the 2-D map `a` (box: 64 columns x 1 row); row i of group
-  // g is x[gather_rows[gather_off[g] + i]] (the round-major row list). Null: tiled A loads.
-  const int32_t* gather_rows;
-  const int32_t* gather_off;
   // Debug bounds checks (MOE_FLAG_DEBUG_BOUNDS): a group's row count above rows_cap (the buffer
   // rows a group may hold) is recorded in the header dbg and clamped. rows_cap 0: unchecked.
   int rows_cap;
   int32_t* dbg;
+  // TMA-store epilogue (CTA-pair form, per-expert outputs only): the output as a 3-D map [groups]
+  // [rows][n_total] with 32 x 32 boxes and the 64-byte swizzle. Null: 16-byte stores per thread.
+  const CUtensorMap* out_map;
 };
 
 // Rows of group g (clamped to rows_cap under the debug bounds checks).
@@ -295,9 +301,6 @@ __device__ __forceinline__ void store_bf16(uint32_t tb, int cols, uint16_t* orow
 // Runs the CTA's share of the tiles of the phase planned in slot `which`. Returns when this
 // warp's role work is issued/done (the epilogue warps return after their last store). Every warp
 // leaves converged: a CTA barrier (which requires whole warps) may follow directly.
-// kGather: the phase gathers its A rows (Phase::gather_rows); a separate instantiation, so that the
-// tiled form keeps its register budget.
-template <bool kGather>
 __device__ __forceinline__ void run_phase(const Smem& s, uint32_t tmem_base, const Phase& p, int which,
                                           Pipe& pipe, int32_t* status) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -324,60 +327,7 @@ __device__ __forceinline__ void run_phase(const Smem& s, uint32_t tmem_base, con
     nt = local - mt * n_tiles;
   };
 
-  if (kGather && warp == 0) {
-    // ---------------------------------------------------------------- TMA producer, fused gather
-    // The whole warp produces: lane l gathers rows 4l .. 4l+3 of the A tile (one 4-row TMA
-    // gather per k block, 512 bytes of the tile each), lane 0 also loads the B tile. Every lane
-    // keeps the same pipeline counters.
-    const CUtensorMap* mb = b_map;
-    const uint32_t tx = static_cast<uint32_t>(kABytes + bn * BK * 2);
-    bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-      int g, mt, nt;
-      decode(tile, g, mt, nt);
-      const int rows_g = group_rows(p, g);
-      const int first = p.gather_off[g];
-      int tok[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {   // rows past the group's end repeat its first row (never stored)
-        const int i = mt * BM + 4 * lane + q;
-        tok[q] = p.gather_rows[first + (i < rows_g ? i : 0)];
-      }
-      for (int kb = 0; kb < p.num_k_blocks; ++kb) {
-        if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&s.empty[pipe.stage]), pipe.phase ^ 1u, s.abort))) {
-          ok = false;
-          break;
-        }
-        const uint32_t sA = smem_addr(s.stage + pipe.stage * stage_bytes);
-        const uint32_t sB = sA + kABytes;
-        const uint32_t fb = smem_addr(&s.full[pipe.stage]);
-        if (lane == 0) mbar_arrive_expect_tx(fb, tx);
-        __syncwarp();
-        tma_gather4_2d(sA + lane * 4 * BK * 2, p.a, fb, kb * BK, tok[0], tok[1], tok[2], tok[3]);
-        if (lane == 0) {
-          if (p.mode == kSwiGLU) {
-            tma_load_3d(sB, mb, fb, kb * BK, nt * width, g);
-            tma_load_3d(sB + width * BK * 2, mb, fb, kb * BK, p.b_second_row + nt * width, g);
-          } else {
-            tma_load_3d(sB, mb, fb, kb * BK, nt * width, g);
-          }
-        }
-        pipe.issued |= 1u << pipe.stage;
-        pipe.issued_parity = (pipe.issued_parity & ~(1u << pipe.stage)) | (pipe.phase << pipe.stage);
-        if (++pipe.stage == nstages) {
-          pipe.stage = 0;
-          pipe.phase ^= 1u;
-        }
-      }
-    }
-    if (!ok && lane == 0) {
-      atomicOr(status, kStatusTimeoutProducer);
-      *s.abort = 1;
-      for (int i = 0; i < nstages; ++i)   // let issued loads land before shared memory is reused
-        if ((pipe.issued >> i) & 1u) mbar_wait(smem_addr(&s.full[i]), (pipe.issued_parity >> i) & 1u, nullptr);
-    }
-    __syncwarp();
-  } else if (warp == 0) {
+  if (warp == 0) {
     if (lane == 0) {
     // ---------------------------------------------------------------- TMA producer
     const CUtensorMap* mb = b_map;
@@ -639,22 +589,10 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
     // ---------------------------------------------------------------- TMA producer (both CTAs)
     const uint32_t tx = 2u * kPairStageBytes;   // the pair's bytes per stage, counted by the leader
     bool ok = true;
-    const bool gather = p.gather_rows != nullptr;
     for (int tile = pair; ok && tile < total; tile += pairs) {
       int g, mp, nt;
       decode(tile, g, mp, nt);
-      const int row0 = mp * kPairRows + static_cast<int>(cta) * BM;   // this CTA's first A row
-      int tok[4] = {0, 0, 0, 0};
-      if (gather) {
-        const int rows_g = group_rows(p, g);
-        const int first = p.gather_off[g];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {   // rows past the group's end repeat its first row (never stored)
-          const int i = row0 + 4 * lane + q;
-          tok[q] = p.gather_rows[first + (i < rows_g ? i : 0)];
-        }
-      }
-      int a_row = row0, a_grp = g;
+      int a_row = mp * kPairRows + static_cast<int>(cta) * BM, a_grp = g;   // this CTA's first A row
       if (p.group_row) {
         a_row += p.group_row[g] - *p.group_row_base;
         a_grp = 0;
@@ -670,12 +608,10 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
         const uint32_t fb = peer_addr(fb_local, 0);   // the leader's full barrier
         if (cta == 0 && lane == 0) mbar_arrive_expect_tx(fb_local, tx);
         __syncwarp();
-        if (gather) {
-          tma_gather4_2d_pair(sA + lane * 4 * BK * 2, p.a, fb, kb * BK, tok[0], tok[1], tok[2], tok[3]);
-        } else if (lane == 0) {
+        if (lane == 0) {
           tma_load_3d_pair(sA, p.a, fb, kb * BK, a_row, a_grp);
+          tma_load_3d_pair(sB, p.b[0], fb, kb * BK, b_row(nt), g);
         }
-        if (lane == 0) tma_load_3d_pair(sB, p.b[0], fb, kb * BK, b_row(nt), g);
         pipe.issued |= 1u << pipe.stage;
         if (++pipe.stage == kPairStages) {
           pipe.stage = 0;
@@ -739,6 +675,8 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
   } else if (warp < 6) {
     // ---------------------------------------------------------------- epilogue (both CTAs)
     const int q = warp & 3;
+    uint32_t ochunk = 0;   // chunks this warp has staged (alternates its two buffers)
+    const uint32_t stage0 = smem_addr(s.out_stage + q * 2 * kOutChunkBytes);
     for (int tile = pair; tile < total; tile += pairs) {
       int g, mp, nt;
       decode(tile, g, mp, nt);
@@ -758,24 +696,67 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
                                      ? static_cast<long long>(p.group_row[g] - *p.group_row_base + row) * p.out_ld
                                      : g * p.out_group_stride + static_cast<long long>(row) * p.out_ld;
       uint16_t* orow = static_cast<uint16_t*>(p.out) + orow_off + nt * width;
-      if (p.mode == kSwiGLU)
+      if (p.out_map != nullptr) {
+        // 32-column chunks: TMEM -> registers -> this warp's staging buffer -> one bulk store of
+        // its 32 rows. Rows of the box past the group's rows hold junk; they fall in the expert's
+        // unused rows [n, C) (never read) or past C (clipped by the map).
+        const int row_base = mp * kPairRows + static_cast<int>(cta) * BM + q * 32;
+        const int chunks = (p.mode == kSwiGLU ? width : kPairBn) / kOutChunkCols;
+        for (int c = 0; c < chunks; ++c) {
+          uint32_t pk[16];
+          if (p.mode == kSwiGLU) {
+            uint32_t gv[32], uv[32];
+            tmem_ld32(tb + c * kOutChunkCols, gv);
+            tmem_ld32(tb + width + c * kOutChunkCols, uv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(silu_f(__uint_as_float(gv[2 * i])) * __uint_as_float(uv[2 * i]),
+                                  silu_f(__uint_as_float(gv[2 * i + 1])) * __uint_as_float(uv[2 * i + 1]));
+          } else {
+            uint32_t v[32];
+            tmem_ld32(tb + c * kOutChunkCols, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+          }
+          const uint32_t buf_off = (ochunk & 1u) * kOutChunkBytes;
+          if (lane == 0) bulk_wait_read_1();   // the store that last used this buffer has read it
+          __syncwarp();
+          uint8_t* row_ptr = s.out_stage + q * 2 * kOutChunkBytes + buf_off + lane * 64;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)   // 64-byte swizzle: piece j of row r at j ^ ((r >> 1) & 3)
+            *reinterpret_cast<uint4*>(row_ptr + ((j ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(p.out_map, stage0 + buf_off, nt * width + c * kOutChunkCols, row_base, g);
+            bulk_commit();
+          }
+          ++ochunk;
+        }
+      } else if (p.mode == kSwiGLU) {
         store_swiglu(tb, width, orow, valid);
-      else
+      } else {
         store_bf16(tb, kPairBn, orow, valid);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(peer_addr(smem_addr(&s.tempty[pipe.acc]), 0));
       pipe.acc ^= 1;
       if (pipe.acc == 0) pipe.acc_phase ^= 1u;
     }
+    if (lane == 0 && ochunk > 0) bulk_wait_all();   // this warp's stores are written before it exits
     __syncwarp();
   }
 }
 
-// Host side: tensor maps (cached) for a 3-D bf16 tensor [groups][rows][inner], box = 64 x
-// box_rows x 1, 128-byte swizzle, zero fill out of bounds.
+// Host side: tensor maps (cached) for a 3-D bf16 tensor [groups][rows][inner], box = box_inner
+// x box_rows x 1, zero fill out of bounds; 128-byte swizzle for 64-column operand boxes, 64-byte
+// swizzle for the 32-column output boxes of the TMA-store epilogue.
 cudaError_t make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
-                     uint64_t groups, uint32_t box_rows);
+                     uint64_t groups, uint32_t box_rows, uint32_t box_inner = BK);
 
 }  // namespace gemm
 }  // namespace moe

@@ -22,6 +22,17 @@ constexpr int kLaunchThreads = kThreads + 32 * kCopyWarps;
 
 enum SideKind : int { kSideNone = 0, kSideDispatch = 1, kSideCombine = 2 };
 
+// The copy warps' accesses carry an L2 evict-first policy (copy_phases.cuh, kStream).
+#ifndef MOE_STREAM_SIDE
+#define MOE_STREAM_SIDE 1
+#endif
+constexpr bool kStreamSide = MOE_STREAM_SIDE != 0;
+// Columns per lane per pass of a combine on the copy warps (copy_phases.cuh, accumulate_token).
+#ifndef MOE_SIDE_LANE_COLS
+#define MOE_SIDE_LANE_COLS 32
+#endif
+constexpr int kSideLaneCols = MOE_SIDE_LANE_COLS;
+
 struct SideArgs {
   int kind;
   int r;                       // round the side work belongs to
@@ -42,8 +53,8 @@ __device__ __forceinline__ void side_work(const SideArgs& sa) {
   const int cw = blockIdx.x * kCopyWarps + ((threadIdx.x >> 5) - kThreads / 32);
   const int warps = gridDim.x * kCopyWarps;
   if (sa.kind == kSideDispatch) {
-    copy::dispatch_rows(sa.x, sa.buf, sa.row_token, sa.row_dst, sa.row_start[sa.r], sa.row_start[sa.r + 1],
-                        sa.vecs, cw, warps, sa.dbg, sa.T, sa.buf_rows);
+    copy::dispatch_rows<kStreamSide>(sa.x, sa.buf, sa.row_token, sa.row_dst, sa.row_start[sa.r],
+                                     sa.row_start[sa.r + 1], sa.vecs, cw, warps, sa.dbg, sa.T, sa.buf_rows);
   } else if (sa.kind == kSideCombine) {
     if (sa.by_rows) {
       const int begin = sa.row_start[sa.r], end = sa.row_start[sa.r + 1];
@@ -53,10 +64,10 @@ __device__ __forceinline__ void side_work(const SideArgs& sa) {
           if ((threadIdx.x & 31) == 0) record_bad(sa.dbg, kBadCombineToken, row);
           continue;
         }
-        copy::combine_token(sa.comb, t, sa.r, sa.row_dst[row]);
+        copy::combine_token<kSideLaneCols, kStreamSide>(sa.comb, t, sa.r, sa.row_dst[row]);
       }
     } else {
-      for (int t = cw; t < sa.comb.T; t += warps) copy::combine_token(sa.comb, t, sa.r);
+      for (int t = cw; t < sa.comb.T; t += warps) copy::combine_token<kSideLaneCols, kStreamSide>(sa.comb, t, sa.r);
     }
   }
 }
@@ -79,12 +90,10 @@ struct KernelArgs {
   int32_t* status;
   const int32_t* group_row;        // pooled rows (see Phase), or null
   const int32_t* group_row_base;
-  const int32_t* gather_rows;      // fused gather of the A rows (see Phase), or null
-  const int32_t* gather_off;
   int rows_cap;                    // debug bounds checks (see Phase): 0 = unchecked
+  int tma_out;                     // CTA-pair form: store through the output map (see Phase)
 };
 
-template <bool kGather>
 __global__ void __launch_bounds__(kLaunchThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb0,
                         const __grid_constant__ CUtensorMap tb1, const __grid_constant__ CUtensorMap tb2,
@@ -117,10 +126,9 @@ __global__ void __launch_bounds__(kLaunchThreads, 1)
   p.n_valid = args.n_valid;
   p.group_row = args.group_row;
   p.group_row_base = args.group_row_base;
-  p.gather_rows = args.gather_rows;
-  p.gather_off = args.gather_off;
   p.rows_cap = args.rows_cap;
   p.dbg = args.rows_cap > 0 ? args.status - kHdrStatus : nullptr;
+  p.out_map = nullptr;
   plan_phase(s, p, 0);              // reads only the row counts (plan data)
   __syncthreads();
   // Everything above overlaps the previous kernel; the operands, and the output buffer that
@@ -129,7 +137,7 @@ __global__ void __launch_bounds__(kLaunchThreads, 1)
   pdl_trigger_early();
   Pipe pipe;
   if (threadIdx.x < kThreads)
-    run_phase<kGather>(s, tmem, p, 0, pipe, args.status);
+    run_phase(s, tmem, p, 0, pipe, args.status);
   else
     side_work(side);
   tc_fence_before();
@@ -142,12 +150,14 @@ __global__ void __launch_bounds__(kLaunchThreads, 1)
 // 256 tiles, one B map with 128-row boxes, a fixed width (SwiGLU 128 gate columns, Bf16Out 256).
 __global__ void __launch_bounds__(kLaunchThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
-                             const KernelArgs args, const SideArgs side, int width) {
+                             const __grid_constant__ CUtensorMap tout, const KernelArgs args, const SideArgs side,
+                             int width) {
   extern __shared__ uint8_t smem_raw[];
   const Smem s = carve(smem_raw);
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&ta);
     tma_prefetch_desc(&tb);
+    if (args.tma_out) tma_prefetch_desc(&tout);
   }
   const uint32_t tmem = setup_pair(s);
   Phase p;
@@ -171,10 +181,9 @@ __global__ void __launch_bounds__(kLaunchThreads, 1)
   p.n_valid = args.n_valid;
   p.group_row = args.group_row;
   p.group_row_base = args.group_row_base;
-  p.gather_rows = args.gather_rows;
-  p.gather_off = args.gather_off;
   p.rows_cap = args.rows_cap;
   p.dbg = args.rows_cap > 0 ? args.status - kHdrStatus : nullptr;
+  p.out_map = args.tma_out ? &tout : nullptr;
   plan_phase_pair(s, p, 0, width);
   __syncthreads();
   grid_dependency_wait();
@@ -210,20 +219,20 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// groups == 0 encodes a 2-D map [rows][inner] (the row-gather form: box_rows must be 1).
+// box_inner == BK: operand tiles (64 columns, 128-byte swizzle); box_inner == kOutChunkCols: the
+// TMA-store epilogue's output chunks (32 columns, 64-byte swizzle).
 static cudaError_t encode_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
-                              uint64_t groups, uint32_t box_rows) {
+                              uint64_t groups, uint32_t box_rows, uint32_t box_inner) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
-  const cuuint32_t rank = groups == 0 ? 2 : 3;
   const cuuint64_t dims[3] = {inner, rows, groups};
   const cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(BK), box_rows, 1};
+  const cuuint32_t box[3] = {box_inner, box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult res = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+  const CUresult res = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                          box_inner == BK ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return res == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
@@ -233,10 +242,10 @@ namespace {
 struct MapKey {
   const void* base;
   uint64_t inner, rows, groups;
-  uint32_t box_rows;
+  uint32_t box_rows, box_inner;
   bool operator==(const MapKey& o) const {
     return base == o.base && inner == o.inner && rows == o.rows && groups == o.groups &&
-           box_rows == o.box_rows;
+           box_rows == o.box_rows && box_inner == o.box_inner;
   }
 };
 constexpr int kMapCacheSize = 128;
@@ -250,17 +259,17 @@ std::mutex g_map_mutex;
 }  // namespace
 
 cudaError_t make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
-                     uint64_t groups, uint32_t box_rows) {
-  const MapKey key{base, inner, rows, groups, box_rows};
+                     uint64_t groups, uint32_t box_rows, uint32_t box_inner) {
+  const MapKey key{base, inner, rows, groups, box_rows, box_inner};
   const uint64_t h = ((reinterpret_cast<uintptr_t>(base) >> 8) * 0x9E3779B97F4A7C15ull) ^
-                     ((inner * 31 + rows) * 131 + groups * 7 + box_rows) * 0xC2B2AE3D27D4EB4Full;
+                     ((inner * 31 + rows) * 131 + groups * 7 + box_rows + box_inner * 3) * 0xC2B2AE3D27D4EB4Full;
   MapCacheEntry& slot = g_map_cache[(h >> 40) % kMapCacheSize];
   std::lock_guard<std::mutex> lock(g_map_mutex);
   if (slot.used && slot.key == key) {
     *map = slot.map;
     return cudaSuccess;
   }
-  const cudaError_t e = encode_map(map, base, inner, rows, groups, box_rows);
+  const cudaError_t e = encode_map(map, base, inner, rows, groups, box_rows, box_inner);
   if (e == cudaSuccess) {
     slot.used = true;
     slot.key = key;
@@ -317,21 +326,16 @@ static cudaError_t run(const CUtensorMap& a, const CUtensorMap* b, const KernelA
   cudaGetDevice(&dev);
   const uint64_t bit = 1ull << (dev & 63);
   if (!(configured.load() & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    const cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               kSmemBytes);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
   launch_begin(kind, stream);
   // with side work every SM takes part in the copy; otherwise one CTA per tile, at most one per SM
   const int grid = side.kind != kSideNone ? num_sms() : static_cast<int>(tiles < num_sms() ? tiles : num_sms());
-  const cudaError_t err = args.gather_rows
-                              ? launch_pdl(grouped_gemm_kernel<true>, dim3(grid), dim3(kLaunchThreads), kSmemBytes,
-                                           stream, a, b[0], b[1], b[2], args, side)
-                              : launch_pdl(grouped_gemm_kernel<false>, dim3(grid), dim3(kLaunchThreads), kSmemBytes,
-                                           stream, a, b[0], b[1], b[2], args, side);
+  const cudaError_t err = launch_pdl(grouped_gemm_kernel, dim3(grid), dim3(kLaunchThreads), kSmemBytes, stream,
+                                     a, b[0], b[1], b[2], args, side);
   launch_end(kind, stream);
   return err;
 }
@@ -385,8 +389,8 @@ static bool use_pair(const int32_t* n_host, int groups, int n_total, int width) 
   return clusters > 0 && pair_tiles >= clusters && rows_pair * 100 <= rows_single * 115;
 }
 
-static cudaError_t run_pair(const CUtensorMap& a, const CUtensorMap& b, const KernelArgs& args, int width,
-                            const SideArgs& side, int kind, cudaStream_t stream) {
+static cudaError_t run_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& out,
+                            const KernelArgs& args, int width, const SideArgs& side, int kind, cudaStream_t stream) {
   const int clusters = pair_clusters();   // every cluster takes part; the device counts the tiles
   launch_begin(kind, stream);
   cudaLaunchConfig_t cfg = {};
@@ -403,7 +407,7 @@ static cudaError_t run_pair(const CUtensorMap& a, const CUtensorMap& b, const Ke
   attr[1].val.programmaticStreamSerializationAllowed = MOE_PDL;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  const cudaError_t err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel, a, b, args, side, width);
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel, a, b, out, args, side, width);
   launch_end(kind, stream);
   return err;
 }
@@ -456,14 +460,10 @@ static gemm::SideArgs make_side(const RoundCopy* copy) {
 cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint16_t* h,
                            const int32_t* n_dev, const int32_t* n_host, int E, int C, int d, int F,
                            int32_t* status, const RoundCopy* copy, const int32_t* group_row,
-                           const int32_t* group_row_base, const GatherA* gather, cudaStream_t stream,
-                           int rows_cap) {
+                           const int32_t* group_row_base, cudaStream_t stream, int rows_cap) {
   CUtensorMap ma, mb[3];
   cudaError_t e = make_gate_up_maps(buf, w_gate_up, E, C, d, F, &ma, mb, group_row != nullptr);
   if (e != cudaSuccess) return e;
-  if (gather != nullptr) {   // A rows straight from x: a 2-D map whose box is one row high
-    if ((e = gemm::make_map(&ma, gather->x, d, gather->T, 0, 1)) != cudaSuccess) return e;
-  }
   gemm::KernelArgs a{};
   a.mode = gemm::kSwiGLU;
   for (int i = 0; i < 3; ++i) a.widths[i] = kGateUpWidths[i];
@@ -478,11 +478,13 @@ cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint1
   a.status = status;
   a.group_row = group_row;
   a.group_row_base = group_row_base;
-  a.gather_rows = gather ? gather->row_token : nullptr;
-  a.gather_off = gather ? gather->row_off : nullptr;
   a.rows_cap = rows_cap;
-  if (gemm::use_pair(n_host, E, F, 128))   // mb[0]: 128-row boxes of W1 and of W3
-    return gemm::run_pair(ma, mb[0], a, 128, make_side(copy), kKindGateUp, stream);
+  if (gemm::use_pair(n_host, E, F, 128)) {   // mb[0]: 128-row boxes of W1 and of W3
+    CUtensorMap mo{};
+    a.tma_out = group_row == nullptr;          // per-expert h [E][C][F]: stored by TMA
+    if (a.tma_out && (e = gemm::make_map(&mo, h, F, C, E, 32, gemm::kOutChunkCols)) != cudaSuccess) return e;
+    return gemm::run_pair(ma, mb[0], mo, a, 128, make_side(copy), kKindGateUp, stream);
+  }
   const long long tiles = gemm::choose_width(n_host, E, 0, F, a);
   return gemm::run(ma, mb, a, tiles, make_side(copy), kKindGateUp, stream);
 }
@@ -509,9 +511,11 @@ cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out
   a.group_row_base = group_row_base;
   a.rows_cap = rows_cap;
   if (gemm::use_pair(n_host, E, d, gemm::kPairBn)) {   // each CTA loads 128 of the tile's 256 W2 rows
-    CUtensorMap mb_half;
+    CUtensorMap mb_half, mo{};
     if ((e = gemm::make_map(&mb_half, w_down, F, d, E, gemm::kPairBHalf)) != cudaSuccess) return e;
-    return gemm::run_pair(ma, mb_half, a, gemm::kPairBn, make_side(copy), kKindDown, stream);
+    a.tma_out = group_row == nullptr;          // per-expert out [E][C][d]: stored by TMA
+    if (a.tma_out && (e = gemm::make_map(&mo, out, d, C, E, 32, gemm::kOutChunkCols)) != cudaSuccess) return e;
+    return gemm::run_pair(ma, mb_half, mo, a, gemm::kPairBn, make_side(copy), kKindDown, stream);
   }
   const long long tiles = gemm::choose_width(n_host, E, 0, d, a);
   return gemm::run(ma, mb, a, tiles, make_side(copy), kKindDown, stream);

@@ -196,16 +196,6 @@ struct RoundCopy {
   int32_t* dbg;              // the header when MOE_FLAG_DEBUG_BOUNDS is set, else null
 };
 
-// Fused gather of a gate/up GEMM's A rows: row i of expert e's rows in the round is
-// x[row_token[row_off[e] + i]] (row_off: the round's row of the row_off table), read by TMA row
-// gathers instead of from the dispatch buffer, which the round then never needs.
-struct GatherA {
-  const uint16_t* x;         // [T, d] bf16
-  int T;
-  const int32_t* row_token;  // the round-major row list's source tokens
-  const int32_t* row_off;    // [E]: position of expert e's first row of the round in the list
-};
-
 // rows_cap > 0 (debug bounds checks): an expert's device row count above it is recorded in the
 // header and clamped.
 // n_dev: rows per expert this round on the device (read by the kernel); n_host: the same on
@@ -215,8 +205,7 @@ struct GatherA {
 cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint16_t* h,
                            const int32_t* n_dev, const int32_t* n_host, int E, int C, int d, int F,
                            int32_t* status, const RoundCopy* copy, const int32_t* group_row,
-                           const int32_t* group_row_base, const GatherA* gather, cudaStream_t stream,
-                           int rows_cap = 0);
+                           const int32_t* group_row_base, cudaStream_t stream, int rows_cap = 0);
 // down: out[e][s] = bf16(h[e][s] W2_e^T), s < n_dev[e]
 cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out, const int32_t* n_dev,
                         const int32_t* n_host, int E, int C, int d, int F, int32_t* status,

@@ -312,22 +312,18 @@ RoundCopy make_copy(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
   return c;
 }
 
-// x_gather: gather the round's A rows from x (the forward's own rounds), or null to read them
-// from the dispatch buffer that moe_round_dispatch filled.
 int do_gate_up(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
                const moe_workspace_layout_t& L, int r, const uint16_t* w13, const RoundCopy* copy,
-               const uint16_t* x_gather, cudaStream_t stream) {
+               cudaStream_t stream) {
   int32_t n_host[MOE_MAX_EXPERTS];
   int rows = 0;
   round_rows(s, info, r, n_host, &rows);
   const bool pooled = borrowing(s);
-  GatherA g{x_gather, s->T, at<int32_t>(ws, L.row_token), at<int32_t>(ws, L.row_off) + static_cast<size_t>(r) * s->E};
   return cuda_status(launch_gate_up(at<uint16_t>(ws, L.buf), w13, at<uint16_t>(ws, L.h),
                                     at<int32_t>(ws, L.n) + static_cast<size_t>(r) * s->E, n_host, s->E,
                                     s->C, s->d, s->d_ff, at<int32_t>(ws, L.header) + kHdrStatus, copy,
                                     pooled ? at<int32_t>(ws, L.row_off) + static_cast<size_t>(r) * s->E : nullptr,
-                                    pooled ? at<int32_t>(ws, L.row_start) + r : nullptr,
-                                    x_gather ? &g : nullptr, stream, rows_cap(s)));
+                                    pooled ? at<int32_t>(ws, L.row_start) + r : nullptr, stream, rows_cap(s)));
 }
 
 int do_down(const moe_shape_t* s, const moe_plan_info_t* info, void* ws,
@@ -601,7 +597,7 @@ int moe_round_gate_up(const moe_shape_t* shape, const moe_plan_info_t* info, voi
   if (st != MOE_OK) return st;
   if (r < 0 || r >= info->R || w_gate_up == nullptr) return MOE_ERR_INVALID_ARG;
   if (!aligned(w_gate_up, 16)) return MOE_ERR_MISALIGNED;
-  return do_gate_up(shape, info, ws, L, r, w_gate_up, nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream));
+  return do_gate_up(shape, info, ws, L, r, w_gate_up, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int moe_round_down(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
@@ -665,47 +661,51 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
     // borrowing and the debug bounds checks run per round only
     while (r0 > 0 && thin(r0 - 1)) --r0;
   }
-  // Per-round launch order. The gate/up GEMM of a round gathers its rows straight from x (TMA
-  // row gathers of the round-major row list), so these rounds need no dispatch step. A round's
-  // combine rides on the next round's gate/up launch as its copy warps when it is small (at most
-  // kFuseCopyBytes of rows) or when its estimated time there stays below that GEMM's; otherwise it
-  // runs as its own full-bandwidth kernel right after its down GEMM. Each launch depends only on
-  // the one before it (PDL wait), and no two steps of one launch touch the same buffer: gate/up
-  // reads x and writes h, down reads h and writes out, combine reads out and updates y. The first
-  // pipelined round is dispatched into buf here too (on the last per-round down GEMM's copy warps,
-  // or by the dispatch kernel), so the pipelined launch starts with its rows in place.
+  // Per-round launch order. A round's copy steps ride on the neighbouring GEMM launches as
+  // their copy warps -- combine(r-1) on gate/up(r), dispatch(r+1) on down(r) -- when they are
+  // small (at most kFuseCopyBytes of rows) or when their estimated time there stays below that
+  // GEMM's; otherwise they run as their own full-bandwidth kernels, dispatch(r+1) right after
+  // down(r), combine(r) after that. Each launch depends only on the one before it (PDL wait), and
+  // no two steps of one launch touch the same buffer: dispatch writes buf, gate/up reads buf and
+  // writes h, down reads h and writes out, combine reads out and updates y. The first pipelined
+  // round is dispatched here too, so the pipelined launch starts with its rows in place.
   auto rows_of = [&](int rr) {
     int32_t n_host[MOE_MAX_EXPERTS];
     int rows = 0;
     round_rows(shape, info, rr, n_host, &rows);
     return rows;
   };
-  auto combine_rides = [&](int rc, int rg) {
+  // copy warps move about kSideCopyGBs while the GEMM runs at about kGemmTflops
+  auto side_s = [&](double bytes) { return bytes / (kSideCopyGBs * 1e9); };
+  auto gemm_s = [&](double flops) { return flops / (kGemmTflops * 1e12); };
+  auto combine_rides = [&](int rc, int rg) {   // combine(rc) on gate/up(rg)
     if (small(rc)) return true;
-    // copy warps move about kSideCopyGBs; the GEMM runs at about kGemmTflops
     const double rows_c = rows_of(rc), tokens_c = rows_c < shape->T ? rows_c : shape->T;
-    const double t_copy = (2.0 * rows_c + 8.0 * tokens_c) * shape->d / (kSideCopyGBs * 1e9);
-    const double t_gemm = 4.0 * rows_of(rg) * shape->d * shape->d_ff / (kGemmTflops * 1e12);
-    return t_copy <= t_gemm;
+    return side_s((2.0 * rows_c + 8.0 * tokens_c) * shape->d) <=
+           gemm_s(4.0 * rows_of(rg) * shape->d * shape->d_ff);
+  };
+  auto dispatch_rides = [&](int rd, int rg) {   // dispatch(rd) on down(rg)
+    if (small(rd)) return true;
+    return side_s(4.0 * rows_of(rd) * shape->d) <= gemm_s(2.0 * rows_of(rg) * shape->d * shape->d_ff);
   };
   auto per_round = [&](int rb, int re) -> int {
     int rc = MOE_OK;
     for (int r = rb; r < re; ++r) {
       const bool fuse_combine = r > rb && combine_rides(r - 1, r);
       const RoundCopy comb = make_copy(shape, info, ws, L, true, r > 0 ? r - 1 : 0, x, y);
-      if ((rc = do_gate_up(shape, info, ws, L, r, w_gate_up, fuse_combine ? &comb : nullptr, x, stream)) != MOE_OK)
+      if ((rc = do_gate_up(shape, info, ws, L, r, w_gate_up, fuse_combine ? &comb : nullptr, stream)) != MOE_OK)
         return rc;
-      const bool pipe_next = r + 1 == re && re < R;   // the pipelined launch takes round r + 1
-      const bool fuse_dispatch = pipe_next && small(r + 1);
-      const RoundCopy disp = make_copy(shape, info, ws, L, false, pipe_next ? r + 1 : r, x, y);
+      const bool next = r + 1 < R;
+      const bool fuse_dispatch = next && dispatch_rides(r + 1, r);
+      const RoundCopy disp = make_copy(shape, info, ws, L, false, next ? r + 1 : r, x, y);
       if ((rc = do_down(shape, info, ws, L, r, w_down, fuse_dispatch ? &disp : nullptr, stream)) != MOE_OK) return rc;
-      if (pipe_next && !fuse_dispatch && (rc = do_dispatch(shape, info, ws, L, r + 1, x, stream)) != MOE_OK) return rc;
+      if (next && !fuse_dispatch && (rc = do_dispatch(shape, info, ws, L, r + 1, x, stream)) != MOE_OK) return rc;
       if (!(r + 1 < re && combine_rides(r, r + 1)) && (rc = do_combine(shape, info, ws, L, r, y, stream)) != MOE_OK)
         return rc;
     }
     return rc;
   };
-  if (r0 == 0 && (st = do_dispatch(shape, info, ws, L, 0, x, stream)) != MOE_OK) return st;
+  if ((st = do_dispatch(shape, info, ws, L, 0, x, stream)) != MOE_OK) return st;
   if ((st = per_round(0, r0)) != MOE_OK) return st;
   if (r0 < R) {
     PipelineArgs p{};
