@@ -21,7 +21,7 @@ LIB_DIR = os.path.join(PKG, "lib")
 LIB_PATH = os.path.join(LIB_DIR, "libmoe.so")
 
 SOURCES = ["moe_api.cu", "router.cu", "plan.cu", "dispatch_combine.cu", "grouped_gemm.cu",
-           "round_pipeline.cu", "noalloc.cu", "backward.cu", "ep_plan.cu"]
+           "round_pipeline.cu", "noalloc.cu", "backward.cu", "ep_plan.cu", "ep_round.cu"]
 HEADERS = ["kernels.h", "backward.h", "sm100.cuh", "gemm_sm100.cuh", "copy_phases.cuh"]
 
 NVCC_FLAGS = [

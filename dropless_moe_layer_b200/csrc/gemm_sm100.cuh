@@ -164,7 +164,12 @@ struct Phase {
   // TMA-store epilogue (CTA-pair form, per-expert outputs only): the output as a 3-D map [groups]
   // [rows][n_total] with 32 x 32 boxes and the 64-byte swizzle. Null: 16-byte stores per thread.
   const CUtensorMap* out_map;
+  // Weights of group g: expert group_expert[g] of the B map (expert parallelism: a group is one
+  // source rank's rows of one local expert). Null: expert g.
+  const int32_t* group_expert;
 };
+
+__device__ __forceinline__ int group_weights(const Phase& p, int g) { return p.group_expert ? p.group_expert[g] : g; }
 
 // Rows of group g (clamped to rows_cap under the debug bounds checks).
 __device__ __forceinline__ int group_rows(const Phase& p, int g) {
@@ -352,10 +357,10 @@ __device__ __forceinline__ void run_phase(const Smem& s, uint32_t tmem_base, con
         mbar_arrive_expect_tx(fb, tx);
         tma_load_3d(sA, p.a, fb, kb * BK, a_row, a_grp);
         if (p.mode == kSwiGLU) {
-          tma_load_3d(sB, mb, fb, kb * BK, nt * width, g);
-          tma_load_3d(sB + width * BK * 2, mb, fb, kb * BK, p.b_second_row + nt * width, g);
+          tma_load_3d(sB, mb, fb, kb * BK, nt * width, group_weights(p, g));
+          tma_load_3d(sB + width * BK * 2, mb, fb, kb * BK, p.b_second_row + nt * width, group_weights(p, g));
         } else {
-          tma_load_3d(sB, mb, fb, kb * BK, nt * width, g);
+          tma_load_3d(sB, mb, fb, kb * BK, nt * width, group_weights(p, g));
         }
         pipe.issued |= 1u << pipe.stage;
         pipe.issued_parity = (pipe.issued_parity & ~(1u << pipe.stage)) | (pipe.phase << pipe.stage);
@@ -610,7 +615,7 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
         __syncwarp();
         if (lane == 0) {
           tma_load_3d_pair(sA, p.a, fb, kb * BK, a_row, a_grp);
-          tma_load_3d_pair(sB, p.b[0], fb, kb * BK, b_row(nt), g);
+          tma_load_3d_pair(sB, p.b[0], fb, kb * BK, b_row(nt), group_weights(p, g));
         }
         pipe.issued |= 1u << pipe.stage;
         if (++pipe.stage == kPairStages) {
@@ -677,6 +682,8 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
     const int q = warp & 3;
     uint32_t ochunk = 0;   // chunks this warp has staged (alternates its two buffers)
     const uint32_t stage0 = smem_addr(s.out_stage + q * 2 * kOutChunkBytes);
+    // the outputs stream out: first in line for eviction, behind the tiles the MMAs still reuse
+    const uint64_t out_policy = policy_evict_first();
     for (int tile = pair; tile < total; tile += pairs) {
       int g, mp, nt;
       decode(tile, g, mp, nt);
@@ -731,7 +738,7 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
           fence_async_shared();
           __syncwarp();
           if (lane == 0) {
-            tma_store_3d(p.out_map, stage0 + buf_off, nt * width + c * kOutChunkCols, row_base, g);
+            tma_store_3d(p.out_map, stage0 + buf_off, nt * width + c * kOutChunkCols, row_base, g, out_policy);
             bulk_commit();
           }
           ++ochunk;

@@ -29,7 +29,7 @@ enum SideKind : int { kSideNone = 0, kSideDispatch = 1, kSideCombine = 2 };
 constexpr bool kStreamSide = MOE_STREAM_SIDE != 0;
 // Columns per lane per pass of a combine on the copy warps (copy_phases.cuh, accumulate_token).
 #ifndef MOE_SIDE_LANE_COLS
-#define MOE_SIDE_LANE_COLS 32
+#define MOE_SIDE_LANE_COLS 16
 #endif
 constexpr int kSideLaneCols = MOE_SIDE_LANE_COLS;
 
@@ -92,6 +92,7 @@ struct KernelArgs {
   const int32_t* group_row_base;
   int rows_cap;                    // debug bounds checks (see Phase): 0 = unchecked
   int tma_out;                     // CTA-pair form: store through the output map (see Phase)
+  const int32_t* group_expert;     // weights of each group (see Phase), or null
 };
 
 __global__ void __launch_bounds__(kLaunchThreads, 1)
@@ -129,6 +130,7 @@ __global__ void __launch_bounds__(kLaunchThreads, 1)
   p.rows_cap = args.rows_cap;
   p.dbg = args.rows_cap > 0 ? args.status - kHdrStatus : nullptr;
   p.out_map = nullptr;
+  p.group_expert = args.group_expert;
   plan_phase(s, p, 0);              // reads only the row counts (plan data)
   __syncthreads();
   // Everything above overlaps the previous kernel; the operands, and the output buffer that
@@ -184,6 +186,7 @@ __global__ void __launch_bounds__(kLaunchThreads, 1)
   p.rows_cap = args.rows_cap;
   p.dbg = args.rows_cap > 0 ? args.status - kHdrStatus : nullptr;
   p.out_map = args.tma_out ? &tout : nullptr;
+  p.group_expert = args.group_expert;
   plan_phase_pair(s, p, 0, width);
   __syncthreads();
   grid_dependency_wait();
@@ -340,6 +343,10 @@ static cudaError_t run(const CUtensorMap& a, const CUtensorMap* b, const KernelA
   return err;
 }
 
+#ifndef MOE_TMA_OUT_GATE_UP
+#define MOE_TMA_OUT_GATE_UP 1   // 0: the pair gate/up GEMM stores h with per-thread stores
+#endif
+
 #ifndef MOE_GEMM_PAIR
 #define MOE_GEMM_PAIR 1   // 0: never use the CTA-pair form
 #endif
@@ -481,7 +488,7 @@ cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint1
   a.rows_cap = rows_cap;
   if (gemm::use_pair(n_host, E, F, 128)) {   // mb[0]: 128-row boxes of W1 and of W3
     CUtensorMap mo{};
-    a.tma_out = group_row == nullptr;          // per-expert h [E][C][F]: stored by TMA
+    a.tma_out = MOE_TMA_OUT_GATE_UP && group_row == nullptr;   // per-expert h [E][C][F]: stored by TMA
     if (a.tma_out && (e = gemm::make_map(&mo, h, F, C, E, 32, gemm::kOutChunkCols)) != cudaSuccess) return e;
     return gemm::run_pair(ma, mb[0], mo, a, 128, make_side(copy), kKindGateUp, stream);
   }
@@ -519,6 +526,63 @@ cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out
   }
   const long long tiles = gemm::choose_width(n_host, E, 0, d, a);
   return gemm::run(ma, mb, a, tiles, make_side(copy), kKindDown, stream);
+}
+
+cudaError_t launch_ep_experts(const uint16_t* recv, const uint16_t* w_gate_up, const uint16_t* w_down, uint16_t* h,
+                              uint16_t* out, int groups, const int32_t* rows_dev, const int32_t* rows_host,
+                              const int32_t* group_row_dev, const int32_t* group_expert_dev, long long buf_rows,
+                              int E_local, int d, int F, int32_t* status, cudaStream_t stream) {
+  // gate/up: h[rows of group g] = bf16(silu(recv W1_e^T) * (recv W3_e^T)), e = group_expert[g]
+  CUtensorMap ma, mb[3];
+  cudaError_t e = gemm::make_map(&ma, recv, d, static_cast<uint64_t>(buf_rows), 1, gemm::BM);
+  if (e != cudaSuccess) return e;
+  if ((e = gemm::make_b_maps(mb, w_gate_up, d, 2ull * F, E_local, kGateUpWidths, F)) != cudaSuccess) return e;
+  gemm::KernelArgs a{};
+  a.mode = gemm::kSwiGLU;
+  for (int i = 0; i < 3; ++i) a.widths[i] = kGateUpWidths[i];
+  a.rows = rows_dev;
+  a.groups = groups;
+  a.num_k_blocks = d / gemm::BK;
+  a.n_total = F;
+  a.b_second_row = F;
+  a.out = h;
+  a.out_ld = F;
+  a.status = status;
+  a.group_row = group_row_dev;        // groups are packed from row 0: group 0 starts at offset 0,
+  a.group_row_base = group_row_dev;   // so its entry doubles as the base
+  a.group_expert = group_expert_dev;
+  const gemm::SideArgs none = make_side(nullptr);
+  if (gemm::use_pair(rows_host, groups, F, 128)) {
+    CUtensorMap unused{};
+    e = gemm::run_pair(ma, mb[0], unused, a, 128, none, kKindGateUp, stream);
+  } else {
+    const long long tiles = gemm::choose_width(rows_host, groups, 0, F, a);
+    e = gemm::run(ma, mb, a, tiles, none, kKindGateUp, stream);
+  }
+  if (e != cudaSuccess) return e;
+  // down: out[rows of group g] = bf16(h W2_e^T)
+  if ((e = gemm::make_map(&ma, h, F, static_cast<uint64_t>(buf_rows), 1, gemm::BM)) != cudaSuccess) return e;
+  gemm::KernelArgs b{};
+  b.mode = gemm::kBf16Out;
+  for (int i = 0; i < 3; ++i) b.widths[i] = kDownWidths[i];
+  b.rows = rows_dev;
+  b.groups = groups;
+  b.num_k_blocks = F / gemm::BK;
+  b.n_total = d;
+  b.out = out;
+  b.out_ld = d;
+  b.status = status;
+  b.group_row = group_row_dev;
+  b.group_row_base = group_row_dev;
+  b.group_expert = group_expert_dev;
+  if (gemm::use_pair(rows_host, groups, d, gemm::kPairBn)) {
+    CUtensorMap mb_half, unused{};
+    if ((e = gemm::make_map(&mb_half, w_down, F, d, E_local, gemm::kPairBHalf)) != cudaSuccess) return e;
+    return gemm::run_pair(ma, mb_half, unused, b, gemm::kPairBn, none, kKindDown, stream);
+  }
+  if ((e = gemm::make_b_maps(mb, w_down, F, d, E_local, kDownWidths, d)) != cudaSuccess) return e;
+  const long long tiles = gemm::choose_width(rows_host, groups, 0, d, b);
+  return gemm::run(ma, mb, b, tiles, none, kKindDown, stream);
 }
 
 cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* w_router, const float* bias,

@@ -240,6 +240,16 @@ struct PipelineArgs {
 };
 cudaError_t launch_round_pipeline(const PipelineArgs& a, cudaStream_t stream);
 
+// Expert parallelism, owner side of round r: both grouped GEMMs over the rows received from every
+// source rank, one group per (source rank, local expert) in that order, packed from row 0 of
+// recv (group g at row group_row[g], rows[g] rows), weights of local expert group_expert[g] of
+// w_gate_up [E_local, 2 d_ff, d] and w_down [E_local, d, d_ff]; h and out hold the same rows.
+// recv, h and out have buf_rows rows each.
+cudaError_t launch_ep_experts(const uint16_t* recv, const uint16_t* w_gate_up, const uint16_t* w_down, uint16_t* h,
+                              uint16_t* out, int groups, const int32_t* rows_dev, const int32_t* rows_host,
+                              const int32_t* group_row_dev, const int32_t* group_expert_dev, long long buf_rows,
+                              int E_local, int d, int F, int32_t* status, cudaStream_t stream);
+
 // router GEMM: logits[t][e] = x[t] . w_router[e] + bias[e] (fp32 out)
 cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* w_router, const float* bias,
                                float* logits, int T, int d, int E, int32_t* status,

@@ -103,6 +103,14 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_plan_noalloc": (ctypes.c_int, [P(Shape), c_vp, c_vp, c_vp, c_vp, c_vp, P(c_i32), P(c_i32), c_vp]),
         "moe_ep_exchange_plan": (ctypes.c_int, [P(Shape), c_i32, c_i32, P(c_i32), c_i32, P(c_i32), P(c_i32),
                                                 P(c_i32), P(c_i32), P(c_i32), P(c_i32), P(c_i32)]),
+        "moe_ep_workspace_bytes": (c_sz, [P(Shape), c_i32]),
+        "moe_ep_plan": (ctypes.c_int, [P(Shape), c_i32, c_i32, P(c_i32), P(PlanInfo), c_vp, c_sz, c_vp, c_sz,
+                                       P(c_i32), c_vp]),
+        "moe_ep_round_pack": (ctypes.c_int, [P(Shape), c_i32, c_i32, P(c_i32), c_vp, c_sz, c_i32, c_vp, c_vp, c_vp]),
+        "moe_ep_round_experts": (ctypes.c_int, [P(Shape), c_i32, c_i32, P(c_i32), c_vp, c_sz, c_i32, c_vp, c_vp,
+                                                c_vp, c_vp, c_vp, ctypes.c_int64, c_vp, c_vp]),
+        "moe_ep_round_combine": (ctypes.c_int, [P(Shape), c_i32, c_i32, P(c_i32), c_vp, c_sz, c_vp, c_sz, c_i32,
+                                                c_vp, c_vp, c_vp]),
         "moe_backward_workspace_bytes": (c_sz, [P(Shape)]),
         "moe_backward_workspace_layout": (ctypes.c_int, [P(Shape), P(BackwardLayout)]),
         "moe_backward": (ctypes.c_int, [P(Shape), P(PlanInfo), c_vp, c_sz, c_vp, c_sz, c_vp, c_vp, c_vp,

@@ -10,6 +10,7 @@ appears a known number of times) or as a quick check that a shape runs on this G
 --tokens N replaces the workload's token count (the other sizes, the routing recipe and the
 seed stay), so a kernel can be profiled on a case that holds less device memory.
 --plan-only skips the expert weights and runs only the router and the planner.
+--backward also runs the backward pass (moe_backward) after each forward.
 """
 from __future__ import annotations
 
@@ -31,6 +32,7 @@ def main() -> None:
     ap.add_argument("--plan-only", action="store_true", help="router + planner only (no expert weights)")
     ap.add_argument("--schedule", default="auto", choices=sorted(moe.SCHEDULES))
     ap.add_argument("--borrow", action="store_true")
+    ap.add_argument("--backward", action="store_true", help="also run the backward pass after each forward")
     args = ap.parse_args()
     w = wl.BY_NAME[args.workload]
     if args.tokens > 0:
@@ -42,12 +44,15 @@ def main() -> None:
     layer = moe.DroplessMoE(w.T, w.d, w.E, w.k, w.F, w.C, device=dev, schedule=args.schedule,
                             borrow=args.borrow)
     y = None if args.plan_only else torch.empty(w.T, w.d, dtype=torch.float32, device=dev)
+    dy = wl.generate_dy(w, dev) if args.backward and not args.plan_only else None
     before = moe.launch_count()
     for _ in range(args.steps):
         layer.plan(logits=inp["logits"], x=inp["x"] if w.router == "gemm" else None,
                    w_router=inp["w_router"], bias=inp["bias"])
         if not args.plan_only:
             layer.forward(inp["x"], inp["w_gate_up"], inp["w_down"], y=y)
+        if dy is not None:
+            layer.backward(inp["x"], inp["w_gate_up"], inp["w_down"], dy)
     torch.cuda.synchronize(dev)
     status = layer.device_status()
     print(json.dumps({"workload": w.name, "T": w.T, "steps": args.steps, "rounds": layer.info.R,

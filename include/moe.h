@@ -334,6 +334,44 @@ MOE_API int moe_ep_exchange_plan(const moe_shape_t* shape, int32_t G, int32_t ra
                                  int32_t* send_offsets, int32_t* recv_counts, int32_t* recv_offsets,
                                  int32_t* n_owned);
 
+/* Device data path of the expert-parallel layer, one round at a time (same sources and
+ * readings as moe_ep_exchange_plan above). Every rank holds T tokens. Per round r, each rank:
+ *   moe_ep_round_pack:     its pairs of round r, in (expert, slot) order, x rows -> sendbuf; the
+ *                          rows for owner g are the chunk at send_offsets[r][g] (send_counts)
+ *   (the caller's all-to-all: chunk g of every rank's sendbuf -> rank g's recvbuf, in source order)
+ *   moe_ep_round_experts:  on the owner, both grouped GEMMs straight over the received rows, one
+ *                          group per (source rank, local expert): h = bf16(silu(recv W1^T) *
+ *                          (recv W3^T)), out = bf16(h W2^T), out in the order of recvbuf
+ *   (the all-to-all back: chunk s of out -> rank s's retbuf)
+ *   moe_ep_round_combine:  y[t] (+)= gate * retbuf row for its pairs of round r, j ascending
+ * The rank's plan comes from moe_plan on its own tokens (without MOE_FLAG_BORROW) followed by
+ * moe_ep_plan, which re-ranks every pair among all ranks' pairs of its expert. Buffers (device,
+ * caller-owned, bf16, 16-byte aligned): sendbuf and retbuf hold min(T*k, E*C) rows of d; recvbuf
+ * and out hold buf_rows >= E/G * C rows of d, h buf_rows rows of d_ff. loads is the host [G, E]
+ * table of every rank's pair counts (all-gathered), the same on every rank.
+ *
+ * Bytes of the plan tables of one rank over G ranks (0 for an invalid shape or G). */
+MOE_API size_t moe_ep_workspace_bytes(const moe_shape_t* shape, int32_t G);
+/* Re-plans this rank's pairs (info/ws from moe_plan on this rank's tokens): global round, slot
+ * within the rank's rows of (round, expert), packed row list. R: host out, the job's rounds.
+ * Synchronizes `stream` once. MOE_ERR_INVALID_ARG if loads do not match info's loads, a rank
+ * holds more than T tokens, or the plan used borrowing. */
+MOE_API int moe_ep_plan(const moe_shape_t* shape, int32_t G, int32_t rank, const int32_t* loads,
+                        const moe_plan_info_t* info, void* ws, size_t ws_bytes, void* ep_ws, size_t ep_bytes,
+                        int32_t* R, moe_stream_t stream);
+MOE_API int moe_ep_round_pack(const moe_shape_t* shape, int32_t G, int32_t rank, const int32_t* loads,
+                              void* ep_ws, size_t ep_bytes, int32_t r, const uint16_t* x, uint16_t* sendbuf,
+                              moe_stream_t stream);
+/* w_gate_up [E/G, 2*d_ff, d] and w_down [E/G, d, d_ff]: this rank's own experts. ws: this rank's
+ * workspace (its status word records bounded-wait time-outs). Synchronizes `stream` once. */
+MOE_API int moe_ep_round_experts(const moe_shape_t* shape, int32_t G, int32_t rank, const int32_t* loads,
+                                 void* ep_ws, size_t ep_bytes, int32_t r, const uint16_t* recvbuf,
+                                 const uint16_t* w_gate_up, const uint16_t* w_down, uint16_t* h, uint16_t* out,
+                                 int64_t buf_rows, void* ws, moe_stream_t stream);
+MOE_API int moe_ep_round_combine(const moe_shape_t* shape, int32_t G, int32_t rank, const int32_t* loads,
+                                 void* ws, size_t ws_bytes, void* ep_ws, size_t ep_bytes, int32_t r,
+                                 const uint16_t* retbuf, float* y, moe_stream_t stream);
+
 /* Routing and round plan with no device allocation at all.
  *
  * The pages have no counterpart to this call; it exists for callers that cannot

@@ -104,3 +104,13 @@ def test_exchange_plan_rejects_bad_arguments():
     bad = ok.copy()
     bad[1, 0] = -1
     assert call(2, 0, bad) == -1
+
+
+def test_ep_workspace_size_is_fixed_by_shape_and_ranks():
+    lib = moe.load_library()
+    s = moe.make_shape(256, 128, 8, 2, 256, 32)
+    n2, n4 = lib.moe_ep_workspace_bytes(__import__("ctypes").byref(s), 2), lib.moe_ep_workspace_bytes(
+        __import__("ctypes").byref(s), 4)
+    assert 0 < n2 < n4                               # more ranks: more possible rounds to plan
+    assert lib.moe_ep_workspace_bytes(__import__("ctypes").byref(s), 3) == 0     # 8 experts over 3 ranks
+    assert lib.moe_ep_workspace_bytes(__import__("ctypes").byref(s), 0) == 0
