@@ -284,6 +284,40 @@ def combine_bytes(w, round_np, rounds=None):
     return total
 
 
+# The library's rule for which copy steps ride on a neighbouring GEMM launch (moe_api.cu,
+# moe_forward): small steps always; larger ones when their bytes at the copy warps' rate stay
+# below the GEMM's flops at its rate. Mirrored here only to split the work between kernel kinds.
+FUSE_COPY_BYTES = 32 << 20
+SIDE_COPY_GBS = 2000.0
+GEMM_TFLOPS = 1100.0
+
+
+def ride_plan(w, n, r0):
+    """For per-round rounds [0, r0): sets of rounds whose combine rides on the next gate/up launch
+    and whose dispatch rides on the previous down launch (n: rows per (round, expert))."""
+    rows = [int(v) for v in np.asarray(n).sum(axis=1)]
+    R = len(rows)
+
+    def small(r):
+        return rows[r] * w.d * 2 <= FUSE_COPY_BYTES
+
+    def combine_rides(rc, rg):
+        if small(rc):
+            return True
+        tokens = min(rows[rc], w.T)
+        return (2.0 * rows[rc] + 8.0 * tokens) * w.d / (SIDE_COPY_GBS * 1e9) <= \
+            4.0 * rows[rg] * w.d * w.F / (GEMM_TFLOPS * 1e12)
+
+    def dispatch_rides(rd, rg):
+        if small(rd):
+            return True
+        return 4.0 * rows[rd] * w.d / (SIDE_COPY_GBS * 1e9) <= 2.0 * rows[rg] * w.d * w.F / (GEMM_TFLOPS * 1e12)
+
+    comb = {r for r in range(r0) if r + 1 < r0 and combine_rides(r, r + 1)}
+    disp = {r + 1 for r in range(r0) if r + 1 < R and dispatch_rides(r + 1, r)}
+    return comb, disp
+
+
 def algorithmic_work(w, info, r0, round_np, n_plan=None):
     """Per kernel kind, the algorithmic units of one step, from the plan alone (padding rows
     C - n never count). Per-round kernels cover rounds [0, r0), the pipelined launch [r0, R).
@@ -296,16 +330,19 @@ def algorithmic_work(w, info, r0, round_np, n_plan=None):
     pipe = n[r0:]
     prow = int(pipe.sum())
     d, F = w.d, w.F
+    rode_comb, rode_disp = ride_plan(w, n, r0)
+    # stand-alone copy kernels: round 0's dispatch, and the per-round steps that do not ride
+    disp_rounds = [r for r in range(min(r0 + 1, info.R)) if r == 0 or r not in rode_disp]
+    comb_rounds = {r for r in range(r0) if r not in rode_comb}
     work = {
         "router_gemm": ("hbm", (w.T * w.d * 2 + w.E * w.d * 2 + w.T * w.E * 4) if w.router == "gemm" else 0),
         "topk": ("hbm", w.T * w.E * 4 + w.T * w.k * 8),
         "plan": ("hbm", w.T * w.k * 4 * 6),
-        # the per-round gate/up GEMMs gather their rows from x; only the pipelined launch's first
-        # round is dispatched into a buffer (x rows in, buffer rows out) before that launch
-        "dispatch": ("hbm", 2 * int(pipe[0].sum()) * d * 2 if len(pipe) else 0),
+        # copy steps that ride on a GEMM launch are done inside that launch (its kind's time)
+        "dispatch": ("hbm", 2 * int(sum(n[r].sum() for r in disp_rounds)) * d * 2),
         "gate_up": ("tensor", 4 * int(per) * d * F),
         "down": ("tensor", 2 * int(per) * F * d),
-        "combine": ("hbm", combine_bytes(w, round_np, set(range(r0))) if r0 > 0 else 0),
+        "combine": ("hbm", combine_bytes(w, round_np, comb_rounds) if comb_rounds else 0),
     }
     if prow:
         flops = 6 * prow * d * F

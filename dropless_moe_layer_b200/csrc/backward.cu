@@ -86,6 +86,8 @@ struct GemmArgs {
   float* dgate_part;          // kDh: [E * C][dgate_ld] partial sums of <W2^T dy, h>
   int dgate_ld;
   int overwrite;              // kWgrad: store the tile instead of adding it (round 0)
+  int tma_out;                // kWgrad: write the tile through the phase's fp32 output map (TMA
+                              // store, or TMA reduce-add) instead of per-thread read-add-write
   int32_t* status;
 };
 
@@ -280,6 +282,43 @@ __device__ __forceinline__ void epi_wgrad(const GemmArgs& p, uint32_t tb, int g,
   }
 }
 
+// The same through TMA: each 32-column slice of the accumulator row goes to this warp's staging
+// buffer as two 16-column fp32 chunks (64-byte swizzle, 32 rows by 64 bytes), which one bulk
+// store (round 0) or one bulk reduce-add (later rounds) writes into the gradient. The add happens
+// in the memory system; every element still gets one fp32 addition per round, in round order.
+__device__ __forceinline__ void epi_wgrad_tma(const GemmArgs& p, const CUtensorMap* map, uint32_t tb, int g,
+                                              int row_base, int nt, uint8_t* stage, uint32_t& ochunk) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t stage_addr = smem_addr(stage);
+  for (int c = 0; c < p.width; c += 32) {
+    uint32_t v[32];
+    tmem_ld32(tb + c, v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t buf_off = (ochunk & 1u) * gemm::kOutChunkBytes;
+      if (lane == 0) bulk_wait_read_1();   // the write that last used this buffer has read it
+      __syncwarp();
+      uint8_t* row_ptr = stage + buf_off + lane * 64;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)   // 64-byte swizzle: piece j of row r at j ^ ((r >> 1) & 3)
+        *reinterpret_cast<uint4*>(row_ptr + ((j ^ ((lane >> 1) & 3)) << 4)) =
+            make_uint4(v[16 * h + 4 * j], v[16 * h + 4 * j + 1], v[16 * h + 4 * j + 2], v[16 * h + 4 * j + 3]);
+      fence_async_shared();
+      __syncwarp();
+      if (lane == 0) {
+        const int col = nt * p.width + c + 16 * h;
+        if (p.overwrite)
+          tma_store_3d_plain(map, stage_addr + buf_off, col, row_base, g);
+        else
+          tma_reduce_add_3d(map, stage_addr + buf_off, col, row_base, g);
+        bulk_commit();
+      }
+      ++ochunk;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- the GEMM kernel
 
 // One launch runs up to three independent GEMMs ("phases") back to back over one tile list:
@@ -307,6 +346,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap tb0,
                     const __grid_constant__ CUtensorMap ta1, const __grid_constant__ CUtensorMap tb1,
                     const __grid_constant__ CUtensorMap ta2, const __grid_constant__ CUtensorMap tb2,
+                    const __grid_constant__ CUtensorMap tout1, const __grid_constant__ CUtensorMap tout2,
                     const __grid_constant__ Launch L) {
   extern __shared__ uint8_t smem_raw[];
   const Smem s = gemm::carve(smem_raw);
@@ -459,6 +499,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   } else {
     // -------------------------------------------------------------- epilogue (warps 2..5)
     const int qw = warp & 3;
+    uint32_t ochunk = 0;   // fp32 chunks this warp has staged (alternates its two buffers)
+    uint8_t* stage = s.out_stage + qw * 2 * gemm::kOutChunkBytes;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       int q, g, mt, nt;
       decode(tile, q, g, mt, nt);
@@ -482,6 +524,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       } else if (p.mode == kDx) {
         uint16_t* orow = static_cast<uint16_t*>(p.out) + row_of(p, g, row) * p.out_ld + nt * p.width;
         gemm::store_bf16(tbase, p.width, orow, valid);
+      } else if (p.tma_out) {
+        epi_wgrad_tma(p, q == 1 ? &tout1 : &tout2, tbase, g, mt * BM + qw * 32, nt, stage, ochunk);
       } else {
         epi_wgrad(p, tbase, g, row, valid, nt);
       }
@@ -490,6 +534,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       pipe.acc ^= 1;
       if (pipe.acc == 0) pipe.acc_phase ^= 1u;
     }
+    if (lane == 0 && ochunk > 0) bulk_wait_all();   // the gradient writes are done before exit
     __syncwarp();
   }
   tc_fence_before();
@@ -778,8 +823,9 @@ int pick_width(const int* widths, int n_widths, long long mtiles, int n_total) {
 }
 
 // One launch of up to three GEMM phases (maps a[q], b[q], args[q]); tiles = the sum of their tiles.
+// out: fp32 output maps of phases 1 and 2 (their weight gradients written through TMA), or null.
 cudaError_t run_gemm(const CUtensorMap* a, const CUtensorMap* b, const bwd::GemmArgs* args, int phases,
-                     long long tiles, int kind, cudaStream_t stream) {
+                     long long tiles, int kind, cudaStream_t stream, const CUtensorMap* out = nullptr) {
   if (tiles <= 0) return cudaSuccess;
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
@@ -798,10 +844,12 @@ cudaError_t run_gemm(const CUtensorMap* a, const CUtensorMap* b, const bwd::Gemm
   const CUtensorMap& b1 = b[phases > 1 ? 1 : 0];
   const CUtensorMap& a2 = a[phases > 2 ? 2 : 0];
   const CUtensorMap& b2 = b[phases > 2 ? 2 : 0];
+  const CUtensorMap& o1 = out ? out[1] : a[0];   // unused unless a phase sets tma_out
+  const CUtensorMap& o2 = out ? out[2] : a[0];
   const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
   launch_begin(kind, stream);
   const cudaError_t err = launch_pdl(bwd::bwd_gemm_kernel, dim3(grid), dim3(gemm::kThreads), bwd::kSmemBytes,
-                                     stream, a[0], b[0], a1, b1, a2, b2, L);
+                                     stream, a[0], b[0], a1, b1, a2, b2, o1, o2, L);
   launch_end(kind, stream);
   return err;
 }
@@ -925,7 +973,7 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
   // one launch: dx rows = dab W13, dW2 (+)= dyT hgT^T, dW13 (+)= dabT xT^T (K = the round's rows)
   {
     bwd::GemmArgs g[3] = {base, base, base};
-    CUtensorMap ma[3], mb[3];
+    CUtensorMap ma[3], mb[3], mo[3];
     long long tiles = 0;
     g[0].mode = bwd::kDx;
     g[0].width = pick_width(kWide, 3, mt, d);
@@ -947,6 +995,8 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g[1].overwrite = r == 0;
     g[1].out_group_stride = static_cast<long long>(d) * F;
     g[1].out_ld = F;
+    g[1].tma_out = 1;   // dW2 [E][d][F] fp32 through TMA (store in round 0, reduce-add after)
+    if ((e = gemm::make_map_f32(&mo[1], a.dw_down, F, d, E, 16, 32)) != cudaSuccess) return e;
     if ((e = gemm::make_map(&ma[1], a.dyt, static_cast<uint64_t>(t_ld), d, groups, gemm::BM)) != cudaSuccess) return e;
     if ((e = gemm::make_map(&mb[1], a.hgt, static_cast<uint64_t>(t_ld), F, groups, static_cast<uint32_t>(g[1].width))) !=
         cudaSuccess)
@@ -960,13 +1010,16 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g[2].overwrite = r == 0;
     g[2].out_group_stride = 2ll * F * d;
     g[2].out_ld = d;
+    g[2].tma_out = 1;   // dW13 [E][2F][d] fp32 through TMA
+    if ((e = gemm::make_map_f32(&mo[2], a.dw_gate_up, d, 2ull * F, E, 16, 32)) != cudaSuccess) return e;
     if ((e = gemm::make_map(&ma[2], a.dabt, static_cast<uint64_t>(t_ld), 2ull * F, groups, gemm::BM)) != cudaSuccess)
       return e;
     if ((e = gemm::make_map(&mb[2], a.xt, static_cast<uint64_t>(t_ld), d, groups, static_cast<uint32_t>(g[2].width))) !=
         cudaSuccess)
       return e;
     tiles += mt_w13 * (d / g[2].width);
-    if ((e = run_gemm(ma, mb, g, 3, tiles, kKindBackwardDxWgrad, stream)) != cudaSuccess) return e;
+    mo[0] = ma[0];
+    if ((e = run_gemm(ma, mb, g, 3, tiles, kKindBackwardDxWgrad, stream, mo)) != cudaSuccess) return e;
   }
   // combine dx and gather dgate
   {

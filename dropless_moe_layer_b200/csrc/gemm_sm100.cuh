@@ -764,6 +764,9 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
 // swizzle for the 32-column output boxes of the TMA-store epilogue.
 cudaError_t make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
                      uint64_t groups, uint32_t box_rows, uint32_t box_inner = BK);
+// fp32 [groups][rows][inner], box box_inner x box_rows x 1, 64-byte swizzle (box_inner * 4 == 64).
+cudaError_t make_map_f32(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t groups,
+                         uint32_t box_inner, uint32_t box_rows);
 
 }  // namespace gemm
 }  // namespace moe

@@ -281,6 +281,35 @@ cudaError_t make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_
   return e;
 }
 
+// fp32 output map [groups][rows][inner] with box_inner x box_rows x 1 boxes and the 64-byte
+// swizzle (box_inner * 4 must be 64): the backward's weight-gradient tiles. Cached like the bf16 maps.
+cudaError_t make_map_f32(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t groups,
+                         uint32_t box_inner, uint32_t box_rows) {
+  const MapKey key{base, inner, rows, groups, box_rows, box_inner | 0x80000000u};
+  const uint64_t h = ((reinterpret_cast<uintptr_t>(base) >> 8) * 0x9E3779B97F4A7C15ull) ^
+                     ((inner * 31 + rows) * 131 + groups * 7 + box_rows + box_inner * 5 + 1) * 0xC2B2AE3D27D4EB4Full;
+  MapCacheEntry& slot = g_map_cache[(h >> 40) % kMapCacheSize];
+  std::lock_guard<std::mutex> lock(g_map_mutex);
+  if (slot.used && slot.key == key) {
+    *map = slot.map;
+    return cudaSuccess;
+  }
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {inner, rows, groups};
+  const cuuint64_t strides[2] = {inner * 4, inner * rows * 4};
+  const cuuint32_t box[3] = {box_inner, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult res = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (res != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  slot.used = true;
+  slot.key = key;
+  slot.map = *map;
+  return cudaSuccess;
+}
+
 // B maps for the candidate widths; a candidate that does not divide the N extent (never chosen
 // on the device) repeats the map of the first one that does.
 static cudaError_t make_b_maps(CUtensorMap* mb, const void* base, uint64_t inner, uint64_t rows,

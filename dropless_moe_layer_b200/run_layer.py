@@ -11,6 +11,8 @@ appears a known number of times) or as a quick check that a shape runs on this G
 seed stay), so a kernel can be profiled on a case that holds less device memory.
 --plan-only skips the expert weights and runs only the router and the planner.
 --backward also runs the backward pass (moe_backward) after each forward.
+--per-step runs the rounds through moe_round_dispatch / gate_up / down / combine, each its own
+kernel, so that every step of a large round can be profiled on its own.
 """
 from __future__ import annotations
 
@@ -33,6 +35,9 @@ def main() -> None:
     ap.add_argument("--schedule", default="auto", choices=sorted(moe.SCHEDULES))
     ap.add_argument("--borrow", action="store_true")
     ap.add_argument("--backward", action="store_true", help="also run the backward pass after each forward")
+    ap.add_argument("--per-step", action="store_true",
+                    help="run the rounds through the per-round step calls (stand-alone dispatch, gate/up, "
+                         "down and combine kernels) instead of moe_forward")
     args = ap.parse_args()
     w = wl.BY_NAME[args.workload]
     if args.tokens > 0:
@@ -49,7 +54,13 @@ def main() -> None:
     for _ in range(args.steps):
         layer.plan(logits=inp["logits"], x=inp["x"] if w.router == "gemm" else None,
                    w_router=inp["w_router"], bias=inp["bias"])
-        if not args.plan_only:
+        if not args.plan_only and args.per_step:
+            for r in range(layer.info.R):
+                layer.round_step("dispatch", r, inp["x"])
+                layer.round_step("gate_up", r, inp["w_gate_up"])
+                layer.round_step("down", r, inp["w_down"])
+                layer.round_step("combine", r, y)
+        elif not args.plan_only:
             layer.forward(inp["x"], inp["w_gate_up"], inp["w_down"], y=y)
         if dy is not None:
             layer.backward(inp["x"], inp["w_gate_up"], inp["w_down"], dy)

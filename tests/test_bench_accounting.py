@@ -30,9 +30,13 @@ def test_work_totals_do_not_depend_on_the_split(name):
         if "pipeline" in work:
             flops += work["pipeline"][1][0]
         assert flops == 6 * pairs * w.d * w.F                      # every pair's GEMM work once
-        comb = work["combine"][1] + (bench.combine_bytes(w, p["round"], set(range(r0, p["R"])))
-                                     if r0 < p["R"] else 0)
-        assert comb == bench.combine_bytes(w, p["round"])          # combine bytes split exactly
+        # combine bytes split exactly between stand-alone launches, the steps that ride on a GEMM
+        # launch and the pipelined launch
+        rode_comb, rode_disp = bench.ride_plan(w, p["n"], r0)
+        assert rode_comb <= set(range(r0)) and rode_disp <= set(range(1, p["R"]))
+        comb = work["combine"][1] + bench.combine_bytes(w, p["round"], rode_comb) + (
+            bench.combine_bytes(w, p["round"], set(range(r0, p["R"]))) if r0 < p["R"] else 0)
+        assert comb == bench.combine_bytes(w, p["round"])
         assert ("pipeline" in work) == (r0 < p["R"])
 
 
@@ -71,3 +75,21 @@ def test_backward_flops_split_by_launch_kind():
     w = wl.BY_NAME["4k-zipf1"]
     assert set(bench.BWD_KIND_FLOPS) == set(moe.BACKWARD_GEMM_KINDS)
     assert sum(bench.BWD_KIND_FLOPS.values()) * w.T * w.k * w.d * w.F == bench.backward_flops(w)
+
+
+def test_ride_plan_follows_the_size_rule():
+    """Small copy steps (at most 32 MiB of rows) always ride; a large one rides only when the GEMM
+    it would ride on is long enough to hide it at the copy warps' rate."""
+    w = wl.BY_NAME["32k-zipf1.2-router-gemm"]
+    n = np.zeros((3, w.E), dtype=np.int64)
+    n[0, :] = w.C                       # a full round: 262144 rows
+    n[1, :4] = w.C                      # 8192 rows (117 MB: not small)
+    n[2, 0] = 100                       # a thin round
+    comb, disp = bench.ride_plan(w, n, 3)
+    assert comb == set()                # round 0's combine outlasts round 1's gate/up; round 1's, round 2's
+    assert disp == {1, 2}               # round 1's dispatch hides under round 0's down; round 2's is small
+    n2 = np.zeros((2, w.E), dtype=np.int64)
+    n2[0, :4] = w.C
+    n2[1, :] = w.C
+    comb, disp = bench.ride_plan(w, n2, 2)
+    assert comb == {0} and disp == set()   # the small round's combine hides under the full round's
