@@ -46,11 +46,19 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch of a kernel, from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum per launch; summaries in profiles/), valid only while the kernel's
 # sources, with comments and blank space taken out, hash to the recorded value.
+GEMM_SOURCES = ["sm100.cuh", "gemm_sm100.cuh", "copy_phases.cuh", "kernels.h", "grouped_gemm.cu"]
 TRAFFIC = {
-    ("4k-zipf1", "pipeline"): {
-        "bytes_per_launch": 67.653888e6 + 13.169408e6,
-        "sources": ["sm100.cuh", "gemm_sm100.cuh", "copy_phases.cuh", "kernels.h", "round_pipeline.cu"],
-        "sources_sha1": "5eedc768a5e12125b43c8dc1e1ed41004ae8d580"},
+    # 16 gate/up launches of one step, dram__bytes_read.sum + dram__bytes_write.sum by ncu on the
+    # full workload (one-pass counters), averaged per launch
+    ("32k-zipf1.2-router-gemm", "gate_up"): {
+        "bytes_per_launch": 49.5184e9 / 16,
+        "sources": GEMM_SOURCES,
+        "sources_sha1": "885cff12e941df85df232b4e2ac9867b694c3aed"},
+    # the 3 gate/up launches of one step (profiles/gate_up_pair_gemm_16k-uniform.md's capture)
+    ("16k-uniform", "gate_up"): {
+        "bytes_per_launch": (3.669719e9 + 0.198734e9 + 4.317842e9 + 0.338580e9 + 0.788634e9 + 0.006991e9) / 3,
+        "sources": GEMM_SOURCES,
+        "sources_sha1": "885cff12e941df85df232b4e2ac9867b694c3aed"},
 }
 
 

@@ -67,12 +67,6 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 enum Mode : int { kSwiGLU = 0, kBf16Out = 1, kF32Bias = 2 };
 
-// Order of a phase's tiles within an expert: N tile major (1, the default), so that the weight
-// slice of one N tile is read once for all of the expert's row blocks, or row block major (0).
-#ifndef MOE_TILE_ORDER_N_MAJOR
-#define MOE_TILE_ORDER_N_MAJOR 1
-#endif
-
 struct Smem {
   uint8_t* stage;
   uint8_t* out_stage;       // TMA-store staging of the epilogue warps (1024-byte aligned)
@@ -334,17 +328,8 @@ __device__ __forceinline__ void run_phase(const Smem& s, uint32_t tmem_base, con
     }
     g = lo;
     const int local = tile - ts[g];
-#if MOE_TILE_ORDER_N_MAJOR
-    // (expert, N tile, row block): the CTAs working at once share each weight slice across the
-    // expert's row blocks, and the expert's rows stay in the L2 from one N tile to the next
-    const int mtiles = (group_rows(p, g) + BM - 1) / BM;
-    (void)n_tiles;
-    nt = local / mtiles;
-    mt = local - nt * mtiles;
-#else
     mt = local / n_tiles;
     nt = local - mt * n_tiles;
-#endif
   };
 
   if (warp == 0) {
@@ -596,15 +581,8 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
     }
     g = lo;
     const int local = tile - ts[g];
-#if MOE_TILE_ORDER_N_MAJOR
-    const int mtiles = (group_rows(p, g) + kPairRows - 1) / kPairRows;   // (expert, N tile, row block)
-    (void)n_tiles;
-    nt = local / mtiles;
-    mp = local - nt * mtiles;
-#else
     mp = local / n_tiles;
     nt = local - mp * n_tiles;
-#endif
   };
   // B rows of this CTA's half of a tile
   auto b_row = [&](int nt) {
