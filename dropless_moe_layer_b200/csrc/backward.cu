@@ -96,10 +96,11 @@ __device__ __forceinline__ uint16_t bf16_bits(float v) {
   return *reinterpret_cast<const uint16_t*>(&b);
 }
 
-__device__ __forceinline__ int tiles_of(const GemmArgs& p, int g, int n_tiles) {
+// Tiles of expert g: row blocks of `bm` rows (128, or 256 in the CTA-pair form) x n_tiles.
+__device__ __forceinline__ int tiles_of(const GemmArgs& p, int g, int n_tiles, int bm) {
   const int rows = p.rows[g];
-  if (p.mode == kWgrad) return rows > 0 ? ((p.m_total + BM - 1) / BM) * n_tiles : 0;
-  return ((rows + BM - 1) / BM) * n_tiles;
+  if (p.mode == kWgrad) return rows > 0 ? ((p.m_total + bm - 1) / bm) * n_tiles : 0;
+  return ((rows + bm - 1) / bm) * n_tiles;
 }
 
 __device__ __forceinline__ int k_blocks_of(const GemmArgs& p, int g) {
@@ -129,9 +130,9 @@ __device__ __forceinline__ void warp_prefix(int* out, int groups, Count cnt_of) 
 
 // Warp 0 writes the tile prefix over the experts into ts[0 .. groups] and, for pooled rows, the
 // experts' first columns in the transposed buffers into seg[0 .. groups].
-__device__ __forceinline__ void plan_tiles(int* ts, int* seg, const GemmArgs& p, int n_tiles) {
+__device__ __forceinline__ void plan_tiles(int* ts, int* seg, const GemmArgs& p, int n_tiles, int bm) {
   if ((threadIdx.x >> 5) != 0) return;
-  warp_prefix(ts, p.groups, [&](int g) { return tiles_of(p, g, n_tiles); });
+  warp_prefix(ts, p.groups, [&](int g) { return tiles_of(p, g, n_tiles, bm); });
   if (p.group_row) warp_prefix(seg, p.groups, [&](int g) { return (p.rows[g] + BK - 1) / BK * BK; });
 }
 
@@ -322,17 +323,28 @@ __device__ __forceinline__ void epi_wgrad_tma(const GemmArgs& p, const CUtensorM
 // ---------------------------------------------------------------- the GEMM kernel
 
 // One launch runs up to three independent GEMMs ("phases") back to back over one tile list:
-// phase 0's tiles, then phase 1's, then phase 2's. All phases share one stage geometry (the
-// widest: a 128-row A tile and a 256-row B tile, 48 KB, 4 stages), because the ring's slot
-// barriers assume that a slot always covers the same bytes.
+// phase 0's tiles, then phase 1's, then phase 2's. All phases share one stage geometry, because
+// the ring's slot barriers assume that a slot always covers the same bytes.
+//
+// Two forms, as in the forward's grouped GEMM:
+// - single CTA: 128-row tiles, a 128-row A tile and up to 256 B rows per stage (48 KB, 4
+//   stages), M = 128 MMAs;
+// - CTA pair (cta_group::2, clusters of two): 256-row tiles of 256 columns. CTA c of the pair
+//   loads A rows [128 c, 128 c + 128) of the tile and B rows [128 c, 128 c + 128) of its 256
+//   (recompute: c = 0 the tile's 128 W1 rows, c = 1 the same W3 rows, so that a and b land in
+//   accumulator columns [0, 128) and [128, 256) as in the single-CTA form) into its own shared
+//   memory (32 KB per stage, 6 stages); the leader's one thread issues the M = 256 MMAs for
+//   both, and accumulator rows [128 c, 128 c + 128) land in CTA c's TMEM, where the same
+//   epilogues as in the single-CTA form read them. Half the shared-memory bytes per flop.
+//   Barriers: full[s] and tempty[a] in the leader, empty[s] and tfull[a] in both (the leader's
+//   commits arrive on both). No load is multicast.
 constexpr int kMaxPhases = 3;
 constexpr int kStageBytes = gemm::kABytes + 256 * BK * 2;
 constexpr int kStages = gemm::kRingBytes / kStageBytes;
 static_assert(kStages >= 2 && kStages <= gemm::kMaxStages, "ring stages");
 constexpr int kTileStride = gemm::kMaxGroups + 1;
-// gemm::carve's layout (ring, the forward's output staging, which this kernel leaves unused,
-// barriers, misc words), with room for a tile prefix and a pooled-column prefix per phase after
-// the misc words.
+// gemm::carve's layout (ring, output staging for the weight-gradient TMA writes, barriers, misc
+// words), with room for a tile prefix and a pooled-column prefix per phase after the misc words.
 constexpr int kSmemBytes = 1024 + gemm::kRingBytes + gemm::kOutStagingBytes + gemm::kBarBytes +
                            gemm::kMiscWords * 4 + 2 * kMaxPhases * kTileStride * 4;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -342,19 +354,26 @@ struct Launch {
   int phases;
 };
 
+template <bool kPair>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap tb0,
                     const __grid_constant__ CUtensorMap ta1, const __grid_constant__ CUtensorMap tb1,
                     const __grid_constant__ CUtensorMap ta2, const __grid_constant__ CUtensorMap tb2,
                     const __grid_constant__ CUtensorMap tout1, const __grid_constant__ CUtensorMap tout2,
                     const __grid_constant__ Launch L) {
+  constexpr int kRows = kPair ? gemm::kPairRows : BM;                   // rows of a tile
+  constexpr int kSlot = kPair ? gemm::kPairStageBytes : kStageBytes;    // bytes of a ring slot
+  constexpr int kSlots = kPair ? gemm::kPairStages : kStages;
   extern __shared__ uint8_t smem_raw[];
   const Smem s = gemm::carve(smem_raw);
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&ta0);
     tma_prefetch_desc(&tb0);
   }
-  const uint32_t tmem_base = gemm::setup(s);
+  const uint32_t tmem_base = kPair ? gemm::setup_pair(s) : gemm::setup(s);
+  const uint32_t cta = kPair ? cluster_rank() : 0u;
+  const int unit = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int units = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   int* ts[kMaxPhases];
   int* seg[kMaxPhases];
   for (int q = 0; q < kMaxPhases; ++q) {
@@ -362,7 +381,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     seg[q] = s.tile_start[0] + (kMaxPhases + q) * kTileStride;
   }
   for (int q = 0; q < L.phases; ++q)     // reads only the round's row counts (plan data)
-    plan_tiles(ts[q], seg[q], L.ph[q], L.ph[q].n_total / L.ph[q].width);
+    plan_tiles(ts[q], seg[q], L.ph[q], L.ph[q].n_total / L.ph[q].width, kRows);
   __syncthreads();
   grid_dependency_wait();
   pdl_trigger_early();
@@ -397,45 +416,60 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ------------------------------------------------------------ TMA producer
+      // ------------------------------------------------------------ TMA producer (both CTAs)
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      for (int tile = unit; ok && tile < total; tile += units) {
         int q, g, mt, nt;
         decode(tile, q, g, mt, nt);
         const GemmArgs& p = L.ph[q];
         const CUtensorMap* ma = map_a(q);
         const CUtensorMap* mb = map_b(q);
-        const uint32_t tx = static_cast<uint32_t>(gemm::kABytes + bn_of(p) * BK * 2);
+        // the pair's bytes per stage land on the leader's barrier; the leader counts both halves
+        const uint32_t tx = kPair ? 2u * gemm::kPairStageBytes
+                                  : static_cast<uint32_t>(gemm::kABytes + bn_of(p) * BK * 2);
         const int kbs = k_blocks_of(p, g);
+        const int m0 = mt * kRows + static_cast<int>(cta) * BM;   // this CTA's first A row of the tile
         for (int kb = 0; kb < kbs; ++kb) {
           if (!mbar_wait(smem_addr(&s.empty[pipe.stage]), pipe.phase ^ 1u, s.abort)) {
             ok = false;
             break;
           }
-          const uint32_t sA = smem_addr(s.stage + pipe.stage * kStageBytes);
+          const uint32_t sA = smem_addr(s.stage + pipe.stage * kSlot);
           const uint32_t sB = sA + gemm::kABytes;
-          const uint32_t fb = smem_addr(&s.full[pipe.stage]);
-          mbar_arrive_expect_tx(fb, tx);
+          const uint32_t fb_local = smem_addr(&s.full[pipe.stage]);
+          const uint32_t fb = kPair ? peer_addr(fb_local, 0) : fb_local;
+          if (cta == 0) mbar_arrive_expect_tx(fb_local, tx);
+          auto load = [&](uint32_t dst, const CUtensorMap* m, int c0, int c1, int c2) {
+            if (kPair)
+              tma_load_3d_pair(dst, m, fb, c0, c1, c2);
+            else
+              tma_load_3d(dst, m, fb, c0, c1, c2);
+          };
           if (p.mode == kWgrad) {
             // both operands are transposed buffers, K = the expert's rows: per expert, or from
             // its pooled first column (a multiple of 64, so the coordinate stays 16-byte aligned)
             const int k0 = p.group_row ? seg[q][g] + kb * BK : kb * BK;
             const int grp = p.group_row ? 0 : g;
-            tma_load_3d(sA, ma, fb, k0, mt * BM, grp);
-            tma_load_3d(sB, mb, fb, k0, nt * p.width, grp);
+            load(sA, ma, k0, m0, grp);
+            load(sB, mb, k0, kPair ? nt * p.width + static_cast<int>(cta) * gemm::kPairBHalf : nt * p.width, grp);
           } else {
-            const int a_row = p.group_row ? static_cast<int>(row_of(p, g, mt * BM)) : mt * BM;
-            tma_load_3d(sA, ma, fb, kb * BK, a_row, p.group_row ? 0 : g);
-            if (p.mode == kRecompute) {
-              tma_load_3d(sB, mb, fb, kb * BK, nt * p.width, g);
-              tma_load_3d(sB + p.width * BK * 2, mb, fb, kb * BK, p.F + nt * p.width, g);
+            const int a_row = p.group_row ? static_cast<int>(row_of(p, g, m0)) : m0;
+            load(sA, ma, kb * BK, a_row, p.group_row ? 0 : g);
+            if (kPair) {
+              // recompute: CTA 0 the tile's W1 rows, CTA 1 the same W3 rows; else 128 of the 256
+              const int b_row = p.mode == kRecompute ? static_cast<int>(cta) * p.F + nt * p.width
+                                                     : nt * p.width + static_cast<int>(cta) * gemm::kPairBHalf;
+              load(sB, mb, kb * BK, b_row, g);
+            } else if (p.mode == kRecompute) {
+              load(sB, mb, kb * BK, nt * p.width, g);
+              load(sB + p.width * BK * 2, mb, kb * BK, p.F + nt * p.width, g);
             } else {
-              tma_load_3d(sB, mb, fb, kb * BK, nt * p.width, g);
+              load(sB, mb, kb * BK, nt * p.width, g);
             }
           }
           pipe.issued |= 1u << pipe.stage;
           pipe.issued_parity = (pipe.issued_parity & ~(1u << pipe.stage)) | (pipe.phase << pipe.stage);
-          if (++pipe.stage == kStages) {
+          if (++pipe.stage == kSlots) {
             pipe.stage = 0;
             pipe.phase ^= 1u;
           }
@@ -444,20 +478,28 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       if (!ok) {
         atomicOr(status, kStatusTimeoutProducer);
         *s.abort = 1;
-        for (int i = 0; i < kStages; ++i)   // let issued loads land before the CTA exits
-          if ((pipe.issued >> i) & 1u) mbar_wait(smem_addr(&s.full[i]), (pipe.issued_parity >> i) & 1u, nullptr);
+        if (kPair) {
+          // loads already issued complete on the leader's barriers, which the peer cannot wait
+          // on: give them time to land before the pair's shared memory is released
+          const uint64_t t0 = global_timer_ns();
+          while (global_timer_ns() - t0 < 200000ull) {
+          }
+        } else {
+          for (int i = 0; i < kSlots; ++i)   // let issued loads land before the CTA exits
+            if ((pipe.issued >> i) & 1u) mbar_wait(smem_addr(&s.full[i]), (pipe.issued_parity >> i) & 1u, nullptr);
+        }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && cta == 0) {
+      // ------------------------------------------------------------ MMA issuer (the leader)
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      for (int tile = unit; ok && tile < total; tile += units) {
         int q, g, mt, nt;
         decode(tile, q, g, mt, nt);
         const GemmArgs& p = L.ph[q];
-        const uint32_t idesc = idesc_bf16_f32(BM, bn_of(p));
+        const uint32_t idesc = idesc_bf16_f32(kRows, bn_of(p));
         const int kbs = k_blocks_of(p, g);
         if (!mbar_wait(smem_addr(&s.tempty[pipe.acc]), pipe.acc_phase ^ 1u, s.abort)) {
           ok = false;
@@ -471,27 +513,40 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sA = smem_addr(s.stage + pipe.stage * kStageBytes);
+          const uint32_t sA = smem_addr(s.stage + pipe.stage * kSlot);
           const uint64_t adesc = smem_desc_sw128(sA);
           const uint64_t bdesc = smem_desc_sw128(sA + gemm::kABytes);
 #pragma unroll
-          for (int kk = 0; kk < BK / gemm::UMMA_K; ++kk)
-            mma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
-          mma_commit(smem_addr(&s.empty[pipe.stage]));
-          if (++pipe.stage == kStages) {
+          for (int kk = 0; kk < BK / gemm::UMMA_K; ++kk) {
+            if (kPair)
+              mma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+            else
+              mma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          if (kPair)
+            mma_commit_pair(smem_addr(&s.empty[pipe.stage]), 3);
+          else
+            mma_commit(smem_addr(&s.empty[pipe.stage]));
+          if (++pipe.stage == kSlots) {
             pipe.stage = 0;
             pipe.phase ^= 1u;
           }
         }
         if (!ok) break;
-        mma_commit(smem_addr(&s.tfull[pipe.acc]));
+        if (kPair)
+          mma_commit_pair(smem_addr(&s.tfull[pipe.acc]), 3);
+        else
+          mma_commit(smem_addr(&s.tfull[pipe.acc]));
         pipe.acc ^= 1;
         if (pipe.acc == 0) pipe.acc_phase ^= 1u;
       }
       if (!ok) {
         atomicOr(status, kStatusTimeoutMma);
         *s.abort = 1;
-        mma_commit(smem_addr(s.drain));   // wait for every MMA already issued
+        if (kPair)
+          mma_commit_pair(smem_addr(s.drain), 1);   // wait for every MMA already issued
+        else
+          mma_commit(smem_addr(s.drain));
         mbar_wait(smem_addr(s.drain), 0, nullptr);
       }
     }
@@ -501,7 +556,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     const int qw = warp & 3;
     uint32_t ochunk = 0;   // fp32 chunks this warp has staged (alternates its two buffers)
     uint8_t* stage = s.out_stage + qw * 2 * gemm::kOutChunkBytes;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    for (int tile = unit; tile < total; tile += units) {
       int q, g, mt, nt;
       decode(tile, q, g, mt, nt);
       const GemmArgs& p = L.ph[q];
@@ -513,7 +568,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int row = mt * BM + qw * 32 + lane;
+      const int row0 = mt * kRows + static_cast<int>(cta) * BM + qw * 32;   // this warp's first row
+      const int row = row0 + lane;
       const bool valid = row < (p.mode == kWgrad ? p.m_total : p.rows[g]);
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) +
                              static_cast<uint32_t>(pipe.acc * gemm::kAccCols);
@@ -525,12 +581,17 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         uint16_t* orow = static_cast<uint16_t*>(p.out) + row_of(p, g, row) * p.out_ld + nt * p.width;
         gemm::store_bf16(tbase, p.width, orow, valid);
       } else if (p.tma_out) {
-        epi_wgrad_tma(p, q == 1 ? &tout1 : &tout2, tbase, g, mt * BM + qw * 32, nt, stage, ochunk);
+        epi_wgrad_tma(p, q == 1 ? &tout1 : &tout2, tbase, g, row0, nt, stage, ochunk);
       } else {
         epi_wgrad(p, tbase, g, row, valid, nt);
       }
       tc_fence_before();
-      mbar_arrive(smem_addr(&s.tempty[pipe.acc]));
+      if (kPair) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(peer_addr(smem_addr(&s.tempty[pipe.acc]), 0));
+      } else {
+        mbar_arrive(smem_addr(&s.tempty[pipe.acc]));
+      }
       pipe.acc ^= 1;
       if (pipe.acc == 0) pipe.acc_phase ^= 1u;
     }
@@ -540,7 +601,10 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   pdl_trigger_late();
-  gemm::release_tmem(tmem_base);
+  if (kPair)
+    gemm::release_tmem_pair(tmem_base);
+  else
+    gemm::release_tmem(tmem_base);
 }
 
 // ---------------------------------------------------------------- copy and small kernels
@@ -594,15 +658,16 @@ __global__ void __launch_bounds__(256) transpose_kernel(const TransposeArgs a) {
 }
 
 // Dispatch and transpose of round r in one pass. A block takes 64 rows of one expert's rows in
-// the round and 64 columns (c0 ..): the rows' tokens come from the round-major row list
-// (row_off[r][e] + s), their x and dy slices are copied row-major into xbuf and dybuf (dy as
+// the round and 64 columns (c0 = 64 * blockIdx.y): the rows' tokens come from the round-major row
+// list (row_off[r][e] + s), their x and dy slices are copied row-major into xbuf and dybuf (dy as
 // bf16) and, through a shared-memory tile, transposed into xT and dyT; rows from n[r][e] up to
 // the next multiple of 64 are zeros in the transposed copies only. The blocks of the first
 // column slice also write each row's gate.
-// Per-expert rows (no borrowing): block (x, y, e) takes expert e's rows 64y.., at e * C + s in the
-// row-major buffers and at [e][c][s] (t_ld per row) in the transposed ones. Pooled rows
-// (borrowing): block (x, y) takes pooled transposed columns 64y.., which lie in the segment of
-// one expert (segments are the experts' rows rounded up to 64, in expert order) or past the last.
+// The grid's x covers only the round's rows: block b is the b-th 64-row block in expert order
+// (expert e holds ceil(n[r][e] / 64) of them), so a round with few rows launches few blocks.
+// Per-expert rows (no borrowing): expert e's rows s at e * C + s in the row-major buffers and at
+// [e][c][s] (t_ld per row) in the transposed ones. Pooled rows (borrowing): the transposed
+// column of block b is 64 b (segments are the experts' rows rounded up to 64, in expert order).
 struct GatherArgs {
   const uint16_t* x;
   const float* dy;
@@ -624,44 +689,50 @@ __global__ void __launch_bounds__(256) bwd_gather_kernel(const __grid_constant__
   __shared__ uint16_t tx_tile[64][66];
   __shared__ uint16_t ty_tile[64][66];
   __shared__ int tok[64];
-  __shared__ int blk[3];      // expert, its first row of this block, its rows (pooled mode)
+  __shared__ int blk[3];      // expert, its first row in this block, its rows in the round
   grid_dependency_wait();
-  const int c0 = blockIdx.x * 64;
+  const int c0 = blockIdx.y * 64;
   const int32_t* nr = a.n + static_cast<size_t>(a.r) * a.E;
-  int e, s0, ne;
-  if (!a.pooled) {
-    e = blockIdx.z;
-    s0 = blockIdx.y * 64;
-    ne = nr[e];
-  } else {
-    if (threadIdx.x == 0) {
-      const int col = blockIdx.y * 64;
-      int acc = 0, found = -1, first = 0, rows = 0;
-      for (int x = 0; x < a.E; ++x) {
-        const int len = (nr[x] + 63) / 64 * 64;
-        if (col < acc + len) {
-          found = x;
-          first = col - acc;
-          rows = nr[x];
-          break;
-        }
-        acc += len;
+  if (threadIdx.x < 32) {
+    // warp 0: the expert whose 64-row blocks hold block b (a running prefix over the experts)
+    const int lane = threadIdx.x;
+    const int b = static_cast<int>(blockIdx.x);
+    int acc = 0, found = -1, first = 0, rows = 0;
+    for (int x0 = 0; x0 < a.E; x0 += 32) {
+      const int x = x0 + lane;
+      const int nx = x < a.E ? nr[x] : 0;
+      const int cnt = (nx + 63) / 64;
+      int incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
       }
+      const int excl = acc + incl - cnt;
+      const unsigned hit = __ballot_sync(0xffffffffu, cnt > 0 && b >= excl && b < excl + cnt);
+      if (hit != 0u) {
+        const int src = __ffs(hit) - 1;
+        found = x0 + src;
+        first = (b - __shfl_sync(0xffffffffu, excl, src)) * 64;
+        rows = __shfl_sync(0xffffffffu, nx, src);
+        break;
+      }
+      acc += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
       blk[0] = found;
       blk[1] = first;
       blk[2] = rows;
     }
-    __syncthreads();
-    e = blk[0];
-    s0 = blk[1];
-    ne = blk[2];
   }
+  __syncthreads();
+  const int e = blk[0], s0 = blk[1], ne = blk[2];
   const int fill = (ne + 63) / 64 * 64;
   if (e >= 0 && s0 < fill) {
     const int base = a.row_off[static_cast<size_t>(a.r) * a.E + e];
     const long long dst0 = a.pooled ? static_cast<long long>(base - a.row_start[a.r])
                                     : static_cast<long long>(e) * a.C;   // row-major row of s = 0
-    const long long tcol0 = a.pooled ? static_cast<long long>(blockIdx.y) * 64
+    const long long tcol0 = a.pooled ? static_cast<long long>(blockIdx.x) * 64
                                      : static_cast<long long>(e) * a.d * a.t_ld + s0;   // + c * t_ld
     if (threadIdx.x < 64) {
       const int sr = s0 + threadIdx.x;
@@ -822,21 +893,89 @@ int pick_width(const int* widths, int n_widths, long long mtiles, int n_total) {
   return last;
 }
 
-// One launch of up to three GEMM phases (maps a[q], b[q], args[q]); tiles = the sum of their tiles.
-// out: fp32 output maps of phases 1 and 2 (their weight gradients written through TMA), or null.
-cudaError_t run_gemm(const CUtensorMap* a, const CUtensorMap* b, const bwd::GemmArgs* args, int phases,
-                     long long tiles, int kind, cudaStream_t stream, const CUtensorMap* out = nullptr) {
-  if (tiles <= 0) return cudaSuccess;
+#ifndef MOE_BWD_PAIR
+#define MOE_BWD_PAIR 1   // 0: the backward GEMMs never use the CTA-pair form
+#endif
+
+// Sets the kernels' shared-memory size once per device; false on failure.
+bool configure_kernels() {
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
   cudaGetDevice(&dev);
   const uint64_t bit = 1ull << (dev & 63);
-  if (!(configured.load() & bit)) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(bwd::bwd_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured.fetch_or(bit);
+  if (configured.load() & bit) return true;
+  if (cudaFuncSetAttribute(bwd::bwd_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           bwd::kSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(bwd::bwd_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           bwd::kSmemBytes) != cudaSuccess)
+    return false;
+  configured.fetch_or(bit);
+  return true;
+}
+
+// Clusters of two of the pair form that fit on the device at once (one CTA per SM), per device
+// ordinal; -1 when the pair form cannot run.
+int pair_clusters() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  dev &= 63;
+  int v = cached[dev].load();
+  if (v != 0) return v;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (num_sms() / 2));
+  cfg.blockDim = dim3(gemm::kThreads);
+  cfg.dynamicSmemBytes = bwd::kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (!configure_kernels() || cudaOccupancyMaxActiveClusters(&n, bwd::bwd_gemm_kernel<true>, &cfg) != cudaSuccess ||
+      n <= 0) {
+    cudaGetLastError();
+    n = -1;
   }
+  cached[dev].store(n);
+  return n;
+}
+
+// Row blocks of the round: 256-row blocks (pair form) and the rows that 256- and 128-row tiles
+// cover.
+struct RowBlocks {
+  long long blocks256 = 0, rows256 = 0, rows128 = 0;
+};
+
+RowBlocks row_blocks(const int32_t* n_host, int E) {
+  RowBlocks b;
+  for (int g = 0; g < E; ++g) {
+    const long long p = (n_host[g] + gemm::kPairRows - 1) / gemm::kPairRows;
+    b.blocks256 += p;
+    b.rows256 += p * gemm::kPairRows;
+    b.rows128 += static_cast<long long>((n_host[g] + gemm::BM - 1) / gemm::BM) * gemm::BM;
+  }
+  return b;
+}
+
+// Whether a launch whose tiles are the round's 256-row blocks x n_tiles runs in the pair form:
+// enough tiles for every cluster, and at most 15% more rows than 128-row tiles would cover.
+bool use_pair(const RowBlocks& b, long long n_tiles) {
+  if (!MOE_BWD_PAIR || n_tiles <= 0) return false;
+  const int clusters = pair_clusters();
+  return clusters > 0 && b.blocks256 * n_tiles >= clusters && b.rows256 * 100 <= b.rows128 * 115;
+}
+
+// One launch of up to three GEMM phases (maps a[q], b[q], args[q]); tiles = the sum of their tiles
+// (single-CTA form; the pair form runs one cluster per pair of SMs and counts tiles on the device).
+// out: fp32 output maps of phases 1 and 2 (their weight gradients written through TMA), or null.
+cudaError_t run_gemm(const CUtensorMap* a, const CUtensorMap* b, const bwd::GemmArgs* args, int phases,
+                     long long tiles, int kind, cudaStream_t stream, const CUtensorMap* out = nullptr,
+                     bool pair = false) {
+  if (tiles <= 0) return cudaSuccess;
+  if (!configure_kernels()) return cudaGetLastError();
   bwd::Launch L{};
   L.phases = phases;
   for (int q = 0; q < phases; ++q) L.ph[q] = args[q];
@@ -846,10 +985,29 @@ cudaError_t run_gemm(const CUtensorMap* a, const CUtensorMap* b, const bwd::Gemm
   const CUtensorMap& b2 = b[phases > 2 ? 2 : 0];
   const CUtensorMap& o1 = out ? out[1] : a[0];   // unused unless a phase sets tma_out
   const CUtensorMap& o2 = out ? out[2] : a[0];
-  const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
   launch_begin(kind, stream);
-  const cudaError_t err = launch_pdl(bwd::bwd_gemm_kernel, dim3(grid), dim3(gemm::kThreads), bwd::kSmemBytes,
-                                     stream, a[0], b[0], a1, b1, a2, b2, o1, o2, L);
+  cudaError_t err;
+  if (pair) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pair_clusters());
+    cfg.blockDim = dim3(gemm::kThreads);
+    cfg.dynamicSmemBytes = bwd::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = MOE_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    err = cudaLaunchKernelEx(&cfg, bwd::bwd_gemm_kernel<true>, a[0], b[0], a1, b1, a2, b2, o1, o2, L);
+  } else {
+    const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
+    err = launch_pdl(bwd::bwd_gemm_kernel<false>, dim3(grid), dim3(gemm::kThreads), bwd::kSmemBytes, stream, a[0],
+                     b[0], a1, b1, a2, b2, o1, o2, L);
+  }
   launch_end(kind, stream);
   return err;
 }
@@ -909,11 +1067,14 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
   {
     const bwd::GatherArgs ga{a.x, a.dy, a.idx, a.gate, a.n, a.row_off, a.row_start, a.row_token, a.xbuf, a.dybuf,
                              a.row_gate, a.xt, a.dyt, r, E, C, d, a.k, static_cast<int>(t_ld), pooled ? 1 : 0};
-    launch_begin(kKindBackwardCopy, stream);
-    e = launch_pdl(bwd::bwd_gather_kernel, dim3(d / 64, static_cast<unsigned>(t_ld / 64), pooled ? 1 : E), dim3(256),
-                   0, stream, ga);
-    launch_end(kKindBackwardCopy, stream);
-    if (e != cudaSuccess) return e;
+    long long blocks = 0;   // the round's 64-row blocks, expert by expert
+    for (int x = 0; x < E; ++x) blocks += (n_host[x] + 63) / 64;
+    if (blocks > 0) {
+      launch_begin(kKindBackwardCopy, stream);
+      e = launch_pdl(bwd::bwd_gather_kernel, dim3(static_cast<unsigned>(blocks), d / 64), dim3(256), 0, stream, ga);
+      launch_end(kKindBackwardCopy, stream);
+      if (e != cudaSuccess) return e;
+    }
   }
 
   long long mt = 0;
@@ -922,6 +1083,7 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     mt += (n_host[g] + gemm::BM - 1) / gemm::BM;
     active += n_host[g] > 0 ? 1 : 0;
   }
+  const RowBlocks rb = row_blocks(n_host, E);
   bwd::GemmArgs base{};
   base.rows = n_dev;
   base.groups = E;
@@ -932,13 +1094,16 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
   base.group_row_base = pooled ? a.row_start + r : nullptr;
   base.status = a.status;
   static const int kWide[3] = {256, 128, 64};
+  // pair form: 256-row tiles, 128 B rows per CTA (recompute: 128 W1 rows and the same W3 rows)
+  const uint32_t pair_box = gemm::kPairBHalf;
 
   // recompute: [a | b] = xbuf W13^T
   {
     static const int kW[3] = {128, 64, 32};
+    const bool pair = F % 128 == 0 && use_pair(rb, F / 128);
     bwd::GemmArgs g = base;
     g.mode = bwd::kRecompute;
-    g.width = pick_width(kW, 3, mt, F);
+    g.width = pair ? 128 : pick_width(kW, 3, mt, F);
     g.n_total = F;
     g.num_k_blocks = d / gemm::BK;
     g.out = a.ab;
@@ -946,16 +1111,20 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g.row_gate = a.row_gate;
     CUtensorMap ma, mb;
     if ((e = gemm::make_map(&ma, a.xbuf, d, a_rows, groups, gemm::BM)) != cudaSuccess) return e;
-    if ((e = gemm::make_map(&mb, a.w_gate_up, d, 2ull * F, E, static_cast<uint32_t>(g.width))) != cudaSuccess) return e;
-    if ((e = run_gemm(&ma, &mb, &g, 1, mt * (F / g.width), kKindBackwardRecompute, stream)) != cudaSuccess)
+    if ((e = gemm::make_map(&mb, a.w_gate_up, d, 2ull * F, E, pair ? pair_box : static_cast<uint32_t>(g.width))) !=
+        cudaSuccess)
+      return e;
+    if ((e = run_gemm(&ma, &mb, &g, 1, mt * (F / g.width), kKindBackwardRecompute, stream, nullptr, pair)) !=
+        cudaSuccess)
       return e;
   }
   // dh = W2^T dy with the SwiGLU backward in its epilogue
   int parts = 0;
   {
+    const bool pair = F % 256 == 0 && use_pair(rb, F / 256);
     bwd::GemmArgs g = base;
     g.mode = bwd::kDh;
-    g.width = pick_width(kWide, 3, mt, F);
+    g.width = pair ? 256 : pick_width(kWide, 3, mt, F);
     parts = F / g.width;
     g.n_total = F;
     g.num_k_blocks = d / gemm::BK;
@@ -967,22 +1136,27 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g.dgate_ld = F / 64;
     CUtensorMap ma, mb;
     if ((e = gemm::make_map(&ma, a.dybuf, d, a_rows, groups, gemm::BM)) != cudaSuccess) return e;
-    if ((e = gemm::make_map(&mb, a.w2t, d, F, E, static_cast<uint32_t>(g.width))) != cudaSuccess) return e;
-    if ((e = run_gemm(&ma, &mb, &g, 1, mt * parts, kKindBackwardDh, stream)) != cudaSuccess) return e;
+    if ((e = gemm::make_map(&mb, a.w2t, d, F, E, pair ? pair_box : static_cast<uint32_t>(g.width))) != cudaSuccess)
+      return e;
+    if ((e = run_gemm(&ma, &mb, &g, 1, mt * parts, kKindBackwardDh, stream, nullptr, pair)) != cudaSuccess) return e;
   }
   // one launch: dx rows = dab W13, dW2 (+)= dyT hgT^T, dW13 (+)= dabT xT^T (K = the round's rows)
   {
+    // the weight gradients' tiles cover d x F and 2F x d per active expert whatever the round's
+    // rows; the dx phase decides, as in the other launches
+    const bool pair = d % 256 == 0 && F % 256 == 0 && use_pair(rb, d / 256);
     bwd::GemmArgs g[3] = {base, base, base};
     CUtensorMap ma[3], mb[3], mo[3];
     long long tiles = 0;
     g[0].mode = bwd::kDx;
-    g[0].width = pick_width(kWide, 3, mt, d);
+    g[0].width = pair ? 256 : pick_width(kWide, 3, mt, d);
     g[0].n_total = d;
     g[0].num_k_blocks = 2 * F / gemm::BK;
     g[0].out = a.dxbuf;
     g[0].out_ld = d;
     if ((e = gemm::make_map(&ma[0], a.dab, 2ull * F, a_rows, groups, gemm::BM)) != cudaSuccess) return e;
-    if ((e = gemm::make_map(&mb[0], a.w13t, 2ull * F, d, E, static_cast<uint32_t>(g[0].width))) != cudaSuccess)
+    if ((e = gemm::make_map(&mb[0], a.w13t, 2ull * F, d, E, pair ? pair_box : static_cast<uint32_t>(g[0].width))) !=
+        cudaSuccess)
       return e;
     tiles += mt * (d / g[0].width);
     const long long mt_w2 = static_cast<long long>(active) * ((d + gemm::BM - 1) / gemm::BM);
@@ -990,7 +1164,7 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g[1].mode = bwd::kWgrad;
     g[1].m_total = d;
     g[1].n_total = F;
-    g[1].width = pick_width(kWide, 3, mt_w2, F);
+    g[1].width = pair ? 256 : pick_width(kWide, 3, mt_w2, F);
     g[1].out = a.dw_down;
     g[1].overwrite = r == 0;
     g[1].out_group_stride = static_cast<long long>(d) * F;
@@ -998,14 +1172,14 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g[1].tma_out = 1;   // dW2 [E][d][F] fp32 through TMA (store in round 0, reduce-add after)
     if ((e = gemm::make_map_f32(&mo[1], a.dw_down, F, d, E, 16, 32)) != cudaSuccess) return e;
     if ((e = gemm::make_map(&ma[1], a.dyt, static_cast<uint64_t>(t_ld), d, groups, gemm::BM)) != cudaSuccess) return e;
-    if ((e = gemm::make_map(&mb[1], a.hgt, static_cast<uint64_t>(t_ld), F, groups, static_cast<uint32_t>(g[1].width))) !=
-        cudaSuccess)
+    if ((e = gemm::make_map(&mb[1], a.hgt, static_cast<uint64_t>(t_ld), F, groups,
+                            pair ? pair_box : static_cast<uint32_t>(g[1].width))) != cudaSuccess)
       return e;
     tiles += mt_w2 * (F / g[1].width);
     g[2].mode = bwd::kWgrad;
     g[2].m_total = 2 * F;
     g[2].n_total = d;
-    g[2].width = pick_width(kWide, 3, mt_w13, d);
+    g[2].width = pair ? 256 : pick_width(kWide, 3, mt_w13, d);
     g[2].out = a.dw_gate_up;
     g[2].overwrite = r == 0;
     g[2].out_group_stride = 2ll * F * d;
@@ -1014,12 +1188,12 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     if ((e = gemm::make_map_f32(&mo[2], a.dw_gate_up, d, 2ull * F, E, 16, 32)) != cudaSuccess) return e;
     if ((e = gemm::make_map(&ma[2], a.dabt, static_cast<uint64_t>(t_ld), 2ull * F, groups, gemm::BM)) != cudaSuccess)
       return e;
-    if ((e = gemm::make_map(&mb[2], a.xt, static_cast<uint64_t>(t_ld), d, groups, static_cast<uint32_t>(g[2].width))) !=
-        cudaSuccess)
+    if ((e = gemm::make_map(&mb[2], a.xt, static_cast<uint64_t>(t_ld), d, groups,
+                            pair ? pair_box : static_cast<uint32_t>(g[2].width))) != cudaSuccess)
       return e;
     tiles += mt_w13 * (d / g[2].width);
     mo[0] = ma[0];
-    if ((e = run_gemm(ma, mb, g, 3, tiles, kKindBackwardDxWgrad, stream, mo)) != cudaSuccess) return e;
+    if ((e = run_gemm(ma, mb, g, 3, tiles, kKindBackwardDxWgrad, stream, mo, pair)) != cudaSuccess) return e;
   }
   // combine dx and gather dgate
   {

@@ -8,5 +8,5 @@ from .moe_oracle import (bf16_to_f64, router_logits, select_topk, gates, plan, p
                          round_rows, silu, expert_hidden, expert_ffn, forward,
                          forward_rounds, layer)
 from .moe_backward import (silu_grad, expert_backward, gates_backward, router_backward,  # noqa: F401
-                           backward, backward_rounds)
+                           backward, backward_sampled, backward_rounds)
 from .moe_ep import owner, ep_plan, ep_forward  # noqa: F401

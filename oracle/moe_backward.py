@@ -32,7 +32,10 @@ The gate function is the forward oracle's reading (softmax over all E, then top-
 pages never name: "parity unpinned" for that choice, as in the forward; the gradients of the
 chosen function are pinned (finite differences, autograd, exact identities).
 
-`backward` is that definition, pair by pair, with no schedule; `backward_rounds` is the
+`backward` is that definition, pair by pair, with no schedule; `backward_sampled` is the same
+definition evaluated only for some tokens and some experts (every gradient entry depends on a
+token's own pairs or on one expert's pairs alone), for sizes where the whole is too slow;
+`backward_rounds` is the
 literal round-by-round form with recompute: each round re-dispatches its rows of x and of
 gate * dy into fixed buffers of E*C rows, recomputes a, b and h for them, and adds the
 round's weight gradients into per-expert accumulators, so nothing it keeps grows with the
@@ -138,6 +141,47 @@ def backward(x_bits, w_gate_up_bits, w_down_bits, z, idx, dy, renorm: bool = Fal
         dx = dx + dx_terms[:, j, :]
     return dict(dx=dx, dw_gate_up=dw_gate_up, dw_down=dw_down, dgate=dgate,
                 dz=gates_backward(z, idx, dgate, renorm))
+
+
+def backward_sampled(x_bits, w_gate_up_bits, w_down_bits, z, idx, dy, tokens, experts,
+                     renorm: bool = False, gate=None) -> dict:
+    """Entries of `backward` at sizes where computing all of them is too slow.
+
+    dx, dgate and dz of token t depend only on token t's own k pairs (its row through each of
+    its experts), and expert e's weight gradients only on the pairs routed to e. So this takes
+    the same definition over those pairs alone: for each sampled token, its k pairs; for each
+    sampled expert, all of its pairs in one `expert_backward`. Returns dx [len(tokens), d],
+    dgate and dz of those tokens, dw_gate_up [len(experts), 2F, d], dw_down [len(experts), d, F].
+    `gate` (full [T, k]) as in `backward`."""
+    idx = np.asarray(idx)
+    z = np.asarray(z)
+    tokens = np.asarray(tokens, dtype=np.int64)
+    T, k = idx.shape
+    d = w_down_bits.shape[1]
+    g = gates(z, idx, renorm) if gate is None else np.asarray(gate, dtype=np.float64)
+    dyd = np.asarray(dy, dtype=np.float64)
+    dx = np.zeros((tokens.size, d), dtype=np.float64)
+    dgate = np.zeros((tokens.size, k), dtype=np.float64)
+    for i, t in enumerate(tokens):
+        xt = bf16_to_f64(x_bits[t:t + 1])
+        for j in range(k):
+            e = int(idx[t, j])
+            gr = expert_backward(xt, bf16_to_f64(w_gate_up_bits[e]), bf16_to_f64(w_down_bits[e]),
+                                 g[t, j] * dyd[t:t + 1])
+            dx[i] += gr["dx"][0]
+            dgate[i, j] = float(np.dot(dyd[t], gr["out"][0]))
+    dz = gates_backward(z[tokens], idx[tokens], dgate, renorm)
+    dw_gate_up = np.zeros((len(experts),) + tuple(w_gate_up_bits.shape[1:]), dtype=np.float64)
+    dw_down = np.zeros((len(experts),) + tuple(w_down_bits.shape[1:]), dtype=np.float64)
+    for i, e in enumerate(experts):
+        tt, jj = np.nonzero(idx == e)
+        if tt.size == 0:
+            continue
+        gr = expert_backward(bf16_to_f64(x_bits[tt]), bf16_to_f64(w_gate_up_bits[e]),
+                             bf16_to_f64(w_down_bits[e]), g[tt, jj][:, None] * dyd[tt])
+        dw_gate_up[i] = gr["dw_gate_up"]
+        dw_down[i] = gr["dw_down"]
+    return dict(dx=dx, dgate=dgate, dz=dz, dw_gate_up=dw_gate_up, dw_down=dw_down)
 
 
 def backward_rounds(x_bits, w_gate_up_bits, w_down_bits, z, idx, dy, C: int,

@@ -137,3 +137,46 @@ def test_backward_borrow_edge_shapes(cfg):
     dy = wl.generate_dy(w, "cuda")
     layer, g = run_backward(w, inp, dy, borrow=True)
     check(w, inp, dy, g)
+
+
+# Round 0 of this shape holds 16 experts x ~512 rows: 32 row blocks of 256 times 4 to 8 column
+# tiles, enough for every SM pair, so its GEMMs run in the CTA-pair form (256-row tiles, ragged
+# where an expert has fewer than 512 rows); the short later rounds run in the single-CTA form.
+PAIR_SHAPE = dict(T=4096, d=1024, E=16, k=2, F=1024, C=512)
+
+
+@pytest.mark.parametrize("borrow", [False, True], ids=["per-expert", "borrow"])
+def test_backward_pair_form_full_parity(borrow):
+    w = wl.custom(name="pair", bias="none", seed=11, **PAIR_SHAPE)
+    inp = wl.generate(w, "cuda")
+    dy = wl.generate_dy(w, "cuda")
+    layer, g = run_backward(w, inp, dy, borrow=borrow)
+    check(w, inp, dy, g)
+    g2 = layer.backward(inp["x"], inp["w_gate_up"], inp["w_down"], dy)
+    torch.cuda.synchronize()
+    for n in NAMES:
+        assert torch.equal(g[n], g2[n]), n
+
+
+def test_backward_16k_uniform_sampled_parity():
+    """The benchmark's backward workload at full size, in the launch configuration it times:
+    dx, dgate and dz of sampled tokens and the weight gradients of the experts with the most and
+    the fewest pairs against the oracle's entries (each token's and each expert's pairs alone)."""
+    w = wl.BY_NAME["16k-uniform"]
+    inp = wl.generate(w, "cuda")
+    dy = wl.generate_dy(w, "cuda")
+    layer, g = run_backward(w, inp, dy)
+    assert layer.info.R >= 2
+    z = inp["logits"].cpu().numpy()
+    idx = oracle.select_topk(z, w.k)
+    load = np.bincount(idx.ravel(), minlength=w.E)
+    experts = [int(np.argmax(load)), int(np.argmin(load))]
+    rng = np.random.default_rng(0)
+    tokens = np.concatenate([[0, w.T - 1], rng.choice(w.T, 14, replace=False)])
+    ref = oracle.backward_sampled(wl.bf16_bits(inp["x"]), wl.bf16_bits(inp["w_gate_up"]),
+                                  wl.bf16_bits(inp["w_down"]), z, idx, dy.cpu().numpy().astype(np.float64),
+                                  tokens, experts)
+    got = {"dx": g["dx"][tokens], "dz": g["dz"][tokens],
+           "dw_gate_up": g["dw_gate_up"][experts], "dw_down": g["dw_down"][experts]}
+    errs = {n: rel_err(got[n].cpu().numpy().astype(np.float64), ref[n]) for n in got}
+    assert all(e <= G_TOL for e in errs.values()), errs

@@ -204,3 +204,28 @@ def test_rounds_with_recompute_equal_the_definition(C, borrow):
     for name in ("dx", "dw_gate_up", "dw_down", "dgate", "dz"):
         scale = 1 + np.abs(ref[name]).max()
         assert np.abs(got[name] - ref[name]).max() <= 1e-12 * scale, name
+
+
+@pytest.mark.parametrize("renorm", [False, True])
+def test_sampled_entries_equal_the_definition(renorm):
+    """The sampled evaluation takes each token's and each expert's pairs alone; the entries it
+    returns must be the full backward's, for any choice of tokens (repeats, unsorted) and of
+    experts (one with no pairs included)."""
+    rng = np.random.default_rng(9)
+    T, d, E, k, F = 30, 8, 5, 2, 6
+    xb, w13b, w2b = _bits(rng, (T, d)), _bits(rng, (E, 2 * F, d), 0.3), _bits(rng, (E, d, F), 0.3)
+    z = (rng.standard_normal((T, E)) - 8.0 * (np.arange(E) == 4)).astype(np.float32)   # expert 4 unused
+    idx = oracle.select_topk(z, k)
+    assert not np.any(idx == 4)
+    dy = rng.standard_normal((T, d))
+    ref = oracle.backward(xb, w13b, w2b, z, idx, dy, renorm=renorm)
+    tokens = [7, 0, 29, 7, 13]
+    experts = [3, 4, 0]
+    got = oracle.backward_sampled(xb, w13b, w2b, z, idx, dy, tokens, experts, renorm=renorm)
+    for name in ("dx", "dgate", "dz"):
+        scale = 1 + np.abs(ref[name]).max()
+        assert np.abs(got[name] - ref[name][tokens]).max() <= 1e-12 * scale, name
+    for name in ("dw_gate_up", "dw_down"):
+        scale = 1 + np.abs(ref[name]).max()
+        assert np.abs(got[name] - ref[name][experts]).max() <= 1e-12 * scale, name
+    assert np.count_nonzero(got["dw_gate_up"][1]) == 0 and np.count_nonzero(got["dw_down"][1]) == 0
