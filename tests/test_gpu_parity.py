@@ -352,3 +352,34 @@ def test_borrow_sampled_parity_hot_expert():
                          tokens=tok)
     got = y[torch.as_tensor(tok, device="cuda")].cpu().numpy().astype(np.float64)
     assert rel_err(got, ref) <= Y_TOL
+
+
+# Every round of this shape leaves each expert a short last row block: C = 300 rows are one
+# 256-row tile and 44 rows, which the CTA-pair GEMMs run as swapped tiles (weights on the MMA's
+# M side, the 44 rows rounded up to 48 on its N side); the last round's blocks range from a few
+# rows to more than 128 (then a 256-row tile again).
+SWAP_SHAPE = dict(T=8192, d=1024, E=32, k=4, F=1024, C=300)
+
+
+@pytest.mark.parametrize("borrow", [False, True], ids=["per-expert", "borrow"])
+@pytest.mark.parametrize("bias", ["none", "zipf"])
+def test_swapped_tail_tiles_full_parity(bias, borrow):
+    w = wl.custom(name="swap", bias=bias, zipf_s=0.5, seed=21, **SWAP_SHAPE)
+    inp = wl.generate(w, "cuda")
+    layer, y = run_gpu(w, inp, schedule="per_round", borrow=borrow)
+    z = inp["logits"].cpu().numpy()
+    idx, g, p = check_plan(layer, w, w.C, z, borrow=borrow)
+    assert p["R"] >= 3
+    ref = oracle.forward(bits(inp["x"]), LazyExperts(inp["w_gate_up"]), LazyExperts(inp["w_down"]), idx, g)
+    assert rel_err(y.cpu().numpy().astype(np.float64), ref) <= Y_TOL
+
+
+def test_swapped_tail_tiles_match_the_pipelined_bits():
+    """A swapped tile computes each output as the same K-ordered fp32 sum of the same products
+    as a 128-row tile of the single-CTA kernel that runs the pipelined rounds, so the two
+    schedules agree bit for bit on a shape whose per-round GEMMs use swapped tiles."""
+    w = wl.custom(name="swap", bias="none", seed=21, **SWAP_SHAPE)
+    inp = wl.generate(w, "cuda")
+    _, y_round = run_gpu(w, inp, schedule="per_round")
+    _, y_pipe = run_gpu(w, inp, schedule="pipeline")
+    assert torch.equal(y_round, y_pipe)
