@@ -143,6 +143,9 @@ struct PlanBuffers {
 };
 cudaError_t launch_plan(const PlanBuffers& b, int T, int k, int E, int C, int max_rounds,
                         cudaStream_t stream);
+// One block copies n words from device memory to dst, host memory mapped into the device's
+// address space (a kernel's stores, not a copy engine).
+cudaError_t launch_copy_words(const int32_t* src, int32_t* dst, int n, cudaStream_t stream);
 
 // ---- dispatch / combine (dispatch_combine.cu)
 // dbg: the workspace header when MOE_FLAG_DEBUG_BOUNDS is set (row checks against T tokens and

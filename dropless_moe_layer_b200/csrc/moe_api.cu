@@ -73,6 +73,44 @@ using namespace moe;
 
 namespace {
 
+// Host words mapped into the device's address space, for reading the plan summary without a
+// copy engine (moe_plan). One buffer per host thread and device: moe_plan returns only after
+// reading it, so a thread never has two reads of its buffer in flight. Allocated on first use
+// (kHdrWords words of pinned host memory) and kept for the thread's lifetime; null if the
+// allocation fails (moe_plan then copies with cudaMemcpyAsync).
+struct MappedWords {
+  volatile int32_t* host = nullptr;
+  int32_t* dev = nullptr;
+};
+
+#ifndef MOE_PLAN_MAPPED
+#define MOE_PLAN_MAPPED 1   // 0: moe_plan reads its summary back with cudaMemcpyAsync
+#endif
+
+const MappedWords* mapped_words() {
+  if (!MOE_PLAN_MAPPED) return nullptr;
+  thread_local MappedWords per_device[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  MappedWords& m = per_device[dev & 63];
+  if (m.host == nullptr) {
+    void* h = nullptr;
+    void* d = nullptr;
+    if (cudaHostAlloc(&h, kHdrWords * sizeof(int32_t), cudaHostAllocMapped) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    if (cudaHostGetDevicePointer(&d, h, 0) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFreeHost(h);
+      return nullptr;
+    }
+    m.host = static_cast<volatile int32_t*>(h);
+    m.dev = static_cast<int32_t*>(d);
+  }
+  return &m;
+}
+
 int check_shape(const moe_shape_t* s) {
   if (s == nullptr) return MOE_ERR_INVALID_ARG;
   if (s->flags & ~static_cast<uint32_t>(MOE_FLAG_RENORM_TOPK | MOE_FLAG_PER_ROUND | MOE_FLAG_PIPELINE_ALL |
@@ -560,10 +598,21 @@ int moe_plan(const moe_shape_t* shape, const float* logits, const uint16_t* x,
   pb.dbg = debug_bounds(&s) ? header : nullptr;
   if ((st = cuda_status(launch_plan(pb, s.T, s.k, s.E, s.C, L.max_rounds, stream))) != MOE_OK) return st;
 
+  // The plan summary comes home through host memory mapped into the device, written by a
+  // kernel: a copy-engine transfer would queue behind any large transfer the caller has in
+  // flight in the same direction on another stream (a result going back to the host while
+  // the next batch is planned), and moe_plan would wait for it.
   int32_t host[kHdrWords];
-  if (cudaMemcpyAsync(host, header, sizeof(host), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  const MappedWords* mw = mapped_words();
+  if (mw != nullptr) {
+    if ((st = cuda_status(launch_copy_words(header, mw->dev, kHdrWords, stream))) != MOE_OK) return st;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+    std::memcpy(host, const_cast<const int32_t*>(mw->host), sizeof(host));
+  } else {
+    if (cudaMemcpyAsync(host, header, sizeof(host), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  }
   if (host[kHdrStatus] != 0) return MOE_ERR_TIMEOUT;
 
   info->R = host[kHdrR];

@@ -304,7 +304,24 @@ __global__ void __launch_bounds__(kTPB) plan_rank_kernel(const int32_t* __restri
   }
 }
 
+// dst[i] = src[i] for i < n, with the stores made visible system-wide (dst is host memory
+// mapped into the device's address space).
+__global__ void __launch_bounds__(kTPB) copy_words_kernel(const int32_t* __restrict__ src, int32_t* dst, int n) {
+  sm100::grid_dependency_wait();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) dst[i] = src[i];
+  __threadfence_system();
+  sm100::pdl_trigger_early();
+  sm100::pdl_trigger_late();
+}
+
 }  // namespace
+
+cudaError_t launch_copy_words(const int32_t* src, int32_t* dst, int n, cudaStream_t stream) {
+  launch_begin(kKindPlan, stream);
+  const cudaError_t err = launch_pdl(copy_words_kernel, dim3(1), dim3(kTPB), 0, stream, src, dst, n);
+  launch_end(kKindPlan, stream);
+  return err;
+}
 
 cudaError_t launch_plan(const PlanBuffers& b, int T, int k, int E, int C, int max_rounds,
                         cudaStream_t stream) {

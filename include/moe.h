@@ -31,7 +31,8 @@
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller, row-major, contiguous,
  *     16-byte aligned. bf16 is passed as its uint16_t bit pattern. The workspace must be
- *     256-byte aligned. The library allocates no device memory.
+ *     256-byte aligned. The library allocates no device memory (moe_plan keeps one small
+ *     pinned, device-mapped host buffer per host thread and device; see moe_plan).
  *   - Entry points return MOE_OK (0) or a negative moe_status; invalid arguments are found
  *     on the host before any kernel is launched, and no entry point aborts the process.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).
@@ -183,6 +184,11 @@ MOE_API int moe_workspace_layout(const moe_shape_t* shape, moe_workspace_layout_
  *   bias     [E] fp32 or NULL (used only when logits == NULL).
  * Writes topk/gate/round/slot/load/offsets/n and the round-major row list into `ws`,
  * then synchronizes `stream` once and fills *info (R, max_load, load[], device pointers).
+ * The summary (1280 bytes) comes home through pinned host memory mapped into the device,
+ * written by a one-block kernel rather than by a copy engine, so that a large device-to-host
+ * copy the caller has in flight on another stream does not delay moe_plan until it ends. That
+ * buffer is allocated on the first call of each host thread on each device and kept for the
+ * thread's lifetime; if it cannot be allocated, moe_plan copies with cudaMemcpyAsync instead.
  * Non-finite logits give undefined routing. */
 MOE_API int moe_plan(const moe_shape_t* shape, const float* logits, const uint16_t* x,
              const uint16_t* w_router, const float* bias, void* ws, size_t ws_bytes,
