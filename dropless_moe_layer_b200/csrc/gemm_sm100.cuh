@@ -167,9 +167,6 @@ struct Phase {
   // Weights of group g: expert group_expert[g] of the B map (expert parallelism: a group is one
   // source rank's rows of one local expert). Null: expert g.
   const int32_t* group_expert;
-  // CTA-pair form: a group whose last row block holds at most kSwapRows rows runs that block as
-  // swapped tiles (weights as the MMA's M side, the rows as its N side; see run_phase_pair).
-  int swap_tail;
 };
 
 __device__ __forceinline__ int group_weights(const Phase& p, int g) { return p.group_expert ? p.group_expert[g] : g; }
@@ -500,25 +497,6 @@ constexpr int kPairStages = kRingBytes / kPairStageBytes;        // 6
 static_assert(kPairStages <= kMaxStages, "pair ring stages");
 constexpr int kEpiWarpsPair = 8;         // arrivals on the leader's tempty per tile
 
-// Swapped tiles. A group's last row block with at most kSwapRows rows (an expert's few leftover
-// rows, common in a round that holds every expert) would waste most of a 256-row tile. It runs
-// instead as n_total / 256 swapped tiles: the MMA's M side is 256 weight rows (output columns;
-// CTA c loads 128 of them) and its N side the block's rows, rounded up to 16 (CTA c loads rows
-// [N/2 c, N/2 c + N/2) of them; the A map's 128-row box, the rest unused). The accumulator is
-// then transposed: TMEM lane = output column, TMEM column = row. SwiGLU needs gate and up of a
-// column in one lane, so its swapped tile takes two ring slots per k block (W1 rows with the
-// token rows, then the same W3 rows) and two MMAs, into accumulator columns [0, N) and
-// [128, 128 + N); a swapped tile covers 256 output columns in either mode.
-constexpr int kSwapRows = 128;
-
-// Tiles of a group with `rows` rows in the pair form (n_tiles column tiles per 256-row block).
-__device__ __forceinline__ int pair_tiles_of(const Phase& p, int rows, int n_tiles) {
-  const int full = rows / kPairRows, tail = rows - full * kPairRows;
-  if (tail == 0) return full * n_tiles;
-  if (p.swap_tail && tail <= kSwapRows) return full * n_tiles + p.n_total / kPairBn;
-  return (full + 1) * n_tiles;
-}
-
 // Set-up of both CTAs of a pair: barriers (thread 0 of each), the pair's TMEM (warp 1 of each),
 // then a cluster barrier, so that no CTA signals its peer before the peer's barriers exist.
 __device__ __forceinline__ uint32_t setup_pair(const Smem& s) {
@@ -568,7 +546,10 @@ __device__ __forceinline__ void plan_phase_pair(const Smem& s, const Phase& p, i
   for (int g0 = 0; g0 < p.groups; g0 += 32) {
     const int g = g0 + lane;
     int cnt = 0;
-    if (g < p.groups) cnt = pair_tiles_of(p, group_rows(p, g), n_tiles);
+    if (g < p.groups) {
+      const int rows = group_rows(p, g);
+      cnt = ((rows + kPairRows - 1) / kPairRows) * n_tiles;
+    }
     int incl = cnt;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -592,45 +573,17 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
   const int* ts = s.tile_start[which];
   const int n_tiles = p.n_total / width;
   const int total = ts[p.groups];
-  // A tile: group g; a 256-row tile (row block mp, column tile nt) or a swapped tile (256-column
-  // block sb over the group's last n <= kSwapRows rows, from row rows0).
-  struct Tile {
-    int g, mp, nt, sb, rows0, n;
-    bool swap;
-  };
-  auto decode = [&](int tile) {
-    Tile t;
+  auto decode = [&](int tile, int& g, int& mp, int& nt) {
     int lo = 0, hi = p.groups - 1;   // largest g with ts[g] <= tile
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
       if (ts[mid] <= tile) lo = mid; else hi = mid - 1;
     }
-    t.g = lo;
-    const int local = tile - ts[t.g];
-    const int rows = group_rows(p, t.g);
-    const int full = rows / kPairRows, tail = rows - full * kPairRows;
-    const bool swap_ok = p.swap_tail && tail > 0 && tail <= kSwapRows;
-    const int normal = (swap_ok || tail == 0 ? full : full + 1) * n_tiles;
-    t.swap = local >= normal;
-    if (t.swap) {
-      t.mp = full;
-      t.nt = 0;
-      t.sb = local - normal;
-      t.rows0 = full * kPairRows;
-      t.n = tail;
-    } else {
-      t.mp = local / n_tiles;
-      t.nt = local - t.mp * n_tiles;
-      t.sb = 0;
-      t.rows0 = t.mp * kPairRows;
-      t.n = 0;
-    }
-    return t;
+    g = lo;
+    const int local = tile - ts[g];
+    mp = local / n_tiles;
+    nt = local - mp * n_tiles;
   };
-  // MMA N of a swapped tile: its rows rounded up to 16
-  auto swap_n = [](int n) { return (n + 15) & ~15; };
-  // ring slots per k block: SwiGLU swapped tiles take two (W1 rows with the token rows, W3 rows)
-  const int swap_slots = p.mode == kSwiGLU ? 2 : 1;
   // B rows of this CTA's half of a tile
   auto b_row = [&](int nt) {
     return p.mode == kSwiGLU ? static_cast<int>(cta) * p.b_second_row + nt * width
@@ -639,53 +592,35 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer (both CTAs)
+    const uint32_t tx = 2u * kPairStageBytes;   // the pair's bytes per stage, counted by the leader
     bool ok = true;
-    // one ring slot: wait for it to be free, count the pair's bytes on the leader's barrier and
-    // load up to two boxes into it (A part at the slot's start, B part after kABytes)
-    auto fill_slot = [&](uint32_t tx, const CUtensorMap* ma, int ka, int ra, int ga, const CUtensorMap* mb, int kb_,
-                         int rb, int gb) {
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&s.empty[pipe.stage]), pipe.phase ^ 1u, s.abort)))
-        return false;
-      const uint32_t sA = smem_addr(s.stage + pipe.stage * kPairStageBytes);
-      const uint32_t fb_local = smem_addr(&s.full[pipe.stage]);
-      const uint32_t fb = peer_addr(fb_local, 0);   // the leader's full barrier
-      if (cta == 0 && lane == 0) mbar_arrive_expect_tx(fb_local, tx);
-      __syncwarp();
-      if (lane == 0) {
-        tma_load_3d_pair(sA, ma, fb, ka, ra, ga);
-        if (mb != nullptr) tma_load_3d_pair(sA + kABytes, mb, fb, kb_, rb, gb);
-      }
-      pipe.issued |= 1u << pipe.stage;
-      if (++pipe.stage == kPairStages) {
-        pipe.stage = 0;
-        pipe.phase ^= 1u;
-      }
-      return true;
-    };
     for (int tile = pair; ok && tile < total; tile += pairs) {
-      const Tile t = decode(tile);
-      const int g = t.g;
-      // this CTA's first row of the group's rows in the A operand, and the A map's group
-      int a_row = t.rows0, a_grp = g;
+      int g, mp, nt;
+      decode(tile, g, mp, nt);
+      int a_row = mp * kPairRows + static_cast<int>(cta) * BM, a_grp = g;   // this CTA's first A row
       if (p.group_row) {
         a_row += p.group_row[g] - *p.group_row_base;
         a_grp = 0;
       }
-      if (!t.swap) {
-        a_row += static_cast<int>(cta) * BM;
-        for (int kb = 0; ok && kb < p.num_k_blocks; ++kb)
-          ok = fill_slot(2u * kPairStageBytes, p.a, kb * BK, a_row, a_grp, p.b[0], kb * BK, b_row(t.nt),
-                         group_weights(p, g));
-      } else {
-        // M side: 128 weight rows of the 256-column block per CTA; N side: half the rows each
-        a_row += static_cast<int>(cta) * (swap_n(t.n) / 2);
-        const int w_row = t.sb * kPairBn + static_cast<int>(cta) * kPairBHalf;
-        for (int kb = 0; ok && kb < p.num_k_blocks; ++kb) {
-          ok = fill_slot(2u * kPairStageBytes, p.b[0], kb * BK, w_row, group_weights(p, g), p.a, kb * BK, a_row,
-                         a_grp);
-          if (ok && swap_slots == 2)
-            ok = fill_slot(2u * kABytes, p.b[0], kb * BK, p.b_second_row + w_row, group_weights(p, g), nullptr, 0,
-                           0, 0);
+      for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&s.empty[pipe.stage]), pipe.phase ^ 1u, s.abort))) {
+          ok = false;
+          break;
+        }
+        const uint32_t sA = smem_addr(s.stage + pipe.stage * kPairStageBytes);
+        const uint32_t sB = sA + kABytes;
+        const uint32_t fb_local = smem_addr(&s.full[pipe.stage]);
+        const uint32_t fb = peer_addr(fb_local, 0);   // the leader's full barrier
+        if (cta == 0 && lane == 0) mbar_arrive_expect_tx(fb_local, tx);
+        __syncwarp();
+        if (lane == 0) {
+          tma_load_3d_pair(sA, p.a, fb, kb * BK, a_row, a_grp);
+          tma_load_3d_pair(sB, p.b[0], fb, kb * BK, b_row(nt), group_weights(p, g));
+        }
+        pipe.issued |= 1u << pipe.stage;
+        if (++pipe.stage == kPairStages) {
+          pipe.stage = 0;
+          pipe.phase ^= 1u;
         }
       }
     }
@@ -702,53 +637,32 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
   } else if (warp == 1) {
     if (lane == 0 && cta == 0) {
     // ---------------------------------------------------------------- MMA issuer (leader only)
+    const uint32_t idesc = idesc_bf16_f32(kPairRows, kPairBn);
     bool ok = true;
-    // waits for the next ring slot to be full and moves past it; returns its index (-1: gave up)
-    auto take_slot = [&]() -> int {
-      if (!mbar_wait(smem_addr(&s.full[pipe.stage]), pipe.phase, s.abort)) return -1;
-      tc_fence_after();
-      const int slot = pipe.stage;
-      if (++pipe.stage == kPairStages) {
-        pipe.stage = 0;
-        pipe.phase ^= 1u;
-      }
-      return slot;
-    };
-    auto slot_addr = [&](int slot) { return smem_addr(s.stage + slot * kPairStageBytes); };
-    // a slot is free again once the MMAs issued so far (all that read it) are done
-    auto free_slot = [&](int slot) { mma_commit_pair(smem_addr(&s.empty[slot]), 3); };
     for (int tile = pair; ok && tile < total; tile += pairs) {
-      const Tile t = decode(tile);
       if (!mbar_wait(smem_addr(&s.tempty[pipe.acc]), pipe.acc_phase ^ 1u, s.abort)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(pipe.acc * kAccCols);
-      const uint32_t idesc = idesc_bf16_f32(kPairRows, t.swap ? swap_n(t.n) : kPairBn);
-      const bool two = t.swap && swap_slots == 2;
       for (int kb = 0; kb < p.num_k_blocks; ++kb) {
-        const int s0 = take_slot();
-        const int s1 = (s0 >= 0 && two) ? take_slot() : 0;
-        if (s0 < 0 || s1 < 0) {
+        if (!mbar_wait(smem_addr(&s.full[pipe.stage]), pipe.phase, s.abort)) {
           ok = false;
           break;
         }
-        const uint32_t sA = slot_addr(s0);
+        tc_fence_after();
+        const uint32_t sA = smem_addr(s.stage + pipe.stage * kPairStageBytes);
         const uint64_t adesc = smem_desc_sw128(sA);
         const uint64_t bdesc = smem_desc_sw128(sA + kABytes);
 #pragma unroll
         for (int kk = 0; kk < BK / UMMA_K; ++kk)
           mma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
-        if (two) {
-          // the W3 rows of the same k block against the same token rows: up into columns 128..
-          const uint64_t udesc = smem_desc_sw128(slot_addr(s1));
-#pragma unroll
-          for (int kk = 0; kk < BK / UMMA_K; ++kk)
-            mma_bf16_pair(d_tmem + kPairBHalf, udesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+        mma_commit_pair(smem_addr(&s.empty[pipe.stage]), 3);
+        if (++pipe.stage == kPairStages) {
+          pipe.stage = 0;
+          pipe.phase ^= 1u;
         }
-        free_slot(s0);
-        if (two) free_slot(s1);
       }
       if (!ok) break;
       mma_commit_pair(smem_addr(&s.tfull[pipe.acc]), 3);
@@ -771,8 +685,8 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
     // the outputs stream out: first in line for eviction, behind the tiles the MMAs still reuse
     const uint64_t out_policy = policy_evict_first();
     for (int tile = pair; tile < total; tile += pairs) {
-      const Tile t = decode(tile);
-      const int g = t.g;
+      int g, mp, nt;
+      decode(tile, g, mp, nt);
       const bool ready = __all_sync(0xffffffffu, mbar_wait(smem_addr(&s.tfull[pipe.acc]), pipe.acc_phase, s.abort));
       if (!ready) {
         if (lane == 0) atomicOr(status, kStatusTimeoutEpilogue);
@@ -780,88 +694,59 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
         break;
       }
       tc_fence_after();
+      const int row = mp * kPairRows + static_cast<int>(cta) * BM + q * 32 + lane;
+      const int rows_g = group_rows(p, g);
+      const bool valid = row < rows_g;
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(pipe.acc * kAccCols);
-      // output row `row` of group g, as an element offset into out
-      auto out_row = [&](int row) {
-        return p.group_row ? static_cast<long long>(p.group_row[g] - *p.group_row_base + row) * p.out_ld
-                           : g * p.out_group_stride + static_cast<long long>(row) * p.out_ld;
-      };
-      if (t.swap) {
-        // transposed accumulator: this thread's lane is one output column, TMEM columns are the
-        // rows; each store instruction of the warp writes 32 adjacent columns (64 bytes) of a row
-        const int col = t.sb * kPairBn + static_cast<int>(cta) * kPairBHalf + q * 32 + lane;
-        uint16_t* out = static_cast<uint16_t*>(p.out);
-        for (int c0 = 0; c0 < t.n; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld32(tb + c0, v);
+      const long long orow_off = p.group_row
+                                     ? static_cast<long long>(p.group_row[g] - *p.group_row_base + row) * p.out_ld
+                                     : g * p.out_group_stride + static_cast<long long>(row) * p.out_ld;
+      uint16_t* orow = static_cast<uint16_t*>(p.out) + orow_off + nt * width;
+      if (p.out_map != nullptr) {
+        // 32-column chunks: TMEM -> registers -> this warp's staging buffer -> one bulk store of
+        // its 32 rows. Rows of the box past the group's rows hold junk; they fall in the expert's
+        // unused rows [n, C) (never read) or past C (clipped by the map).
+        const int row_base = mp * kPairRows + static_cast<int>(cta) * BM + q * 32;
+        const int chunks = (p.mode == kSwiGLU ? width : kPairBn) / kOutChunkCols;
+        for (int c = 0; c < chunks; ++c) {
+          uint32_t pk[16];
           if (p.mode == kSwiGLU) {
-            uint32_t u[32];
-            tmem_ld32(tb + kPairBHalf + c0, u);
+            uint32_t gv[32], uv[32];
+            tmem_ld32(tb + c * kOutChunkCols, gv);
+            tmem_ld32(tb + width + c * kOutChunkCols, uv);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              v[i] = __float_as_uint(silu_f(__uint_as_float(v[i])) * __uint_as_float(u[i]));
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(silu_f(__uint_as_float(gv[2 * i])) * __uint_as_float(uv[2 * i]),
+                                  silu_f(__uint_as_float(gv[2 * i + 1])) * __uint_as_float(uv[2 * i + 1]));
           } else {
+            uint32_t v[32];
+            tmem_ld32(tb + c * kOutChunkCols, v);
             tmem_wait_ld();
-          }
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (c0 + i < t.n) {
-              const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(v[i]));
-              out[out_row(t.rows0 + c0 + i) + col] = *reinterpret_cast<const uint16_t*>(&b);
-            }
+            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
           }
+          const uint32_t buf_off = (ochunk & 1u) * kOutChunkBytes;
+          if (lane == 0) bulk_wait_read_1();   // the store that last used this buffer has read it
+          __syncwarp();
+          uint8_t* row_ptr = s.out_stage + q * 2 * kOutChunkBytes + buf_off + lane * 64;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)   // 64-byte swizzle: piece j of row r at j ^ ((r >> 1) & 3)
+            *reinterpret_cast<uint4*>(row_ptr + ((j ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(p.out_map, stage0 + buf_off, nt * width + c * kOutChunkCols, row_base, g, out_policy);
+            bulk_commit();
+          }
+          ++ochunk;
         }
+      } else if (p.mode == kSwiGLU) {
+        store_swiglu(tb, width, orow, valid);
       } else {
-        const int row = t.rows0 + static_cast<int>(cta) * BM + q * 32 + lane;
-        const bool valid = row < group_rows(p, g);
-        uint16_t* orow = static_cast<uint16_t*>(p.out) + out_row(row) + t.nt * width;
-        if (p.out_map != nullptr) {
-          // 32-column chunks: TMEM -> registers -> this warp's staging buffer -> one bulk store of
-          // its 32 rows. Rows of the box past the group's rows hold junk; they fall in the
-          // expert's unused rows [n, C) (never read) or past C (clipped by the map).
-          const int row_base = t.rows0 + static_cast<int>(cta) * BM + q * 32;
-          const int chunks = (p.mode == kSwiGLU ? width : kPairBn) / kOutChunkCols;
-          for (int c = 0; c < chunks; ++c) {
-            uint32_t pk[16];
-            if (p.mode == kSwiGLU) {
-              uint32_t gv[32], uv[32];
-              tmem_ld32(tb + c * kOutChunkCols, gv);
-              tmem_ld32(tb + width + c * kOutChunkCols, uv);
-              tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                pk[i] = pack_bf16x2(silu_f(__uint_as_float(gv[2 * i])) * __uint_as_float(uv[2 * i]),
-                                    silu_f(__uint_as_float(gv[2 * i + 1])) * __uint_as_float(uv[2 * i + 1]));
-            } else {
-              uint32_t v[32];
-              tmem_ld32(tb + c * kOutChunkCols, v);
-              tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-            }
-            const uint32_t buf_off = (ochunk & 1u) * kOutChunkBytes;
-            if (lane == 0) bulk_wait_read_1();   // the store that last used this buffer has read it
-            __syncwarp();
-            uint8_t* row_ptr = s.out_stage + q * 2 * kOutChunkBytes + buf_off + lane * 64;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)   // 64-byte swizzle: piece j of row r at j ^ ((r >> 1) & 3)
-              *reinterpret_cast<uint4*>(row_ptr + ((j ^ ((lane >> 1) & 3)) << 4)) =
-                  make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-            fence_async_shared();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_3d(p.out_map, stage0 + buf_off, t.nt * width + c * kOutChunkCols, row_base, g, out_policy);
-              bulk_commit();
-            }
-            ++ochunk;
-          }
-        } else if (p.mode == kSwiGLU) {
-          store_swiglu(tb, width, orow, valid);
-        } else {
-          store_bf16(tb, kPairBn, orow, valid);
-        }
+        store_bf16(tb, kPairBn, orow, valid);
       }
       tc_fence_before();
       __syncwarp();

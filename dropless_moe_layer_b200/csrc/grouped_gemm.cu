@@ -93,7 +93,6 @@ struct KernelArgs {
   int rows_cap;                    // debug bounds checks (see Phase): 0 = unchecked
   int tma_out;                     // CTA-pair form: store through the output map (see Phase)
   const int32_t* group_expert;     // weights of each group (see Phase), or null
-  int swap_tail;                   // CTA-pair form: swapped tiles for short last row blocks (see Phase)
 };
 
 __global__ void __launch_bounds__(kLaunchThreads, 1)
@@ -132,7 +131,6 @@ __global__ void __launch_bounds__(kLaunchThreads, 1)
   p.dbg = args.rows_cap > 0 ? args.status - kHdrStatus : nullptr;
   p.out_map = nullptr;
   p.group_expert = args.group_expert;
-  p.swap_tail = 0;
   plan_phase(s, p, 0);              // reads only the row counts (plan data)
   __syncthreads();
   // Everything above overlaps the previous kernel; the operands, and the output buffer that
@@ -189,7 +187,6 @@ __global__ void __launch_bounds__(kLaunchThreads, 1)
   p.dbg = args.rows_cap > 0 ? args.status - kHdrStatus : nullptr;
   p.out_map = args.tma_out ? &tout : nullptr;
   p.group_expert = args.group_expert;
-  p.swap_tail = args.swap_tail;
   plan_phase_pair(s, p, 0, width);
   __syncthreads();
   grid_dependency_wait();
@@ -413,36 +410,17 @@ static int pair_clusters() {
   return n;
 }
 
-#ifndef MOE_GEMM_SWAP
-#define MOE_GEMM_SWAP 1   // 0: the CTA-pair form never uses swapped tiles for short last row blocks
-#endif
-
-// Whether the pair form may run a group's short last row block as swapped tiles (256 output
-// columns each, so n_total must be a multiple of 256).
-static bool swap_ok(int n_total) { return MOE_GEMM_SWAP && n_total % kPairBn == 0; }
-
-// Whether a round's GEMM runs in the CTA-pair form: its tiles must keep every cluster busy and
-// cover at most 15 % more rows than the 128-row tiles of the single-CTA form. With swapped
-// tiles a short last row block costs its rows rounded up to 16 instead of a 256-row tile.
+// Whether a round's GEMM runs in the CTA-pair form: its 256-row tiles must keep every cluster
+// busy and pad at most kPairPadding more rows than the 128-row tiles of the single-CTA form.
 static bool use_pair(const int32_t* n_host, int groups, int n_total, int width) {
   if (!MOE_GEMM_PAIR || n_host == nullptr || n_total % width != 0) return false;
-  const bool swap = swap_ok(n_total);
-  const long long n_tiles = n_total / width;
   long long pair_tiles = 0, rows_pair = 0, rows_single = 0;
   for (int g = 0; g < groups; ++g) {
-    const long long full = n_host[g] / kPairRows, tail = n_host[g] - full * kPairRows;
-    if (tail == 0) {
-      pair_tiles += full * n_tiles;
-      rows_pair += full * kPairRows;
-    } else if (swap && tail <= kSwapRows) {
-      pair_tiles += full * n_tiles + n_total / kPairBn;
-      rows_pair += full * kPairRows + (tail + 15) / 16 * 16;
-    } else {
-      pair_tiles += (full + 1) * n_tiles;
-      rows_pair += (full + 1) * kPairRows;
-    }
+    pair_tiles += (n_host[g] + kPairRows - 1) / kPairRows;
+    rows_pair += static_cast<long long>((n_host[g] + kPairRows - 1) / kPairRows) * kPairRows;
     rows_single += static_cast<long long>((n_host[g] + BM - 1) / BM) * BM;
   }
+  pair_tiles *= n_total / width;
   const int clusters = pair_clusters();
   return clusters > 0 && pair_tiles >= clusters && rows_pair * 100 <= rows_single * 115;
 }
@@ -541,7 +519,6 @@ cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint1
     CUtensorMap mo{};
     a.tma_out = MOE_TMA_OUT_GATE_UP && group_row == nullptr;   // per-expert h [E][C][F]: stored by TMA
     if (a.tma_out && (e = gemm::make_map(&mo, h, F, C, E, 32, gemm::kOutChunkCols)) != cudaSuccess) return e;
-    a.swap_tail = gemm::swap_ok(F);
     return gemm::run_pair(ma, mb[0], mo, a, 128, make_side(copy), kKindGateUp, stream);
   }
   const long long tiles = gemm::choose_width(n_host, E, 0, F, a);
@@ -574,7 +551,6 @@ cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out
     if ((e = gemm::make_map(&mb_half, w_down, F, d, E, gemm::kPairBHalf)) != cudaSuccess) return e;
     a.tma_out = group_row == nullptr;          // per-expert out [E][C][d]: stored by TMA
     if (a.tma_out && (e = gemm::make_map(&mo, out, d, C, E, 32, gemm::kOutChunkCols)) != cudaSuccess) return e;
-    a.swap_tail = gemm::swap_ok(d);
     return gemm::run_pair(ma, mb_half, mo, a, gemm::kPairBn, make_side(copy), kKindDown, stream);
   }
   const long long tiles = gemm::choose_width(n_host, E, 0, d, a);
@@ -607,7 +583,6 @@ cudaError_t launch_ep_experts(const uint16_t* recv, const uint16_t* w_gate_up, c
   const gemm::SideArgs none = make_side(nullptr);
   if (gemm::use_pair(rows_host, groups, F, 128)) {
     CUtensorMap unused{};
-    a.swap_tail = gemm::swap_ok(F);
     e = gemm::run_pair(ma, mb[0], unused, a, 128, none, kKindGateUp, stream);
   } else {
     const long long tiles = gemm::choose_width(rows_host, groups, 0, F, a);
@@ -632,7 +607,6 @@ cudaError_t launch_ep_experts(const uint16_t* recv, const uint16_t* w_gate_up, c
   if (gemm::use_pair(rows_host, groups, d, gemm::kPairBn)) {
     CUtensorMap mb_half, unused{};
     if ((e = gemm::make_map(&mb_half, w_down, F, d, E_local, gemm::kPairBHalf)) != cudaSuccess) return e;
-    b.swap_tail = gemm::swap_ok(d);
     return gemm::run_pair(ma, mb_half, unused, b, gemm::kPairBn, none, kKindDown, stream);
   }
   if ((e = gemm::make_b_maps(mb, w_down, F, d, E_local, kDownWidths, d)) != cudaSuccess) return e;

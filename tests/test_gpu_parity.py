@@ -354,31 +354,32 @@ def test_borrow_sampled_parity_hot_expert():
     assert rel_err(got, ref) <= Y_TOL
 
 
-# Every round of this shape leaves each expert a short last row block: C = 300 rows are one
-# 256-row tile and 44 rows, which the CTA-pair GEMMs run as swapped tiles (weights on the MMA's
-# M side, the 44 rows rounded up to 48 on its N side); the last round's blocks range from a few
-# rows to more than 128 (then a 256-row tile again).
-SWAP_SHAPE = dict(T=8192, d=1024, E=32, k=4, F=1024, C=300)
+# Round 0 of this shape gives each expert C = 1100 rows: four 256-row tiles of the CTA-pair
+# GEMMs and a last tile with 76 rows; later rounds leave ragged last tiles of other sizes. The
+# per-round GEMMs of round 0 run in the pair form (their 256-row tiles cover at most 15 % more
+# rows than 128-row tiles).
+RAGGED_SHAPE = dict(T=16384, d=512, E=32, k=4, F=512, C=1100)
 
 
 @pytest.mark.parametrize("borrow", [False, True], ids=["per-expert", "borrow"])
 @pytest.mark.parametrize("bias", ["none", "zipf"])
-def test_swapped_tail_tiles_full_parity(bias, borrow):
-    w = wl.custom(name="swap", bias=bias, zipf_s=0.5, seed=21, **SWAP_SHAPE)
+def test_ragged_pair_tiles_full_parity(bias, borrow):
+    w = wl.custom(name="ragged", bias=bias, zipf_s=0.5, seed=21, **RAGGED_SHAPE)
     inp = wl.generate(w, "cuda")
     layer, y = run_gpu(w, inp, schedule="per_round", borrow=borrow)
     z = inp["logits"].cpu().numpy()
     idx, g, p = check_plan(layer, w, w.C, z, borrow=borrow)
-    assert p["R"] >= 3
+    assert p["R"] >= 2
     ref = oracle.forward(bits(inp["x"]), LazyExperts(inp["w_gate_up"]), LazyExperts(inp["w_down"]), idx, g)
     assert rel_err(y.cpu().numpy().astype(np.float64), ref) <= Y_TOL
 
 
-def test_swapped_tail_tiles_match_the_pipelined_bits():
-    """A swapped tile computes each output as the same K-ordered fp32 sum of the same products
-    as a 128-row tile of the single-CTA kernel that runs the pipelined rounds, so the two
-    schedules agree bit for bit on a shape whose per-round GEMMs use swapped tiles."""
-    w = wl.custom(name="swap", bias="none", seed=21, **SWAP_SHAPE)
+def test_ragged_pair_tiles_match_the_pipelined_bits():
+    """The CTA-pair tiles of the per-round launches and the 128-row tiles of the single-CTA
+    kernel that runs the pipelined rounds compute each output as the same K-ordered fp32 sum,
+    so the two schedules agree bit for bit on a shape whose per-round GEMMs run in the pair
+    form with ragged last row blocks."""
+    w = wl.custom(name="ragged", bias="none", seed=21, **RAGGED_SHAPE)
     inp = wl.generate(w, "cuda")
     _, y_round = run_gpu(w, inp, schedule="per_round")
     _, y_pipe = run_gpu(w, inp, schedule="pipeline")
