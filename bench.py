@@ -51,14 +51,9 @@ TRAFFIC = {
     # 16 gate/up launches of one step, dram__bytes_read.sum + dram__bytes_write.sum by ncu on the
     # full workload (one-pass counters), averaged per launch
     ("32k-zipf1.2-router-gemm", "gate_up"): {
-        "bytes_per_launch": 49.5184e9 / 16,
+        "bytes_per_launch": 47.90227328e9 / 16,
         "sources": GEMM_SOURCES,
-        "sources_sha1": "885cff12e941df85df232b4e2ac9867b694c3aed"},
-    # the 3 gate/up launches of one step (profiles/gate_up_pair_gemm_16k-uniform.md's capture)
-    ("16k-uniform", "gate_up"): {
-        "bytes_per_launch": (3.669719e9 + 0.198734e9 + 4.317842e9 + 0.338580e9 + 0.788634e9 + 0.006991e9) / 3,
-        "sources": GEMM_SOURCES,
-        "sources_sha1": "885cff12e941df85df232b4e2ac9867b694c3aed"},
+        "sources_sha1": "a1a1b075c49c76fb449b808adbc8f6ec433d4e01"},
 }
 
 

@@ -22,10 +22,10 @@
 //              multiple of 64); the pair's gate -> row_gate
 //   recompute  [a | b] = xbuf W13^T (tensor cores); epilogue keeps a, b (bf16, row-major) and
 //              writes bf16(gate * h) transposed (hgT, F rows)
-//   dh         W2^T dy as dybuf (W2^T)^T (tensor cores, B = W2 transposed once per call);
+//   dh         W2^T dy as dybuf (W2^T)^T (tensor cores, B = W2 read MN-major as stored);
 //              epilogue: the SwiGLU backward (da, db from a, b and the gate), dgate partial sums
 //              <W2^T dy, h> per 64..256-column tile, dab = [da | db] row-major and transposed
-//   dx         dab W13 (tensor cores, B = W13 transposed once per call) -> dxbuf (bf16)
+//   dx         dab W13 (tensor cores, B = W13 read MN-major as stored) -> dxbuf (bf16)
 //   combine    dx[t] = (first round of t ? 0 : dx[t]) + sum of the token's dxbuf rows, ascending
 //              j; dgate[t, j] = sum of its row's partials in tile order (no atomics anywhere)
 //   wgrad      dW2 += dyT hgT^T and dW13 += dabT xT^T over K = the round's rows of each expert
@@ -88,8 +88,14 @@ struct GemmArgs {
   int overwrite;              // kWgrad: store the tile instead of adding it (round 0)
   int tma_out;                // kWgrad: write the tile through the phase's fp32 output map (TMA
                               // store, or TMA reduce-add) instead of per-thread read-add-write
+  int b_mn;                   // kDh, kDx: B is the weight itself, MN-major ([E][K][N] in memory:
+                              // W2 [E][d][d_ff] for dh, W13 [E][2 d_ff][d] for dx), loaded as
+                              // 64 x 64 boxes (64 N by 64 K), instead of a transposed copy
   int32_t* status;
 };
+
+constexpr int kMnBox = 64;                         // MN-major B boxes: 64 N x 64 K rows
+constexpr int kMnBoxBytes = kMnBox * BK * 2;       // 8 KB
 
 __device__ __forceinline__ uint16_t bf16_bits(float v) {
   const __nv_bfloat16 b = __float2bfloat16_rn(v);
@@ -455,7 +461,12 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           } else {
             const int a_row = p.group_row ? static_cast<int>(row_of(p, g, m0)) : m0;
             load(sA, ma, kb * BK, a_row, p.group_row ? 0 : g);
-            if (kPair) {
+            if (p.b_mn) {
+              // MN-major weights: this CTA's B columns as 64-column boxes, 8 KB apart
+              const int n0 = nt * p.width + (kPair ? static_cast<int>(cta) * gemm::kPairBHalf : 0);
+              const int nb = kPair ? gemm::kPairBHalf / kMnBox : p.width / kMnBox;
+              for (int j = 0; j < nb; ++j) load(sB + j * kMnBoxBytes, mb, n0 + j * kMnBox, kb * BK, g);
+            } else if (kPair) {
               // recompute: CTA 0 the tile's W1 rows, CTA 1 the same W3 rows; else 128 of the 256
               const int b_row = p.mode == kRecompute ? static_cast<int>(cta) * p.F + nt * p.width
                                                      : nt * p.width + static_cast<int>(cta) * gemm::kPairBHalf;
@@ -499,7 +510,9 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         int q, g, mt, nt;
         decode(tile, q, g, mt, nt);
         const GemmArgs& p = L.ph[q];
-        const uint32_t idesc = idesc_bf16_f32(kRows, bn_of(p));
+        const uint32_t idesc = p.b_mn ? idesc_bf16_f32_bmn(kRows, bn_of(p)) : idesc_bf16_f32(kRows, bn_of(p));
+        // one K step of 16: +32 B along a K-major row, +16 rows of 128 B in an MN-major box
+        const uint32_t b_step = p.b_mn ? (16u * 128u) >> 4 : 2u;
         const int kbs = k_blocks_of(p, g);
         if (!mbar_wait(smem_addr(&s.tempty[pipe.acc]), pipe.acc_phase ^ 1u, s.abort)) {
           ok = false;
@@ -515,13 +528,14 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           tc_fence_after();
           const uint32_t sA = smem_addr(s.stage + pipe.stage * kSlot);
           const uint64_t adesc = smem_desc_sw128(sA);
-          const uint64_t bdesc = smem_desc_sw128(sA + gemm::kABytes);
+          const uint64_t bdesc = p.b_mn ? smem_desc_sw128_mn(sA + gemm::kABytes, kMnBoxBytes)
+                                        : smem_desc_sw128(sA + gemm::kABytes);
 #pragma unroll
           for (int kk = 0; kk < BK / gemm::UMMA_K; ++kk) {
             if (kPair)
-              mma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+              mma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + b_step * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
             else
-              mma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+              mma_bf16(d_tmem, adesc + 2 * kk, bdesc + b_step * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           if (kPair)
             mma_commit_pair(smem_addr(&s.empty[pipe.stage]), 3);
@@ -610,52 +624,6 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
 // ---------------------------------------------------------------- copy and small kernels
 
 constexpr int kWarps = 8;
-
-// Batched transpose of bf16 [G][R][Ccols] into [G][Ccols][Rp]: dst[g][c][r] = src[g][r][c] for
-// r < valid(g), 0 for valid(g) <= r < fill(g), nothing written past fill(g). valid(g) = R and
-// fill(g) = R without `valid_rows`; with it valid(g) = valid_rows[g] and fill(g) = valid(g)
-// rounded up to 64. A block moves one 64 x 64 tile through shared memory; Ccols, R (without
-// valid_rows) and Rp are multiples of 64. Two tensors can share the launch (blockIdx.z >= G
-// picks the second pair).
-struct TransposeArgs {
-  const uint16_t* src[2];
-  uint16_t* dst[2];
-  int G, R, Ccols, Rp;
-  const int32_t* valid_rows;   // [G] or null
-};
-
-__global__ void __launch_bounds__(256) transpose_kernel(const TransposeArgs a) {
-  __shared__ uint16_t tile[64][66];
-  grid_dependency_wait();
-  const int which = blockIdx.z >= a.G ? 1 : 0;
-  const int g = blockIdx.z - which * a.G;
-  const int c0 = blockIdx.x * 64, r0 = blockIdx.y * 64;
-  const int valid = a.valid_rows ? a.valid_rows[g] : a.R;
-  const int fill = a.valid_rows ? (valid + 63) / 64 * 64 : a.R;
-  if (r0 < fill) {
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
-    const uint16_t* src = (which ? a.src[1] : a.src[0]) + static_cast<size_t>(g) * a.R * a.Ccols;
-    uint16_t* dst = (which ? a.dst[1] : a.dst[0]) + static_cast<size_t>(g) * a.Ccols * a.Rp;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int rr = ty + 8 * i;
-      const int r = r0 + rr;
-      uint32_t v = 0;
-      if (r < valid) v = *reinterpret_cast<const uint32_t*>(src + static_cast<size_t>(r) * a.Ccols + c0 + 2 * tx);
-      tile[rr][2 * tx] = static_cast<uint16_t>(v & 0xFFFFu);
-      tile[rr][2 * tx + 1] = static_cast<uint16_t>(v >> 16);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int cc = ty + 8 * i;
-      const uint32_t v = static_cast<uint32_t>(tile[2 * tx][cc]) | (static_cast<uint32_t>(tile[2 * tx + 1][cc]) << 16);
-      *reinterpret_cast<uint32_t*>(dst + static_cast<size_t>(c0 + cc) * a.Rp + r0 + 2 * tx) = v;
-    }
-  }
-  pdl_trigger_early();
-  pdl_trigger_late();
-}
 
 // Dispatch and transpose of round r in one pass. A block takes 64 rows of one expert's rows in
 // the round and 64 columns (c0 = 64 * blockIdx.y): the rows' tokens come from the round-major row
@@ -1031,17 +999,6 @@ cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_h
     if ((e = cudaMemsetAsync(a.dw_gate_up + x * per13, 0, per13 * 4, stream)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(a.dw_down + x * per2, 0, per2 * 4, stream)) != cudaSuccess) return e;
   }
-  // W2 [E][d][F] -> W2^T [E][F][d]; W13 [E][2F][d] -> W13^T [E][d][2F]
-  bwd::TransposeArgs t1{{a.w_down, nullptr}, {a.w2t, nullptr}, E, d, F, d, nullptr};
-  launch_begin(kKindBackwardCopy, stream);
-  e = launch_pdl(bwd::transpose_kernel, dim3(F / 64, d / 64, E), dim3(256), 0, stream, t1);
-  launch_end(kKindBackwardCopy, stream);
-  if (e != cudaSuccess) return e;
-  bwd::TransposeArgs t2{{a.w_gate_up, nullptr}, {a.w13t, nullptr}, E, 2 * F, d, 2 * F, nullptr};
-  launch_begin(kKindBackwardCopy, stream);
-  e = launch_pdl(bwd::transpose_kernel, dim3(d / 64, 2 * F / 64, E), dim3(256), 0, stream, t2);
-  launch_end(kKindBackwardCopy, stream);
-  if (e != cudaSuccess) return e;
   const long long pairs = static_cast<long long>(a.T) * a.k;
   if (pairs > 0) {
     launch_begin(kKindBackwardCopy, stream);
@@ -1136,8 +1093,8 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g.dgate_ld = F / 64;
     CUtensorMap ma, mb;
     if ((e = gemm::make_map(&ma, a.dybuf, d, a_rows, groups, gemm::BM)) != cudaSuccess) return e;
-    if ((e = gemm::make_map(&mb, a.w2t, d, F, E, pair ? pair_box : static_cast<uint32_t>(g.width))) != cudaSuccess)
-      return e;
+    g.b_mn = 1;   // B[n = column of d_ff][k = column of d] = W2[k][n]: W2 as stored, MN-major
+    if ((e = gemm::make_map(&mb, a.w_down, F, d, E, bwd::kMnBox, bwd::kMnBox)) != cudaSuccess) return e;
     if ((e = run_gemm(&ma, &mb, &g, 1, mt * parts, kKindBackwardDh, stream, nullptr, pair)) != cudaSuccess) return e;
   }
   // one launch: dx rows = dab W13, dW2 (+)= dyT hgT^T, dW13 (+)= dabT xT^T (K = the round's rows)
@@ -1155,9 +1112,8 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g[0].out = a.dxbuf;
     g[0].out_ld = d;
     if ((e = gemm::make_map(&ma[0], a.dab, 2ull * F, a_rows, groups, gemm::BM)) != cudaSuccess) return e;
-    if ((e = gemm::make_map(&mb[0], a.w13t, 2ull * F, d, E, pair ? pair_box : static_cast<uint32_t>(g[0].width))) !=
-        cudaSuccess)
-      return e;
+    g[0].b_mn = 1;   // B[n = column of d][k = row of W13] = W13[k][n]: W13 as stored, MN-major
+    if ((e = gemm::make_map(&mb[0], a.w_gate_up, d, 2ull * F, E, bwd::kMnBox, bwd::kMnBox)) != cudaSuccess) return e;
     tiles += mt * (d / g[0].width);
     const long long mt_w2 = static_cast<long long>(active) * ((d + gemm::BM - 1) / gemm::BM);
     const long long mt_w13 = static_cast<long long>(active) * ((2 * F + gemm::BM - 1) / gemm::BM);

@@ -52,8 +52,6 @@ struct BackwardArgs {
   uint16_t* dxbuf;            // [E * C, d]
   float* dgate;               // [T, k]
   float* ones;                // [T, k]
-  uint16_t* w2t;              // [E, F, d]
-  uint16_t* w13t;             // [E, d, 2F]
   int32_t* status;
   int T, k, E, C, d, F, renorm;
   int pooled;                 // capacity borrowing: pooled round rows (see the plan's row_off)

@@ -416,8 +416,6 @@ void make_backward_layout(const moe_shape_t* s, moe_backward_layout_t* L) {
   L->dxbuf = take(E * C * d * 2);
   L->dgate = take(T * k * 4);
   L->ones = take(T * k * 4);
-  L->w2t = take(E * F * d * 2);
-  L->w13t = take(E * d * 2 * F * 2);
   L->total_bytes = off;
   L->cpad = static_cast<int32_t>(t_ld);
 }
@@ -501,8 +499,6 @@ int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws
   a.dxbuf = at<uint16_t>(bws, B.dxbuf);
   a.dgate = at<float>(bws, B.dgate);
   a.ones = at<float>(bws, B.ones);
-  a.w2t = at<uint16_t>(bws, B.w2t);
-  a.w13t = at<uint16_t>(bws, B.w13t);
   a.status = at<int32_t>(ws, L.header) + kHdrStatus;
   a.T = shape->T;
   a.k = shape->k;

@@ -223,6 +223,22 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   return desc;
 }
 
+// The same for an MN-major bf16 tile (the operand's M or N index contiguous in memory), as TMA
+// writes it from a [K rows][MN] tensor with 64 x 64 boxes and the 128-byte swizzle: each box is
+// 64 K rows of 64 MN elements (128 B), 8-row swizzle atoms 1024 B apart; boxes along MN are
+// `mn_stride` bytes apart. Fields: leading byte offset = the stride between 64-element MN
+// blocks, stride byte offset = the stride between 8-row K groups (1024 B). One K step of 16
+// rows advances the start address by 2048 B.
+__device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr, uint32_t mn_stride) {
+  uint64_t desc = 0;
+  desc |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  desc |= static_cast<uint64_t>((mn_stride >> 4) & 0x3FFFu) << 16;
+  desc |= static_cast<uint64_t>(1024u >> 4) << 32;
+  desc |= static_cast<uint64_t>(1u) << 46;
+  desc |= static_cast<uint64_t>(2u) << 61;
+  return desc;
+}
+
 // Instruction descriptor of kind::f16 with bf16 A and B, fp32 D, both K-major:
 // D format (bits 4-5) = 1 (f32), A format (bits 7-9) = 1 (bf16), B format
 // (bits 10-12) = 1 (bf16), N >> 3 (bits 17-22), M >> 4 (bits 24-28).
@@ -230,6 +246,9 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
+
+// The same with an MN-major B operand (transpose-B bit 16).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) { return idesc_bf16_f32(M, N) | (1u << 16); }
 
 // ---------------------------------------------------------------- CTA pairs (cta_group::2)
 //

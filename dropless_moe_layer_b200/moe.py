@@ -54,7 +54,7 @@ class WorkspaceLayout(ctypes.Structure):
 class BackwardLayout(ctypes.Structure):
     _fields_ = [(name, c_sz) for name in (
         "total_bytes", "xbuf", "dybuf", "row_gate", "xt", "dyt", "ab", "hgt", "dab", "dabt",
-        "dgate_part", "dxbuf", "dgate", "ones", "w2t", "w13t")
+        "dgate_part", "dxbuf", "dgate", "ones")
     ] + [("cpad", c_i32)]
 
 

@@ -235,8 +235,9 @@ MOE_API int moe_round_combine(const moe_shape_t* shape, const moe_plan_info_t* i
  * dy rows, recomputes the SwiGLU pre-activations on the tensor cores, and adds the round's
  * weight gradients into the caller's fp32 gradients; nothing it holds grows with the routing.
  *
- * Its own workspace `bws` (device, caller-owned, 256-byte aligned) holds the per-round buffers
- * and transposed copies of the weights; its size depends on the shape only. */
+ * Its own workspace `bws` (device, caller-owned, 256-byte aligned) holds the per-round buffers;
+ * its size depends on the shape only. The weights are read as they are stored (the GEMMs that
+ * need them transposed load them MN-major). */
 typedef struct moe_backward_layout {
   size_t total_bytes;
   size_t xbuf;        /* bf16 [E * C, d]     the round's x rows */
@@ -253,8 +254,6 @@ typedef struct moe_backward_layout {
   size_t dxbuf;       /* bf16 [E * C, d]     per-pair dx rows of the round */
   size_t dgate;       /* f32  [T, k]         dL/dgate */
   size_t ones;        /* f32  [T, k]         unit gates of the dx combine */
-  size_t w2t;         /* bf16 [E, d_ff, d]   W2 transposed */
-  size_t w13t;        /* bf16 [E, d, 2 d_ff] W13 transposed */
   int32_t cpad;       /* elements per row of the transposed buffers: C rounded up to 128 (one
                          buffer per expert); with MOE_FLAG_BORROW, E * C + 64 * E rounded up to
                          128 (one pooled buffer, every expert's rows rounded up to 64) */
