@@ -167,6 +167,11 @@ struct Phase {
   // Weights of group g: expert group_expert[g] of the B map (expert parallelism: a group is one
   // source rank's rows of one local expert). Null: expert g.
   const int32_t* group_expert;
+  // CTA-pair form: a group's last row block of at most 128 rows runs as half-height tiles (M =
+  // 128; see run_phase_pair), read through these two maps with 64-row boxes: the A operand's,
+  // and (SwiGLU) the weights'. Null: 256-row tiles throughout.
+  const CUtensorMap* a_rows64;
+  const CUtensorMap* b_rows64;
 };
 
 __device__ __forceinline__ int group_weights(const Phase& p, int g) { return p.group_expert ? p.group_expert[g] : g; }
@@ -497,6 +502,26 @@ constexpr int kPairStages = kRingBytes / kPairStageBytes;        // 6
 static_assert(kPairStages <= kMaxStages, "pair ring stages");
 constexpr int kEpiWarpsPair = 8;         // arrivals on the leader's tempty per tile
 
+// Half-height tiles. A group's last row block with at most 128 rows (an expert's leftover rows,
+// common in a round that holds every expert) would leave at least half of a 256-row tile as
+// padding. It runs instead as M = 128 tiles of the same columns: CTA c loads 64 A rows [64 c,
+// 64 c + 64) of the block and the same 128 B rows as in a full tile, except that for SwiGLU CTA c
+// takes W1 rows [64 c, 64 c + 64) of the tile's 128 gate columns and the same W3 rows (64-row
+// boxes). In this shape the accumulator of each CTA holds its 64 rows twice over the TMEM lanes:
+// lanes [0, 64) take the MMA's columns [0, 128) (CTA 0's B rows), lanes [64, 128) columns
+// [128, 256) (CTA 1's), each at TMEM columns [0, 128). So epilogue warp q handles rows
+// 32 (q & 1) .. + 32 of the CTA's 64 and the B half q >> 1: SwiGLU gate columns at [0, 64) and
+// up at [64, 128) for the 64 gate columns 64 c' (c' = q >> 1) of the tile; Bf16Out the tile's
+// columns 128 (q >> 1) .. + 128. Half the MMA work of a padded 256-row tile, the same weights.
+constexpr int kHalfRows = BM / 2;        // A rows per CTA in a half-height tile
+constexpr int kHalfStageBytes = kHalfRows * BK * 2 + kPairBHalf * BK * 2;   // 24 KB per CTA
+
+// Whether row block mp of a group with `rows` rows is its short last block (half-height tiles).
+__device__ __forceinline__ bool half_block(const Phase& p, int rows, int mp) {
+  const int tail = rows - mp * kPairRows;
+  return p.a_rows64 != nullptr && tail > 0 && tail <= BM;
+}
+
 // Set-up of both CTAs of a pair: barriers (thread 0 of each), the pair's TMEM (warp 1 of each),
 // then a cluster barrier, so that no CTA signals its peer before the peer's barriers exist.
 __device__ __forceinline__ uint32_t setup_pair(const Smem& s) {
@@ -592,12 +617,15 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer (both CTAs)
-    const uint32_t tx = 2u * kPairStageBytes;   // the pair's bytes per stage, counted by the leader
     bool ok = true;
     for (int tile = pair; ok && tile < total; tile += pairs) {
       int g, mp, nt;
       decode(tile, g, mp, nt);
-      int a_row = mp * kPairRows + static_cast<int>(cta) * BM, a_grp = g;   // this CTA's first A row
+      const bool half = half_block(p, group_rows(p, g), mp);
+      // the pair's bytes per stage, counted by the leader
+      const uint32_t tx = 2u * (half ? kHalfStageBytes : kPairStageBytes);
+      // this CTA's first A row
+      int a_row = mp * kPairRows + static_cast<int>(cta) * (half ? kHalfRows : BM), a_grp = g;
       if (p.group_row) {
         a_row += p.group_row[g] - *p.group_row_base;
         a_grp = 0;
@@ -614,8 +642,20 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
         if (cta == 0 && lane == 0) mbar_arrive_expect_tx(fb_local, tx);
         __syncwarp();
         if (lane == 0) {
-          tma_load_3d_pair(sA, p.a, fb, kb * BK, a_row, a_grp);
-          tma_load_3d_pair(sB, p.b[0], fb, kb * BK, b_row(nt), group_weights(p, g));
+          if (!half) {
+            tma_load_3d_pair(sA, p.a, fb, kb * BK, a_row, a_grp);
+            tma_load_3d_pair(sB, p.b[0], fb, kb * BK, b_row(nt), group_weights(p, g));
+          } else {
+            tma_load_3d_pair(sA, p.a_rows64, fb, kb * BK, a_row, a_grp);
+            if (p.mode == kSwiGLU) {   // 64 W1 rows, then the same 64 W3 rows
+              const int w1 = nt * width + static_cast<int>(cta) * kHalfRows;
+              tma_load_3d_pair(sB, p.b_rows64, fb, kb * BK, w1, group_weights(p, g));
+              tma_load_3d_pair(sB + kHalfRows * BK * 2, p.b_rows64, fb, kb * BK, p.b_second_row + w1,
+                               group_weights(p, g));
+            } else {
+              tma_load_3d_pair(sB, p.b[0], fb, kb * BK, b_row(nt), group_weights(p, g));
+            }
+          }
         }
         pipe.issued |= 1u << pipe.stage;
         if (++pipe.stage == kPairStages) {
@@ -637,9 +677,11 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
   } else if (warp == 1) {
     if (lane == 0 && cta == 0) {
     // ---------------------------------------------------------------- MMA issuer (leader only)
-    const uint32_t idesc = idesc_bf16_f32(kPairRows, kPairBn);
     bool ok = true;
     for (int tile = pair; ok && tile < total; tile += pairs) {
+      int g, mp, nt;
+      decode(tile, g, mp, nt);
+      const uint32_t idesc = idesc_bf16_f32(half_block(p, group_rows(p, g), mp) ? BM : kPairRows, kPairBn);
       if (!mbar_wait(smem_addr(&s.tempty[pipe.acc]), pipe.acc_phase ^ 1u, s.abort)) {
         ok = false;
         break;
@@ -694,27 +736,35 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
         break;
       }
       tc_fence_after();
-      const int row = mp * kPairRows + static_cast<int>(cta) * BM + q * 32 + lane;
       const int rows_g = group_rows(p, g);
+      const bool half = half_block(p, rows_g, mp);
+      // this warp's first row, and the output columns it holds (from TMEM column 0 on): a full
+      // tile's warp q has rows 32 q .. of the CTA's 128 and all the tile's columns; a half-height
+      // tile's has rows 32 (q & 1) .. of the CTA's 64 and the columns of B half q >> 1
+      const int row_base = mp * kPairRows + (half ? static_cast<int>(cta) * kHalfRows + (q & 1) * 32
+                                                  : static_cast<int>(cta) * BM + q * 32);
+      const int row = row_base + lane;
       const bool valid = row < rows_g;
+      const int out_cols = (p.mode == kSwiGLU ? width : kPairBn) / (half ? 2 : 1);
+      const int col0 = nt * width + (half ? (q >> 1) * out_cols : 0);
+      const int up_off = out_cols;   // SwiGLU: TMEM offset of the up columns
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(pipe.acc * kAccCols);
       const long long orow_off = p.group_row
                                      ? static_cast<long long>(p.group_row[g] - *p.group_row_base + row) * p.out_ld
                                      : g * p.out_group_stride + static_cast<long long>(row) * p.out_ld;
-      uint16_t* orow = static_cast<uint16_t*>(p.out) + orow_off + nt * width;
+      uint16_t* orow = static_cast<uint16_t*>(p.out) + orow_off + col0;
       if (p.out_map != nullptr) {
         // 32-column chunks: TMEM -> registers -> this warp's staging buffer -> one bulk store of
         // its 32 rows. Rows of the box past the group's rows hold junk; they fall in the expert's
         // unused rows [n, C) (never read) or past C (clipped by the map).
-        const int row_base = mp * kPairRows + static_cast<int>(cta) * BM + q * 32;
-        const int chunks = (p.mode == kSwiGLU ? width : kPairBn) / kOutChunkCols;
+        const int chunks = out_cols / kOutChunkCols;
         for (int c = 0; c < chunks; ++c) {
           uint32_t pk[16];
           if (p.mode == kSwiGLU) {
             uint32_t gv[32], uv[32];
             tmem_ld32(tb + c * kOutChunkCols, gv);
-            tmem_ld32(tb + width + c * kOutChunkCols, uv);
+            tmem_ld32(tb + up_off + c * kOutChunkCols, uv);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -738,15 +788,15 @@ __device__ __forceinline__ void run_phase_pair(const Smem& s, uint32_t tmem_base
           fence_async_shared();
           __syncwarp();
           if (lane == 0) {
-            tma_store_3d(p.out_map, stage0 + buf_off, nt * width + c * kOutChunkCols, row_base, g, out_policy);
+            tma_store_3d(p.out_map, stage0 + buf_off, col0 + c * kOutChunkCols, row_base, g, out_policy);
             bulk_commit();
           }
           ++ochunk;
         }
       } else if (p.mode == kSwiGLU) {
-        store_swiglu(tb, width, orow, valid);
+        store_swiglu(tb, out_cols, orow, valid);
       } else {
-        store_bf16(tb, kPairBn, orow, valid);
+        store_bf16(tb, out_cols, orow, valid);
       }
       tc_fence_before();
       __syncwarp();

@@ -93,6 +93,7 @@ struct KernelArgs {
   int rows_cap;                    // debug bounds checks (see Phase): 0 = unchecked
   int tma_out;                     // CTA-pair form: store through the output map (see Phase)
   const int32_t* group_expert;     // weights of each group (see Phase), or null
+  int half_tiles;                  // CTA-pair form: half-height tiles for short last row blocks
 };
 
 __global__ void __launch_bounds__(kLaunchThreads, 1)
@@ -131,6 +132,8 @@ __global__ void __launch_bounds__(kLaunchThreads, 1)
   p.dbg = args.rows_cap > 0 ? args.status - kHdrStatus : nullptr;
   p.out_map = nullptr;
   p.group_expert = args.group_expert;
+  p.a_rows64 = nullptr;
+  p.b_rows64 = nullptr;
   plan_phase(s, p, 0);              // reads only the row counts (plan data)
   __syncthreads();
   // Everything above overlaps the previous kernel; the operands, and the output buffer that
@@ -152,7 +155,8 @@ __global__ void __launch_bounds__(kLaunchThreads, 1)
 // 256 tiles, one B map with 128-row boxes, a fixed width (SwiGLU 128 gate columns, Bf16Out 256).
 __global__ void __launch_bounds__(kLaunchThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
-                             const __grid_constant__ CUtensorMap tout, const KernelArgs args, const SideArgs side,
+                             const __grid_constant__ CUtensorMap tout, const __grid_constant__ CUtensorMap ta64,
+                             const __grid_constant__ CUtensorMap tb64, const KernelArgs args, const SideArgs side,
                              int width) {
   extern __shared__ uint8_t smem_raw[];
   const Smem s = carve(smem_raw);
@@ -187,6 +191,8 @@ __global__ void __launch_bounds__(kLaunchThreads, 1)
   p.dbg = args.rows_cap > 0 ? args.status - kHdrStatus : nullptr;
   p.out_map = args.tma_out ? &tout : nullptr;
   p.group_expert = args.group_expert;
+  p.a_rows64 = args.half_tiles ? &ta64 : nullptr;
+  p.b_rows64 = args.half_tiles ? &tb64 : nullptr;
   plan_phase_pair(s, p, 0, width);
   __syncthreads();
   grid_dependency_wait();
@@ -410,14 +416,21 @@ static int pair_clusters() {
   return n;
 }
 
-// Whether a round's GEMM runs in the CTA-pair form: its 256-row tiles must keep every cluster
-// busy and pad at most kPairPadding more rows than the 128-row tiles of the single-CTA form.
+#ifndef MOE_GEMM_HALF
+#define MOE_GEMM_HALF 1   // 0: no half-height tiles; a short last row block takes a 256-row tile
+#endif
+
+// Whether a round's GEMM runs in the CTA-pair form: its tiles must keep every cluster busy and
+// cover at most 15 % more rows than the 128-row tiles of the single-CTA form (a short last row
+// block, at most 128 rows, costs 128 rows with half-height tiles, else 256).
 static bool use_pair(const int32_t* n_host, int groups, int n_total, int width) {
   if (!MOE_GEMM_PAIR || n_host == nullptr || n_total % width != 0) return false;
   long long pair_tiles = 0, rows_pair = 0, rows_single = 0;
   for (int g = 0; g < groups; ++g) {
-    pair_tiles += (n_host[g] + kPairRows - 1) / kPairRows;
-    rows_pair += static_cast<long long>((n_host[g] + kPairRows - 1) / kPairRows) * kPairRows;
+    const long long blocks = (n_host[g] + kPairRows - 1) / kPairRows;
+    const long long tail = n_host[g] - (blocks - 1) * kPairRows;
+    pair_tiles += blocks;
+    rows_pair += blocks * kPairRows - ((MOE_GEMM_HALF && blocks > 0 && tail <= BM) ? BM : 0);
     rows_single += static_cast<long long>((n_host[g] + BM - 1) / BM) * BM;
   }
   pair_tiles *= n_total / width;
@@ -425,8 +438,12 @@ static bool use_pair(const int32_t* n_host, int groups, int n_total, int width) 
   return clusters > 0 && pair_tiles >= clusters && rows_pair * 100 <= rows_single * 115;
 }
 
-static cudaError_t run_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& out,
-                            const KernelArgs& args, int width, const SideArgs& side, int kind, cudaStream_t stream) {
+// a64, b64: the A operand's and the weights' maps with 64-row boxes (half-height tiles; b64 is
+// read for SwiGLU only).
+static cudaError_t run_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& out, const CUtensorMap& a64,
+                            const CUtensorMap& b64, KernelArgs args, int width, const SideArgs& side, int kind,
+                            cudaStream_t stream) {
+  args.half_tiles = MOE_GEMM_HALF;
   const int clusters = pair_clusters();   // every cluster takes part; the device counts the tiles
   launch_begin(kind, stream);
   cudaLaunchConfig_t cfg = {};
@@ -443,7 +460,7 @@ static cudaError_t run_pair(const CUtensorMap& a, const CUtensorMap& b, const CU
   attr[1].val.programmaticStreamSerializationAllowed = MOE_PDL;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  const cudaError_t err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel, a, b, out, args, side, width);
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel, a, b, out, a64, b64, args, side, width);
   launch_end(kind, stream);
   return err;
 }
@@ -460,6 +477,12 @@ cudaError_t make_gate_up_maps(const uint16_t* buf, const uint16_t* w_gate_up, in
                          : gemm::make_map(ma, buf, d, C, E, gemm::BM);
   if (e != cudaSuccess) return e;
   return gemm::make_b_maps(mb, w_gate_up, d, 2ull * F, E, kGateUpWidths, F);
+}
+
+// A round buffer ([E][C][inner] per expert, or pooled [1][E*C][inner]) with 64-row boxes.
+static cudaError_t make_rows64_map(CUtensorMap* m, const uint16_t* rows, int inner, int E, int C, bool pooled) {
+  return pooled ? gemm::make_map(m, rows, inner, static_cast<uint64_t>(E) * C, 1, gemm::kHalfRows)
+                : gemm::make_map(m, rows, inner, C, E, gemm::kHalfRows);
 }
 
 cudaError_t make_down_maps(const uint16_t* h, const uint16_t* w_down, int E, int C, int d, int F,
@@ -519,7 +542,11 @@ cudaError_t launch_gate_up(const uint16_t* buf, const uint16_t* w_gate_up, uint1
     CUtensorMap mo{};
     a.tma_out = MOE_TMA_OUT_GATE_UP && group_row == nullptr;   // per-expert h [E][C][F]: stored by TMA
     if (a.tma_out && (e = gemm::make_map(&mo, h, F, C, E, 32, gemm::kOutChunkCols)) != cudaSuccess) return e;
-    return gemm::run_pair(ma, mb[0], mo, a, 128, make_side(copy), kKindGateUp, stream);
+    CUtensorMap ma64, mb64;   // 64-row boxes of the rows and of W1 / W3 (half-height tiles)
+    if ((e = make_rows64_map(&ma64, buf, d, E, C, group_row != nullptr)) != cudaSuccess ||
+        (e = gemm::make_map(&mb64, w_gate_up, d, 2ull * F, E, gemm::kHalfRows)) != cudaSuccess)
+      return e;
+    return gemm::run_pair(ma, mb[0], mo, ma64, mb64, a, 128, make_side(copy), kKindGateUp, stream);
   }
   const long long tiles = gemm::choose_width(n_host, E, 0, F, a);
   return gemm::run(ma, mb, a, tiles, make_side(copy), kKindGateUp, stream);
@@ -551,7 +578,9 @@ cudaError_t launch_down(const uint16_t* h, const uint16_t* w_down, uint16_t* out
     if ((e = gemm::make_map(&mb_half, w_down, F, d, E, gemm::kPairBHalf)) != cudaSuccess) return e;
     a.tma_out = group_row == nullptr;          // per-expert out [E][C][d]: stored by TMA
     if (a.tma_out && (e = gemm::make_map(&mo, out, d, C, E, 32, gemm::kOutChunkCols)) != cudaSuccess) return e;
-    return gemm::run_pair(ma, mb_half, mo, a, gemm::kPairBn, make_side(copy), kKindDown, stream);
+    CUtensorMap ma64;   // 64-row boxes of h (half-height tiles)
+    if ((e = make_rows64_map(&ma64, h, F, E, C, group_row != nullptr)) != cudaSuccess) return e;
+    return gemm::run_pair(ma, mb_half, mo, ma64, mb_half, a, gemm::kPairBn, make_side(copy), kKindDown, stream);
   }
   const long long tiles = gemm::choose_width(n_host, E, 0, d, a);
   return gemm::run(ma, mb, a, tiles, make_side(copy), kKindDown, stream);
@@ -582,8 +611,11 @@ cudaError_t launch_ep_experts(const uint16_t* recv, const uint16_t* w_gate_up, c
   a.group_expert = group_expert_dev;
   const gemm::SideArgs none = make_side(nullptr);
   if (gemm::use_pair(rows_host, groups, F, 128)) {
-    CUtensorMap unused{};
-    e = gemm::run_pair(ma, mb[0], unused, a, 128, none, kKindGateUp, stream);
+    CUtensorMap unused{}, ma64, mb64;
+    if ((e = gemm::make_map(&ma64, recv, d, static_cast<uint64_t>(buf_rows), 1, gemm::kHalfRows)) != cudaSuccess ||
+        (e = gemm::make_map(&mb64, w_gate_up, d, 2ull * F, E_local, gemm::kHalfRows)) != cudaSuccess)
+      return e;
+    e = gemm::run_pair(ma, mb[0], unused, ma64, mb64, a, 128, none, kKindGateUp, stream);
   } else {
     const long long tiles = gemm::choose_width(rows_host, groups, 0, F, a);
     e = gemm::run(ma, mb, a, tiles, none, kKindGateUp, stream);
@@ -607,7 +639,9 @@ cudaError_t launch_ep_experts(const uint16_t* recv, const uint16_t* w_gate_up, c
   if (gemm::use_pair(rows_host, groups, d, gemm::kPairBn)) {
     CUtensorMap mb_half, unused{};
     if ((e = gemm::make_map(&mb_half, w_down, F, d, E_local, gemm::kPairBHalf)) != cudaSuccess) return e;
-    return gemm::run_pair(ma, mb_half, unused, b, gemm::kPairBn, none, kKindDown, stream);
+    CUtensorMap ma64;
+    if ((e = gemm::make_map(&ma64, h, F, static_cast<uint64_t>(buf_rows), 1, gemm::kHalfRows)) != cudaSuccess) return e;
+    return gemm::run_pair(ma, mb_half, unused, ma64, mb_half, b, gemm::kPairBn, none, kKindDown, stream);
   }
   if ((e = gemm::make_b_maps(mb, w_down, F, d, E_local, kDownWidths, d)) != cudaSuccess) return e;
   const long long tiles = gemm::choose_width(rows_host, groups, 0, d, b);
