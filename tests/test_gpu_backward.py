@@ -158,25 +158,58 @@ def test_backward_pair_form_full_parity(borrow):
         assert torch.equal(g[n], g2[n]), n
 
 
-def test_backward_16k_uniform_sampled_parity():
-    """The benchmark's backward workload at full size, in the launch configuration it times:
-    dx, dgate and dz of sampled tokens and the weight gradients of the experts with the most and
-    the fewest pairs against the oracle's entries (each token's and each expert's pairs alone)."""
-    w = wl.BY_NAME["16k-uniform"]
+class _LazyExperts:
+    """Expert weights fetched from the GPU one expert at a time, as bf16 bits."""
+
+    def __init__(self, t):
+        self.t = t
+        self.shape = tuple(t.shape)
+
+    def __getitem__(self, e):
+        return wl.bf16_bits(self.t[e])
+
+
+def _sampled_backward_check(w, pick_experts):
+    """Full-size backward on the GPU; dx and dz of 16 sampled tokens and the weight gradients of
+    the experts `pick_experts(load)` names, against the oracle's entries (each token's and each
+    expert's pairs alone)."""
     inp = wl.generate(w, "cuda")
     dy = wl.generate_dy(w, "cuda")
-    layer, g = run_backward(w, inp, dy)
+    if w.router == "gemm":
+        layer = moe.DroplessMoE(w.T, w.d, w.E, w.k, w.F, w.C)
+        layer(inp["x"], inp["w_gate_up"], inp["w_down"], w_router=inp["w_router"], bias=inp["bias"])
+        g = layer.backward(inp["x"], inp["w_gate_up"], inp["w_down"], dy)
+        torch.cuda.synchronize()
+        assert layer.device_status() == 0
+        z = layer.plan_tensors()["logits"].cpu().numpy()     # the logits the GPU routed on
+    else:
+        layer, g = run_backward(w, inp, dy)
+        z = inp["logits"].cpu().numpy()
     assert layer.info.R >= 2
-    z = inp["logits"].cpu().numpy()
     idx = oracle.select_topk(z, w.k)
     load = np.bincount(idx.ravel(), minlength=w.E)
-    experts = [int(np.argmax(load)), int(np.argmin(load))]
+    experts = pick_experts(load)
     rng = np.random.default_rng(0)
     tokens = np.concatenate([[0, w.T - 1], rng.choice(w.T, 14, replace=False)])
-    ref = oracle.backward_sampled(wl.bf16_bits(inp["x"]), wl.bf16_bits(inp["w_gate_up"]),
-                                  wl.bf16_bits(inp["w_down"]), z, idx, dy.cpu().numpy().astype(np.float64),
+    ref = oracle.backward_sampled(wl.bf16_bits(inp["x"]), _LazyExperts(inp["w_gate_up"]),
+                                  _LazyExperts(inp["w_down"]), z, idx, dy.cpu().numpy().astype(np.float64),
                                   tokens, experts)
     got = {"dx": g["dx"][tokens], "dz": g["dz"][tokens],
            "dw_gate_up": g["dw_gate_up"][experts], "dw_down": g["dw_down"][experts]}
     errs = {n: rel_err(got[n].cpu().numpy().astype(np.float64), ref[n]) for n in got}
     assert all(e <= G_TOL for e in errs.values()), errs
+
+
+def test_backward_16k_uniform_sampled_parity():
+    """16k-uniform at full size: the experts with the most and the fewest pairs."""
+    _sampled_backward_check(wl.BY_NAME["16k-uniform"], lambda load: [int(np.argmax(load)), int(np.argmin(load))])
+
+
+def test_backward_32k_sampled_parity():
+    """The bench's default workload at full size (router-GEMM logits, 16 rounds, round 0 in the
+    pair form with most experts' rows in one short block): the experts with the fewest pairs and
+    with the median count (the hottest expert's 32k rows would take the float64 oracle minutes)."""
+    def pick(load):
+        order = np.argsort(load, kind="stable")
+        return [int(order[0]), int(order[len(order) // 2])]
+    _sampled_backward_check(wl.BY_NAME["32k-zipf1.2-router-gemm"], pick)
