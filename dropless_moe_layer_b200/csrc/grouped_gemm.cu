@@ -152,7 +152,9 @@ __global__ void __launch_bounds__(kLaunchThreads, 1)
 }
 
 // The CTA-pair form (gemm_sm100.cuh, run_phase_pair), launched as clusters of two CTAs: 256 x
-// 256 tiles, one B map with 128-row boxes, a fixed width (SwiGLU 128 gate columns, Bf16Out 256).
+// 256 tiles, one B map with 128-row boxes, a fixed width (SwiGLU 128 gate columns, Bf16Out 256);
+// ta64 / tb64 are the A operand and the weights with 64-row boxes, read by the half-height tiles
+// of a group's short last row block (tb64 by SwiGLU only).
 __global__ void __launch_bounds__(kLaunchThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
                              const __grid_constant__ CUtensorMap tout, const __grid_constant__ CUtensorMap ta64,
