@@ -414,6 +414,42 @@ def backward_flops(w):
     return 16 * w.T * w.k * w.d * w.F
 
 
+def backward_roofline_s(w, info, round_np, peaks, tensor_tflops, n_plan=None):
+    """Lower bound on one backward pass from its algorithmic work, per round and launch kind
+    the larger of its tensor-core time and its DRAM time (the copies at the DRAM peak alone).
+    Bytes counted: the round's x and dy rows read once and kept as bf16 rows, the expert
+    weights each GEMM reads once per active expert, the recomputed a, b and gate*h written once
+    and read where used, [da | db] likewise, the per-pair dx rows, every token's dx read-add-write
+    in each round it has pairs in, and the fp32 weight gradients stored (round 0) or
+    read-added (later rounds) per active expert. The transposed copies the kernels make are
+    not counted: they are this implementation's choice, not the method's. Returns (seconds,
+    parts)."""
+    n = round_rows(w, info, n_plan)
+    d, F = w.d, w.F
+    bw = peaks["hbm_gbs"] * 1e9
+    pt = tensor_tflops * 1e12
+    parts = {"recompute": 0.0, "dh": 0.0, "dx_wgrad": 0.0, "copies": 0.0}
+    rnd = np.asarray(round_np)
+    for r in range(n.shape[0]):
+        P = int(n[r].sum())
+        A = int((n[r] > 0).sum())
+        tokens = int((rnd == r).any(axis=1).sum())
+        first = int(((rnd == r).any(axis=1) & ~(rnd < r).any(axis=1)).sum())   # tokens whose dx starts here
+        w13, w2 = A * 2 * F * d * 2, A * d * F * 2
+        grads = A * 3 * d * F * 4 * (1 if r == 0 else 2)
+        kinds = {
+            "recompute": (4 * P * d * F, P * d * 2 + w13 + P * 2 * F * 2 + P * F * 2),
+            "dh": (2 * P * d * F, P * d * 2 + w2 + P * 2 * F * 2 + P * 2 * F * 2),
+            "dx_wgrad": (10 * P * d * F,
+                         2 * P * 2 * F * 2 + w13 + P * d * 2 + P * F * 2 + P * d * 2 + P * d * 2 + grads),
+        }
+        for k, (fl, by) in kinds.items():
+            parts[k] += max(fl / pt, by / bw)
+        parts["copies"] += (P * d * (2 + 4) + P * d * 4 + P * d * 2 + tokens * d * 8 - first * d * 4) / bw
+    parts["copies"] += (w.T * w.E * 8 + w.T * w.k * 8) / bw      # dz from the logits and dgate
+    return sum(parts.values()), {k: v * 1e3 for k, v in parts.items()}
+
+
 def backward_cpu_baseline(w, budget_s=12.0):
     """The oracle's backward on the host cores, on a seeded token sample (all the sampled tokens'
     pairs), scaled to tokens/s."""
@@ -515,6 +551,8 @@ def bench_backward(args, w):
     tensor_key = "bf16_tflops_sustained" if power_capped and "bf16_tflops_sustained" in peaks else "bf16_tflops"
     peak = peaks[tensor_key]
     ms = total_ms / args.steps
+    pass_s, pass_parts = backward_roofline_s(w, info, layer.plan_tensors()["round"].cpu().numpy(), peaks, peak,
+                                             layer.plan_tensors()["n"].cpu().numpy())
     line = {
         "metric": BWD_METRIC, "pass": "backward", "value": w.T / (ms / 1e3), "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -525,6 +563,11 @@ def bench_backward(args, w):
                      "peak_source": f"{peak_src} ({tensor_key})", "traffic": None,
                      "frac_vs_burst": achieved / peaks["bf16_tflops"], "flops_per_step": flops},
         "whole_pass_tflops": flops / (ms / 1e3) / 1e12,
+        "pass_frac": pass_s * 1e3 / ms,
+        "pass_roofline": {"ms": pass_s * 1e3, **{k + "_ms": round(v, 4) for k, v in pass_parts.items()},
+                          "peaks": f"{peak_src}: hbm_gbs {peaks['hbm_gbs']}, {tensor_key} {peak}",
+                          "formula": "per round and launch kind max(tensor flops at the peak, algorithmic DRAM "
+                                     "bytes at the copy peak); copies at the copy peak"},
         "kernels": {k: dict({"launches": c, "ms": round(t, 4)},
                             **({"TFLOP/s": round(BWD_KIND_FLOPS[k] * w.T * w.k * w.d * w.F / (t / 1e3) / 1e12, 1)}
                                if k in BWD_KIND_FLOPS else {}))

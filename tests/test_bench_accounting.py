@@ -93,3 +93,30 @@ def test_ride_plan_follows_the_size_rule():
     n2[1, :] = w.C
     comb, disp = bench.ride_plan(w, n2, 2)
     assert comb == {0} and disp == set()   # the small round's combine hides under the full round's
+
+
+def test_backward_roofline_counts():
+    """One round, two experts (3 and 1 rows), four tokens each with one pair: the copy part is
+    the gather (x bf16 and dy fp32 read, both written back as bf16 rows), the dx rows read by the
+    combine and each token's first dx write, plus dz from the logits and dgate; with an
+    unbounded tensor peak every GEMM kind is its bytes at the copy peak, and the weight
+    gradients are stored once (round 0)."""
+    w = wl.custom(name="t", T=4, d=64, E=2, k=1, F=64, C=4)
+    info = types.SimpleNamespace(load=[3, 1] + [0] * 254, R=1)
+    rnd = np.zeros((4, 1), dtype=np.int64)
+    n = np.array([[3, 1]])
+    peaks = {"hbm_gbs": 1.0}     # 1 GB/s: seconds = bytes / 1e9
+    s, parts = bench.backward_roofline_s(w, info, rnd, peaks, 1e30, n)
+    P, A, d, F, T, E, k = 4, 2, 64, 64, 4, 2, 1
+    copies = P * d * 6 + P * d * 4 + P * d * 2 + T * d * 4 + T * E * 8 + T * k * 8
+    assert parts["copies"] == pytest.approx(copies / 1e9 * 1e3)
+    grads = A * 3 * d * F * 4
+    assert parts["dx_wgrad"] * 1e6 == pytest.approx(4 * P * 2 * F + A * 2 * F * d * 2 + 3 * P * d * 2 + P * F * 2
+                                                     + grads)
+    assert s * 1e3 == pytest.approx(sum(parts.values()))
+    # a second round holding the same rows again: its gradients are read and written (2x)
+    rnd2 = np.array([[0, 1]] * 4)
+    info2 = types.SimpleNamespace(load=[6, 2] + [0] * 254, R=2)
+    w2 = wl.custom(name="t", T=4, d=64, E=2, k=2, F=64, C=3)
+    _, parts2 = bench.backward_roofline_s(w2, info2, rnd2, peaks, 1e30, np.array([[3, 1], [3, 1]]))
+    assert parts2["dx_wgrad"] - 2 * parts["dx_wgrad"] == pytest.approx(grads / 1e9 * 1e3)
