@@ -421,9 +421,7 @@ def backward_roofline_s(w, info, round_np, peaks, tensor_tflops, n_plan=None):
     weights each GEMM reads once per active expert, the recomputed a, b and gate*h written once
     and read where used, [da | db] likewise, the per-pair dx rows, every token's dx read-add-write
     in each round it has pairs in, and the fp32 weight gradients stored (round 0) or
-    read-added (later rounds) per active expert. The transposed copies the kernels make are
-    not counted: they are this implementation's choice, not the method's. Returns (seconds,
-    parts)."""
+    read-added (later rounds) per active expert. Returns (seconds, parts)."""
     n = round_rows(w, info, n_plan)
     d, F = w.d, w.F
     bw = peaks["hbm_gbs"] * 1e9

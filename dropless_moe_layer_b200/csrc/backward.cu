@@ -13,32 +13,31 @@
 //   dW2_e += (gate dy) h^T = dy (gate h)^T  dW1_e += da x^T, dW3_e += db x^T
 //   dz = softmax Jacobian applied to dgate (renormalised gates: the quotient rule first).
 //
-// Per round r, with the forward's plan (rows of expert e in round r at e * C + slot; with
-// capacity borrowing pooled, at row_off[r][e] - row_start[r] + slot):
-//   gather     x rows -> xbuf, bf16(dy) rows -> dybuf (row-major) and, in the same pass, xT, dyT
-//              (K-major over the round's rows for the weight-gradient GEMMs: [E][d][Cp] with
-//              Cp = C rounded up to 128, or pooled [d][E * C + 64 E rounded up to 128] with each
-//              expert's rows rounded up to 64; zeros past the expert's rows up to the next
-//              multiple of 64); the pair's gate -> row_gate
-//   recompute  [a | b] = xbuf W13^T (tensor cores); epilogue keeps a, b (bf16, row-major) and
-//              writes bf16(gate * h) transposed (hgT, F rows)
+// Per round r, with the forward's plan. The round's rows live in buffers of E * C rows, expert
+// e's at e * C + slot; with capacity borrowing in buffers of E * C + 64 E rows, expert e's at
+// seg_off[r][e] + slot, where each expert's segment starts at a multiple of 64:
+//   gather     x rows -> xbuf, bf16(dy) rows -> dybuf; the pair's gate -> row_gate
+//   recompute  [a | b] = xbuf W13^T (tensor cores); epilogue keeps a, b (bf16) and writes
+//              hg = bf16(gate * h)
 //   dh         W2^T dy as dybuf (W2^T)^T (tensor cores, B = W2 read MN-major as stored);
 //              epilogue: the SwiGLU backward (da, db from a, b and the gate), dgate partial sums
-//              <W2^T dy, h> per 64..256-column tile, dab = [da | db] row-major and transposed
+//              <W2^T dy, h> per 64..256-column tile, dab = [da | db]
 //   dx         dab W13 (tensor cores, B = W13 read MN-major as stored) -> dxbuf (bf16)
 //   combine    dx[t] = (first round of t ? 0 : dx[t]) + sum of the token's dxbuf rows, ascending
 //              j; dgate[t, j] = sum of its row's partials in tile order (no atomics anywhere)
-//   wgrad      dW2 += dyT hgT^T and dW13 += dabT xT^T over K = the round's rows of each expert
-//              (tensor cores; fp32 read-add-write of the caller's gradient, one CTA per tile;
-//              round 0 stores instead: it holds every expert that has rows); one launch with
-//              the dx GEMM, as the three are independent
+//   wgrad      dW2 += dy^T hg and dW13 += dab^T x over K = the round's rows of each expert
+//              (tensor cores, both operands the row-major round buffers read MN-major; the fp32
+//              gradient tiles are stored in round 0, which holds every expert that has rows,
+//              and reduce-added through TMA after); one launch with the dx GEMM, as the three
+//              are independent
 // After the last round: dz from dgate and the logits (one warp per token).
 //
 // Every operand of a tensor-core step is bf16 (fp32 accumulate); a and b are kept as bf16 between
 // the recompute and the dh epilogue. Rows of a tile past the expert's row count never reach a
-// row-major store; in the transposed buffers they are written as zeros up to the next multiple of
-// 64 (and no further: with pooled rows the next expert's rows follow), so the weight-gradient
-// GEMMs may read K in blocks of 64 without a mask.
+// store, except that the rows from the count up to the next multiple of 64 (within the expert's
+// C rows, or its segment) are written as zeros in xbuf, dybuf, hg and dab: the weight-gradient
+// GEMMs read K, the rows, in blocks of 64 without a mask, and with pooled rows the next expert's
+// segment starts right after.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -69,18 +68,15 @@ struct GemmArgs {
   int n_total;                // output columns per expert
   int num_k_blocks;           // K / 64 (all but kWgrad, whose K is the expert's rows)
   int C, F;
-  int t_ld;                   // elements per row of the transposed buffers: C rounded up to 128
-                              // per expert, or the pooled width with capacity borrowing
   // Pooled round rows (capacity borrowing): expert g's rows of the round start at row
-  // group_row[g] - *group_row_base of the E*C-row buffers, and at column seg(g) = sum over
-  // g' < g of rows(g') rounded up to 64 of the single [rows_t][t_ld] transposed buffers. Null:
-  // rows at g * C, transposed buffers per expert ([E][rows_t][t_ld]).
+  // group_row[g] - *group_row_base of the round buffers, a multiple of 64 (the backward's own
+  // segment table). Null: rows at g * C.
   const int32_t* group_row;
   const int32_t* group_row_base;
   void* out;                  // kRecompute: ab; kDh: dab; kDx: dxbuf; kWgrad: the fp32 gradient
   long long out_group_stride; // elements (kWgrad)
   int out_ld;                 // elements (kWgrad, kDx)
-  uint16_t* out_t;            // kRecompute: hgT (F rows); kDh: dabT (2F rows)
+  uint16_t* out_hg;           // kRecompute: hg [rows][F] = bf16(gate * silu(a) * b)
   const uint16_t* ab;         // kDh: [E * C][2F] a | b
   const float* row_gate;      // kRecompute, kDh: [E * C] gate of the pair in each row
   float* dgate_part;          // kDh: [E * C][dgate_ld] partial sums of <W2^T dy, h>
@@ -88,14 +84,19 @@ struct GemmArgs {
   int overwrite;              // kWgrad: store the tile instead of adding it (round 0)
   int tma_out;                // kWgrad: write the tile through the phase's fp32 output map (TMA
                               // store, or TMA reduce-add) instead of per-thread read-add-write
-  int b_mn;                   // kDh, kDx: B is the weight itself, MN-major ([E][K][N] in memory:
-                              // W2 [E][d][d_ff] for dh, W13 [E][2 d_ff][d] for dx), loaded as
-                              // 64 x 64 boxes (64 N by 64 K), instead of a transposed copy
+  int b_mn;                   // B is MN-major ([K][N] in memory), loaded as 64 x 64 boxes (64 N
+                              // by 64 K): kDh W2 [E][d][d_ff], kDx W13 [E][2 d_ff][d], kWgrad
+                              // the round's row-major hg or xbuf ([rows][N], K = the rows)
+  int a_mn;                   // A is MN-major the same way: kWgrad the round's dybuf or dab
   int32_t* status;
 };
 
-constexpr int kMnBox = 64;                         // MN-major B boxes: 64 N x 64 K rows
+constexpr int kMnBox = 64;                         // MN-major boxes: 64 M or N x 64 K rows
 constexpr int kMnBoxBytes = kMnBox * BK * 2;       // 8 KB
+
+// Instruction descriptor bits of kind::f16: A MN-major (transpose A, bit 15), B MN-major (bit 16).
+constexpr uint32_t kIdescAMn = 1u << 15;
+constexpr uint32_t kIdescBMn = 1u << 16;
 
 __device__ __forceinline__ uint16_t bf16_bits(float v) {
   const __nv_bfloat16 b = __float2bfloat16_rn(v);
@@ -134,36 +135,33 @@ __device__ __forceinline__ void warp_prefix(int* out, int groups, Count cnt_of) 
   __syncwarp();
 }
 
-// Warp 0 writes the tile prefix over the experts into ts[0 .. groups] and, for pooled rows, the
-// experts' first columns in the transposed buffers into seg[0 .. groups].
-__device__ __forceinline__ void plan_tiles(int* ts, int* seg, const GemmArgs& p, int n_tiles, int bm) {
+// Warp 0 writes the tile prefix over the experts into ts[0 .. groups].
+__device__ __forceinline__ void plan_tiles(int* ts, const GemmArgs& p, int n_tiles, int bm) {
   if ((threadIdx.x >> 5) != 0) return;
   warp_prefix(ts, p.groups, [&](int g) { return tiles_of(p, g, n_tiles, bm); });
-  if (p.group_row) warp_prefix(seg, p.groups, [&](int g) { return (p.rows[g] + BK - 1) / BK * BK; });
 }
 
-// Row of expert g's row `row` in the E*C-row buffers.
+// Row of expert g's row `row` in the round buffers.
 __device__ __forceinline__ long long row_of(const GemmArgs& p, int g, int row) {
   return p.group_row ? static_cast<long long>(p.group_row[g] - *p.group_row_base) + row
                      : static_cast<long long>(g) * p.C + row;
 }
 
-// Element (r, c) of expert g's part of a transposed buffer with rows_t rows: c is the expert's row.
-__device__ __forceinline__ long long t_index(const GemmArgs& p, const int* seg, int g, int rows_t, int r,
-                                             int c) {
-  return p.group_row ? static_cast<long long>(r) * p.t_ld + seg[g] + c
-                     : (static_cast<long long>(g) * rows_t + r) * p.t_ld + c;
+// Whether `row` of expert g is a padding row that must hold zeros: at or past the expert's rows,
+// below the next multiple of 64 (the weight-gradient GEMMs read K in blocks of 64), and inside
+// the rows the expert owns (its C rows; with pooled rows its segment).
+__device__ __forceinline__ bool pad_row(const GemmArgs& p, int g, int row) {
+  const int n = p.rows[g];
+  return row >= n && row < (n + BK - 1) / BK * BK && (p.group_row != nullptr || row < p.C);
 }
 
 // ---------------------------------------------------------------- epilogues (one row per thread)
 
-// a, b of 32 columns: row-major bf16 into ab, and bf16(gate * silu(a) * b) transposed into hgT.
-__device__ __forceinline__ void epi_recompute(const GemmArgs& p, const int* seg, uint32_t tb, int g, int row,
-                                              bool valid, int nt) {
+// a, b of 32-column chunks: row-major bf16 into ab, and bf16(gate * silu(a) * b) into hg. A
+// padding row of the expert (see pad_row) gets zeros in hg.
+__device__ __forceinline__ void epi_recompute(const GemmArgs& p, uint32_t tb, int g, int row, bool valid, int nt) {
   const long long rrow = row_of(p, g, row);
-  // transposed rows are written up to the expert's rows rounded up to 64 (zeros past them): the
-  // weight-gradient GEMMs read K in blocks of 64, and with pooled rows the next expert follows
-  const bool in_t = row < (p.rows[g] + BK - 1) / BK * BK;
+  const bool pad = !valid && pad_row(p, g, row);
   const float gv = valid ? p.row_gate[rrow] : 0.f;
   uint16_t* ab = static_cast<uint16_t*>(p.out);
   for (int c = 0; c < p.width; c += 32) {
@@ -172,12 +170,16 @@ __device__ __forceinline__ void epi_recompute(const GemmArgs& p, const int* seg,
     tmem_ld32(tb + p.width + c, bv);
     tmem_wait_ld();
     const int col0 = nt * p.width + c;
+    uint4* hq = reinterpret_cast<uint4*>(p.out_hg + rrow * p.F + col0);
     if (valid) {
-      uint32_t pa[16], pb[16];
+      uint32_t pa[16], pb[16], ph[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        pa[i] = gemm::pack_bf16x2(__uint_as_float(av[2 * i]), __uint_as_float(av[2 * i + 1]));
-        pb[i] = gemm::pack_bf16x2(__uint_as_float(bv[2 * i]), __uint_as_float(bv[2 * i + 1]));
+        const float a0 = __uint_as_float(av[2 * i]), a1 = __uint_as_float(av[2 * i + 1]);
+        const float b0 = __uint_as_float(bv[2 * i]), b1 = __uint_as_float(bv[2 * i + 1]);
+        pa[i] = gemm::pack_bf16x2(a0, a1);
+        pb[i] = gemm::pack_bf16x2(b0, b1);
+        ph[i] = gemm::pack_bf16x2(gv * gemm::silu_f(a0) * b0, gv * gemm::silu_f(a1) * b1);
       }
       uint4* da = reinterpret_cast<uint4*>(ab + rrow * 2 * p.F + col0);
       uint4* db = reinterpret_cast<uint4*>(ab + rrow * 2 * p.F + p.F + col0);
@@ -185,24 +187,20 @@ __device__ __forceinline__ void epi_recompute(const GemmArgs& p, const int* seg,
       for (int i = 0; i < 4; ++i) {
         da[i] = make_uint4(pa[4 * i], pa[4 * i + 1], pa[4 * i + 2], pa[4 * i + 3]);
         db[i] = make_uint4(pb[4 * i], pb[4 * i + 1], pb[4 * i + 2], pb[4 * i + 3]);
+        hq[i] = make_uint4(ph[4 * i], ph[4 * i + 1], ph[4 * i + 2], ph[4 * i + 3]);
       }
-    }
-    if (in_t) {
-      uint16_t* tcol = p.out_t + t_index(p, seg, g, p.F, col0, row);
+    } else if (pad) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float a = __uint_as_float(av[i]), b = __uint_as_float(bv[i]);
-        tcol[static_cast<long long>(i) * p.t_ld] = valid ? bf16_bits(gv * gemm::silu_f(a) * b) : uint16_t(0);
-      }
+      for (int i = 0; i < 4; ++i) hq[i] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
 }
 
 // The accumulator holds W2^T dy for 32-column chunks of the tile; a, b come from the recompute.
-__device__ __forceinline__ void epi_dh(const GemmArgs& p, const int* seg, uint32_t tb, int g, int row, bool valid,
-                                       int nt) {
+// [da | db] goes row-major into dab; a padding row of the expert gets zeros there.
+__device__ __forceinline__ void epi_dh(const GemmArgs& p, uint32_t tb, int g, int row, bool valid, int nt) {
   const long long rrow = row_of(p, g, row);
-  const bool in_t = row < (p.rows[g] + BK - 1) / BK * BK;
+  const bool pad = !valid && pad_row(p, g, row);
   const float gv = valid ? p.row_gate[rrow] : 0.f;
   uint16_t* dab = static_cast<uint16_t*>(p.out);
   float part = 0.f;
@@ -211,8 +209,8 @@ __device__ __forceinline__ void epi_dh(const GemmArgs& p, const int* seg, uint32
     tmem_ld32(tb + c, v);
     tmem_wait_ld();
     const int col0 = nt * p.width + c;
-    uint16_t* tda = p.out_t + t_index(p, seg, g, 2 * p.F, col0, row);
-    uint16_t* tdb = tda + static_cast<long long>(p.F) * p.t_ld;
+    uint4* oda = reinterpret_cast<uint4*>(dab + rrow * 2 * p.F + col0);
+    uint4* odb = reinterpret_cast<uint4*>(dab + rrow * 2 * p.F + p.F + col0);
     if (valid) {
       const uint4* aq = reinterpret_cast<const uint4*>(p.ab + rrow * 2 * p.F + col0);
       const uint4* bq = reinterpret_cast<const uint4*>(p.ab + rrow * 2 * p.F + p.F + col0);
@@ -240,25 +238,16 @@ __device__ __forceinline__ void epi_dh(const GemmArgs& p, const int* seg, uint32
           pdb[4 * u + i] = gemm::pack_bf16x2(dbv[2 * i], dbv[2 * i + 1]);
         }
       }
-      uint4* oda = reinterpret_cast<uint4*>(dab + rrow * 2 * p.F + col0);
-      uint4* odb = reinterpret_cast<uint4*>(dab + rrow * 2 * p.F + p.F + col0);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         oda[i] = make_uint4(pda[4 * i], pda[4 * i + 1], pda[4 * i + 2], pda[4 * i + 3]);
         odb[i] = make_uint4(pdb[4 * i], pdb[4 * i + 1], pdb[4 * i + 2], pdb[4 * i + 3]);
       }
+    } else if (pad) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        tda[static_cast<long long>(2 * i) * p.t_ld] = static_cast<uint16_t>(pda[i] & 0xFFFFu);
-        tda[static_cast<long long>(2 * i + 1) * p.t_ld] = static_cast<uint16_t>(pda[i] >> 16);
-        tdb[static_cast<long long>(2 * i) * p.t_ld] = static_cast<uint16_t>(pdb[i] & 0xFFFFu);
-        tdb[static_cast<long long>(2 * i + 1) * p.t_ld] = static_cast<uint16_t>(pdb[i] >> 16);
-      }
-    } else if (in_t) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        tda[static_cast<long long>(i) * p.t_ld] = 0;
-        tdb[static_cast<long long>(i) * p.t_ld] = 0;
+      for (int i = 0; i < 4; ++i) {
+        oda[i] = make_uint4(0u, 0u, 0u, 0u);
+        odb[i] = make_uint4(0u, 0u, 0u, 0u);
       }
     }
   }
@@ -381,13 +370,9 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   const int unit = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int units = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   int* ts[kMaxPhases];
-  int* seg[kMaxPhases];
-  for (int q = 0; q < kMaxPhases; ++q) {
-    ts[q] = s.tile_start[0] + q * kTileStride;
-    seg[q] = s.tile_start[0] + (kMaxPhases + q) * kTileStride;
-  }
+  for (int q = 0; q < kMaxPhases; ++q) ts[q] = s.tile_start[0] + q * kTileStride;
   for (int q = 0; q < L.phases; ++q)     // reads only the round's row counts (plan data)
-    plan_tiles(ts[q], seg[q], L.ph[q], L.ph[q].n_total / L.ph[q].width, kRows);
+    plan_tiles(ts[q], L.ph[q], L.ph[q].n_total / L.ph[q].width, kRows);
   __syncthreads();
   grid_dependency_wait();
   pdl_trigger_early();
@@ -452,12 +437,15 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
               tma_load_3d(dst, m, fb, c0, c1, c2);
           };
           if (p.mode == kWgrad) {
-            // both operands are transposed buffers, K = the expert's rows: per expert, or from
-            // its pooled first column (a multiple of 64, so the coordinate stays 16-byte aligned)
-            const int k0 = p.group_row ? seg[q][g] + kb * BK : kb * BK;
+            // both operands are the round's row-major buffers read MN-major, K = the expert's
+            // rows (from row 0 of its C rows, or from its segment's first row): this CTA's 128
+            // A columns and its B columns as 64-column boxes, 8 KB apart
+            const int k0 = static_cast<int>(row_of(p, g, 0)) - (p.group_row ? 0 : g * p.C) + kb * BK;
             const int grp = p.group_row ? 0 : g;
-            load(sA, ma, k0, m0, grp);
-            load(sB, mb, k0, kPair ? nt * p.width + static_cast<int>(cta) * gemm::kPairBHalf : nt * p.width, grp);
+            for (int j = 0; j < BM / kMnBox; ++j) load(sA + j * kMnBoxBytes, ma, m0 + j * kMnBox, k0, grp);
+            const int n0 = nt * p.width + (kPair ? static_cast<int>(cta) * gemm::kPairBHalf : 0);
+            const int nb = kPair ? gemm::kPairBHalf / kMnBox : p.width / kMnBox;
+            for (int j = 0; j < nb; ++j) load(sB + j * kMnBoxBytes, mb, n0 + j * kMnBox, k0, grp);
           } else {
             const int a_row = p.group_row ? static_cast<int>(row_of(p, g, m0)) : m0;
             load(sA, ma, kb * BK, a_row, p.group_row ? 0 : g);
@@ -510,9 +498,11 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         int q, g, mt, nt;
         decode(tile, q, g, mt, nt);
         const GemmArgs& p = L.ph[q];
-        const uint32_t idesc = p.b_mn ? idesc_bf16_f32_bmn(kRows, bn_of(p)) : idesc_bf16_f32(kRows, bn_of(p));
+        const uint32_t idesc =
+            idesc_bf16_f32(kRows, bn_of(p)) | (p.a_mn ? kIdescAMn : 0u) | (p.b_mn ? kIdescBMn : 0u);
         // one K step of 16: +32 B along a K-major row, +16 rows of 128 B in an MN-major box
         const uint32_t b_step = p.b_mn ? (16u * 128u) >> 4 : 2u;
+        const uint32_t a_step = p.a_mn ? (16u * 128u) >> 4 : 2u;
         const int kbs = k_blocks_of(p, g);
         if (!mbar_wait(smem_addr(&s.tempty[pipe.acc]), pipe.acc_phase ^ 1u, s.abort)) {
           ok = false;
@@ -527,15 +517,15 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           }
           tc_fence_after();
           const uint32_t sA = smem_addr(s.stage + pipe.stage * kSlot);
-          const uint64_t adesc = smem_desc_sw128(sA);
+          const uint64_t adesc = p.a_mn ? smem_desc_sw128_mn(sA, kMnBoxBytes) : smem_desc_sw128(sA);
           const uint64_t bdesc = p.b_mn ? smem_desc_sw128_mn(sA + gemm::kABytes, kMnBoxBytes)
                                         : smem_desc_sw128(sA + gemm::kABytes);
 #pragma unroll
           for (int kk = 0; kk < BK / gemm::UMMA_K; ++kk) {
             if (kPair)
-              mma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + b_step * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+              mma_bf16_pair(d_tmem, adesc + a_step * kk, bdesc + b_step * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
             else
-              mma_bf16(d_tmem, adesc + 2 * kk, bdesc + b_step * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+              mma_bf16(d_tmem, adesc + a_step * kk, bdesc + b_step * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           if (kPair)
             mma_commit_pair(smem_addr(&s.empty[pipe.stage]), 3);
@@ -588,9 +578,9 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) +
                              static_cast<uint32_t>(pipe.acc * gemm::kAccCols);
       if (p.mode == kRecompute) {
-        epi_recompute(p, seg[q], tbase, g, row, valid, nt);
+        epi_recompute(p, tbase, g, row, valid, nt);
       } else if (p.mode == kDh) {
-        epi_dh(p, seg[q], tbase, g, row, valid, nt);
+        epi_dh(p, tbase, g, row, valid, nt);
       } else if (p.mode == kDx) {
         uint16_t* orow = static_cast<uint16_t*>(p.out) + row_of(p, g, row) * p.out_ld + nt * p.width;
         gemm::store_bf16(tbase, p.width, orow, valid);
@@ -625,17 +615,16 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
 
 constexpr int kWarps = 8;
 
-// Dispatch and transpose of round r in one pass. A block takes 64 rows of one expert's rows in
-// the round and 64 columns (c0 = 64 * blockIdx.y): the rows' tokens come from the round-major row
-// list (row_off[r][e] + s), their x and dy slices are copied row-major into xbuf and dybuf (dy as
-// bf16) and, through a shared-memory tile, transposed into xT and dyT; rows from n[r][e] up to
-// the next multiple of 64 are zeros in the transposed copies only. The blocks of the first
+// Dispatch of round r. A block takes 64 rows of one expert's rows in the round and 64 columns
+// (c0 = 64 * blockIdx.y): the rows' tokens come from the round-major row list (row_off[r][e] +
+// s); their x and dy slices are copied into xbuf and dybuf (dy as bf16). The expert's padding
+// rows (from n[r][e] up to the next multiple of 64, within its C rows or its pooled segment) get
+// zeros: the weight-gradient GEMMs read the rows as K in blocks of 64. The blocks of the first
 // column slice also write each row's gate.
 // The grid's x covers only the round's rows: block b is the b-th 64-row block in expert order
 // (expert e holds ceil(n[r][e] / 64) of them), so a round with few rows launches few blocks.
-// Per-expert rows (no borrowing): expert e's rows s at e * C + s in the row-major buffers and at
-// [e][c][s] (t_ld per row) in the transposed ones. Pooled rows (borrowing): the transposed
-// column of block b is 64 b (segments are the experts' rows rounded up to 64, in expert order).
+// Rows s of expert e are at e * C + s, or with pooled rows at 64 b + (s mod 64): each expert's
+// segment starts at a multiple of 64 (the table seg_off the GEMMs and the combine read).
 struct GatherArgs {
   const uint16_t* x;
   const float* dy;
@@ -643,19 +632,14 @@ struct GatherArgs {
   const float* gate;
   const int32_t* n;           // [max_rounds, E]
   const int32_t* row_off;     // [max_rounds, E] first row of (round, expert) in the row list
-  const int32_t* row_start;   // [max_rounds + 1]
   const int32_t* row_token;
   uint16_t* xbuf;
   uint16_t* dybuf;
   float* row_gate;
-  uint16_t* xt;
-  uint16_t* dyt;
-  int r, E, C, d, k, t_ld, pooled;
+  int r, E, C, d, k, pooled;
 };
 
 __global__ void __launch_bounds__(256) bwd_gather_kernel(const __grid_constant__ GatherArgs a) {
-  __shared__ uint16_t tx_tile[64][66];
-  __shared__ uint16_t ty_tile[64][66];
   __shared__ int tok[64];
   __shared__ int blk[3];      // expert, its first row in this block, its rows in the round
   grid_dependency_wait();
@@ -695,13 +679,11 @@ __global__ void __launch_bounds__(256) bwd_gather_kernel(const __grid_constant__
   }
   __syncthreads();
   const int e = blk[0], s0 = blk[1], ne = blk[2];
-  const int fill = (ne + 63) / 64 * 64;
-  if (e >= 0 && s0 < fill) {
+  if (e >= 0) {
     const int base = a.row_off[static_cast<size_t>(a.r) * a.E + e];
-    const long long dst0 = a.pooled ? static_cast<long long>(base - a.row_start[a.r])
-                                    : static_cast<long long>(e) * a.C;   // row-major row of s = 0
-    const long long tcol0 = a.pooled ? static_cast<long long>(blockIdx.x) * 64
-                                     : static_cast<long long>(e) * a.d * a.t_ld + s0;   // + c * t_ld
+    // row-major row of s = 0 (pooled: this block's first row is 64 b)
+    const long long dst0 = a.pooled ? static_cast<long long>(blockIdx.x) * 64 - s0
+                                    : static_cast<long long>(e) * a.C;
     if (threadIdx.x < 64) {
       const int sr = s0 + threadIdx.x;
       tok[threadIdx.x] = sr < ne ? a.row_token[base + sr] : -1;
@@ -711,30 +693,18 @@ __global__ void __launch_bounds__(256) bwd_gather_kernel(const __grid_constant__
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int rr = ty + 8 * i;
+      const int sr = s0 + rr;
+      if (!a.pooled && sr >= a.C) continue;   // past the expert's C rows: the next expert's
       const int t = tok[rr];
       uint32_t xv = 0, yv = 0;
       if (t >= 0) {
         xv = *reinterpret_cast<const uint32_t*>(a.x + static_cast<size_t>(t) * a.d + c0 + 2 * tx);
         const float2 dv = *reinterpret_cast<const float2*>(a.dy + static_cast<size_t>(t) * a.d + c0 + 2 * tx);
         yv = gemm::pack_bf16x2(dv.x, dv.y);
-        const size_t orow = static_cast<size_t>(dst0 + s0 + rr) * a.d + c0 + 2 * tx;
-        *reinterpret_cast<uint32_t*>(a.xbuf + orow) = xv;
-        *reinterpret_cast<uint32_t*>(a.dybuf + orow) = yv;
       }
-      tx_tile[rr][2 * tx] = static_cast<uint16_t>(xv & 0xFFFFu);
-      tx_tile[rr][2 * tx + 1] = static_cast<uint16_t>(xv >> 16);
-      ty_tile[rr][2 * tx] = static_cast<uint16_t>(yv & 0xFFFFu);
-      ty_tile[rr][2 * tx + 1] = static_cast<uint16_t>(yv >> 16);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int cc = ty + 8 * i;
-      const size_t o = static_cast<size_t>(tcol0 + static_cast<long long>(c0 + cc) * a.t_ld) + 2 * tx;
-      *reinterpret_cast<uint32_t*>(a.xt + o) =
-          static_cast<uint32_t>(tx_tile[2 * tx][cc]) | (static_cast<uint32_t>(tx_tile[2 * tx + 1][cc]) << 16);
-      *reinterpret_cast<uint32_t*>(a.dyt + o) =
-          static_cast<uint32_t>(ty_tile[2 * tx][cc]) | (static_cast<uint32_t>(ty_tile[2 * tx + 1][cc]) << 16);
+      const size_t orow = static_cast<size_t>(dst0 + sr) * a.d + c0 + 2 * tx;
+      *reinterpret_cast<uint32_t*>(a.xbuf + orow) = xv;
+      *reinterpret_cast<uint32_t*>(a.dybuf + orow) = yv;
     }
     if (c0 == 0 && threadIdx.x < 64) {
       const int t = tok[threadIdx.x];
@@ -744,6 +714,34 @@ __global__ void __launch_bounds__(256) bwd_gather_kernel(const __grid_constant__
         a.row_gate[dst0 + s0 + threadIdx.x] = a.gate[static_cast<size_t>(t) * a.k + j];
       }
     }
+  }
+  pdl_trigger_early();
+  pdl_trigger_late();
+}
+
+// The pooled segment table of rounds 0 .. R-1 (one block per round): seg_off[r][e] = the sum over
+// e' < e of n[r][e'] rounded up to 64, and zeros[r] = 0 (zeros[R] too).
+__global__ void __launch_bounds__(32) seg_table_kernel(const int32_t* __restrict__ n, int E, int32_t* seg_off,
+                                                       int32_t* zeros) {
+  grid_dependency_wait();
+  const int r = blockIdx.x, lane = threadIdx.x;
+  const int32_t* nr = n + static_cast<size_t>(r) * E;
+  int running = 0;
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const int e = e0 + lane;
+    const int cnt = e < E ? (nr[e] + 63) / 64 * 64 : 0;
+    int incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (e < E) seg_off[static_cast<size_t>(r) * E + e] = running + incl - cnt;
+    running += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) {
+    zeros[r] = 0;
+    if (r == static_cast<int>(gridDim.x) - 1) zeros[r + 1] = 0;
   }
   pdl_trigger_early();
   pdl_trigger_late();
@@ -982,12 +980,11 @@ cudaError_t run_gemm(const CUtensorMap* a, const CUtensorMap* b, const bwd::Gemm
 
 }  // namespace
 
-long long backward_t_ld(int E, int C, bool pooled) {
-  const long long w = pooled ? static_cast<long long>(E) * C + 64ll * E : static_cast<long long>(C);
-  return (w + 127) / 128 * 128;
+long long backward_rows(int E, int C, bool pooled) {
+  return static_cast<long long>(E) * C + (pooled ? 64ll * E : 0ll);
 }
 
-cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_host, cudaStream_t stream) {
+cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_host, int R, cudaStream_t stream) {
   const int E = a.E, d = a.d, F = a.F;
   cudaError_t e;
   // Round 0 holds every expert that has rows at all (an expert with rows in round r > 0 has C
@@ -998,6 +995,12 @@ cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_h
     if (load_host[x] > 0) continue;
     if ((e = cudaMemsetAsync(a.dw_gate_up + x * per13, 0, per13 * 4, stream)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(a.dw_down + x * per2, 0, per2 * 4, stream)) != cudaSuccess) return e;
+  }
+  if (R > 0) {   // the pooled segment table (read only with pooled rows; cheap either way)
+    launch_begin(kKindBackwardCopy, stream);
+    e = launch_pdl(bwd::seg_table_kernel, dim3(R), dim3(32), 0, stream, a.n, E, a.seg_off, a.zeros);
+    launch_end(kKindBackwardCopy, stream);
+    if (e != cudaSuccess) return e;
   }
   const long long pairs = static_cast<long long>(a.T) * a.k;
   if (pairs > 0) {
@@ -1013,17 +1016,16 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
                                   cudaStream_t stream) {
   (void)rows;
   const int E = a.E, C = a.C, d = a.d, F = a.F;
-  const long long t_ld = a.t_ld;
   const bool pooled = a.pooled != 0;
   const int32_t* n_dev = a.n + static_cast<size_t>(r) * E;
-  // A operands [E][C][K] per expert, or pooled [1][E * C][K]; transposed [E][rows][t_ld] or [1][rows][t_ld]
-  const uint64_t a_rows = pooled ? static_cast<uint64_t>(E) * C : static_cast<uint64_t>(C);
+  // round buffers as 3-D maps: [E][C][K] per expert, or pooled [1][rows][K]
+  const uint64_t a_rows = pooled ? static_cast<uint64_t>(a.rows) : static_cast<uint64_t>(C);
   const uint64_t groups = pooled ? 1 : static_cast<uint64_t>(E);
   cudaError_t e;
-  // dispatch and transpose x, dy; the rows' gates
+  // dispatch x and dy; the rows' gates
   {
-    const bwd::GatherArgs ga{a.x, a.dy, a.idx, a.gate, a.n, a.row_off, a.row_start, a.row_token, a.xbuf, a.dybuf,
-                             a.row_gate, a.xt, a.dyt, r, E, C, d, a.k, static_cast<int>(t_ld), pooled ? 1 : 0};
+    const bwd::GatherArgs ga{a.x, a.dy, a.idx, a.gate, a.n, a.row_off, a.row_token, a.xbuf, a.dybuf,
+                             a.row_gate, r, E, C, d, a.k, pooled ? 1 : 0};
     long long blocks = 0;   // the round's 64-row blocks, expert by expert
     for (int x = 0; x < E; ++x) blocks += (n_host[x] + 63) / 64;
     if (blocks > 0) {
@@ -1046,9 +1048,8 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
   base.groups = E;
   base.C = C;
   base.F = F;
-  base.t_ld = static_cast<int>(t_ld);
-  base.group_row = pooled ? a.row_off + static_cast<size_t>(r) * E : nullptr;
-  base.group_row_base = pooled ? a.row_start + r : nullptr;
+  base.group_row = pooled ? a.seg_off + static_cast<size_t>(r) * E : nullptr;   // 64-aligned segments
+  base.group_row_base = pooled ? a.zeros + r : nullptr;
   base.status = a.status;
   static const int kWide[3] = {256, 128, 64};
   // pair form: 256-row tiles, 128 B rows per CTA (recompute: 128 W1 rows and the same W3 rows)
@@ -1064,7 +1065,7 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g.n_total = F;
     g.num_k_blocks = d / gemm::BK;
     g.out = a.ab;
-    g.out_t = a.hgt;
+    g.out_hg = a.hg;
     g.row_gate = a.row_gate;
     CUtensorMap ma, mb;
     if ((e = gemm::make_map(&ma, a.xbuf, d, a_rows, groups, gemm::BM)) != cudaSuccess) return e;
@@ -1086,7 +1087,6 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g.n_total = F;
     g.num_k_blocks = d / gemm::BK;
     g.out = a.dab;
-    g.out_t = a.dabt;
     g.ab = a.ab;
     g.row_gate = a.row_gate;
     g.dgate_part = a.dgate_part;
@@ -1097,7 +1097,8 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     if ((e = gemm::make_map(&mb, a.w_down, F, d, E, bwd::kMnBox, bwd::kMnBox)) != cudaSuccess) return e;
     if ((e = run_gemm(&ma, &mb, &g, 1, mt * parts, kKindBackwardDh, stream, nullptr, pair)) != cudaSuccess) return e;
   }
-  // one launch: dx rows = dab W13, dW2 (+)= dyT hgT^T, dW13 (+)= dabT xT^T (K = the round's rows)
+  // one launch: dx rows = dab W13, dW2 (+)= dy^T hg and dW13 (+)= dab^T x over K = the round's
+  // rows of each expert (both operands the row-major round buffers, read MN-major)
   {
     // the weight gradients' tiles cover d x F and 2F x d per active expert whatever the round's
     // rows; the dx phase decides, as in the other launches
@@ -1127,9 +1128,9 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g[1].out_ld = F;
     g[1].tma_out = 1;   // dW2 [E][d][F] fp32 through TMA (store in round 0, reduce-add after)
     if ((e = gemm::make_map_f32(&mo[1], a.dw_down, F, d, E, 16, 32)) != cudaSuccess) return e;
-    if ((e = gemm::make_map(&ma[1], a.dyt, static_cast<uint64_t>(t_ld), d, groups, gemm::BM)) != cudaSuccess) return e;
-    if ((e = gemm::make_map(&mb[1], a.hgt, static_cast<uint64_t>(t_ld), F, groups,
-                            pair ? pair_box : static_cast<uint32_t>(g[1].width))) != cudaSuccess)
+    g[1].a_mn = g[1].b_mn = 1;   // A[m = column of d][k = row] = dybuf[k][m], B[n][k] = hg[k][n]
+    if ((e = gemm::make_map(&ma[1], a.dybuf, d, a_rows, groups, bwd::kMnBox, bwd::kMnBox)) != cudaSuccess ||
+        (e = gemm::make_map(&mb[1], a.hg, F, a_rows, groups, bwd::kMnBox, bwd::kMnBox)) != cudaSuccess)
       return e;
     tiles += mt_w2 * (F / g[1].width);
     g[2].mode = bwd::kWgrad;
@@ -1142,10 +1143,9 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g[2].out_ld = d;
     g[2].tma_out = 1;   // dW13 [E][2F][d] fp32 through TMA
     if ((e = gemm::make_map_f32(&mo[2], a.dw_gate_up, d, 2ull * F, E, 16, 32)) != cudaSuccess) return e;
-    if ((e = gemm::make_map(&ma[2], a.dabt, static_cast<uint64_t>(t_ld), 2ull * F, groups, gemm::BM)) != cudaSuccess)
-      return e;
-    if ((e = gemm::make_map(&mb[2], a.xt, static_cast<uint64_t>(t_ld), d, groups,
-                            pair ? pair_box : static_cast<uint32_t>(g[2].width))) != cudaSuccess)
+    g[2].a_mn = g[2].b_mn = 1;   // A[m = column of 2 d_ff][k = row] = dab[k][m], B[n][k] = xbuf[k][n]
+    if ((e = gemm::make_map(&ma[2], a.dab, 2ull * F, a_rows, groups, bwd::kMnBox, bwd::kMnBox)) != cudaSuccess ||
+        (e = gemm::make_map(&mb[2], a.xbuf, d, a_rows, groups, bwd::kMnBox, bwd::kMnBox)) != cudaSuccess)
       return e;
     tiles += mt_w13 * (d / g[2].width);
     mo[0] = ma[0];
@@ -1153,8 +1153,9 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
   }
   // combine dx and gather dgate
   {
+    // pooled rows: the pair's row is seg_off[r][e] - zeros[r] + slot
     const copy::CombineArgs ca{a.dxbuf, a.dx, a.idx, a.ones, a.round, a.slot, a.T, a.k, C, d,
-                               pooled ? a.row_off : nullptr, pooled ? a.row_start : nullptr, E};
+                               pooled ? a.seg_off : nullptr, pooled ? a.zeros : nullptr, E};
     launch_begin(kKindBackwardCopy, stream);
     e = launch_pdl(bwd::bwd_combine_kernel, dim3(grid_for(a.T)), dim3(32 * bwd::kWarps), 0, stream, ca, r,
                    static_cast<const float*>(a.dgate_part), F / 64, parts, a.dgate);

@@ -38,34 +38,34 @@ struct BackwardArgs {
   float* dw_gate_up;          // [E, 2F, d]
   float* dw_down;             // [E, d, F]
   float* dz;                  // [T, E]
-  // backward workspace
-  uint16_t* xbuf;             // [E * C, d]
-  uint16_t* dybuf;            // [E * C, d]
-  float* row_gate;            // [E * C]
-  uint16_t* xt;               // [E, d, t_ld], or [d, t_ld] pooled
-  uint16_t* dyt;              // the same
-  uint16_t* ab;               // [E * C, 2F]
-  uint16_t* hgt;              // [E, F, t_ld], or [F, t_ld] pooled
-  uint16_t* dab;              // [E * C, 2F]
-  uint16_t* dabt;             // [E, 2F, t_ld], or [2F, t_ld] pooled
-  float* dgate_part;          // [E * C, F / 64]
-  uint16_t* dxbuf;            // [E * C, d]
+  // backward workspace: per-round buffers of `rows` rows (E * C, or with pooled rows E * C + 64 E:
+  // expert e's rows of round r from seg_off[r][e], a multiple of 64)
+  uint16_t* xbuf;             // [rows, d]
+  uint16_t* dybuf;            // [rows, d]
+  float* row_gate;            // [rows]
+  uint16_t* ab;               // [rows, 2F]
+  uint16_t* hg;               // [rows, F]
+  uint16_t* dab;              // [rows, 2F]
+  float* dgate_part;          // [rows, F / 64]
+  uint16_t* dxbuf;            // [rows, d]
   float* dgate;               // [T, k]
   float* ones;                // [T, k]
+  int32_t* seg_off;           // [max_rounds, E] pooled rows: each expert's first row in a round
+  int32_t* zeros;             // [max_rounds + 1]
   int32_t* status;
   int T, k, E, C, d, F, renorm;
   int pooled;                 // capacity borrowing: pooled round rows (see the plan's row_off)
-  long long t_ld;             // elements per row of the transposed buffers
+  int rows;                   // rows of the per-round buffers
 };
-// Elements per row of the transposed per-round buffers: C rounded up to 128 (a whole GEMM row
-// tile) per expert; with pooled rows E * C + 64 * E (every expert's segment rounded up to 64)
-// rounded up to 128, one row for all experts.
-long long backward_t_ld(int E, int C, bool pooled);
-// Zeroes the weight gradients of experts without rows (load_host: host copy of the loads),
-// transposes the weights, fills the unit gates.
-cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_host, cudaStream_t stream);
-// One round: dispatch, transposes, recompute, dh (+ SwiGLU backward), dx GEMM, dx combine and
-// dgate, weight gradients. n_host / rows: the round's rows per expert and in total.
+// Rows of the per-round buffers: E * C per expert (expert e's rows at e * C), or with pooled rows
+// E * C + 64 E (each expert's segment rounded up to 64 rows, in expert order).
+long long backward_rows(int E, int C, bool pooled);
+// Zeroes the weight gradients of experts without rows (load_host: host copy of the loads), fills
+// the unit gates, and writes the segment table seg_off of the R rounds (from the plan's n on the
+// device) and the zero words.
+cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_host, int R, cudaStream_t stream);
+// One round: dispatch, recompute, dh (+ SwiGLU backward), dx GEMM, dx combine and dgate, weight
+// gradients. n_host / rows: the round's rows per expert and in total.
 cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n_host, int rows,
                                   cudaStream_t stream);
 // dz from dgate and the logits, after the last round.

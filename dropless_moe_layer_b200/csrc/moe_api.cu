@@ -399,30 +399,29 @@ void make_backward_layout(const moe_shape_t* s, moe_backward_layout_t* L) {
     off += (static_cast<size_t>(bytes) + 255) & ~static_cast<size_t>(255);
     return o;
   };
-  const long long T = s->T, E = s->E, k = s->k, C = s->C, d = s->d, F = s->d_ff;
-  const bool pooled = (s->flags & MOE_FLAG_BORROW) != 0;
-  const long long t_ld = backward_t_ld(s->E, s->C, pooled);
-  const long long tg = pooled ? 1 : E;   // transposed buffers: one per expert, or one pooled
-  L->xbuf = take(E * C * d * 2);
-  L->dybuf = take(E * C * d * 2);
-  L->row_gate = take(E * C * 4);
-  L->xt = take(tg * d * t_ld * 2);
-  L->dyt = take(tg * d * t_ld * 2);
-  L->ab = take(E * C * 2 * F * 2);
-  L->hgt = take(tg * F * t_ld * 2);
-  L->dab = take(E * C * 2 * F * 2);
-  L->dabt = take(tg * 2 * F * t_ld * 2);
-  L->dgate_part = take(E * C * (F / 64) * 4);
-  L->dxbuf = take(E * C * d * 2);
+  const long long T = s->T, E = s->E, k = s->k, d = s->d, F = s->d_ff;
+  const long long rows = backward_rows(s->E, s->C, (s->flags & MOE_FLAG_BORROW) != 0);
+  const long long mr = max_rounds_of(s);
+  L->xbuf = take(rows * d * 2);
+  L->dybuf = take(rows * d * 2);
+  L->row_gate = take(rows * 4);
+  L->ab = take(rows * 2 * F * 2);
+  L->hg = take(rows * F * 2);
+  L->dab = take(rows * 2 * F * 2);
+  L->dgate_part = take(rows * (F / 64) * 4);
+  L->dxbuf = take(rows * d * 2);
   L->dgate = take(T * k * 4);
   L->ones = take(T * k * 4);
+  L->seg_off = take(mr * E * 4);
+  L->zeros = take((mr + 1) * 4);
   L->total_bytes = off;
-  L->cpad = static_cast<int32_t>(t_ld);
+  L->rows = static_cast<int32_t>(rows);
 }
 
-// The pooled transposed row (borrowing) must stay within int32 element offsets.
+// The per-round buffers' rows (and the element offsets within them) must fit int32.
 bool backward_shape_ok(const moe_shape_t* s) {
-  return backward_t_ld(s->E, s->C, (s->flags & MOE_FLAG_BORROW) != 0) < (1ll << 31);
+  const long long rows = backward_rows(s->E, s->C, (s->flags & MOE_FLAG_BORROW) != 0);
+  return rows * 2 * s->d_ff < (1ll << 31) && rows * s->d < (1ll << 31);
 }
 
 }  // namespace
@@ -489,12 +488,11 @@ int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws
   a.xbuf = at<uint16_t>(bws, B.xbuf);
   a.dybuf = at<uint16_t>(bws, B.dybuf);
   a.row_gate = at<float>(bws, B.row_gate);
-  a.xt = at<uint16_t>(bws, B.xt);
-  a.dyt = at<uint16_t>(bws, B.dyt);
   a.ab = at<uint16_t>(bws, B.ab);
-  a.hgt = at<uint16_t>(bws, B.hgt);
+  a.hg = at<uint16_t>(bws, B.hg);
   a.dab = at<uint16_t>(bws, B.dab);
-  a.dabt = at<uint16_t>(bws, B.dabt);
+  a.seg_off = at<int32_t>(bws, B.seg_off);
+  a.zeros = at<int32_t>(bws, B.zeros);
   a.dgate_part = at<float>(bws, B.dgate_part);
   a.dxbuf = at<uint16_t>(bws, B.dxbuf);
   a.dgate = at<float>(bws, B.dgate);
@@ -508,8 +506,8 @@ int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws
   a.F = shape->d_ff;
   a.renorm = (shape->flags & MOE_FLAG_RENORM_TOPK) ? 1 : 0;
   a.pooled = borrowing(shape) ? 1 : 0;
-  a.t_ld = B.cpad;
-  if ((st = cuda_status(launch_backward_prepare(a, info->load, stream))) != MOE_OK) return st;
+  a.rows = B.rows;
+  if ((st = cuda_status(launch_backward_prepare(a, info->load, info->R, stream))) != MOE_OK) return st;
   for (int r = 0; r < info->R; ++r) {
     int32_t n_host[MOE_MAX_EXPERTS];
     int rows = 0;

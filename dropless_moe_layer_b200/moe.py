@@ -53,9 +53,9 @@ class WorkspaceLayout(ctypes.Structure):
 
 class BackwardLayout(ctypes.Structure):
     _fields_ = [(name, c_sz) for name in (
-        "total_bytes", "xbuf", "dybuf", "row_gate", "xt", "dyt", "ab", "hgt", "dab", "dabt",
-        "dgate_part", "dxbuf", "dgate", "ones")
-    ] + [("cpad", c_i32)]
+        "total_bytes", "xbuf", "dybuf", "row_gate", "ab", "hg", "dab", "dgate_part", "dxbuf", "dgate",
+        "ones", "seg_off", "zeros")
+    ] + [("rows", c_i32)]
 
 
 class MoeError(RuntimeError):

@@ -236,27 +236,29 @@ MOE_API int moe_round_combine(const moe_shape_t* shape, const moe_plan_info_t* i
  * weight gradients into the caller's fp32 gradients; nothing it holds grows with the routing.
  *
  * Its own workspace `bws` (device, caller-owned, 256-byte aligned) holds the per-round buffers;
- * its size depends on the shape only. The weights are read as they are stored (the GEMMs that
- * need them transposed load them MN-major). */
+ * its size depends on the shape only. Weights and activations are read as they are stored: the
+ * GEMMs that need an operand transposed load it MN-major, so no transposed copy is made. */
 typedef struct moe_backward_layout {
   size_t total_bytes;
-  size_t xbuf;        /* bf16 [E * C, d]     the round's x rows */
-  size_t dybuf;       /* bf16 [E * C, d]     the round's dy rows */
-  size_t row_gate;    /* f32  [E * C]        the gate of the pair in each row */
-  size_t xt;          /* bf16 [E, d, cpad]   xbuf transposed per expert (K-major over rows);
-                         with MOE_FLAG_BORROW [d, cpad], pooled */
-  size_t dyt;         /* bf16, dybuf transposed, the same shape */
-  size_t ab;          /* bf16 [E * C, 2 d_ff] recomputed a = W1 x, b = W3 x */
-  size_t hgt;         /* bf16 [E, d_ff, cpad] gate * silu(a) * b, transposed ([d_ff, cpad] pooled) */
-  size_t dab;         /* bf16 [E * C, 2 d_ff] [da | db] */
-  size_t dabt;        /* bf16 [E, 2 d_ff, cpad] [da | db] transposed ([2 d_ff, cpad] pooled) */
-  size_t dgate_part;  /* f32  [E * C, d_ff / 64] per-tile partial sums of dgate */
-  size_t dxbuf;       /* bf16 [E * C, d]     per-pair dx rows of the round */
+  /* The per-round buffers have `rows` rows: E * C, expert e's rows of the round at e * C + slot;
+     with MOE_FLAG_BORROW E * C + 64 * E, expert e's rows at the round's seg_off[r][e] + slot,
+     where each expert's segment starts at a multiple of 64 rows (the experts' rows rounded up to
+     64, in expert order). Rows from an expert's count up to the next multiple of 64 (within its
+     C rows, or within its segment) hold zeros in xbuf, dybuf, hg and dab: the weight-gradient
+     GEMMs read K, the rows, in blocks of 64. */
+  size_t xbuf;        /* bf16 [rows, d]      the round's x rows */
+  size_t dybuf;       /* bf16 [rows, d]      the round's dy rows */
+  size_t row_gate;    /* f32  [rows]         the gate of the pair in each row */
+  size_t ab;          /* bf16 [rows, 2 d_ff] recomputed a = W1 x, b = W3 x */
+  size_t hg;          /* bf16 [rows, d_ff]   gate * silu(a) * b */
+  size_t dab;         /* bf16 [rows, 2 d_ff] [da | db] */
+  size_t dgate_part;  /* f32  [rows, d_ff / 64] per-tile partial sums of dgate */
+  size_t dxbuf;       /* bf16 [rows, d]      per-pair dx rows of the round */
   size_t dgate;       /* f32  [T, k]         dL/dgate */
   size_t ones;        /* f32  [T, k]         unit gates of the dx combine */
-  int32_t cpad;       /* elements per row of the transposed buffers: C rounded up to 128 (one
-                         buffer per expert); with MOE_FLAG_BORROW, E * C + 64 * E rounded up to
-                         128 (one pooled buffer, every expert's rows rounded up to 64) */
+  size_t seg_off;     /* i32  [max_rounds, E] MOE_FLAG_BORROW: first row of each expert's segment */
+  size_t zeros;       /* i32  [max_rounds + 1] zeros (row offsets of the segment tables) */
+  int32_t rows;       /* rows of the per-round buffers (above) */
 } moe_backward_layout_t;
 
 /* Bytes of the backward workspace for `shape` (0 for an invalid shape). */

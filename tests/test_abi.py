@@ -139,16 +139,17 @@ def test_forward_argument_errors_without_gpu(lib):
 
 
 def _backward_bytes_model(w, borrow=False):
-    """Backward workspace from its layout rules: per-round buffers of E*C rows, the transposed
-    copies with C rounded up to 128 per expert (with borrowing one pooled copy whose rows hold
-    E*C + 64*E columns rounded up to 128), [T, k] dgate and unit gates. No copy of the weights."""
+    """Backward workspace from its layout rules: per-round buffers of E*C rows (with borrowing
+    E*C + 64*E: each expert's segment starts at a multiple of 64), [T, k] dgate and unit gates,
+    the segment table [max_rounds, E] and max_rounds + 1 zero words. No copy of the weights and
+    no transposed copy of the activations."""
     def a(n):
         return (n + 255) // 256 * 256
     T, E, k, C, d, F = w.T, w.E, w.k, w.C, w.d, w.F
-    cp = (E * C + 64 * E + 127) // 128 * 128 if borrow else (C + 127) // 128 * 128
-    tg = 1 if borrow else E
-    return (3 * a(E * C * d * 2) + a(E * C * 4) + 2 * a(tg * d * cp * 2) + 2 * a(E * C * 2 * F * 2)
-            + a(tg * F * cp * 2) + a(tg * 2 * F * cp * 2) + a(E * C * (F // 64) * 4) + 2 * a(T * k * 4))
+    rows = E * C + (64 * E if borrow else 0)
+    mr = (T + C - 1) // C
+    return (3 * a(rows * d * 2) + a(rows * 4) + 2 * a(rows * 2 * F * 2) + a(rows * F * 2)
+            + a(rows * (F // 64) * 4) + 2 * a(T * k * 4) + a(mr * E * 4) + a((mr + 1) * 4))
 
 
 @pytest.mark.parametrize("w", wl.WORKLOADS, ids=lambda w: w.name)
@@ -157,13 +158,13 @@ def test_backward_workspace_is_fixed_by_shape(lib, w):
     n = moe.backward_workspace_bytes(s)
     assert n == _backward_bytes_model(w)
     lay = moe.backward_layout(s)
-    assert lay.total_bytes == n and lay.cpad % 128 == 0 and w.C <= lay.cpad < w.C + 128
-    offs = [lay.xbuf, lay.dybuf, lay.row_gate, lay.xt, lay.dyt, lay.ab, lay.hgt, lay.dab, lay.dabt,
-            lay.dgate_part, lay.dxbuf, lay.dgate, lay.ones]
+    assert lay.total_bytes == n and lay.rows == w.E * w.C
+    offs = [lay.xbuf, lay.dybuf, lay.row_gate, lay.ab, lay.hg, lay.dab, lay.dgate_part, lay.dxbuf, lay.dgate,
+            lay.ones, lay.seg_off, lay.zeros]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     sb = moe.make_shape(w.T, w.d, w.E, w.k, w.F, w.C, borrow=True)
     assert moe.backward_workspace_bytes(sb) == _backward_bytes_model(w, borrow=True)
-    assert moe.backward_layout(sb).cpad == (w.E * w.C + 64 * w.E + 127) // 128 * 128
+    assert moe.backward_layout(sb).rows == w.E * w.C + 64 * w.E
     s.flags = 32          # not a flag
     assert moe.backward_workspace_bytes(s) == 0
 
