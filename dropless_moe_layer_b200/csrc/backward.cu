@@ -18,10 +18,10 @@
 // seg_off[r][e] + slot, where each expert's segment starts at a multiple of 64:
 //   gather     x rows -> xbuf, bf16(dy) rows -> dybuf; the pair's gate -> row_gate
 //   recompute  [a | b] = xbuf W13^T (tensor cores); epilogue keeps a, b (bf16) and writes
-//              hg = bf16(gate * h)
+//              hg = bf16(gate * h), through TMA stores of 32 x 32 chunks
 //   dh         W2^T dy as dybuf (W2^T)^T (tensor cores, B = W2 read MN-major as stored);
 //              epilogue: the SwiGLU backward (da, db from a, b and the gate), dgate partial sums
-//              <W2^T dy, h> per 64..256-column tile, dab = [da | db]
+//              <W2^T dy, h> per 64..256-column tile, dab = [da | db] (TMA stores)
 //   dx         dab W13 (tensor cores, B = W13 read MN-major as stored) -> dxbuf (bf16)
 //   combine    dx[t] = (first round of t ? 0 : dx[t]) + sum of the token's dxbuf rows, ascending
 //              j; dgate[t, j] = sum of its row's partials in tile order (no atomics anywhere)
@@ -76,7 +76,6 @@ struct GemmArgs {
   void* out;                  // kRecompute: ab; kDh: dab; kDx: dxbuf; kWgrad: the fp32 gradient
   long long out_group_stride; // elements (kWgrad)
   int out_ld;                 // elements (kWgrad, kDx)
-  uint16_t* out_hg;           // kRecompute: hg [rows][F] = bf16(gate * silu(a) * b)
   const uint16_t* ab;         // kDh: [E * C][2F] a | b
   const float* row_gate;      // kRecompute, kDh: [E * C] gate of the pair in each row
   float* dgate_part;          // kDh: [E * C][dgate_ld] partial sums of <W2^T dy, h>
@@ -147,74 +146,103 @@ __device__ __forceinline__ long long row_of(const GemmArgs& p, int g, int row) {
                      : static_cast<long long>(g) * p.C + row;
 }
 
-// Whether `row` of expert g is a padding row that must hold zeros: at or past the expert's rows,
-// below the next multiple of 64 (the weight-gradient GEMMs read K in blocks of 64), and inside
-// the rows the expert owns (its C rows; with pooled rows its segment).
-__device__ __forceinline__ bool pad_row(const GemmArgs& p, int g, int row) {
-  const int n = p.rows[g];
-  return row >= n && row < (n + BK - 1) / BK * BK && (p.group_row != nullptr || row < p.C);
-}
-
 // ---------------------------------------------------------------- epilogues (one row per thread)
 
-// a, b of 32-column chunks: row-major bf16 into ab, and bf16(gate * silu(a) * b) into hg. A
-// padding row of the expert (see pad_row) gets zeros in hg.
-__device__ __forceinline__ void epi_recompute(const GemmArgs& p, uint32_t tb, int g, int row, bool valid, int nt) {
-  const long long rrow = row_of(p, g, row);
-  const bool pad = !valid && pad_row(p, g, row);
-  const float gv = valid ? p.row_gate[rrow] : 0.f;
-  uint16_t* ab = static_cast<uint16_t*>(p.out);
+// One 32 x 32 bf16 chunk of this warp's 32 rows (lane = row; pk = the lane's 32 values packed in
+// pairs) through one of the warp's two staging buffers (64-byte swizzle) and one bulk tensor
+// store at (col, row, grp) of `map`. ochunk counts the warp's staged chunks (alternates buffers).
+__device__ __forceinline__ void store_chunk(const CUtensorMap* map, const uint32_t (&pk)[16], int col, int row,
+                                            int grp, uint8_t* stage, uint32_t& ochunk) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t buf_off = (ochunk & 1u) * gemm::kOutChunkBytes;
+  if (lane == 0) bulk_wait_read_1();   // the store that last used this buffer has read it
+  __syncwarp();
+  uint8_t* row_ptr = stage + buf_off + lane * 64;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)   // 64-byte swizzle: piece j of row r at j ^ ((r >> 1) & 3)
+    *reinterpret_cast<uint4*>(row_ptr + ((j ^ ((lane >> 1) & 3)) << 4)) =
+        make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+  fence_async_shared();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_3d_plain(map, smem_addr(stage) + buf_off, col, row, grp);
+    bulk_commit();
+  }
+  ++ochunk;
+}
+
+// Where this warp's 32 rows [row_base, row_base + 32) of expert g go, and which of them it
+// stores: `rows_out` the map coordinates (row within the expert's C rows and group, or the
+// pooled row and group 0); `keep_ab` whether the box holds a row of the expert (the ab box:
+// rows past the expert's count in it are junk no one reads, and stay inside the expert's
+// rows); `keep_pad` whether it starts below the count rounded up to 64 (the hg / dab box: rows
+// past the count get zeros, and the box ends at or before that multiple of 64).
+struct ChunkRows {
+  int row, grp;
+  bool keep_ab, keep_pad;
+};
+
+__device__ __forceinline__ ChunkRows chunk_rows(const GemmArgs& p, int g, int row_base) {
+  ChunkRows c;
+  const int n = p.rows[g];
+  c.row = p.group_row ? static_cast<int>(row_of(p, g, row_base)) : row_base;
+  c.grp = p.group_row ? 0 : g;
+  c.keep_ab = row_base < n;
+  c.keep_pad = row_base < (n + BK - 1) / BK * BK;
+  return c;
+}
+
+// a, b of 32-column chunks into ab, and hg = bf16(gate * silu(a) * b), all row-major, through
+// TMA stores of 32 x 32 chunks (maps: ab [.][2F], hg [.][F]). The expert's padding rows get
+// zeros in hg.
+__device__ __forceinline__ void epi_recompute(const GemmArgs& p, const CUtensorMap* ab_map, const CUtensorMap* hg_map,
+                                              uint32_t tb, int g, int row_base, bool valid, int nt, uint8_t* stage,
+                                              uint32_t& ochunk) {
+  const int lane = threadIdx.x & 31;
+  const ChunkRows cr = chunk_rows(p, g, row_base);
+  const float gv = valid ? p.row_gate[row_of(p, g, row_base + lane)] : 0.f;
   for (int c = 0; c < p.width; c += 32) {
     uint32_t av[32], bv[32];
     tmem_ld32(tb + c, av);
     tmem_ld32(tb + p.width + c, bv);
     tmem_wait_ld();
     const int col0 = nt * p.width + c;
-    uint4* hq = reinterpret_cast<uint4*>(p.out_hg + rrow * p.F + col0);
-    if (valid) {
-      uint32_t pa[16], pb[16], ph[16];
+    uint32_t pa[16], pb[16], ph[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float a0 = __uint_as_float(av[2 * i]), a1 = __uint_as_float(av[2 * i + 1]);
-        const float b0 = __uint_as_float(bv[2 * i]), b1 = __uint_as_float(bv[2 * i + 1]);
-        pa[i] = gemm::pack_bf16x2(a0, a1);
-        pb[i] = gemm::pack_bf16x2(b0, b1);
-        ph[i] = gemm::pack_bf16x2(gv * gemm::silu_f(a0) * b0, gv * gemm::silu_f(a1) * b1);
-      }
-      uint4* da = reinterpret_cast<uint4*>(ab + rrow * 2 * p.F + col0);
-      uint4* db = reinterpret_cast<uint4*>(ab + rrow * 2 * p.F + p.F + col0);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        da[i] = make_uint4(pa[4 * i], pa[4 * i + 1], pa[4 * i + 2], pa[4 * i + 3]);
-        db[i] = make_uint4(pb[4 * i], pb[4 * i + 1], pb[4 * i + 2], pb[4 * i + 3]);
-        hq[i] = make_uint4(ph[4 * i], ph[4 * i + 1], ph[4 * i + 2], ph[4 * i + 3]);
-      }
-    } else if (pad) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) hq[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = 0; i < 16; ++i) {
+      const float a0 = __uint_as_float(av[2 * i]), a1 = __uint_as_float(av[2 * i + 1]);
+      const float b0 = __uint_as_float(bv[2 * i]), b1 = __uint_as_float(bv[2 * i + 1]);
+      pa[i] = gemm::pack_bf16x2(a0, a1);
+      pb[i] = gemm::pack_bf16x2(b0, b1);
+      ph[i] = valid ? gemm::pack_bf16x2(gv * gemm::silu_f(a0) * b0, gv * gemm::silu_f(a1) * b1) : 0u;
     }
+    if (cr.keep_ab) {
+      store_chunk(ab_map, pa, col0, cr.row, cr.grp, stage, ochunk);
+      store_chunk(ab_map, pb, p.F + col0, cr.row, cr.grp, stage, ochunk);
+    }
+    if (cr.keep_pad) store_chunk(hg_map, ph, col0, cr.row, cr.grp, stage, ochunk);
   }
 }
 
 // The accumulator holds W2^T dy for 32-column chunks of the tile; a, b come from the recompute.
-// [da | db] goes row-major into dab; a padding row of the expert gets zeros there.
-__device__ __forceinline__ void epi_dh(const GemmArgs& p, uint32_t tb, int g, int row, bool valid, int nt) {
-  const long long rrow = row_of(p, g, row);
-  const bool pad = !valid && pad_row(p, g, row);
+// [da | db] goes row-major into dab through TMA stores of 32 x 32 chunks (map dab [.][2F]); the
+// expert's padding rows get zeros there.
+__device__ __forceinline__ void epi_dh(const GemmArgs& p, const CUtensorMap* dab_map, uint32_t tb, int g, int row_base,
+                                       bool valid, int nt, uint8_t* stage, uint32_t& ochunk) {
+  const int lane = threadIdx.x & 31;
+  const ChunkRows cr = chunk_rows(p, g, row_base);
+  const long long rrow = row_of(p, g, row_base + lane);
   const float gv = valid ? p.row_gate[rrow] : 0.f;
-  uint16_t* dab = static_cast<uint16_t*>(p.out);
   float part = 0.f;
   for (int c = 0; c < p.width; c += 32) {
     uint32_t v[32];
     tmem_ld32(tb + c, v);
     tmem_wait_ld();
     const int col0 = nt * p.width + c;
-    uint4* oda = reinterpret_cast<uint4*>(dab + rrow * 2 * p.F + col0);
-    uint4* odb = reinterpret_cast<uint4*>(dab + rrow * 2 * p.F + p.F + col0);
+    uint32_t pda[16], pdb[16];
     if (valid) {
       const uint4* aq = reinterpret_cast<const uint4*>(p.ab + rrow * 2 * p.F + col0);
       const uint4* bq = reinterpret_cast<const uint4*>(p.ab + rrow * 2 * p.F + p.F + col0);
-      uint32_t pda[16], pdb[16];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         float af[8], bf[8];
@@ -238,17 +266,13 @@ __device__ __forceinline__ void epi_dh(const GemmArgs& p, uint32_t tb, int g, in
           pdb[4 * u + i] = gemm::pack_bf16x2(dbv[2 * i], dbv[2 * i + 1]);
         }
       }
+    } else {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        oda[i] = make_uint4(pda[4 * i], pda[4 * i + 1], pda[4 * i + 2], pda[4 * i + 3]);
-        odb[i] = make_uint4(pdb[4 * i], pdb[4 * i + 1], pdb[4 * i + 2], pdb[4 * i + 3]);
-      }
-    } else if (pad) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        oda[i] = make_uint4(0u, 0u, 0u, 0u);
-        odb[i] = make_uint4(0u, 0u, 0u, 0u);
-      }
+      for (int i = 0; i < 16; ++i) pda[i] = pdb[i] = 0u;
+    }
+    if (cr.keep_pad) {
+      store_chunk(dab_map, pda, col0, cr.row, cr.grp, stage, ochunk);
+      store_chunk(dab_map, pdb, p.F + col0, cr.row, cr.grp, stage, ochunk);
     }
   }
   if (valid) p.dgate_part[rrow * p.dgate_ld + nt] = part;
@@ -578,9 +602,9 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) +
                              static_cast<uint32_t>(pipe.acc * gemm::kAccCols);
       if (p.mode == kRecompute) {
-        epi_recompute(p, tbase, g, row, valid, nt);
+        epi_recompute(p, &tout1, &tout2, tbase, g, row0, valid, nt, stage, ochunk);
       } else if (p.mode == kDh) {
-        epi_dh(p, tbase, g, row, valid, nt);
+        epi_dh(p, &tout1, tbase, g, row0, valid, nt, stage, ochunk);
       } else if (p.mode == kDx) {
         uint16_t* orow = static_cast<uint16_t*>(p.out) + row_of(p, g, row) * p.out_ld + nt * p.width;
         gemm::store_bf16(tbase, p.width, orow, valid);
@@ -936,7 +960,8 @@ bool use_pair(const RowBlocks& b, long long n_tiles) {
 
 // One launch of up to three GEMM phases (maps a[q], b[q], args[q]); tiles = the sum of their tiles
 // (single-CTA form; the pair form runs one cluster per pair of SMs and counts tiles on the device).
-// out: fp32 output maps of phases 1 and 2 (their weight gradients written through TMA), or null.
+// out: the epilogues' TMA-store maps out[1] and out[2] (the recompute's ab and hg, dh's dab, or
+// the fp32 weight gradients of phases 1 and 2), or null.
 cudaError_t run_gemm(const CUtensorMap* a, const CUtensorMap* b, const bwd::GemmArgs* args, int phases,
                      long long tiles, int kind, cudaStream_t stream, const CUtensorMap* out = nullptr,
                      bool pair = false) {
@@ -949,7 +974,7 @@ cudaError_t run_gemm(const CUtensorMap* a, const CUtensorMap* b, const bwd::Gemm
   const CUtensorMap& b1 = b[phases > 1 ? 1 : 0];
   const CUtensorMap& a2 = a[phases > 2 ? 2 : 0];
   const CUtensorMap& b2 = b[phases > 2 ? 2 : 0];
-  const CUtensorMap& o1 = out ? out[1] : a[0];   // unused unless a phase sets tma_out
+  const CUtensorMap& o1 = out ? out[1] : a[0];   // unused unless an epilogue stores through TMA
   const CUtensorMap& o2 = out ? out[2] : a[0];
   launch_begin(kind, stream);
   cudaError_t err;
@@ -1065,14 +1090,18 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     g.n_total = F;
     g.num_k_blocks = d / gemm::BK;
     g.out = a.ab;
-    g.out_hg = a.hg;
     g.row_gate = a.row_gate;
     CUtensorMap ma, mb;
     if ((e = gemm::make_map(&ma, a.xbuf, d, a_rows, groups, gemm::BM)) != cudaSuccess) return e;
     if ((e = gemm::make_map(&mb, a.w_gate_up, d, 2ull * F, E, pair ? pair_box : static_cast<uint32_t>(g.width))) !=
         cudaSuccess)
       return e;
-    if ((e = run_gemm(&ma, &mb, &g, 1, mt * (F / g.width), kKindBackwardRecompute, stream, nullptr, pair)) !=
+    CUtensorMap mo[3];   // the epilogue's TMA stores: 1 = ab [.][2F], 2 = hg [.][F], 32 x 32 chunks
+    if ((e = gemm::make_map(&mo[1], a.ab, 2ull * F, a_rows, groups, 32, gemm::kOutChunkCols)) != cudaSuccess ||
+        (e = gemm::make_map(&mo[2], a.hg, F, a_rows, groups, 32, gemm::kOutChunkCols)) != cudaSuccess)
+      return e;
+    mo[0] = mo[1];
+    if ((e = run_gemm(&ma, &mb, &g, 1, mt * (F / g.width), kKindBackwardRecompute, stream, mo, pair)) !=
         cudaSuccess)
       return e;
   }
@@ -1095,7 +1124,10 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     if ((e = gemm::make_map(&ma, a.dybuf, d, a_rows, groups, gemm::BM)) != cudaSuccess) return e;
     g.b_mn = 1;   // B[n = column of d_ff][k = column of d] = W2[k][n]: W2 as stored, MN-major
     if ((e = gemm::make_map(&mb, a.w_down, F, d, E, bwd::kMnBox, bwd::kMnBox)) != cudaSuccess) return e;
-    if ((e = run_gemm(&ma, &mb, &g, 1, mt * parts, kKindBackwardDh, stream, nullptr, pair)) != cudaSuccess) return e;
+    CUtensorMap mo[3];   // the epilogue's TMA stores: 1 = dab [.][2F], 32 x 32 chunks
+    if ((e = gemm::make_map(&mo[1], a.dab, 2ull * F, a_rows, groups, 32, gemm::kOutChunkCols)) != cudaSuccess) return e;
+    mo[0] = mo[2] = mo[1];
+    if ((e = run_gemm(&ma, &mb, &g, 1, mt * parts, kKindBackwardDh, stream, mo, pair)) != cudaSuccess) return e;
   }
   // one launch: dx rows = dab W13, dW2 (+)= dy^T hg and dW13 (+)= dab^T x over K = the round's
   // rows of each expert (both operands the row-major round buffers, read MN-major)
