@@ -872,15 +872,24 @@ int grid_for(long long warps_needed) {
   return static_cast<int>(blocks < 1 ? 1 : blocks < cap ? blocks : cap);
 }
 
-// Widest candidate whose tile count reaches the SM count, else the narrowest that divides n_total.
-int pick_width(const int* widths, int n_widths, long long mtiles, int n_total) {
-  int last = -1;
+// The candidate N width (dividing n_total) with the least streaming time: each SM streams a
+// tile's 128 A rows and its B rows (width x b_per_col) over the same K, once per wave of
+// tiles, so the time goes as waves x (128 + width x b_per_col). Ties go to the wider tile
+// (fewer A re-reads in all). b_per_col: 2 for the recompute (W1 and W3 rows), else 1.
+int pick_width(const int* widths, int n_widths, long long mtiles, int n_total, int b_per_col = 1) {
+  int best = -1;
+  long long best_cost = 0;
   for (int i = 0; i < n_widths; ++i) {
     if (n_total % widths[i] != 0) continue;
-    last = widths[i];
-    if (mtiles * (n_total / widths[i]) >= num_sms()) return widths[i];
+    const long long tiles = mtiles * (n_total / widths[i]);
+    const long long waves = (tiles + num_sms() - 1) / num_sms();
+    const long long cost = waves * (gemm::BM + static_cast<long long>(widths[i]) * b_per_col);
+    if (best < 0 || cost < best_cost || (cost == best_cost && widths[i] > best)) {
+      best = widths[i];
+      best_cost = cost;
+    }
   }
-  return last;
+  return best;
 }
 
 #ifndef MOE_BWD_PAIR
@@ -1086,7 +1095,7 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     const bool pair = F % 128 == 0 && use_pair(rb, F / 128);
     bwd::GemmArgs g = base;
     g.mode = bwd::kRecompute;
-    g.width = pair ? 128 : pick_width(kW, 3, mt, F);
+    g.width = pair ? 128 : pick_width(kW, 3, mt, F, 2);
     g.n_total = F;
     g.num_k_blocks = d / gemm::BK;
     g.out = a.ab;
