@@ -97,6 +97,11 @@ def measured_traffic(workload, kernel):
     return rec["bytes_per_launch"]
 
 
+# B200 datasheet figures, for the fractions reported beside the measured ones: dense bf16 tensor
+# throughput and HBM3e bandwidth.
+DATASHEET = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -559,7 +564,8 @@ def bench_backward(args, w):
                      "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{peak_src} ({tensor_key})", "traffic": None,
-                     "frac_vs_burst": achieved / peaks["bf16_tflops"], "flops_per_step": flops},
+                     "frac_vs_burst": achieved / peaks["bf16_tflops"],
+                     "frac_vs_datasheet": achieved / DATASHEET["bf16_tflops"], "flops_per_step": flops},
         "whole_pass_tflops": flops / (ms / 1e3) / 1e12,
         "pass_frac": pass_s * 1e3 / ms,
         "pass_roofline": {"ms": pass_s * 1e3, **{k + "_ms": round(v, 4) for k, v in pass_parts.items()},
@@ -725,6 +731,9 @@ def main():
         achieved, peak, unit = per_launch_units / avg_launch_s / 1e9, peaks["hbm_gbs"], "GB/s"
     layer_s, layer_parts = layer_roofline_s(w, info, rnd, peaks, peaks[tensor_key],
                                             layer.plan_tensors()["n"].cpu().numpy())
+    # the same bound with the datasheet's peaks (dense bf16 2.25 PFLOP/s, HBM3e 8 TB/s)
+    layer_ds_s, _ = layer_roofline_s(w, info, rnd, {"hbm_gbs": DATASHEET["hbm_gbs"]}, DATASHEET["bf16_tflops"],
+                                     layer.plan_tensors()["n"].cpu().numpy())
     per_kernel = {}
     for k, (c, t) in kinds.items():
         b, u = resolve(k)
@@ -847,8 +856,11 @@ def main():
                               "frac": achieved / peak,
                               "peak_source": f"{peak_src} ({tensor_key if bound == 'tensor' else 'hbm_gbs copy'})",
                               "traffic": measured_traffic(w.name, dom)},
-                             **({"frac_vs_burst": achieved / peaks["bf16_tflops"]} if bound == "tensor" else {})),
+                             **({"frac_vs_burst": achieved / peaks["bf16_tflops"]} if bound == "tensor" else {}),
+                             frac_vs_datasheet=achieved / (DATASHEET["bf16_tflops"] if bound == "tensor"
+                                                           else DATASHEET["hbm_gbs"])),
             "layer_frac": layer_s * 1e3 / (total_ms / args.steps),
+            "layer_frac_vs_datasheet": layer_ds_s * 1e3 / (total_ms / args.steps),
             "layer_roofline": dict(layer_parts, ms=layer_s * 1e3,
                                    peaks=f"{peak_src}: hbm_gbs {peaks['hbm_gbs']}, {tensor_key} {peaks[tensor_key]}",
                                    formula="router/top-k/plan/dispatch/combine bytes at HBM + sum over active "
