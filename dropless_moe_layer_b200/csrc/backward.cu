@@ -24,7 +24,9 @@
 //              <W2^T dy, h> per 64..256-column tile, dab = [da | db] (TMA stores)
 //   dx         dab W13 (tensor cores, B = W13 read MN-major as stored) -> dxbuf (bf16)
 //   combine    dx[t] = (first round of t ? 0 : dx[t]) + sum of the token's dxbuf rows, ascending
-//              j; dgate[t, j] = sum of its row's partials in tile order (no atomics anywhere)
+//              j; dgate[t, j] = sum of its row's partials in tile order (no atomics anywhere);
+//              the next round's gather runs in the same launch (other blocks), so a round after
+//              the first takes four launches
 //   wgrad      dW2 += dy^T hg and dW13 += dab^T x over K = the round's rows of each expert
 //              (tensor cores, both operands the row-major round buffers read MN-major; the fp32
 //              gradient tiles are stored in round 0, which holds every expert that has rows,
@@ -663,16 +665,17 @@ struct GatherArgs {
   int r, E, C, d, k, pooled;
 };
 
-__global__ void __launch_bounds__(256) bwd_gather_kernel(const __grid_constant__ GatherArgs a) {
+// Block (bx, by) of the gather: 64 rows (the bx-th 64-row block of the round) x 64 columns
+// (c0 = 64 by). The whole block runs it (256 threads).
+__device__ __forceinline__ void gather_block(const GatherArgs& a, int bx, int by) {
   __shared__ int tok[64];
   __shared__ int blk[3];      // expert, its first row in this block, its rows in the round
-  grid_dependency_wait();
-  const int c0 = blockIdx.y * 64;
+  const int c0 = by * 64;
   const int32_t* nr = a.n + static_cast<size_t>(a.r) * a.E;
   if (threadIdx.x < 32) {
     // warp 0: the expert whose 64-row blocks hold block b (a running prefix over the experts)
     const int lane = threadIdx.x;
-    const int b = static_cast<int>(blockIdx.x);
+    const int b = bx;
     int acc = 0, found = -1, first = 0, rows = 0;
     for (int x0 = 0; x0 < a.E; x0 += 32) {
       const int x = x0 + lane;
@@ -706,7 +709,7 @@ __global__ void __launch_bounds__(256) bwd_gather_kernel(const __grid_constant__
   if (e >= 0) {
     const int base = a.row_off[static_cast<size_t>(a.r) * a.E + e];
     // row-major row of s = 0 (pooled: this block's first row is 64 b)
-    const long long dst0 = a.pooled ? static_cast<long long>(blockIdx.x) * 64 - s0
+    const long long dst0 = a.pooled ? static_cast<long long>(bx) * 64 - s0
                                     : static_cast<long long>(e) * a.C;
     if (threadIdx.x < 64) {
       const int sr = s0 + threadIdx.x;
@@ -739,6 +742,11 @@ __global__ void __launch_bounds__(256) bwd_gather_kernel(const __grid_constant__
       }
     }
   }
+}
+
+__global__ void __launch_bounds__(256) bwd_gather_kernel(const __grid_constant__ GatherArgs a) {
+  grid_dependency_wait();
+  gather_block(a, static_cast<int>(blockIdx.x), static_cast<int>(blockIdx.y));
   pdl_trigger_early();
   pdl_trigger_late();
 }
@@ -773,13 +781,23 @@ __global__ void __launch_bounds__(32) seg_table_kernel(const int32_t* __restrict
 
 // One warp per token with pairs in round r: dx[t] (+)= its pairs' dxbuf rows (gate 1, ascending j),
 // dgate[t, j] = sum over the row's `parts` partials, in order.
-__global__ void __launch_bounds__(32 * kWarps)
-    bwd_combine_kernel(const copy::CombineArgs a, int r, const float* __restrict__ dgate_part, int dgate_ld,
-                       int parts, float* __restrict__ dgate) {
-  grid_dependency_wait();
+// The combine's arguments besides the copy step's.
+struct CombineExtra {
+  int r;
+  const float* dgate_part;
+  int dgate_ld, parts;
+  float* dgate;
+};
+
+// Block `block` of `blocks` blocks of the combine (kWarps warps each).
+__device__ __forceinline__ void combine_blocks(const copy::CombineArgs& a, const CombineExtra& x, int block,
+                                               int blocks) {
+  const int r = x.r, parts = x.parts, dgate_ld = x.dgate_ld;
+  const float* __restrict__ dgate_part = x.dgate_part;
+  float* __restrict__ dgate = x.dgate;
   const int lane = threadIdx.x & 31;
-  const int warps = gridDim.x * kWarps;
-  for (int t = blockIdx.x * kWarps + (threadIdx.x >> 5); t < a.T; t += warps) {
+  const int warps = blocks * kWarps;
+  for (int t = block * kWarps + (threadIdx.x >> 5); t < a.T; t += warps) {
     const copy::PairLoads l = copy::load_pairs(a, t);
     const copy::TokenPairs tp = copy::token_pairs(a, l, r);
     if (tp.npairs == 0) continue;
@@ -792,6 +810,31 @@ __global__ void __launch_bounds__(32 * kWarps)
       for (int i = 0; i < parts; ++i) sum += pr[i];
       dgate[static_cast<size_t>(t) * a.k + j] = sum;
     }
+  }
+}
+
+__global__ void __launch_bounds__(32 * kWarps) bwd_combine_kernel(const copy::CombineArgs a, const CombineExtra x) {
+  grid_dependency_wait();
+  combine_blocks(a, x, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x));
+  pdl_trigger_early();
+  pdl_trigger_late();
+}
+
+// The combine of round r (blocks [0, comb_blocks)) and the gather of round r + 1 (the other
+// blocks, gather block (b mod gx, b / gx) for b = blockIdx.x - comb_blocks) in one launch: the
+// combine reads only dxbuf and the dgate partials, which the gather does not write, and the
+// gather writes only what round r's GEMMs have finished reading.
+__global__ void __launch_bounds__(32 * kWarps)
+    bwd_combine_gather_kernel(const copy::CombineArgs a, const CombineExtra x, const __grid_constant__ GatherArgs g,
+                              int comb_blocks, int gx) {
+  static_assert(32 * kWarps == 256, "the gather's blocks are 256 threads");
+  grid_dependency_wait();
+  const int b = static_cast<int>(blockIdx.x);
+  if (b < comb_blocks) {
+    combine_blocks(a, x, b, comb_blocks);
+  } else {
+    const int bg = b - comb_blocks;
+    gather_block(g, bg % gx, bg / gx);
   }
   pdl_trigger_early();
   pdl_trigger_late();
@@ -1046,8 +1089,24 @@ cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_h
   return e;
 }
 
+namespace {
+
+// The gather of round r: its arguments and its 64-row blocks, expert by expert.
+bwd::GatherArgs gather_args(const BackwardArgs& a, int r) {
+  return bwd::GatherArgs{a.x, a.dy, a.idx, a.gate, a.n, a.row_off, a.row_token, a.xbuf, a.dybuf,
+                         a.row_gate, r, a.E, a.C, a.d, a.k, a.pooled != 0 ? 1 : 0};
+}
+
+long long gather_blocks(const int32_t* n_host, int E) {
+  long long blocks = 0;
+  for (int x = 0; x < E; ++x) blocks += (n_host[x] + 63) / 64;
+  return blocks;
+}
+
+}  // namespace
+
 cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n_host, int rows,
-                                  cudaStream_t stream) {
+                                  const int32_t* n_next, cudaStream_t stream) {
   (void)rows;
   const int E = a.E, C = a.C, d = a.d, F = a.F;
   const bool pooled = a.pooled != 0;
@@ -1056,15 +1115,14 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
   const uint64_t a_rows = pooled ? static_cast<uint64_t>(a.rows) : static_cast<uint64_t>(C);
   const uint64_t groups = pooled ? 1 : static_cast<uint64_t>(E);
   cudaError_t e;
-  // dispatch x and dy; the rows' gates
-  {
-    const bwd::GatherArgs ga{a.x, a.dy, a.idx, a.gate, a.n, a.row_off, a.row_token, a.xbuf, a.dybuf,
-                             a.row_gate, r, E, C, d, a.k, pooled ? 1 : 0};
-    long long blocks = 0;   // the round's 64-row blocks, expert by expert
-    for (int x = 0; x < E; ++x) blocks += (n_host[x] + 63) / 64;
+  // dispatch x and dy; the rows' gates (rounds after the first: in the previous round's combine
+  // launch)
+  if (r == 0) {
+    const long long blocks = gather_blocks(n_host, E);
     if (blocks > 0) {
       launch_begin(kKindBackwardCopy, stream);
-      e = launch_pdl(bwd::bwd_gather_kernel, dim3(static_cast<unsigned>(blocks), d / 64), dim3(256), 0, stream, ga);
+      e = launch_pdl(bwd::bwd_gather_kernel, dim3(static_cast<unsigned>(blocks), d / 64), dim3(256), 0, stream,
+                     gather_args(a, r));
       launch_end(kKindBackwardCopy, stream);
       if (e != cudaSuccess) return e;
     }
@@ -1192,14 +1250,21 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     mo[0] = ma[0];
     if ((e = run_gemm(ma, mb, g, 3, tiles, kKindBackwardDxWgrad, stream, mo, pair)) != cudaSuccess) return e;
   }
-  // combine dx and gather dgate
+  // combine dx and gather dgate; with the next round's gather in the same launch
   {
     // pooled rows: the pair's row is seg_off[r][e] - zeros[r] + slot
     const copy::CombineArgs ca{a.dxbuf, a.dx, a.idx, a.ones, a.round, a.slot, a.T, a.k, C, d,
                                pooled ? a.seg_off : nullptr, pooled ? a.zeros : nullptr, E};
+    const bwd::CombineExtra cx{r, a.dgate_part, F / 64, parts, a.dgate};
+    const int comb_blocks = grid_for(a.T);
+    const long long next_blocks = n_next ? gather_blocks(n_next, E) * (d / 64) : 0;
     launch_begin(kKindBackwardCopy, stream);
-    e = launch_pdl(bwd::bwd_combine_kernel, dim3(grid_for(a.T)), dim3(32 * bwd::kWarps), 0, stream, ca, r,
-                   static_cast<const float*>(a.dgate_part), F / 64, parts, a.dgate);
+    if (next_blocks > 0)
+      e = launch_pdl(bwd::bwd_combine_gather_kernel, dim3(static_cast<unsigned>(comb_blocks + next_blocks)),
+                     dim3(32 * bwd::kWarps), 0, stream, ca, cx, gather_args(a, r + 1), comb_blocks,
+                     static_cast<int>(next_blocks / (d / 64)));
+    else
+      e = launch_pdl(bwd::bwd_combine_kernel, dim3(comb_blocks), dim3(32 * bwd::kWarps), 0, stream, ca, cx);
     launch_end(kKindBackwardCopy, stream);
   }
   return e;

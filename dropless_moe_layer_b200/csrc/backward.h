@@ -64,10 +64,12 @@ long long backward_rows(int E, int C, bool pooled);
 // the unit gates, and writes the segment table seg_off of the R rounds (from the plan's n on the
 // device) and the zero words.
 cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_host, int R, cudaStream_t stream);
-// One round: dispatch, recompute, dh (+ SwiGLU backward), dx GEMM, dx combine and dgate, weight
-// gradients. n_host / rows: the round's rows per expert and in total.
+// One round: dispatch (round 0 only), recompute, dh (+ SwiGLU backward), dx GEMM and weight
+// gradients, dx combine and dgate. n_host / rows: the round's rows per expert and in total;
+// n_next: the next round's rows per expert, whose dispatch then runs in this round's combine
+// launch (null after the last round).
 cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n_host, int rows,
-                                  cudaStream_t stream);
+                                  const int32_t* n_next, cudaStream_t stream);
 // dz from dgate and the logits, after the last round.
 cudaError_t launch_backward_gates(const BackwardArgs& a, cudaStream_t stream);
 

@@ -508,11 +508,16 @@ int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws
   a.pooled = borrowing(shape) ? 1 : 0;
   a.rows = B.rows;
   if ((st = cuda_status(launch_backward_prepare(a, info->load, info->R, stream))) != MOE_OK) return st;
+  int32_t n_rounds[2][MOE_MAX_EXPERTS];
+  int rows[2] = {0, 0};
+  if (info->R > 0) round_rows(shape, info, 0, n_rounds[0], &rows[0]);
   for (int r = 0; r < info->R; ++r) {
-    int32_t n_host[MOE_MAX_EXPERTS];
-    int rows = 0;
-    round_rows(shape, info, r, n_host, &rows);
-    if ((st = cuda_status(launch_backward_round(a, r, n_host, rows, stream))) != MOE_OK) return st;
+    const int cur = r & 1, nxt = cur ^ 1;
+    const bool more = r + 1 < info->R;
+    if (more) round_rows(shape, info, r + 1, n_rounds[nxt], &rows[nxt]);
+    if ((st = cuda_status(launch_backward_round(a, r, n_rounds[cur], rows[cur], more ? n_rounds[nxt] : nullptr,
+                                                stream))) != MOE_OK)
+      return st;
   }
   return cuda_status(launch_backward_gates(a, stream));
 }
