@@ -1047,7 +1047,10 @@ cudaError_t run_gemm(const CUtensorMap* a, const CUtensorMap* b, const bwd::Gemm
     cfg.numAttrs = 2;
     err = cudaLaunchKernelEx(&cfg, bwd::bwd_gemm_kernel<true>, a[0], b[0], a1, b1, a2, b2, o1, o2, L);
   } else {
-    const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
+    // the fewest CTAs that take the tiles in as many waves as one CTA per SM would: the SMs left
+    // over serve the other stream's launches when two rounds overlap
+    const long long waves = (tiles + num_sms() - 1) / num_sms();
+    const int grid = static_cast<int>((tiles + waves - 1) / waves);
     err = launch_pdl(bwd::bwd_gemm_kernel<false>, dim3(grid), dim3(gemm::kThreads), bwd::kSmemBytes, stream, a[0],
                      b[0], a1, b1, a2, b2, o1, o2, L);
   }
@@ -1059,6 +1062,11 @@ cudaError_t run_gemm(const CUtensorMap* a, const CUtensorMap* b, const bwd::Gemm
 
 long long backward_rows(int E, int C, bool pooled) {
   return static_cast<long long>(E) * C + (pooled ? 64ll * E : 0ll);
+}
+
+long long backward_rows2(int E, int C) {
+  const long long eighth = (static_cast<long long>(E) * C + 7) / 8;
+  return (eighth + 63) / 64 * 64 + 64ll * E;
 }
 
 cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_host, int R, cudaStream_t stream) {
@@ -1105,19 +1113,62 @@ long long gather_blocks(const int32_t* n_host, int E) {
 
 }  // namespace
 
-cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n_host, int rows,
-                                  const int32_t* n_next, cudaStream_t stream) {
-  (void)rows;
-  const int E = a.E, C = a.C, d = a.d, F = a.F;
+namespace {
+
+// What the launches of one round share: the round's row counts, its row blocks and the GEMMs'
+// common arguments, and the round buffers' 3-D map extents ([E][C][K] per expert, or pooled
+// [1][rows][K]).
+struct RoundGeom {
+  long long mt = 0;     // 128-row blocks of the round
+  int active = 0;       // experts with rows
+  RowBlocks rb;
+  bwd::GemmArgs base{};
+  uint64_t a_rows = 0, groups = 0;
+};
+
+RoundGeom round_geom(const BackwardArgs& a, int r, const int32_t* n_host) {
+  RoundGeom q;
+  const int E = a.E;
   const bool pooled = a.pooled != 0;
-  const int32_t* n_dev = a.n + static_cast<size_t>(r) * E;
-  // round buffers as 3-D maps: [E][C][K] per expert, or pooled [1][rows][K]
-  const uint64_t a_rows = pooled ? static_cast<uint64_t>(a.rows) : static_cast<uint64_t>(C);
-  const uint64_t groups = pooled ? 1 : static_cast<uint64_t>(E);
+  for (int g = 0; g < E; ++g) {
+    q.mt += (n_host[g] + gemm::BM - 1) / gemm::BM;
+    q.active += n_host[g] > 0 ? 1 : 0;
+  }
+  q.rb = row_blocks(n_host, E);
+  q.base.rows = a.n + static_cast<size_t>(r) * E;
+  q.base.groups = E;
+  q.base.C = a.C;
+  q.base.F = a.F;
+  q.base.group_row = pooled ? a.seg_off + static_cast<size_t>(r) * E : nullptr;   // 64-aligned segments
+  q.base.group_row_base = pooled ? a.zeros + r : nullptr;
+  q.base.status = a.status;
+  q.a_rows = pooled ? static_cast<uint64_t>(a.rows) : static_cast<uint64_t>(a.C);
+  q.groups = pooled ? 1 : static_cast<uint64_t>(E);
+  return q;
+}
+
+constexpr int kWide[3] = {256, 128, 64};
+
+}  // namespace
+
+bool backward_front_is_thin(const BackwardArgs& a, const int32_t* n_host) {
+  const int F = a.F;
+  long long mt = 0;
+  for (int g = 0; g < a.E; ++g) mt += (n_host[g] + gemm::BM - 1) / gemm::BM;
+  const RowBlocks rb = row_blocks(n_host, a.E);
+  static const int kW[3] = {128, 64, 32};
+  if ((F % 128 == 0 && use_pair(rb, F / 128)) || (F % 256 == 0 && use_pair(rb, F / 256))) return false;
+  const long long rec = mt * (F / pick_width(kW, 3, mt, F, 2));
+  const long long dh = mt * (F / pick_width(kWide, 3, mt, F));
+  return rec < num_sms() && dh < num_sms();
+}
+
+cudaError_t launch_backward_front(const BackwardArgs& a, int r, const int32_t* n_host, bool gather, int* parts_out,
+                                  cudaStream_t stream) {
+  const int E = a.E, d = a.d, F = a.F;
   cudaError_t e;
-  // dispatch x and dy; the rows' gates (rounds after the first: in the previous round's combine
-  // launch)
-  if (r == 0) {
+  // dispatch x and dy; the rows' gates
+  if (gather) {
     const long long blocks = gather_blocks(n_host, E);
     if (blocks > 0) {
       launch_begin(kKindBackwardCopy, stream);
@@ -1127,23 +1178,11 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
       if (e != cudaSuccess) return e;
     }
   }
-
-  long long mt = 0;
-  int active = 0;
-  for (int g = 0; g < E; ++g) {
-    mt += (n_host[g] + gemm::BM - 1) / gemm::BM;
-    active += n_host[g] > 0 ? 1 : 0;
-  }
-  const RowBlocks rb = row_blocks(n_host, E);
-  bwd::GemmArgs base{};
-  base.rows = n_dev;
-  base.groups = E;
-  base.C = C;
-  base.F = F;
-  base.group_row = pooled ? a.seg_off + static_cast<size_t>(r) * E : nullptr;   // 64-aligned segments
-  base.group_row_base = pooled ? a.zeros + r : nullptr;
-  base.status = a.status;
-  static const int kWide[3] = {256, 128, 64};
+  const RoundGeom q = round_geom(a, r, n_host);
+  const long long mt = q.mt;
+  const RowBlocks& rb = q.rb;
+  const bwd::GemmArgs& base = q.base;
+  const uint64_t a_rows = q.a_rows, groups = q.groups;
   // pair form: 256-row tiles, 128 B rows per CTA (recompute: 128 W1 rows and the same W3 rows)
   const uint32_t pair_box = gemm::kPairBHalf;
 
@@ -1196,6 +1235,21 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
     mo[0] = mo[2] = mo[1];
     if ((e = run_gemm(&ma, &mb, &g, 1, mt * parts, kKindBackwardDh, stream, mo, pair)) != cudaSuccess) return e;
   }
+  *parts_out = parts;
+  return cudaSuccess;
+}
+
+cudaError_t launch_backward_back(const BackwardArgs& a, int r, const int32_t* n_host, int parts,
+                                 const BackwardArgs* a_next, const int32_t* n_next, cudaStream_t stream) {
+  const int E = a.E, C = a.C, d = a.d, F = a.F;
+  const bool pooled = a.pooled != 0;
+  cudaError_t e;
+  const RoundGeom q = round_geom(a, r, n_host);
+  const long long mt = q.mt;
+  const int active = q.active;
+  const RowBlocks& rb = q.rb;
+  const bwd::GemmArgs& base = q.base;
+  const uint64_t a_rows = q.a_rows, groups = q.groups;
   // one launch: dx rows = dab W13, dW2 (+)= dy^T hg and dW13 (+)= dab^T x over K = the round's
   // rows of each expert (both operands the row-major round buffers, read MN-major)
   {
@@ -1257,11 +1311,11 @@ cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n
                                pooled ? a.seg_off : nullptr, pooled ? a.zeros : nullptr, E};
     const bwd::CombineExtra cx{r, a.dgate_part, F / 64, parts, a.dgate};
     const int comb_blocks = grid_for(a.T);
-    const long long next_blocks = n_next ? gather_blocks(n_next, E) * (d / 64) : 0;
+    const long long next_blocks = a_next && n_next ? gather_blocks(n_next, E) * (d / 64) : 0;
     launch_begin(kKindBackwardCopy, stream);
     if (next_blocks > 0)
       e = launch_pdl(bwd::bwd_combine_gather_kernel, dim3(static_cast<unsigned>(comb_blocks + next_blocks)),
-                     dim3(32 * bwd::kWarps), 0, stream, ca, cx, gather_args(a, r + 1), comb_blocks,
+                     dim3(32 * bwd::kWarps), 0, stream, ca, cx, gather_args(*a_next, r + 1), comb_blocks,
                      static_cast<int>(next_blocks / (d / 64)));
     else
       e = launch_pdl(bwd::bwd_combine_kernel, dim3(comb_blocks), dim3(32 * bwd::kWarps), 0, stream, ca, cx);

@@ -60,16 +60,26 @@ struct BackwardArgs {
 // Rows of the per-round buffers: E * C per expert (expert e's rows at e * C), or with pooled rows
 // E * C + 64 E (each expert's segment rounded up to 64 rows, in expert order).
 long long backward_rows(int E, int C, bool pooled);
+// Rows of the second, smaller buffer set (always pooled): E * C / 8 rounded up to 64, plus 64 E.
+long long backward_rows2(int E, int C);
 // Zeroes the weight gradients of experts without rows (load_host: host copy of the loads), fills
 // the unit gates, and writes the segment table seg_off of the R rounds (from the plan's n on the
 // device) and the zero words.
 cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_host, int R, cudaStream_t stream);
-// One round: dispatch (round 0 only), recompute, dh (+ SwiGLU backward), dx GEMM and weight
-// gradients, dx combine and dgate. n_host / rows: the round's rows per expert and in total;
-// n_next: the next round's rows per expert, whose dispatch then runs in this round's combine
-// launch (null after the last round).
-cudaError_t launch_backward_round(const BackwardArgs& a, int r, const int32_t* n_host, int rows,
-                                  const int32_t* n_next, cudaStream_t stream);
+// A round in two halves, each on a stream of its own choosing. n_host: the round's rows per
+// expert. a: the round's buffer set (its pointers, pooled and rows).
+// Whether a round's front half runs in the single-CTA form with fewer tiles per GEMM than the
+// device has SMs (so that it leaves SMs to the round before's back half).
+bool backward_front_is_thin(const BackwardArgs& a, const int32_t* n_host);
+// Front: the dispatch of x and dy (when `gather`; else the previous round's combine launch ran
+// it), the recompute and dh (+ the SwiGLU backward); *parts: dgate partials per row, for the back.
+cudaError_t launch_backward_front(const BackwardArgs& a, int r, const int32_t* n_host, bool gather, int* parts,
+                                  cudaStream_t stream);
+// Back: the dx GEMM and the weight gradients (one launch), the dx combine and dgate. With a_next
+// and n_next (the next round's buffer set and rows per expert) the next round's dispatch runs in
+// the combine's launch.
+cudaError_t launch_backward_back(const BackwardArgs& a, int r, const int32_t* n_host, int parts,
+                                 const BackwardArgs* a_next, const int32_t* n_next, cudaStream_t stream);
 // dz from dgate and the logits, after the last round.
 cudaError_t launch_backward_gates(const BackwardArgs& a, cudaStream_t stream);
 

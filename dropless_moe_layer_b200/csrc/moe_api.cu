@@ -414,11 +414,54 @@ void make_backward_layout(const moe_shape_t* s, moe_backward_layout_t* L) {
   L->ones = take(T * k * 4);
   L->seg_off = take(mr * E * 4);
   L->zeros = take((mr + 1) * 4);
+  // the second buffer set (none with MOE_FLAG_PER_ROUND, which runs the rounds one at a time)
+  const long long rows2 = (s->flags & MOE_FLAG_PER_ROUND) ? 0 : backward_rows2(s->E, s->C);
+  L->xbuf2 = take(rows2 * d * 2);
+  L->dybuf2 = take(rows2 * d * 2);
+  L->row_gate2 = take(rows2 * 4);
+  L->ab2 = take(rows2 * 2 * F * 2);
+  L->hg2 = take(rows2 * F * 2);
+  L->dab2 = take(rows2 * 2 * F * 2);
+  L->dgate_part2 = take(rows2 * (F / 64) * 4);
+  L->dxbuf2 = take(rows2 * d * 2);
+  if (rows2 == 0) L->xbuf2 = L->dybuf2 = L->row_gate2 = L->ab2 = L->hg2 = L->dab2 = L->dgate_part2 = L->dxbuf2 = 0;
   L->total_bytes = off;
   L->rows = static_cast<int32_t>(rows);
+  L->rows2 = static_cast<int32_t>(rows2);
 }
 
 // The per-round buffers' rows (and the element offsets within them) must fit int32.
+// The backward's second stream (the highest priority: it carries the rounds' serial back
+// halves) and its events, per host thread and device, created on first use.
+struct SideStream {
+  cudaStream_t stream;
+  cudaEvent_t front, back[2];
+};
+
+cudaError_t side_stream(SideStream* out) {
+  thread_local SideStream cache[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  SideStream& c = cache[dev & 63];
+  if (c.stream == nullptr) {
+    SideStream n{};
+    int least = 0, greatest = 0;
+    if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess ||
+        (e = cudaStreamCreateWithPriority(&n.stream, cudaStreamNonBlocking, greatest)) != cudaSuccess)
+      return e;
+    if ((e = cudaEventCreateWithFlags(&n.front, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&n.back[0], cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&n.back[1], cudaEventDisableTiming)) != cudaSuccess) {
+      cudaStreamDestroy(n.stream);
+      return e;
+    }
+    c = n;
+  }
+  *out = c;
+  return cudaSuccess;
+}
+
 bool backward_shape_ok(const moe_shape_t* s) {
   const long long rows = backward_rows(s->E, s->C, (s->flags & MOE_FLAG_BORROW) != 0);
   return rows * 2 * s->d_ff < (1ll << 31) && rows * s->d < (1ll << 31);
@@ -507,16 +550,80 @@ int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws
   a.renorm = (shape->flags & MOE_FLAG_RENORM_TOPK) ? 1 : 0;
   a.pooled = borrowing(shape) ? 1 : 0;
   a.rows = B.rows;
+  // The second buffer set: a thin round (its front half's GEMMs have fewer tiles than the device
+  // has SMs) whose pooled rows fit in it runs there when the round before ran in the first set,
+  // so that its front half (dispatch, recompute, dh) on the caller's stream overlaps the round
+  // before's back half (dx and weight gradients, combine) on a second stream. Large rounds are
+  // not overlapped: two GEMM launches that each fill the device only slow each other down.
+  // The back halves keep their round order on that stream (the fp32 weight gradients and dx are
+  // accumulated round by round), so the results are those of running the rounds one at a time.
+  BackwardArgs a2 = a;
+  SideStream side{};
+  bool overlap = B.rows2 > 0 && info->R > 1;
+  if (overlap) {
+    a2.xbuf = at<uint16_t>(bws, B.xbuf2);
+    a2.dybuf = at<uint16_t>(bws, B.dybuf2);
+    a2.row_gate = at<float>(bws, B.row_gate2);
+    a2.ab = at<uint16_t>(bws, B.ab2);
+    a2.hg = at<uint16_t>(bws, B.hg2);
+    a2.dab = at<uint16_t>(bws, B.dab2);
+    a2.dgate_part = at<float>(bws, B.dgate_part2);
+    a2.dxbuf = at<uint16_t>(bws, B.dxbuf2);
+    a2.pooled = 1;
+    a2.rows = B.rows2;
+    if ((st = cuda_status(side_stream(&side))) != MOE_OK) return st;
+  }
   if ((st = cuda_status(launch_backward_prepare(a, info->load, info->R, stream))) != MOE_OK) return st;
   int32_t n_rounds[2][MOE_MAX_EXPERTS];
   int rows[2] = {0, 0};
+  auto pooled_rows = [&](const int32_t* n) {
+    long long p = 0;
+    for (int e = 0; e < shape->E; ++e) p += (n[e] + 63) / 64 * 64;
+    return p;
+  };
+  // set of round r + 1 given round r's: the second set only right after the first
+  auto next_set = [&](int set, const int32_t* n_next) {
+    return overlap && set == 0 && pooled_rows(n_next) <= B.rows2 && backward_front_is_thin(a2, n_next) ? 1 : 0;
+  };
   if (info->R > 0) round_rows(shape, info, 0, n_rounds[0], &rows[0]);
+  int set = 0;
+  bool gathered = false;     // the round's dispatch ran in the previous round's combine launch
+  bool back_used[2] = {false, false};
+  cudaStream_t back_stream = overlap ? side.stream : stream;
   for (int r = 0; r < info->R; ++r) {
     const int cur = r & 1, nxt = cur ^ 1;
     const bool more = r + 1 < info->R;
     if (more) round_rows(shape, info, r + 1, n_rounds[nxt], &rows[nxt]);
-    if ((st = cuda_status(launch_backward_round(a, r, n_rounds[cur], rows[cur], more ? n_rounds[nxt] : nullptr,
-                                                stream))) != MOE_OK)
+    const BackwardArgs& ar = set ? a2 : a;
+    // front half on the caller's stream, after the last back half that read this set
+    if (overlap && back_used[set] && (st = cuda_status(cudaStreamWaitEvent(stream, side.back[set], 0))) != MOE_OK)
+      return st;
+    int parts = 0;
+    if ((st = cuda_status(launch_backward_front(ar, r, n_rounds[cur], !gathered, &parts, stream))) != MOE_OK)
+      return st;
+    // back half: the next round's dispatch joins its combine launch when the next round uses
+    // the same set (its front half waits for this back half anyway)
+    const int set_next = more ? next_set(set, n_rounds[nxt]) : 0;
+    const bool merge = more && set_next == set;
+    if (overlap) {
+      if ((st = cuda_status(cudaEventRecord(side.front, stream))) != MOE_OK ||
+          (st = cuda_status(cudaStreamWaitEvent(back_stream, side.front, 0))) != MOE_OK)
+        return st;
+    }
+    if ((st = cuda_status(launch_backward_back(ar, r, n_rounds[cur], parts, merge ? &ar : nullptr,
+                                               merge ? n_rounds[nxt] : nullptr, back_stream))) != MOE_OK)
+      return st;
+    if (overlap) {
+      if ((st = cuda_status(cudaEventRecord(side.back[set], back_stream))) != MOE_OK) return st;
+      back_used[set] = true;
+    }
+    gathered = merge;
+    set = set_next;
+  }
+  // dz after the last combine (the back halves ran in round order on the second stream)
+  if (overlap) {
+    if ((st = cuda_status(cudaEventRecord(side.front, back_stream))) != MOE_OK ||
+        (st = cuda_status(cudaStreamWaitEvent(stream, side.front, 0))) != MOE_OK)
       return st;
   }
   return cuda_status(launch_backward_gates(a, stream));

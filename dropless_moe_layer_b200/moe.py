@@ -55,7 +55,9 @@ class BackwardLayout(ctypes.Structure):
     _fields_ = [(name, c_sz) for name in (
         "total_bytes", "xbuf", "dybuf", "row_gate", "ab", "hg", "dab", "dgate_part", "dxbuf", "dgate",
         "ones", "seg_off", "zeros")
-    ] + [("rows", c_i32)]
+    ] + [("rows", c_i32)] + [(name, c_sz) for name in (
+        "xbuf2", "dybuf2", "row_gate2", "ab2", "hg2", "dab2", "dgate_part2", "dxbuf2")
+    ] + [("rows2", c_i32)]
 
 
 class MoeError(RuntimeError):

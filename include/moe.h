@@ -256,9 +256,16 @@ typedef struct moe_backward_layout {
   size_t dxbuf;       /* bf16 [rows, d]      per-pair dx rows of the round */
   size_t dgate;       /* f32  [T, k]         dL/dgate */
   size_t ones;        /* f32  [T, k]         unit gates of the dx combine */
-  size_t seg_off;     /* i32  [max_rounds, E] MOE_FLAG_BORROW: first row of each expert's segment */
+  size_t seg_off;     /* i32  [max_rounds, E] first row of each expert's segment in pooled rows */
   size_t zeros;       /* i32  [max_rounds + 1] zeros (row offsets of the segment tables) */
   int32_t rows;       /* rows of the per-round buffers (above) */
+  /* A second, smaller set of the per-round buffers, laid out like the first but with rows2 =
+     E * C / 8 (rounded up to 64) + 64 * E rows, always pooled (expert e's rows of the round at
+     seg_off[r][e] + slot). A round whose pooled rows fit runs in it when the round before ran in
+     the first set, so that its dispatch, recompute and dh overlap that round's dx, weight
+     gradients and combine (unless MOE_FLAG_PER_ROUND). */
+  size_t xbuf2, dybuf2, row_gate2, ab2, hg2, dab2, dgate_part2, dxbuf2;
+  int32_t rows2;
 } moe_backward_layout_t;
 
 /* Bytes of the backward workspace for `shape` (0 for an invalid shape). */

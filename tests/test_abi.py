@@ -138,18 +138,30 @@ def test_forward_argument_errors_without_gpu(lib):
     assert lib.moe_forward(P(sb), P(info), ws, need_b, 4096, 4096, 4096, 4096, None) == -1
 
 
-def _backward_bytes_model(w, borrow=False):
+def _backward_rows2(w, per_round=False):
+    """Rows of the second buffer set: E*C/8 rounded up to 64, plus 64 per expert (none with the
+    per-round flag)."""
+    if per_round:
+        return 0
+    return (-(-w.E * w.C // 8) + 63) // 64 * 64 + 64 * w.E
+
+
+def _backward_bytes_model(w, borrow=False, per_round=False):
     """Backward workspace from its layout rules: per-round buffers of E*C rows (with borrowing
     E*C + 64*E: each expert's segment starts at a multiple of 64), [T, k] dgate and unit gates,
-    the segment table [max_rounds, E] and max_rounds + 1 zero words. No copy of the weights and
-    no transposed copy of the activations."""
+    the segment table [max_rounds, E], max_rounds + 1 zero words, and the second set of the
+    per-round buffers. No copy of the weights and no transposed copy of the activations."""
     def a(n):
         return (n + 255) // 256 * 256
     T, E, k, C, d, F = w.T, w.E, w.k, w.C, w.d, w.F
+
+    def round_buffers(rows):
+        return (3 * a(rows * d * 2) + a(rows * 4) + 2 * a(rows * 2 * F * 2) + a(rows * F * 2)
+                + a(rows * (F // 64) * 4))
     rows = E * C + (64 * E if borrow else 0)
     mr = (T + C - 1) // C
-    return (3 * a(rows * d * 2) + a(rows * 4) + 2 * a(rows * 2 * F * 2) + a(rows * F * 2)
-            + a(rows * (F // 64) * 4) + 2 * a(T * k * 4) + a(mr * E * 4) + a((mr + 1) * 4))
+    return (round_buffers(rows) + 2 * a(T * k * 4) + a(mr * E * 4) + a((mr + 1) * 4)
+            + round_buffers(_backward_rows2(w, per_round)))
 
 
 @pytest.mark.parametrize("w", wl.WORKLOADS, ids=lambda w: w.name)
@@ -162,9 +174,16 @@ def test_backward_workspace_is_fixed_by_shape(lib, w):
     offs = [lay.xbuf, lay.dybuf, lay.row_gate, lay.ab, lay.hg, lay.dab, lay.dgate_part, lay.dxbuf, lay.dgate,
             lay.ones, lay.seg_off, lay.zeros]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert lay.rows2 == _backward_rows2(w)
+    offs2 = [lay.xbuf2, lay.dybuf2, lay.row_gate2, lay.ab2, lay.hg2, lay.dab2, lay.dgate_part2, lay.dxbuf2]
+    assert offs2 == sorted(offs2) and offs2[0] > lay.zeros and all(o % 256 == 0 for o in offs2)
     sb = moe.make_shape(w.T, w.d, w.E, w.k, w.F, w.C, borrow=True)
     assert moe.backward_workspace_bytes(sb) == _backward_bytes_model(w, borrow=True)
     assert moe.backward_layout(sb).rows == w.E * w.C + 64 * w.E
+    sp = moe.make_shape(w.T, w.d, w.E, w.k, w.F, w.C, schedule="per_round")
+    assert moe.backward_workspace_bytes(sp) == _backward_bytes_model(w, per_round=True)
+    lp = moe.backward_layout(sp)
+    assert lp.rows2 == 0 and lp.xbuf2 == 0 and lp.dxbuf2 == 0
     s.flags = 32          # not a flag
     assert moe.backward_workspace_bytes(s) == 0
 

@@ -102,6 +102,36 @@ def test_backward_is_deterministic():
         assert torch.equal(g1[n], g2[n]), n
 
 
+OVERLAP_CASES = ["4k-zipf1", "16k-hot-expert", "C1", "C130"]
+
+
+@pytest.mark.parametrize("name", OVERLAP_CASES)
+def test_backward_overlapped_rounds_equal_one_at_a_time(name):
+    """Rounds in the second buffer set overlap the round before (two streams); the per-round
+    schedule runs every round in the first set, one after another. The gradients are bitwise
+    equal: the weight gradients and dx are accumulated in round order either way, and a round's
+    arithmetic does not depend on which set its rows live in."""
+    if name in wl.BY_NAME:
+        w = wl.BY_NAME[name]
+    else:
+        cfg = {"C1": EDGE[1], "C130": EDGE[7]}[name]
+        w = wl.custom(name="edge", T=cfg["T"], d=cfg["d"], E=cfg["E"], k=cfg["k"], F=cfg["F"], C=cfg["C"],
+                      bias="zipf", zipf_s=1.0, seed=cfg["T"])
+    inp = wl.generate(w, "cuda")
+    dy = wl.generate_dy(w, "cuda")
+    out = {}
+    for sched in ("auto", "per_round"):
+        layer = moe.DroplessMoE(w.T, w.d, w.E, w.k, w.F, w.C, schedule=sched)
+        layer(inp["x"], inp["w_gate_up"], inp["w_down"], logits=inp["logits"])
+        assert layer.info.R >= 3
+        out[sched] = layer.backward(inp["x"], inp["w_gate_up"], inp["w_down"], dy)
+        torch.cuda.synchronize()
+        assert layer.device_status() == 0
+        del layer
+    for n in NAMES:
+        assert torch.equal(out["auto"][n], out["per_round"][n]), n
+
+
 def test_backward_empty_batch():
     """No tokens: no rounds; the weight gradients are all zero."""
     layer = moe.DroplessMoE(0, 128, 8, 2, 128, 16)
