@@ -409,8 +409,11 @@ BWD_METRIC = ("routed tokens/s per MoE layer backward with per-round recompute (
               "% of tensor roofline")
 
 
-# Tensor-core flops per routed pair, in units of d * d_ff, of each backward GEMM launch kind.
-BWD_KIND_FLOPS = {"backward_recompute": 4, "backward_dh": 2, "backward_dx_wgrad": 10}
+# Tensor-core flops per routed pair, in units of d * d_ff, of each backward GEMM launch kind. The
+# recompute and dh run as two launches in rounds whose GEMMs use the CTA-pair form and as one
+# (backward_recompute_dh) in the others, so they are rated together ("front" GEMMs).
+BWD_KIND_FLOPS = {"backward_recompute": 4, "backward_dh": 2, "backward_recompute_dh": 6, "backward_dx_wgrad": 10}
+BWD_FRONT_KINDS = ("backward_recompute", "backward_dh", "backward_recompute_dh")
 
 
 def backward_flops(w):
@@ -549,6 +552,7 @@ def bench_backward(args, w):
     peaks, peak_src = load_peaks()
     flops = backward_flops(w)
     gemm_ms = sum(prof[k][1] for k in moe.BACKWARD_GEMM_KINDS if k in prof)
+    front_ms = sum(prof[k][1] for k in BWD_FRONT_KINDS if k in prof)
     achieved = flops / (gemm_ms / 1e3) / 1e12
     power_capped = bool(clk and "sw_power_cap" in clk.get("reasons", []))
     tensor_key = "bf16_tflops_sustained" if power_capped and "bf16_tflops_sustained" in peaks else "bf16_tflops"
@@ -574,8 +578,9 @@ def bench_backward(args, w):
                                      "bytes at the copy peak); copies at the copy peak"},
         "kernels": {k: dict({"launches": c, "ms": round(t, 4)},
                             **({"TFLOP/s": round(BWD_KIND_FLOPS[k] * w.T * w.k * w.d * w.F / (t / 1e3) / 1e12, 1)}
-                               if k in BWD_KIND_FLOPS else {}))
+                               if k == "backward_dx_wgrad" else {}))
                     for k, (c, t) in prof.items()},
+        "front_gemms_TFLOP/s": round(6 * w.T * w.k * w.d * w.F / (front_ms / 1e3) / 1e12, 1) if front_ms > 0 else None,
         "cpu_baseline": None if args.no_cpu_baseline else backward_cpu_baseline(w),
         "gpu_launches": launches,
         "clocks": clk,

@@ -22,6 +22,10 @@
 //   dh         W2^T dy as dybuf (W2^T)^T (tensor cores, B = W2 read MN-major as stored);
 //              epilogue: the SwiGLU backward (da, db from a, b and the gate), dgate partial sums
 //              <W2^T dy, h> per 64..256-column tile, dab = [da | db] (TMA stores)
+//              Rounds whose GEMMs run in the single-CTA form may run recompute and dh as one
+//              launch (kRecDh, when it streams less per SM than two launches): a tile of 64 d_ff
+//              columns accumulates [a | b] and W2^T dy side by side in TMEM, and one epilogue
+//              writes hg and dab from fp32 a and b (ab is not written).
 //   dx         dab W13 (tensor cores, B = W13 read MN-major as stored) -> dxbuf (bf16)
 //   combine    dx[t] = (first round of t ? 0 : dx[t]) + sum of the token's dxbuf rows, ascending
 //              j; dgate[t, j] = sum of its row's partials in tile order (no atomics anywhere);
@@ -35,7 +39,7 @@
 // After the last round: dz from dgate and the logits (one warp per token).
 //
 // Every operand of a tensor-core step is bf16 (fp32 accumulate); a and b are kept as bf16 between
-// the recompute and the dh epilogue. Rows of a tile past the expert's row count never reach a
+// the recompute and the dh epilogue (fp32 in TMEM in the fused launch). Rows of a tile past the expert's row count never reach a
 // store, except that the rows from the count up to the next multiple of 64 (within the expert's
 // C rows, or its segment) are written as zeros in xbuf, dybuf, hg and dab: the weight-gradient
 // GEMMs read K, the rows, in blocks of 64 without a mask, and with pooled rows the next expert's
@@ -59,7 +63,14 @@ using gemm::BM;
 using gemm::Pipe;
 using gemm::Smem;
 
-enum Mode : int { kRecompute = 0, kDh = 1, kDx = 2, kWgrad = 3 };
+enum Mode : int { kRecompute = 0, kDh = 1, kDx = 2, kWgrad = 3, kRecDh = 4 };
+
+// kRecDh (single-CTA form only): the recompute and dh of the same 64 d_ff columns in one tile.
+// K blocks [0, num_k_blocks) accumulate [a | b] = x W13^T (MMA N = 128) into accumulator columns
+// [0, 128), K blocks [num_k_blocks, 2 num_k_blocks) accumulate W2^T dy (N = 64, W2 read
+// MN-major) into columns [128, 192); the epilogue has a, b and W2^T dy of its rows at once, so
+// a and b are never stored.
+constexpr int kRecDhWidth = 64;
 
 struct GemmArgs {
   int mode;
@@ -112,7 +123,7 @@ __device__ __forceinline__ int tiles_of(const GemmArgs& p, int g, int n_tiles, i
 }
 
 __device__ __forceinline__ int k_blocks_of(const GemmArgs& p, int g) {
-  return p.mode == kWgrad ? (p.rows[g] + BK - 1) / BK : p.num_k_blocks;
+  return p.mode == kWgrad ? (p.rows[g] + BK - 1) / BK : p.mode == kRecDh ? 2 * p.num_k_blocks : p.num_k_blocks;
 }
 
 // Exclusive prefix over the experts of cnt(g), written to out[0 .. groups] by warp 0.
@@ -280,6 +291,83 @@ __device__ __forceinline__ void epi_dh(const GemmArgs& p, const CUtensorMap* dab
   if (valid) p.dgate_part[rrow * p.dgate_ld + nt] = part;
 }
 
+// 16 accumulator columns of this warp's 32 lanes (one row each).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// kRecDh: a, b (accumulator columns [0, 64) and [64, 128)) and W2^T dy ([128, 192)) of 64 d_ff
+// columns, all fp32, read 16 columns at a time. Per 32 columns: hg = bf16(gate * silu(a) * b)
+// into hg, then [da | db] into dab (a and b read again), through TMA stores of 32 x 32 chunks
+// (the expert's padding rows get zeros in both); the row's dgate partial <W2^T dy, h> over the
+// tile's columns goes into dgate_part.
+__device__ __forceinline__ void epi_recdh(const GemmArgs& p, const CUtensorMap* dab_map, const CUtensorMap* hg_map,
+                                          uint32_t tb, int g, int row_base, bool valid, int nt, uint8_t* stage,
+                                          uint32_t& ochunk) {
+  const int lane = threadIdx.x & 31;
+  const ChunkRows cr = chunk_rows(p, g, row_base);
+  const long long rrow = row_of(p, g, row_base + lane);
+  const float gv = valid ? p.row_gate[rrow] : 0.f;
+  float part = 0.f;
+  for (int c = 0; c < kRecDhWidth; c += 32) {
+    const int col0 = nt * kRecDhWidth + c;
+    {
+      uint32_t ph[16];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t av[16], bv[16];
+        tmem_ld16(tb + c + 16 * h, av);
+        tmem_ld16(tb + kRecDhWidth + c + 16 * h, bv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float a0 = __uint_as_float(av[2 * i]), a1 = __uint_as_float(av[2 * i + 1]);
+          const float b0 = __uint_as_float(bv[2 * i]), b1 = __uint_as_float(bv[2 * i + 1]);
+          ph[8 * h + i] = valid ? gemm::pack_bf16x2(gv * gemm::silu_f(a0) * b0, gv * gemm::silu_f(a1) * b1) : 0u;
+        }
+      }
+      if (cr.keep_pad) store_chunk(hg_map, ph, col0, cr.row, cr.grp, stage, ochunk);
+    }
+    uint32_t pda[16], pdb[16];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t av[16], bv[16], dv[16];
+      tmem_ld16(tb + c + 16 * h, av);
+      tmem_ld16(tb + kRecDhWidth + c + 16 * h, bv);
+      tmem_ld16(tb + 2 * kRecDhWidth + c + 16 * h, dv);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float dav[2], dbv[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const float a = __uint_as_float(av[2 * i + u]), b = __uint_as_float(bv[2 * i + u]);
+          const float dhu = __uint_as_float(dv[2 * i + u]);
+          const float sig = __fdividef(1.0f, 1.0f + __expf(-a));
+          const float s = a * sig;
+          part = __fmaf_rn(dhu, s * b, part);
+          const float dh = gv * dhu;
+          dbv[u] = dh * s;
+          dav[u] = dh * b * (sig * (1.0f + a * (1.0f - sig)));
+        }
+        pda[8 * h + i] = valid ? gemm::pack_bf16x2(dav[0], dav[1]) : 0u;
+        pdb[8 * h + i] = valid ? gemm::pack_bf16x2(dbv[0], dbv[1]) : 0u;
+      }
+    }
+    if (cr.keep_pad) {
+      store_chunk(dab_map, pda, col0, cr.row, cr.grp, stage, ochunk);
+      store_chunk(dab_map, pdb, p.F + col0, cr.row, cr.grp, stage, ochunk);
+    }
+  }
+  if (valid) p.dgate_part[rrow * p.dgate_ld + nt] = part;
+}
+
 // fp32 gradient tile row: out[g][row][nt * width + c] += accumulator (= accumulator when
 // `overwrite`: round 0, the first round of every expert that has rows at all).
 __device__ __forceinline__ void epi_wgrad(const GemmArgs& p, uint32_t tb, int g, int row, bool valid, int nt) {
@@ -427,7 +515,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   };
   auto map_a = [&](int q) { return q == 0 ? &ta0 : q == 1 ? &ta1 : &ta2; };
   auto map_b = [&](int q) { return q == 0 ? &tb0 : q == 1 ? &tb1 : &tb2; };
-  auto bn_of = [&](const GemmArgs& p) { return p.mode == kRecompute ? 2 * p.width : p.width; };
+  auto bn_of = [&](const GemmArgs& p) { return p.mode == kRecompute || p.mode == kRecDh ? 2 * p.width : p.width; };
   Pipe pipe;
   int32_t* status = L.ph[0].status;
 
@@ -442,8 +530,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         const CUtensorMap* ma = map_a(q);
         const CUtensorMap* mb = map_b(q);
         // the pair's bytes per stage land on the leader's barrier; the leader counts both halves
-        const uint32_t tx = kPair ? 2u * gemm::kPairStageBytes
-                                  : static_cast<uint32_t>(gemm::kABytes + bn_of(p) * BK * 2);
+        const uint32_t tx0 = kPair ? 2u * gemm::kPairStageBytes
+                                   : static_cast<uint32_t>(gemm::kABytes + bn_of(p) * BK * 2);
         const int kbs = k_blocks_of(p, g);
         const int m0 = mt * kRows + static_cast<int>(cta) * BM;   // this CTA's first A row of the tile
         for (int kb = 0; kb < kbs; ++kb) {
@@ -455,6 +543,9 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           const uint32_t sB = sA + gemm::kABytes;
           const uint32_t fb_local = smem_addr(&s.full[pipe.stage]);
           const uint32_t fb = kPair ? peer_addr(fb_local, 0) : fb_local;
+          // kRecDh's dh half: A and one 64 x 64 MN-major box of W2 per stage
+          const bool dh_half = !kPair && p.mode == kRecDh && kb >= p.num_k_blocks;
+          const uint32_t tx = dh_half ? static_cast<uint32_t>(gemm::kABytes + kMnBoxBytes) : tx0;
           if (cta == 0) mbar_arrive_expect_tx(fb_local, tx);
           auto load = [&](uint32_t dst, const CUtensorMap* m, int c0, int c1, int c2) {
             if (kPair)
@@ -472,6 +563,20 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
             const int n0 = nt * p.width + (kPair ? static_cast<int>(cta) * gemm::kPairBHalf : 0);
             const int nb = kPair ? gemm::kPairBHalf / kMnBox : p.width / kMnBox;
             for (int j = 0; j < nb; ++j) load(sB + j * kMnBoxBytes, mb, n0 + j * kMnBox, k0, grp);
+          } else if (!kPair && p.mode == kRecDh) {
+            // K blocks of the recompute (x, W13 rows of the tile's gate and up columns), then
+            // those of dh (dy, the tile's 64 columns of W2 as one MN-major box)
+            const int a_row = p.group_row ? static_cast<int>(row_of(p, g, m0)) : m0;
+            const int grp = p.group_row ? 0 : g;
+            if (!dh_half) {
+              load(sA, &ta0, kb * BK, a_row, grp);
+              load(sB, &tb0, kb * BK, nt * kRecDhWidth, g);
+              load(sB + kRecDhWidth * BK * 2, &tb0, kb * BK, p.F + nt * kRecDhWidth, g);
+            } else {
+              const int kk = kb - p.num_k_blocks;
+              load(sA, &ta1, kk * BK, a_row, grp);
+              load(sB, &tb1, nt * kRecDhWidth, kk * BK, g);
+            }
           } else {
             const int a_row = p.group_row ? static_cast<int>(row_of(p, g, m0)) : m0;
             load(sA, ma, kb * BK, a_row, p.group_row ? 0 : g);
@@ -526,6 +631,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         const GemmArgs& p = L.ph[q];
         const uint32_t idesc =
             idesc_bf16_f32(kRows, bn_of(p)) | (p.a_mn ? kIdescAMn : 0u) | (p.b_mn ? kIdescBMn : 0u);
+        // kRecDh's dh half: N = 64, B MN-major, accumulator columns from 128
+        const uint32_t idesc_dh = idesc_bf16_f32(kRows, kRecDhWidth) | kIdescBMn;
         // one K step of 16: +32 B along a K-major row, +16 rows of 128 B in an MN-major box
         const uint32_t b_step = p.b_mn ? (16u * 128u) >> 4 : 2u;
         const uint32_t a_step = p.a_mn ? (16u * 128u) >> 4 : 2u;
@@ -544,14 +651,24 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           tc_fence_after();
           const uint32_t sA = smem_addr(s.stage + pipe.stage * kSlot);
           const uint64_t adesc = p.a_mn ? smem_desc_sw128_mn(sA, kMnBoxBytes) : smem_desc_sw128(sA);
-          const uint64_t bdesc = p.b_mn ? smem_desc_sw128_mn(sA + gemm::kABytes, kMnBoxBytes)
-                                        : smem_desc_sw128(sA + gemm::kABytes);
+          if (!kPair && p.mode == kRecDh && kb >= p.num_k_blocks) {
+            const int kd = kb - p.num_k_blocks;
+            const uint64_t bdesc = smem_desc_sw128_mn(sA + gemm::kABytes, kMnBoxBytes);
+            const uint32_t mn_step = (16u * 128u) >> 4;
 #pragma unroll
-          for (int kk = 0; kk < BK / gemm::UMMA_K; ++kk) {
-            if (kPair)
-              mma_bf16_pair(d_tmem, adesc + a_step * kk, bdesc + b_step * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
-            else
-              mma_bf16(d_tmem, adesc + a_step * kk, bdesc + b_step * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < BK / gemm::UMMA_K; ++kk)
+              mma_bf16(d_tmem + 2 * kRecDhWidth, adesc + 2u * kk, bdesc + mn_step * kk, idesc_dh,
+                       (kd | kk) != 0 ? 1u : 0u);
+          } else {
+            const uint64_t bdesc = p.b_mn ? smem_desc_sw128_mn(sA + gemm::kABytes, kMnBoxBytes)
+                                          : smem_desc_sw128(sA + gemm::kABytes);
+#pragma unroll
+            for (int kk = 0; kk < BK / gemm::UMMA_K; ++kk) {
+              if (kPair)
+                mma_bf16_pair(d_tmem, adesc + a_step * kk, bdesc + b_step * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+              else
+                mma_bf16(d_tmem, adesc + a_step * kk, bdesc + b_step * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
           }
           if (kPair)
             mma_commit_pair(smem_addr(&s.empty[pipe.stage]), 3);
@@ -607,6 +724,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         epi_recompute(p, &tout1, &tout2, tbase, g, row0, valid, nt, stage, ochunk);
       } else if (p.mode == kDh) {
         epi_dh(p, &tout1, tbase, g, row0, valid, nt, stage, ochunk);
+      } else if (p.mode == kRecDh) {
+        if constexpr (!kPair) epi_recdh(p, &tout1, &tout2, tbase, g, row0, valid, nt, stage, ochunk);
       } else if (p.mode == kDx) {
         uint16_t* orow = static_cast<uint16_t*>(p.out) + row_of(p, g, row) * p.out_ld + nt * p.width;
         gemm::store_bf16(tbase, p.width, orow, valid);
@@ -1022,8 +1141,10 @@ cudaError_t run_gemm(const CUtensorMap* a, const CUtensorMap* b, const bwd::Gemm
   bwd::Launch L{};
   L.phases = phases;
   for (int q = 0; q < phases; ++q) L.ph[q] = args[q];
-  const CUtensorMap& a1 = a[phases > 1 ? 1 : 0];
-  const CUtensorMap& b1 = b[phases > 1 ? 1 : 0];
+  // kRecDh (one phase) reads its dh operands through the second map pair
+  const bool rec_dh = args[0].mode == bwd::kRecDh;
+  const CUtensorMap& a1 = a[phases > 1 || rec_dh ? 1 : 0];
+  const CUtensorMap& b1 = b[phases > 1 || rec_dh ? 1 : 0];
   const CUtensorMap& a2 = a[phases > 2 ? 2 : 0];
   const CUtensorMap& b2 = b[phases > 2 ? 2 : 0];
   const CUtensorMap& o1 = out ? out[1] : a[0];   // unused unless an epilogue stores through TMA
@@ -1151,16 +1272,45 @@ constexpr int kWide[3] = {256, 128, 64};
 
 }  // namespace
 
-bool backward_front_is_thin(const BackwardArgs& a, const int32_t* n_host) {
-  const int F = a.F;
+namespace {
+
+constexpr int kRecW[3] = {128, 64, 32};   // the recompute's tile widths (gate columns)
+
+// How a round's front half runs: `pair` when either GEMM takes the CTA-pair form (then as two
+// launches); else as one fused recompute + dh launch (kRecDh) when that streams less per SM than
+// the two launches, counting a launch as 550 KB of streaming (about 5.5 us at 100 GB/s per SM).
+// Costs are in rows of K = d per SM: waves x (A rows + B rows) of each launch. `tiles`: the most
+// tiles of one of its launches.
+struct FrontPlan {
+  bool pair = false, fused = false;
+  int w_rec = 0, w_dh = 0;
+  long long tiles = 0;
+};
+
+FrontPlan front_plan(const int32_t* n_host, int E, int d, int F) {
+  FrontPlan f;
   long long mt = 0;
-  for (int g = 0; g < a.E; ++g) mt += (n_host[g] + gemm::BM - 1) / gemm::BM;
-  const RowBlocks rb = row_blocks(n_host, a.E);
-  static const int kW[3] = {128, 64, 32};
-  if ((F % 128 == 0 && use_pair(rb, F / 128)) || (F % 256 == 0 && use_pair(rb, F / 256))) return false;
-  const long long rec = mt * (F / pick_width(kW, 3, mt, F, 2));
-  const long long dh = mt * (F / pick_width(kWide, 3, mt, F));
-  return rec < num_sms() && dh < num_sms();
+  for (int g = 0; g < E; ++g) mt += (n_host[g] + gemm::BM - 1) / gemm::BM;
+  const RowBlocks rb = row_blocks(n_host, E);
+  f.pair = (F % 128 == 0 && use_pair(rb, F / 128)) || (F % 256 == 0 && use_pair(rb, F / 256));
+  f.w_rec = pick_width(kRecW, 3, mt, F, 2);
+  f.w_dh = pick_width(kWide, 3, mt, F);
+  const long long sms = num_sms();
+  auto waves = [&](long long tiles) { return (tiles + sms - 1) / sms; };
+  const long long t_rec = mt * (F / f.w_rec), t_dh = mt * (F / f.w_dh), t_f = mt * (F / bwd::kRecDhWidth);
+  const long long separate = waves(t_rec) * (gemm::BM + 2 * f.w_rec) + waves(t_dh) * (gemm::BM + f.w_dh) +
+                             (550ll * 1024) / (2ll * d);
+  const long long fused = waves(t_f) * (gemm::BM + 2 * bwd::kRecDhWidth + gemm::BM + bwd::kRecDhWidth);
+  f.fused = !f.pair && F % bwd::kRecDhWidth == 0 && fused < separate;
+  f.tiles = f.fused ? t_f : (t_rec > t_dh ? t_rec : t_dh);
+  return f;
+}
+
+}  // namespace
+
+bool backward_front_is_thin(const BackwardArgs& a, const int32_t* n_host) {
+  const FrontPlan f = front_plan(n_host, a.E, a.d, a.F);
+  return !f.pair && f.tiles <= num_sms();
 }
 
 cudaError_t launch_backward_front(const BackwardArgs& a, int r, const int32_t* n_host, bool gather, int* parts_out,
@@ -1186,13 +1336,41 @@ cudaError_t launch_backward_front(const BackwardArgs& a, int r, const int32_t* n
   // pair form: 256-row tiles, 128 B rows per CTA (recompute: 128 W1 rows and the same W3 rows)
   const uint32_t pair_box = gemm::kPairBHalf;
 
+  const FrontPlan fp = front_plan(n_host, E, d, F);
+  // single-CTA form: recompute and dh of the same 64 d_ff columns in one tile (a, b stay in TMEM)
+  if (fp.fused) {
+    constexpr int w = bwd::kRecDhWidth;
+    bwd::GemmArgs g = base;
+    g.mode = bwd::kRecDh;
+    g.width = w;
+    g.n_total = F;
+    g.num_k_blocks = d / gemm::BK;
+    g.out = a.dab;
+    g.row_gate = a.row_gate;
+    g.dgate_part = a.dgate_part;
+    g.dgate_ld = F / 64;
+    CUtensorMap ma[2], mb[2], mo[3];
+    if ((e = gemm::make_map(&ma[0], a.xbuf, d, a_rows, groups, gemm::BM)) != cudaSuccess ||
+        (e = gemm::make_map(&mb[0], a.w_gate_up, d, 2ull * F, E, w)) != cudaSuccess ||
+        (e = gemm::make_map(&ma[1], a.dybuf, d, a_rows, groups, gemm::BM)) != cudaSuccess ||
+        (e = gemm::make_map(&mb[1], a.w_down, F, d, E, bwd::kMnBox, bwd::kMnBox)) != cudaSuccess)
+      return e;
+    // the epilogue's TMA stores: 1 = dab [.][2F], 2 = hg [.][F], 32 x 32 chunks
+    if ((e = gemm::make_map(&mo[1], a.dab, 2ull * F, a_rows, groups, 32, gemm::kOutChunkCols)) != cudaSuccess ||
+        (e = gemm::make_map(&mo[2], a.hg, F, a_rows, groups, 32, gemm::kOutChunkCols)) != cudaSuccess)
+      return e;
+    mo[0] = mo[1];
+    if ((e = run_gemm(ma, mb, &g, 1, mt * (F / w), kKindBackwardRecDh, stream, mo, false)) != cudaSuccess) return e;
+    *parts_out = F / w;
+    return cudaSuccess;
+  }
+
   // recompute: [a | b] = xbuf W13^T
   {
-    static const int kW[3] = {128, 64, 32};
     const bool pair = F % 128 == 0 && use_pair(rb, F / 128);
     bwd::GemmArgs g = base;
     g.mode = bwd::kRecompute;
-    g.width = pair ? 128 : pick_width(kW, 3, mt, F, 2);
+    g.width = pair ? 128 : fp.w_rec;
     g.n_total = F;
     g.num_k_blocks = d / gemm::BK;
     g.out = a.ab;
@@ -1217,7 +1395,7 @@ cudaError_t launch_backward_front(const BackwardArgs& a, int r, const int32_t* n
     const bool pair = F % 256 == 0 && use_pair(rb, F / 256);
     bwd::GemmArgs g = base;
     g.mode = bwd::kDh;
-    g.width = pair ? 256 : pick_width(kWide, 3, mt, F);
+    g.width = pair ? 256 : fp.w_dh;
     parts = F / g.width;
     g.n_total = F;
     g.num_k_blocks = d / gemm::BK;

@@ -15,6 +15,7 @@ constexpr int kKindBackwardRecompute = 8;
 constexpr int kKindBackwardDh = 9;
 constexpr int kKindBackwardDxWgrad = 10;
 constexpr int kKindBackwardCopy = 11;
+constexpr int kKindBackwardRecDh = 12;
 
 // ---- backward with per-round recompute (backward.cu)
 // Device pointers of one backward call: the forward's plan (read only), the caller's tensors and
@@ -68,8 +69,9 @@ long long backward_rows2(int E, int C);
 cudaError_t launch_backward_prepare(const BackwardArgs& a, const int32_t* load_host, int R, cudaStream_t stream);
 // A round in two halves, each on a stream of its own choosing. n_host: the round's rows per
 // expert. a: the round's buffer set (its pointers, pooled and rows).
-// Whether a round's front half runs in the single-CTA form with fewer tiles per GEMM than the
-// device has SMs (so that it leaves SMs to the round before's back half).
+// Whether a round's front half is one fused recompute + dh launch in the single-CTA form with at
+// most as many tiles as the device has SMs (so that it leaves SMs to the round before's back
+// half).
 bool backward_front_is_thin(const BackwardArgs& a, const int32_t* n_host);
 // Front: the dispatch of x and dy (when `gather`; else the previous round's combine launch ran
 // it), the recompute and dh (+ the SwiGLU backward); *parts: dgate partials per row, for the back.

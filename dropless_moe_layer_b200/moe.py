@@ -16,10 +16,11 @@ from .build import LIB_PATH, ROOT
 c_i32, c_u32, c_sz, c_vp = ctypes.c_int32, ctypes.c_uint32, ctypes.c_size_t, ctypes.c_void_p
 
 MAX_EXPERTS = 256
-PROFILE_KINDS = 12
+PROFILE_KINDS = 13
 PROFILE_NAMES = ["router_gemm", "topk", "plan", "dispatch", "gate_up", "down", "combine", "pipeline",
-                 "backward_recompute", "backward_dh", "backward_dx_wgrad", "backward_copy"]
-BACKWARD_GEMM_KINDS = ("backward_recompute", "backward_dh", "backward_dx_wgrad")
+                 "backward_recompute", "backward_dh", "backward_dx_wgrad", "backward_copy",
+                 "backward_recompute_dh"]
+BACKWARD_GEMM_KINDS = ("backward_recompute", "backward_dh", "backward_recompute_dh", "backward_dx_wgrad")
 FLAG_RENORM_TOPK = 1
 FLAG_PER_ROUND = 2
 FLAG_PIPELINE_ALL = 4

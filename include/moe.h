@@ -307,9 +307,10 @@ MOE_API uint64_t moe_launch_count(void);
  * 0 router GEMM, 1 top-k, 2 plan, 3 dispatch, 4 gate_up GEMM, 5 down GEMM, 6 combine,
  * 7 pipelined rounds (all four steps of its rounds in one launch); backward: 8 recompute GEMM,
  * 9 dh GEMM (with the SwiGLU backward), 10 dx and weight-gradient GEMMs (one launch a round),
- * 11 its other launches (gather, dx combine, gate gradient, segment table, fills).
+ * 11 its other launches (gather, dx combine, gate gradient, segment table, fills), 12 recompute
+ * and dh GEMMs in one launch (rounds whose GEMMs run in the single-CTA form).
  * Up to 4096 launches are recorded between enable and read. Not thread-safe. */
-#define MOE_PROFILE_KINDS 12
+#define MOE_PROFILE_KINDS 13
 MOE_API int moe_profile_enable(int on);
 MOE_API int moe_profile_read(int32_t counts[MOE_PROFILE_KINDS], double ms[MOE_PROFILE_KINDS]);
 

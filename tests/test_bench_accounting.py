@@ -70,11 +70,14 @@ def test_traffic_record_ignores_comments_not_code():
 
 def test_backward_flops_split_by_launch_kind():
     """The backward's GEMM launch kinds account for all of its tensor-core work: 16 d d_ff flops
-    per routed pair (recompute 4, dh 2, dx 4, dW2 2, dW1 and dW3 4)."""
+    per routed pair (recompute 4, dh 2, dx 4, dW2 2, dW1 and dW3 4); a round runs its recompute
+    and dh either as two launches or as one fused launch, never both."""
     from dropless_moe_layer_b200 import moe
     w = wl.BY_NAME["4k-zipf1"]
-    assert set(bench.BWD_KIND_FLOPS) == set(moe.BACKWARD_GEMM_KINDS)
-    assert sum(bench.BWD_KIND_FLOPS.values()) * w.T * w.k * w.d * w.F == bench.backward_flops(w)
+    f = bench.BWD_KIND_FLOPS
+    assert set(f) == set(moe.BACKWARD_GEMM_KINDS) and set(bench.BWD_FRONT_KINDS) <= set(f)
+    assert f["backward_recompute"] + f["backward_dh"] == f["backward_recompute_dh"]
+    assert (f["backward_recompute_dh"] + f["backward_dx_wgrad"]) * w.T * w.k * w.d * w.F == bench.backward_flops(w)
 
 
 def test_ride_plan_follows_the_size_rule():
