@@ -529,11 +529,56 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         const GemmArgs& p = L.ph[q];
         const CUtensorMap* ma = map_a(q);
         const CUtensorMap* mb = map_b(q);
+        // The tile's load plan, in registers: the loop below issues only the loads and the
+        // K coordinate (the TMA and barrier asm statements clobber memory, so anything read
+        // from the launch arguments inside the loop would be read again at every stage).
+        enum : int { kLdWgrad, kLdBmn, kLdB1, kLdB2, kLdRecDh };
+        const int mode = p.mode;
+        const int m0 = mt * kRows + static_cast<int>(cta) * BM;   // this CTA's first A row of the tile
+        const int grp = p.group_row ? 0 : g;
+        const int kbs = k_blocks_of(p, g);
+        const int nkb = p.num_k_blocks;
+        int ld, a_c = 0, b_c = 0, b_c2 = 0, nbox = 0;
+        if (mode == kWgrad) {
+          // both operands are the round's row-major buffers read MN-major, K = the expert's
+          // rows (from row 0 of its C rows, or from its segment's first row): this CTA's 128
+          // A columns and its B columns as 64-column boxes, 8 KB apart
+          ld = kLdWgrad;
+          a_c = static_cast<int>(row_of(p, g, 0)) - (p.group_row ? 0 : g * p.C);   // K base
+          b_c = nt * p.width + (kPair ? static_cast<int>(cta) * gemm::kPairBHalf : 0);
+          nbox = kPair ? gemm::kPairBHalf / kMnBox : p.width / kMnBox;
+        } else {
+          a_c = p.group_row ? static_cast<int>(row_of(p, g, m0)) : m0;   // A row
+          if (!kPair && mode == kRecDh) {
+            // K blocks of the recompute (x, W13 rows of the tile's gate and up columns), then
+            // those of dh (dy, the tile's 64 columns of W2 as one MN-major box)
+            ld = kLdRecDh;
+            b_c = nt * kRecDhWidth;
+            b_c2 = p.F + nt * kRecDhWidth;
+          } else if (p.b_mn) {
+            // MN-major weights: this CTA's B columns as 64-column boxes, 8 KB apart
+            ld = kLdBmn;
+            b_c = nt * p.width + (kPair ? static_cast<int>(cta) * gemm::kPairBHalf : 0);
+            nbox = kPair ? gemm::kPairBHalf / kMnBox : p.width / kMnBox;
+          } else if (kPair) {
+            // recompute: CTA 0 the tile's W1 rows, CTA 1 the same W3 rows; else 128 of the 256
+            ld = kLdB1;
+            b_c = mode == kRecompute ? static_cast<int>(cta) * p.F + nt * p.width
+                                     : nt * p.width + static_cast<int>(cta) * gemm::kPairBHalf;
+          } else if (mode == kRecompute) {
+            ld = kLdB2;
+            b_c = nt * p.width;
+            b_c2 = p.F + nt * p.width;
+          } else {
+            ld = kLdB1;
+            b_c = nt * p.width;
+          }
+        }
+        const uint32_t b2_off = static_cast<uint32_t>(p.width) * BK * 2;   // kLdB2: the up rows
         // the pair's bytes per stage land on the leader's barrier; the leader counts both halves
         const uint32_t tx0 = kPair ? 2u * gemm::kPairStageBytes
                                    : static_cast<uint32_t>(gemm::kABytes + bn_of(p) * BK * 2);
-        const int kbs = k_blocks_of(p, g);
-        const int m0 = mt * kRows + static_cast<int>(cta) * BM;   // this CTA's first A row of the tile
+        const uint32_t tx_dh = static_cast<uint32_t>(gemm::kABytes + kMnBoxBytes);
         for (int kb = 0; kb < kbs; ++kb) {
           if (!mbar_wait(smem_addr(&s.empty[pipe.stage]), pipe.phase ^ 1u, s.abort)) {
             ok = false;
@@ -544,57 +589,34 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           const uint32_t fb_local = smem_addr(&s.full[pipe.stage]);
           const uint32_t fb = kPair ? peer_addr(fb_local, 0) : fb_local;
           // kRecDh's dh half: A and one 64 x 64 MN-major box of W2 per stage
-          const bool dh_half = !kPair && p.mode == kRecDh && kb >= p.num_k_blocks;
-          const uint32_t tx = dh_half ? static_cast<uint32_t>(gemm::kABytes + kMnBoxBytes) : tx0;
-          if (cta == 0) mbar_arrive_expect_tx(fb_local, tx);
+          const bool dh_half = !kPair && ld == kLdRecDh && kb >= nkb;
+          if (cta == 0) mbar_arrive_expect_tx(fb_local, dh_half ? tx_dh : tx0);
           auto load = [&](uint32_t dst, const CUtensorMap* m, int c0, int c1, int c2) {
             if (kPair)
               tma_load_3d_pair(dst, m, fb, c0, c1, c2);
             else
               tma_load_3d(dst, m, fb, c0, c1, c2);
           };
-          if (p.mode == kWgrad) {
-            // both operands are the round's row-major buffers read MN-major, K = the expert's
-            // rows (from row 0 of its C rows, or from its segment's first row): this CTA's 128
-            // A columns and its B columns as 64-column boxes, 8 KB apart
-            const int k0 = static_cast<int>(row_of(p, g, 0)) - (p.group_row ? 0 : g * p.C) + kb * BK;
-            const int grp = p.group_row ? 0 : g;
-            for (int j = 0; j < BM / kMnBox; ++j) load(sA + j * kMnBoxBytes, ma, m0 + j * kMnBox, k0, grp);
-            const int n0 = nt * p.width + (kPair ? static_cast<int>(cta) * gemm::kPairBHalf : 0);
-            const int nb = kPair ? gemm::kPairBHalf / kMnBox : p.width / kMnBox;
-            for (int j = 0; j < nb; ++j) load(sB + j * kMnBoxBytes, mb, n0 + j * kMnBox, k0, grp);
-          } else if (!kPair && p.mode == kRecDh) {
-            // K blocks of the recompute (x, W13 rows of the tile's gate and up columns), then
-            // those of dh (dy, the tile's 64 columns of W2 as one MN-major box)
-            const int a_row = p.group_row ? static_cast<int>(row_of(p, g, m0)) : m0;
-            const int grp = p.group_row ? 0 : g;
+          const int k = kb * BK;
+          if (ld == kLdWgrad) {
+            for (int j = 0; j < BM / kMnBox; ++j) load(sA + j * kMnBoxBytes, ma, m0 + j * kMnBox, a_c + k, grp);
+            for (int j = 0; j < nbox; ++j) load(sB + j * kMnBoxBytes, mb, b_c + j * kMnBox, a_c + k, grp);
+          } else if (ld == kLdRecDh) {
             if (!dh_half) {
-              load(sA, &ta0, kb * BK, a_row, grp);
-              load(sB, &tb0, kb * BK, nt * kRecDhWidth, g);
-              load(sB + kRecDhWidth * BK * 2, &tb0, kb * BK, p.F + nt * kRecDhWidth, g);
+              load(sA, &ta0, k, a_c, grp);
+              load(sB, &tb0, k, b_c, g);
+              load(sB + kRecDhWidth * BK * 2, &tb0, k, b_c2, g);
             } else {
-              const int kk = kb - p.num_k_blocks;
-              load(sA, &ta1, kk * BK, a_row, grp);
-              load(sB, &tb1, nt * kRecDhWidth, kk * BK, g);
+              load(sA, &ta1, k - nkb * BK, a_c, grp);
+              load(sB, &tb1, b_c, k - nkb * BK, g);
             }
           } else {
-            const int a_row = p.group_row ? static_cast<int>(row_of(p, g, m0)) : m0;
-            load(sA, ma, kb * BK, a_row, p.group_row ? 0 : g);
-            if (p.b_mn) {
-              // MN-major weights: this CTA's B columns as 64-column boxes, 8 KB apart
-              const int n0 = nt * p.width + (kPair ? static_cast<int>(cta) * gemm::kPairBHalf : 0);
-              const int nb = kPair ? gemm::kPairBHalf / kMnBox : p.width / kMnBox;
-              for (int j = 0; j < nb; ++j) load(sB + j * kMnBoxBytes, mb, n0 + j * kMnBox, kb * BK, g);
-            } else if (kPair) {
-              // recompute: CTA 0 the tile's W1 rows, CTA 1 the same W3 rows; else 128 of the 256
-              const int b_row = p.mode == kRecompute ? static_cast<int>(cta) * p.F + nt * p.width
-                                                     : nt * p.width + static_cast<int>(cta) * gemm::kPairBHalf;
-              load(sB, mb, kb * BK, b_row, g);
-            } else if (p.mode == kRecompute) {
-              load(sB, mb, kb * BK, nt * p.width, g);
-              load(sB + p.width * BK * 2, mb, kb * BK, p.F + nt * p.width, g);
+            load(sA, ma, k, a_c, grp);
+            if (ld == kLdBmn) {
+              for (int j = 0; j < nbox; ++j) load(sB + j * kMnBoxBytes, mb, b_c + j * kMnBox, k, g);
             } else {
-              load(sB, mb, kb * BK, nt * p.width, g);
+              load(sB, mb, k, b_c, g);
+              if (ld == kLdB2) load(sB + b2_off, mb, k, b_c2, g);
             }
           }
           pipe.issued |= 1u << pipe.stage;
@@ -637,6 +659,10 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         const uint32_t b_step = p.b_mn ? (16u * 128u) >> 4 : 2u;
         const uint32_t a_step = p.a_mn ? (16u * 128u) >> 4 : 2u;
         const int kbs = k_blocks_of(p, g);
+        // in registers: the asm statements below clobber memory
+        const bool a_mn = p.a_mn != 0, b_mn = p.b_mn != 0;
+        const bool rec_dh = !kPair && p.mode == kRecDh;
+        const int nkb = p.num_k_blocks;
         if (!mbar_wait(smem_addr(&s.tempty[pipe.acc]), pipe.acc_phase ^ 1u, s.abort)) {
           ok = false;
           break;
@@ -650,9 +676,9 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           }
           tc_fence_after();
           const uint32_t sA = smem_addr(s.stage + pipe.stage * kSlot);
-          const uint64_t adesc = p.a_mn ? smem_desc_sw128_mn(sA, kMnBoxBytes) : smem_desc_sw128(sA);
-          if (!kPair && p.mode == kRecDh && kb >= p.num_k_blocks) {
-            const int kd = kb - p.num_k_blocks;
+          const uint64_t adesc = a_mn ? smem_desc_sw128_mn(sA, kMnBoxBytes) : smem_desc_sw128(sA);
+          if (rec_dh && kb >= nkb) {
+            const int kd = kb - nkb;
             const uint64_t bdesc = smem_desc_sw128_mn(sA + gemm::kABytes, kMnBoxBytes);
             const uint32_t mn_step = (16u * 128u) >> 4;
 #pragma unroll
@@ -660,8 +686,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
               mma_bf16(d_tmem + 2 * kRecDhWidth, adesc + 2u * kk, bdesc + mn_step * kk, idesc_dh,
                        (kd | kk) != 0 ? 1u : 0u);
           } else {
-            const uint64_t bdesc = p.b_mn ? smem_desc_sw128_mn(sA + gemm::kABytes, kMnBoxBytes)
-                                          : smem_desc_sw128(sA + gemm::kABytes);
+            const uint64_t bdesc = b_mn ? smem_desc_sw128_mn(sA + gemm::kABytes, kMnBoxBytes)
+                                        : smem_desc_sw128(sA + gemm::kABytes);
 #pragma unroll
             for (int kk = 0; kk < BK / gemm::UMMA_K; ++kk) {
               if (kPair)
