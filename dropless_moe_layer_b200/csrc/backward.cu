@@ -786,8 +786,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
 
 constexpr int kWarps = 8;
 
-// Dispatch of round r. A block takes 64 rows of one expert's rows in the round and 64 columns
-// (c0 = 64 * blockIdx.y): the rows' tokens come from the round-major row list (row_off[r][e] +
+// Dispatch of round r. A block takes 64 rows of one expert's rows in the round and 256 columns
+// (c0 = 256 * blockIdx.y): the rows' tokens come from the round-major row list (row_off[r][e] +
 // s); their x and dy slices are copied into xbuf and dybuf (dy as bf16). The expert's padding
 // rows (from n[r][e] up to the next multiple of 64, within its C rows or its pooled segment) get
 // zeros: the weight-gradient GEMMs read the rows as K in blocks of 64. The blocks of the first
@@ -796,6 +796,8 @@ constexpr int kWarps = 8;
 // (expert e holds ceil(n[r][e] / 64) of them), so a round with few rows launches few blocks.
 // Rows s of expert e are at e * C + s, or with pooled rows at 64 b + (s mod 64): each expert's
 // segment starts at a multiple of 64 (the table seg_off the GEMMs and the combine read).
+constexpr int kGatherCols = 256;   // columns of a gather block (8 per lane)
+
 struct GatherArgs {
   const uint16_t* x;
   const float* dy;
@@ -810,12 +812,12 @@ struct GatherArgs {
   int r, E, C, d, k, pooled;
 };
 
-// Block (bx, by) of the gather: 64 rows (the bx-th 64-row block of the round) x 64 columns
-// (c0 = 64 by). The whole block runs it (256 threads).
+// Block (bx, by) of the gather: 64 rows (the bx-th 64-row block of the round) x kGatherCols
+// columns (c0 = kGatherCols by). The whole block runs it (256 threads).
 __device__ __forceinline__ void gather_block(const GatherArgs& a, int bx, int by) {
   __shared__ int tok[64];
   __shared__ int blk[3];      // expert, its first row in this block, its rows in the round
-  const int c0 = by * 64;
+  const int c0 = by * kGatherCols;
   const int32_t* nr = a.n + static_cast<size_t>(a.r) * a.E;
   if (threadIdx.x < 32) {
     // warp 0: the expert whose 64-row blocks hold block b (a running prefix over the experts)
@@ -861,22 +863,29 @@ __device__ __forceinline__ void gather_block(const GatherArgs& a, int bx, int by
       tok[threadIdx.x] = sr < ne ? a.row_token[base + sr] : -1;
     }
     __syncthreads();
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int rr = ty + 8 * i;
-      const int sr = s0 + rr;
-      if (!a.pooled && sr >= a.C) continue;   // past the expert's C rows: the next expert's
-      const int t = tok[rr];
-      uint32_t xv = 0, yv = 0;
-      if (t >= 0) {
-        xv = *reinterpret_cast<const uint32_t*>(a.x + static_cast<size_t>(t) * a.d + c0 + 2 * tx);
-        const float2 dv = *reinterpret_cast<const float2*>(a.dy + static_cast<size_t>(t) * a.d + c0 + 2 * tx);
-        yv = gemm::pack_bf16x2(dv.x, dv.y);
+    // 32 x 8 threads: a lane takes 8 columns (16-byte x and bf16 dy stores, two 16-byte dy
+    // loads), a warp 256 columns of one row at a time
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    const int c = c0 + 8 * tx;
+    if (c < a.d) {
+#pragma unroll 4
+      for (int i = 0; i < 8; ++i) {
+        const int rr = ty + 8 * i;
+        const int sr = s0 + rr;
+        if (!a.pooled && sr >= a.C) continue;   // past the expert's C rows: the next expert's
+        const int t = tok[rr];
+        uint4 xv = make_uint4(0u, 0u, 0u, 0u), yv = make_uint4(0u, 0u, 0u, 0u);
+        if (t >= 0) {
+          xv = __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.d + c));
+          const float4* dq = reinterpret_cast<const float4*>(a.dy + static_cast<size_t>(t) * a.d + c);
+          const float4 d0 = __ldg(dq), d1 = __ldg(dq + 1);
+          yv = make_uint4(gemm::pack_bf16x2(d0.x, d0.y), gemm::pack_bf16x2(d0.z, d0.w), gemm::pack_bf16x2(d1.x, d1.y),
+                          gemm::pack_bf16x2(d1.z, d1.w));
+        }
+        const size_t orow = static_cast<size_t>(dst0 + sr) * a.d + c;
+        *reinterpret_cast<uint4*>(a.xbuf + orow) = xv;
+        *reinterpret_cast<uint4*>(a.dybuf + orow) = yv;
       }
-      const size_t orow = static_cast<size_t>(dst0 + sr) * a.d + c0 + 2 * tx;
-      *reinterpret_cast<uint32_t*>(a.xbuf + orow) = xv;
-      *reinterpret_cast<uint32_t*>(a.dybuf + orow) = yv;
     }
     if (c0 == 0 && threadIdx.x < 64) {
       const int t = tok[threadIdx.x];
@@ -1348,7 +1357,7 @@ cudaError_t launch_backward_front(const BackwardArgs& a, int r, const int32_t* n
     const long long blocks = gather_blocks(n_host, E);
     if (blocks > 0) {
       launch_begin(kKindBackwardCopy, stream);
-      e = launch_pdl(bwd::bwd_gather_kernel, dim3(static_cast<unsigned>(blocks), d / 64), dim3(256), 0, stream,
+      e = launch_pdl(bwd::bwd_gather_kernel, dim3(static_cast<unsigned>(blocks), (d + bwd::kGatherCols - 1) / bwd::kGatherCols), dim3(256), 0, stream,
                      gather_args(a, r));
       launch_end(kKindBackwardCopy, stream);
       if (e != cudaSuccess) return e;
@@ -1515,12 +1524,13 @@ cudaError_t launch_backward_back(const BackwardArgs& a, int r, const int32_t* n_
                                pooled ? a.seg_off : nullptr, pooled ? a.zeros : nullptr, E};
     const bwd::CombineExtra cx{r, a.dgate_part, F / 64, parts, a.dgate};
     const int comb_blocks = grid_for(a.T);
-    const long long next_blocks = a_next && n_next ? gather_blocks(n_next, E) * (d / 64) : 0;
+    const int gy = (d + bwd::kGatherCols - 1) / bwd::kGatherCols;   // column blocks of the gather
+    const long long next_blocks = a_next && n_next ? gather_blocks(n_next, E) * gy : 0;
     launch_begin(kKindBackwardCopy, stream);
     if (next_blocks > 0)
       e = launch_pdl(bwd::bwd_combine_gather_kernel, dim3(static_cast<unsigned>(comb_blocks + next_blocks)),
                      dim3(32 * bwd::kWarps), 0, stream, ca, cx, gather_args(*a_next, r + 1), comb_blocks,
-                     static_cast<int>(next_blocks / (d / 64)));
+                     static_cast<int>(next_blocks / gy));
     else
       e = launch_pdl(bwd::bwd_combine_kernel, dim3(comb_blocks), dim3(32 * bwd::kWarps), 0, stream, ca, cx);
     launch_end(kKindBackwardCopy, stream);
