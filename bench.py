@@ -528,10 +528,13 @@ def bench_backward(args, w):
         step()
     torch.cuda.synchronize(dev)
     launches0 = moe.launch_count()
+    host_s = 0.0   # host time to enqueue the calls (their launches, events and waits)
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
         starts[i].record(stream)
+        h0 = time.perf_counter()
         step()
+        host_s += time.perf_counter() - h0
         ends[i].record(stream)
     torch.cuda.synchronize(dev)
     launches = moe.launch_count() - launches0
@@ -571,6 +574,7 @@ def bench_backward(args, w):
                      "frac_vs_burst": achieved / peaks["bf16_tflops"],
                      "frac_vs_datasheet": achieved / DATASHEET["bf16_tflops"], "flops_per_step": flops},
         "whole_pass_tflops": flops / (ms / 1e3) / 1e12,
+        "host_enqueue_ms_per_call": host_s * 1e3 / args.steps,
         "pass_frac": pass_s * 1e3 / ms,
         "pass_roofline": {"ms": pass_s * 1e3, **{k + "_ms": round(v, 4) for k, v in pass_parts.items()},
                           "peaks": f"{peak_src}: hbm_gbs {peaks['hbm_gbs']}, {tensor_key} {peak}",
