@@ -83,7 +83,9 @@ typedef enum moe_status {
  * launches. The pipelined launch
  * alternates two sets of round buffers, so the workspace holds a second set unless
  * MOE_FLAG_PER_ROUND is given. */
-#define MOE_FLAG_PER_ROUND 2u       /* every round as per-round launches */
+#define MOE_FLAG_PER_ROUND 2u       /* every round as per-round launches; moe_backward runs its
+                                       rounds one after another on `stream`, without the second
+                                       buffer set of its workspace (same results) */
 #define MOE_FLAG_PIPELINE_ALL 4u    /* every round in the pipelined launch */
 /* Capacity borrowing ("Frontier Pre-training at Microsoft AI (MAI-Base-2)", Key claims,
  * multi-round dropless MoE item: overflow tokens use unused capacity of other experts of the
@@ -284,7 +286,11 @@ MOE_API int moe_backward_workspace_layout(const moe_shape_t* shape, moe_backward
  * w_down as in moe_forward; dy [T, d] fp32. Operands of the tensor-core steps are bf16 (dy, a,
  * b, gate * h, da, db rounded to bf16) with fp32 accumulation. Plans made with MOE_FLAG_BORROW
  * run on their pooled round rows. A bounded wait that gives up sets the status word
- * (moe_device_status). Asynchronous: no synchronization. */
+ * (moe_device_status). Asynchronous: no synchronization. Thin rounds overlap the round before
+ * them: their dispatch, recompute and dh run on `stream` while the round before's dx, weight
+ * gradients and combine run on a second stream of the library's (one per host thread and
+ * device, created on first use), joined back to `stream` before the call's last launch; the
+ * results are those of one round at a time, bit for bit. */
 MOE_API int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws, size_t ws_bytes,
                          void* bws, size_t bws_bytes, const uint16_t* x, const uint16_t* w_gate_up,
                          const uint16_t* w_down, const float* dy, float* dx, float* dw_gate_up,
