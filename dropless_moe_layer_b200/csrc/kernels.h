@@ -78,8 +78,9 @@ constexpr int kPlanTokensPerBlock = 256;
 // dependency counters inside the workspace ("sync" region, int32, all zero between launches).
 // Round r of a launch starting at round r0 uses buffer set p = (r - r0) & 1.
 constexpr int kPipeRowBlock = 128;   // rows of a tile (one 128-row block of an expert's C rows)
-constexpr int kPipeGuWidth = 32;     // gate columns per gate/up tile (MMA N = 64)
-constexpr int kPipeDnWidth = 64;     // output columns per down tile (MMA N = 64)
+// Gate columns per gate/up tile (MMA N = twice that); a down tile has twice as many output
+// columns, so both GEMMs share one stage geometry. 64 when d is a multiple of 128, else 32.
+__host__ __device__ inline int pipe_gate_width(int d) { return d % 128 == 0 ? 64 : 32; }
 // Every counter has its own 32-byte sector (a stride of 8 words) and the round-level counters
 // their own 256-byte slots, so that polls and atomic adds on different counters do not queue
 // behind each other in one L2 line.
@@ -240,6 +241,7 @@ struct PipelineArgs {
   int32_t* status;
   int T, k, E, C, d, F, r0, R;
   int r0_dispatched;         // 1: round r0's rows are already in buf (set 0) when the launch starts
+  int gw;                    // gate columns per gate/up tile (pipe_gate_width(d)); down tiles 2 gw
 };
 cudaError_t launch_round_pipeline(const PipelineArgs& a, cudaStream_t stream);
 

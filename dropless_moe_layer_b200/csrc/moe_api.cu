@@ -894,6 +894,7 @@ int moe_forward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws,
     p.r0 = r0;
     p.R = R;
     p.r0_dispatched = 1;
+    p.gw = pipe_gate_width(shape->d);
     const cudaError_t e = launch_round_pipeline(p, stream);
     if (e == cudaErrorCooperativeLaunchTooLarge) {
       // not every SM is available to this context (a partitioned GPU): run those rounds per round

@@ -16,9 +16,11 @@
 //                 index to the MMA and epilogue warps through a small shared-memory ring;
 //   warps 6..9    dispatch warps: each round's rows, in contiguous slices per warp of the grid;
 //   warps 10..15  combine warps: each owns a fixed set of tokens and combines them round by round.
-// GEMM tile list: gate/up tiles (128 rows x 32 gate columns, MMA N = 64, every column slice of
-// a 128-row block before the next block) and down tiles (128 rows x 64 output columns), phase
-// by phase in the order G(r0) G(r0+1) N(r0) G(r0+2) N(r0+1) ... N(R-1).
+// GEMM tile list: gate/up tiles (128 rows x GW gate columns, MMA N = 2 GW, every column slice
+// of a 128-row block before the next block) and down tiles (128 rows x 2 GW output columns),
+// phase by phase in the order G(r0) G(r0+1) N(r0) G(r0+2) N(r0+1) ... N(R-1). GW is 64 when d
+// is a multiple of 128 (fewer, wider tiles: each tile's fixed costs are paid for twice the
+// columns), else 32 (a template parameter of the kernel; both use the same 192 KB ring).
 //
 // Round r uses buffer set p = (r - r0) & 1 (buf, h and out exist twice), so a round's buffers
 // are reused two rounds later and consecutive rounds do not wait on each other's reads.
@@ -61,11 +63,15 @@ namespace {
 
 using namespace gemm;
 
-constexpr int kBN = 2 * kPipeGuWidth;                      // MMA N of both GEMMs
-constexpr int kPStageBytes = kABytes + kBN * BK * 2;       // 24 KB
-constexpr int kPStages = kRingBytes / kPStageBytes;        // 8
-static_assert(kPStages <= kMaxStages, "ring stages");
-static_assert(kPipeDnWidth == kBN, "both GEMMs use one stage geometry");
+// Stage geometry for GW gate columns per gate/up tile: MMA N = 2 GW for both GEMMs (a down
+// tile has 2 GW output columns), so one ring serves both.
+template <int GW>
+struct Geom {
+  static constexpr int kBN = 2 * GW;                               // MMA N of both GEMMs
+  static constexpr int kStageBytes = kABytes + kBN * BK * 2;       // 24 KB (GW 32), 32 KB (GW 64)
+  static constexpr int kStages = kRingBytes / kStageBytes;         // 8, 6
+  static_assert(kStages >= 2 && kStages <= kMaxStages, "ring stages");
+};
 static_assert(kPipeRowBlock == BM, "row blocks are GEMM tiles");
 constexpr int kDispWarps = 4;
 constexpr int kCombWarps = 6;
@@ -132,7 +138,7 @@ struct Cursor {
 
 __device__ __forceinline__ void cursor_load(Cursor& c, const PipelineArgs& a) {
   const int mblocks = a.mb_prefix[static_cast<size_t>(c.r) * (a.E + 1) + a.E];
-  c.end = c.base + mblocks * (c.gu ? a.F / kPipeGuWidth : a.d / kPipeDnWidth);
+  c.end = c.base + mblocks * (c.gu ? a.F / a.gw : a.d / (2 * a.gw));
 }
 
 __device__ __forceinline__ void cursor_init(Cursor& c, const PipelineArgs& a) {
@@ -178,7 +184,7 @@ __device__ __forceinline__ void decode(const Cursor& c, const PipelineArgs& a, i
   const int local = task - c.base;
   t.r = c.r;
   t.gu = c.gu;
-  const int per = c.gu ? a.F / kPipeGuWidth : a.d / kPipeDnWidth;
+  const int per = c.gu ? a.F / a.gw : a.d / (2 * a.gw);
   t.kb = c.gu ? a.d / BK : a.F / BK;
   const int blk = local / per;
   t.nt = local - blk * per;
@@ -226,9 +232,9 @@ __device__ bool wait_inputs(const PipelineArgs& a, const Counters& cn, const Cur
     // round r0's rows were dispatched by an earlier kernel: set 0 counts them as present
     const int pre = a.r0_dispatched && p == 0 ? full : 0;
     if (!wait_counter(a, cn.disp[p] + blk, q * full + rows - pre)) return false;
-    if (q > 0 && !wait_counter(a, cn.dn[p] + blk, q * kEpiWarps * (a.d / kPipeDnWidth))) return false;
+    if (q > 0 && !wait_counter(a, cn.dn[p] + blk, q * kEpiWarps * (a.d / (2 * a.gw)))) return false;
   } else {
-    if (!wait_counter(a, cn.gu[p] + blk, (q + 1) * kEpiWarps * (a.F / kPipeGuWidth))) return false;
+    if (!wait_counter(a, cn.gu[p] + blk, (q + 1) * kEpiWarps * (a.F / a.gw))) return false;
     if (q > 0 && !wait_counter(a, cn.rd[p] + blk, q * min(BM, a.C - t.m * BM))) return false;
   }
   return true;
@@ -245,7 +251,7 @@ __device__ void dispatch_role(const PipelineArgs& a, const Counters& cn) {
     const int p = (r - a.r0) & 1;
     const int q = (r - a.r0) >> 1;
     // block (e, m) of buf[p] is free once every gate/up tile of it in round r-2 has read it
-    const int war_target = q * kEpiWarps * (a.F / kPipeGuWidth);
+    const int war_target = q * kEpiWarps * (a.F / a.gw);
     const int begin = a.row_start[r], rows = a.row_start[r + 1] - begin;
     const int chunk = (rows + W - 1) / W;
     const int lo = gw * chunk, hi = min(rows, lo + chunk);
@@ -296,8 +302,8 @@ __device__ void combine_role(const PipelineArgs& a, const Counters& cn) {
     const int p = (r - a.r0) & 1;
     const int q = (r - a.r0) >> 1;
     const int mblocks = a.mb_prefix[static_cast<size_t>(r) * (a.E + 1) + a.E];
-    dn_cum[p] += mblocks * kEpiWarps * (a.d / kPipeDnWidth);
-    const int blk_target = (q + 1) * kEpiWarps * (a.d / kPipeDnWidth);
+    dn_cum[p] += mblocks * kEpiWarps * (a.d / (2 * a.gw));
+    const int blk_target = (q + 1) * kEpiWarps * (a.d / (2 * a.gw));
     const copy::CombineArgs comb{a.out[p], a.y, a.idx, a.gate, a.round, a.slot, a.T, a.k, a.C, a.d};
     bool round_done = false;   // every down tile of round r seen finished
     for (long long c0 = gw; c0 < a.T; c0 += span) {
@@ -331,11 +337,15 @@ __device__ void combine_role(const PipelineArgs& a, const Counters& cn) {
   }
 }
 
+template <int GW>
 __global__ void __launch_bounds__(kPipeThreads, 1)
     round_pipeline_kernel(const __grid_constant__ CUtensorMap a_gu0, const __grid_constant__ CUtensorMap a_gu1,
                           const __grid_constant__ CUtensorMap b_gu, const __grid_constant__ CUtensorMap a_dn0,
                           const __grid_constant__ CUtensorMap a_dn1, const __grid_constant__ CUtensorMap b_dn,
                           const PipelineArgs a) {
+  constexpr int kBN = Geom<GW>::kBN;
+  constexpr int kPStageBytes = Geom<GW>::kStageBytes;
+  constexpr int kPStages = Geom<GW>::kStages;
   extern __shared__ uint8_t smem_raw[];
   __shared__ int last_cta;
   // tile ring: the producer publishes each claimed tile (-1: no more) to the MMA issuer and the
@@ -370,10 +380,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       bool ok = true;
       auto load_b = [&](const Tile& t, int kb, uint32_t sB, uint32_t fb) {
         if (t.gu) {
-          tma_load_3d(sB, &b_gu, fb, kb * BK, t.nt * kPipeGuWidth, t.e);
-          tma_load_3d(sB + kPipeGuWidth * BK * 2, &b_gu, fb, kb * BK, a.F + t.nt * kPipeGuWidth, t.e);
+          tma_load_3d(sB, &b_gu, fb, kb * BK, t.nt * GW, t.e);
+          tma_load_3d(sB + GW * BK * 2, &b_gu, fb, kb * BK, a.F + t.nt * GW, t.e);
         } else {
-          tma_load_3d(sB, &b_dn, fb, kb * BK, t.nt * kPipeDnWidth, t.e);
+          tma_load_3d(sB, &b_dn, fb, kb * BK, t.nt * kBN, t.e);
         }
       };
       int slot = 0;
@@ -561,11 +571,11 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kAccCols);
       const int p = (t.r - a.r0) & 1;
       if (t.gu) {
-        uint16_t* orow = a.h[p] + (static_cast<size_t>(t.e) * a.C + row) * a.F + t.nt * kPipeGuWidth;
-        store_swiglu(tb, kPipeGuWidth, orow, valid);
+        uint16_t* orow = a.h[p] + (static_cast<size_t>(t.e) * a.C + row) * a.F + t.nt * GW;
+        store_swiglu(tb, GW, orow, valid);
       } else {
-        uint16_t* orow = a.out[p] + (static_cast<size_t>(t.e) * a.C + row) * a.d + t.nt * kPipeDnWidth;
-        store_bf16(tb, kPipeDnWidth, orow, valid);
+        uint16_t* orow = a.out[p] + (static_cast<size_t>(t.e) * a.C + row) * a.d + t.nt * kBN;
+        store_bf16(tb, kBN, orow, valid);
       }
       tc_fence_before();
       mbar_arrive(smem_addr(&s.tempty[acc]));
@@ -617,15 +627,19 @@ cudaError_t launch_round_pipeline(const PipelineArgs& a, cudaStream_t stream) {
     e = gemm::make_map(&m_agu[p], a.buf[p], a.d, a.C, a.E, BM);
     if (e == cudaSuccess) e = gemm::make_map(&m_adn[p], a.h[p], a.F, a.C, a.E, BM);
   }
-  if (e == cudaSuccess) e = gemm::make_map(&m_bgu, a.w_gate_up, a.d, 2ull * a.F, a.E, kPipeGuWidth);
-  if (e == cudaSuccess) e = gemm::make_map(&m_bdn, a.w_down, a.F, a.d, a.E, kPipeDnWidth);
+  const int gw = a.gw;
+  if (gw != pipe_gate_width(a.d) || a.F % gw != 0 || a.d % (2 * gw) != 0) return cudaErrorInvalidValue;
+  if (e == cudaSuccess) e = gemm::make_map(&m_bgu, a.w_gate_up, a.d, 2ull * a.F, a.E, gw);
+  if (e == cudaSuccess) e = gemm::make_map(&m_bdn, a.w_down, a.F, a.d, a.E, 2 * gw);
   if (e != cudaSuccess) return e;
   static std::atomic<uint64_t> configured{0};   // one bit per device ordinal
   int dev = 0;
   cudaGetDevice(&dev);
   const uint64_t bit = 1ull << (dev & 63);
   if (!(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(round_pipeline_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    e = cudaFuncSetAttribute(round_pipeline_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(round_pipeline_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
@@ -642,7 +656,10 @@ cudaError_t launch_round_pipeline(const PipelineArgs& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   launch_begin(kKindPipeline, stream);
-  e = cudaLaunchKernelEx(&cfg, round_pipeline_kernel, m_agu[0], m_agu[1], m_bgu, m_adn[0], m_adn[1], m_bdn, a);
+  if (gw == 64)
+    e = cudaLaunchKernelEx(&cfg, round_pipeline_kernel<64>, m_agu[0], m_agu[1], m_bgu, m_adn[0], m_adn[1], m_bdn, a);
+  else
+    e = cudaLaunchKernelEx(&cfg, round_pipeline_kernel<32>, m_agu[0], m_agu[1], m_bgu, m_adn[0], m_adn[1], m_bdn, a);
   launch_end(kKindPipeline, stream);
   return e;
 }
