@@ -1473,7 +1473,9 @@ cudaError_t launch_backward_back(const BackwardArgs& a, int r, const int32_t* n_
     CUtensorMap ma[3], mb[3], mo[3];
     long long tiles = 0;
     g[0].mode = bwd::kDx;
-    g[0].width = pair ? 256 : pick_width(kWide, 3, mt, d);
+    // single-CTA form: the widest tiles when they divide (each tile's fixed costs, its pipeline
+    // fill and its epilogue, then cover the most columns), else the least streaming time
+    g[0].width = pair || d % 256 == 0 ? 256 : pick_width(kWide, 3, mt, d);
     g[0].n_total = d;
     g[0].num_k_blocks = 2 * F / gemm::BK;
     g[0].out = a.dxbuf;
@@ -1487,7 +1489,7 @@ cudaError_t launch_backward_back(const BackwardArgs& a, int r, const int32_t* n_
     g[1].mode = bwd::kWgrad;
     g[1].m_total = d;
     g[1].n_total = F;
-    g[1].width = pair ? 256 : pick_width(kWide, 3, mt_w2, F);
+    g[1].width = pair || F % 256 == 0 ? 256 : pick_width(kWide, 3, mt_w2, F);
     g[1].out = a.dw_down;
     g[1].overwrite = r == 0;
     g[1].out_group_stride = static_cast<long long>(d) * F;
@@ -1502,7 +1504,7 @@ cudaError_t launch_backward_back(const BackwardArgs& a, int r, const int32_t* n_
     g[2].mode = bwd::kWgrad;
     g[2].m_total = 2 * F;
     g[2].n_total = d;
-    g[2].width = pair ? 256 : pick_width(kWide, 3, mt_w13, d);
+    g[2].width = pair || d % 256 == 0 ? 256 : pick_width(kWide, 3, mt_w13, d);
     g[2].out = a.dw_gate_up;
     g[2].overwrite = r == 0;
     g[2].out_group_stride = 2ll * F * d;
