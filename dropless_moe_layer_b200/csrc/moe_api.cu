@@ -590,6 +590,17 @@ int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws
   bool gathered = false;     // the round's dispatch ran in the previous round's combine launch
   bool back_used[2] = {false, false};
   cudaStream_t back_stream = overlap ? side.stream : stream;
+  // the caller's stream waits for everything the second stream was given (also on an error
+  // return, so that no work of this call is left unordered behind the caller's next launches)
+  auto join = [&]() {
+    if (!overlap) return cudaSuccess;
+    const cudaError_t e = cudaEventRecord(side.front, back_stream);
+    return e == cudaSuccess ? cudaStreamWaitEvent(stream, side.front, 0) : e;
+  };
+  auto fail = [&](int code) {
+    join();
+    return code;
+  };
   for (int r = 0; r < info->R; ++r) {
     const int cur = r & 1, nxt = cur ^ 1;
     const bool more = r + 1 < info->R;
@@ -597,10 +608,10 @@ int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws
     const BackwardArgs& ar = set ? a2 : a;
     // front half on the caller's stream, after the last back half that read this set
     if (overlap && back_used[set] && (st = cuda_status(cudaStreamWaitEvent(stream, side.back[set], 0))) != MOE_OK)
-      return st;
+      return fail(st);
     int parts = 0;
     if ((st = cuda_status(launch_backward_front(ar, r, n_rounds[cur], !gathered, &parts, stream))) != MOE_OK)
-      return st;
+      return fail(st);
     // back half: the next round's dispatch joins its combine launch when the next round uses
     // the same set (its front half waits for this back half anyway)
     const int set_next = more ? next_set(set, n_rounds[nxt]) : 0;
@@ -608,24 +619,20 @@ int moe_backward(const moe_shape_t* shape, const moe_plan_info_t* info, void* ws
     if (overlap) {
       if ((st = cuda_status(cudaEventRecord(side.front, stream))) != MOE_OK ||
           (st = cuda_status(cudaStreamWaitEvent(back_stream, side.front, 0))) != MOE_OK)
-        return st;
+        return fail(st);
     }
     if ((st = cuda_status(launch_backward_back(ar, r, n_rounds[cur], parts, merge ? &ar : nullptr,
                                                merge ? n_rounds[nxt] : nullptr, back_stream))) != MOE_OK)
-      return st;
+      return fail(st);
     if (overlap) {
-      if ((st = cuda_status(cudaEventRecord(side.back[set], back_stream))) != MOE_OK) return st;
+      if ((st = cuda_status(cudaEventRecord(side.back[set], back_stream))) != MOE_OK) return fail(st);
       back_used[set] = true;
     }
     gathered = merge;
     set = set_next;
   }
   // dz after the last combine (the back halves ran in round order on the second stream)
-  if (overlap) {
-    if ((st = cuda_status(cudaEventRecord(side.front, back_stream))) != MOE_OK ||
-        (st = cuda_status(cudaStreamWaitEvent(stream, side.front, 0))) != MOE_OK)
-      return st;
-  }
+  if ((st = cuda_status(join())) != MOE_OK) return st;
   return cuda_status(launch_backward_gates(a, stream));
 }
 
